@@ -1,0 +1,353 @@
+"""Benchmark of the momentum selective scan on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one mm_scan_fwd call over one batch of the named workload (default:
+fp32, batch 4, L 2048, D 1536, N 16, beta 0.9, alpha 1.0), i.e. every step of
+the scan: staging, discretisation, velocity and hidden recurrences, read-out,
+final state.  Inputs are synthetic and seeded (see workloads.py).
+
+* value: state updates/s (batch * L * D * N per step, summed over ranks) with
+  inputs resident in HBM, timed with CUDA events on the launching stream over
+  exactly K steps between barriers; several input sets rotate so that the
+  bytes a step reads were evicted from the 126 MB L2 by the steps before it.
+* e2e: the same metric through the public host-memory call: every step copies
+  the inputs from pinned host memory, scans, and copies y, hT, vT back.
+* roofline: the scan kernel is bound by its exponentials (one MUFU ex2 per
+  state update, 16 per clock per SM); peak = 16 * 148 SMs * max SM clock.
+* cpu_baseline: the fp64 oracle on the host cores (rank 0, N = 1), on a
+  bounded sample of the same workload.
+* --impl reference: the oracle alone as the reference arm.
+
+Multi-GPU (launched by torchrun): one process per GPU, each scanning its own
+batch; there is no collective on the data path, only a barrier and a max of
+the per-rank times (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from selective_state_space_momentum_b200 import workloads as wl  # noqa: E402
+
+METRIC = "selective-scan state updates/s (B·L·D·N) and % of roofline, 1×B200"
+UNIT = "state updates/s"
+MUFU_EX2_PER_CLK_PER_SM = 16
+B200_SMS = 148
+FALLBACK_SM_MAX_MHZ = 1965.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126e6
+
+WORKLOADS = {w.name: w for w in wl.SCAN_WORKLOADS}
+ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
+           "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name}
+DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MAX_MHZ}, "fallback"
+
+
+def algorithmic_bytes(w: wl.ScanWorkload) -> int:
+    """Bytes one call must move: x, delta, y once; B, C once; A; hT, vT."""
+    eb = 4 if w.io == "f32" else 2
+    bdl = w.batch * w.dim * w.seqlen
+    return 3 * bdl * eb + 2 * w.batch * w.dstate * w.seqlen * eb + w.dim * w.dstate * 4 \
+        + 2 * w.batch * w.dim * w.dstate * 4
+
+
+# ------------------------------------------------------------ clocks -------
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:  # no NVML: report that, do not fail the bench
+            self.error = f"{type(e).__name__}: {e}"
+        return self
+
+    def _sample(self):
+        n = self._nvml
+        self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+        mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+        return False
+
+    def summary(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+               "samples": len(self.samples)}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# ------------------------------------------------------------ helpers ------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0):
+    """Time the fp64 oracle (as it stands) on whole passes over the workload,
+    or on a channel slice of it when one pass would exceed the budget."""
+    import oracle
+    inp = wl.scan_inputs(w)
+    nch = w.batch * w.dim
+    # calibrate on a small slice
+    probe = np.arange(min(nch, 64), dtype=np.int64)
+    t = time.perf_counter()
+    oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=probe)
+    per_chan = (time.perf_counter() - t) / len(probe)
+    if per_chan * nch <= budget_s:
+        chans, passes = None, max(1, int(budget_s // max(per_chan * nch, 1e-9)))
+        passes = min(passes, 3)
+        sample = f"{passes} full pass(es) over all {nch} channels"
+    else:
+        k = max(1, int(budget_s / per_chan))
+        chans, passes = np.linspace(0, nch - 1, k).astype(np.int64), 1
+        sample = f"{k} of {nch} channels (evenly spaced), 1 pass"
+    updates = (nch if chans is None else len(chans)) * w.seqlen * w.dstate * passes
+    t = time.perf_counter()
+    for _ in range(passes):
+        oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=chans)
+    dt = time.perf_counter() - t
+    return {"value": updates / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": sample + f", beta={beta}, alpha={alpha}, fp64, {dt:.2f} s wall"}
+
+
+def run_reference(args, w, beta, alpha):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    cb = cpu_baseline(w, beta, alpha, budget_s=args.reference_budget)
+    line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
+                       "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------- main -------
+def main(argv=None):
+    ap = argparse.ArgumentParser(description="momentum selective scan benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--beta", type=float, default=None)
+    ap.add_argument("--alpha", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-budget", type=float, default=12.0)
+    ap.add_argument("--tile", default=None, help="force SPTxWARPS, e.g. 4x2 (tuning)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[ALIASES.get(args.workload, args.workload)]
+    default = (0.9, 1.0) if (0.9, 1.0) in w.runs else w.runs[0]
+    beta = args.beta if args.beta is not None else default[0]
+    alpha = args.alpha if args.alpha is not None else default[1]
+    if args.impl == "reference":
+        return run_reference(args, w, beta, alpha)
+
+    import torch
+    import selective_state_space_momentum_b200 as mm
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if args.tile:
+        spt, warps = (int(v) for v in args.tile.split("x"))
+        mm.mm_scan_set_tile(spt, warps)
+
+    # Each rank scans its own batch (seed offset by rank): weak scaling.
+    inp = wl.scan_inputs(w, seed=wl.seed_of(w.seed_index) + 1000 * rank)
+    iodt = torch.float32 if w.io == "f32" else torch.bfloat16
+    host = {k: torch.from_numpy(v) for k, v in inp.items()}
+    step_bytes = algorithmic_bytes(w)
+    # enough input sets that a step's bytes were evicted by the steps before it
+    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    sets = []
+    for _ in range(nsets):
+        s = {k: host[k].to(dev).to(iodt if k in ("x", "delta", "B", "C") else torch.float32).contiguous()
+             for k in host}
+        s["y"] = torch.empty_like(s["x"])
+        s["hT"] = torch.empty((w.batch, w.dim, w.dstate), device=dev)
+        s["vT"] = torch.empty_like(s["hT"])
+        sets.append(s)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % nsets]
+        mm.mm_scan_fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha,
+                       s["y"], s["hT"], s["vT"], stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if world == 1 else local) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    updates = w.updates
+    value = updates * world / (ms_step * 1e-3)
+
+    # ---- end to end through the host-memory call -------------------------
+    e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
+    pinned = {k: v.to(iodt if k in ("x", "delta", "B", "C") else torch.float32).pin_memory()
+              for k, v in host.items()}
+    out = {"y": torch.empty(tuple(inp["x"].shape), dtype=iodt, pin_memory=True),
+           "hT": torch.empty((w.batch, w.dim, w.dstate), pin_memory=True),
+           "vT": torch.empty((w.batch, w.dim, w.dstate), pin_memory=True)}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in out.values())
+    for _ in range(2):
+        mm.scan_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
+                         beta=beta, alpha=alpha, out=out)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        mm.scan_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
+                         beta=beta, alpha=alpha, out=out, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    barrier()
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        clocks = clk.summary()
+        sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
+        mufu_peak = MUFU_EX2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
+        achieved = updates / (ms_step * 1e-3)      # one ex2 per update, per launch
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        hbm_achieved = step_bytes / (ms_step * 1e-3) / 1e9
+        cb = None
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(w, beta, alpha)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
+                       "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
+                       "global_batch": w.batch * world, "parallelism": f"dp{world}",
+                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
+            "roofline": {"bound": "alu", "kernel": "scan_fwd_kernel",
+                         "achieved": achieved / 1e9, "peak": mufu_peak / 1e9, "unit": "Gex2/s",
+                         "frac": achieved / mufu_peak, "traffic": None,
+                         "peak_source": f"16 ex2/clk/SM x 148 SMs x {sm_max:.0f} MHz",
+                         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": hbm_achieved / hbm_peak, "peak_source": peak_kind,
+                                 "algorithmic_bytes": step_bytes}},
+            "e2e": {"value": updates * world / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+        if cb is not None:
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

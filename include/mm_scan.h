@@ -1,0 +1,195 @@
+/*
+ * mm_scan.h -- C ABI of libmmscan.so: the forward selective scan of Mamba-1
+ * with the Momentum Mamba extension, and its Mamba-2 scalar-A chunked (SSD)
+ * form, on NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named as device buffers must be CUDA device (or managed) memory
+ *   of the current device; the caller allocates and owns every buffer.  The
+ *   library allocates no memory and keeps no state between calls except a
+ *   per-thread copy of the last error message (mm_last_error).
+ * - Every base pointer must be 16-byte aligned (MM_ERR_ALIGN otherwise).
+ *   Tensors are dense and contiguous in the stated layout, last index
+ *   fastest.
+ * - All argument checks run on the host before anything is launched; a call
+ *   that returns an error has launched nothing and touched no buffer.
+ * - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *   legacy default stream) and runs asynchronously: the call returns once
+ *   the kernels are queued.  Faults during execution surface at the caller's
+ *   next synchronisation with that stream, as for any CUDA kernel.
+ * - Calls on different streams that write the same output buffers race.
+ */
+#ifndef MM_SCAN_H
+#define MM_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MM_OK = 0,
+    MM_ERR_NULL = 1,           /* a required pointer is NULL                      */
+    MM_ERR_DIMS = 2,           /* a size is < 1, or sizes are inconsistent         */
+    MM_ERR_SCALAR = 3,         /* beta outside [0, 1), alpha < 0, or non-finite    */
+    MM_ERR_DTYPE = 4,          /* unknown storage type code                        */
+    MM_ERR_ALIGN = 5,          /* a base pointer is not 16-byte aligned            */
+    MM_ERR_UNSUPPORTED = 6,    /* valid request outside what this build supports   */
+    MM_ERR_CUDA = 7,           /* a CUDA runtime call or a launch failed           */
+    MM_ERR_DEVICE_TIMEOUT = 8, /* a bounded device-side wait gave up               */
+    MM_ERR_ALIAS = 9           /* an output overlaps an input it may not overlap   */
+} mm_status;
+
+/* Storage type of the streamed tensors (x, delta, B, C, y). */
+typedef enum { MM_F32 = 0, MM_BF16 = 1 } mm_dtype;
+
+/* Sizes of one Mamba-1 scan call. */
+typedef struct {
+    int64_t batch;   /* b: independent sequences                          */
+    int64_t seqlen;  /* L: time steps                                      */
+    int64_t dim;     /* D: channels (d_inner)                              */
+    int64_t dstate;  /* N: states per channel, 1..16                       */
+    int32_t io;      /* mm_dtype of x, delta, B, C and y                   */
+} mm_scan_dims;
+
+/*
+ * mm_scan_fwd -- momentum selective scan, forward.
+ *
+ * Computes, for every batch row b, channel d and state n
+ * ("Momentum Mamba: Enhanced State Space Models with Momentum", sections
+ * "Momentum Mamba Recurrence" and "Discretization Note"):
+ *
+ *     v_t = beta * v_{t-1} + alpha * delta_t * B_t[n] * x_t
+ *     h_t = exp(delta_t * A[d,n]) * h_{t-1} + v_t
+ *     y_t = sum_n C_t[n] * h_t[n]
+ *
+ * beta = 0, alpha = 1 is the plain Mamba scan (same page, "Hyperparameters").
+ * This is the core of the page's `selective_scan_fn` (section
+ * "selective_scan_fn") with D = z = delta_bias = None and
+ * delta_softplus = False: delta is taken as given, already positive.
+ *
+ * Arguments (device buffers unless noted):
+ *   x      (batch, dim, L)     io     input u
+ *   delta  (batch, dim, L)     io     step size
+ *   A      (dim, dstate)       fp32   state matrix (any finite values)
+ *   B, C   (batch, dstate, L)  io     input / output projections, shared
+ *                                      by all channels of a batch row
+ *   h0, v0 (batch, dim, dstate) fp32  initial hidden state / velocity, or
+ *                                      NULL for zero (the page initialises
+ *                                      the velocity to zero)
+ *   beta   host scalar in [0, 1)      momentum decay
+ *   alpha  host scalar, finite, >= 0  momentum scale
+ *   y      (batch, dim, L)     io     output, rounded to nearest-even for bf16
+ *   hT, vT (batch, dim, dstate) fp32  final h_{L-1} and v_{L-1}, or NULL to
+ *                                      skip ("return_last_state")
+ *   dims   host struct of sizes; stream: cudaStream_t or NULL
+ *
+ * Arithmetic is fp32 with the state held in registers.  exp is evaluated
+ * as a base-2 exponential of delta * (A * log2 e).
+ *
+ * Aliasing: hT may be the same buffer as h0 and vT the same as v0 (in-place
+ * streaming: every lane reads its initial state before writing its final
+ * one); no other overlap between outputs and inputs is allowed
+ * (MM_ERR_ALIAS).
+ *
+ * Streaming: for a fixed (batch, dim, dstate, io), calling with the first
+ * L1 steps and then with the remaining steps, passing (hT, vT) of the first
+ * call as (h0, v0) of the second, gives final states bit-identical to one
+ * call over all steps, and the same y within rounding of the read-out.
+ *
+ * Errors: MM_ERR_NULL (x, delta, A, B, C, y or dims NULL), MM_ERR_DIMS
+ * (a size < 1), MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE,
+ * MM_ERR_SCALAR, MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA (launch failure;
+ * mm_last_error has CUDA's message).
+ */
+mm_status mm_scan_fwd(const void *x, const void *delta, const float *A,
+                      const void *B, const void *C,
+                      const float *h0, const float *v0,
+                      float beta, float alpha,
+                      void *y, float *hT, float *vT,
+                      const mm_scan_dims *dims, void *stream);
+
+/* Sizes of one Mamba-2 SSD call. */
+typedef struct {
+    int64_t batch;    /* b                                                  */
+    int64_t seqlen;   /* L                                                  */
+    int64_t nheads;   /* H                                                  */
+    int64_t headdim;  /* P (the page's head dimension, 64 in its example)   */
+    int64_t dstate;   /* N                                                  */
+    int64_t ngroups;  /* G: B/C groups; head h reads group h / (H / G)      */
+    int64_t chunk;    /* Q: chunk length of the 4-step algorithm            */
+} mm_ssd_dims;
+
+/*
+ * mm_ssd_workspace_size -- bytes of device workspace mm_ssd_fwd needs for
+ * these sizes (written to *bytes).  The caller allocates it (any 256-byte
+ * aligned device buffer of at least that size) and passes it to every call
+ * with the same sizes; the library keeps nothing in it between calls.
+ * Errors: MM_ERR_NULL, MM_ERR_DIMS, MM_ERR_UNSUPPORTED as for mm_ssd_fwd.
+ */
+mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
+
+/*
+ * mm_ssd_fwd -- Mamba-2 scalar-A multi-head scan through the chunked (SSD)
+ * algorithm ("Mamba-2 -- SSM = structured matrix multiply", sections
+ * "4-Step Algorithm" and "Multi-Head Expansion"; first-order
+ * discretization B_bar = delta * B as in the Momentum Mamba page).
+ *
+ * For every batch row b, head h, head channel p and state n:
+ *     h_t[p, n] = exp(delta_t[h] * A[h]) * h_{t-1}[p, n]
+ *                 + alpha * delta_t[h] * B_t[g(h), n] * x_t[h, p]
+ *     y_t[h, p] = sum_n C_t[g(h), n] * h_t[p, n]
+ * computed per chunk of Q steps as: intra-chunk products C B^T masked by
+ * the decay, the chunk's own final state, a scan of the states across
+ * chunks, and the read-out of the carried state (tensor-core GEMMs for the
+ * three dense steps).
+ *
+ * Arguments (device buffers unless noted):
+ *   x      (batch, L, H, P)  bf16   input
+ *   delta  (batch, L, H)     fp32   step size per head
+ *   A      (H)               fp32   one decay rate per head
+ *   B, C   (batch, L, G, N)  bf16
+ *   h0     (batch, H, P, N)  fp32   initial state or NULL (zero)
+ *   beta   must be 0 (momentum in chunked form is not built: MM_ERR_UNSUPPORTED)
+ *   alpha  finite, >= 0
+ *   y      (batch, L, H, P)  bf16   output (round to nearest-even)
+ *   hT     (batch, H, P, N)  fp32   final state or NULL; may equal h0
+ *   workspace, workspace_bytes      device scratch of at least
+ *                                   mm_ssd_workspace_size() bytes
+ * Supported sizes: headdim 64, dstate 128, chunk 256 (power of two),
+ * seqlen any >= 1, H a multiple of G.
+ * Errors: as mm_scan_fwd, plus MM_ERR_DIMS for a workspace that is too
+ * small.
+ */
+mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
+                     const void *B, const void *C, const float *h0,
+                     float beta, float alpha,
+                     void *y, float *hT,
+                     void *workspace, size_t workspace_bytes,
+                     const mm_ssd_dims *dims, void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *mm_status_string(mm_status status);
+
+/* Detail of the last error returned on this host thread ("" if none). */
+const char *mm_last_error(void);
+
+/*
+ * Tuning knob for benchmarks: force the scan's per-thread state count
+ * (2 or 4) and warps per block (1, 2 or 4); 0, 0 restores the automatic
+ * choice.  Process-wide, not thread-safe with concurrent calls.  Returns
+ * MM_ERR_UNSUPPORTED for a combination that is not built.
+ */
+mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MM_SCAN_H */

@@ -1,0 +1,251 @@
+"""B200-native Momentum Mamba selective scan (and its Mamba-2 SSD form).
+
+Thin Python binding over ``libmmscan.so`` (include/mm_scan.h).  Functions
+named like the C entry points (``mm_scan_fwd``, ``mm_ssd_fwd``, ...) only
+marshal arguments: every step of the computation runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.  There is no CPU
+fallback: without the built library (``python -m
+selective_state_space_momentum_b200.build``) every compute call raises.
+
+Convenience wrappers allocate outputs:
+
+* :func:`scan_fwd` -- ``(y, last_state, last_velocity)`` like the Momentum
+  Mamba page's ``selective_scan_fn`` with D, z, delta_bias unset and no
+  softplus on delta.
+* :func:`ssd_fwd` -- ``(y, last_state)`` of the multi-head scalar-A form.
+* :func:`scan_fwd_host` -- end-to-end call on host arrays (copies in, scan,
+  copies out) for callers whose data lives in host memory.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
+    "mm_scan_fwd", "mm_ssd_fwd", "mm_ssd_workspace_size", "mm_status_string",
+    "mm_last_error", "mm_scan_set_tile", "mm_version",
+    "scan_fwd", "ssd_fwd", "scan_fwd_host", "EXPORTED_SYMBOLS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libmmscan.so")
+_lock = threading.Lock()
+_lib = None
+
+MM_F32 = 0
+MM_BF16 = 1
+
+STATUS_NAMES = {
+    0: "MM_OK", 1: "MM_ERR_NULL", 2: "MM_ERR_DIMS", 3: "MM_ERR_SCALAR", 4: "MM_ERR_DTYPE",
+    5: "MM_ERR_ALIGN", 6: "MM_ERR_UNSUPPORTED", 7: "MM_ERR_CUDA", 8: "MM_ERR_DEVICE_TIMEOUT",
+    9: "MM_ERR_ALIAS",
+}
+
+# Every function include/mm_scan.h declares.
+EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_ssd_workspace_size", "mm_ssd_fwd", "mm_status_string",
+                    "mm_last_error", "mm_scan_set_tile", "mm_version")
+
+
+class MMError(RuntimeError):
+    """A libmmscan call returned a status other than MM_OK."""
+
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        self.name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{where}: {self.name}: {detail}")
+
+
+class ScanDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("io", ctypes.c_int32)]
+
+
+class SSDDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64),
+                ("ngroups", ctypes.c_int64), ("chunk", ctypes.c_int64)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _declare(lib):
+    vp, f = ctypes.c_void_p, ctypes.c_float
+    lib.mm_scan_fwd.restype = ctypes.c_int
+    lib.mm_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp,
+                                ctypes.POINTER(ScanDims), vp]
+    lib.mm_ssd_workspace_size.restype = ctypes.c_int
+    lib.mm_ssd_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.POINTER(ctypes.c_size_t)]
+    lib.mm_ssd_fwd.restype = ctypes.c_int
+    lib.mm_ssd_fwd.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, ctypes.c_size_t,
+                               ctypes.POINTER(SSDDims), vp]
+    lib.mm_status_string.restype = ctypes.c_char_p
+    lib.mm_status_string.argtypes = [ctypes.c_int]
+    lib.mm_last_error.restype = ctypes.c_char_p
+    lib.mm_last_error.argtypes = []
+    lib.mm_scan_set_tile.restype = ctypes.c_int
+    lib.mm_scan_set_tile.argtypes = [ctypes.c_int, ctypes.c_int]
+    lib.mm_version.restype = ctypes.c_int
+    lib.mm_version.argtypes = []
+    return lib
+
+
+def load_library(path: str | None = None):
+    """Load libmmscan.so (raises if it has not been built)."""
+    global _lib
+    if path is not None:
+        return _declare(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m selective_state_space_momentum_b200.build` (needs nvcc)")
+            _lib = _declare(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        lib = load_library()
+        raise MMError(rc, where, lib.mm_last_error().decode())
+
+
+# ------------------------------------------------------- C-named calls -----
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _io_code(dtype) -> int:
+    import torch
+    if dtype == torch.float32:
+        return MM_F32
+    if dtype == torch.bfloat16:
+        return MM_BF16
+    raise TypeError(f"unsupported storage type {dtype}; use float32 or bfloat16")
+
+
+def mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
+    """C entry point mm_scan_fwd on torch CUDA tensors (marshalling only).
+
+    Shapes: x, delta, y (batch, dim, L); A (dim, N) fp32; B, C (batch, N, L);
+    h0, v0, hT, vT (batch, dim, N) fp32 or None.  x, delta, B, C, y share one
+    storage type (fp32 or bf16).  Raises MMError on a non-OK status.
+    """
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_fwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
+                                    _ptr(v0), float(beta), float(alpha), _ptr(y), _ptr(hT), _ptr(vT),
+                                    ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_fwd")
+
+
+def mm_ssd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk) -> int:
+    dims = SSDDims(batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
+    out = ctypes.c_size_t(0)
+    _check(load_library().mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(out)),
+           "mm_ssd_workspace_size")
+    return int(out.value)
+
+
+def mm_ssd_fwd(x, delta, A, B, C, h0, beta, alpha, y, hT, workspace, chunk, stream=None):
+    """C entry point mm_ssd_fwd on torch CUDA tensors (marshalling only).
+
+    x, y (batch, L, H, P) bf16; delta (batch, L, H) fp32; A (H) fp32;
+    B, C (batch, L, G, N) bf16; h0, hT (batch, H, P, N) fp32 or None;
+    workspace: a uint8 CUDA tensor of mm_ssd_workspace_size() bytes.
+    """
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dims = SSDDims(batch, L, H, P, N, G, chunk)
+    rc = load_library().mm_ssd_fwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
+                                   float(beta), float(alpha), _ptr(y), _ptr(hT), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(),
+                                   ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_ssd_fwd")
+
+
+def mm_status_string(status: int) -> str:
+    return load_library().mm_status_string(status).decode()
+
+
+def mm_last_error() -> str:
+    return load_library().mm_last_error().decode()
+
+
+def mm_scan_set_tile(states_per_thread: int, warps_per_block: int):
+    _check(load_library().mm_scan_set_tile(states_per_thread, warps_per_block), "mm_scan_set_tile")
+
+
+def mm_version() -> int:
+    return int(load_library().mm_version())
+
+
+# ------------------------------------------------------------ wrappers -----
+def scan_fwd(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0,
+             return_last_state=True, stream=None):
+    """Allocate outputs and run mm_scan_fwd; returns (y, hT, vT) (states None
+    when ``return_last_state`` is False)."""
+    import torch
+    y = torch.empty_like(x)
+    hT = vT = None
+    if return_last_state:
+        shape = (x.shape[0], x.shape[1], A.shape[1])
+        hT = torch.empty(shape, device=x.device, dtype=torch.float32)
+        vT = torch.empty(shape, device=x.device, dtype=torch.float32)
+    mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream)
+    return y, hT, vT
+
+
+def ssd_fwd(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, return_last_state=True,
+            workspace=None, stream=None):
+    """Allocate outputs (and workspace if not given) and run mm_ssd_fwd;
+    returns (y, hT)."""
+    import torch
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    need = mm_ssd_workspace_size(batch, L, H, P, N, G, chunk)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, device=x.device, dtype=torch.uint8)
+    y = torch.empty_like(x)
+    hT = torch.empty((batch, H, P, N), device=x.device, dtype=torch.float32) if return_last_state else None
+    mm_ssd_fwd(x, delta, A, B, C, h0, 0.0, alpha, y, hT, workspace, chunk, stream)
+    return y, hT
+
+
+def scan_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, device="cuda",
+                  out=None, stream=None):
+    """End-to-end scan of host (CPU, ideally pinned) tensors.
+
+    Copies the inputs to the device, runs mm_scan_fwd, and copies y, hT and
+    vT back into ``out`` (a dict of host tensors, allocated if None).
+    Returns that dict after synchronising the stream.
+    """
+    import torch
+    s = stream or torch.cuda.current_stream(device)
+    with torch.cuda.stream(s):
+        dev = [t.to(device, non_blocking=True) if t is not None else None
+               for t in (x, delta, A, B, C, h0, v0)]
+        y, hT, vT = scan_fwd(*dev[:5], h0=dev[5], v0=dev[6], beta=beta, alpha=alpha, stream=s)
+        if out is None:
+            out = {"y": torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
+                   "hT": torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True),
+                   "vT": torch.empty(vT.shape, dtype=vT.dtype, pin_memory=True)}
+        out["y"].copy_(y, non_blocking=True)
+        out["hT"].copy_(hT, non_blocking=True)
+        out["vT"].copy_(vT, non_blocking=True)
+    s.synchronize()
+    return out

@@ -1,0 +1,249 @@
+// mm_api.cpp -- the C ABI of libmmscan (declared in include/mm_scan.h):
+// host-side argument checks, variant choice and launch.  Every check runs
+// before anything is enqueued; a rejected call touches no buffer.
+#include "mm_scan.h"
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "mm_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+mm_status fail(mm_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+mm_status ok() {
+    g_last_error.clear();
+    return MM_OK;
+}
+
+std::atomic<int> g_forced_spt{0};
+std::atomic<int> g_forced_warps{0};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// a * b * ... without int64 overflow; false on overflow.
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+struct Range {
+    const char* name;
+    uintptr_t lo, hi;   // [lo, hi)
+};
+
+Range rng(const char* name, const void* p, int64_t bytes) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    return Range{name, lo, p ? lo + static_cast<uintptr_t>(bytes) : lo};
+}
+
+bool overlap(const Range& a, const Range& b) {
+    if (a.lo == a.hi || b.lo == b.hi) return false;   // NULL / empty
+    return a.lo < b.hi && b.lo < a.hi;
+}
+
+// Fault-injection hook for the host-side error path: with
+// MMSCAN_FAULT_INJECT=launch a call that passed its checks returns
+// MM_ERR_CUDA without launching anything.
+bool inject_launch_failure() {
+    const char* v = std::getenv("MMSCAN_FAULT_INJECT");
+    return v && std::strcmp(v, "launch") == 0;
+}
+
+mm_status from_cuda(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return ok();
+    return fail(MM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mm_status_string(mm_status s) {
+    switch (s) {
+        case MM_OK: return "ok";
+        case MM_ERR_NULL: return "a required pointer is NULL";
+        case MM_ERR_DIMS: return "invalid sizes";
+        case MM_ERR_SCALAR: return "beta must be in [0, 1) and alpha finite and >= 0";
+        case MM_ERR_DTYPE: return "unknown storage type";
+        case MM_ERR_ALIGN: return "a base pointer is not 16-byte aligned";
+        case MM_ERR_UNSUPPORTED: return "request outside what this build supports";
+        case MM_ERR_CUDA: return "CUDA error";
+        case MM_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+        case MM_ERR_ALIAS: return "an output overlaps an input";
+    }
+    return "unknown status";
+}
+
+const char* mm_last_error(void) { return g_last_error.c_str(); }
+
+int mm_version(void) { return 100; }
+
+mm_status mm_scan_set_tile(int spt, int warps) {
+    if (spt == 0 && warps == 0) {
+        g_forced_spt = 0;
+        g_forced_warps = 0;
+        return ok();
+    }
+    if (!mmscan::scan_tile_supported(spt, warps))
+        return fail(MM_ERR_UNSUPPORTED, "scan tile spt=%d warps=%d is not built", spt, warps);
+    g_forced_spt = spt;
+    g_forced_warps = warps;
+    return ok();
+}
+
+mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const void* B,
+                      const void* C, const float* h0, const float* v0, float beta, float alpha,
+                      void* y, float* hT, float* vT, const mm_scan_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !y)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
+    const int64_t bsz = dims->batch, L = dims->seqlen, D = dims->dim, N = dims->dstate;
+    if (bsz < 1 || L < 1 || D < 1 || N < 1)
+        return fail(MM_ERR_DIMS, "sizes must be >= 1 (batch=%lld seqlen=%lld dim=%lld dstate=%lld)",
+                    (long long)bsz, (long long)L, (long long)D, (long long)N);
+    if (N > 16) return fail(MM_ERR_UNSUPPORTED, "dstate=%lld > 16", (long long)N);
+    if (dims->io != MM_F32 && dims->io != MM_BF16)
+        return fail(MM_ERR_DTYPE, "io=%d is not MM_F32 or MM_BF16", (int)dims->io);
+    if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
+        return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
+    if (!std::isfinite(alpha) || alpha < 0.0f)
+        return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
+    const int64_t esize = dims->io == MM_F32 ? 4 : 2;
+    int64_t bd, bdl, seq_bytes, bn, bnl, bc_bytes, dn, a_bytes, bdn, st_bytes;
+    if (!mul_ok(bsz, D, &bd) || !mul_ok(bd, L, &bdl) || !mul_ok(bdl, esize, &seq_bytes) ||
+        !mul_ok(bsz, N, &bn) || !mul_ok(bn, L, &bnl) || !mul_ok(bnl, esize, &bc_bytes) ||
+        !mul_ok(D, N, &dn) || !mul_ok(dn, 4, &a_bytes) || !mul_ok(bd, N, &bdn) ||
+        !mul_ok(bdn, 4, &st_bytes))
+        return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
+    const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT};
+    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "y", "hT", "vT"};
+    for (int i = 0; i < 10; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+
+    const Range rx = rng("x", x, seq_bytes), rd = rng("delta", delta, seq_bytes),
+                rA = rng("A", A, a_bytes), rB = rng("B", B, bc_bytes), rC = rng("C", C, bc_bytes),
+                rh0 = rng("h0", h0, st_bytes), rv0 = rng("v0", v0, st_bytes),
+                ry = rng("y", y, seq_bytes), rhT = rng("hT", hT, st_bytes),
+                rvT = rng("vT", vT, st_bytes);
+    const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0, &rv0};
+    for (const Range* in : inputs)
+        if (overlap(ry, *in)) return fail(MM_ERR_ALIAS, "y overlaps %s", in->name);
+    for (const Range* out : {&rhT, &rvT}) {
+        for (const Range* in : inputs) {
+            const bool same_state = (out == &rhT && in == &rh0) || (out == &rvT && in == &rv0);
+            if (!overlap(*out, *in)) continue;
+            if (same_state && out->lo == in->lo) continue;   // in-place streaming
+            return fail(MM_ERR_ALIAS, "%s overlaps %s", out->name, in->name);
+        }
+        if (overlap(*out, ry)) return fail(MM_ERR_ALIAS, "%s overlaps y", out->name);
+    }
+    if (overlap(rhT, rvT)) return fail(MM_ERR_ALIAS, "hT overlaps vT");
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+
+    mmscan::ScanArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.h0 = h0; a.v0 = v0;
+    a.y = y; a.hT = hT; a.vT = vT;
+    a.batch = bsz; a.seqlen = L; a.dim = D; a.dstate = (int)N;
+    a.beta = beta; a.alpha = alpha;
+    a.vec_ok = ((L * esize) % 16) == 0;
+    const mmscan::ScanTileChoice t =
+        mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load());
+    return from_cuda(mmscan::launch_scan_fwd(a, t, dims->io, static_cast<cudaStream_t>(stream)),
+                     "mm_scan_fwd launch");
+}
+
+mm_status mm_ssd_workspace_size(const mm_ssd_dims* dims, size_t* bytes) {
+    if (!dims || !bytes) return fail(MM_ERR_NULL, "dims and bytes are required");
+    if (dims->batch < 1 || dims->seqlen < 1 || dims->nheads < 1 || dims->headdim < 1 ||
+        dims->dstate < 1 || dims->ngroups < 1 || dims->chunk < 1 ||
+        dims->nheads % dims->ngroups != 0)
+        return fail(MM_ERR_DIMS, "invalid SSD sizes");
+    if (!mmscan::ssd_shape_supported(dims->headdim, dims->dstate, dims->chunk))
+        return fail(MM_ERR_UNSUPPORTED, "SSD with headdim=%lld dstate=%lld chunk=%lld is not built",
+                    (long long)dims->headdim, (long long)dims->dstate, (long long)dims->chunk);
+    *bytes = mmscan::ssd_workspace_bytes(dims->batch, dims->seqlen, dims->nheads, dims->headdim,
+                                         dims->dstate, dims->chunk);
+    return ok();
+}
+
+mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const void* B,
+                     const void* C, const float* h0, float beta, float alpha, void* y, float* hT,
+                     void* workspace, size_t workspace_bytes, const mm_ssd_dims* dims,
+                     void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !y || !workspace)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C, y and workspace are required");
+    size_t need = 0;
+    mm_status st = mm_ssd_workspace_size(dims, &need);
+    if (st != MM_OK) return st;
+    if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
+        return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
+    if (beta != 0.0f)
+        return fail(MM_ERR_UNSUPPORTED, "momentum (beta != 0) in the chunked SSD form is not built");
+    if (!std::isfinite(alpha) || alpha < 0.0f)
+        return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
+    if (workspace_bytes < need)
+        return fail(MM_ERR_DIMS, "workspace of %zu bytes is smaller than the %zu needed",
+                    workspace_bytes, need);
+    const int64_t bsz = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
+                  N = dims->dstate, G = dims->ngroups;
+    int64_t blh, xy_bytes, bl, d_bytes, blg, bc_elems, bc_bytes, st_elems, st_bytes;
+    if (!mul_ok(bsz * L, H, &blh) || !mul_ok(blh, P * 2, &xy_bytes) || !mul_ok(bsz, L, &bl) ||
+        !mul_ok(bl, H * 4, &d_bytes) || !mul_ok(bl, G, &blg) || !mul_ok(blg, N, &bc_elems) ||
+        !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz * H, P * N, &st_elems) ||
+        !mul_ok(st_elems, 4, &st_bytes))
+        return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
+    const void* ptrs[] = {x, delta, A, B, C, h0, y, hT, workspace};
+    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "y", "hT", "workspace"};
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    const Range rx = rng("x", x, xy_bytes), rd = rng("delta", delta, d_bytes),
+                rA = rng("A", A, H * 4), rB = rng("B", B, bc_bytes), rC = rng("C", C, bc_bytes),
+                rh0 = rng("h0", h0, st_bytes), ry = rng("y", y, xy_bytes),
+                rhT = rng("hT", hT, st_bytes),
+                rw = rng("workspace", workspace, (int64_t)workspace_bytes);
+    const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0};
+    for (const Range* out : {&ry, &rhT, &rw}) {
+        for (const Range* in : inputs) {
+            if (!overlap(*out, *in)) continue;
+            if (out == &rhT && in == &rh0 && out->lo == in->lo) continue;
+            return fail(MM_ERR_ALIAS, "%s overlaps %s", out->name, in->name);
+        }
+    }
+    if (overlap(ry, rhT) || overlap(ry, rw) || overlap(rhT, rw))
+        return fail(MM_ERR_ALIAS, "outputs and workspace overlap");
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+
+    mmscan::SSDArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.h0 = h0; a.y = y; a.hT = hT;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
+    a.chunk = dims->chunk; a.alpha = alpha;
+    const cudaError_t e = mmscan::launch_ssd_fwd(a, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported)
+        return fail(MM_ERR_UNSUPPORTED, "the SSD kernels are not part of this build");
+    return from_cuda(e, "mm_ssd_fwd launch");
+}
+
+}  // extern "C"

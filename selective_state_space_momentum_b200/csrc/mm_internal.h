@@ -1,0 +1,62 @@
+// mm_internal.h -- declarations shared by the translation units of
+// libmmscan (argument blocks and launchers).  Not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mmscan {
+
+// Arguments of one scan launch (device pointers; sizes as in mm_scan_dims).
+struct ScanArgs {
+    const void* x;
+    const void* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* h0;
+    const float* v0;
+    void* y;
+    float* hT;
+    float* vT;
+    int64_t batch, seqlen, dim;
+    int dstate;
+    int tiles_per_batch;   // filled by the launcher
+    float beta, alpha;
+    int vec_ok;            // rows of L elements are whole 16-byte pieces
+};
+
+struct ScanTileChoice {
+    int np;      // states padded to a power of two (2, 4, 8, 16)
+    int spt;     // states per lane (2 or 4)
+    int warps;   // warps per CTA (1, 2 or 4)
+};
+
+bool scan_tile_supported(int spt, int warps);
+ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
+                                int forced_spt, int forced_warps);
+cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s);
+
+// Arguments of one SSD call.
+struct SSDArgs {
+    const void* x;
+    const float* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* h0;
+    void* y;
+    float* hT;
+    void* workspace;
+    size_t workspace_bytes;
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
+    float alpha;
+};
+
+size_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                           int64_t dstate, int64_t chunk);
+bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk);
+cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t s);
+
+}  // namespace mmscan

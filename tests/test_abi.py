@@ -1,0 +1,139 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/*.h declares, and rejects bad arguments on the host.
+
+No test here launches anything: every call either fails a host-side check
+(which returns before any CUDA call) or takes the fault-injection path that
+returns MM_ERR_CUDA without launching.  Pointers are fake, aligned integers.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import selective_state_space_momentum_b200 as mm
+from selective_state_space_momentum_b200 import build as mmbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mmbuild.build()
+    return mm.load_library()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(mm_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_function_is_exported(lib):
+    declared = _declared_functions()
+    assert declared, "no declarations found in include/*.h"
+    assert declared == set(mm.EXPORTED_SYMBOLS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_library_needs_no_cuda_shared_object():
+    path = mmbuild.build()
+    out = os.popen(f"ldd {path}").read()
+    assert "libcudart" not in out and "libcuda.so" not in out
+
+
+def test_status_strings(lib):
+    for code in range(10):
+        assert lib.mm_status_string(code)
+    assert mm.mm_version() >= 100
+
+
+A16 = 1 << 20   # a fake, 16-byte aligned address
+
+
+def _fake(k):
+    return ctypes.c_void_p(A16 * (k + 1))
+
+
+def _scan(lib, dims, beta=0.9, alpha=1.0, **over):
+    args = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), h0=None, v0=None,
+                y=_fake(5), hT=None, vT=None)
+    args.update(over)
+    return lib.mm_scan_fwd(args["x"], args["delta"], args["A"], args["B"], args["C"], args["h0"],
+                           args["v0"], beta, alpha, args["y"], args["hT"], args["vT"],
+                           ctypes.byref(dims) if dims is not None else None, None)
+
+
+def D(batch=1, L=64, dim=8, N=16, io=0):
+    return mm.ScanDims(batch, L, dim, N, io)
+
+
+def test_scan_rejects_bad_arguments(lib):
+    assert _scan(lib, None) == 1                                  # dims NULL
+    assert _scan(lib, D(), x=None) == 1
+    assert _scan(lib, D(), y=None) == 1
+    assert _scan(lib, D(L=0)) == 2
+    assert _scan(lib, D(batch=-1)) == 2
+    assert _scan(lib, D(N=17)) == 6
+    assert _scan(lib, D(io=7)) == 4
+    assert _scan(lib, D(), beta=1.0) == 3
+    assert _scan(lib, D(), beta=-0.1) == 3
+    assert _scan(lib, D(), beta=float("nan")) == 3
+    assert _scan(lib, D(), alpha=-1.0) == 3
+    assert _scan(lib, D(), alpha=float("inf")) == 3
+    assert _scan(lib, D(), x=ctypes.c_void_p(A16 + 4)) == 5      # misaligned
+    assert "x is not 16-byte aligned" in mm.mm_last_error()
+
+
+def test_scan_rejects_aliasing(lib):
+    # y on top of delta
+    assert _scan(lib, D(), y=_fake(1)) == 9
+    # hT on top of A (sizes: A = 8*16*4 bytes)
+    assert _scan(lib, D(), hT=_fake(2)) == 9
+    # hT overlapping vT
+    assert _scan(lib, D(), hT=_fake(6), vT=ctypes.c_void_p(A16 * 7 + 64)) == 9
+
+
+def test_scan_fault_injection_returns_cuda_error(lib, monkeypatch):
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    # in-place streaming (hT == h0, vT == v0) is allowed and reaches the launch step
+    rc = _scan(lib, D(), h0=_fake(6), hT=_fake(6), v0=_fake(7), vT=_fake(7))
+    assert rc == 7
+    assert "injected" in mm.mm_last_error()
+
+
+def test_set_tile(lib):
+    assert lib.mm_scan_set_tile(3, 2) == 6
+    assert lib.mm_scan_set_tile(4, 2) == 0
+    assert lib.mm_scan_set_tile(0, 0) == 0
+
+
+def test_ssd_rejects_bad_arguments(lib):
+    dims = mm.SSDDims(1, 512, 4, 64, 128, 1, 256)
+    size = ctypes.c_size_t(0)
+    assert lib.mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == 0
+    assert size.value > 0
+    bad = mm.SSDDims(1, 512, 4, 64, 128, 3, 256)                  # H % G != 0
+    assert lib.mm_ssd_workspace_size(ctypes.byref(bad), ctypes.byref(size)) == 2
+    odd = mm.SSDDims(1, 512, 4, 48, 128, 1, 256)
+    assert lib.mm_ssd_workspace_size(ctypes.byref(odd), ctypes.byref(size)) == 6
+
+    def call(beta=0.0, alpha=1.0, ws=1 << 30, **over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), h0=None,
+                 y=_fake(5), hT=None, w=_fake(8))
+        a.update(over)
+        return lib.mm_ssd_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["h0"], beta, alpha,
+                              a["y"], a["hT"], a["w"], ws, ctypes.byref(dims), None)
+    assert call(x=None) == 1
+    assert call(w=None) == 1
+    assert call(beta=0.5) == 6
+    assert call(beta=1.5) == 3
+    assert call(alpha=-2.0) == 3
+    assert call(ws=16) == 2
+    assert call(y=_fake(0)) == 9
