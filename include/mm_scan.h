@@ -125,9 +125,10 @@ typedef struct {
 
 /*
  * mm_ssd_workspace_size -- bytes of device workspace mm_ssd_fwd needs for
- * these sizes (written to *bytes).  The caller allocates it (any 256-byte
- * aligned device buffer of at least that size) and passes it to every call
- * with the same sizes; the library keeps nothing in it between calls.
+ * these sizes (written to *bytes).  This build needs none (0): the state
+ * never leaves the SM.  When the size is non-zero the caller allocates a
+ * 256-byte aligned device buffer of at least that size and passes it to
+ * every call with the same sizes; nothing is kept in it between calls.
  * Errors: MM_ERR_NULL, MM_ERR_DIMS, MM_ERR_UNSUPPORTED as for mm_ssd_fwd.
  */
 mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
@@ -147,6 +148,13 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
  * chunks, and the read-out of the carried state (tensor-core GEMMs for the
  * three dense steps).
  *
+ * The kernel keeps the state of a (batch row, head) on one SM and walks the
+ * sequence in blocks of 128 rows: each block's diagonal 128 x 128 part of
+ * the masked decay matrix is formed densely; for chunk = 256 the
+ * off-diagonal block of a chunk is applied through its rank-N factors
+ * (the block state), the structured-matrix property the page describes.
+ * Results equal the chunked recurrence up to rounding.
+ *
  * Arguments (device buffers unless noted):
  *   x      (batch, L, H, P)  bf16   input
  *   delta  (batch, L, H)     fp32   step size per head
@@ -158,9 +166,10 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
  *   y      (batch, L, H, P)  bf16   output (round to nearest-even)
  *   hT     (batch, H, P, N)  fp32   final state or NULL; may equal h0
  *   workspace, workspace_bytes      device scratch of at least
- *                                   mm_ssd_workspace_size() bytes
- * Supported sizes: headdim 64, dstate 128, chunk 256 (power of two),
- * seqlen any >= 1, H a multiple of G.
+ *                                   mm_ssd_workspace_size() bytes (may be
+ *                                   NULL when that size is 0)
+ * Supported sizes: headdim 64, dstate 128, chunk 128 or 256, seqlen any
+ * >= 1, H a multiple of G.  All of x, B, C must be 16-byte aligned.
  * Errors: as mm_scan_fwd, plus MM_ERR_DIMS for a workspace that is too
  * small.
  */
@@ -170,6 +179,16 @@ mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
                      void *y, float *hT,
                      void *workspace, size_t workspace_bytes,
                      const mm_ssd_dims *dims, void *stream);
+
+/*
+ * mm_device_status -- synchronise the current device, then report whether
+ * any kernel of this library gave up a bounded device-side wait since the
+ * previous call (MM_ERR_DEVICE_TIMEOUT: the outputs of that call are
+ * incomplete).  Kernels never wait without a limit (2 s); a wait that runs
+ * out records the fact here and the kernel returns.  Clears the record.
+ * MM_ERR_CUDA if the synchronisation itself reports an error.
+ */
+mm_status mm_device_status(void);
 
 /* Static description of a status code (never NULL). */
 const char *mm_status_string(mm_status status);

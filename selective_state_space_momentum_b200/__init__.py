@@ -25,7 +25,7 @@ import threading
 __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
     "mm_scan_fwd", "mm_ssd_fwd", "mm_ssd_workspace_size", "mm_status_string",
-    "mm_last_error", "mm_scan_set_tile", "mm_version",
+    "mm_last_error", "mm_scan_set_tile", "mm_version", "mm_device_status",
     "scan_fwd", "ssd_fwd", "scan_fwd_host", "EXPORTED_SYMBOLS",
 ]
 
@@ -44,8 +44,8 @@ STATUS_NAMES = {
 }
 
 # Every function include/mm_scan.h declares.
-EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_ssd_workspace_size", "mm_ssd_fwd", "mm_status_string",
-                    "mm_last_error", "mm_scan_set_tile", "mm_version")
+EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_ssd_workspace_size", "mm_ssd_fwd", "mm_device_status",
+                    "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
 
 
 class MMError(RuntimeError):
@@ -90,6 +90,8 @@ def _declare(lib):
     lib.mm_scan_set_tile.argtypes = [ctypes.c_int, ctypes.c_int]
     lib.mm_version.restype = ctypes.c_int
     lib.mm_version.argtypes = []
+    lib.mm_device_status.restype = ctypes.c_int
+    lib.mm_device_status.argtypes = []
     return lib
 
 
@@ -192,6 +194,11 @@ def mm_scan_set_tile(states_per_thread: int, warps_per_block: int):
 
 def mm_version() -> int:
     return int(load_library().mm_version())
+
+
+def mm_device_status():
+    """Synchronise the device; raise MMError if a kernel gave up a bounded wait."""
+    _check(load_library().mm_device_status(), "mm_device_status")
 
 
 # ------------------------------------------------------------ wrappers -----

@@ -97,6 +97,15 @@ const char* mm_last_error(void) { return g_last_error.c_str(); }
 
 int mm_version(void) { return 100; }
 
+mm_status mm_device_status(void) {
+    const cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return from_cuda(e, "mm_device_status: synchronize");
+    const unsigned int w = mmscan::scan_read_and_clear_device_error() |
+                           mmscan::ssd_read_and_clear_device_error();
+    if (w) return fail(MM_ERR_DEVICE_TIMEOUT, "a device-side wait ran past its limit (word 0x%x)", w);
+    return ok();
+}
+
 mm_status mm_scan_set_tile(int spt, int warps) {
     if (spt == 0 && warps == 0) {
         g_forced_spt = 0;
@@ -191,11 +200,13 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
                      void* workspace, size_t workspace_bytes, const mm_ssd_dims* dims,
                      void* stream) {
     if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
-    if (!x || !delta || !A || !B || !C || !y || !workspace)
-        return fail(MM_ERR_NULL, "x, delta, A, B, C, y and workspace are required");
+    if (!x || !delta || !A || !B || !C || !y)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
     size_t need = 0;
     mm_status st = mm_ssd_workspace_size(dims, &need);
     if (st != MM_OK) return st;
+    if (need > 0 && !workspace)
+        return fail(MM_ERR_NULL, "a workspace of %zu bytes is required", need);
     if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
         return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
     if (beta != 0.0f)
@@ -240,10 +251,7 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
     a.chunk = dims->chunk; a.alpha = alpha;
-    const cudaError_t e = mmscan::launch_ssd_fwd(a, static_cast<cudaStream_t>(stream));
-    if (e == cudaErrorNotSupported)
-        return fail(MM_ERR_UNSUPPORTED, "the SSD kernels are not part of this build");
-    return from_cuda(e, "mm_ssd_fwd launch");
+    return from_cuda(mmscan::launch_ssd_fwd(a, static_cast<cudaStream_t>(stream)), "mm_ssd_fwd launch");
 }
 
 }  // extern "C"

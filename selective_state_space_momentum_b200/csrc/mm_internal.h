@@ -37,6 +37,9 @@ bool scan_tile_supported(int spt, int warps);
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
                                 int forced_spt, int forced_warps);
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s);
+// Read (and reset) the device error word of the scan / SSD kernels.
+unsigned int scan_read_and_clear_device_error();
+unsigned int ssd_read_and_clear_device_error();
 
 // Arguments of one SSD call.
 struct SSDArgs {

@@ -9,137 +9,136 @@
 //
 // Design (B200-first; the page's CUB two-stage block scan is prior art only):
 //  * Work split.  A CTA owns CH channels of one batch row (B_t and C_t are
-//    shared by all channels of a row) and walks the whole sequence.  Inside
-//    it, G = NP / SPT consecutive lanes share a channel; each lane keeps SPT
-//    consecutive states (v, h) in fp32 registers for the whole call, so the
-//    recurrence runs exactly in time order with no carry recombination.
-//  * Staging.  The sequence is cut into chunks of T steps.  For each chunk
-//    the CTA copies its x and delta rows and the B/C rows of its batch row
-//    into shared memory with cp.async (16-byte, zero-filled past L), three
-//    chunks in flight.  B and C are then transposed to [t][n] in fp32 with
-//    alpha folded into B, so a lane reads its SPT states of one step in one
-//    vector load.
-//  * Arithmetic.  Per step and state: one MUFU ex2 for exp(delta A) (A is
-//    pre-scaled by log2 e), and packed f32x2 multiply / FMA for the write,
-//    the velocity, the hidden state and the read-out, two states per
-//    instruction.  exp of a step is never stored; no (L, D, N) tensor exists.
-//  * Read-out.  Each lane forms its partial C_t . h_t over its SPT states;
-//    the G partials of a channel meet in shared memory and one pass sums
-//    them and writes y with coalesced 16-byte (fp32) or 8-byte (bf16) stores,
-//    rounding to nearest-even for bf16.
-//  * Final state.  (h, v) after the last step are written to hT, vT.  The
-//    per-state operation sequence does not depend on how the sequence is
-//    cut into calls, so split calls reproduce hT, vT bit for bit.
+//    shared by all channels of a row) and walks the whole sequence.  G = NP /
+//    SPT consecutive lanes share a channel; each lane keeps SPT consecutive
+//    states (v, h) in fp32 registers for the whole call, so the recurrence
+//    runs in time order and needs no carry recombination.
+//  * Staging.  The sequence is cut into chunks of T = 64 steps.  One thread
+//    issues TMA tile loads (no multicast) of the chunk's x and delta rows and
+//    of the batch row's B and C into shared memory, 128-byte swizzled, with
+//    three chunks in flight on mbarriers.  TMA zero-fills past L, D and N.
+//    Rows whose byte length is not a multiple of 16 cannot be described to
+//    TMA; for them the same tiles are filled element by element.
+//  * B and C are transposed to [t][n] fp32 (alpha folded into B) in 4x4
+//    blocks, double-buffered, so a lane reads its SPT states of a step with
+//    one vector load and the CTA needs one barrier per chunk.
+//  * Arithmetic, per group of 8 steps: one MUFU ex2 per (step, state) for
+//    exp(delta A) (A pre-scaled by log2 e), and packed f32x2 multiply / FMA
+//    for the write, the velocity, the hidden state and the read-out -- two
+//    states per instruction.  Nothing of size (L, D, N) is ever stored.
+//  * Read-out.  The G lanes of a channel add their partial C_t . h_t through
+//    a small per-warp buffer (no CTA barrier) and store y directly: the G
+//    lanes write G consecutive steps of their channel.
+//  * Final state.  (h, v) after the last step go to hT, vT.  The per-state
+//    operation sequence does not depend on where the sequence is cut into
+//    calls, so split calls reproduce hT, vT bit for bit.
+#include <cuda.h>
+
 #include <atomic>
+#include <mutex>
 
 #include "mm_common.cuh"
 #include "mm_internal.h"
 
 namespace mmscan {
 
+// Device error word of this file's kernels (bounded waits that gave up).
+static __device__ unsigned int g_scan_dev_err = 0;
+
 template <typename IO, int NP, int SPT, int WARPS>
 struct ScanTile {
-    static constexpr int G = NP / SPT;          // lanes per channel
-    static constexpr int CPW = 32 / G;          // channels per warp
-    static constexpr int CH = WARPS * CPW;      // channels per CTA
-    static constexpr int NT = WARPS * 32;       // threads per CTA
-    static constexpr int T = 32;                // steps per chunk
-    static constexpr int STAGES = 3;            // chunks in flight
+    static constexpr int G = NP / SPT;           // lanes per channel
+    static constexpr int CPW = 32 / G;           // channels per warp
+    static constexpr int CH = WARPS * CPW;       // channels per CTA
+    static constexpr int NT = WARPS * 32;        // threads per CTA
+    static constexpr int NPAIR = SPT / 2;
     static constexpr int EB = IOTraits<IO>::kBytes;
-    static constexpr int XP = T + 16 / EB;      // row pitch (elements) of staged rows
-    static constexpr int BP = NP + 4;           // row pitch (floats) of transposed B/C
-    static constexpr int YP = T + 4;            // row pitch (floats) of read-out partials
-    static constexpr int ROWS = 2 * CH + 2 * NP;
-    static constexpr int STAGE_ELEMS = ROWS * XP;
-    static constexpr int STAGE_BYTES = STAGE_ELEMS * EB;
-    static constexpr int BT_FLOATS = T * BP;
-    static constexpr int YPART_FLOATS = CH * G * YP;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + (2 * BT_FLOATS + YPART_FLOATS) * 4;
-    static constexpr int PPR = T * EB / 16;     // 16-byte pieces per staged row
+    static constexpr int BOX_T = 128 / EB;       // steps in one 128-byte swizzled row
+    static constexpr int T = 64;                 // steps per chunk
+    static constexpr int NBOX = T / BOX_T;       // boxes per row per chunk
+    static constexpr int STAGES = 3;             // chunks in flight
+    static constexpr int NPT = NP < 8 ? 8 : NP;  // B/C rows per box (whole swizzle atoms)
+    static constexpr int XBOX = CH * 128;        // bytes of one x (or delta) box
+    static constexpr int BBOX = NPT * 128;       // bytes of one B (or C) box
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_D = NBOX * XBOX;
+    static constexpr int OFF_B = 2 * NBOX * XBOX;
+    static constexpr int OFF_C = OFF_B + NBOX * BBOX;
+    static constexpr int STAGE_BYTES = OFF_C + NBOX * BBOX;
+    static constexpr int TX_BYTES = STAGE_BYTES;  // every box is written in full
+    static constexpr int BP = NP + 4;            // row pitch (floats) of transposed B/C
+    static constexpr int BT_BYTES = T * BP * 4;
+    static constexpr int R = 8;                  // steps per inner group
+    static constexpr int YW_PITCH = R * G + G;   // floats per channel in the read-out buffer
+    static constexpr int YW_BYTES = CPW * YW_PITCH * 4;   // per warp
+    static constexpr int OFF_BT = STAGES * STAGE_BYTES;    // 2 buffers of B^T, then 2 of C^T
+    static constexpr int OFF_YW = OFF_BT + 4 * BT_BYTES;
+    static constexpr int OFF_BAR = OFF_YW + WARPS * YW_BYTES;
+    static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
 
-    static_assert(G >= 1 && (G & (G - 1)) == 0 && 32 % G == 0, "lanes per channel");
-    static_assert(SPT % 2 == 0 && SPT <= 8, "states per lane are processed in pairs");
-    static_assert(T % 4 == 0 && (T * EB) % 16 == 0, "chunk length");
-    static_assert((XP * EB) % 16 == 0 && (STAGE_BYTES % 16) == 0, "16-byte rows");
+    static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "lanes per channel");
+    static_assert(SPT % 2 == 0 && SPT <= 8, "states per lane come in pairs");
+    static_assert(R % G == 0 && BOX_T % R == 0 && T % BOX_T == 0, "step grouping");
+    static_assert(CH % 8 == 0, "x tiles must be whole 1024-byte swizzle atoms");
+    static_assert(STAGE_BYTES % 1024 == 0 && (OFF_BT % 16) == 0, "alignment");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// Copy chunk `k` (steps t0 .. t0+T-1) of the CTA's rows into stage buffer `sbuf`.
-template <typename IO, int NP, int SPT, int WARPS>
-__device__ __forceinline__ void stage_chunk(const ScanArgs& p, IO* sbuf, int64_t b, int64_t d0,
-                                            int64_t t0, int tid) {
-    using TL = ScanTile<IO, NP, SPT, WARPS>;
-    const int64_t L = p.seqlen;
-    const int nval = (int)((L - t0) < TL::T ? (L - t0) : TL::T);
-    const IO* xg = static_cast<const IO*>(p.x);
-    const IO* dg = static_cast<const IO*>(p.delta);
-    const IO* Bg = static_cast<const IO*>(p.B);
-    const IO* Cg = static_cast<const IO*>(p.C);
-
-    // row r -> (global row start, number of valid elements)
-    auto row_src = [&](int r, int& valid) -> const IO* {
-        if (r < 2 * TL::CH) {
-            const int c = r < TL::CH ? r : r - TL::CH;
-            const int64_t d = d0 + c;
-            valid = d < p.dim ? nval : 0;
-            const IO* base = r < TL::CH ? xg : dg;
-            return valid ? base + ((b * p.dim + d) * L + t0) : base;
+// Store `cnt` consecutive steps of one output row.
+template <typename IO>
+__device__ __forceinline__ void store_steps(IO* dst, const float* v, int cnt, bool vec) {
+    if constexpr (sizeof(IO) == 4) {
+        if (vec && cnt == 2) {
+            *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+            return;
         }
-        const int rr = r - 2 * TL::CH;
-        const int n = rr < NP ? rr : rr - NP;
-        valid = n < p.dstate ? nval : 0;
-        const IO* base = rr < NP ? Bg : Cg;
-        return valid ? base + ((b * p.dstate + n) * L + t0) : base;
-    };
-
-    if (p.vec_ok) {
-        constexpr int EPP = 16 / TL::EB;  // elements per 16-byte piece
-        for (int i = tid; i < TL::ROWS * TL::PPR; i += TL::NT) {
-            const int r = i / TL::PPR;
-            const int j = i - r * TL::PPR;
-            int valid;
-            const IO* src = row_src(r, valid);
-            int bytes = (valid - j * EPP) * TL::EB;
-            bytes = bytes < 0 ? 0 : (bytes > 16 ? 16 : bytes);
-            cp_async_16(sbuf + r * TL::XP + j * EPP, bytes ? src + j * EPP : src, bytes);
-        }
-    } else if constexpr (TL::EB == 4) {
-        for (int i = tid; i < TL::ROWS * TL::T; i += TL::NT) {
-            const int r = i / TL::T;
-            const int e = i - r * TL::T;
-            int valid;
-            const IO* src = row_src(r, valid);
-            const bool ok = e < valid;
-            cp_async_4(sbuf + r * TL::XP + e, ok ? src + e : src, ok ? 4 : 0);
+        if (vec && cnt == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+            return;
         }
     } else {
-        // 2-byte elements on rows that are not 4-byte aligned: plain loads.
-        for (int i = tid; i < TL::ROWS * TL::T; i += TL::NT) {
-            const int r = i / TL::T;
-            const int e = i - r * TL::T;
-            int valid;
-            const IO* src = row_src(r, valid);
-            sbuf[r * TL::XP + e] = e < valid ? src[e] : IO(0.0f);
+        if (vec && cnt == 2) {
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v[0], v[1]);
+            return;
+        }
+        if (vec && cnt == 4) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+            return;
         }
     }
 }
 
+template <typename IO, int PER>
+__device__ __forceinline__ void store_steps_n(IO* dst, const float (&v)[PER], int cnt, bool vec) {
+    if (vec && cnt == PER && (PER == 2 || PER == 4)) {
+        store_steps<IO>(dst, v, PER, true);
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        if (i < cnt) store1(dst + i, v[i]);
+}
+
 template <typename IO, int NP, int SPT, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32)
-scan_fwd_kernel(const ScanArgs p) {
+scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
+                const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+                const ScanArgs p) {
     using TL = ScanTile<IO, NP, SPT, WARPS>;
-    constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T;
-    constexpr int ST = TL::STAGES, NPAIR = SPT / 2;
+    constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
+    constexpr int ST = TL::STAGES, NPAIR = TL::NPAIR, EB = TL::EB, BP = TL::BP;
 
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    IO* stages = reinterpret_cast<IO*>(smem_raw);
-    float* Bt = reinterpret_cast<float*>(smem_raw + ST * TL::STAGE_BYTES);
-    float* Ct = Bt + TL::BT_FLOATS;
-    float* ypart = Ct + TL::BT_FLOATS;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (base - raw_addr);
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int g = lane % G;
-    const int c = (tid >> 5) * CPW + lane / G;      // channel within the CTA
+    const int cw = lane / G;
+    const int c = warp * CPW + cw;                   // channel within the CTA
     const int64_t b = blockIdx.x / p.tiles_per_batch;
     const int64_t d0 = (int64_t)(blockIdx.x % p.tiles_per_batch) * CH;
     const int64_t d = d0 + c;
@@ -147,167 +146,273 @@ scan_fwd_kernel(const ScanArgs p) {
     const int64_t L = p.seqlen;
     const int N = p.dstate;
     const int64_t nchunks = (L + T - 1) / T;
+    const bool use_tma = p.vec_ok != 0;
+    const uint32_t bar0 = base + TL::OFF_BAR;
+
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, use_tma ? 1u : (uint32_t)NT);
+        fence_barrier_init();
+    }
+    __syncthreads();
 
     // ---- per-lane constants and state ------------------------------------
-    float A2[SPT];          // A[d, n] * log2 e
+    float2 A2p[SPT];        // (A[d,n] log2 e) twice, for two steps at once
     float2 vv[NPAIR], hh[NPAIR];
 #pragma unroll
     for (int s = 0; s < SPT; ++s) {
         const int n = g * SPT + s;
-        A2[s] = (active && n < N) ? p.A[d * N + n] * kLog2e : 0.0f;
+        const float a2 = (active && n < N) ? p.A[d * N + n] * kLog2e : 0.0f;
+        A2p[s] = f2(a2, a2);
     }
 #pragma unroll
     for (int q = 0; q < NPAIR; ++q) {
-        float hv[2] = {0.0f, 0.0f}, vvv[2] = {0.0f, 0.0f};
+        float hv[2] = {0.0f, 0.0f}, vw[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int n = g * SPT + 2 * q + e;
             if (active && n < N) {
-                const int64_t si = ((b * p.dim + d) * N + n);
+                const int64_t si = (b * p.dim + d) * N + n;
                 if (p.h0) hv[e] = p.h0[si];
-                if (p.v0) vvv[e] = p.v0[si];
+                if (p.v0) vw[e] = p.v0[si];
             }
         }
         hh[q] = f2(hv[0], hv[1]);
-        vv[q] = f2(vvv[0], vvv[1]);
+        vv[q] = f2(vw[0], vw[1]);
     }
     const float2 beta2 = f2(p.beta, p.beta);
     const float alpha = p.alpha;
-    float2 A2p[SPT];        // (A2[s], A2[s]) for two steps at once
-#pragma unroll
-    for (int s = 0; s < SPT; ++s) A2p[s] = f2(A2[s], A2[s]);
 
-    // ---- pipeline prologue -----------------------------------------------
+    // ---- staging of one chunk into a stage buffer --------------------------
+    auto issue = [&](int64_t k, int s) {
+        const int64_t t0 = k * T;
+        const uint32_t sb = base + s * TL::STAGE_BYTES;
+        const uint32_t bar = bar0 + 8 * s;
+        if (use_tma) {
+            if (tid == 0) {
+                mbar_expect_tx(bar, TL::TX_BYTES);
 #pragma unroll
-    for (int s = 0; s < ST - 1; ++s) {
-        if (s < nchunks)
-            stage_chunk<IO, NP, SPT, WARPS>(p, stages + s * TL::STAGE_ELEMS, b, d0, (int64_t)s * T, tid);
-        cp_async_commit();
-    }
+                for (int bx = 0; bx < TL::NBOX; ++bx) {
+                    const int tc = (int)(t0 + bx * TL::BOX_T);
+                    tma_load_3d(sb + TL::OFF_X + bx * TL::XBOX, &tm_x, bar, tc, (int)d0, (int)b);
+                    tma_load_3d(sb + TL::OFF_D + bx * TL::XBOX, &tm_d, bar, tc, (int)d0, (int)b);
+                    tma_load_3d(sb + TL::OFF_B + bx * TL::BBOX, &tm_B, bar, tc, 0, (int)b);
+                    tma_load_3d(sb + TL::OFF_C + bx * TL::BBOX, &tm_C, bar, tc, 0, (int)b);
+                }
+            }
+            return;
+        }
+        // Element-wise fill of the same swizzled tiles (rows not 16-byte multiples).
+        const IO* xg = static_cast<const IO*>(p.x);
+        const IO* dg = static_cast<const IO*>(p.delta);
+        const IO* Bg = static_cast<const IO*>(p.B);
+        const IO* Cg = static_cast<const IO*>(p.C);
+        constexpr int ROWS = 2 * CH + 2 * TL::NPT;
+        for (int i = tid; i < ROWS * T; i += NT) {
+            const int r = i / T;
+            const int tau = i - r * T;
+            const int bx = tau / TL::BOX_T;
+            const int col = tau - bx * TL::BOX_T;
+            const int64_t t = t0 + tau;
+            const IO* src = nullptr;
+            uint32_t off;
+            if (r < 2 * CH) {
+                const int cc = r < CH ? r : r - CH;
+                off = (r < CH ? TL::OFF_X : TL::OFF_D) + bx * TL::XBOX + sw128(cc, col * EB);
+                if (d0 + cc < p.dim && t < L) src = (r < CH ? xg : dg) + ((b * p.dim + d0 + cc) * L + t);
+            } else {
+                const int rr = r - 2 * CH;
+                const int n = rr < TL::NPT ? rr : rr - TL::NPT;
+                off = (rr < TL::NPT ? TL::OFF_B : TL::OFF_C) + bx * TL::BBOX + sw128(n, col * EB);
+                if (n < N && t < L) src = (rr < TL::NPT ? Bg : Cg) + ((b * N + n) * L + t);
+            }
+            if constexpr (EB == 4) {
+                cp_async_4(smem + s * TL::STAGE_BYTES + off, src ? src : xg, src ? 4 : 0);
+            } else {
+                *reinterpret_cast<IO*>(smem + s * TL::STAGE_BYTES + off) = src ? *src : IO(0.0f);
+            }
+        }
+        if constexpr (EB == 4) cp_async_mbar_arrive(bar);
+        else mbar_arrive(bar);
+    };
+
+    // ---- pipeline prologue ---------------------------------------------------
+#pragma unroll
+    for (int s = 0; s < ST - 1; ++s)
+        if (s < nchunks) issue(s, s);
+
+    float* yw = reinterpret_cast<float*>(smem + TL::OFF_YW + warp * TL::YW_BYTES) + cw * TL::YW_PITCH;
+    IO* yrow = static_cast<IO*>(p.y) + (b * p.dim + (active ? d : 0)) * L;
+    const bool vec_out = use_tma;
 
     for (int64_t k = 0; k < nchunks; ++k) {
-        const int buf = (int)(k % ST);
+        const int s = (int)(k % ST);
         const int64_t t0 = k * T;
         const int nval = (int)((L - t0) < T ? (L - t0) : T);
-        cp_async_wait<ST - 2>();
-        __syncthreads();
+        if (!mbar_wait(bar0 + 8 * s, (uint32_t)((k / ST) & 1), &g_scan_dev_err)) return;
+        const unsigned char* sbuf = smem + s * TL::STAGE_BYTES;
+        float* Bt = reinterpret_cast<float*>(smem + TL::OFF_BT + (int)(k & 1) * TL::BT_BYTES);
+        float* Ct = reinterpret_cast<float*>(smem + TL::OFF_BT + (2 + (int)(k & 1)) * TL::BT_BYTES);
+
+        // ---- transpose B, C to [t][n] fp32 in 4x4 blocks (alpha into B) ----
         {
-            const int64_t kn = k + ST - 1;
-            if (kn < nchunks)
-                stage_chunk<IO, NP, SPT, WARPS>(p, stages + (int)(kn % ST) * TL::STAGE_ELEMS, b, d0,
-                                                kn * T, tid);
-            cp_async_commit();
-        }
-        const IO* sb = stages + buf * TL::STAGE_ELEMS;
-
-        // ---- transpose B, C to [t][n] fp32 (alpha folded into B) ---------
-        {
-            const IO* Braw = sb + 2 * CH * TL::XP;
-            const IO* Craw = Braw + NP * TL::XP;
-            constexpr int PER = NP * (T / 4);
-            for (int i = tid; i < 2 * PER; i += NT) {
-                const int which = i / PER;
-                const int rem = i - which * PER;
-                const int n = rem % NP;
-                const int t4 = (rem / NP) * 4;
-                const IO* src = (which ? Craw : Braw) + n * TL::XP + t4;
-                float4 v4 = load4(src);
-                if (!which) {
-                    v4.x *= alpha; v4.y *= alpha; v4.z *= alpha; v4.w *= alpha;
-                }
-                float* dst = (which ? Ct : Bt) + t4 * TL::BP + n;
-                dst[0] = v4.x;
-                dst[TL::BP] = v4.y;
-                dst[2 * TL::BP] = v4.z;
-                dst[3 * TL::BP] = v4.w;
-            }
-        }
-        __syncthreads();
-
-        // ---- the recurrence over this chunk -------------------------------
-        {
-            const IO* xrow = sb + c * TL::XP;
-            const IO* drow = sb + (CH + c) * TL::XP;
-            float* yrow = ypart + (c * G + g) * TL::YP;
-            const float* Bg = Bt + g * SPT;
-            const float* Cg = Ct + g * SPT;
-
-            auto step = [&](int t, float u, const float* a) -> float {
-                const float2 uu = f2(u, u);
-                float2 yy = f2(0.0f, 0.0f);
+            constexpr int NB4 = NP / 4 > 0 ? NP / 4 : 1;
+            constexpr int ITEMS = NB4 * (T / 4);
+            for (int i = tid; i < 2 * ITEMS; i += NT) {
+                const int which = i / ITEMS;
+                const int rem = i - which * ITEMS;
+                const int n0 = (rem % NB4) * 4;
+                const int t4 = (rem / NB4) * 4;
+                const int bx = t4 / TL::BOX_T;
+                const int col = t4 - bx * TL::BOX_T;
+                const unsigned char* tile = sbuf + (which ? TL::OFF_C : TL::OFF_B) + bx * TL::BBOX;
+                float m[4][4];   // m[row n][step]
 #pragma unroll
-                for (int q = 0; q < NPAIR; ++q) {
-                    const float2 bq = *reinterpret_cast<const float2*>(Bg + t * TL::BP + 2 * q);
-                    const float2 cq = *reinterpret_cast<const float2*>(Cg + t * TL::BP + 2 * q);
-                    const float2 w = __fmul2_rn(uu, bq);
-                    vv[q] = __ffma2_rn(beta2, vv[q], w);
-                    hh[q] = __ffma2_rn(f2(a[2 * q], a[2 * q + 1]), hh[q], vv[q]);
-                    yy = __ffma2_rn(cq, hh[q], yy);
+                for (int r = 0; r < 4; ++r) {
+                    if (n0 + r < NP) {
+                        const float4 q = load4(reinterpret_cast<const IO*>(tile + sw128(n0 + r, col * EB)));
+                        m[r][0] = q.x; m[r][1] = q.y; m[r][2] = q.z; m[r][3] = q.w;
+                    } else {
+                        m[r][0] = m[r][1] = m[r][2] = m[r][3] = 0.0f;
+                    }
                 }
-                return yy.x + yy.y;
-            };
-
-            const int nfull = nval & ~3;
-#pragma unroll 2
-            for (int tau = 0; tau < nfull; tau += 4) {
-                const float4 dq = load4(drow + tau);
-                const float4 xq = load4(xrow + tau);
-                const float2 u01 = __fmul2_rn(f2(dq.x, dq.y), f2(xq.x, xq.y));
-                const float2 u23 = __fmul2_rn(f2(dq.z, dq.w), f2(xq.z, xq.w));
-                float a0[SPT], a1[SPT], a2[SPT], a3[SPT];
+                const float sc = which ? 1.0f : alpha;
+                float* dst = (which ? Ct : Bt) + t4 * BP + n0;
 #pragma unroll
-                for (int s = 0; s < SPT; ++s) {
-                    const float2 r01 = __fmul2_rn(f2(dq.x, dq.y), A2p[s]);
-                    const float2 r23 = __fmul2_rn(f2(dq.z, dq.w), A2p[s]);
-                    a0[s] = ex2_approx(r01.x);
-                    a1[s] = ex2_approx(r01.y);
-                    a2[s] = ex2_approx(r23.x);
-                    a3[s] = ex2_approx(r23.y);
-                }
-                float4 yo;
-                yo.x = step(tau + 0, u01.x, a0);
-                yo.y = step(tau + 1, u01.y, a1);
-                yo.z = step(tau + 2, u23.x, a2);
-                yo.w = step(tau + 3, u23.y, a3);
-                *reinterpret_cast<float4*>(yrow + tau) = yo;
-            }
-            if (nfull < nval) {   // ragged last steps of the sequence (uniform)
-                for (int t = nfull; t < nval; ++t) {
-                    const float dt = load1(drow + t);
-                    const float u = dt * load1(xrow + t);
-                    float a[SPT];
-#pragma unroll
-                    for (int s = 0; s < SPT; ++s) a[s] = ex2_approx(dt * A2[s]);
-                    yrow[t] = step(t, u, a);
+                for (int j = 0; j < 4; ++j) {
+                    if constexpr (NP >= 4) {
+                        *reinterpret_cast<float4*>(dst + j * BP) =
+                            make_float4(m[0][j] * sc, m[1][j] * sc, m[2][j] * sc, m[3][j] * sc);
+                    } else {
+                        dst[j * BP] = m[0][j] * sc;
+                        dst[j * BP + 1] = m[1][j] * sc;
+                    }
                 }
             }
         }
         __syncthreads();
+        // Every thread is past compute(k-1): its stage and B^T/C^T buffers are free.
+        if (k + ST - 1 < nchunks) issue(k + ST - 1, (int)((k + ST - 1) % ST));
 
-        // ---- sum the G partials of each channel and store y -------------
-        {
-            IO* yg = static_cast<IO*>(p.y);
-            constexpr int Q4 = T / 4;
-            for (int i = tid; i < CH * Q4; i += NT) {
-                const int cc = i / Q4;
-                const int t4 = (i - cc * Q4) * 4;
-                const int64_t dd = d0 + cc;
-                if (dd >= p.dim || t4 >= nval) continue;
-                const float* src = ypart + cc * G * TL::YP + t4;
-                float4 s4 = *reinterpret_cast<const float4*>(src);
+        // ---- the recurrence over this chunk, R steps at a time -------------
+        const float* Bg = Bt + g * SPT;
+        const float* Cg = Ct + g * SPT;
+        const int ngroups = (nval + R - 1) / R;
+        for (int gi = 0; gi < ngroups; ++gi) {
+            const int tau0 = gi * R;
+            const int kmax = nval - tau0 < R ? nval - tau0 : R;
+            const int bx = tau0 / TL::BOX_T;
+            const int col = tau0 - bx * TL::BOX_T;
+            const unsigned char* xt = sbuf + TL::OFF_X + bx * TL::XBOX;
+            const unsigned char* dtl = sbuf + TL::OFF_D + bx * TL::XBOX;
+            float dl[R], xl[R];
 #pragma unroll
-                for (int gg = 1; gg < G; ++gg) {
-                    const float4 o = *reinterpret_cast<const float4*>(src + gg * TL::YP);
-                    s4.x += o.x; s4.y += o.y; s4.z += o.z; s4.w += o.w;
-                }
-                IO* dst = yg + ((b * p.dim + dd) * L + t0 + t4);
-                if (p.vec_ok && t4 + 4 <= nval) {
-                    store4(dst, s4);
-                } else {
-                    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-                    for (int e = 0; e < 4 && t4 + e < nval; ++e) store1(dst + e, sv[e]);
+            for (int j = 0; j < R; j += 4) {
+                const float4 dq = load4(reinterpret_cast<const IO*>(dtl + sw128(c, (col + j) * EB)));
+                const float4 xq = load4(reinterpret_cast<const IO*>(xt + sw128(c, (col + j) * EB)));
+                dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
+                xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
+            }
+            float u[R];
+#pragma unroll
+            for (int j = 0; j < R; j += 2) {
+                const float2 uu = __fmul2_rn(f2(dl[j], dl[j + 1]), f2(xl[j], xl[j + 1]));
+                u[j] = uu.x;
+                u[j + 1] = uu.y;
+            }
+            float a[R][SPT];
+#pragma unroll
+            for (int sI = 0; sI < SPT; ++sI) {
+#pragma unroll
+                for (int j = 0; j < R; j += 2) {
+                    const float2 r2 = __fmul2_rn(f2(dl[j], dl[j + 1]), A2p[sI]);
+                    a[j][sI] = ex2_approx(r2.x);
+                    a[j + 1][sI] = ex2_approx(r2.y);
                 }
             }
+            float yk[R];
+            if (kmax == R) {
+#pragma unroll
+                for (int j = 0; j < R; ++j) {
+                    const float* brow = Bg + (tau0 + j) * BP;
+                    const float* crow = Cg + (tau0 + j) * BP;
+                    float bq[SPT], cq[SPT];
+#pragma unroll
+                    for (int q = 0; q < SPT; q += 4 > SPT ? SPT : 4) {
+                        if constexpr (SPT >= 4) {
+                            const float4 b4 = *reinterpret_cast<const float4*>(brow + q);
+                            const float4 c4 = *reinterpret_cast<const float4*>(crow + q);
+                            bq[q] = b4.x; bq[q + 1] = b4.y; bq[q + 2] = b4.z; bq[q + 3] = b4.w;
+                            cq[q] = c4.x; cq[q + 1] = c4.y; cq[q + 2] = c4.z; cq[q + 3] = c4.w;
+                        } else {
+                            const float2 b2 = *reinterpret_cast<const float2*>(brow + q);
+                            const float2 c2 = *reinterpret_cast<const float2*>(crow + q);
+                            bq[q] = b2.x; bq[q + 1] = b2.y;
+                            cq[q] = c2.x; cq[q + 1] = c2.y;
+                        }
+                    }
+                    const float2 uu = f2(u[j], u[j]);
+                    float2 yy = f2(0.0f, 0.0f);
+#pragma unroll
+                    for (int q = 0; q < NPAIR; ++q) {
+                        const float2 w = __fmul2_rn(uu, f2(bq[2 * q], bq[2 * q + 1]));
+                        vv[q] = __ffma2_rn(beta2, vv[q], w);
+                        hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
+                        yy = __ffma2_rn(f2(cq[2 * q], cq[2 * q + 1]), hh[q], yy);
+                    }
+                    yk[j] = yy.x + yy.y;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < R; ++j) {       // ragged end of the sequence
+                    yk[j] = 0.0f;
+                    if (j < kmax) {
+                        const float* brow = Bg + (tau0 + j) * BP;
+                        const float* crow = Cg + (tau0 + j) * BP;
+                        const float2 uu = f2(u[j], u[j]);
+                        float2 yy = f2(0.0f, 0.0f);
+#pragma unroll
+                        for (int q = 0; q < NPAIR; ++q) {
+                            const float2 w = __fmul2_rn(uu, f2(brow[2 * q], brow[2 * q + 1]));
+                            vv[q] = __ffma2_rn(beta2, vv[q], w);
+                            hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
+                            yy = __ffma2_rn(f2(crow[2 * q], crow[2 * q + 1]), hh[q], yy);
+                        }
+                        yk[j] = yy.x + yy.y;
+                    }
+                }
+            }
+
+            // ---- add the G partials of each channel; store y -------------
+            constexpr int PER = R / G;      // steps each lane finishes
+            float out[PER];
+            if constexpr (G == 1) {
+#pragma unroll
+                for (int j = 0; j < R; ++j) out[j] = yk[j];
+            } else {
+#pragma unroll
+                for (int j = 0; j < R; ++j) yw[j * G + g] = yk[j];
+                __syncwarp();
+#pragma unroll
+                for (int e = 0; e < PER; ++e) {
+                    const float* src = yw + (g * PER + e) * G;
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int gg = 0; gg < G; gg += (G >= 4 ? 4 : G)) {
+                        if constexpr (G >= 4) {
+                            const float4 q4 = *reinterpret_cast<const float4*>(src + gg);
+                            acc += (q4.x + q4.y) + (q4.z + q4.w);
+                        } else {
+                            const float2 q2 = *reinterpret_cast<const float2*>(src + gg);
+                            acc += q2.x + q2.y;
+                        }
+                    }
+                    out[e] = acc;
+                }
+                __syncwarp();
+            }
+            const int first = tau0 + g * PER;      // step (within the chunk) of out[0]
+            const int cnt = nval - first < PER ? nval - first : PER;
+            if (active && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
         }
     }
 
@@ -319,7 +424,7 @@ scan_fwd_kernel(const ScanArgs p) {
             for (int e = 0; e < 2; ++e) {
                 const int n = g * SPT + 2 * q + e;
                 if (n < N) {
-                    const int64_t si = ((b * p.dim + d) * N + n);
+                    const int64_t si = (b * p.dim + d) * N + n;
                     if (p.hT) p.hT[si] = e ? hh[q].y : hh[q].x;
                     if (p.vT) p.vT[si] = e ? vv[q].y : vv[q].x;
                 }
@@ -331,13 +436,61 @@ scan_fwd_kernel(const ScanArgs p) {
 // ------------------------------------------------------------- launch -----
 namespace {
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 3-D tiled map over a (d2, d1, d0 = innermost) tensor, 128-byte swizzle.
+cudaError_t make_map_3d(CUtensorMap* m, const void* base, bool bf16_elems, uint64_t d0n, uint64_t d1n,
+                        uint64_t d2n, uint32_t box0, uint32_t box1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const uint64_t eb = bf16_elems ? 2 : 4;
+    const cuuint64_t dims[3] = {d0n, d1n, d2n};
+    const cuuint64_t strides[2] = {d0n * eb, d0n * d1n * eb};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, bf16_elems ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <typename IO, int NP, int SPT, int WARPS>
 cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
     using TL = ScanTile<IO, NP, SPT, WARPS>;
     ScanArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t grid = a.batch * a.tiles_per_batch;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (grid > 0x7fffffffLL || a.dim > 0x7fffffffLL || a.batch > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    CUtensorMap mx, md, mB, mC;
+    memset(&mx, 0, sizeof(mx)); memset(&md, 0, sizeof(md));
+    memset(&mB, 0, sizeof(mB)); memset(&mC, 0, sizeof(mC));
+    if (a.vec_ok) {
+        const bool bf = sizeof(IO) == 2;
+        const uint64_t L = (uint64_t)a.seqlen;
+        cudaError_t e;
+        if ((e = make_map_3d(&mx, a.x, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&md, a.delta, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
+    }
     auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS>;
     // The dynamic shared-memory limit is raised once per device and variant.
     static std::atomic<uint64_t> attr_done{0};
@@ -350,63 +503,68 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_done.fetch_or(bit, std::memory_order_release);
     }
-    kern<<<(unsigned)grid, TL::NT, TL::SMEM_BYTES, stream>>>(a);
+    kern<<<(unsigned)grid, TL::NT, TL::SMEM_BYTES, stream>>>(mx, md, mB, mC, a);
     return cudaGetLastError();
 }
 
-template <typename IO, int NP>
-cudaError_t launch_np(const ScanArgs& a, int spt, int warps, cudaStream_t s) {
-    if constexpr (NP >= 4) {
-        if (spt == 4) {
-            if (warps == 1) return launch_variant<IO, NP, 4, 1>(a, s);
-            if (warps == 2) return launch_variant<IO, NP, 4, 2>(a, s);
-            if (warps == 4) return launch_variant<IO, NP, 4, 4>(a, s);
-        }
-    }
-    if (spt == 2) {
-        if (warps == 1) return launch_variant<IO, NP, 2, 1>(a, s);
-        if (warps == 2) return launch_variant<IO, NP, 2, 2>(a, s);
-        if (warps == 4) return launch_variant<IO, NP, 2, 4>(a, s);
-    }
-    return cudaErrorInvalidValue;
-}
-
+// Variants that are built: (states per lane, warps per CTA) for 16 padded states,
+// and the natural choices for smaller state counts.
 template <typename IO>
 cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, cudaStream_t s) {
     switch (np) {
-        case 2: return launch_np<IO, 2>(a, 2, warps, s);
-        case 4: return launch_np<IO, 4>(a, spt, warps, s);
-        case 8: return launch_np<IO, 8>(a, spt, warps, s);
-        case 16: return launch_np<IO, 16>(a, spt, warps, s);
-        default: return cudaErrorInvalidValue;
+        case 16:
+            if (spt == 2 && warps == 2) return launch_variant<IO, 16, 2, 2>(a, s);
+            if (spt == 2 && warps == 4) return launch_variant<IO, 16, 2, 4>(a, s);
+            if (spt == 2 && warps == 8) return launch_variant<IO, 16, 2, 8>(a, s);
+            if (spt == 4 && warps == 1) return launch_variant<IO, 16, 4, 1>(a, s);
+            if (spt == 4 && warps == 2) return launch_variant<IO, 16, 4, 2>(a, s);
+            if (spt == 4 && warps == 4) return launch_variant<IO, 16, 4, 4>(a, s);
+            break;
+        case 8:
+            if (spt == 2) return launch_variant<IO, 8, 2, 2>(a, s);
+            return launch_variant<IO, 8, 4, 2>(a, s);
+        case 4:
+            return launch_variant<IO, 4, 2, 2>(a, s);
+        case 2:
+            return launch_variant<IO, 2, 2, 1>(a, s);
+        default:
+            break;
     }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 bool scan_tile_supported(int spt, int warps) {
-    return (spt == 2 || spt == 4) && (warps == 1 || warps == 2 || warps == 4);
+    return (spt == 2 && (warps == 2 || warps == 4 || warps == 8)) ||
+           (spt == 4 && (warps == 1 || warps == 2 || warps == 4));
 }
 
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
                                 int forced_spt, int forced_warps) {
+    (void)batch; (void)dim; (void)io;
     ScanTileChoice t;
     t.np = dstate <= 2 ? 2 : dstate <= 4 ? 4 : dstate <= 8 ? 8 : 16;
-    if (forced_spt) {
+    t.spt = 2;
+    t.warps = 4;
+    if (t.np == 16 && forced_spt) {
         t.spt = forced_spt;
         t.warps = forced_warps;
-    } else {
-        (void)batch; (void)dim; (void)io;
-        t.spt = 4;
-        t.warps = 2;
     }
-    if (t.np == 2) t.spt = 2;
+    if (t.np == 8 && forced_spt) t.spt = forced_spt;
     return t;
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s) {
     if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, s);
     return launch_io<bf16>(a, t.np, t.spt, t.warps, s);
+}
+
+unsigned int scan_read_and_clear_device_error() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_scan_dev_err, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_scan_dev_err, &z, sizeof(z));
+    return v;
 }
 
 }  // namespace mmscan

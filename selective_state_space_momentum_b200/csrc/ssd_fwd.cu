@@ -1,19 +1,452 @@
-// ssd_fwd.cu -- Mamba-2 scalar-A chunked (SSD) forward on sm_100a.
+// ssd_fwd.cu -- Mamba-2 scalar-A multi-head scan through the chunked (SSD)
+// algorithm on sm_100a tensor cores (tcgen05 / TMEM).
+//
+// What it computes ("Mamba-2 -- SSM = structured matrix multiply", "4-Step
+// Algorithm" and "Multi-Head Expansion"; first-order discretization
+// B_bar = delta B as on the Momentum Mamba page), for batch row b, head h
+// (group g = h / (H/G)), head channel p, state n:
+//     h_t[p, n] = exp(delta_t A_h) h_{t-1}[p, n] + alpha delta_t B_t[n] x_t[p]
+//     y_t[p]    = sum_n C_t[n] h_t[p, n]
+//
+// Design.  One persistent CTA per (b, h) walks the sequence in blocks of
+// 128 rows, so the state S (N x P = 128 x 64, fp32) never leaves the SM.
+// For a block with in-block cumulative log-decay cs_i = sum_{t<=i} delta_t A_h:
+//  1. intra-block:  CB = C . B^T (128 x 128, K = N) on the tensor core into
+//     TMEM; the compute warps turn it into the masked, decayed matrix
+//     M_ij = CB_ij exp(cs_i - cs_j) alpha delta_j (j <= i), written back into
+//     TMEM as bf16 pairs, and Y_diag = M . X runs with A read from TMEM.
+//  2. block state:  s = B^T . (w o X), w_j = exp(cs_last - cs_j) alpha delta_j.
+//  3. inter-block:  S <- exp(cs_last) S + s, in registers of the compute
+//     warps (thread n holds row n of S).
+//  4. output:       Y_off = C . S_prev^T on the tensor core with S_prev in
+//     shared memory as bf16; y = Y_diag + exp(cs_i) Y_off, stored as bf16.
+// A chunk of Q = 256 rows is processed as two such blocks: its two diagonal
+// 128 x 128 blocks of the masked matrix are formed densely and its
+// off-diagonal block, which is rank <= N (the semiseparable structure the
+// page describes), is applied through the block state of step 2-4.  The
+// result is the same chunked recurrence up to rounding.
+//
+// Roles (6 warps): warp 4 issues TMA loads (no multicast) of X, B, C blocks
+// into a 2-deep ring; warp 5 issues all tcgen05.mma; warps 0-3 own TMEM
+// lanes 0-127 and do the element-wise work.  Every wait is an mbarrier wait
+// bounded by kWaitLimitNs; on give-up the kernel records the fact and every
+// role leaves its loop, TMEM is freed and the kernel returns.
+#include <cuda.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "mm_common.cuh"
 #include "mm_internal.h"
 
 namespace mmscan {
 
+static __device__ unsigned int g_ssd_dev_err = 0;
+
+namespace ssd {
+constexpr int P = 64;                 // head dimension
+constexpr int NS = 128;               // states
+constexpr int UB = 128;               // rows per block
+constexpr int NCOMP = 128;            // compute threads (warps 0-3)
+constexpr int NTHREADS = NCOMP + 64;  // + producer warp + MMA warp
+constexpr int X_TILE = UB * P * 2;          // 16 KB: [128 rows][64] bf16, swizzled
+constexpr int BC_SLAB = UB * 64 * 2;        // 16 KB: [128 rows][64 states]
+constexpr int BC_TILE = 2 * BC_SLAB;        // 32 KB
+constexpr int SLOT = X_TILE + 2 * BC_TILE;  // 80 KB: X, B, C of one block
+constexpr int OFF_XHAT = 2 * SLOT;
+constexpr int S_SLAB = P * 64 * 2;          // 8 KB: [64 rows p][64 states]
+constexpr int S_TILE = 2 * S_SLAB;          // 16 KB
+constexpr int OFF_S = OFF_XHAT + X_TILE;    // 2 S buffers
+constexpr int OFF_CS = OFF_S + 2 * S_TILE;  // cs[2][128] fp32
+constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha*delta[2][128]
+constexpr int OFF_RED = OFF_DA + 2 * UB * 4;
+constexpr int OFF_BAR = OFF_RED + 64;
+constexpr int NBAR = 16;
+constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
+constexpr int OFF_ABORT = OFF_TSLOT + 8;
+constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+// TMEM columns: CB/M + Y_diag for two blocks, Y_off for two blocks, block state.
+__device__ __forceinline__ uint32_t tm_cb(int k) { return (uint32_t)k * 128u; }        // 0, 128
+__device__ __forceinline__ uint32_t tm_yoff(int k) { return 256u + (uint32_t)k * 64u; }  // 256, 320
+constexpr uint32_t TM_STATE = 384;
+constexpr uint32_t TM_COLS = 512;
+// barriers
+enum { B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_TFREE = 10,
+       B_XHAT = 12, B_STATE = 13, B_SFREE = 14, B_SREADY = 15 };
+constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
+constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . Xhat (both MN-major)
+constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // M(tmem) . X (X MN-major)
+constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 0);   // C . S^T
+}  // namespace ssd
+
+struct SSDKArgs {
+    const float* delta;
+    const float* A;
+    const float* h0;
+    bf16* y;
+    float* hT;
+    int64_t batch, seqlen, nheads, ngroups;
+    int nblocks;
+    float alpha;
+};
+
+__global__ void __launch_bounds__(ssd::NTHREADS, 1)
+ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
+               const __grid_constant__ CUtensorMap tm_C, const SSDKArgs p) {
+    using namespace ssd;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (base - raw_addr);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t b = blockIdx.x / p.nheads;
+    const int64_t h = blockIdx.x % p.nheads;
+    const int64_t g = h / (p.nheads / p.ngroups);
+    const int64_t L = p.seqlen;
+    const int nblk = p.nblocks;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    auto bar = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
+
+    if (tid == 0) {
+        mbar_init(bar(B_FULL + 0), 1); mbar_init(bar(B_FULL + 1), 1);
+        mbar_init(bar(B_EMPTY + 0), 1); mbar_init(bar(B_EMPTY + 1), 1);
+        mbar_init(bar(B_CB + 0), 1); mbar_init(bar(B_CB + 1), 1);
+        mbar_init(bar(B_M + 0), NCOMP); mbar_init(bar(B_M + 1), NCOMP);
+        mbar_init(bar(B_Y + 0), 1); mbar_init(bar(B_Y + 1), 1);
+        mbar_init(bar(B_TFREE + 0), NCOMP); mbar_init(bar(B_TFREE + 1), NCOMP);
+        mbar_init(bar(B_XHAT), NCOMP);
+        mbar_init(bar(B_STATE), 1);
+        mbar_init(bar(B_SFREE), NCOMP);
+        mbar_init(bar(B_SREADY), NCOMP);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(base + OFF_TSLOT, TM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT);
+
+    auto wait = [&](int i, uint32_t parity) -> bool {
+        if (*abort_flag) return false;
+        if (!mbar_wait(bar(i), parity, &g_ssd_dev_err)) {
+            *abort_flag = 1;
+            return false;
+        }
+        return true;
+    };
+
+    if (warp == 4) {
+        // ------------------------------------------------------ producer ----
+        if (lane == 0) {
+            for (int u = 0; u < nblk; ++u) {
+                const int s = u & 1;
+                if (!wait(B_EMPTY + s, (uint32_t)(((u >> 1) + 1) & 1))) break;
+                const uint32_t slot = base + s * SLOT;
+                const uint32_t fb = bar(B_FULL + s);
+                mbar_expect_tx(fb, SLOT);
+                const int t0 = u * UB;
+                tma_load_4d(slot, &tm_x, fb, 0, (int)h, t0, (int)b);
+                tma_load_4d(slot + X_TILE, &tm_B, fb, 0, (int)g, t0, (int)b);
+                tma_load_4d(slot + X_TILE + BC_SLAB, &tm_B, fb, 64, (int)g, t0, (int)b);
+                tma_load_4d(slot + X_TILE + BC_TILE, &tm_C, fb, 0, (int)g, t0, (int)b);
+                tma_load_4d(slot + X_TILE + BC_TILE + BC_SLAB, &tm_C, fb, 64, (int)g, t0, (int)b);
+            }
+        }
+    } else if (warp == 5) {
+        // ----------------------------------------------------------- MMA ----
+        if (lane == 0) {
+            const uint32_t xhat = base + OFF_XHAT;
+            for (int u = 0; u < nblk; ++u) {
+                const int s = u & 1, k = u & 1;
+                const uint32_t slot = base + s * SLOT;
+                const uint32_t xs = slot, bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
+                if (!wait(B_FULL + s, (uint32_t)((u >> 1) & 1))) break;
+                if (!wait(B_TFREE + k, (uint32_t)(((u >> 1) + 1) & 1))) break;
+                tc_fence_after();
+                // 1. CB = C . B^T: M = 128 rows i, N = 128 rows j, K = 128 states
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
+                    umma_ss(tmem + tm_cb(k), umma_desc_sw128(cs + koff, 16, 1024),
+                            umma_desc_sw128(bs + koff, 16, 1024), ID_CB, ks > 0);
+                }
+                umma_commit(bar(B_CB + k));
+                // 2. block state = B^T . Xhat: M = 128 states, N = 64, K = 128 rows
+                if (!wait(B_XHAT, (uint32_t)(u & 1))) break;
+                if (!wait(B_SFREE, (uint32_t)((u + 1) & 1))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ss(tmem + TM_STATE, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
+                            umma_desc_sw128(xhat + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
+                umma_commit(bar(B_STATE));
+                // 3. Y_diag = M(tmem) . X and Y_off = C . S_prev^T
+                if (!wait(B_M + k, (uint32_t)((u >> 1) & 1))) break;
+                if (!wait(B_SREADY, (uint32_t)(u & 1))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ts(tmem + tm_cb(k) + 64, tmem + tm_cb(k) + ks * 8,
+                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
+                const uint32_t sb = base + OFF_S + (u & 1) * S_TILE;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff_c = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
+                    const uint32_t koff_s = (ks >> 2) * S_SLAB + (ks & 3) * 32;
+                    umma_ss(tmem + tm_yoff(k), umma_desc_sw128(cs + koff_c, 16, 1024),
+                            umma_desc_sw128(sb + koff_s, 16, 1024), ID_YO, ks > 0);
+                }
+                umma_commit(bar(B_Y + k));
+                umma_commit(bar(B_EMPTY + s));
+            }
+            // Drain: the last commit must land before the CTA may exit.
+            if (nblk > 0 && !*abort_flag) {
+                const int u = nblk - 1;
+                wait(B_EMPTY + (u & 1), (uint32_t)((u >> 1) & 1));
+            }
+        }
+    } else {
+        // ------------------------------------------------- compute warps ----
+        const int t = tid;                         // TMEM lane = row i = state n
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float a_h = p.A[h] * kLog2e;          // log2-scaled decay rate
+        float* red = reinterpret_cast<float*>(smem + OFF_RED);
+        float S[P];                                 // row n = t of the state, fp32
+        {
+            const float* h0 = p.h0 ? p.h0 + (((b * p.nheads + h) * P) * NS) : nullptr;
+#pragma unroll
+            for (int q = 0; q < P; ++q) S[q] = h0 ? h0[q * NS + t] : 0.0f;
+        }
+        auto write_S = [&](int buf) {
+            unsigned char* sb = smem + OFF_S + buf * S_TILE + (t >> 6) * S_SLAB;
+            const uint32_t col = (uint32_t)(t & 63) * 2;
+#pragma unroll
+            for (int q = 0; q < P; ++q)
+                *reinterpret_cast<bf16*>(sb + sw128(q, col)) = __float2bfloat16_rn(S[q]);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_SREADY));
+        };
+        write_S(0);
+
+        bool ok = true;
+        for (int u = 0; u < nblk && ok; ++u) {
+            const int s = u & 1, k = u & 1;
+            const int64_t t0 = (int64_t)u * UB;
+            const int nrow = (L - t0) < UB ? (int)(L - t0) : UB;
+            float* cs_sm = reinterpret_cast<float*>(smem + OFF_CS) + k * UB;
+            float* da_sm = reinterpret_cast<float*>(smem + OFF_DA) + k * UB;
+            // (a) cumulative log2-decay over the block (scan over 128 threads)
+            const float dt = t < nrow ? p.delta[((b * L + t0 + t) * p.nheads) + h] : 0.0f;
+            float cs = dt * a_h;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, cs, off);
+                if (lane >= off) cs += o;
+            }
+            if (lane == 31) red[(u & 1) * 4 + warp] = cs;
+            named_bar_sync(1, NCOMP);
+            float prefix = 0.0f, total = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float v = red[(u & 1) * 4 + w];
+                if (w < warp) prefix += v;
+                total += v;
+            }
+            cs += prefix;
+            cs_sm[t] = cs;
+            da_sm[t] = p.alpha * dt;
+            const float wt = ex2_approx(total - cs) * p.alpha * dt;   // exp(cs_last - cs_t) alpha delta_t
+            const float et = ex2_approx(cs);                          // exp(cs_t)
+            const float gam = ex2_approx(total);                      // exp(cs_last)
+            named_bar_sync(1, NCOMP);
+
+            // (b) Xhat = diag(w) X  (row t; same swizzled layout as X)
+            if (!(ok = wait(B_FULL + s, (uint32_t)((u >> 1) & 1)))) break;
+            {
+                const unsigned char* xrow = smem + s * SLOT + t * 128;
+                unsigned char* xh = smem + OFF_XHAT + t * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 q = *reinterpret_cast<const uint4*>(xrow + c * 16);
+                    uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w4[e] = pack_bf16x2(bf16_lo(w4[e]) * wt, bf16_hi(w4[e]) * wt);
+                    *reinterpret_cast<uint4*>(xh + c * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_XHAT));
+
+            // (c) M = CB o exp(cs_i - cs_j) alpha delta_j (j <= i), packed bf16 into TMEM
+            if (!(ok = wait(B_CB + k, (uint32_t)((u >> 1) & 1)))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+                if (cb > warp) {               // block entirely above the diagonal
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                } else {
+                    float m[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = cb * 32 + jj;
+                        const float f = ex2_approx(cs - cs_sm[j]) * da_sm[j];
+                        m[jj] = (cb < warp || j <= t) ? __uint_as_float(r[jj]) * f : 0.0f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
+                }
+                tmem_st16(tmem + lane_base + tm_cb(k) + cb * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_M + k));
+
+            // (d) S <- exp(cs_last) S + block state; publish S for the next block
+            if (!(ok = wait(B_STATE, (uint32_t)(u & 1)))) break;
+            tc_fence_after();
+            {
+                uint32_t r[32];
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    tmem_ld32(tmem + lane_base + TM_STATE + hc * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) S[hc * 32 + q] = fmaf(gam, S[hc * 32 + q], __uint_as_float(r[q]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_SFREE));
+            write_S((u + 1) & 1);
+
+            // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of the block
+            if (!(ok = wait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
+            tc_fence_after();
+            {
+                bf16* yrow = p.y + ((b * L + t0 + t) * p.nheads + h) * P;
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t rd[32], ro[32];
+                    tmem_ld32(tmem + lane_base + tm_cb(k) + 64 + hc * 32, rd);
+                    tmem_ld32(tmem + lane_base + tm_yoff(k) + hc * 32, ro);
+                    tmem_wait_ld();
+                    if (t < nrow) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int q = c * 8 + 2 * e;
+                                w4[e] = pack_bf16x2(fmaf(et, __uint_as_float(ro[q]), __uint_as_float(rd[q])),
+                                                    fmaf(et, __uint_as_float(ro[q + 1]), __uint_as_float(rd[q + 1])));
+                            }
+                            *reinterpret_cast<uint4*>(yrow + hc * 32 + c * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_TFREE + k));
+        }
+        if (ok && p.hT) {
+            float* hT = p.hT + ((b * p.nheads + h) * P) * NS;
+#pragma unroll
+            for (int q = 0; q < P; ++q) hT[q * NS + t] = S[q];
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+// ------------------------------------------------------------- launch -----
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 4-D bf16 map (d0 innermost), box (64, 1, 128, 1), 128-byte swizzle.
+cudaError_t make_map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
 bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk) {
-    return headdim == 64 && dstate == 128 && chunk == 256;
+    return headdim == ssd::P && dstate == ssd::NS && (chunk == 128 || chunk == 256);
 }
 
-size_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
-                           int64_t dstate, int64_t chunk) {
-    (void)batch; (void)seqlen; (void)nheads; (void)headdim; (void)dstate; (void)chunk;
-    return 256;
+size_t ssd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t) { return 0; }
+
+cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t stream) {
+    if (a.batch * a.nheads > 0x7fffffffLL || a.seqlen > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    CUtensorMap mx, mB, mC;
+    cudaError_t e;
+    if ((e = make_map_4d(&mx, a.x, ssd::P, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
+    if ((e = make_map_4d(&mB, a.B, ssd::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
+    if ((e = make_map_4d(&mC, a.C, ssd::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
+    SSDKArgs k{};
+    k.delta = a.delta; k.A = a.A; k.h0 = a.h0;
+    k.y = static_cast<bf16*>(a.y); k.hT = a.hT;
+    k.batch = a.batch; k.seqlen = a.seqlen; k.nheads = a.nheads; k.ngroups = a.ngroups;
+    k.nblocks = (int)((a.seqlen + ssd::UB - 1) / ssd::UB);
+    k.alpha = a.alpha;
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ssd::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done.fetch_or(bit, std::memory_order_release);
+    }
+    ssd_fwd_kernel<<<(unsigned)(a.batch * a.nheads), ssd::NTHREADS, ssd::SMEM_BYTES, stream>>>(mx, mB, mC, k);
+    return cudaGetLastError();
 }
 
-cudaError_t launch_ssd_fwd(const SSDArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+unsigned int ssd_read_and_clear_device_error() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_ssd_dev_err, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_ssd_dev_err, &z, sizeof(z));
+    return v;
+}
 
 }  // namespace mmscan

@@ -114,26 +114,30 @@ def test_set_tile(lib):
     assert lib.mm_scan_set_tile(0, 0) == 0
 
 
-def test_ssd_rejects_bad_arguments(lib):
+def test_ssd_rejects_bad_arguments(lib, monkeypatch):
     dims = mm.SSDDims(1, 512, 4, 64, 128, 1, 256)
-    size = ctypes.c_size_t(0)
+    size = ctypes.c_size_t(123)
     assert lib.mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == 0
-    assert size.value > 0
+    assert size.value == 0                                        # the state stays on chip
     bad = mm.SSDDims(1, 512, 4, 64, 128, 3, 256)                  # H % G != 0
     assert lib.mm_ssd_workspace_size(ctypes.byref(bad), ctypes.byref(size)) == 2
-    odd = mm.SSDDims(1, 512, 4, 48, 128, 1, 256)
-    assert lib.mm_ssd_workspace_size(ctypes.byref(odd), ctypes.byref(size)) == 6
+    for odd in (mm.SSDDims(1, 512, 4, 48, 128, 1, 256), mm.SSDDims(1, 512, 4, 64, 64, 1, 256),
+                mm.SSDDims(1, 512, 4, 64, 128, 1, 64)):
+        assert lib.mm_ssd_workspace_size(ctypes.byref(odd), ctypes.byref(size)) == 6
 
-    def call(beta=0.0, alpha=1.0, ws=1 << 30, **over):
+    def call(beta=0.0, alpha=1.0, ws=0, **over):
         a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), h0=None,
-                 y=_fake(5), hT=None, w=_fake(8))
+                 y=_fake(5), hT=None, w=None)
         a.update(over)
         return lib.mm_ssd_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["h0"], beta, alpha,
                               a["y"], a["hT"], a["w"], ws, ctypes.byref(dims), None)
     assert call(x=None) == 1
-    assert call(w=None) == 1
     assert call(beta=0.5) == 6
     assert call(beta=1.5) == 3
     assert call(alpha=-2.0) == 3
-    assert call(ws=16) == 2
     assert call(y=_fake(0)) == 9
+    assert call(hT=_fake(3)) == 9
+    assert call(B=ctypes.c_void_p(A16 * 4 + 8)) == 5
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call() == 7                                            # no workspace needed
+    assert call(h0=_fake(6), hT=_fake(6)) == 7                   # in-place final state

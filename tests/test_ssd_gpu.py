@@ -1,0 +1,119 @@
+"""GPU parity of mm_ssd_fwd (tcgen05 chunked SSD) against the fp64 oracle.
+
+x, B, C and y are bf16 with fp32 accumulation, so the bar is the task's
+bf16 one: relative L2 error <= 1e-2 for y, and the same bar for the final
+state.  Small problems are compared over the whole output; the full-size
+workload (batch 4, L 4096, 32 heads of 64, N 128) on a seeded sample of
+(batch, head, channel) lanes that the oracle computes on their own.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import selective_state_space_momentum_b200 as mm
+from selective_state_space_momentum_b200 import workloads as wl
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+def _dev(inp):
+    return {"x": torch.from_numpy(inp["x"]).cuda().to(torch.bfloat16).contiguous(),
+            "delta": torch.from_numpy(inp["delta"]).cuda().contiguous(),
+            "A": torch.from_numpy(inp["A"]).cuda().contiguous(),
+            "B": torch.from_numpy(inp["B"]).cuda().to(torch.bfloat16).contiguous(),
+            "C": torch.from_numpy(inp["C"]).cuda().to(torch.bfloat16).contiguous()}
+
+
+def _run(dev, h0=None, alpha=1.0, chunk=256):
+    y, hT = mm.ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=h0, alpha=alpha,
+                       chunk=chunk)
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    return y.float().cpu().numpy(), hT.cpu().numpy()
+
+
+def _rel(got, ref):
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+def _lanes_of(y, hT, lanes):
+    """GPU outputs of flat lanes (b*H + h)*P + p as oracle-shaped rows."""
+    Bsz, L, H, P = y.shape
+    b = lanes // (H * P)
+    h = (lanes // P) % H
+    p = lanes % P
+    return y[b, :, h, p], hT[b, h, p, :]
+
+
+def _compare(inp, y, hT, h0=None, alpha=1.0, lanes=None, what=""):
+    Bsz, L, H, P = inp["x"].shape
+    h0r = None if h0 is None else h0.astype(np.float64)
+    yr, hr, _ = oracle.ssd_seq(**inp, h0=h0r, beta=0.0, alpha=alpha, lane=lanes)
+    if lanes is None:
+        lanes = np.arange(Bsz * H * P)
+    yg, hg = _lanes_of(y, hT, lanes)
+    ry, rh = _rel(yg, yr), _rel(hg, hr)
+    assert ry <= TOL, f"{what}: y relative L2 {ry:.3e}"
+    assert rh <= TOL, f"{what}: hT relative L2 {rh:.3e}"
+    return ry, rh
+
+
+@pytest.mark.parametrize("chunk", [128, 256])
+def test_small_full_output(chunk):
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=512, nheads=2)
+    y, hT = _run(_dev(inp), chunk=chunk)
+    _compare(inp, y, hT, what=f"small chunk={chunk}")
+
+
+def test_ragged_length_groups_initial_state_alpha():
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=2, seqlen=300, nheads=4, ngroups=2)
+    rng = np.random.default_rng(5)
+    h0 = (0.5 * rng.standard_normal((2, 4, 64, 128))).astype(np.float32)
+    y, hT = _run(_dev(inp), h0=torch.from_numpy(h0).cuda(), alpha=0.7)
+    _compare(inp, y, hT, h0=h0, alpha=0.7, what="ragged")
+
+
+@pytest.mark.parametrize("L", [1, 127, 129])
+def test_short_and_odd_lengths(L):
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=L, nheads=2)
+    y, hT = _run(_dev(inp))
+    _compare(inp, y, hT, what=f"L={L}")
+
+
+def test_full_size_workload_sampled_lanes():
+    w = wl.SSD_MH
+    inp = wl.ssd_inputs(w)
+    y, hT = _run(_dev(inp), chunk=w.chunk)
+    rng = np.random.default_rng(0)
+    nl = w.batch * w.nheads * w.headdim
+    lanes = np.unique(np.concatenate([rng.choice(nl, 30, replace=False), [0, nl - 1]])).astype(np.int64)
+    _compare(inp, y, hT, lanes=lanes, what="full size")
+
+
+def test_in_place_state_and_determinism():
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=384, nheads=2)
+    dev = _dev(inp)
+    rng = np.random.default_rng(9)
+    h0 = rng.standard_normal((1, 2, 64, 128)).astype(np.float32)
+    st = torch.from_numpy(h0).cuda()
+    y = torch.empty_like(dev["x"])
+    mm.mm_ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], st, 0.0, 1.0, y, st,
+                  torch.empty(0, dtype=torch.uint8, device="cuda"), 256)
+    torch.cuda.synchronize()
+    _compare(inp, y.float().cpu().numpy(), st.cpu().numpy(), h0=h0, what="in place")
+    a = _run(dev)
+    b = _run(dev)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_momentum_is_rejected():
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=128, nheads=1)
+    dev = _dev(inp)
+    y = torch.empty_like(dev["x"])
+    with pytest.raises(mm.MMError) as e:
+        mm.mm_ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], None, 0.5, 1.0, y, None,
+                      torch.empty(0, dtype=torch.uint8, device="cuda"), 256)
+    assert e.value.name == "MM_ERR_UNSUPPORTED"
