@@ -51,8 +51,9 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126e6
 
 WORKLOADS = {w.name: w for w in wl.SCAN_WORKLOADS}
+WORKLOADS[wl.SSD_MH.name] = wl.SSD_MH
 ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
-           "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name}
+           "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name, "ssd": wl.SSD_MH.name}
 DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
 
 
@@ -192,6 +193,166 @@ def run_reference(args, w, beta, alpha):
     return 0
 
 
+def ssd_algorithmic_flops(w: wl.SSDWorkload) -> float:
+    """Tensor FLOPs of the chunked algorithm with chunk Q, full squares:
+    C.B^T once per (batch, chunk) (groups share it), then per head the
+    masked product with X, the chunk state and the read-out of the carried
+    state."""
+    nchunk = math.ceil(w.seqlen / w.chunk)
+    Q, P, N = w.chunk, w.headdim, w.dstate
+    per_bc = 2 * Q * Q * N * w.ngroups
+    per_head = 2 * Q * Q * P + 2 * Q * N * P + 2 * Q * N * P
+    return w.batch * nchunk * (per_bc + w.nheads * per_head)
+
+
+def ssd_executed_flops(w: wl.SSDWorkload) -> float:
+    """Tensor FLOPs the kernel issues: per head and 128-row block, C.B^T
+    (128x128x128), M.X, B^T.Xhat and C.S^T (128x64x128 each)."""
+    nblk = math.ceil(w.seqlen / 128)
+    return w.batch * w.nheads * nblk * (2 * 128 * 128 * 128 + 3 * 2 * 128 * 128 * 64)
+
+
+def ssd_bytes(w: wl.SSDWorkload) -> int:
+    blh = w.batch * w.seqlen * w.nheads
+    return 2 * blh * w.headdim * 2 + 2 * w.batch * w.seqlen * w.ngroups * w.dstate * 2 + blh * 4 \
+        + w.batch * w.nheads * w.headdim * w.dstate * 4
+
+
+def run_ssd(args, w, rank, world, local):
+    import torch
+    import selective_state_space_momentum_b200 as mm
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = wl.ssd_inputs(w, seed=wl.seed_of(w.seed_index) + 1000 * rank)
+    host = {k: torch.from_numpy(v) for k, v in inp.items()}
+    bf = {"x", "B", "C"}
+    step_bytes = ssd_bytes(w)
+    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    sets = []
+    for _ in range(nsets):
+        st = {k: host[k].to(dev).to(torch.bfloat16 if k in bf else torch.float32).contiguous() for k in host}
+        st["y"] = torch.empty_like(st["x"])
+        st["hT"] = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), device=dev)
+        sets.append(st)
+    ws = torch.empty(mm.mm_ssd_workspace_size(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate,
+                                              w.ngroups, w.chunk), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        st = sets[i % nsets]
+        mm.mm_ssd_fwd(st["x"], st["delta"], st["A"], st["B"], st["C"], None, 0.0, w.alpha,
+                      st["y"], st["hT"], ws, w.chunk, stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if world == 1 else local) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    mm.mm_device_status()
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = w.updates * world / (ms_step * 1e-3)
+
+    # end to end from pinned host memory
+    pinned = {k: v.to(torch.bfloat16 if k in bf else torch.float32).pin_memory() for k, v in host.items()}
+    out_y = torch.empty(tuple(inp["x"].shape), dtype=torch.bfloat16, pin_memory=True)
+    out_h = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_y.numel() * 2 + out_h.numel() * 4
+    e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
+
+    def e2e_step():
+        d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], alpha=w.alpha, chunk=w.chunk,
+                           workspace=ws)
+        out_y.copy_(y, non_blocking=True)
+        out_h.copy_(hT, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    barrier()
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        tf_peak = float(peaks.get("bf16_tflops", 1590.0))
+        alg = ssd_algorithmic_flops(w)
+        exe = ssd_executed_flops(w)
+        achieved = alg / (ms_step * 1e-3) / 1e12
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        hbm_achieved = step_bytes / (ms_step * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads,
+                       "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
+                       "beta": w.beta, "alpha": w.alpha, "global_batch": w.batch * world,
+                       "parallelism": f"dp{world}",
+                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": "ssd_fwd_kernel", "achieved": achieved,
+                         "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved / tf_peak, "traffic": None,
+                         "peak_source": f"{peak_kind} cuBLAS bf16 burst",
+                         "algorithmic_flops": alg, "executed_flops": exe,
+                         "executed_tflops": exe / (ms_step * 1e-3) / 1e12,
+                         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": hbm_achieved / hbm_peak, "algorithmic_bytes": step_bytes}},
+            "e2e": {"value": w.updates * world / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = ssd_cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def ssd_cpu_baseline(w: wl.SSDWorkload, budget_s: float = 12.0):
+    """The fp64 oracle (sequential definition) on a sample of (b, h, p) lanes."""
+    import oracle
+    inp = wl.ssd_inputs(w)
+    nl = w.batch * w.nheads * w.headdim
+    probe = np.arange(8, dtype=np.int64)
+    t = time.perf_counter()
+    oracle.ssd_seq(**inp, beta=0.0, alpha=w.alpha, lane=probe)
+    per = (time.perf_counter() - t) / len(probe)
+    k = int(max(8, min(nl, budget_s / max(per, 1e-9))))
+    lanes = np.linspace(0, nl - 1, k).astype(np.int64)
+    t = time.perf_counter()
+    oracle.ssd_seq(**inp, beta=0.0, alpha=w.alpha, lane=lanes)
+    dt = time.perf_counter() - t
+    return {"value": k * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{k} of {nl} (batch, head, channel) lanes, fp64, {dt:.2f} s wall"}
+
+
 # -------------------------------------------------------------- main -------
 def main(argv=None):
     ap = argparse.ArgumentParser(description="momentum selective scan benchmark")
@@ -210,6 +371,34 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[ALIASES.get(args.workload, args.workload)]
+    if isinstance(w, wl.SSDWorkload):
+        if args.impl == "reference":
+            rank, world, _ = dist_env()
+            if rank != 0:
+                return 0
+            cb = ssd_cpu_baseline(w, budget_s=args.reference_budget)
+            print(json.dumps({"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                              "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                              "dtype": "f64", "data": "synthetic", "impl": "reference",
+                              "config": {"workload": w.name}, "cpu_baseline": cb,
+                              "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+            return 0
+        import torch
+        rank, world, local = dist_env()
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            torch.cuda.set_device(0)
+        rc = run_ssd(args, w, rank, world, local)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
     default = (0.9, 1.0) if (0.9, 1.0) in w.runs else w.runs[0]
     beta = args.beta if args.beta is not None else default[0]
     alpha = args.alpha if args.alpha is not None else default[1]

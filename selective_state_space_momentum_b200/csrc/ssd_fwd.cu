@@ -42,6 +42,8 @@
 namespace mmscan {
 
 static __device__ unsigned int g_ssd_dev_err = 0;
+// First wait that gave up: 0x80000000 | role << 24 | barrier << 16 | block.
+static __device__ unsigned int g_ssd_dev_where = 0;
 
 namespace ssd {
 constexpr int P = 64;                 // head dimension
@@ -54,14 +56,14 @@ constexpr int BC_SLAB = UB * 64 * 2;        // 16 KB: [128 rows][64 states]
 constexpr int BC_TILE = 2 * BC_SLAB;        // 32 KB
 constexpr int SLOT = X_TILE + 2 * BC_TILE;  // 80 KB: X, B, C of one block
 constexpr int OFF_XHAT = 2 * SLOT;
-constexpr int S_SLAB = P * 64 * 2;          // 8 KB: [64 rows p][64 states]
-constexpr int S_TILE = 2 * S_SLAB;          // 16 KB
+constexpr int S_TILE = NS * P * 2;         // 16 KB: [128 rows n][64 p] bf16, swizzled
 constexpr int OFF_S = OFF_XHAT + X_TILE;    // 2 S buffers
-constexpr int OFF_CS = OFF_S + 2 * S_TILE;  // cs[2][128] fp32
+constexpr int OFF_CS = OFF_S + 2 * S_TILE;  // cs[2][128] fp32 (log2 units)
 constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha*delta[2][128]
-constexpr int OFF_RED = OFF_DA + 2 * UB * 4;
+constexpr int OFF_CF = OFF_DA + 2 * UB * 4; // column factors [2][128]
+constexpr int OFF_RED = OFF_CF + 2 * UB * 4;
 constexpr int OFF_BAR = OFF_RED + 64;
-constexpr int NBAR = 16;
+constexpr int NBAR = 18;
 constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TSLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
@@ -72,12 +74,15 @@ __device__ __forceinline__ uint32_t tm_yoff(int k) { return 256u + (uint32_t)k *
 constexpr uint32_t TM_STATE = 384;
 constexpr uint32_t TM_COLS = 512;
 // barriers
+// One "ready" barrier per S buffer: the compute warps may publish the state
+// of the next block before the MMA warp has consumed this one, so a single
+// barrier could run two phases ahead of its waiter.
 enum { B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_TFREE = 10,
-       B_XHAT = 12, B_STATE = 13, B_SFREE = 14, B_SREADY = 15 };
+       B_XHAT = 12, B_STATE = 13, B_SFREE = 14, B_SREADY = 15 /* and 16 */ };
 constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
 constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . Xhat (both MN-major)
 constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // M(tmem) . X (X MN-major)
-constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 0);   // C . S^T
+constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 1);   // C . S^T (S MN-major)
 }  // namespace ssd
 
 struct SSDKArgs {
@@ -121,7 +126,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         mbar_init(bar(B_XHAT), NCOMP);
         mbar_init(bar(B_STATE), 1);
         mbar_init(bar(B_SFREE), NCOMP);
-        mbar_init(bar(B_SREADY), NCOMP);
+        mbar_init(bar(B_SREADY + 0), NCOMP); mbar_init(bar(B_SREADY + 1), NCOMP);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -131,9 +136,13 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT);
 
+    int role = warp == 4 ? 1 : warp == 5 ? 2 : 3;
+    int cur_blk = 0;
     auto wait = [&](int i, uint32_t parity) -> bool {
         if (*abort_flag) return false;
         if (!mbar_wait(bar(i), parity, &g_ssd_dev_err)) {
+            atomicCAS(&g_ssd_dev_where, 0u, 0x80000000u | ((uint32_t)role << 24) | ((uint32_t)i << 16) |
+                                                ((uint32_t)cur_blk & 0xffffu));
             *abort_flag = 1;
             return false;
         }
@@ -144,6 +153,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // ------------------------------------------------------ producer ----
         if (lane == 0) {
             for (int u = 0; u < nblk; ++u) {
+                cur_blk = u;
                 const int s = u & 1;
                 if (!wait(B_EMPTY + s, (uint32_t)(((u >> 1) + 1) & 1))) break;
                 const uint32_t slot = base + s * SLOT;
@@ -162,6 +172,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         if (lane == 0) {
             const uint32_t xhat = base + OFF_XHAT;
             for (int u = 0; u < nblk; ++u) {
+                cur_blk = u;
                 const int s = u & 1, k = u & 1;
                 const uint32_t slot = base + s * SLOT;
                 const uint32_t xs = slot, bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
@@ -187,7 +198,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 umma_commit(bar(B_STATE));
                 // 3. Y_diag = M(tmem) . X and Y_off = C . S_prev^T
                 if (!wait(B_M + k, (uint32_t)((u >> 1) & 1))) break;
-                if (!wait(B_SREADY, (uint32_t)(u & 1))) break;
+                if (!wait(B_SREADY + (u & 1), (uint32_t)((u >> 1) & 1))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -197,9 +208,8 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t koff_c = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
-                    const uint32_t koff_s = (ks >> 2) * S_SLAB + (ks & 3) * 32;
                     umma_ss(tmem + tm_yoff(k), umma_desc_sw128(cs + koff_c, 16, 1024),
-                            umma_desc_sw128(sb + koff_s, 16, 1024), ID_YO, ks > 0);
+                            umma_desc_sw128(sb + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
                 }
                 umma_commit(bar(B_Y + k));
                 umma_commit(bar(B_EMPTY + s));
@@ -222,89 +232,129 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
             for (int q = 0; q < P; ++q) S[q] = h0 ? h0[q * NS + t] : 0.0f;
         }
+        // S as the bf16 B operand of C . S^T: MN-major, row n holds 64 p.
         auto write_S = [&](int buf) {
-            unsigned char* sb = smem + OFF_S + buf * S_TILE + (t >> 6) * S_SLAB;
-            const uint32_t col = (uint32_t)(t & 63) * 2;
+            unsigned char* row = smem + OFF_S + buf * S_TILE + t * 128;
 #pragma unroll
-            for (int q = 0; q < P; ++q)
-                *reinterpret_cast<bf16*>(sb + sw128(q, col)) = __float2bfloat16_rn(S[q]);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(S[c * 8 + 2 * e], S[c * 8 + 2 * e + 1]);
+                *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
             fence_proxy_async_smem();
-            mbar_arrive(bar(B_SREADY));
+            mbar_arrive(bar(B_SREADY + buf));
         };
-        write_S(0);
-
-        bool ok = true;
-        for (int u = 0; u < nblk && ok; ++u) {
-            const int s = u & 1, k = u & 1;
+        auto nrow_of = [&](int u) -> int {
             const int64_t t0 = (int64_t)u * UB;
-            const int nrow = (L - t0) < UB ? (int)(L - t0) : UB;
+            return (L - t0) < UB ? (int)(L - t0) : UB;
+        };
+        auto load_dt = [&](int u) -> float {
+            return t < nrow_of(u) ? p.delta[((b * L + (int64_t)u * UB + t) * p.nheads) + h] : 0.0f;
+        };
+        // Per-block scalars of row t: cumulative log2-decay and the factors derived from it.
+        struct Blk { float cs, wt, et, gam; };
+        auto scan_block = [&](int u, float dt) -> Blk {
+            const int k = u & 1;
             float* cs_sm = reinterpret_cast<float*>(smem + OFF_CS) + k * UB;
             float* da_sm = reinterpret_cast<float*>(smem + OFF_DA) + k * UB;
-            // (a) cumulative log2-decay over the block (scan over 128 threads)
-            const float dt = t < nrow ? p.delta[((b * L + t0 + t) * p.nheads) + h] : 0.0f;
+            float* cf_sm = reinterpret_cast<float*>(smem + OFF_CF) + k * UB;
             float cs = dt * a_h;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float o = __shfl_up_sync(0xffffffffu, cs, off);
                 if (lane >= off) cs += o;
             }
-            if (lane == 31) red[(u & 1) * 4 + warp] = cs;
+            if (lane == 31) red[k * 4 + warp] = cs;
             named_bar_sync(1, NCOMP);
             float prefix = 0.0f, total = 0.0f;
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const float v = red[(u & 1) * 4 + w];
+                const float v = red[k * 4 + w];
                 if (w < warp) prefix += v;
                 total += v;
             }
             cs += prefix;
+            const float da = p.alpha * dt;
             cs_sm[t] = cs;
-            da_sm[t] = p.alpha * dt;
-            const float wt = ex2_approx(total - cs) * p.alpha * dt;   // exp(cs_last - cs_t) alpha delta_t
-            const float et = ex2_approx(cs);                          // exp(cs_t)
-            const float gam = ex2_approx(total);                      // exp(cs_last)
+            da_sm[t] = da;
+            // column factor of column t against the last column of its 32-column batch
+            const float cs_ref = __shfl_sync(0xffffffffu, cs, 31);
+            cf_sm[t] = ex2_approx(cs_ref - cs) * da;
             named_bar_sync(1, NCOMP);
-
-            // (b) Xhat = diag(w) X  (row t; same swizzled layout as X)
-            if (!(ok = wait(B_FULL + s, (uint32_t)((u >> 1) & 1)))) break;
-            {
-                const unsigned char* xrow = smem + s * SLOT + t * 128;
-                unsigned char* xh = smem + OFF_XHAT + t * 128;
+            Blk r;
+            r.cs = cs;
+            r.wt = ex2_approx(total - cs) * da;     // exp(cs_last - cs_t) alpha delta_t
+            r.et = ex2_approx(cs);                  // exp(cs_t)
+            r.gam = ex2_approx(total);              // exp(cs_last)
+            return r;
+        };
+        // Xhat = diag(w) X, row t, same swizzled layout as X.
+        auto make_xhat = [&](int u, float wt) -> bool {
+            if (!wait(B_FULL + (u & 1), (uint32_t)((u >> 1) & 1))) return false;
+            const unsigned char* xrow = smem + (u & 1) * SLOT + t * 128;
+            unsigned char* xh = smem + OFF_XHAT + t * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 q = *reinterpret_cast<const uint4*>(xrow + c * 16);
-                    uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+            for (int c = 0; c < 8; ++c) {
+                uint4 q = *reinterpret_cast<const uint4*>(xrow + c * 16);
+                uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w4[e] = pack_bf16x2(bf16_lo(w4[e]) * wt, bf16_hi(w4[e]) * wt);
-                    *reinterpret_cast<uint4*>(xh + c * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
+                for (int e = 0; e < 4; ++e)
+                    w4[e] = pack_bf16x2(bf16_lo(w4[e]) * wt, bf16_hi(w4[e]) * wt);
+                *reinterpret_cast<uint4*>(xh + c * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(B_XHAT));
+            return true;
+        };
 
-            // (c) M = CB o exp(cs_i - cs_j) alpha delta_j (j <= i), packed bf16 into TMEM
+        write_S(0);
+        float dt_next = nblk > 1 ? load_dt(1) : 0.0f;
+        Blk cur = scan_block(0, load_dt(0));
+        bool ok = make_xhat(0, cur.wt);
+        for (int u = 0; u < nblk && ok; ++u) {
+            cur_blk = u;
+            const int k = u & 1;
+            const int64_t t0 = (int64_t)u * UB;
+            const int nrow = nrow_of(u);
+            const float* cs_sm = reinterpret_cast<const float*>(smem + OFF_CS) + k * UB;
+            const float* da_sm = reinterpret_cast<const float*>(smem + OFF_DA) + k * UB;
+            const float* cf_sm = reinterpret_cast<const float*>(smem + OFF_CF) + k * UB;
+
+            // (c) M = CB o exp(cs_i - cs_j) alpha delta_j (j <= i), bf16 pairs into TMEM.
+            //     Batches below the diagonal use exp(cs_i - cs_r) exp(cs_r - cs_j), both <= 1.
             if (!(ok = wait(B_CB + k, (uint32_t)((u >> 1) & 1)))) break;
             tc_fence_after();
 #pragma unroll 1
             for (int cb = 0; cb < 4; ++cb) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
-                tmem_wait_ld();
                 uint32_t pk[16];
-                if (cb > warp) {               // block entirely above the diagonal
+                if (cb > warp) {                   // entirely above the diagonal
 #pragma unroll
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 } else {
-                    float m[32];
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
+                    tmem_wait_ld();
+                    if (cb < warp) {
+                        const float rowf = ex2_approx(cur.cs - cs_sm[cb * 32 + 31]);
+                        const float2 rr = f2(rowf, rowf);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = cb * 32 + jj;
-                        const float f = ex2_approx(cs - cs_sm[j]) * da_sm[j];
-                        m[jj] = (cb < warp || j <= t) ? __uint_as_float(r[jj]) * f : 0.0f;
+                        for (int e = 0; e < 16; ++e) {
+                            const float2 cf = *reinterpret_cast<const float2*>(cf_sm + cb * 32 + 2 * e);
+                            const float2 m = __fmul2_rn(__fmul2_rn(f2(__uint_as_float(r[2 * e]),
+                                                                       __uint_as_float(r[2 * e + 1])), cf), rr);
+                            pk[e] = pack_bf16x2(m.x, m.y);
+                        }
+                    } else {
+                        float m[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = cb * 32 + jj;
+                            m[jj] = j <= t ? __uint_as_float(r[jj]) * (ex2_approx(cur.cs - cs_sm[j]) * da_sm[j]) : 0.0f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
                     }
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
                 }
                 tmem_st16(tmem + lane_base + tm_cb(k) + cb * 16, pk);
             }
@@ -322,14 +372,23 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tmem_ld32(tmem + lane_base + TM_STATE + hc * 32, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) S[hc * 32 + q] = fmaf(gam, S[hc * 32 + q], __uint_as_float(r[q]));
+                    for (int q = 0; q < 32; ++q) S[hc * 32 + q] = fmaf(cur.gam, S[hc * 32 + q], __uint_as_float(r[q]));
                 }
             }
             tc_fence_before();
             mbar_arrive(bar(B_SFREE));
             write_S((u + 1) & 1);
 
-            // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of the block
+            // next block's scan and Xhat while this block's output MMAs run
+            const float et = cur.et;
+            if (u + 1 < nblk) {
+                const float dt = dt_next;
+                if (u + 2 < nblk) dt_next = load_dt(u + 2);
+                cur = scan_block(u + 1, dt);
+                if (!(ok = make_xhat(u + 1, cur.wt))) break;
+            }
+
+            // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of block u
             if (!(ok = wait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
             tc_fence_after();
             {
@@ -443,10 +502,13 @@ cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t stream) {
 }
 
 unsigned int ssd_read_and_clear_device_error() {
-    unsigned int v = 0, z = 0;
+    unsigned int v = 0, w = 0, z = 0;
     if (cudaMemcpyFromSymbol(&v, g_ssd_dev_err, sizeof(v)) != cudaSuccess) return 0;
+    if (!v) return 0;
+    cudaMemcpyFromSymbol(&w, g_ssd_dev_where, sizeof(w));
     cudaMemcpyToSymbol(g_ssd_dev_err, &z, sizeof(z));
-    return v;
+    cudaMemcpyToSymbol(g_ssd_dev_where, &z, sizeof(z));
+    return w ? w : v;
 }
 
 }  // namespace mmscan

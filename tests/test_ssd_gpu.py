@@ -117,3 +117,20 @@ def test_momentum_is_rejected():
         mm.mm_ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], None, 0.5, 1.0, y, None,
                       torch.empty(0, dtype=torch.uint8, device="cuda"), 256)
     assert e.value.name == "MM_ERR_UNSUPPORTED"
+
+
+def test_repeated_runs_odd_block_counts_finish_without_device_timeout():
+    """Several block counts (odd and even) run back to back; every call must
+    complete its handshakes (mm_device_status raises on a bounded wait that
+    gave up) and match the oracle."""
+    for L in (300, 640, 1000):
+        inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=L, nheads=3)
+        dev = _dev(inp)
+        first = None
+        for _ in range(3):
+            y, hT = _run(dev)
+            if first is None:
+                first = (y, hT)
+                _compare(inp, y, hT, what=f"repeat L={L}")
+            else:
+                assert np.array_equal(first[0], y) and np.array_equal(first[1], hT)
