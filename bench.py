@@ -57,6 +57,24 @@ ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
 DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
 
 
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes of one launch from the committed ncu summary (profiles/),
+    or None when there is none for this workload or the kernel source has
+    changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+        if not rec or rec.get("workload") != workload:
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != rec["source_sha256_16"]:
+                return None
+        return float(rec["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -141,6 +159,27 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ helpers ------
+def rank_seed(index: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): a distinct, fixed seed."""
+    return wl.seed_of(index) + 1000 * rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of x over all ranks (the job's time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -222,7 +261,7 @@ def run_ssd(args, w, rank, world, local):
     import torch
     import selective_state_space_momentum_b200 as mm
     dev = torch.device("cuda", torch.cuda.current_device())
-    inp = wl.ssd_inputs(w, seed=wl.seed_of(w.seed_index) + 1000 * rank)
+    inp = wl.ssd_inputs(w, seed=rank_seed(w.seed_index, rank))
     host = {k: torch.from_numpy(v) for k, v in inp.items()}
     bf = {"x", "B", "C"}
     step_bytes = ssd_bytes(w)
@@ -261,13 +300,9 @@ def run_ssd(args, w, rank, world, local):
         torch.cuda.synchronize()
     mm.mm_device_status()
     barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms_total / args.steps
-    value = w.updates * world / (ms_step * 1e-3)
+    value = whole_job_rate(w.updates, world, ms_step)
 
     # end to end from pinned host memory
     pinned = {k: v.to(torch.bfloat16 if k in bf else torch.float32).pin_memory() for k, v in host.items()}
@@ -294,11 +329,7 @@ def run_ssd(args, w, rank, world, local):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     barrier()
     if rank == 0:
         peaks, peak_kind = measured_peaks()
@@ -318,13 +349,14 @@ def run_ssd(args, w, rank, world, local):
                        "parallelism": f"dp{world}",
                        "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": "ssd_fwd_kernel", "achieved": achieved,
-                         "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved / tf_peak, "traffic": None,
+                         "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved / tf_peak,
+                         "traffic": measured_traffic("ssd_fwd_kernel", w.name),
                          "peak_source": f"{peak_kind} cuBLAS bf16 burst",
                          "algorithmic_flops": alg, "executed_flops": exe,
                          "executed_tflops": exe / (ms_step * 1e-3) / 1e12,
                          "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
                                  "frac": hbm_achieved / hbm_peak, "algorithmic_bytes": step_bytes}},
-            "e2e": {"value": w.updates * world / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+            "e2e": {"value": whole_job_rate(w.updates, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
@@ -423,7 +455,7 @@ def main(argv=None):
         mm.mm_scan_set_tile(spt, warps)
 
     # Each rank scans its own batch (seed offset by rank): weak scaling.
-    inp = wl.scan_inputs(w, seed=wl.seed_of(w.seed_index) + 1000 * rank)
+    inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))
     iodt = torch.float32 if w.io == "f32" else torch.bfloat16
     host = {k: torch.from_numpy(v) for k, v in inp.items()}
     step_bytes = algorithmic_bytes(w)
@@ -462,14 +494,10 @@ def main(argv=None):
         torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms_total / args.steps
     updates = w.updates
-    value = updates * world / (ms_step * 1e-3)
+    value = whole_job_rate(updates, world, ms_step)
 
     # ---- end to end through the host-memory call -------------------------
     e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
@@ -492,11 +520,7 @@ def main(argv=None):
                          beta=beta, alpha=alpha, out=out, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     barrier()
 
     if rank == 0:
@@ -520,12 +544,13 @@ def main(argv=None):
                        "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
             "roofline": {"bound": "alu", "kernel": "scan_fwd_kernel",
                          "achieved": achieved / 1e9, "peak": mufu_peak / 1e9, "unit": "Gex2/s",
-                         "frac": achieved / mufu_peak, "traffic": None,
+                         "frac": achieved / mufu_peak,
+                         "traffic": measured_traffic("scan_fwd_kernel", w.name),
                          "peak_source": f"16 ex2/clk/SM x 148 SMs x {sm_max:.0f} MHz",
                          "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
                                  "frac": hbm_achieved / hbm_peak, "peak_source": peak_kind,
                                  "algorithmic_bytes": step_bytes}},
-            "e2e": {"value": updates * world / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+            "e2e": {"value": whole_job_rate(updates, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
             "clocks": clocks,

@@ -296,10 +296,10 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // ---- the recurrence over this chunk, R steps at a time -------------
         const float* Bg = Bt + g * SPT;
         const float* Cg = Ct + g * SPT;
-        const int ngroups = (nval + R - 1) / R;
-        for (int gi = 0; gi < ngroups; ++gi) {
+
+        // Loads, delta*x and exponentials of the R steps of group gi.
+        auto prep = [&](int gi, float (&u)[R], float (&a)[R][SPT]) {
             const int tau0 = gi * R;
-            const int kmax = nval - tau0 < R ? nval - tau0 : R;
             const int bx = tau0 / TL::BOX_T;
             const int col = tau0 - bx * TL::BOX_T;
             const unsigned char* xt = sbuf + TL::OFF_X + bx * TL::XBOX;
@@ -312,14 +312,12 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
                 xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
             }
-            float u[R];
 #pragma unroll
             for (int j = 0; j < R; j += 2) {
                 const float2 uu = __fmul2_rn(f2(dl[j], dl[j + 1]), f2(xl[j], xl[j + 1]));
                 u[j] = uu.x;
                 u[j + 1] = uu.y;
             }
-            float a[R][SPT];
 #pragma unroll
             for (int sI = 0; sI < SPT; ++sI) {
 #pragma unroll
@@ -329,90 +327,183 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     a[j + 1][sI] = ex2_approx(r2.y);
                 }
             }
-            float yk[R];
-            if (kmax == R) {
-#pragma unroll
-                for (int j = 0; j < R; ++j) {
-                    const float* brow = Bg + (tau0 + j) * BP;
-                    const float* crow = Cg + (tau0 + j) * BP;
-                    float bq[SPT], cq[SPT];
-#pragma unroll
-                    for (int q = 0; q < SPT; q += 4 > SPT ? SPT : 4) {
-                        if constexpr (SPT >= 4) {
-                            const float4 b4 = *reinterpret_cast<const float4*>(brow + q);
-                            const float4 c4 = *reinterpret_cast<const float4*>(crow + q);
-                            bq[q] = b4.x; bq[q + 1] = b4.y; bq[q + 2] = b4.z; bq[q + 3] = b4.w;
-                            cq[q] = c4.x; cq[q + 1] = c4.y; cq[q + 2] = c4.z; cq[q + 3] = c4.w;
-                        } else {
-                            const float2 b2 = *reinterpret_cast<const float2*>(brow + q);
-                            const float2 c2 = *reinterpret_cast<const float2*>(crow + q);
-                            bq[q] = b2.x; bq[q + 1] = b2.y;
-                            cq[q] = c2.x; cq[q + 1] = c2.y;
+        };
+
+        auto reduce_store = [&](int tau0, const float (&yk)[R]) {
+                // ---- add the G partials of each channel; store y -------------
+                constexpr int PER = R / G;      // steps each lane finishes
+                float out[PER];
+                if constexpr (G == 1) {
+    #pragma unroll
+                    for (int j = 0; j < R; ++j) out[j] = yk[j];
+                } else {
+    #pragma unroll
+                    for (int j = 0; j < R; ++j) yw[j * G + g] = yk[j];
+                    __syncwarp();
+    #pragma unroll
+                    for (int e = 0; e < PER; ++e) {
+                        const float* src = yw + (g * PER + e) * G;
+                        float acc = 0.0f;
+    #pragma unroll
+                        for (int gg = 0; gg < G; gg += (G >= 4 ? 4 : G)) {
+                            if constexpr (G >= 4) {
+                                const float4 q4 = *reinterpret_cast<const float4*>(src + gg);
+                                acc += (q4.x + q4.y) + (q4.z + q4.w);
+                            } else {
+                                const float2 q2 = *reinterpret_cast<const float2*>(src + gg);
+                                acc += q2.x + q2.y;
+                            }
                         }
+                        out[e] = acc;
                     }
-                    const float2 uu = f2(u[j], u[j]);
-                    float2 yy = f2(0.0f, 0.0f);
-#pragma unroll
-                    for (int q = 0; q < NPAIR; ++q) {
-                        const float2 w = __fmul2_rn(uu, f2(bq[2 * q], bq[2 * q + 1]));
-                        vv[q] = __ffma2_rn(beta2, vv[q], w);
-                        hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
-                        yy = __ffma2_rn(f2(cq[2 * q], cq[2 * q + 1]), hh[q], yy);
-                    }
-                    yk[j] = yy.x + yy.y;
+                    __syncwarp();
                 }
-            } else {
+                const int first = tau0 + g * PER;      // step (within the chunk) of out[0]
+                const int cnt = nval - first < PER ? nval - first : PER;
+                if (active && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
+        };
+
+        // The R full steps of group gi, then the read-out reduction and store.
+        auto full_steps = [&](int gi, const float (&u)[R], const float (&a)[R][SPT]) {
+            const int tau0 = gi * R;
+            float yk[R];
 #pragma unroll
-                for (int j = 0; j < R; ++j) {       // ragged end of the sequence
-                    yk[j] = 0.0f;
-                    if (j < kmax) {
+            for (int j = 0; j < R; ++j) {
+                const float* brow = Bg + (tau0 + j) * BP;
+                const float* crow = Cg + (tau0 + j) * BP;
+                float bq[SPT], cq[SPT];
+                if constexpr (SPT >= 4) {
+#pragma unroll
+                    for (int q = 0; q < SPT; q += 4) {
+                        const float4 b4 = *reinterpret_cast<const float4*>(brow + q);
+                        const float4 c4 = *reinterpret_cast<const float4*>(crow + q);
+                        bq[q] = b4.x; bq[q + 1] = b4.y; bq[q + 2] = b4.z; bq[q + 3] = b4.w;
+                        cq[q] = c4.x; cq[q + 1] = c4.y; cq[q + 2] = c4.z; cq[q + 3] = c4.w;
+                    }
+                } else {
+                    const float2 b2 = *reinterpret_cast<const float2*>(brow);
+                    const float2 c2 = *reinterpret_cast<const float2*>(crow);
+                    bq[0] = b2.x; bq[1] = b2.y;
+                    cq[0] = c2.x; cq[1] = c2.y;
+                }
+                const float2 uu = f2(u[j], u[j]);
+                float2 yy = f2(0.0f, 0.0f);
+#pragma unroll
+                for (int q = 0; q < NPAIR; ++q) {
+                    const float2 w = __fmul2_rn(uu, f2(bq[2 * q], bq[2 * q + 1]));
+                    vv[q] = __ffma2_rn(beta2, vv[q], w);
+                    hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
+                    yy = __ffma2_rn(f2(cq[2 * q], cq[2 * q + 1]), hh[q], yy);
+                }
+                yk[j] = yy.x + yy.y;
+            }
+            reduce_store(tau0, yk);
+        };
+
+        if (nval == T) {
+            // Full chunk: groups unrolled, each group's exponentials issued one group ahead.
+            constexpr int NG = T / R;
+            float uA[R], uB[R], aA[R][SPT], aB[R][SPT];
+            prep(0, uA, aA);
+#pragma unroll
+            for (int gi = 0; gi < NG; ++gi) {
+                if ((gi & 1) == 0) {
+                    if (gi + 1 < NG) prep(gi + 1, uB, aB);
+                    full_steps(gi, uA, aA);
+                } else {
+                    if (gi + 1 < NG) prep(gi + 1, uA, aA);
+                    full_steps(gi, uB, aB);
+                }
+            }
+        } else {
+            const int ngroups = (nval + R - 1) / R;
+            for (int gi = 0; gi < ngroups; ++gi) {
+                const int tau0 = gi * R;
+                const int kmax = nval - tau0 < R ? nval - tau0 : R;
+                const int bx = tau0 / TL::BOX_T;
+                const int col = tau0 - bx * TL::BOX_T;
+                const unsigned char* xt = sbuf + TL::OFF_X + bx * TL::XBOX;
+                const unsigned char* dtl = sbuf + TL::OFF_D + bx * TL::XBOX;
+                float dl[R], xl[R];
+    #pragma unroll
+                for (int j = 0; j < R; j += 4) {
+                    const float4 dq = load4(reinterpret_cast<const IO*>(dtl + sw128(c, (col + j) * EB)));
+                    const float4 xq = load4(reinterpret_cast<const IO*>(xt + sw128(c, (col + j) * EB)));
+                    dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
+                    xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
+                }
+                float u[R];
+    #pragma unroll
+                for (int j = 0; j < R; j += 2) {
+                    const float2 uu = __fmul2_rn(f2(dl[j], dl[j + 1]), f2(xl[j], xl[j + 1]));
+                    u[j] = uu.x;
+                    u[j + 1] = uu.y;
+                }
+                float a[R][SPT];
+    #pragma unroll
+                for (int sI = 0; sI < SPT; ++sI) {
+    #pragma unroll
+                    for (int j = 0; j < R; j += 2) {
+                        const float2 r2 = __fmul2_rn(f2(dl[j], dl[j + 1]), A2p[sI]);
+                        a[j][sI] = ex2_approx(r2.x);
+                        a[j + 1][sI] = ex2_approx(r2.y);
+                    }
+                }
+                float yk[R];
+                if (kmax == R) {
+    #pragma unroll
+                    for (int j = 0; j < R; ++j) {
                         const float* brow = Bg + (tau0 + j) * BP;
                         const float* crow = Cg + (tau0 + j) * BP;
+                        float bq[SPT], cq[SPT];
+    #pragma unroll
+                        for (int q = 0; q < SPT; q += 4 > SPT ? SPT : 4) {
+                            if constexpr (SPT >= 4) {
+                                const float4 b4 = *reinterpret_cast<const float4*>(brow + q);
+                                const float4 c4 = *reinterpret_cast<const float4*>(crow + q);
+                                bq[q] = b4.x; bq[q + 1] = b4.y; bq[q + 2] = b4.z; bq[q + 3] = b4.w;
+                                cq[q] = c4.x; cq[q + 1] = c4.y; cq[q + 2] = c4.z; cq[q + 3] = c4.w;
+                            } else {
+                                const float2 b2 = *reinterpret_cast<const float2*>(brow + q);
+                                const float2 c2 = *reinterpret_cast<const float2*>(crow + q);
+                                bq[q] = b2.x; bq[q + 1] = b2.y;
+                                cq[q] = c2.x; cq[q + 1] = c2.y;
+                            }
+                        }
                         const float2 uu = f2(u[j], u[j]);
                         float2 yy = f2(0.0f, 0.0f);
-#pragma unroll
+    #pragma unroll
                         for (int q = 0; q < NPAIR; ++q) {
-                            const float2 w = __fmul2_rn(uu, f2(brow[2 * q], brow[2 * q + 1]));
+                            const float2 w = __fmul2_rn(uu, f2(bq[2 * q], bq[2 * q + 1]));
                             vv[q] = __ffma2_rn(beta2, vv[q], w);
                             hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
-                            yy = __ffma2_rn(f2(crow[2 * q], crow[2 * q + 1]), hh[q], yy);
+                            yy = __ffma2_rn(f2(cq[2 * q], cq[2 * q + 1]), hh[q], yy);
                         }
                         yk[j] = yy.x + yy.y;
                     }
-                }
-            }
-
-            // ---- add the G partials of each channel; store y -------------
-            constexpr int PER = R / G;      // steps each lane finishes
-            float out[PER];
-            if constexpr (G == 1) {
-#pragma unroll
-                for (int j = 0; j < R; ++j) out[j] = yk[j];
-            } else {
-#pragma unroll
-                for (int j = 0; j < R; ++j) yw[j * G + g] = yk[j];
-                __syncwarp();
-#pragma unroll
-                for (int e = 0; e < PER; ++e) {
-                    const float* src = yw + (g * PER + e) * G;
-                    float acc = 0.0f;
-#pragma unroll
-                    for (int gg = 0; gg < G; gg += (G >= 4 ? 4 : G)) {
-                        if constexpr (G >= 4) {
-                            const float4 q4 = *reinterpret_cast<const float4*>(src + gg);
-                            acc += (q4.x + q4.y) + (q4.z + q4.w);
-                        } else {
-                            const float2 q2 = *reinterpret_cast<const float2*>(src + gg);
-                            acc += q2.x + q2.y;
+                } else {
+    #pragma unroll
+                    for (int j = 0; j < R; ++j) {       // ragged end of the sequence
+                        yk[j] = 0.0f;
+                        if (j < kmax) {
+                            const float* brow = Bg + (tau0 + j) * BP;
+                            const float* crow = Cg + (tau0 + j) * BP;
+                            const float2 uu = f2(u[j], u[j]);
+                            float2 yy = f2(0.0f, 0.0f);
+    #pragma unroll
+                            for (int q = 0; q < NPAIR; ++q) {
+                                const float2 w = __fmul2_rn(uu, f2(brow[2 * q], brow[2 * q + 1]));
+                                vv[q] = __ffma2_rn(beta2, vv[q], w);
+                                hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
+                                yy = __ffma2_rn(f2(crow[2 * q], crow[2 * q + 1]), hh[q], yy);
+                            }
+                            yk[j] = yy.x + yy.y;
                         }
                     }
-                    out[e] = acc;
                 }
-                __syncwarp();
+
+                reduce_store(tau0, yk);
             }
-            const int first = tau0 + g * PER;      // step (within the chunk) of out[0]
-            const int cnt = nval - first < PER ? nval - first : PER;
-            if (active && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
         }
     }
 
@@ -519,6 +610,8 @@ cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, cudaStream_
             if (spt == 4 && warps == 1) return launch_variant<IO, 16, 4, 1>(a, s);
             if (spt == 4 && warps == 2) return launch_variant<IO, 16, 4, 2>(a, s);
             if (spt == 4 && warps == 4) return launch_variant<IO, 16, 4, 4>(a, s);
+            if (spt == 8 && warps == 1) return launch_variant<IO, 16, 8, 1>(a, s);
+            if (spt == 8 && warps == 2) return launch_variant<IO, 16, 8, 2>(a, s);
             break;
         case 8:
             if (spt == 2) return launch_variant<IO, 8, 2, 2>(a, s);
@@ -537,21 +630,33 @@ cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, cudaStream_
 
 bool scan_tile_supported(int spt, int warps) {
     return (spt == 2 && (warps == 2 || warps == 4 || warps == 8)) ||
-           (spt == 4 && (warps == 1 || warps == 2 || warps == 4));
+           (spt == 4 && (warps == 1 || warps == 2 || warps == 4)) ||
+           (spt == 8 && (warps == 1 || warps == 2));
 }
 
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
                                 int forced_spt, int forced_warps) {
-    (void)batch; (void)dim; (void)io;
+    (void)io;
+    // The choice depends on (batch * dim, dstate) only, never on L, so calls
+    // that split one sequence use the same variant.  Fewer states per lane
+    // give more warps (needed when there are few channels); more states per
+    // lane need fewer instructions per update.
     ScanTileChoice t;
     t.np = dstate <= 2 ? 2 : dstate <= 4 ? 4 : dstate <= 8 ? 8 : 16;
-    t.spt = 2;
-    t.warps = 4;
+    const int64_t channels = batch * dim;
+    if (channels >= 4096) {
+        t.spt = 4;
+        t.warps = 2;
+    } else {
+        t.spt = 2;
+        t.warps = 2;
+    }
     if (t.np == 16 && forced_spt) {
         t.spt = forced_spt;
         t.warps = forced_warps;
     }
-    if (t.np == 8 && forced_spt) t.spt = forced_spt;
+    if (t.np == 8 && forced_spt) t.spt = forced_spt == 8 ? 4 : forced_spt;
+    if (t.np == 8 && t.spt > 4) t.spt = 4;
     return t;
 }
 
