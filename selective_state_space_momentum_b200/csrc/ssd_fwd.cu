@@ -49,8 +49,9 @@ namespace ssd {
 constexpr int P = 64;                 // head dimension
 constexpr int NS = 128;               // states
 constexpr int UB = 128;               // rows per block
-constexpr int NCOMP = 128;            // compute threads (warps 0-3)
-constexpr int NTHREADS = NCOMP + 64;  // + producer warp + MMA warp
+constexpr int NCOMP = 128;            // threads of one compute warpgroup
+constexpr int NTHREADS = 2 * NCOMP + 64;  // mask warpgroup + state warpgroup + producer + MMA
+constexpr int W_PROD = 8, W_MMA = 9;  // warp indices of the producer and the MMA issuer
 constexpr int X_TILE = UB * P * 2;          // 16 KB: [128 rows][64] bf16, swizzled
 constexpr int BC_SLAB = UB * 64 * 2;        // 16 KB: [128 rows][64 states]
 constexpr int BC_TILE = 2 * BC_SLAB;        // 32 KB
@@ -61,9 +62,12 @@ constexpr int OFF_S = OFF_XHAT + X_TILE;    // 2 S buffers
 constexpr int OFF_CS = OFF_S + 2 * S_TILE;  // cs[2][128] fp32 (log2 units)
 constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha*delta[2][128]
 constexpr int OFF_CF = OFF_DA + 2 * UB * 4; // column factors [2][128]
-constexpr int OFF_RED = OFF_CF + 2 * UB * 4;
+constexpr int OFF_ET = OFF_CF + 2 * UB * 4; // exp(cs_t) [2][128]
+constexpr int OFF_WT = OFF_ET + 2 * UB * 4;  // exp(cs_last - cs_t) alpha delta_t [2][128]
+constexpr int OFF_GAM = OFF_WT + 2 * UB * 4;   // exp(cs_last) [2]
+constexpr int OFF_RED = OFF_GAM + 16;
 constexpr int OFF_BAR = OFF_RED + 64;
-constexpr int NBAR = 18;
+constexpr int NBAR = 20;
 constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TSLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
@@ -78,12 +82,28 @@ constexpr uint32_t TM_COLS = 512;
 // of the next block before the MMA warp has consumed this one, so a single
 // barrier could run two phases ahead of its waiter.
 enum { B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_TFREE = 10,
-       B_XHAT = 12, B_STATE = 13, B_SFREE = 14, B_SREADY = 15 /* and 16 */ };
+       B_XHAT = 12, B_STATE = 13, B_SFREE = 14, B_SREADY = 15 /* and 16 */,
+       B_SCAL = 17 /* and 18: per-block scalars ready for the state warpgroup */ };
 constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
 constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . Xhat (both MN-major)
 constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // M(tmem) . X (X MN-major)
 constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 1);   // C . S^T (S MN-major)
 }  // namespace ssd
+
+// Xhat row t, 16-byte chunks c0..c0+3 (logical order; the physical chunk
+// index is swizzled so a warp touches 8 different bank groups).
+__device__ __forceinline__ void ssd_scale_row_half(const unsigned char* xrow, unsigned char* xh, int t,
+                                                   int c0, float wt) {
+#pragma unroll
+    for (int c = c0; c < c0 + 4; ++c) {
+        const int pc = (c ^ (t & 7)) << 4;
+        const uint4 q = *reinterpret_cast<const uint4*>(xrow + pc);
+        uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(bf16_lo(w4[e]) * wt, bf16_hi(w4[e]) * wt);
+        *reinterpret_cast<uint4*>(xh + pc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+}
 
 struct SSDKArgs {
     const float* delta;
@@ -123,10 +143,11 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         mbar_init(bar(B_M + 0), NCOMP); mbar_init(bar(B_M + 1), NCOMP);
         mbar_init(bar(B_Y + 0), 1); mbar_init(bar(B_Y + 1), 1);
         mbar_init(bar(B_TFREE + 0), NCOMP); mbar_init(bar(B_TFREE + 1), NCOMP);
-        mbar_init(bar(B_XHAT), NCOMP);
+        mbar_init(bar(B_XHAT), 2 * NCOMP);   // both warpgroups write half of each row
         mbar_init(bar(B_STATE), 1);
         mbar_init(bar(B_SFREE), NCOMP);
         mbar_init(bar(B_SREADY + 0), NCOMP); mbar_init(bar(B_SREADY + 1), NCOMP);
+        mbar_init(bar(B_SCAL + 0), NCOMP); mbar_init(bar(B_SCAL + 1), NCOMP);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -136,7 +157,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT);
 
-    int role = warp == 4 ? 1 : warp == 5 ? 2 : 3;
+    int role = warp == W_PROD ? 1 : warp == W_MMA ? 2 : warp < 4 ? 3 : 4;
     int cur_blk = 0;
     auto wait = [&](int i, uint32_t parity) -> bool {
         if (*abort_flag) return false;
@@ -149,7 +170,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         return true;
     };
 
-    if (warp == 4) {
+    if (warp == W_PROD) {
         // ------------------------------------------------------ producer ----
         if (lane == 0) {
             for (int u = 0; u < nblk; ++u) {
@@ -167,38 +188,48 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tma_load_4d(slot + X_TILE + BC_TILE + BC_SLAB, &tm_C, fb, 64, (int)g, t0, (int)b);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == W_MMA) {
         // ----------------------------------------------------------- MMA ----
+        // Issue order per block u: block state(u), C.B^T(u+1) (one block
+        // ahead, so the mask warpgroup can start on it), then Y(u).
         if (lane == 0) {
             const uint32_t xhat = base + OFF_XHAT;
-            for (int u = 0; u < nblk; ++u) {
+            auto issue_cb = [&](int v) -> bool {
+                const int sv = v & 1, kv = v & 1;
+                const uint32_t slot = base + sv * SLOT;
+                const uint32_t bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
+                if (!wait(B_FULL + sv, (uint32_t)((v >> 1) & 1))) return false;
+                if (!wait(B_TFREE + kv, (uint32_t)(((v >> 1) + 1) & 1))) return false;
+                tc_fence_after();
+                // C . B^T: M = 128 rows i, N = 128 rows j, K = 128 states
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
+                    umma_ss(tmem + tm_cb(kv), umma_desc_sw128(cs + koff, 16, 1024),
+                            umma_desc_sw128(bs + koff, 16, 1024), ID_CB, ks > 0);
+                }
+                umma_commit(bar(B_CB + kv));
+                return true;
+            };
+            bool live = nblk > 0 && issue_cb(0);
+            for (int u = 0; u < nblk && live; ++u) {
                 cur_blk = u;
                 const int s = u & 1, k = u & 1;
                 const uint32_t slot = base + s * SLOT;
                 const uint32_t xs = slot, bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
-                if (!wait(B_FULL + s, (uint32_t)((u >> 1) & 1))) break;
-                if (!wait(B_TFREE + k, (uint32_t)(((u >> 1) + 1) & 1))) break;
-                tc_fence_after();
-                // 1. CB = C . B^T: M = 128 rows i, N = 128 rows j, K = 128 states
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
-                    umma_ss(tmem + tm_cb(k), umma_desc_sw128(cs + koff, 16, 1024),
-                            umma_desc_sw128(bs + koff, 16, 1024), ID_CB, ks > 0);
-                }
-                umma_commit(bar(B_CB + k));
-                // 2. block state = B^T . Xhat: M = 128 states, N = 64, K = 128 rows
-                if (!wait(B_XHAT, (uint32_t)(u & 1))) break;
-                if (!wait(B_SFREE, (uint32_t)((u + 1) & 1))) break;
+                // block state = B^T . Xhat: M = 128 states, N = 64, K = 128 rows
+                if (!(live = wait(B_XHAT, (uint32_t)(u & 1)))) break;
+                if (!(live = wait(B_SFREE, (uint32_t)((u + 1) & 1)))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     umma_ss(tmem + TM_STATE, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
                             umma_desc_sw128(xhat + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
                 umma_commit(bar(B_STATE));
-                // 3. Y_diag = M(tmem) . X and Y_off = C . S_prev^T
-                if (!wait(B_M + k, (uint32_t)((u >> 1) & 1))) break;
-                if (!wait(B_SREADY + (u & 1), (uint32_t)((u >> 1) & 1))) break;
+                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
+                // Y_diag = M(tmem) . X and Y_off = C . S_prev^T
+                if (!(live = wait(B_M + k, (uint32_t)((u >> 1) & 1)))) break;
+                if (!(live = wait(B_SREADY + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -220,31 +251,13 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 wait(B_EMPTY + (u & 1), (uint32_t)((u >> 1) & 1));
             }
         }
-    } else {
-        // ------------------------------------------------- compute warps ----
-        const int t = tid;                         // TMEM lane = row i = state n
+    } else if (warp < 4) {
+        // ------------------------------------- mask warpgroup (warps 0-3) ----
+        // Per block: in-block log2-decay scan, w o X, and the masked matrix M.
+        const int t = tid;                         // TMEM lane = row i of the block
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const float a_h = p.A[h] * kLog2e;          // log2-scaled decay rate
+        const float a_h = p.A[h] * kLog2e;
         float* red = reinterpret_cast<float*>(smem + OFF_RED);
-        float S[P];                                 // row n = t of the state, fp32
-        {
-            const float* h0 = p.h0 ? p.h0 + (((b * p.nheads + h) * P) * NS) : nullptr;
-#pragma unroll
-            for (int q = 0; q < P; ++q) S[q] = h0 ? h0[q * NS + t] : 0.0f;
-        }
-        // S as the bf16 B operand of C . S^T: MN-major, row n holds 64 p.
-        auto write_S = [&](int buf) {
-            unsigned char* row = smem + OFF_S + buf * S_TILE + t * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(S[c * 8 + 2 * e], S[c * 8 + 2 * e + 1]);
-                *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_SREADY + buf));
-        };
         auto nrow_of = [&](int u) -> int {
             const int64_t t0 = (int64_t)u * UB;
             return (L - t0) < UB ? (int)(L - t0) : UB;
@@ -252,13 +265,21 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         auto load_dt = [&](int u) -> float {
             return t < nrow_of(u) ? p.delta[((b * L + (int64_t)u * UB + t) * p.nheads) + h] : 0.0f;
         };
-        // Per-block scalars of row t: cumulative log2-decay and the factors derived from it.
-        struct Blk { float cs, wt, et, gam; };
-        auto scan_block = [&](int u, float dt) -> Blk {
+        bool ok = true;
+        float dt_next = nblk > 0 ? load_dt(0) : 0.0f;
+        for (int u = 0; u < nblk && ok; ++u) {
+            cur_blk = u;
             const int k = u & 1;
+            const float dt = dt_next;
+            if (u + 1 < nblk) dt_next = load_dt(u + 1);
             float* cs_sm = reinterpret_cast<float*>(smem + OFF_CS) + k * UB;
             float* da_sm = reinterpret_cast<float*>(smem + OFF_DA) + k * UB;
             float* cf_sm = reinterpret_cast<float*>(smem + OFF_CF) + k * UB;
+            float* et_sm = reinterpret_cast<float*>(smem + OFF_ET) + k * UB;
+            float* gam_sm = reinterpret_cast<float*>(smem + OFF_GAM);
+            // the state warpgroup is done with block u-2's scalars and TMEM buffer k
+            if (u >= 2 && !(ok = wait(B_TFREE + k, (uint32_t)(((u - 2) >> 1) & 1)))) break;
+            // (a) cumulative log2-decay over the block
             float cs = dt * a_h;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -278,48 +299,22 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const float da = p.alpha * dt;
             cs_sm[t] = cs;
             da_sm[t] = da;
-            // column factor of column t against the last column of its 32-column batch
-            const float cs_ref = __shfl_sync(0xffffffffu, cs, 31);
+            const float cs_ref = __shfl_sync(0xffffffffu, cs, 31);   // last column of this 32-batch
             cf_sm[t] = ex2_approx(cs_ref - cs) * da;
+            et_sm[t] = ex2_approx(cs);                               // exp(cs_t)
+            if (t == 0) gam_sm[k] = ex2_approx(total);                // exp(cs_last)
+            const float wt = ex2_approx(total - cs) * da;            // exp(cs_last - cs_t) alpha delta_t
+            (reinterpret_cast<float*>(smem + OFF_WT) + k * UB)[t] = wt;
+            mbar_arrive(bar(B_SCAL + k));
             named_bar_sync(1, NCOMP);
-            Blk r;
-            r.cs = cs;
-            r.wt = ex2_approx(total - cs) * da;     // exp(cs_last - cs_t) alpha delta_t
-            r.et = ex2_approx(cs);                  // exp(cs_t)
-            r.gam = ex2_approx(total);              // exp(cs_last)
-            return r;
-        };
-        // Xhat = diag(w) X, row t, same swizzled layout as X.
-        auto make_xhat = [&](int u, float wt) -> bool {
-            if (!wait(B_FULL + (u & 1), (uint32_t)((u >> 1) & 1))) return false;
-            const unsigned char* xrow = smem + (u & 1) * SLOT + t * 128;
-            unsigned char* xh = smem + OFF_XHAT + t * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 q = *reinterpret_cast<const uint4*>(xrow + c * 16);
-                uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w4[e] = pack_bf16x2(bf16_lo(w4[e]) * wt, bf16_hi(w4[e]) * wt);
-                *reinterpret_cast<uint4*>(xh + c * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
+
+            // (b) first half of Xhat = diag(w) X (the state warpgroup does the other
+            //     half); X_hat is single-buffered: block u-1's state MMA must be done
+            if (u >= 1 && !(ok = wait(B_STATE, (uint32_t)((u - 1) & 1)))) break;
+            if (!(ok = wait(B_FULL + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
+            ssd_scale_row_half(smem + (u & 1) * SLOT + t * 128, smem + OFF_XHAT + t * 128, t, 0, wt);
             fence_proxy_async_smem();
             mbar_arrive(bar(B_XHAT));
-            return true;
-        };
-
-        write_S(0);
-        float dt_next = nblk > 1 ? load_dt(1) : 0.0f;
-        Blk cur = scan_block(0, load_dt(0));
-        bool ok = make_xhat(0, cur.wt);
-        for (int u = 0; u < nblk && ok; ++u) {
-            cur_blk = u;
-            const int k = u & 1;
-            const int64_t t0 = (int64_t)u * UB;
-            const int nrow = nrow_of(u);
-            const float* cs_sm = reinterpret_cast<const float*>(smem + OFF_CS) + k * UB;
-            const float* da_sm = reinterpret_cast<const float*>(smem + OFF_DA) + k * UB;
-            const float* cf_sm = reinterpret_cast<const float*>(smem + OFF_CF) + k * UB;
 
             // (c) M = CB o exp(cs_i - cs_j) alpha delta_j (j <= i), bf16 pairs into TMEM.
             //     Batches below the diagonal use exp(cs_i - cs_r) exp(cs_r - cs_j), both <= 1.
@@ -335,14 +330,25 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
                     tmem_wait_ld();
-                    if (cb < warp) {
-                        const float rowf = ex2_approx(cur.cs - cs_sm[cb * 32 + 31]);
+                    // Row factor 2^(cs_i - cs_r) and column factor 2^(cs_r - cs_j) alpha delta_j,
+                    // r = last column of the batch.  Below the diagonal both are <= 1; in the
+                    // diagonal batch the row factor is >= 1 but bounded by 2^(batch range),
+                    // so it is used only when that range stays far from fp32 overflow.
+                    const float cs_r = cs_sm[cb * 32 + 31];
+                    const bool factored = cb < warp || (cs_sm[cb * 32] - cs_r) <= 100.0f;
+                    if (factored) {
+                        const float rowf = ex2_approx(cs - cs_r);
                         const float2 rr = f2(rowf, rowf);
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const float2 cf = *reinterpret_cast<const float2*>(cf_sm + cb * 32 + 2 * e);
-                            const float2 m = __fmul2_rn(__fmul2_rn(f2(__uint_as_float(r[2 * e]),
-                                                                       __uint_as_float(r[2 * e + 1])), cf), rr);
+                            float2 m = __fmul2_rn(__fmul2_rn(f2(__uint_as_float(r[2 * e]),
+                                                                 __uint_as_float(r[2 * e + 1])), cf), rr);
+                            if (cb == warp) {      // causal mask inside the diagonal batch
+                                const int j = cb * 32 + 2 * e;
+                                m.x = j <= t ? m.x : 0.0f;
+                                m.y = j + 1 <= t ? m.y : 0.0f;
+                            }
                             pk[e] = pack_bf16x2(m.x, m.y);
                         }
                     } else {
@@ -350,7 +356,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
                             const int j = cb * 32 + jj;
-                            m[jj] = j <= t ? __uint_as_float(r[jj]) * (ex2_approx(cur.cs - cs_sm[j]) * da_sm[j]) : 0.0f;
+                            m[jj] = j <= t ? __uint_as_float(r[jj]) * (ex2_approx(cs - cs_sm[j]) * da_sm[j]) : 0.0f;
                         }
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
@@ -361,6 +367,52 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(B_M + k));
+        }
+    } else {
+        // ------------------------------------ state warpgroup (warps 4-7) ----
+        // Per block: S <- exp(cs_last) S + block state, the bf16 S operand for
+        // the next block, and the output y = Y_diag + exp(cs_i) Y_off.
+        const int t = tid - NCOMP;                 // TMEM lane = state n = row i
+        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        float S[P];                                 // row n = t of the state, fp32
+        {
+            const float* h0 = p.h0 ? p.h0 + (((b * p.nheads + h) * P) * NS) : nullptr;
+#pragma unroll
+            for (int q = 0; q < P; ++q) S[q] = h0 ? h0[q * NS + t] : 0.0f;
+        }
+        // S as the bf16 B operand of C . S^T: MN-major, row n holds 64 p.
+        auto write_S = [&](int buf) {
+            unsigned char* row = smem + OFF_S + buf * S_TILE + t * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(S[c * 8 + 2 * e], S[c * 8 + 2 * e + 1]);
+                *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_SREADY + buf));
+        };
+        // Second half of the rows of Xhat for block v (needs its w and its X tile).
+        auto xhat_half = [&](int v) -> bool {
+            if (!wait(B_SCAL + (v & 1), (uint32_t)((v >> 1) & 1))) return false;
+            if (!wait(B_FULL + (v & 1), (uint32_t)((v >> 1) & 1))) return false;
+            const float wt = (reinterpret_cast<const float*>(smem + OFF_WT) + (v & 1) * UB)[t];
+            ssd_scale_row_half(smem + (v & 1) * SLOT + t * 128, smem + OFF_XHAT + t * 128, t, 4, wt);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_XHAT));
+            return true;
+        };
+        write_S(0);
+        bool ok = nblk == 0 || xhat_half(0);
+        for (int u = 0; u < nblk && ok; ++u) {
+            cur_blk = u;
+            const int k = u & 1;
+            const int64_t t0 = (int64_t)u * UB;
+            const int nrow = (L - t0) < UB ? (int)(L - t0) : UB;
+            if (!(ok = wait(B_SCAL + k, (uint32_t)((u >> 1) & 1)))) break;
+            const float gam = reinterpret_cast<const float*>(smem + OFF_GAM)[k];
+            const float et = (reinterpret_cast<const float*>(smem + OFF_ET) + k * UB)[t];
 
             // (d) S <- exp(cs_last) S + block state; publish S for the next block
             if (!(ok = wait(B_STATE, (uint32_t)(u & 1)))) break;
@@ -372,21 +424,14 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tmem_ld32(tmem + lane_base + TM_STATE + hc * 32, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) S[hc * 32 + q] = fmaf(cur.gam, S[hc * 32 + q], __uint_as_float(r[q]));
+                    for (int q = 0; q < 32; ++q) S[hc * 32 + q] = fmaf(gam, S[hc * 32 + q], __uint_as_float(r[q]));
                 }
             }
             tc_fence_before();
             mbar_arrive(bar(B_SFREE));
             write_S((u + 1) & 1);
-
-            // next block's scan and Xhat while this block's output MMAs run
-            const float et = cur.et;
-            if (u + 1 < nblk) {
-                const float dt = dt_next;
-                if (u + 2 < nblk) dt_next = load_dt(u + 2);
-                cur = scan_block(u + 1, dt);
-                if (!(ok = make_xhat(u + 1, cur.wt))) break;
-            }
+            // block u's state MMA is complete, so X_hat may take block u+1
+            if (u + 1 < nblk && !(ok = xhat_half(u + 1))) break;
 
             // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of block u
             if (!(ok = wait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
