@@ -398,7 +398,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget", type=float, default=12.0)
-    ap.add_argument("--tile", default=None, help="force SPTxWARPS, e.g. 4x2 (tuning)")
+    ap.add_argument("--tile", default=None, help="force SPTxWARPS[xTIME_LANES], e.g. 4x2 or 4x2x2 (tuning)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -451,8 +451,8 @@ def main(argv=None):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     if args.tile:
-        spt, warps = (int(v) for v in args.tile.split("x"))
-        mm.mm_scan_set_tile(spt, warps)
+        parts = [int(v) for v in args.tile.split("x")]
+        mm.mm_scan_set_tile(parts[0], parts[1], parts[2] if len(parts) > 2 else 1)
 
     # Each rank scans its own batch (seed offset by rank): weak scaling.
     inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))

@@ -96,9 +96,12 @@ typedef struct {
  * (MM_ERR_ALIAS).
  *
  * Streaming: for a fixed (batch, dim, dstate, io), calling with the first
- * L1 steps and then with the remaining steps, passing (hT, vT) of the first
- * call as (h0, v0) of the second, gives final states bit-identical to one
- * call over all steps, and the same y within rounding of the read-out.
+ * L1 steps (L1 a multiple of 64) and then with the remaining steps,
+ * passing (hT, vT) of the first call as (h0, v0) of the second, gives final
+ * states bit-identical to one call over all steps, and the same y within
+ * rounding of the read-out.  (With one lane along time per state group the
+ * steps are applied in order and any L1 gives the same; the time split
+ * carries its state across 32-step chunks.)
  *
  * Errors: MM_ERR_NULL (x, delta, A, B, C, y or dims NULL), MM_ERR_DIMS
  * (a size < 1), MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE,
@@ -198,11 +201,13 @@ const char *mm_last_error(void);
 
 /*
  * Tuning knob for benchmarks: force the scan's per-thread state count
- * (2 or 4) and warps per block (1, 2 or 4); 0, 0 restores the automatic
- * choice.  Process-wide, not thread-safe with concurrent calls.  Returns
- * MM_ERR_UNSUPPORTED for a combination that is not built.
+ * (2, 4 or 8), warps per block (1, 2, 4 or 8) and lanes along time per
+ * state group (1, or 2 for the time split: fp32 I/O and 9..16 states
+ * only; other calls fall back to one lane).  0, 0, any restores the
+ * automatic choice.  Process-wide, not thread-safe with concurrent calls.
+ * Returns MM_ERR_UNSUPPORTED for a combination that is not built.
  */
-mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block);
+mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_lanes);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mm_version(void);

@@ -87,7 +87,7 @@ def _declare(lib):
     lib.mm_last_error.restype = ctypes.c_char_p
     lib.mm_last_error.argtypes = []
     lib.mm_scan_set_tile.restype = ctypes.c_int
-    lib.mm_scan_set_tile.argtypes = [ctypes.c_int, ctypes.c_int]
+    lib.mm_scan_set_tile.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.mm_version.restype = ctypes.c_int
     lib.mm_version.argtypes = []
     lib.mm_device_status.restype = ctypes.c_int
@@ -188,8 +188,9 @@ def mm_last_error() -> str:
     return load_library().mm_last_error().decode()
 
 
-def mm_scan_set_tile(states_per_thread: int, warps_per_block: int):
-    _check(load_library().mm_scan_set_tile(states_per_thread, warps_per_block), "mm_scan_set_tile")
+def mm_scan_set_tile(states_per_thread: int, warps_per_block: int, time_lanes: int = 1):
+    _check(load_library().mm_scan_set_tile(states_per_thread, warps_per_block, time_lanes),
+           "mm_scan_set_tile")
 
 
 def mm_version() -> int:

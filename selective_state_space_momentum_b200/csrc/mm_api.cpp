@@ -34,6 +34,7 @@ mm_status ok() {
 
 std::atomic<int> g_forced_spt{0};
 std::atomic<int> g_forced_warps{0};
+std::atomic<int> g_forced_ts{1};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -106,16 +107,19 @@ mm_status mm_device_status(void) {
     return ok();
 }
 
-mm_status mm_scan_set_tile(int spt, int warps) {
+mm_status mm_scan_set_tile(int spt, int warps, int time_lanes) {
     if (spt == 0 && warps == 0) {
         g_forced_spt = 0;
         g_forced_warps = 0;
+        g_forced_ts = 1;
         return ok();
     }
-    if (!mmscan::scan_tile_supported(spt, warps))
-        return fail(MM_ERR_UNSUPPORTED, "scan tile spt=%d warps=%d is not built", spt, warps);
+    if (!mmscan::scan_tile_supported(spt, warps, time_lanes))
+        return fail(MM_ERR_UNSUPPORTED, "scan tile spt=%d warps=%d time_lanes=%d is not built", spt,
+                    warps, time_lanes);
     g_forced_spt = spt;
     g_forced_warps = warps;
+    g_forced_ts = time_lanes;
     return ok();
 }
 
@@ -176,7 +180,8 @@ mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const vo
     a.beta = beta; a.alpha = alpha;
     a.vec_ok = ((L * esize) % 16) == 0;
     const mmscan::ScanTileChoice t =
-        mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load());
+        mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load(),
+                                 g_forced_ts.load());
     return from_cuda(mmscan::launch_scan_fwd(a, t, dims->io, static_cast<cudaStream_t>(stream)),
                      "mm_scan_fwd launch");
 }

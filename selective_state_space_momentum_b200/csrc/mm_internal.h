@@ -30,12 +30,13 @@ struct ScanArgs {
 struct ScanTileChoice {
     int np;      // states padded to a power of two (2, 4, 8, 16)
     int spt;     // states per lane (2 or 4)
-    int warps;   // warps per CTA (1, 2 or 4)
+    int warps;   // warps per CTA (1, 2, 4 or 8)
+    int ts;      // lanes along time per state group (1, or 2 for the time split)
 };
 
-bool scan_tile_supported(int spt, int warps);
+bool scan_tile_supported(int spt, int warps, int time_lanes);
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
-                                int forced_spt, int forced_warps);
+                                int forced_spt, int forced_warps, int forced_ts);
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s);
 // Read (and reset) the device error word of the scan / SSD kernels.
 unsigned int scan_read_and_clear_device_error();

@@ -45,16 +45,19 @@ namespace mmscan {
 // Device error word of this file's kernels (bounded waits that gave up).
 static __device__ unsigned int g_scan_dev_err = 0;
 
-template <typename IO, int NP, int SPT, int WARPS>
+template <typename IO, int NP, int SPT, int WARPS, int TS>
 struct ScanTile {
-    static constexpr int G = NP / SPT;           // lanes per channel
-    static constexpr int CPW = 32 / G;           // channels per warp
+    static constexpr int G = NP / SPT;           // lanes per (channel, time-lane)
+    static constexpr int CPW = 32 / (G * TS);    // channels per warp
     static constexpr int CH = WARPS * CPW;       // channels per CTA
     static constexpr int NT = WARPS * 32;        // threads per CTA
+    // The time split doubles the warps; 12 resident warps per SM (<= 168 registers)
+    // hold the medium-size grids in one wave.
+    static constexpr int MIN_CTAS = TS == 2 ? (12 / WARPS > 0 ? 12 / WARPS : 1) : 1;
     static constexpr int NPAIR = SPT / 2;
     static constexpr int EB = IOTraits<IO>::kBytes;
     static constexpr int BOX_T = 128 / EB;       // steps in one 128-byte swizzled row
-    static constexpr int T = 64;                 // steps per chunk
+    static constexpr int T = TS == 1 ? 64 : 32;  // steps per chunk
     static constexpr int NBOX = T / BOX_T;       // boxes per row per chunk
     static constexpr int STAGES = 3;             // chunks in flight
     static constexpr int NPT = NP < 8 ? 8 : NP;  // B/C rows per box (whole swizzle atoms)
@@ -69,11 +72,8 @@ struct ScanTile {
     static constexpr int BP = NP + 4;            // row pitch (floats) of transposed B/C
     static constexpr int BT_BYTES = T * BP * 4;
     static constexpr int R = 8;                  // steps per inner group
-    static constexpr int YW_PITCH = R * G + G;   // floats per channel in the read-out buffer
-    static constexpr int YW_BYTES = CPW * YW_PITCH * 4;   // per warp
     static constexpr int OFF_BT = STAGES * STAGE_BYTES;    // 2 buffers of B^T, then 2 of C^T
-    static constexpr int OFF_YW = OFF_BT + 4 * BT_BYTES;
-    static constexpr int OFF_BAR = OFF_YW + WARPS * YW_BYTES;
+    static constexpr int OFF_BAR = OFF_BT + 4 * BT_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
 
     static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "lanes per channel");
@@ -82,6 +82,8 @@ struct ScanTile {
     static_assert(CH % 8 == 0, "x tiles must be whole 1024-byte swizzle atoms");
     static_assert(STAGE_BYTES % 1024 == 0 && (OFF_BT % 16) == 0, "alignment");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+    static_assert(TS == 1 || (TS == 2 && EB == 4 && T == 2 * 2 * R && (G == 4 || G == 8)),
+                  "time split: fp32 I/O, two groups per lane, 4 or 8 lanes per channel");
 };
 
 // Store `cnt` consecutive steps of one output row.
@@ -119,12 +121,44 @@ __device__ __forceinline__ void store_steps_n(IO* dst, const float (&v)[PER], in
         if (i < cnt) store1(dst + i, v[i]);
 }
 
-template <typename IO, int NP, int SPT, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32)
+// Sum, over the G consecutive lanes of a group, of K per-lane partials: a
+// butterfly that halves the values each lane carries at every stage (the lane
+// whose bit m is set keeps the upper half), so that group lane g ends with
+// the sums of entries [g K/G, (g+1) K/G) after log2 G exchanges of K/2, K/4,
+// ... values.  The exchanges stay in registers: no shared-memory traffic.
+template <int G, int K>
+__device__ __forceinline__ void butterfly_sum(const float (&v)[K], float (&out)[K / G], int g) {
+    static_assert((G & (G - 1)) == 0 && K % G == 0, "power-of-two group dividing K");
+    float cur[K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) cur[i] = v[i];
+#pragma unroll
+    for (int m = G / 2, n = K; m >= 1; m >>= 1, n >>= 1) {
+        const bool upper = (g & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float keep = upper ? cur[n / 2 + i] : cur[i];
+            const float send = upper ? cur[i] : cur[n / 2 + i];
+            cur[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < K / G; ++e) out[e] = cur[e];
+}
+
+__device__ __forceinline__ float2 shfl_up_f2(float2 v, int delta) {
+    return f2(__shfl_up_sync(0xffffffffu, v.x, delta), __shfl_up_sync(0xffffffffu, v.y, delta));
+}
+__device__ __forceinline__ float2 shfl_down_f2(float2 v, int delta) {
+    return f2(__shfl_down_sync(0xffffffffu, v.x, delta), __shfl_down_sync(0xffffffffu, v.y, delta));
+}
+
+template <typename IO, int NP, int SPT, int WARPS, int TS>
+__global__ void __launch_bounds__(WARPS * 32, ScanTile<IO, NP, SPT, WARPS, TS>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                 const ScanArgs p) {
-    using TL = ScanTile<IO, NP, SPT, WARPS>;
+    using TL = ScanTile<IO, NP, SPT, WARPS, TS>;
     constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
     constexpr int ST = TL::STAGES, NPAIR = TL::NPAIR, EB = TL::EB, BP = TL::BP;
 
@@ -137,12 +171,16 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int g = lane % G;
-    const int cw = lane / G;
+    const int yrow_id = lane / G;                    // (time-lane, channel) row of the read-out buffer
+    const int j_t = yrow_id % TS;                    // time-lane: which half of each chunk (TS == 2)
+    const int cw = yrow_id / TS;
     const int c = warp * CPW + cw;                   // channel within the CTA
     const int64_t b = blockIdx.x / p.tiles_per_batch;
     const int64_t d0 = (int64_t)(blockIdx.x % p.tiles_per_batch) * CH;
     const int64_t d = d0 + c;
     const bool active = d < p.dim;
+    // Lanes that own the carried state, store y and write the final state.
+    const bool writer = active && (TS == 1 || j_t == 0);
     const int64_t L = p.seqlen;
     const int N = p.dstate;
     const int64_t nchunks = (L + T - 1) / T;
@@ -170,7 +208,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int n = g * SPT + 2 * q + e;
-            if (active && n < N) {
+            if (writer && n < N) {
                 const int64_t si = (b * p.dim + d) * N + n;
                 if (p.h0) hv[e] = p.h0[si];
                 if (p.v0) vw[e] = p.v0[si];
@@ -240,7 +278,6 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     for (int s = 0; s < ST - 1; ++s)
         if (s < nchunks) issue(s, s);
 
-    float* yw = reinterpret_cast<float*>(smem + TL::OFF_YW + warp * TL::YW_BYTES) + cw * TL::YW_PITCH;
     IO* yrow = static_cast<IO*>(p.y) + (b * p.dim + (active ? d : 0)) * L;
     const bool vec_out = use_tma;
 
@@ -329,44 +366,28 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
         };
 
+        // ---- add the G partials of each channel; store y --------------------
         auto reduce_store = [&](int tau0, const float (&yk)[R]) {
-                // ---- add the G partials of each channel; store y -------------
-                constexpr int PER = R / G;      // steps each lane finishes
-                float out[PER];
-                if constexpr (G == 1) {
-    #pragma unroll
-                    for (int j = 0; j < R; ++j) out[j] = yk[j];
-                } else {
-    #pragma unroll
-                    for (int j = 0; j < R; ++j) yw[j * G + g] = yk[j];
-                    __syncwarp();
-    #pragma unroll
-                    for (int e = 0; e < PER; ++e) {
-                        const float* src = yw + (g * PER + e) * G;
-                        float acc = 0.0f;
-    #pragma unroll
-                        for (int gg = 0; gg < G; gg += (G >= 4 ? 4 : G)) {
-                            if constexpr (G >= 4) {
-                                const float4 q4 = *reinterpret_cast<const float4*>(src + gg);
-                                acc += (q4.x + q4.y) + (q4.z + q4.w);
-                            } else {
-                                const float2 q2 = *reinterpret_cast<const float2*>(src + gg);
-                                acc += q2.x + q2.y;
-                            }
-                        }
-                        out[e] = acc;
-                    }
-                    __syncwarp();
-                }
-                const int first = tau0 + g * PER;      // step (within the chunk) of out[0]
-                const int cnt = nval - first < PER ? nval - first : PER;
-                if (active && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
+            constexpr int PER = R / G;      // steps each lane finishes
+            float out[PER];
+            butterfly_sum<G, R>(yk, out, g);
+            const int first = tau0 + g * PER;      // step (within the chunk) of out[0]
+            const int cnt = nval - first < PER ? nval - first : PER;
+            if (writer && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
+        };
+        // The same for the 16 steps of one half chunk (time split); both halves store.
+        auto reduce16_store = [&](int tau0, const float (&yk)[16]) {
+            constexpr int PER = 16 / G;
+            float out[PER];
+            butterfly_sum<G, 16>(yk, out, g);
+            const int first = tau0 + g * PER;
+            const int cnt = nval - first < PER ? nval - first : PER;
+            if (active && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
         };
 
-        // The R full steps of group gi, then the read-out reduction and store.
-        auto full_steps = [&](int gi, const float (&u)[R], const float (&a)[R][SPT]) {
+        // The R full steps of group gi from the lane's state; per-lane partial y into yk.
+        auto group_steps = [&](int gi, const float (&u)[R], const float (&a)[R][SPT], float (&yk)[R]) {
             const int tau0 = gi * R;
-            float yk[R];
 #pragma unroll
             for (int j = 0; j < R; ++j) {
                 const float* brow = Bg + (tau0 + j) * BP;
@@ -397,25 +418,15 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 yk[j] = yy.x + yy.y;
             }
-            reduce_store(tau0, yk);
+        };
+        auto full_steps = [&](int gi, const float (&u)[R], const float (&a)[R][SPT]) {
+            float yk[R];
+            group_steps(gi, u, a, yk);
+            reduce_store(gi * R, yk);
         };
 
-        if (nval == T) {
-            // Full chunk: groups unrolled, each group's exponentials issued one group ahead.
-            constexpr int NG = T / R;
-            float uA[R], uB[R], aA[R][SPT], aB[R][SPT];
-            prep(0, uA, aA);
-#pragma unroll
-            for (int gi = 0; gi < NG; ++gi) {
-                if ((gi & 1) == 0) {
-                    if (gi + 1 < NG) prep(gi + 1, uB, aB);
-                    full_steps(gi, uA, aA);
-                } else {
-                    if (gi + 1 < NG) prep(gi + 1, uA, aA);
-                    full_steps(gi, uB, aB);
-                }
-            }
-        } else {
+        // The remaining nval < T steps of the sequence, one group at a time.
+        auto ragged_chunk = [&]() {
             const int ngroups = (nval + R - 1) / R;
             for (int gi = 0; gi < ngroups; ++gi) {
                 const int tau0 = gi * R;
@@ -504,11 +515,116 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
                 reduce_store(tau0, yk);
             }
+        };
+
+        if constexpr (TS == 1) {
+            if (nval == T) {
+                // Full chunk: groups unrolled, each group's exponentials issued one group ahead.
+                constexpr int NG = T / R;
+                float uA[R], uB[R], aA[R][SPT], aB[R][SPT];
+                prep(0, uA, aA);
+#pragma unroll
+                for (int gi = 0; gi < NG; ++gi) {
+                    if ((gi & 1) == 0) {
+                        if (gi + 1 < NG) prep(gi + 1, uB, aB);
+                        full_steps(gi, uA, aA);
+                    } else {
+                        if (gi + 1 < NG) prep(gi + 1, uA, aA);
+                        full_steps(gi, uB, aB);
+                    }
+                }
+            } else {
+                ragged_chunk();
+            }
+        } else {
+            // ---- time split: lane half j_t runs steps [16 j_t, 16 j_t + 16) ----
+            // The first half starts from the carried state, the second from zero.
+            // The recurrence is linear in its start state (v_in, h_in), so the
+            // second half's true state is its zero-start state plus the response
+            // to (v_in, h_in) alone:  b_t = beta^(t+1) v_in,  c_t = a_t c_{t-1} + b_t
+            // with c_{-1} = h_in, which adds C_t . c_t to y_t and (b, c) at the end
+            // to (v, h).  The 2x2 carry [[beta, 0], [beta, a_t]] is thus applied
+            // across the two halves with one shuffle each way.
+            if (nval == T) {
+                constexpr int HALF = T / 2;
+                const int gi0 = 2 * j_t;
+                float uA[R], uB[R], aA[R][SPT], aB[R][SPT], yk[HALF];
+                prep(gi0, uA, aA);
+                prep(gi0 + 1, uB, aB);
+                {
+                    float y8[R];
+                    group_steps(gi0, uA, aA, y8);
+#pragma unroll
+                    for (int j = 0; j < R; ++j) yk[j] = y8[j];
+                    group_steps(gi0 + 1, uB, aB, y8);
+#pragma unroll
+                    for (int j = 0; j < R; ++j) yk[R + j] = y8[j];
+                }
+                float2 bv[NPAIR], cc[NPAIR];
+                const float2 zero2 = f2(0.0f, 0.0f);
+#pragma unroll
+                for (int q = 0; q < NPAIR; ++q) {      // first-half lanes take zeros: exact no-op
+                    const float2 vi = shfl_up_f2(vv[q], G);
+                    const float2 hi = shfl_up_f2(hh[q], G);
+                    bv[q] = j_t ? vi : zero2;
+                    cc[q] = j_t ? hi : zero2;
+                }
+                const float* Ch = Cg + (gi0 * R) * BP;
+#pragma unroll
+                for (int t = 0; t < HALF; ++t) {
+                    const float* crow = Ch + t * BP;
+                    float cq[SPT];
+                    if constexpr (SPT >= 4) {
+#pragma unroll
+                        for (int q = 0; q < SPT; q += 4) {
+                            const float4 c4 = *reinterpret_cast<const float4*>(crow + q);
+                            cq[q] = c4.x; cq[q + 1] = c4.y; cq[q + 2] = c4.z; cq[q + 3] = c4.w;
+                        }
+                    } else {
+                        const float2 c2 = *reinterpret_cast<const float2*>(crow);
+                        cq[0] = c2.x; cq[1] = c2.y;
+                    }
+                    float2 yy = zero2;
+#pragma unroll
+                    for (int q = 0; q < NPAIR; ++q) {
+                        const float a0 = t < R ? aA[t][2 * q] : aB[t - R][2 * q];
+                        const float a1 = t < R ? aA[t][2 * q + 1] : aB[t - R][2 * q + 1];
+                        bv[q] = __fmul2_rn(beta2, bv[q]);
+                        cc[q] = __ffma2_rn(f2(a0, a1), cc[q], bv[q]);
+                        yy = __ffma2_rn(f2(cq[2 * q], cq[2 * q + 1]), cc[q], yy);
+                    }
+                    yk[t] += yy.x + yy.y;
+                }
+#pragma unroll
+                for (int q = 0; q < NPAIR; ++q) {
+                    vv[q] = __fadd2_rn(vv[q], bv[q]);
+                    hh[q] = __fadd2_rn(hh[q], cc[q]);
+                }
+                reduce16_store(gi0 * R, yk);
+                // The second half's end state is the next chunk's start, in the first half's lanes.
+#pragma unroll
+                for (int q = 0; q < NPAIR; ++q) {
+                    const float2 vn = shfl_down_f2(vv[q], G);
+                    const float2 hn = shfl_down_f2(hh[q], G);
+                    vv[q] = j_t ? zero2 : vn;
+                    hh[q] = j_t ? zero2 : hn;
+                }
+            } else {
+                // Ragged end of the sequence: the second half's lanes take the carried
+                // state and repeat the first half's work; only the first half stores.
+#pragma unroll
+                for (int q = 0; q < NPAIR; ++q) {
+                    const float2 vi = shfl_up_f2(vv[q], G);
+                    const float2 hi = shfl_up_f2(hh[q], G);
+                    if (j_t) { vv[q] = vi; hh[q] = hi; }
+                }
+                ragged_chunk();
+            }
         }
     }
 
     // ---- final states -------------------------------------------------------
-    if (active) {
+    if (writer) {
 #pragma unroll
         for (int q = 0; q < NPAIR; ++q) {
 #pragma unroll
@@ -562,9 +678,9 @@ cudaError_t make_map_3d(CUtensorMap* m, const void* base, bool bf16_elems, uint6
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename IO, int NP, int SPT, int WARPS>
+template <typename IO, int NP, int SPT, int WARPS, int TS = 1>
 cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
-    using TL = ScanTile<IO, NP, SPT, WARPS>;
+    using TL = ScanTile<IO, NP, SPT, WARPS, TS>;
     ScanArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t grid = a.batch * a.tiles_per_batch;
@@ -582,7 +698,7 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
         if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
         if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
     }
-    auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS>;
+    auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS, TS>;
     // The dynamic shared-memory limit is raised once per device and variant.
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
@@ -601,7 +717,19 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
 // Variants that are built: (states per lane, warps per CTA) for 16 padded states,
 // and the natural choices for smaller state counts.
 template <typename IO>
-cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, cudaStream_t s) {
+cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, int ts, cudaStream_t s) {
+    if (ts == 2) {
+        // Time split: fp32 I/O and 16 padded states only.
+        if constexpr (sizeof(IO) == 4) {
+            if (np == 16) {
+                if (spt == 4 && warps == 2) return launch_variant<IO, 16, 4, 2, 2>(a, s);
+                if (spt == 4 && warps == 4) return launch_variant<IO, 16, 4, 4, 2>(a, s);
+                if (spt == 2 && warps == 4) return launch_variant<IO, 16, 2, 4, 2>(a, s);
+                if (spt == 2 && warps == 8) return launch_variant<IO, 16, 2, 8, 2>(a, s);
+            }
+        }
+        return cudaErrorInvalidValue;
+    }
     switch (np) {
         case 16:
             if (spt == 2 && warps == 2) return launch_variant<IO, 16, 2, 2>(a, s);
@@ -628,32 +756,38 @@ cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, cudaStream_
 
 }  // namespace
 
-bool scan_tile_supported(int spt, int warps) {
+bool scan_tile_supported(int spt, int warps, int time_lanes) {
+    if (time_lanes == 2)
+        return (spt == 4 && (warps == 2 || warps == 4)) || (spt == 2 && (warps == 4 || warps == 8));
+    if (time_lanes != 1) return false;
     return (spt == 2 && (warps == 2 || warps == 4 || warps == 8)) ||
            (spt == 4 && (warps == 1 || warps == 2 || warps == 4)) ||
            (spt == 8 && (warps == 1 || warps == 2));
 }
 
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
-                                int forced_spt, int forced_warps) {
-    (void)io;
-    // The choice depends on (batch * dim, dstate) only, never on L, so calls
+                                int forced_spt, int forced_warps, int forced_ts) {
+    // The choice depends on (batch * dim, dstate, io) only, never on L, so calls
     // that split one sequence use the same variant.  Fewer states per lane
     // give more warps (needed when there are few channels); more states per
     // lane need fewer instructions per update.
     ScanTileChoice t;
     t.np = dstate <= 2 ? 2 : dstate <= 4 ? 4 : dstate <= 8 ? 8 : 16;
+    t.ts = 1;
+    // Two states per lane (8 lanes per channel) keep about 2.5 warps per
+    // scheduler on the medium and bf16 workloads; four-warp CTAs share each
+    // B/C transpose over 16 channels.
     const int64_t channels = batch * dim;
-    if (channels >= 4096) {
-        t.spt = 4;
-        t.warps = 2;
-    } else {
-        t.spt = 2;
-        t.warps = 2;
-    }
+    t.spt = 2;
+    t.warps = channels >= 2048 ? 4 : 2;
     if (t.np == 16 && forced_spt) {
         t.spt = forced_spt;
         t.warps = forced_warps;
+        t.ts = (forced_ts == 2 && io == 0) ? 2 : 1;
+        if (t.ts == 1 && !scan_tile_supported(t.spt, t.warps, 1)) {
+            t.spt = 4;
+            t.warps = 2;
+        }
     }
     if (t.np == 8 && forced_spt) t.spt = forced_spt == 8 ? 4 : forced_spt;
     if (t.np == 8 && t.spt > 4) t.spt = 4;
@@ -661,8 +795,8 @@ ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int 
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s) {
-    if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, s);
-    return launch_io<bf16>(a, t.np, t.spt, t.warps, s);
+    if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, t.ts, s);
+    return launch_io<bf16>(a, t.np, t.spt, t.warps, t.ts, s);
 }
 
 unsigned int scan_read_and_clear_device_error() {

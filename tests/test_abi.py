@@ -109,9 +109,12 @@ def test_scan_fault_injection_returns_cuda_error(lib, monkeypatch):
 
 
 def test_set_tile(lib):
-    assert lib.mm_scan_set_tile(3, 2) == 6
-    assert lib.mm_scan_set_tile(4, 2) == 0
-    assert lib.mm_scan_set_tile(0, 0) == 0
+    assert lib.mm_scan_set_tile(3, 2, 1) == 6
+    assert lib.mm_scan_set_tile(4, 2, 3) == 6
+    assert lib.mm_scan_set_tile(4, 1, 2) == 6                    # time split needs >= 8 channels per CTA
+    assert lib.mm_scan_set_tile(4, 2, 1) == 0
+    assert lib.mm_scan_set_tile(4, 2, 2) == 0
+    assert lib.mm_scan_set_tile(0, 0, 0) == 0
 
 
 def test_ssd_rejects_bad_arguments(lib, monkeypatch):

@@ -195,14 +195,74 @@ def test_every_tile_variant_matches(io):
     yr, hr, vr = oracle.scan_seq(**inp, beta=0.9, alpha=1.0)
     try:
         for spt, warps in ((2, 2), (2, 4), (2, 8), (4, 1), (4, 2), (4, 4)):
-                mm.mm_scan_set_tile(spt, warps)
+                mm.mm_scan_set_tile(spt, warps, 1)
                 got = _run(dev, 0.9, 1.0)
                 _compare(io, (got[0].reshape(-1, 200), got[1].reshape(-1, 16), got[2].reshape(-1, 16)),
                          (yr, hr, vr), f"tile spt={spt} warps={warps}")
                 # the per-state arithmetic is the same in every variant
                 assert np.array_equal(got[1], base[1]) and np.array_equal(got[2], base[2])
     finally:
-        mm.mm_scan_set_tile(0, 0)
+        mm.mm_scan_set_tile(0, 0, 1)
+
+
+TIME_SPLIT_TILES = ((4, 2), (4, 4), (2, 4), (2, 8))
+
+
+def test_time_split_variants_match_and_agree_on_state():
+    """fp32 variants with two lanes along time per state group: each matches
+    the oracle (ragged last chunk, carried initial state), and all give the
+    same final states, since the per-state arithmetic does not depend on
+    how states are spread over lanes."""
+    inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=2, seqlen=200, dim=70)
+    dev = _dev(inp, "f32")
+    rng = np.random.default_rng(4)
+    h0 = rng.standard_normal((2, 70, 16)).astype(np.float32)
+    v0 = rng.standard_normal((2, 70, 16)).astype(np.float32)
+    th0, tv0 = torch.from_numpy(h0).cuda(), torch.from_numpy(v0).cuda()
+    yr, hr, vr = oracle.scan_seq(**inp, h0=h0.astype(np.float64), v0=v0.astype(np.float64),
+                                 beta=0.9, alpha=1.0)
+    first = None
+    try:
+        for spt, warps in TIME_SPLIT_TILES:
+            mm.mm_scan_set_tile(spt, warps, 2)
+            got = _run(dev, 0.9, 1.0, th0, tv0)
+            _compare("f32", (got[0].reshape(-1, 200), got[1].reshape(-1, 16), got[2].reshape(-1, 16)),
+                     (yr, hr, vr), f"time split spt={spt} warps={warps}")
+            if first is None:
+                first = got
+            assert np.array_equal(got[1], first[1]) and np.array_equal(got[2], first[2])
+    finally:
+        mm.mm_scan_set_tile(0, 0, 1)
+
+
+@pytest.mark.parametrize("L", [1, 31, 32, 33, 64, 65, 130])
+@pytest.mark.parametrize("beta", [0.0, 0.9])
+def test_time_split_lengths(L, beta):
+    inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=1, seqlen=L, dim=24)
+    try:
+        mm.mm_scan_set_tile(4, 2, 2)
+        _full_compare(inp, "f32", beta, 1.0, what=f"time split L={L} beta={beta}")
+    finally:
+        mm.mm_scan_set_tile(0, 0, 1)
+
+
+def test_time_split_streaming_bit_identical():
+    inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=2, seqlen=448, dim=40)
+    dev = _dev(inp, "f32")
+    try:
+        mm.mm_scan_set_tile(4, 2, 2)
+        one = _run(dev, 0.99, 1.0)
+        for half in (64, 192, 384):
+            d1 = {k: (v[..., :half].contiguous() if k in ("x", "delta", "B", "C") else v) for k, v in dev.items()}
+            d2 = {k: (v[..., half:].contiguous() if k in ("x", "delta", "B", "C") else v) for k, v in dev.items()}
+            y1, h1, v1 = mm.scan_fwd(d1["x"], d1["delta"], d1["A"], d1["B"], d1["C"], beta=0.99, alpha=1.0)
+            y2, h2, v2 = mm.scan_fwd(d2["x"], d2["delta"], d2["A"], d2["B"], d2["C"], h0=h1, v0=v1,
+                                     beta=0.99, alpha=1.0)
+            torch.cuda.synchronize()
+            assert np.array_equal(h2.cpu().numpy(), one[1]), f"hT differs (split at {half})"
+            assert np.array_equal(v2.cpu().numpy(), one[2]), f"vT differs (split at {half})"
+    finally:
+        mm.mm_scan_set_tile(0, 0, 1)
 
 
 def test_in_place_streaming_state_and_optional_outputs():
