@@ -59,15 +59,15 @@ constexpr int SLOT = X_TILE + 2 * BC_TILE;  // 80 KB: X, B, C of one block
 constexpr int OFF_XHAT = 2 * SLOT;
 constexpr int S_TILE = NS * P * 2;         // 16 KB: [128 rows n][64 p] bf16, swizzled
 constexpr int OFF_S = OFF_XHAT + X_TILE;    // 2 S buffers
-constexpr int OFF_CS = OFF_S + 2 * S_TILE;  // cs[2][128] fp32 (log2 units)
+constexpr int Y_STAGE = UB * 32 * 2;       // 8 KB: half a y tile, [128 rows][32] bf16, 64-byte swizzle
+constexpr int OFF_YST = OFF_S + 2 * S_TILE;
+constexpr int OFF_CS = OFF_YST + Y_STAGE;   // cs[2][128] fp32 (log2 units)
 constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha*delta[2][128]
 constexpr int OFF_CF = OFF_DA + 2 * UB * 4; // column factors [2][128]
-constexpr int OFF_ET = OFF_CF + 2 * UB * 4; // exp(cs_t) [2][128]
-constexpr int OFF_WT = OFF_ET + 2 * UB * 4;  // exp(cs_last - cs_t) alpha delta_t [2][128]
-constexpr int OFF_GAM = OFF_WT + 2 * UB * 4;   // exp(cs_last) [2]
-constexpr int OFF_RED = OFF_GAM + 16;
+constexpr int OFF_WT = OFF_CF + 2 * UB * 4;  // exp(cs_last - cs_t) alpha delta_t [2][128]
+constexpr int OFF_RED = OFF_WT + 2 * UB * 4;
 constexpr int OFF_BAR = OFF_RED + 64;
-constexpr int NBAR = 20;
+constexpr int NBAR = 24;
 constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TSLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
@@ -83,27 +83,13 @@ constexpr uint32_t TM_COLS = 512;
 // barrier could run two phases ahead of its waiter.
 enum { B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_TFREE = 10,
        B_XHAT = 12, B_STATE = 13, B_SFREE = 14, B_SREADY = 15 /* and 16 */,
-       B_SCAL = 17 /* and 18: per-block scalars ready for the state warpgroup */ };
+       B_SCAL = 17 /* and 18: per-block scalars ready for the state warpgroup */,
+       B_FULLX = 19, B_EMPTYX = 21 /* X part of a slot; B_FULL / B_EMPTY cover its B and C */ };
 constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
 constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . Xhat (both MN-major)
 constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // M(tmem) . X (X MN-major)
 constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 1);   // C . S^T (S MN-major)
 }  // namespace ssd
-
-// Xhat row t, 16-byte chunks c0..c0+3 (logical order; the physical chunk
-// index is swizzled so a warp touches 8 different bank groups).
-__device__ __forceinline__ void ssd_scale_row_half(const unsigned char* xrow, unsigned char* xh, int t,
-                                                   int c0, float wt) {
-#pragma unroll
-    for (int c = c0; c < c0 + 4; ++c) {
-        const int pc = (c ^ (t & 7)) << 4;
-        const uint4 q = *reinterpret_cast<const uint4*>(xrow + pc);
-        uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(bf16_lo(w4[e]) * wt, bf16_hi(w4[e]) * wt);
-        *reinterpret_cast<uint4*>(xh + pc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-    }
-}
 
 struct SSDKArgs {
     const float* delta;
@@ -118,7 +104,8 @@ struct SSDKArgs {
 
 __global__ void __launch_bounds__(ssd::NTHREADS, 1)
 ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
-               const __grid_constant__ CUtensorMap tm_C, const SSDKArgs p) {
+               const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
+               const SSDKArgs p) {
     using namespace ssd;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -139,11 +126,13 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     if (tid == 0) {
         mbar_init(bar(B_FULL + 0), 1); mbar_init(bar(B_FULL + 1), 1);
         mbar_init(bar(B_EMPTY + 0), 1); mbar_init(bar(B_EMPTY + 1), 1);
+        mbar_init(bar(B_FULLX + 0), 1); mbar_init(bar(B_FULLX + 1), 1);
+        mbar_init(bar(B_EMPTYX + 0), 1); mbar_init(bar(B_EMPTYX + 1), 1);
         mbar_init(bar(B_CB + 0), 1); mbar_init(bar(B_CB + 1), 1);
         mbar_init(bar(B_M + 0), NCOMP); mbar_init(bar(B_M + 1), NCOMP);
         mbar_init(bar(B_Y + 0), 1); mbar_init(bar(B_Y + 1), 1);
         mbar_init(bar(B_TFREE + 0), NCOMP); mbar_init(bar(B_TFREE + 1), NCOMP);
-        mbar_init(bar(B_XHAT), 2 * NCOMP);   // both warpgroups write half of each row
+        mbar_init(bar(B_XHAT), NCOMP);
         mbar_init(bar(B_STATE), 1);
         mbar_init(bar(B_SFREE), NCOMP);
         mbar_init(bar(B_SREADY + 0), NCOMP); mbar_init(bar(B_SREADY + 1), NCOMP);
@@ -176,22 +165,29 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             for (int u = 0; u < nblk; ++u) {
                 cur_blk = u;
                 const int s = u & 1;
+                // B and C of a slot are released once the block's state and Y_off
+                // products are done, X only after Y_diag, which waits for the mask:
+                // the two parts are refilled separately.
                 if (!wait(B_EMPTY + s, (uint32_t)(((u >> 1) + 1) & 1))) break;
                 const uint32_t slot = base + s * SLOT;
                 const uint32_t fb = bar(B_FULL + s);
-                mbar_expect_tx(fb, SLOT);
+                mbar_expect_tx(fb, 2 * BC_TILE);
                 const int t0 = u * UB;
-                tma_load_4d(slot, &tm_x, fb, 0, (int)h, t0, (int)b);
                 tma_load_4d(slot + X_TILE, &tm_B, fb, 0, (int)g, t0, (int)b);
                 tma_load_4d(slot + X_TILE + BC_SLAB, &tm_B, fb, 64, (int)g, t0, (int)b);
                 tma_load_4d(slot + X_TILE + BC_TILE, &tm_C, fb, 0, (int)g, t0, (int)b);
                 tma_load_4d(slot + X_TILE + BC_TILE + BC_SLAB, &tm_C, fb, 64, (int)g, t0, (int)b);
+                if (!wait(B_EMPTYX + s, (uint32_t)(((u >> 1) + 1) & 1))) break;
+                const uint32_t fx = bar(B_FULLX + s);
+                mbar_expect_tx(fx, X_TILE);
+                tma_load_4d(slot, &tm_x, fx, 0, (int)h, t0, (int)b);
             }
         }
     } else if (warp == W_MMA) {
         // ----------------------------------------------------------- MMA ----
-        // Issue order per block u: block state(u), C.B^T(u+1) (one block
-        // ahead, so the mask warpgroup can start on it), then Y(u).
+        // Issue order per block u: block state(u), Y_off(u) (needs only the
+        // previous state, and frees the block's B and C), C.B^T(u+1) (one block
+        // ahead, so the mask warpgroup can start on it), then Y_diag(u).
         if (lane == 0) {
             const uint32_t xhat = base + OFF_XHAT;
             auto issue_cb = [&](int v) -> bool {
@@ -226,15 +222,9 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     umma_ss(tmem + TM_STATE, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
                             umma_desc_sw128(xhat + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
                 umma_commit(bar(B_STATE));
-                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
-                // Y_diag = M(tmem) . X and Y_off = C . S_prev^T
-                if (!(live = wait(B_M + k, (uint32_t)((u >> 1) & 1)))) break;
+                // Y_off = C . S_prev^T
                 if (!(live = wait(B_SREADY + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_ts(tmem + tm_cb(k) + 64, tmem + tm_cb(k) + ks * 8,
-                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
                 const uint32_t sb = base + OFF_S + (u & 1) * S_TILE;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
@@ -242,94 +232,84 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     umma_ss(tmem + tm_yoff(k), umma_desc_sw128(cs + koff_c, 16, 1024),
                             umma_desc_sw128(sb + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
                 }
-                umma_commit(bar(B_Y + k));
                 umma_commit(bar(B_EMPTY + s));
+                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
+                // Y_diag = M(tmem) . X
+                if (!(live = wait(B_M + k, (uint32_t)((u >> 1) & 1)))) break;
+                if (!(live = wait(B_FULLX + s, (uint32_t)((u >> 1) & 1)))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ts(tmem + tm_cb(k) + 64, tmem + tm_cb(k) + ks * 8,
+                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
+                umma_commit(bar(B_Y + k));
+                umma_commit(bar(B_EMPTYX + s));
             }
             // Drain: the last commit must land before the CTA may exit.
             if (nblk > 0 && !*abort_flag) {
                 const int u = nblk - 1;
-                wait(B_EMPTY + (u & 1), (uint32_t)((u >> 1) & 1));
+                wait(B_EMPTYX + (u & 1), (uint32_t)((u >> 1) & 1));
             }
         }
     } else if (warp < 4) {
         // ------------------------------------- mask warpgroup (warps 0-3) ----
-        // Per block: in-block log2-decay scan, w o X, and the masked matrix M.
+        // Per block: w o X and the masked matrix M.
         const int t = tid;                         // TMEM lane = row i of the block
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const float a_h = p.A[h] * kLog2e;
-        float* red = reinterpret_cast<float*>(smem + OFF_RED);
-        auto nrow_of = [&](int u) -> int {
-            const int64_t t0 = (int64_t)u * UB;
-            return (L - t0) < UB ? (int)(L - t0) : UB;
-        };
-        auto load_dt = [&](int u) -> float {
-            return t < nrow_of(u) ? p.delta[((b * L + (int64_t)u * UB + t) * p.nheads) + h] : 0.0f;
-        };
+        // Waits are made uniform over the warpgroup (all leave the loop together),
+        // since the named barriers below need every one of its threads.
+        auto gwait = [&](int i, uint32_t par) { return named_bar_and(1, NCOMP, wait(i, par)); };
         bool ok = true;
-        float dt_next = nblk > 0 ? load_dt(0) : 0.0f;
+        bool lok = true;    // this thread's own waits since the last uniform check
         for (int u = 0; u < nblk && ok; ++u) {
             cur_blk = u;
             const int k = u & 1;
-            const float dt = dt_next;
-            if (u + 1 < nblk) dt_next = load_dt(u + 1);
-            float* cs_sm = reinterpret_cast<float*>(smem + OFF_CS) + k * UB;
-            float* da_sm = reinterpret_cast<float*>(smem + OFF_DA) + k * UB;
-            float* cf_sm = reinterpret_cast<float*>(smem + OFF_CF) + k * UB;
-            float* et_sm = reinterpret_cast<float*>(smem + OFF_ET) + k * UB;
-            float* gam_sm = reinterpret_cast<float*>(smem + OFF_GAM);
-            // the state warpgroup is done with block u-2's scalars and TMEM buffer k
-            if (u >= 2 && !(ok = wait(B_TFREE + k, (uint32_t)(((u - 2) >> 1) & 1)))) break;
-            // (a) cumulative log2-decay over the block
-            float cs = dt * a_h;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, cs, off);
-                if (lane >= off) cs += o;
-            }
-            if (lane == 31) red[k * 4 + warp] = cs;
-            named_bar_sync(1, NCOMP);
-            float prefix = 0.0f, total = 0.0f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float v = red[k * 4 + w];
-                if (w < warp) prefix += v;
-                total += v;
-            }
-            cs += prefix;
-            const float da = p.alpha * dt;
-            cs_sm[t] = cs;
-            da_sm[t] = da;
-            const float cs_ref = __shfl_sync(0xffffffffu, cs, 31);   // last column of this 32-batch
-            cf_sm[t] = ex2_approx(cs_ref - cs) * da;
-            et_sm[t] = ex2_approx(cs);                               // exp(cs_t)
-            if (t == 0) gam_sm[k] = ex2_approx(total);                // exp(cs_last)
-            const float wt = ex2_approx(total - cs) * da;            // exp(cs_last - cs_t) alpha delta_t
-            (reinterpret_cast<float*>(smem + OFF_WT) + k * UB)[t] = wt;
-            mbar_arrive(bar(B_SCAL + k));
-            named_bar_sync(1, NCOMP);
+            const float* cs_sm = reinterpret_cast<const float*>(smem + OFF_CS) + k * UB;
+            const float* da_sm = reinterpret_cast<const float*>(smem + OFF_DA) + k * UB;
+            const float* cf_sm = reinterpret_cast<const float*>(smem + OFF_CF) + k * UB;
+            // (a) the state warpgroup has published block u's decay scalars
+            ok = named_bar_and(1, NCOMP, lok && wait(B_SCAL + k, (uint32_t)((u >> 1) & 1)));
+            if (!ok) break;
+            const float cs = cs_sm[t];
 
-            // (b) first half of Xhat = diag(w) X (the state warpgroup does the other
-            //     half); X_hat is single-buffered: block u-1's state MMA must be done
-            if (u >= 1 && !(ok = wait(B_STATE, (uint32_t)((u - 1) & 1)))) break;
-            if (!(ok = wait(B_FULL + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
-            ssd_scale_row_half(smem + (u & 1) * SLOT + t * 128, smem + OFF_XHAT + t * 128, t, 0, wt);
+            // (b) Xhat = diag(w) X.  X_hat is single-buffered: block u-1's state MMA
+            //     must be done.  Warp q scales its own range of rows: the warps
+            //     with fewer mask batches in (c) take more rows, so that the two
+            //     steps together take about as long in every warp.
+            if (u >= 1 && !(ok = gwait(B_STATE, (uint32_t)((u - 1) & 1)))) break;
+            if (!(ok = gwait(B_FULLX + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
+            {
+                const float* wt_sm = reinterpret_cast<const float*>(smem + OFF_WT) + k * UB;
+                const unsigned char* xs = smem + (u & 1) * SLOT;
+                unsigned char* xh = smem + OFF_XHAT;
+                const int r0 = warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116;
+                const int r1 = warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128;
+                const int units = (r1 - r0) * 8;
+                for (int i = lane; i < units; i += 32) {
+                    const int r = r0 + (i >> 3);
+                    const int pc = ((i & 7) ^ (r & 7)) << 4;        // swizzled 16-byte chunk
+                    const float w = wt_sm[r];
+                    const uint4 q = *reinterpret_cast<const uint4*>(xs + r * 128 + pc);
+                    uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(bf16_lo(w4[e]) * w, bf16_hi(w4[e]) * w);
+                    *reinterpret_cast<uint4*>(xh + r * 128 + pc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
             fence_proxy_async_smem();
             mbar_arrive(bar(B_XHAT));
 
             // (c) M = CB o exp(cs_i - cs_j) alpha delta_j (j <= i), bf16 pairs into TMEM.
             //     Batches below the diagonal use exp(cs_i - cs_r) exp(cs_r - cs_j), both <= 1.
-            if (!(ok = wait(B_CB + k, (uint32_t)((u >> 1) & 1)))) break;
+            // Not a uniform wait: each warp goes on from its share of X_hat to its
+            // mask batches without waiting for the others.  A failed wait skips
+            // the work; the loop-top check above then ends the loop for all.
+            lok = wait(B_CB + k, (uint32_t)((u >> 1) & 1));
             tc_fence_after();
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t pk[16];
-                if (cb > warp) {                   // entirely above the diagonal
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                } else {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
-                    tmem_wait_ld();
+            if (lok) {
+                // One batch of 32 columns from its TMEM words r: decayed, masked, packed, stored.
+                auto mask_batch = [&](int cb, const uint32_t (&r)[32]) {
+                    uint32_t pk[16];
                     // Row factor 2^(cs_i - cs_r) and column factor 2^(cs_r - cs_j) alpha delta_j,
                     // r = last column of the batch.  Below the diagonal both are <= 1; in the
                     // diagonal batch the row factor is >= 1 but bounded by 2^(batch range),
@@ -340,16 +320,21 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         const float rowf = ex2_approx(cs - cs_r);
                         const float2 rr = f2(rowf, rowf);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 cf = *reinterpret_cast<const float2*>(cf_sm + cb * 32 + 2 * e);
-                            float2 m = __fmul2_rn(__fmul2_rn(f2(__uint_as_float(r[2 * e]),
-                                                                 __uint_as_float(r[2 * e + 1])), cf), rr);
-                            if (cb == warp) {      // causal mask inside the diagonal batch
-                                const int j = cb * 32 + 2 * e;
-                                m.x = j <= t ? m.x : 0.0f;
-                                m.y = j + 1 <= t ? m.y : 0.0f;
+                        for (int e = 0; e < 16; e += 2) {
+                            const float4 cf4 = *reinterpret_cast<const float4*>(cf_sm + cb * 32 + 2 * e);
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const int ee = e + h2;
+                                const float2 cf = h2 ? f2(cf4.z, cf4.w) : f2(cf4.x, cf4.y);
+                                float2 m = __fmul2_rn(__fmul2_rn(f2(__uint_as_float(r[2 * ee]),
+                                                                     __uint_as_float(r[2 * ee + 1])), cf), rr);
+                                if (cb == warp) {      // causal mask inside the diagonal batch
+                                    const int j = cb * 32 + 2 * ee;
+                                    m.x = j <= t ? m.x : 0.0f;
+                                    m.y = j + 1 <= t ? m.y : 0.0f;
+                                }
+                                pk[ee] = pack_bf16x2(m.x, m.y);
                             }
-                            pk[e] = pack_bf16x2(m.x, m.y);
                         }
                     } else {
                         float m[32];
@@ -361,8 +346,30 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(m[2 * e], m[2 * e + 1]);
                     }
+                    tmem_st16(tmem + lane_base + tm_cb(k) + cb * 16, pk);
+                };
+                // The packed batch cb lands on columns 16 cb .. 16 cb + 15 of the same
+                // buffer, i.e. on fp32 batch cb / 2, which is always read by then.
+                // Batches on or below the diagonal are read two at a time, so that one
+                // TMEM round trip covers both; the batches above it are zero and are
+                // written last (they overlap fp32 batches this warp still reads).
+#pragma unroll 1
+                for (int cb = 0; cb <= warp; cb += 2) {
+                    uint32_t r0[32], r1[32];
+                    const bool two = cb + 1 <= warp;
+                    tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r0);
+                    if (two) tmem_ld32(tmem + lane_base + tm_cb(k) + (cb + 1) * 32, r1);
+                    tmem_wait_ld();
+                    mask_batch(cb, r0);
+                    if (two) mask_batch(cb + 1, r1);
                 }
-                tmem_st16(tmem + lane_base + tm_cb(k) + cb * 16, pk);
+#pragma unroll 1
+                for (int cb = warp + 1; cb < 4; ++cb) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    tmem_st16(tmem + lane_base + tm_cb(k) + cb * 16, pk);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -373,13 +380,52 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         // Per block: S <- exp(cs_last) S + block state, the bf16 S operand for
         // the next block, and the output y = Y_diag + exp(cs_i) Y_off.
         const int t = tid - NCOMP;                 // TMEM lane = state n = row i
-        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        const int wq = warp - 4;
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         float S[P];                                 // row n = t of the state, fp32
+        auto gwait = [&](int i, uint32_t par) { return named_bar_and(2, NCOMP, wait(i, par)); };
         {
             const float* h0 = p.h0 ? p.h0 + (((b * p.nheads + h) * P) * NS) : nullptr;
 #pragma unroll
             for (int q = 0; q < P; ++q) S[q] = h0 ? h0[q * NS + t] : 0.0f;
         }
+        const float a_h = p.A[h] * kLog2e;
+        float* red = reinterpret_cast<float*>(smem + OFF_RED);
+        auto load_dt = [&](int v) -> float {
+            const int64_t tv = (int64_t)v * UB + t;
+            return tv < L ? p.delta[((b * L + tv) * p.nheads) + h] : 0.0f;
+        };
+        // In-block log2-decay scan of block v (row t): publishes cs, alpha delta,
+        // the column factors and w for the mask warpgroup (buffer v & 1) and
+        // returns exp(cs_t) and exp(cs_last) for this warpgroup's own use.
+        auto scan_block = [&](int v, float dt, float& et_out, float& gam_out) {
+            const int kv = v & 1;
+            float cs = dt * a_h;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, cs, off);
+                if (lane >= off) cs += o;
+            }
+            if (lane == 31) red[kv * 4 + wq] = cs;
+            named_bar_sync(2, NCOMP);
+            float prefix = 0.0f, total = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float v4 = red[kv * 4 + w];
+                if (w < wq) prefix += v4;
+                total += v4;
+            }
+            cs += prefix;
+            const float da = p.alpha * dt;
+            (reinterpret_cast<float*>(smem + OFF_CS) + kv * UB)[t] = cs;
+            (reinterpret_cast<float*>(smem + OFF_DA) + kv * UB)[t] = da;
+            const float cs_ref = __shfl_sync(0xffffffffu, cs, 31);   // last column of this 32-batch
+            (reinterpret_cast<float*>(smem + OFF_CF) + kv * UB)[t] = ex2_approx(cs_ref - cs) * da;
+            (reinterpret_cast<float*>(smem + OFF_WT) + kv * UB)[t] = ex2_approx(total - cs) * da;
+            mbar_arrive(bar(B_SCAL + kv));
+            et_out = ex2_approx(cs);                                 // exp(cs_t)
+            gam_out = ex2_approx(total);                             // exp(cs_last)
+        };
         // S as the bf16 B operand of C . S^T: MN-major, row n holds 64 p.
         auto write_S = [&](int buf) {
             unsigned char* row = smem + OFF_S + buf * S_TILE + t * 128;
@@ -393,75 +439,81 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             fence_proxy_async_smem();
             mbar_arrive(bar(B_SREADY + buf));
         };
-        // Second half of the rows of Xhat for block v (needs its w and its X tile).
-        auto xhat_half = [&](int v) -> bool {
-            if (!wait(B_SCAL + (v & 1), (uint32_t)((v >> 1) & 1))) return false;
-            if (!wait(B_FULL + (v & 1), (uint32_t)((v >> 1) & 1))) return false;
-            const float wt = (reinterpret_cast<const float*>(smem + OFF_WT) + (v & 1) * UB)[t];
-            ssd_scale_row_half(smem + (v & 1) * SLOT + t * 128, smem + OFF_XHAT + t * 128, t, 4, wt);
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_XHAT));
-            return true;
-        };
+        float et_u = 0.0f, gam_u = 0.0f;            // scalars of the current block
+        float dt_next = nblk > 1 ? load_dt(1) : 0.0f;
+        if (nblk > 0) scan_block(0, load_dt(0), et_u, gam_u);
         write_S(0);
-        bool ok = nblk == 0 || xhat_half(0);
+        bool ok = true;
         for (int u = 0; u < nblk && ok; ++u) {
             cur_blk = u;
             const int k = u & 1;
             const int64_t t0 = (int64_t)u * UB;
-            const int nrow = (L - t0) < UB ? (int)(L - t0) : UB;
-            if (!(ok = wait(B_SCAL + k, (uint32_t)((u >> 1) & 1)))) break;
-            const float gam = reinterpret_cast<const float*>(smem + OFF_GAM)[k];
-            const float et = (reinterpret_cast<const float*>(smem + OFF_ET) + k * UB)[t];
+            const float dt1 = dt_next;               // delta of block u+1, loaded one block ahead
+            if (u + 2 < nblk) dt_next = load_dt(u + 2);
+            // The next block's decay scan first: it needs no result of this block,
+            // and the mask warpgroup starts on the next block with it.
+            float et_n = 0.0f, gam_n = 0.0f;
+            if (u + 1 < nblk) scan_block(u + 1, dt1, et_n, gam_n);
 
             // (d) S <- exp(cs_last) S + block state; publish S for the next block
-            if (!(ok = wait(B_STATE, (uint32_t)(u & 1)))) break;
+            if (!(ok = gwait(B_STATE, (uint32_t)(u & 1)))) break;
             tc_fence_after();
+            const float gam = gam_u, et = et_u;
             {
-                uint32_t r[32];
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_base + TM_STATE, r0);
+                tmem_ld32(tmem + lane_base + TM_STATE + 32, r1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    tmem_ld32(tmem + lane_base + TM_STATE + hc * 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) S[hc * 32 + q] = fmaf(gam, S[hc * 32 + q], __uint_as_float(r[q]));
+                for (int q = 0; q < 32; ++q) {
+                    S[q] = fmaf(gam, S[q], __uint_as_float(r0[q]));
+                    S[32 + q] = fmaf(gam, S[32 + q], __uint_as_float(r1[q]));
                 }
             }
             tc_fence_before();
             mbar_arrive(bar(B_SFREE));
             write_S((u + 1) & 1);
-            // block u's state MMA is complete, so X_hat may take block u+1
-            if (u + 1 < nblk && !(ok = xhat_half(u + 1))) break;
 
-            // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of block u
-            if (!(ok = wait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
+            // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of block u.  Each half
+            //     (32 of the 64 columns) is staged in shared memory in the 64-byte
+            //     swizzled layout of the y tensor map and written by one TMA store,
+            //     which keeps the row-scattered global writes off the LSU pipe (the
+            //     mask warpgroup's loads share it).  Rows past L are clipped by the map.
+            if (!(ok = gwait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
             tc_fence_after();
             {
-                bf16* yrow = p.y + ((b * L + t0 + t) * p.nheads + h) * P;
+                unsigned char* yst = smem + OFF_YST + t * 64;
 #pragma unroll
                 for (int hc = 0; hc < 2; ++hc) {
                     uint32_t rd[32], ro[32];
                     tmem_ld32(tmem + lane_base + tm_cb(k) + 64 + hc * 32, rd);
                     tmem_ld32(tmem + lane_base + tm_yoff(k) + hc * 32, ro);
                     tmem_wait_ld();
-                    if (t < nrow) {
+                    uint32_t w[16];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            uint32_t w4[4];
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(fmaf(et, __uint_as_float(ro[2 * e]), __uint_as_float(rd[2 * e])),
+                                           fmaf(et, __uint_as_float(ro[2 * e + 1]), __uint_as_float(rd[2 * e + 1])));
+                    if (t == 0) bulk_wait_read_all();        // the previous store has read the stage
+                    named_bar_sync(2, NCOMP);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int q = c * 8 + 2 * e;
-                                w4[e] = pack_bf16x2(fmaf(et, __uint_as_float(ro[q]), __uint_as_float(rd[q])),
-                                                    fmaf(et, __uint_as_float(ro[q + 1]), __uint_as_float(rd[q + 1])));
-                            }
-                            *reinterpret_cast<uint4*>(yrow + hc * 32 + c * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                        }
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(yst + ((c ^ ((t >> 1) & 3)) << 4)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    named_bar_sync(2, NCOMP);
+                    if (t == 0) {
+                        tma_store_4d(&tm_y, base + OFF_YST, hc * 32, (int)h, (int)t0, (int)b);
+                        bulk_commit_group();
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(bar(B_TFREE + k));
+            et_u = et_n;
+            gam_u = gam_n;
         }
+        if (t == 0) bulk_wait_all();                 // y stores complete before the CTA exits
         if (ok && p.hT) {
             float* hT = p.hT + ((b * p.nheads + h) * P) * NS;
 #pragma unroll
@@ -498,16 +550,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 4-D bf16 map (d0 innermost), box (64, 1, 128, 1), 128-byte swizzle.
-cudaError_t make_map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+// 4-D bf16 map (d0 innermost), box (box0, 1, 128, 1): 64 columns with the
+// 128-byte swizzle for the loads, 32 columns with the 64-byte swizzle for the y stores.
+cudaError_t make_map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                        uint32_t box0 = 64) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[4] = {d0, d1, d2, d3};
     const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t box[4] = {box0, 1, 128, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          box0 == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -522,11 +577,12 @@ size_t ssd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t)
 
 cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t stream) {
     if (a.batch * a.nheads > 0x7fffffffLL || a.seqlen > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    CUtensorMap mx, mB, mC;
+    CUtensorMap mx, mB, mC, my;
     cudaError_t e;
     if ((e = make_map_4d(&mx, a.x, ssd::P, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = make_map_4d(&mB, a.B, ssd::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = make_map_4d(&mC, a.C, ssd::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
+    if ((e = make_map_4d(&my, a.y, ssd::P, a.nheads, a.seqlen, a.batch, 32)) != cudaSuccess) return e;
     SSDKArgs k{};
     k.delta = a.delta; k.A = a.A; k.h0 = a.h0;
     k.y = static_cast<bf16*>(a.y); k.hT = a.hT;
@@ -542,7 +598,7 @@ cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_done.fetch_or(bit, std::memory_order_release);
     }
-    ssd_fwd_kernel<<<(unsigned)(a.batch * a.nheads), ssd::NTHREADS, ssd::SMEM_BYTES, stream>>>(mx, mB, mC, k);
+    ssd_fwd_kernel<<<(unsigned)(a.batch * a.nheads), ssd::NTHREADS, ssd::SMEM_BYTES, stream>>>(mx, mB, mC, my, k);
     return cudaGetLastError();
 }
 
