@@ -26,11 +26,21 @@
 // page describes), is applied through the block state of step 2-4.  The
 // result is the same chunked recurrence up to rounding.
 //
-// Roles (6 warps): warp 4 issues TMA loads (no multicast) of X, B, C blocks
-// into a 2-deep ring; warp 5 issues all tcgen05.mma; warps 0-3 own TMEM
-// lanes 0-127 and do the element-wise work.  Every wait is an mbarrier wait
-// bounded by kWaitLimitNs; on give-up the kernel records the fact and every
-// role leaves its loop, TMEM is freed and the kernel returns.
+// Factored blocks.  With ref = cs_last / 2, exp(cs_i - cs_j) = e_i g_j where
+// e_i = 2^(cs_i - ref) and g_j = 2^(ref - cs_j) (log2 units).  When every
+// |cs_i - ref| is at most FACTOR_RANGE (the usual case), g_j alpha delta_j is
+// folded into X in place (X~), M is CB with the causal mask only, the block
+// state is 2^(cs_last - ref) B^T . X~, Y_off uses 2^ref S_prev, and Y_diag
+// accumulates onto Y_off, so that y = e_i (M . X~ + C . (2^ref S_prev)^T).
+// Blocks with a wider decay range use the per-element form above.
+//
+// Roles (10 warps): warps 0-3 (mask warpgroup) scale X and form M; warps 4-7
+// (state warpgroup) run the decay scan one block ahead, carry S and write y
+// through TMA stores; warp 8 issues TMA loads (no multicast) into a 2-deep
+// ring whose B/C and X parts are refilled separately; warp 9 issues all
+// tcgen05.mma.  Every wait is an mbarrier wait bounded by kWaitLimitNs; on
+// give-up the kernel records the fact and every role leaves its loop, TMEM
+// is freed and the kernel returns.
 #include <cuda.h>
 
 #include <atomic>
@@ -64,9 +74,10 @@ constexpr int OFF_YST = OFF_S + 2 * S_TILE;
 constexpr int OFF_CS = OFF_YST + Y_STAGE;   // cs[2][128] fp32 (log2 units)
 constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha*delta[2][128]
 constexpr int OFF_CF = OFF_DA + 2 * UB * 4; // column factors [2][128]
-constexpr int OFF_WT = OFF_CF + 2 * UB * 4;  // exp(cs_last - cs_t) alpha delta_t [2][128]
+constexpr int OFF_WT = OFF_CF + 2 * UB * 4;  // row factor of X for the block state [2][128]
 constexpr int OFF_RED = OFF_WT + 2 * UB * 4;
-constexpr int OFF_BAR = OFF_RED + 64;
+constexpr int OFF_MODE = OFF_RED + 64;      // per buffer: 1 = factored block (see the kernel comment)
+constexpr int OFF_BAR = OFF_MODE + 16;
 constexpr int NBAR = 24;
 constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TSLOT + 8;
@@ -89,6 +100,10 @@ constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
 constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . Xhat (both MN-major)
 constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // M(tmem) . X (X MN-major)
 constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 1);   // C . S^T (S MN-major)
+// A block is factored when every |cs_i - cs_last / 2| stays within this many
+// powers of two: the factors 2^(cs_i - ref) and 2^(ref - cs_j) then stay far
+// from the fp32 / bf16 range limits.
+constexpr float FACTOR_RANGE = 60.0f;
 }  // namespace ssd
 
 struct SSDKArgs {
@@ -213,14 +228,17 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 const int s = u & 1, k = u & 1;
                 const uint32_t slot = base + s * SLOT;
                 const uint32_t xs = slot, bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
-                // block state = B^T . Xhat: M = 128 states, N = 64, K = 128 rows
+                // block state = B^T . Xhat: M = 128 states, N = 64, K = 128 rows.  A factored
+                // block has its scaled X in place in the slot, otherwise in the X_hat buffer.
                 if (!(live = wait(B_XHAT, (uint32_t)(u & 1)))) break;
                 if (!(live = wait(B_SFREE, (uint32_t)((u + 1) & 1)))) break;
+                const bool fac = reinterpret_cast<volatile const int*>(smem + OFF_MODE)[k] != 0;
+                const uint32_t xop = fac ? xs : xhat;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     umma_ss(tmem + TM_STATE, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
-                            umma_desc_sw128(xhat + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
+                            umma_desc_sw128(xop + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
                 umma_commit(bar(B_STATE));
                 // Y_off = C . S_prev^T
                 if (!(live = wait(B_SREADY + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
@@ -238,10 +256,12 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 if (!(live = wait(B_M + k, (uint32_t)((u >> 1) & 1)))) break;
                 if (!(live = wait(B_FULLX + s, (uint32_t)((u >> 1) & 1)))) break;
                 tc_fence_after();
+                // factored: accumulate onto Y_off (y = e_i (Y_diag + Y_off)); else its own columns
+                const uint32_t yd = fac ? tmem + tm_yoff(k) : tmem + tm_cb(k) + 64;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_ts(tmem + tm_cb(k) + 64, tmem + tm_cb(k) + ks * 8,
-                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
+                    umma_ts(yd, tmem + tm_cb(k) + ks * 8, umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD,
+                            fac || ks > 0);
                 umma_commit(bar(B_Y + k));
                 umma_commit(bar(B_EMPTYX + s));
             }
@@ -271,19 +291,24 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             ok = named_bar_and(1, NCOMP, lok && wait(B_SCAL + k, (uint32_t)((u >> 1) & 1)));
             if (!ok) break;
             const float cs = cs_sm[t];
+            const bool fac = reinterpret_cast<volatile const int*>(smem + OFF_MODE)[k] != 0;
 
-            // (b) Xhat = diag(w) X.  X_hat is single-buffered: block u-1's state MMA
-            //     must be done.  Warp q scales its own range of rows: the warps
-            //     with fewer mask batches in (c) take more rows, so that the two
-            //     steps together take about as long in every warp.
+            // (b) Xhat = diag(f) X with the row factor f of OFF_WT: in place in the slot
+            //     for a factored block, else into the X_hat buffer, which is
+            //     single-buffered (block u-1's state MMA must be done).  Warp q
+            //     scales its own range of rows: the warps with fewer mask batches
+            //     in (c) take more rows, so that both steps together take about
+            //     as long in every warp.
             if (u >= 1 && !(ok = gwait(B_STATE, (uint32_t)((u - 1) & 1)))) break;
             if (!(ok = gwait(B_FULLX + (u & 1), (uint32_t)((u >> 1) & 1)))) break;
             {
                 const float* wt_sm = reinterpret_cast<const float*>(smem + OFF_WT) + k * UB;
                 const unsigned char* xs = smem + (u & 1) * SLOT;
-                unsigned char* xh = smem + OFF_XHAT;
-                const int r0 = warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116;
-                const int r1 = warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128;
+                unsigned char* xh = fac ? smem + (u & 1) * SLOT : smem + OFF_XHAT;
+                const int r0 = fac ? (warp == 0 ? 0 : warp == 1 ? 38 : warp == 2 ? 72 : 102)
+                                   : (warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116);
+                const int r1 = fac ? (warp == 0 ? 38 : warp == 1 ? 72 : warp == 2 ? 102 : 128)
+                                   : (warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128);
                 const int units = (r1 - r0) * 8;
                 for (int i = lane; i < units; i += 32) {
                     const int r = r0 + (i >> 3);
@@ -300,7 +325,10 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             mbar_arrive(bar(B_XHAT));
 
             // (c) M = CB o exp(cs_i - cs_j) alpha delta_j (j <= i), bf16 pairs into TMEM.
-            //     Batches below the diagonal use exp(cs_i - cs_r) exp(cs_r - cs_j), both <= 1.
+            //     A factored block has both decay factors elsewhere (2^(ref - cs_j)
+            //     alpha delta_j in X, 2^(cs_i - ref) in the epilogue): M is CB with the
+            //     causal mask.  Otherwise batches below the diagonal use
+            //     exp(cs_i - cs_r) exp(cs_r - cs_j), both <= 1.
             // Not a uniform wait: each warp goes on from its share of X_hat to its
             // mask batches without waiting for the others.  A failed wait skips
             // the work; the loop-top check above then ends the loop for all.
@@ -310,6 +338,22 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 // One batch of 32 columns from its TMEM words r: decayed, masked, packed, stored.
                 auto mask_batch = [&](int cb, const uint32_t (&r)[32]) {
                     uint32_t pk[16];
+                    if (fac) {
+                        if (cb == warp) {          // causal mask inside the diagonal batch
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int j = cb * 32 + 2 * e;
+                                pk[e] = pack_bf16x2(j <= t ? __uint_as_float(r[2 * e]) : 0.0f,
+                                                    j + 1 <= t ? __uint_as_float(r[2 * e + 1]) : 0.0f);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                        }
+                        tmem_st16(tmem + lane_base + tm_cb(k) + cb * 16, pk);
+                        return;
+                    }
                     // Row factor 2^(cs_i - cs_r) and column factor 2^(cs_r - cs_j) alpha delta_j,
                     // r = last column of the batch.  Below the diagonal both are <= 1; in the
                     // diagonal batch the row factor is >= 1 but bounded by 2^(batch range),
@@ -395,10 +439,22 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const int64_t tv = (int64_t)v * UB + t;
             return tv < L ? p.delta[((b * L + tv) * p.nheads) + h] : 0.0f;
         };
-        // In-block log2-decay scan of block v (row t): publishes cs, alpha delta,
-        // the column factors and w for the mask warpgroup (buffer v & 1) and
-        // returns exp(cs_t) and exp(cs_last) for this warpgroup's own use.
-        auto scan_block = [&](int v, float dt, float& et_out, float& gam_out) {
+        // In-block log2-decay scan of block v (row t).  It decides whether the
+        // block is factored: with ref = cs_last / 2 and every |cs_i - ref| within
+        // FACTOR_RANGE, exp2(cs_i - cs_j) = 2^(cs_i - ref) 2^(ref - cs_j) splits
+        // into a row factor applied to y and a column factor folded into X.  It
+        // publishes, for the mask warpgroup (buffer v & 1), cs, alpha delta, the
+        // per-batch column factors of the unfactored mask, the X row factor
+        // (2^(ref - cs_j) alpha delta_j if factored, else 2^(cs_last - cs_j)
+        // alpha delta_j) and the mode; it returns this warpgroup's own scalars.
+        struct BlockScal {
+            float et;     // y row factor: 2^(cs_t - ref) if factored, else 2^cs_t
+            float gam;    // 2^cs_last: decay of the carried state over the block
+            float gam2;   // factor of the block state B^T Xhat: 2^(cs_last - ref), or 1
+            float sref;   // factor of S in the Y_off operand: 2^ref, or 1
+            bool fac;
+        };
+        auto scan_block = [&](int v, float dt) -> BlockScal {
             const int kv = v & 1;
             float cs = dt * a_h;
 #pragma unroll
@@ -416,33 +472,41 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 total += v4;
             }
             cs += prefix;
+            const float ref = 0.5f * total;
+            BlockScal bs;
+            bs.fac = named_bar_and(2, NCOMP, fabsf(cs - ref) <= FACTOR_RANGE);
             const float da = p.alpha * dt;
             (reinterpret_cast<float*>(smem + OFF_CS) + kv * UB)[t] = cs;
             (reinterpret_cast<float*>(smem + OFF_DA) + kv * UB)[t] = da;
-            const float cs_ref = __shfl_sync(0xffffffffu, cs, 31);   // last column of this 32-batch
-            (reinterpret_cast<float*>(smem + OFF_CF) + kv * UB)[t] = ex2_approx(cs_ref - cs) * da;
-            (reinterpret_cast<float*>(smem + OFF_WT) + kv * UB)[t] = ex2_approx(total - cs) * da;
+            const float cs_b = __shfl_sync(0xffffffffu, cs, 31);     // last column of this 32-batch
+            (reinterpret_cast<float*>(smem + OFF_CF) + kv * UB)[t] = ex2_approx(cs_b - cs) * da;
+            (reinterpret_cast<float*>(smem + OFF_WT) + kv * UB)[t] = ex2_approx((bs.fac ? ref : total) - cs) * da;
+            if (t == 0) reinterpret_cast<volatile int*>(smem + OFF_MODE)[kv] = bs.fac ? 1 : 0;
             mbar_arrive(bar(B_SCAL + kv));
-            et_out = ex2_approx(cs);                                 // exp(cs_t)
-            gam_out = ex2_approx(total);                             // exp(cs_last)
+            bs.et = ex2_approx(bs.fac ? cs - ref : cs);
+            bs.gam = ex2_approx(total);
+            bs.gam2 = bs.fac ? ex2_approx(total - ref) : 1.0f;
+            bs.sref = bs.fac ? ex2_approx(ref) : 1.0f;
+            return bs;
         };
         // S as the bf16 B operand of C . S^T: MN-major, row n holds 64 p.
-        auto write_S = [&](int buf) {
+        auto write_S = [&](int buf, float scale) {
             unsigned char* row = smem + OFF_S + buf * S_TILE + t * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint32_t w4[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(S[c * 8 + 2 * e], S[c * 8 + 2 * e + 1]);
+                for (int e = 0; e < 4; ++e)
+                    w4[e] = pack_bf16x2(S[c * 8 + 2 * e] * scale, S[c * 8 + 2 * e + 1] * scale);
                 *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(B_SREADY + buf));
         };
-        float et_u = 0.0f, gam_u = 0.0f;            // scalars of the current block
+        BlockScal cur{1.0f, 1.0f, 1.0f, 1.0f, false};   // scalars of the current block
         float dt_next = nblk > 1 ? load_dt(1) : 0.0f;
-        if (nblk > 0) scan_block(0, load_dt(0), et_u, gam_u);
-        write_S(0);
+        if (nblk > 0) cur = scan_block(0, load_dt(0));
+        write_S(0, cur.sref);
         bool ok = true;
         for (int u = 0; u < nblk && ok; ++u) {
             cur_blk = u;
@@ -452,13 +516,13 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             if (u + 2 < nblk) dt_next = load_dt(u + 2);
             // The next block's decay scan first: it needs no result of this block,
             // and the mask warpgroup starts on the next block with it.
-            float et_n = 0.0f, gam_n = 0.0f;
-            if (u + 1 < nblk) scan_block(u + 1, dt1, et_n, gam_n);
+            BlockScal nxt{1.0f, 1.0f, 1.0f, 1.0f, false};
+            if (u + 1 < nblk) nxt = scan_block(u + 1, dt1);
 
             // (d) S <- exp(cs_last) S + block state; publish S for the next block
             if (!(ok = gwait(B_STATE, (uint32_t)(u & 1)))) break;
             tc_fence_after();
-            const float gam = gam_u, et = et_u;
+            const float gam = cur.gam, gam2 = cur.gam2, et = cur.et;
             {
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tmem + lane_base + TM_STATE, r0);
@@ -466,13 +530,13 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 tmem_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    S[q] = fmaf(gam, S[q], __uint_as_float(r0[q]));
-                    S[32 + q] = fmaf(gam, S[32 + q], __uint_as_float(r1[q]));
+                    S[q] = fmaf(gam, S[q], gam2 * __uint_as_float(r0[q]));
+                    S[32 + q] = fmaf(gam, S[32 + q], gam2 * __uint_as_float(r1[q]));
                 }
             }
             tc_fence_before();
             mbar_arrive(bar(B_SFREE));
-            write_S((u + 1) & 1);
+            write_S((u + 1) & 1, nxt.sref);
 
             // (e) y = Y_diag + exp(cs_i) Y_off, bf16, row t of block u.  Each half
             //     (32 of the 64 columns) is staged in shared memory in the 64-byte
@@ -485,15 +549,24 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 unsigned char* yst = smem + OFF_YST + t * 64;
 #pragma unroll
                 for (int hc = 0; hc < 2; ++hc) {
-                    uint32_t rd[32], ro[32];
-                    tmem_ld32(tmem + lane_base + tm_cb(k) + 64 + hc * 32, rd);
-                    tmem_ld32(tmem + lane_base + tm_yoff(k) + hc * 32, ro);
-                    tmem_wait_ld();
                     uint32_t w[16];
+                    if (cur.fac) {                           // y = e_i (Y_diag + Y_off), one accumulator
+                        uint32_t ro[32];
+                        tmem_ld32(tmem + lane_base + tm_yoff(k) + hc * 32, ro);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(fmaf(et, __uint_as_float(ro[2 * e]), __uint_as_float(rd[2 * e])),
-                                           fmaf(et, __uint_as_float(ro[2 * e + 1]), __uint_as_float(rd[2 * e + 1])));
+                        for (int e = 0; e < 16; ++e)
+                            w[e] = pack_bf16x2(et * __uint_as_float(ro[2 * e]), et * __uint_as_float(ro[2 * e + 1]));
+                    } else {
+                        uint32_t rd[32], ro[32];
+                        tmem_ld32(tmem + lane_base + tm_cb(k) + 64 + hc * 32, rd);
+                        tmem_ld32(tmem + lane_base + tm_yoff(k) + hc * 32, ro);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            w[e] = pack_bf16x2(fmaf(et, __uint_as_float(ro[2 * e]), __uint_as_float(rd[2 * e])),
+                                               fmaf(et, __uint_as_float(ro[2 * e + 1]), __uint_as_float(rd[2 * e + 1])));
+                    }
                     if (t == 0) bulk_wait_read_all();        // the previous store has read the stage
                     named_bar_sync(2, NCOMP);
 #pragma unroll
@@ -510,8 +583,7 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             }
             tc_fence_before();
             mbar_arrive(bar(B_TFREE + k));
-            et_u = et_n;
-            gam_u = gam_n;
+            cur = nxt;
         }
         if (t == 0) bulk_wait_all();                 // y stores complete before the CTA exits
         if (ok && p.hT) {

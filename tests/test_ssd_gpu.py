@@ -134,3 +134,18 @@ def test_repeated_runs_odd_block_counts_finish_without_device_timeout():
                 _compare(inp, y, hT, what=f"repeat L={L}")
             else:
                 assert np.array_equal(first[0], y) and np.array_equal(first[1], hT)
+
+
+def test_strong_decay_blocks_and_mode_switches():
+    """Blocks whose decay range is too wide for the factored form take the
+    per-element path; heads and blocks of both kinds, and a sequence that
+    switches between them, all match the oracle."""
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=640, nheads=4)
+    inp["A"] = (inp["A"] * np.array([1.0, 25.0, 1.0, 25.0], dtype=np.float32)).astype(np.float32)
+    d = inp["delta"].copy()
+    d[:, 256:512, :] *= 20.0                  # blocks 2-3 of every head decay fast
+    inp["delta"] = d.astype(np.float32)
+    rng = np.random.default_rng(11)
+    h0 = rng.standard_normal((1, 4, 64, 128)).astype(np.float32)
+    y, hT = _run(_dev(inp), h0=torch.from_numpy(h0).cuda(), alpha=1.3)
+    _compare(inp, y, hT, h0=h0, alpha=1.3, what="strong decay")
