@@ -189,21 +189,24 @@ def dist_env():
 
 def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0):
     """Time the fp64 oracle (as it stands) on whole passes over the workload,
-    or on a channel slice of it when one pass would exceed the budget."""
+    or on a channel slice of it when one pass would exceed the budget.
+    `budget_s` is CPU time (wall time x the oracle's threads)."""
     import oracle
     inp = wl.scan_inputs(w)
     nch = w.batch * w.dim
+    cores = oracle.num_threads()
+    wall_budget = budget_s / max(cores, 1)
     # calibrate on a small slice
-    probe = np.arange(min(nch, 64), dtype=np.int64)
+    probe = np.arange(min(nch, 256), dtype=np.int64)
     t = time.perf_counter()
     oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=probe)
     per_chan = (time.perf_counter() - t) / len(probe)
-    if per_chan * nch <= budget_s:
-        chans, passes = None, max(1, int(budget_s // max(per_chan * nch, 1e-9)))
-        passes = min(passes, 3)
+    if per_chan * nch <= wall_budget:
+        chans = None
+        passes = max(1, min(50, int(wall_budget // max(per_chan * nch, 1e-9))))
         sample = f"{passes} full pass(es) over all {nch} channels"
     else:
-        k = max(1, int(budget_s / per_chan))
+        k = max(1, int(wall_budget / per_chan))
         chans, passes = np.linspace(0, nch - 1, k).astype(np.int64), 1
         sample = f"{k} of {nch} channels (evenly spaced), 1 pass"
     updates = (nch if chans is None else len(chans)) * w.seqlen * w.dstate * passes
@@ -211,8 +214,8 @@ def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float 
     for _ in range(passes):
         oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=chans)
     dt = time.perf_counter() - t
-    return {"value": updates / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": sample + f", beta={beta}, alpha={alpha}, fp64, {dt:.2f} s wall"}
+    return {"value": updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": sample + f", beta={beta}, alpha={alpha}, fp64, {dt:.2f} s wall on {cores} threads"}
 
 
 def run_reference(args, w, beta, alpha):
