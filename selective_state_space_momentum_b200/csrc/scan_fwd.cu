@@ -52,8 +52,10 @@ struct ScanTile {
     static constexpr int CH = WARPS * CPW;       // channels per CTA
     static constexpr int NT = WARPS * 32;        // threads per CTA
     // The time split doubles the warps; 12 resident warps per SM (<= 168 registers)
-    // hold the medium-size grids in one wave.
-    static constexpr int MIN_CTAS = TS == 2 ? (12 / WARPS > 0 ? 12 / WARPS : 1) : 1;
+    // hold the medium-size grids in one wave.  bf16 tiles need less shared memory,
+    // so four 4-warp CTAs fit per SM when registers allow (<= 128 per thread).
+    static constexpr int MIN_CTAS = TS == 2 ? (12 / WARPS > 0 ? 12 / WARPS : 1)
+                                            : (SPT == 2 && WARPS == 4 && sizeof(IO) == 2 ? 4 : 1);
     static constexpr int NPAIR = SPT / 2;
     static constexpr int EB = IOTraits<IO>::kBytes;
     static constexpr int BOX_T = 128 / EB;       // steps in one 128-byte swizzled row
