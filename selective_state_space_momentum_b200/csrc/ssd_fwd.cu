@@ -305,10 +305,8 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 const float* wt_sm = reinterpret_cast<const float*>(smem + OFF_WT) + k * UB;
                 const unsigned char* xs = smem + (u & 1) * SLOT;
                 unsigned char* xh = fac ? smem + (u & 1) * SLOT : smem + OFF_XHAT;
-                const int r0 = fac ? (warp == 0 ? 0 : warp == 1 ? 38 : warp == 2 ? 72 : 102)
-                                   : (warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116);
-                const int r1 = fac ? (warp == 0 ? 38 : warp == 1 ? 72 : warp == 2 ? 102 : 128)
-                                   : (warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128);
+                const int r0 = fac ? warp * 32 : (warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116);
+                const int r1 = fac ? warp * 32 + 32 : (warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128);
                 const int units = (r1 - r0) * 8;
                 for (int i = lane; i < units; i += 32) {
                     const int r = r0 + (i >> 3);
