@@ -201,8 +201,8 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     } else if (warp == W_MMA) {
         // ----------------------------------------------------------- MMA ----
         // Issue order per block u: block state(u), Y_off(u) (needs only the
-        // previous state, and frees the block's B and C), C.B^T(u+1) (one block
-        // ahead, so the mask warpgroup can start on it), then Y_diag(u).
+        // previous state, and frees the block's B and C), Y_diag(u), then
+        // C.B^T(u+1) (one block ahead, so the mask warpgroup can start on it).
         if (lane == 0) {
             const uint32_t xhat = base + OFF_XHAT;
             auto issue_cb = [&](int v) -> bool {
@@ -251,7 +251,6 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             umma_desc_sw128(sb + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
                 }
                 umma_commit(bar(B_EMPTY + s));
-                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
                 // Y_diag = M(tmem) . X
                 if (!(live = wait(B_M + k, (uint32_t)((u >> 1) & 1)))) break;
                 if (!(live = wait(B_FULLX + s, (uint32_t)((u >> 1) & 1)))) break;
@@ -264,6 +263,9 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                             fac || ks > 0);
                 umma_commit(bar(B_Y + k));
                 umma_commit(bar(B_EMPTYX + s));
+                // C.B^T of the next block last: it waits for that block's B and C and
+                // for TMEM buffer k^1, which must not hold up this block's output.
+                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
             }
             // Drain: the last commit must land before the CTA may exit.
             if (nblk > 0 && !*abort_flag) {
