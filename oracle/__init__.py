@@ -60,6 +60,10 @@ def _declare(lib):
     lib.oracle_scan_seq.argtypes = [
         _f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p, _f64, _f64,
         _i64, _i64, _i64, _i64, _i64p, _i64, _f64p, _f64p, _f64p]
+    lib.oracle_scan_gated.restype = ctypes.c_int
+    lib.oracle_scan_gated.argtypes = [
+        _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, ctypes.c_int, _f64p, _f64p,
+        _f64, _f64, _i64, _i64, _i64, _i64, _i64p, _i64, _f64p, _f64p, _f64p]
     lib.oracle_scan_chunked.restype = ctypes.c_int
     lib.oracle_scan_chunked.argtypes = [
         _f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p, _f64, _f64,
@@ -90,6 +94,15 @@ def load(path: str | None = None):
 
 def _f32(a, name):
     a = np.ascontiguousarray(a, dtype=np.float32)
+    return a, a.ctypes.data_as(_f32p)
+
+
+def _f32opt(a, shape, name):
+    if a is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    if a.shape != tuple(shape):
+        raise ValueError(f"{name}: shape {a.shape}, expected {tuple(shape)}")
     return a, a.ctypes.data_as(_f32p)
 
 
@@ -144,6 +157,44 @@ def scan_seq(x, delta, A, B, C, h0=None, v0=None, beta=0.0, alpha=1.0,
                              y.ctypes.data_as(_f64p), hT.ctypes.data_as(_f64p),
                              vT.ctypes.data_as(_f64p))
     _check(rc, "oracle_scan_seq")
+    return y, hT, vT
+
+
+def scan_gated(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+               h0=None, v0=None, beta=0.0, alpha=1.0, chan=None, lib=None):
+    """The full selective_scan_fn forward (mm_oracle.c: oracle_scan_gated).
+
+    Momentum Mamba README, "selective_scan_fn" (arguments D, z, delta_bias,
+    delta_softplus); the gate as placed by "Mamba: Choosing What to Remember
+    Based on the Input", "Where the state computation sits in a Mamba block".
+    delta' = softplus(delta + delta_bias) (each part optional), the momentum
+    recurrence with delta', then out = (y + D x) * silu(z).  D, delta_bias:
+    (dim,) or None; z: (batch, dim, L) or None.  Returns fp64 (out, hT, vT)
+    shaped as :func:`scan_seq`.
+    """
+    lib = lib or load()
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    xs, xp = _f32(x, "x")
+    ds, dp = _f32(delta, "delta")
+    As, Ap = _f32(A, "A")
+    Bs, Bp = _f32(B, "B")
+    Cs, Cp = _f32(C, "C")
+    Ds, Dp = _f32opt(D, (dim,), "D")
+    zs, zp = _f32opt(z, (batch, dim, L), "z")
+    bs, bp = _f32opt(delta_bias, (dim,), "delta_bias")
+    h0s, h0p = _f64opt(h0, (batch, dim, N), "h0")
+    v0s, v0p = _f64opt(v0, (batch, dim, N), "v0")
+    cs, cp, nc = _idx(chan)
+    n = nc if chan is not None else batch * dim
+    y = np.empty((n, L), np.float64)
+    hT = np.empty((n, N), np.float64)
+    vT = np.empty((n, N), np.float64)
+    rc = lib.oracle_scan_gated(xp, dp, Ap, Bp, Cp, Dp, zp, bp, 1 if delta_softplus else 0,
+                               h0p, v0p, float(beta), float(alpha), batch, L, dim, N, cp, nc,
+                               y.ctypes.data_as(_f64p), hT.ctypes.data_as(_f64p),
+                               vT.ctypes.data_as(_f64p))
+    _check(rc, "oracle_scan_gated")
     return y, hT, vT
 
 

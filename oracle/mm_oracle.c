@@ -105,6 +105,87 @@ int oracle_scan_seq(const float *x, const float *delta, const float *A,
 }
 
 /* ------------------------------------------------------------------------ */
+/* The full selective_scan_fn forward: delta bias and softplus, D skip, z gate */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [MM] "selective_scan_fn" lists, besides u (= x), delta, A, B, C and the
+ * momentum pair, a skip weight D (dim), a gate z (batch, dim, L), a delta
+ * bias (dim) and a softplus switch; [SEL] "Where the state computation sits
+ * in a Mamba block" places the gate after the scan: SiLU of the gate branch
+ * multiplies the scan's output elementwise.  Readings (the pages give the
+ * arguments but no formulas):
+ *
+ *     delta'_t = delta_t + delta_bias[d]                   (bias NULL: + 0)
+ *     delta'_t = ln(1 + e^{delta'_t})                      (if softplus)
+ *     y_t      = sum_n C_t[n] h_t[n]   (recurrence above, with delta')
+ *     out_t    = y_t + D[d] * x_t                          (D NULL: + 0)
+ *     out_t    = out_t * z_t / (1 + e^{-z_t})              (z NULL: no gate)
+ *
+ * The states hT, vT are those of the recurrence.  Same layouts, channel
+ * selection and outputs as oracle_scan_seq (y holds out).
+ */
+static double softplus_f64(double u)
+{
+    /* ln(1 + e^u) without overflow: max(u, 0) + ln(1 + e^{-|u|}) */
+    return (u > 0.0 ? u : 0.0) + log1p(exp(-fabs(u)));
+}
+
+int oracle_scan_gated(const float *x, const float *delta, const float *A,
+                      const float *Bm, const float *Cm,
+                      const float *Dv, const float *z, const float *dbias, int softplus,
+                      const double *h0, const double *v0,
+                      double beta, double alpha,
+                      int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                      const int64_t *chan, int64_t nchan,
+                      double *y, double *hT, double *vT)
+{
+    if (!x || !delta || !A || !Bm || !Cm || !y) return ORACLE_ERR_ARG;
+    if (batch < 1 || seqlen < 1 || dim < 1 || dstate < 1) return ORACLE_ERR_ARG;
+    if (!chan) nchan = batch * dim;
+    if (nchan < 0) return ORACLE_ERR_ARG;
+
+    int64_t r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nchan; ++r) {
+        const int64_t c = chan ? chan[r] : r;
+        const int64_t b = c / dim;
+        const int64_t d = c % dim;
+        const float *xr = x + c * seqlen;
+        const float *dr = delta + c * seqlen;
+        double *yr = y + r * seqlen;
+        for (int64_t t = 0; t < seqlen; ++t) yr[t] = 0.0;
+
+        for (int64_t n = 0; n < dstate; ++n) {
+            double h = h0 ? h0[c * dstate + n] : 0.0;
+            double v = v0 ? v0[c * dstate + n] : 0.0;
+            const double a_dn = (double)A[d * dstate + n];
+            const float *Bn = Bm + (b * dstate + n) * seqlen;
+            const float *Cn = Cm + (b * dstate + n) * seqlen;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                double dt = (double)dr[t] + (dbias ? (double)dbias[d] : 0.0);
+                if (softplus) dt = softplus_f64(dt);
+                const double abar = exp(dt * a_dn);
+                v = beta * v + alpha * (dt * (double)Bn[t] * (double)xr[t]);
+                h = abar * h + v;
+                yr[t] += (double)Cn[t] * h;
+            }
+            if (hT) hT[r * dstate + n] = h;
+            if (vT) vT[r * dstate + n] = v;
+        }
+        for (int64_t t = 0; t < seqlen; ++t) {
+            double o = yr[t] + (Dv ? (double)Dv[d] * (double)xr[t] : 0.0);
+            if (z) {
+                const double zt = (double)z[c * seqlen + t];
+                o *= zt / (1.0 + exp(-zt));
+            }
+            yr[t] = o;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* The same scan in chunked form: per-chunk affine maps, then a carry fold.  */
 /* ------------------------------------------------------------------------ */
 

@@ -53,6 +53,56 @@ SSD_MUTANTS = {
 }
 
 
+GATED_MUTANTS = {
+    "softplus_dropped": ("                if (softplus) dt = softplus_f64(dt);\n", ""),
+    "softplus_log_not_log1p": ("return (u > 0.0 ? u : 0.0) + log1p(exp(-fabs(u)));",
+                               "return (u > 0.0 ? u : 0.0) + log(exp(-fabs(u)));"),
+    "bias_sign": ("double dt = (double)dr[t] + (dbias ? (double)dbias[d] : 0.0);",
+                  "double dt = (double)dr[t] - (dbias ? (double)dbias[d] : 0.0);"),
+    "skip_without_x": ("double o = yr[t] + (Dv ? (double)Dv[d] * (double)xr[t] : 0.0);",
+                       "double o = yr[t] + (Dv ? (double)Dv[d] : 0.0);"),
+    "gate_sigmoid_not_silu": ("o *= zt / (1.0 + exp(-zt));", "o *= 1.0 / (1.0 + exp(-zt));"),
+    "skip_after_gate": ("double o = yr[t] + (Dv ? (double)Dv[d] * (double)xr[t] : 0.0);\n            if (z) {\n"
+                        "                const double zt = (double)z[c * seqlen + t];\n"
+                        "                o *= zt / (1.0 + exp(-zt));\n            }",
+                        "double o = yr[t];\n            if (z) {\n"
+                        "                const double zt = (double)z[c * seqlen + t];\n"
+                        "                o *= zt / (1.0 + exp(-zt));\n            }\n"
+                        "            o += (Dv ? (double)Dv[d] * (double)xr[t] : 0.0);"),
+}
+
+
+def _gated_pins(lib):
+    """Pins of tests/test_oracle_gated_pins.py run against `lib`."""
+    from tests import test_oracle_gated_pins as gp
+    failed = []
+    g = json.load(open(GOLDEN))["selective_fig2"]
+    A = math.log(0.5)
+    for case in g["cases"]:
+        bias = math.log(math.expm1(case["delta"]))
+        y, h, _ = gp._one_step_gated([g["h_prev"]], [A], 0.0, [g["B"]], g["u"], [g["C"]],
+                                     delta_bias=bias, softplus=True, lib=lib)
+        if abs(h[0] - case["new_state_derived"]) > 1e-6 * case["new_state_derived"]:
+            failed.append("fig2_softplus")
+            break
+    for case in g["cases"]:
+        y, h, _ = gp._one_step_gated([g["h_prev"]], [A], 0.25 * case["delta"], [g["B"]], g["u"], [g["C"]],
+                                     delta_bias=0.75 * case["delta"], softplus=False, lib=lib)
+        if abs(h[0] - case["new_state_derived"]) > 1e-6 * case["new_state_derived"]:
+            failed.append("fig2_bias")
+            break
+    y, _, _ = gp._one_step_gated([0.0], [-1.0], 0.1, [1.0], 3.0, [0.0], D=2.0, z=1.0, lib=lib)
+    if abs(y - 6.0 * gp.SIGMA1) > 1e-12:
+        failed.append("skip_then_gate")
+    y, _, _ = gp._one_step_gated([0.0], [-1.0], 0.1, [1.0], 3.0, [0.0], D=2.0, z=2.0, lib=lib)
+    if abs(y - 6.0 * gp.SILU2) > 1e-12:
+        failed.append("silu2")
+    y, _, _ = gp._one_step_gated([0.0], [-1.0], 0.1, [1.0], 3.0, [0.0], D=2.0, lib=lib)
+    if y != 6.0:
+        failed.append("skip_C0")
+    return failed
+
+
 def _ssd_pins(lib):
     """Chunked SSD against the sequential definition (tiny, several chunks)."""
     rng = np.random.default_rng(4)
@@ -106,11 +156,12 @@ def _pins(lib):
 def test_real_oracle_passes_the_mutant_pins():
     assert _pins(oracle.load()) == []
     assert _ssd_pins(oracle.load()) == []
+    assert _gated_pins(oracle.load()) == []
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SSD_MUTANTS))
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SSD_MUTANTS) + sorted(GATED_MUTANTS))
 def test_planted_mistake_is_caught(name, tmp_path):
-    old, new = MUTANTS.get(name) or SSD_MUTANTS[name]
+    old, new = MUTANTS.get(name) or SSD_MUTANTS.get(name) or GATED_MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation anchor for {name} not found"
     mut_src = tmp_path / "mm_oracle.c"
@@ -120,5 +171,5 @@ def test_planted_mistake_is_caught(name, tmp_path):
     subprocess.run(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-shared",
                     "-fPIC", "-std=c11", "-o", str(so), str(mut_src), "-lm"], check=True)
     lib = oracle.load(str(so))
-    pins = _pins if name in MUTANTS else _ssd_pins
+    pins = _pins if name in MUTANTS else _ssd_pins if name in SSD_MUTANTS else _gated_pins
     assert pins(lib), f"no pin caught the planted mistake '{name}'"
