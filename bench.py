@@ -55,6 +55,8 @@ WORKLOADS[wl.SSD_MH.name] = wl.SSD_MH
 ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
            "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name, "ssd": wl.SSD_MH.name}
 DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
+IO_KEYS = ("x", "delta", "B", "C", "z")          # tensors in the workload's storage type
+GATED_EXTRAS = "D skip, z SiLU gate, delta_bias, softplus"
 
 
 def measured_traffic(kernel: str, workload: str):
@@ -84,12 +86,14 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MAX_MHZ}, "fallback"
 
 
-def algorithmic_bytes(w: wl.ScanWorkload) -> int:
-    """Bytes one call must move: x, delta, y once; B, C once; A; hT, vT."""
+def algorithmic_bytes(w: wl.ScanWorkload, gated: bool = False) -> int:
+    """Bytes one call must move: x, delta, y once; B, C once; A; hT, vT; with
+    the selective_scan_fn extras also z once and D, delta_bias."""
     eb = 4 if w.io == "f32" else 2
     bdl = w.batch * w.dim * w.seqlen
+    extra = (bdl * eb + 2 * w.dim * 4) if gated else 0
     return 3 * bdl * eb + 2 * w.batch * w.dstate * w.seqlen * eb + w.dim * w.dstate * 4 \
-        + 2 * w.batch * w.dim * w.dstate * 4
+        + 2 * w.batch * w.dim * w.dstate * 4 + extra
 
 
 # ------------------------------------------------------------ clocks -------
@@ -187,19 +191,27 @@ def dist_env():
     return rank, world, local
 
 
-def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0):
+def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0,
+                 gated: bool = False):
     """Time the fp64 oracle (as it stands) on whole passes over the workload,
     or on a channel slice of it when one pass would exceed the budget.
     `budget_s` is CPU time (wall time x the oracle's threads)."""
     import oracle
     inp = wl.scan_inputs(w)
+    if gated:
+        ex = wl.scan_extras(w)
+        run_oracle = lambda **kw: oracle.scan_gated(
+            inp["x"], ex["delta_raw"], inp["A"], inp["B"], inp["C"], D=ex["D"], z=ex["z"],
+            delta_bias=ex["delta_bias"], delta_softplus=True, beta=beta, alpha=alpha, **kw)
+    else:
+        run_oracle = lambda **kw: oracle.scan_seq(**inp, beta=beta, alpha=alpha, **kw)
     nch = w.batch * w.dim
     cores = oracle.num_threads()
     wall_budget = budget_s / max(cores, 1)
     # calibrate on a small slice
     probe = np.arange(min(nch, 256), dtype=np.int64)
     t = time.perf_counter()
-    oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=probe)
+    run_oracle(chan=probe)
     per_chan = (time.perf_counter() - t) / len(probe)
     if per_chan * nch <= wall_budget:
         chans = None
@@ -212,10 +224,11 @@ def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float 
     updates = (nch if chans is None else len(chans)) * w.seqlen * w.dstate * passes
     t = time.perf_counter()
     for _ in range(passes):
-        oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=chans)
+        run_oracle(chan=chans)
     dt = time.perf_counter() - t
     return {"value": updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": sample + f", beta={beta}, alpha={alpha}, fp64, {dt:.2f} s wall on {cores} threads"}
+            "sample": sample + f", beta={beta}, alpha={alpha}{', D, z, delta_bias, softplus' if gated else ''}, "
+                      f"fp64, {dt:.2f} s wall on {cores} threads"}
 
 
 def run_reference(args, w, beta=None, alpha=None):
@@ -245,12 +258,20 @@ def run_reference(args, w, beta=None, alpha=None):
         inp = wl.scan_inputs(w)
         n_units = w.batch * w.dim
         per_unit_updates = w.seqlen * w.dstate
+        ex = wl.scan_extras(w) if args.gated else None
 
         def run(sel):
-            oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=sel)
+            if ex is None:
+                oracle.scan_seq(**inp, beta=beta, alpha=alpha, chan=sel)
+            else:
+                oracle.scan_gated(inp["x"], ex["delta_raw"], inp["A"], inp["B"], inp["C"], D=ex["D"],
+                                  z=ex["z"], delta_bias=ex["delta_bias"], delta_softplus=True,
+                                  beta=beta, alpha=alpha, chan=sel)
         config = {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
                   "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
                   "global_batch": w.batch, "parallelism": "dp1"}
+        if args.gated:
+            config["extras"] = GATED_EXTRAS
         unit_name = "channels"
     probe = np.arange(min(n_units, 64), dtype=np.int64)
     t = time.perf_counter()
@@ -449,11 +470,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget", type=float, default=60.0,
                     help="wall seconds for the whole --impl reference run")
+    ap.add_argument("--gated", action="store_true",
+                    help="time mm_scan_fwd_gated with D, z, delta_bias and softplus (scan workloads)")
     ap.add_argument("--tile", default=None, help="force SPTxWARPS[xTIME_LANES], e.g. 4x2 or 4x2x2 (tuning)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[ALIASES.get(args.workload, args.workload)]
+    if args.gated and isinstance(w, wl.SSDWorkload):
+        ap.error("--gated applies to the scan workloads")
     if isinstance(w, wl.SSDWorkload):
         if args.impl == "reference":
             return run_reference(args, w)
@@ -497,13 +522,17 @@ def main(argv=None):
     # Each rank scans its own batch (seed offset by rank): weak scaling.
     inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))
     iodt = torch.float32 if w.io == "f32" else torch.bfloat16
+    if args.gated:
+        ex = wl.scan_extras(w, seed=rank_seed(w.seed_index, rank))
+        inp["delta"] = ex["delta_raw"]
+        inp.update(z=ex["z"], D=ex["D"], delta_bias=ex["delta_bias"])
     host = {k: torch.from_numpy(v) for k, v in inp.items()}
-    step_bytes = algorithmic_bytes(w)
+    step_bytes = algorithmic_bytes(w, args.gated)
     # enough input sets that a step's bytes were evicted by the steps before it
     nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
     sets = []
     for _ in range(nsets):
-        s = {k: host[k].to(dev).to(iodt if k in ("x", "delta", "B", "C") else torch.float32).contiguous()
+        s = {k: host[k].to(dev).to(iodt if k in IO_KEYS else torch.float32).contiguous()
              for k in host}
         s["y"] = torch.empty_like(s["x"])
         s["hT"] = torch.empty((w.batch, w.dim, w.dstate), device=dev)
@@ -513,8 +542,13 @@ def main(argv=None):
 
     def step(i):
         s = sets[i % nsets]
-        mm.mm_scan_fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha,
-                       s["y"], s["hT"], s["vT"], stream)
+        if args.gated:
+            mm.mm_scan_fwd_gated(s["x"], s["delta"], s["A"], s["B"], s["C"], s["D"], s["z"],
+                                 s["delta_bias"], 1, None, None, beta, alpha, s["y"], s["hT"], s["vT"],
+                                 stream)
+        else:
+            mm.mm_scan_fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha,
+                           s["y"], s["hT"], s["vT"], stream)
 
     def barrier():
         if world > 1:
@@ -541,8 +575,10 @@ def main(argv=None):
 
     # ---- end to end through the host-memory call -------------------------
     e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
-    pinned = {k: v.to(iodt if k in ("x", "delta", "B", "C") else torch.float32).pin_memory()
+    pinned = {k: v.to(iodt if k in IO_KEYS else torch.float32).pin_memory()
               for k, v in host.items()}
+    extras = dict(D=pinned["D"], z=pinned["z"], delta_bias=pinned["delta_bias"],
+                  delta_softplus=True) if args.gated else {}
     out = {"y": torch.empty(tuple(inp["x"].shape), dtype=iodt, pin_memory=True),
            "hT": torch.empty((w.batch, w.dim, w.dstate), pin_memory=True),
            "vT": torch.empty((w.batch, w.dim, w.dstate), pin_memory=True)}
@@ -550,14 +586,14 @@ def main(argv=None):
     d2h = sum(v.numel() * v.element_size() for v in out.values())
     for _ in range(2):
         mm.scan_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
-                         beta=beta, alpha=alpha, out=out)
+                         beta=beta, alpha=alpha, out=out, **extras)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         mm.scan_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
-                         beta=beta, alpha=alpha, out=out, stream=stream)
+                         beta=beta, alpha=alpha, out=out, stream=stream, **extras)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
@@ -573,7 +609,7 @@ def main(argv=None):
         hbm_achieved = step_bytes / (ms_step * 1e-3) / 1e9
         cb = None
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline(w, beta, alpha)
+            cb = cpu_baseline(w, beta, alpha, gated=args.gated)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -581,11 +617,12 @@ def main(argv=None):
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
                        "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
                        "global_batch": w.batch * world, "parallelism": f"dp{world}",
-                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
+                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2",
+                       **({"extras": GATED_EXTRAS} if args.gated else {})},
             "roofline": {"bound": "alu", "kernel": "scan_fwd_kernel",
                          "achieved": achieved / 1e9, "peak": mufu_peak / 1e9, "unit": "Gex2/s",
                          "frac": achieved / mufu_peak,
-                         "traffic": measured_traffic("scan_fwd_kernel", w.name),
+                         "traffic": None if args.gated else measured_traffic("scan_fwd_kernel", w.name),
                          "peak_source": f"16 ex2/clk/SM x 148 SMs x {sm_max:.0f} MHz",
                          "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
                                  "frac": hbm_achieved / hbm_peak, "peak_source": peak_kind,

@@ -115,6 +115,36 @@ mm_status mm_scan_fwd(const void *x, const void *delta, const float *A,
                       void *y, float *hT, float *vT,
                       const mm_scan_dims *dims, void *stream);
 
+/*
+ * mm_scan_fwd_gated -- the full selective_scan_fn forward: mm_scan_fwd plus
+ * the optional arguments the Momentum Mamba README lists for
+ * "selective_scan_fn" (D, z, delta_bias, delta_softplus), with the gate
+ * after the scan as in "Mamba: Choosing What to Remember Based on the
+ * Input", section "Where the state computation sits in a Mamba block":
+ *
+ *   delta'_t = delta_t + delta_bias[d]            (delta_bias NULL: + 0)
+ *   delta'_t = ln(1 + exp(delta'_t))              (delta_softplus != 0)
+ *   the recurrence of mm_scan_fwd with delta'
+ *   out_t    = y_t + D[d] * x_t                   (D NULL: + 0)
+ *   out_t    = out_t * z_t * sigmoid(z_t)         (z NULL: no gate)
+ *
+ * and y receives out.  D, delta_bias: (dim) fp32; z: (batch, dim, L) in the
+ * io dtype; each may be NULL (with delta_softplus = 0 and all three NULL
+ * this is mm_scan_fwd).  hT, vT are the recurrence's final states.  Same
+ * layouts, alignment (16 bytes for every given pointer), aliasing rules (y
+ * may overlap no input, z, D and delta_bias included), streaming property
+ * and errors as mm_scan_fwd.  delta' is computed once per (batch, channel,
+ * step) in fp32 from the loaded delta; the gate uses a fast exponential.
+ */
+mm_status mm_scan_fwd_gated(const void *x, const void *delta, const float *A,
+                            const void *B, const void *C,
+                            const float *D, const void *z,
+                            const float *delta_bias, int delta_softplus,
+                            const float *h0, const float *v0,
+                            float beta, float alpha,
+                            void *y, float *hT, float *vT,
+                            const mm_scan_dims *dims, void *stream);
+
 /* Sizes of one Mamba-2 SSD call. */
 typedef struct {
     int64_t batch;    /* b                                                  */

@@ -24,7 +24,7 @@ import threading
 
 __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
-    "mm_scan_fwd", "mm_ssd_fwd", "mm_ssd_workspace_size", "mm_status_string",
+    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_ssd_fwd", "mm_ssd_workspace_size", "mm_status_string",
     "mm_last_error", "mm_scan_set_tile", "mm_version", "mm_device_status",
     "scan_fwd", "ssd_fwd", "scan_fwd_host", "EXPORTED_SYMBOLS",
 ]
@@ -44,7 +44,8 @@ STATUS_NAMES = {
 }
 
 # Every function include/mm_scan.h declares.
-EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_ssd_workspace_size", "mm_ssd_fwd", "mm_device_status",
+EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_ssd_workspace_size", "mm_ssd_fwd",
+                    "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
 
 
@@ -77,6 +78,9 @@ def _declare(lib):
     lib.mm_scan_fwd.restype = ctypes.c_int
     lib.mm_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp,
                                 ctypes.POINTER(ScanDims), vp]
+    lib.mm_scan_fwd_gated.restype = ctypes.c_int
+    lib.mm_scan_fwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, f, f,
+                                      vp, vp, vp, ctypes.POINTER(ScanDims), vp]
     lib.mm_ssd_workspace_size.restype = ctypes.c_int
     lib.mm_ssd_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.POINTER(ctypes.c_size_t)]
     lib.mm_ssd_fwd.restype = ctypes.c_int
@@ -155,6 +159,21 @@ def mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
     _check(rc, "mm_scan_fwd")
 
 
+def mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
+                      y, hT, vT, stream=None):
+    """C entry point mm_scan_fwd_gated (marshalling only): mm_scan_fwd plus the
+    optional D (dim,) fp32, z (batch, dim, L) in the storage type of x,
+    delta_bias (dim,) fp32 and the softplus switch."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_fwd_gated(
+        _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if delta_softplus else 0, _ptr(h0), _ptr(v0), float(beta), float(alpha), _ptr(y), _ptr(hT),
+        _ptr(vT), ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_fwd_gated")
+
+
 def mm_ssd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk) -> int:
     dims = SSDDims(batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
     out = ctypes.c_size_t(0)
@@ -204,9 +223,11 @@ def mm_device_status():
 
 # ------------------------------------------------------------ wrappers -----
 def scan_fwd(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0,
-             return_last_state=True, stream=None):
-    """Allocate outputs and run mm_scan_fwd; returns (y, hT, vT) (states None
-    when ``return_last_state`` is False)."""
+             return_last_state=True, stream=None, D=None, z=None, delta_bias=None,
+             delta_softplus=False):
+    """Allocate outputs and run mm_scan_fwd, or mm_scan_fwd_gated when any of
+    D, z, delta_bias, delta_softplus is given; returns (y, hT, vT) (states
+    None when ``return_last_state`` is False)."""
     import torch
     y = torch.empty_like(x)
     hT = vT = None
@@ -214,7 +235,11 @@ def scan_fwd(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0,
         shape = (x.shape[0], x.shape[1], A.shape[1])
         hT = torch.empty(shape, device=x.device, dtype=torch.float32)
         vT = torch.empty(shape, device=x.device, dtype=torch.float32)
-    mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream)
+    if D is None and z is None and delta_bias is None and not delta_softplus:
+        mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream)
+    else:
+        mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
+                          y, hT, vT, stream)
     return y, hT, vT
 
 
@@ -235,10 +260,11 @@ def ssd_fwd(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, return_last_state=
 
 
 def scan_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, device="cuda",
-                  out=None, stream=None):
+                  out=None, stream=None, D=None, z=None, delta_bias=None, delta_softplus=False):
     """End-to-end scan of host (CPU, ideally pinned) tensors.
 
-    Copies the inputs to the device, runs mm_scan_fwd, and copies y, hT and
+    Copies the inputs to the device, runs mm_scan_fwd (mm_scan_fwd_gated when
+    any of D, z, delta_bias, delta_softplus is given), and copies y, hT and
     vT back into ``out`` (a dict of host tensors, allocated if None).
     Returns that dict after synchronising the stream.
     """
@@ -246,8 +272,9 @@ def scan_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, devi
     s = stream or torch.cuda.current_stream(device)
     with torch.cuda.stream(s):
         dev = [t.to(device, non_blocking=True) if t is not None else None
-               for t in (x, delta, A, B, C, h0, v0)]
-        y, hT, vT = scan_fwd(*dev[:5], h0=dev[5], v0=dev[6], beta=beta, alpha=alpha, stream=s)
+               for t in (x, delta, A, B, C, h0, v0, D, z, delta_bias)]
+        y, hT, vT = scan_fwd(*dev[:5], h0=dev[5], v0=dev[6], beta=beta, alpha=alpha, stream=s,
+                             D=dev[7], z=dev[8], delta_bias=dev[9], delta_softplus=delta_softplus)
         if out is None:
             out = {"y": torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
                    "hT": torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True),

@@ -126,6 +126,15 @@ mm_status mm_scan_set_tile(int spt, int warps, int time_lanes) {
 mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const void* B,
                       const void* C, const float* h0, const float* v0, float beta, float alpha,
                       void* y, float* hT, float* vT, const mm_scan_dims* dims, void* stream) {
+    return mm_scan_fwd_gated(x, delta, A, B, C, nullptr, nullptr, nullptr, 0, h0, v0, beta, alpha,
+                             y, hT, vT, dims, stream);
+}
+
+mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, const void* B,
+                            const void* C, const float* Dskip, const void* z, const float* delta_bias,
+                            int delta_softplus, const float* h0, const float* v0, float beta,
+                            float alpha, void* y, float* hT, float* vT, const mm_scan_dims* dims,
+                            void* stream) {
     if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
     if (!x || !delta || !A || !B || !C || !y)
         return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
@@ -147,18 +156,22 @@ mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const vo
         !mul_ok(D, N, &dn) || !mul_ok(dn, 4, &a_bytes) || !mul_ok(bd, N, &bdn) ||
         !mul_ok(bdn, 4, &st_bytes))
         return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
-    const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT};
-    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "y", "hT", "vT"};
-    for (int i = 0; i < 10; ++i)
+    const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT, Dskip, z, delta_bias};
+    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "y", "hT", "vT", "D", "z",
+                           "delta_bias"};
+    for (int i = 0; i < 13; ++i)
         if (ptrs[i] && !aligned16(ptrs[i]))
             return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    int64_t d_bytes;
+    if (!mul_ok(D, 4, &d_bytes)) return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
 
     const Range rx = rng("x", x, seq_bytes), rd = rng("delta", delta, seq_bytes),
                 rA = rng("A", A, a_bytes), rB = rng("B", B, bc_bytes), rC = rng("C", C, bc_bytes),
                 rh0 = rng("h0", h0, st_bytes), rv0 = rng("v0", v0, st_bytes),
                 ry = rng("y", y, seq_bytes), rhT = rng("hT", hT, st_bytes),
-                rvT = rng("vT", vT, st_bytes);
-    const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0, &rv0};
+                rvT = rng("vT", vT, st_bytes), rD = rng("D", Dskip, d_bytes),
+                rz = rng("z", z, seq_bytes), rbias = rng("delta_bias", delta_bias, d_bytes);
+    const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0, &rv0, &rD, &rz, &rbias};
     for (const Range* in : inputs)
         if (overlap(ry, *in)) return fail(MM_ERR_ALIAS, "y overlaps %s", in->name);
     for (const Range* out : {&rhT, &rvT}) {
@@ -179,6 +192,8 @@ mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const vo
     a.batch = bsz; a.seqlen = L; a.dim = D; a.dstate = (int)N;
     a.beta = beta; a.alpha = alpha;
     a.vec_ok = ((L * esize) % 16) == 0;
+    a.Dskip = Dskip; a.z = z; a.dbias = delta_bias; a.softplus = delta_softplus ? 1 : 0;
+    a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
     const mmscan::ScanTileChoice t =
         mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load(),
                                  g_forced_ts.load());

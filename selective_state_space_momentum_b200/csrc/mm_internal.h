@@ -25,6 +25,12 @@ struct ScanArgs {
     int tiles_per_batch;   // filled by the launcher
     float beta, alpha;
     int vec_ok;            // rows of L elements are whole 16-byte pieces
+    // selective_scan_fn extras (all absent on the plain path)
+    const float* Dskip;    // (dim) or null
+    const void* z;         // (batch, dim, L) io dtype, or null
+    const float* dbias;    // (dim) or null
+    int softplus;          // delta' = softplus(delta + dbias)
+    int ext;               // any of the four is present
 };
 
 struct ScanTileChoice {

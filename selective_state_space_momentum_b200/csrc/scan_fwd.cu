@@ -45,7 +45,7 @@ namespace mmscan {
 // Device error word of this file's kernels (bounded waits that gave up).
 static __device__ unsigned int g_scan_dev_err = 0;
 
-template <typename IO, int NP, int SPT, int WARPS, int TS>
+template <typename IO, int NP, int SPT, int WARPS, int TS, bool EXT = false>
 struct ScanTile {
     static constexpr int G = NP / SPT;           // lanes per (channel, time-lane)
     static constexpr int CPW = 32 / (G * TS);    // channels per warp
@@ -75,7 +75,13 @@ struct ScanTile {
     static constexpr int BT_BYTES = T * BP * 4;
     static constexpr int R = 8;                  // steps per inner group
     static constexpr int OFF_BT = STAGES * STAGE_BYTES;    // 2 buffers of B^T, then 2 of C^T
-    static constexpr int OFF_BAR = OFF_BT + 4 * BT_BYTES;
+    // selective_scan_fn extras: delta' = softplus(delta + bias) per (channel,
+    // step) as fp32 in the fp32 box layout (32 steps x CH rows of 128 bytes):
+    // in place in the delta tile for fp32 I/O, else in two buffers of its own.
+    static constexpr int XBOX_F32 = CH * 128;    // one 32-step fp32 box of CH rows
+    static constexpr int DP_BYTES = (EXT && EB == 2) ? (T / 32) * XBOX_F32 : 0;
+    static constexpr int OFF_DP = OFF_BT + 4 * BT_BYTES;
+    static constexpr int OFF_BAR = OFF_DP + 2 * DP_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
 
     static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "lanes per channel");
@@ -86,6 +92,7 @@ struct ScanTile {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
     static_assert(TS == 1 || (TS == 2 && EB == 4 && T == 2 * 2 * R && (G == 4 || G == 8)),
                   "time split: fp32 I/O, two groups per lane, 4 or 8 lanes per channel");
+    static_assert(!EXT || TS == 1, "the selective_scan_fn extras run without the time split");
 };
 
 // Store `cnt` consecutive steps of one output row.
@@ -155,12 +162,32 @@ __device__ __forceinline__ float2 shfl_down_f2(float2 v, int delta) {
     return f2(__shfl_down_sync(0xffffffffu, v.x, delta), __shfl_down_sync(0xffffffffu, v.y, delta));
 }
 
-template <typename IO, int NP, int SPT, int WARPS, int TS>
-__global__ void __launch_bounds__(WARPS * 32, ScanTile<IO, NP, SPT, WARPS, TS>::MIN_CTAS)
+// softplus(v) = ln(1 + e^v) = max(v, 0) + ln(1 + u) with u = e^-|v| in (0, 1].
+// ln(1 + u) = 2 atanh(s) for s = u / (2 + u) in (0, 1/3], summed as the odd
+// series s (1 + s^2/3 + s^4/5 + ... + s^14/15): every term is positive (no
+// cancellation) and the first one left out is below 2e-9 of the sum, so the
+// error is that of fp32 rounding and of the two MUFU operations.
+__device__ __forceinline__ float softplus_f32(float v) {
+    const float u = ex2_approx(-fabsf(v) * kLog2e);
+    const float s = __fdividef(u, 2.0f + u);
+    const float q = s * s;
+    float p = 1.0f / 15.0f;
+    p = fmaf(p, q, 1.0f / 13.0f);
+    p = fmaf(p, q, 1.0f / 11.0f);
+    p = fmaf(p, q, 1.0f / 9.0f);
+    p = fmaf(p, q, 1.0f / 7.0f);
+    p = fmaf(p, q, 1.0f / 5.0f);
+    p = fmaf(p, q, 1.0f / 3.0f);
+    p = fmaf(p, q, 1.0f);
+    return fmaxf(v, 0.0f) + 2.0f * s * p;
+}
+
+template <typename IO, int NP, int SPT, int WARPS, int TS, bool EXT>
+__global__ void __launch_bounds__(WARPS * 32, ScanTile<IO, NP, SPT, WARPS, TS, EXT>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                 const ScanArgs p) {
-    using TL = ScanTile<IO, NP, SPT, WARPS, TS>;
+    using TL = ScanTile<IO, NP, SPT, WARPS, TS, EXT>;
     constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
     constexpr int ST = TL::STAGES, NPAIR = TL::NPAIR, EB = TL::EB, BP = TL::BP;
 
@@ -221,6 +248,12 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
     const float2 beta2 = f2(p.beta, p.beta);
     const float alpha = p.alpha;
+    // selective_scan_fn extras
+    const float skip_d = (EXT && p.Dskip && active) ? p.Dskip[d] : 0.0f;
+    const bool has_skip = EXT && p.Dskip != nullptr;
+    const IO* zrow = (EXT && p.z) ? static_cast<const IO*>(p.z) + (b * p.dim + (active ? d : 0)) * p.seqlen
+                                  : nullptr;
+    constexpr int ZN = EXT ? TL::R / G : 1;      // gate values a lane applies per group
 
     // ---- staging of one chunk into a stage buffer --------------------------
     auto issue = [&](int64_t k, int s) {
@@ -328,6 +361,30 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
         }
+        if constexpr (EXT) {
+            // delta' = softplus(delta + bias) once per (channel, step) of the chunk,
+            // four steps per item, as fp32 in the fp32 box layout.
+            if (p.dbias || p.softplus) {
+                unsigned char* dp = (EB == 4) ? smem + s * TL::STAGE_BYTES + TL::OFF_D
+                                              : smem + TL::OFF_DP + (int)(k & 1) * TL::DP_BYTES;
+                for (int i = tid; i < CH * (T / 4); i += NT) {
+                    const int cc = i / (T / 4);
+                    const int t4 = (i - cc * (T / 4)) * 4;
+                    const int bxs = t4 / TL::BOX_T;
+                    const int cols = t4 - bxs * TL::BOX_T;
+                    const float4 q = load4(reinterpret_cast<const IO*>(sbuf + TL::OFF_D + bxs * TL::XBOX +
+                                                                       sw128(cc, cols * EB)));
+                    const float bv = (p.dbias && d0 + cc < p.dim) ? p.dbias[d0 + cc] : 0.0f;
+                    float v[4] = {q.x + bv, q.y + bv, q.z + bv, q.w + bv};
+                    if (p.softplus) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) v[e] = softplus_f32(v[e]);
+                    }
+                    *reinterpret_cast<float4*>(dp + (t4 / 32) * TL::XBOX_F32 + sw128(cc, (t4 % 32) * 4)) =
+                        make_float4(v[0], v[1], v[2], v[3]);
+                }
+            }
+        }
         __syncthreads();
         // Every thread is past compute(k-1): its stage and B^T/C^T buffers are free.
         if (k + ST - 1 < nchunks) issue(k + ST - 1, (int)((k + ST - 1) % ST));
@@ -337,7 +394,9 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const float* Cg = Ct + g * SPT;
 
         // Loads, delta*x and exponentials of the R steps of group gi.
-        auto prep = [&](int gi, float (&u)[R], float (&a)[R][SPT]) {
+        const bool dprime_bf16 = EXT && EB == 2 && (p.dbias || p.softplus);
+        const unsigned char* dpb = smem + TL::OFF_DP + (int)(k & 1) * TL::DP_BYTES;
+        auto prep = [&](int gi, float (&u)[R], float (&a)[R][SPT], float (&zg)[ZN]) {
             const int tau0 = gi * R;
             const int bx = tau0 / TL::BOX_T;
             const int col = tau0 - bx * TL::BOX_T;
@@ -346,10 +405,22 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             float dl[R], xl[R];
 #pragma unroll
             for (int j = 0; j < R; j += 4) {
-                const float4 dq = load4(reinterpret_cast<const IO*>(dtl + sw128(c, (col + j) * EB)));
+                float4 dq;
+                if (dprime_bf16)      // delta' kept as fp32 beside the bf16 tiles
+                    dq = *reinterpret_cast<const float4*>(dpb + ((tau0 + j) / 32) * TL::XBOX_F32 +
+                                                          sw128(c, ((tau0 + j) % 32) * 4));
+                else
+                    dq = load4(reinterpret_cast<const IO*>(dtl + sw128(c, (col + j) * EB)));
                 const float4 xq = load4(reinterpret_cast<const IO*>(xt + sw128(c, (col + j) * EB)));
                 dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
                 xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
+            }
+            if constexpr (EXT) {      // the gate of this lane's outputs, one group ahead
+#pragma unroll
+                for (int e = 0; e < ZN; ++e) {
+                    const int64_t tz = t0 + tau0 + g * ZN + e;
+                    zg[e] = (zrow && active && tz < L) ? load1(zrow + tz) : 0.0f;
+                }
             }
 #pragma unroll
             for (int j = 0; j < R; j += 2) {
@@ -369,12 +440,24 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         };
 
         // ---- add the G partials of each channel; store y --------------------
-        auto reduce_store = [&](int tau0, const float (&yk)[R]) {
+        auto reduce_store = [&](int tau0, const float (&yk)[R], const float (&zg)[ZN]) {
             constexpr int PER = R / G;      // steps each lane finishes
             float out[PER];
             butterfly_sum<G, R>(yk, out, g);
             const int first = tau0 + g * PER;      // step (within the chunk) of out[0]
             const int cnt = nval - first < PER ? nval - first : PER;
+            if constexpr (EXT) {
+#pragma unroll
+                for (int e = 0; e < PER; ++e) {
+                    if (has_skip) {               // + D x, x from the staged tile
+                        const int st = first + e;
+                        const int bxx = st / TL::BOX_T;
+                        out[e] += skip_d * load1(reinterpret_cast<const IO*>(
+                                      sbuf + TL::OFF_X + bxx * TL::XBOX + sw128(c, (st - bxx * TL::BOX_T) * EB)));
+                    }
+                    if (zrow) out[e] *= __fdividef(zg[e], 1.0f + ex2_approx(-zg[e] * kLog2e));   // * silu(z)
+                }
+            }
             if (writer && cnt > 0) store_steps_n<IO, PER>(yrow + t0 + first, out, cnt, vec_out);
         };
         // The same for the 16 steps of one half chunk (time split); both halves store.
@@ -421,10 +504,10 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 yk[j] = yy.x + yy.y;
             }
         };
-        auto full_steps = [&](int gi, const float (&u)[R], const float (&a)[R][SPT]) {
+        auto full_steps = [&](int gi, const float (&u)[R], const float (&a)[R][SPT], const float (&zg)[ZN]) {
             float yk[R];
             group_steps(gi, u, a, yk);
-            reduce_store(gi * R, yk);
+            reduce_store(gi * R, yk, zg);
         };
 
         // The remaining nval < T steps of the sequence, one group at a time.
@@ -433,69 +516,12 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             for (int gi = 0; gi < ngroups; ++gi) {
                 const int tau0 = gi * R;
                 const int kmax = nval - tau0 < R ? nval - tau0 : R;
-                const int bx = tau0 / TL::BOX_T;
-                const int col = tau0 - bx * TL::BOX_T;
-                const unsigned char* xt = sbuf + TL::OFF_X + bx * TL::XBOX;
-                const unsigned char* dtl = sbuf + TL::OFF_D + bx * TL::XBOX;
-                float dl[R], xl[R];
-    #pragma unroll
-                for (int j = 0; j < R; j += 4) {
-                    const float4 dq = load4(reinterpret_cast<const IO*>(dtl + sw128(c, (col + j) * EB)));
-                    const float4 xq = load4(reinterpret_cast<const IO*>(xt + sw128(c, (col + j) * EB)));
-                    dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
-                    xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
-                }
-                float u[R];
-    #pragma unroll
-                for (int j = 0; j < R; j += 2) {
-                    const float2 uu = __fmul2_rn(f2(dl[j], dl[j + 1]), f2(xl[j], xl[j + 1]));
-                    u[j] = uu.x;
-                    u[j + 1] = uu.y;
-                }
-                float a[R][SPT];
-    #pragma unroll
-                for (int sI = 0; sI < SPT; ++sI) {
-    #pragma unroll
-                    for (int j = 0; j < R; j += 2) {
-                        const float2 r2 = __fmul2_rn(f2(dl[j], dl[j + 1]), A2p[sI]);
-                        a[j][sI] = ex2_approx(r2.x);
-                        a[j + 1][sI] = ex2_approx(r2.y);
-                    }
-                }
-                float yk[R];
+                float u[R], a[R][SPT], yk[R], zg[ZN];
+                prep(gi, u, a, zg);
                 if (kmax == R) {
-    #pragma unroll
-                    for (int j = 0; j < R; ++j) {
-                        const float* brow = Bg + (tau0 + j) * BP;
-                        const float* crow = Cg + (tau0 + j) * BP;
-                        float bq[SPT], cq[SPT];
-    #pragma unroll
-                        for (int q = 0; q < SPT; q += 4 > SPT ? SPT : 4) {
-                            if constexpr (SPT >= 4) {
-                                const float4 b4 = *reinterpret_cast<const float4*>(brow + q);
-                                const float4 c4 = *reinterpret_cast<const float4*>(crow + q);
-                                bq[q] = b4.x; bq[q + 1] = b4.y; bq[q + 2] = b4.z; bq[q + 3] = b4.w;
-                                cq[q] = c4.x; cq[q + 1] = c4.y; cq[q + 2] = c4.z; cq[q + 3] = c4.w;
-                            } else {
-                                const float2 b2 = *reinterpret_cast<const float2*>(brow + q);
-                                const float2 c2 = *reinterpret_cast<const float2*>(crow + q);
-                                bq[q] = b2.x; bq[q + 1] = b2.y;
-                                cq[q] = c2.x; cq[q + 1] = c2.y;
-                            }
-                        }
-                        const float2 uu = f2(u[j], u[j]);
-                        float2 yy = f2(0.0f, 0.0f);
-    #pragma unroll
-                        for (int q = 0; q < NPAIR; ++q) {
-                            const float2 w = __fmul2_rn(uu, f2(bq[2 * q], bq[2 * q + 1]));
-                            vv[q] = __ffma2_rn(beta2, vv[q], w);
-                            hh[q] = __ffma2_rn(f2(a[j][2 * q], a[j][2 * q + 1]), hh[q], vv[q]);
-                            yy = __ffma2_rn(f2(cq[2 * q], cq[2 * q + 1]), hh[q], yy);
-                        }
-                        yk[j] = yy.x + yy.y;
-                    }
+                    group_steps(gi, u, a, yk);
                 } else {
-    #pragma unroll
+#pragma unroll
                     for (int j = 0; j < R; ++j) {       // ragged end of the sequence
                         yk[j] = 0.0f;
                         if (j < kmax) {
@@ -503,7 +529,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                             const float* crow = Cg + (tau0 + j) * BP;
                             const float2 uu = f2(u[j], u[j]);
                             float2 yy = f2(0.0f, 0.0f);
-    #pragma unroll
+#pragma unroll
                             for (int q = 0; q < NPAIR; ++q) {
                                 const float2 w = __fmul2_rn(uu, f2(brow[2 * q], brow[2 * q + 1]));
                                 vv[q] = __ffma2_rn(beta2, vv[q], w);
@@ -514,8 +540,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         }
                     }
                 }
-
-                reduce_store(tau0, yk);
+                reduce_store(tau0, yk, zg);
             }
         };
 
@@ -523,16 +548,16 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (nval == T) {
                 // Full chunk: groups unrolled, each group's exponentials issued one group ahead.
                 constexpr int NG = T / R;
-                float uA[R], uB[R], aA[R][SPT], aB[R][SPT];
-                prep(0, uA, aA);
+                float uA[R], uB[R], aA[R][SPT], aB[R][SPT], zA[ZN], zB[ZN];
+                prep(0, uA, aA, zA);
 #pragma unroll
                 for (int gi = 0; gi < NG; ++gi) {
                     if ((gi & 1) == 0) {
-                        if (gi + 1 < NG) prep(gi + 1, uB, aB);
-                        full_steps(gi, uA, aA);
+                        if (gi + 1 < NG) prep(gi + 1, uB, aB, zB);
+                        full_steps(gi, uA, aA, zA);
                     } else {
-                        if (gi + 1 < NG) prep(gi + 1, uA, aA);
-                        full_steps(gi, uB, aB);
+                        if (gi + 1 < NG) prep(gi + 1, uA, aA, zA);
+                        full_steps(gi, uB, aB, zB);
                     }
                 }
             } else {
@@ -550,9 +575,9 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (nval == T) {
                 constexpr int HALF = T / 2;
                 const int gi0 = 2 * j_t;
-                float uA[R], uB[R], aA[R][SPT], aB[R][SPT], yk[HALF];
-                prep(gi0, uA, aA);
-                prep(gi0 + 1, uB, aB);
+                float uA[R], uB[R], aA[R][SPT], aB[R][SPT], yk[HALF], zd[ZN];
+                prep(gi0, uA, aA, zd);
+                prep(gi0 + 1, uB, aB, zd);
                 {
                     float y8[R];
                     group_steps(gi0, uA, aA, y8);
@@ -680,9 +705,9 @@ cudaError_t make_map_3d(CUtensorMap* m, const void* base, bool bf16_elems, uint6
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename IO, int NP, int SPT, int WARPS, int TS = 1>
+template <typename IO, int NP, int SPT, int WARPS, int TS = 1, bool EXT = false>
 cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
-    using TL = ScanTile<IO, NP, SPT, WARPS, TS>;
+    using TL = ScanTile<IO, NP, SPT, WARPS, TS, EXT>;
     ScanArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t grid = a.batch * a.tiles_per_batch;
@@ -700,7 +725,7 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
         if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
         if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
     }
-    auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS, TS>;
+    auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS, TS, EXT>;
     // The dynamic shared-memory limit is raised once per device and variant.
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
@@ -720,6 +745,19 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
 // and the natural choices for smaller state counts.
 template <typename IO>
 cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, int ts, cudaStream_t s) {
+    if (a.ext) {
+        // selective_scan_fn extras: built for the automatic tiles; a forced
+        // tile outside them falls back to the automatic one.
+        switch (np) {
+            case 16:
+                if (spt == 2 && warps == 2) return launch_variant<IO, 16, 2, 2, 1, true>(a, s);
+                return launch_variant<IO, 16, 2, 4, 1, true>(a, s);
+            case 8: return launch_variant<IO, 8, 2, 2, 1, true>(a, s);
+            case 4: return launch_variant<IO, 4, 2, 2, 1, true>(a, s);
+            case 2: return launch_variant<IO, 2, 2, 1, 1, true>(a, s);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (ts == 2) {
         // Time split: fp32 I/O and 16 padded states only.
         if constexpr (sizeof(IO) == 4) {

@@ -191,6 +191,30 @@ def scan_inputs(w: ScanWorkload, *, batch: int | None = None, seqlen: int | None
     return {"x": x, "delta": delta, "A": np.ascontiguousarray(A), "B": B, "C": C}
 
 
+def scan_extras(w: ScanWorkload, *, batch: int | None = None, seqlen: int | None = None,
+                dim: int | None = None, seed: int | None = None):
+    """Draw the selective_scan_fn extras for a scan workload: a raw delta
+    ~ N(0, 0.5) (batch, dim, L) meant to go through softplus(delta + bias),
+    delta_bias = ln(expm1(dt)) with dt log-uniform on [1e-3, 1e-1] per channel
+    (so that softplus(delta + bias) has the workloads' usual size), a skip
+    weight D ~ U(0.5, 1.5) per channel and a gate z ~ N(0, 1) (batch, dim,
+    L).  Their own seed stream (the workload's seed + 1000); for bf16
+    workloads delta and z hold bf16-rounded values."""
+    bsz = batch or w.batch
+    L = seqlen or w.seqlen
+    D = dim or w.dim
+    rd, rb, rs, rz = _streams((seed if seed is not None else seed_of(w.seed_index)) + 1000, 4)
+    delta_raw = _normal(rd, (bsz, D, L), 0.5)
+    dt = _log_uniform(rb, (D,), 1e-3, 1e-1).astype(np.float64)
+    bias = np.log(np.expm1(dt)).astype(np.float32)
+    Dskip = rs.uniform(0.5, 1.5, D).astype(np.float32)
+    z = _normal(rz, (bsz, D, L))
+    if w.io == "bf16":
+        delta_raw = bf16_round(delta_raw)
+        z = bf16_round(z)
+    return {"delta_raw": delta_raw, "delta_bias": bias, "D": Dskip, "z": z}
+
+
 def ssd_inputs(w: SSDWorkload, *, batch: int | None = None, seqlen: int | None = None,
                nheads: int | None = None, headdim: int | None = None,
                dstate: int | None = None, ngroups: int | None = None,

@@ -108,6 +108,23 @@ def test_scan_fault_injection_returns_cuda_error(lib, monkeypatch):
     assert "injected" in mm.mm_last_error()
 
 
+def test_gated_checks_its_extras(lib, monkeypatch):
+    dims = D(L=64, dim=8)
+    def call(**over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), D=None, z=None,
+                 bias=None, sp=0, h0=None, v0=None, y=_fake(5), hT=None, vT=None)
+        a.update(over)
+        return lib.mm_scan_fwd_gated(a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                                     a["bias"], a["sp"], a["h0"], a["v0"], 0.9, 1.0, a["y"], a["hT"],
+                                     a["vT"], ctypes.byref(dims), None)
+    assert call(z=ctypes.c_void_p(A16 * 7 + 4)) == 5              # misaligned gate
+    assert "z is not 16-byte aligned" in mm.mm_last_error()
+    assert call(z=_fake(5)) == 9                                  # y on top of z
+    assert call(D=_fake(5)) == 9                                  # y on top of D
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call(D=_fake(6), z=_fake(7), bias=_fake(8), sp=1) == 7  # passes every check
+
+
 def test_set_tile(lib):
     assert lib.mm_scan_set_tile(3, 2, 1) == 6
     assert lib.mm_scan_set_tile(4, 2, 3) == 6
