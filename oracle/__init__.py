@@ -64,6 +64,11 @@ def _declare(lib):
     lib.oracle_scan_gated.argtypes = [
         _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, ctypes.c_int, _f64p, _f64p,
         _f64, _f64, _i64, _i64, _i64, _i64, _i64p, _i64, _f64p, _f64p, _f64p]
+    lib.oracle_scan_bwd.restype = ctypes.c_int
+    lib.oracle_scan_bwd.argtypes = [
+        _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, ctypes.c_int, _f64p, _f64p,
+        _f64, _f64, _f32p, _f64p, _f64p, _i64, _i64, _i64, _i64, _i64p, _i64, _i64p, _i64,
+        _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p]
     lib.oracle_scan_chunked.restype = ctypes.c_int
     lib.oracle_scan_chunked.argtypes = [
         _f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p, _f64, _f64,
@@ -196,6 +201,56 @@ def scan_gated(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplu
                                vT.ctypes.data_as(_f64p))
     _check(rc, "oracle_scan_gated")
     return y, hT, vT
+
+
+def scan_bwd(x, delta, A, B, C, dout, D=None, z=None, delta_bias=None, delta_softplus=False,
+             h0=None, v0=None, dhT=None, dvT=None, beta=0.0, alpha=1.0, chan=None, bn=None,
+             lib=None):
+    """Gradients of the full selective_scan_fn forward (mm_oracle.c: oracle_scan_bwd).
+
+    Momentum Mamba README, "Gradient Flow" and "Backward Pass: Reconstructed
+    Forward + Reverse Scans", with the adjoint recursions derived from the
+    forward recurrence (the C header states them).  ``dout`` is the gradient
+    reaching the output (batch, dim, L); ``dhT``, ``dvT`` those reaching the
+    final states (batch, dim, N) or None.  Returns a dict of fp64 arrays:
+    dx, ddelta (and dz when z is given) (nchan, L); dh0, dv0 (nchan, N);
+    dA (dim, N); dD, ddelta_bias (dim,); dB, dC (nbn, L).  ``chan`` selects
+    channels b*dim + d for the per-channel results (dA, dD and ddelta_bias
+    then sum only those); ``bn`` selects (b, n) rows b*N + n of dB and dC.
+    """
+    lib = lib or load()
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    xs, xp = _f32(x, "x")
+    ds, dp = _f32(delta, "delta")
+    As, Ap = _f32(A, "A")
+    Bs, Bp = _f32(B, "B")
+    Cs, Cp = _f32(C, "C")
+    os_, op_ = _f32(dout, "dout")
+    Ds, Dp = _f32opt(D, (dim,), "D")
+    zs, zp = _f32opt(z, (batch, dim, L), "z")
+    bs, bp = _f32opt(delta_bias, (dim,), "delta_bias")
+    h0s, h0p = _f64opt(h0, (batch, dim, N), "h0")
+    v0s, v0p = _f64opt(v0, (batch, dim, N), "v0")
+    gTs, gTp = _f64opt(dhT, (batch, dim, N), "dhT")
+    pTs, pTp = _f64opt(dvT, (batch, dim, N), "dvT")
+    cs, cp, nc = _idx(chan)
+    ks, kp, nk = _idx(bn)
+    n = nc if chan is not None else batch * dim
+    m = nk if bn is not None else batch * N
+    out = {"dx": np.empty((n, L)), "ddelta": np.empty((n, L)), "dh0": np.empty((n, N)),
+           "dv0": np.empty((n, N)), "dA": np.empty((dim, N)), "dD": np.empty(dim),
+           "ddelta_bias": np.empty(dim), "dB": np.empty((m, L)), "dC": np.empty((m, L))}
+    if z is not None:
+        out["dz"] = np.empty((n, L))
+    ptr = lambda k: out[k].ctypes.data_as(_f64p) if k in out else None
+    rc = lib.oracle_scan_bwd(xp, dp, Ap, Bp, Cp, Dp, zp, bp, 1 if delta_softplus else 0,
+                             h0p, v0p, float(beta), float(alpha), op_, gTp, pTp,
+                             batch, L, dim, N, cp, nc, kp, nk,
+                             ptr("dx"), ptr("ddelta"), ptr("dz"), ptr("dh0"), ptr("dv0"),
+                             ptr("dA"), ptr("dD"), ptr("ddelta_bias"), ptr("dB"), ptr("dC"))
+    _check(rc, "oracle_scan_bwd")
+    return out
 
 
 def scan_chunked(x, delta, A, B, C, h0=None, v0=None, beta=0.0, alpha=1.0,

@@ -1,6 +1,7 @@
 /*
- * mm_oracle.c -- plain, slow, fp64 CPU oracle for the Momentum Mamba forward
- * selective scan and its Mamba-2 scalar-A chunked (SSD) form.
+ * mm_oracle.c -- plain, slow, fp64 CPU oracle for the Momentum Mamba
+ * selective scan (forward and backward) and its Mamba-2 scalar-A chunked
+ * (SSD) form.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
  * call this file: only the tests, the package's smoke check and the CPU
@@ -17,7 +18,8 @@
  *  [MM]  "Momentum Mamba: Enhanced State Space Models with Momentum"
  *        (t-khanusa/Momentum_Mamba README), sections "Momentum Mamba
  *        Recurrence", "Discretization Note", "selective_scan_fn",
- *        "Mamba Module" (step / velocity_state).
+ *        "Mamba Module" (step / velocity_state), "Gradient Flow" and
+ *        "Backward Pass: Reconstructed Forward + Reverse Scans".
  *  [SEL] "Mamba: Choosing What to Remember Based on the Input", section
  *        "Expressing the update and read as equations" (read-out of the
  *        post-update state).
@@ -180,6 +182,260 @@ int oracle_scan_gated(const float *x, const float *delta, const float *A,
                 o *= zt / (1.0 + exp(-zt));
             }
             yr[t] = o;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the full selective_scan_fn forward                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [MM] "Gradient Flow" and "Backward Pass: Reconstructed Forward + Reverse
+ * Scans": the forward states are rebuilt, then the gradients with respect to
+ * the hidden state and the velocity run backwards in time.  The printed
+ * formulas use one symbol for both of those gradients and leave a term out
+ * of the velocity's, so the recursions are derived here from the forward
+ * recurrence itself.  With G_t = dL/dh_t and P_t = dL/dv_t (total
+ * derivatives: everything that depends on the state later is included),
+ *
+ *     G_t = dy_t C_t[n] + a_{t+1} G_{t+1}      (for t = L-1: + dhT instead)
+ *     P_t = G_t + beta P_{t+1}                 (for t = L-1: + dvT instead)
+ *
+ * because h_t feeds y_t and h_{t+1} (factor a_{t+1}), and v_t feeds h_t
+ * (factor 1) and v_{t+1} (factor beta).  The local terms are the ones the
+ * pages list, with dL/dh_t and dL/dv_t read as G_t and P_t:
+ *
+ *     dx_t       += alpha delta'_t B_t[n] P_t
+ *     ddelta'_t  += alpha B_t[n] x_t P_t + A[d,n] a_t h_{t-1} G_t
+ *     dA[d,n]    += delta'_t a_t h_{t-1} G_t           (all t and b)
+ *     dB_t[n]    += alpha delta'_t x_t P_t             (all d of the batch row)
+ *     dC_t[n]    += dy_t h_t                           (all d of the batch row)
+ *     dh0 = a_0 G_0,   dv0 = beta P_0
+ *
+ * with a_t = exp(delta'_t A[d,n]).  dy is the gradient that reaches the
+ * read-out.  Around it, following the readings of oracle_scan_gated, with
+ * o_t = y_t + D x_t and s_t = 1 / (1 + e^{-z_t}):
+ *
+ *     dy_t = dout_t z_t s_t         (no gate: dy_t = dout_t)
+ *     dz_t = dout_t o_t s_t (1 + z_t (1 - s_t))
+ *     dx_t += D dy_t,   dD += dy_t x_t
+ *     ddelta_t = ddelta'_t / (1 + e^{-(delta_t + bias)})   (softplus; else ddelta'_t)
+ *     dbias += ddelta_t
+ */
+
+/* delta' of channel c and the gradient dy reaching its read-out; dz_r and
+ * the gate-side terms are written when asked for.  The forward over all
+ * states is run once when the gate needs y. */
+static void bwd_channel_prep(int64_t c, const float *x, const float *delta, const float *A,
+                             const float *Bm, const float *Cm, const float *Dv, const float *z,
+                             const float *dbias, int softplus, const double *h0, const double *v0,
+                             double beta, double alpha, const float *dout,
+                             int64_t seqlen, int64_t dim, int64_t dstate,
+                             double *dp, double *dy, double *dz_r)
+{
+    const int64_t b = c / dim;
+    const int64_t d = c % dim;
+    const float *xr = x + c * seqlen;
+    const float *dr = delta + c * seqlen;
+    for (int64_t t = 0; t < seqlen; ++t) {
+        double u = (double)dr[t] + (dbias ? (double)dbias[d] : 0.0);
+        dp[t] = softplus ? softplus_f64(u) : u;
+        dy[t] = (double)dout[c * seqlen + t];
+    }
+    if (!z) return;
+    /* the gate needs o_t = y_t + D x_t */
+    double *o = (double *)calloc((size_t)seqlen, sizeof(double));
+    for (int64_t n = 0; n < dstate; ++n) {
+        double h = h0 ? h0[c * dstate + n] : 0.0;
+        double v = v0 ? v0[c * dstate + n] : 0.0;
+        const double a_dn = (double)A[d * dstate + n];
+        const float *Bn = Bm + (b * dstate + n) * seqlen;
+        const float *Cn = Cm + (b * dstate + n) * seqlen;
+        for (int64_t t = 0; t < seqlen; ++t) {
+            v = beta * v + alpha * (dp[t] * (double)Bn[t] * (double)xr[t]);
+            h = exp(dp[t] * a_dn) * h + v;
+            o[t] += (double)Cn[t] * h;
+        }
+    }
+    for (int64_t t = 0; t < seqlen; ++t) {
+        const double ot = o[t] + (Dv ? (double)Dv[d] * (double)xr[t] : 0.0);
+        const double zt = (double)z[c * seqlen + t];
+        const double st = 1.0 / (1.0 + exp(-zt));
+        if (dz_r) dz_r[t] = dy[t] * ot * st * (1.0 + zt * (1.0 - st));
+        dy[t] = dy[t] * zt * st;
+    }
+    free(o);
+}
+
+/* One (b, d, n) chain: the forward states of every step, then the reverse
+ * sweep giving G_t and P_t.  Returns a_0 G_0 and beta P_0 in *gh0, *gv0. */
+static void bwd_chain(const double *dp, const float *xr, double a_dn, const float *Bn,
+                      const float *Cn, const double *dy, double h_init, double v_init,
+                      double beta, double alpha, double gT, double pT, int64_t seqlen,
+                      double *hs, double *vs, double *as, double *G, double *P,
+                      double *gh0, double *gv0)
+{
+    double h = h_init, v = v_init;
+    for (int64_t t = 0; t < seqlen; ++t) {
+        const double abar = exp(dp[t] * a_dn);
+        v = beta * v + alpha * (dp[t] * (double)Bn[t] * (double)xr[t]);
+        h = abar * h + v;
+        hs[t] = h;
+        vs[t] = v;
+        as[t] = abar;
+    }
+    double cg = gT, cp = pT;          /* a_{t+1} G_{t+1} and beta P_{t+1} */
+    for (int64_t t = seqlen - 1; t >= 0; --t) {
+        const double g = dy[t] * (double)Cn[t] + cg;
+        const double p = g + cp;
+        G[t] = g;
+        P[t] = p;
+        cg = as[t] * g;
+        cp = beta * p;
+    }
+    *gh0 = cg;
+    *gv0 = cp;
+}
+
+/*
+ * Arguments as oracle_scan_gated, plus dout (batch, dim, L) and dhT, dvT
+ * (batch, dim, dstate; NULL = 0), the gradients arriving at the outputs.
+ * Per-channel results are computed for the channels `chan` lists (NULL: all,
+ * in order) and written as rows r: dx, ddelta, dz (nchan, L); dh0, dv0
+ * (nchan, dstate).  dA (dim, dstate), dD and dbias (dim) sum the listed
+ * channels' terms (all channels: the full gradients).  dB and dC rows are
+ * computed for the (b, n) pairs `bn` lists as flat indices b*dstate + n
+ * (NULL: all, in order), each summed over every d: (nbn, L).  Any output
+ * may be NULL.
+ */
+int oracle_scan_bwd(const float *x, const float *delta, const float *A,
+                    const float *Bm, const float *Cm,
+                    const float *Dv, const float *z, const float *dbias, int softplus,
+                    const double *h0, const double *v0, double beta, double alpha,
+                    const float *dout, const double *dhT, const double *dvT,
+                    int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                    const int64_t *chan, int64_t nchan, const int64_t *bn, int64_t nbn,
+                    double *dx, double *ddelta, double *dz, double *dh0, double *dv0,
+                    double *dA, double *dD, double *ddbias, double *dB, double *dC)
+{
+    if (!x || !delta || !A || !Bm || !Cm || !dout) return ORACLE_ERR_ARG;
+    if (batch < 1 || seqlen < 1 || dim < 1 || dstate < 1) return ORACLE_ERR_ARG;
+    if (!chan) nchan = batch * dim;
+    if (!bn) nbn = batch * dstate;
+    if (nchan < 0 || nbn < 0) return ORACLE_ERR_ARG;
+    const size_t L = (size_t)seqlen;
+
+    /* per-channel terms of dA, dD, dbias, summed in channel order afterwards */
+    double *dA_r = (double *)calloc((size_t)nchan * (size_t)dstate, sizeof(double));
+    double *dD_r = (double *)calloc((size_t)nchan, sizeof(double));
+    double *db_r = (double *)calloc((size_t)nchan, sizeof(double));
+
+    int64_t r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nchan; ++r) {
+        const int64_t c = chan ? chan[r] : r;
+        const int64_t b = c / dim;
+        const int64_t d = c % dim;
+        const float *xr = x + c * seqlen;
+        double *buf = (double *)malloc(9 * L * sizeof(double));
+        double *dp = buf, *dy = buf + L, *hs = buf + 2 * L, *vs = buf + 3 * L, *as = buf + 4 * L;
+        double *G = buf + 5 * L, *P = buf + 6 * L, *gx = buf + 7 * L, *gd = buf + 8 * L;
+        bwd_channel_prep(c, x, delta, A, Bm, Cm, Dv, z, dbias, softplus, h0, v0, beta, alpha,
+                         dout, seqlen, dim, dstate, dp, dy, dz ? dz + r * seqlen : NULL);
+        for (size_t t = 0; t < L; ++t) gx[t] = gd[t] = 0.0;
+        for (int64_t n = 0; n < dstate; ++n) {
+            const double a_dn = (double)A[d * dstate + n];
+            const float *Bn = Bm + (b * dstate + n) * seqlen;
+            const float *Cn = Cm + (b * dstate + n) * seqlen;
+            const double hi = h0 ? h0[c * dstate + n] : 0.0;
+            const double vi = v0 ? v0[c * dstate + n] : 0.0;
+            double gh0, gv0;
+            bwd_chain(dp, xr, a_dn, Bn, Cn, dy, hi, vi, beta, alpha,
+                      dhT ? dhT[c * dstate + n] : 0.0, dvT ? dvT[c * dstate + n] : 0.0,
+                      seqlen, hs, vs, as, G, P, &gh0, &gv0);
+            double acc_a = 0.0;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                const double hprev = t > 0 ? hs[t - 1] : hi;
+                const double decay_term = as[t] * hprev * G[t];      /* a_t h_{t-1} G_t */
+                gx[t] += alpha * dp[t] * (double)Bn[t] * P[t];
+                gd[t] += alpha * (double)Bn[t] * (double)xr[t] * P[t] + a_dn * decay_term;
+                acc_a += dp[t] * decay_term;
+            }
+            dA_r[r * dstate + n] = acc_a;
+            if (dh0) dh0[r * dstate + n] = gh0;
+            if (dv0) dv0[r * dstate + n] = gv0;
+        }
+        double accD = 0.0, accb = 0.0;
+        for (int64_t t = 0; t < seqlen; ++t) {
+            double g_delta = gd[t];
+            if (softplus) {
+                const double u = (double)delta[c * seqlen + t] + (dbias ? (double)dbias[d] : 0.0);
+                g_delta *= 1.0 / (1.0 + exp(-u));
+            }
+            const double g_x = gx[t] + (Dv ? (double)Dv[d] * dy[t] : 0.0);
+            if (dx) dx[r * seqlen + t] = g_x;
+            if (ddelta) ddelta[r * seqlen + t] = g_delta;
+            accD += dy[t] * (double)xr[t];
+            accb += g_delta;
+        }
+        dD_r[r] = accD;
+        db_r[r] = accb;
+        free(buf);
+    }
+    if (dA) {
+        for (int64_t i = 0; i < dim * dstate; ++i) dA[i] = 0.0;
+        for (r = 0; r < nchan; ++r) {
+            const int64_t d = (chan ? chan[r] : r) % dim;
+            for (int64_t n = 0; n < dstate; ++n) dA[d * dstate + n] += dA_r[r * dstate + n];
+        }
+    }
+    if (dD || ddbias) {
+        for (int64_t i = 0; i < dim; ++i) {
+            if (dD) dD[i] = 0.0;
+            if (ddbias) ddbias[i] = 0.0;
+        }
+        for (r = 0; r < nchan; ++r) {
+            const int64_t d = (chan ? chan[r] : r) % dim;
+            if (dD) dD[d] += dD_r[r];
+            if (ddbias) ddbias[d] += db_r[r];
+        }
+    }
+    free(dA_r);
+    free(dD_r);
+    free(db_r);
+
+    if (dB || dC) {
+        int64_t k;
+#pragma omp parallel for schedule(dynamic, 1)
+        for (k = 0; k < nbn; ++k) {
+            const int64_t f = bn ? bn[k] : k;
+            const int64_t b = f / dstate;
+            const int64_t n = f % dstate;
+            const float *Bn = Bm + (b * dstate + n) * seqlen;
+            const float *Cn = Cm + (b * dstate + n) * seqlen;
+            double *buf = (double *)malloc(7 * L * sizeof(double));
+            double *dp = buf, *dy = buf + L, *hs = buf + 2 * L, *vs = buf + 3 * L, *as = buf + 4 * L;
+            double *G = buf + 5 * L, *P = buf + 6 * L;
+            if (dB) for (int64_t t = 0; t < seqlen; ++t) dB[k * seqlen + t] = 0.0;
+            if (dC) for (int64_t t = 0; t < seqlen; ++t) dC[k * seqlen + t] = 0.0;
+            for (int64_t d = 0; d < dim; ++d) {
+                const int64_t c = b * dim + d;
+                const float *xr = x + c * seqlen;
+                bwd_channel_prep(c, x, delta, A, Bm, Cm, Dv, z, dbias, softplus, h0, v0, beta,
+                                 alpha, dout, seqlen, dim, dstate, dp, dy, NULL);
+                double gh0, gv0;
+                bwd_chain(dp, xr, (double)A[d * dstate + n], Bn, Cn, dy,
+                          h0 ? h0[c * dstate + n] : 0.0, v0 ? v0[c * dstate + n] : 0.0,
+                          beta, alpha, dhT ? dhT[c * dstate + n] : 0.0,
+                          dvT ? dvT[c * dstate + n] : 0.0, seqlen, hs, vs, as, G, P, &gh0, &gv0);
+                for (int64_t t = 0; t < seqlen; ++t) {
+                    if (dB) dB[k * seqlen + t] += alpha * dp[t] * (double)xr[t] * P[t];
+                    if (dC) dC[k * seqlen + t] += dy[t] * hs[t];
+                }
+            }
+            free(buf);
         }
     }
     return ORACLE_OK;

@@ -72,6 +72,35 @@ GATED_MUTANTS = {
 }
 
 
+# Backward: each is a plausible slip in the adjoint recursions or a local term,
+# the first one the velocity recursion exactly as the pages print it (the
+# read-out gradient only, without the hidden state's full gradient).
+BWD_MUTANTS = {
+    "bwd_velocity_adjoint_as_printed": ("const double p = g + cp;",
+                                        "const double p = dy[t] * (double)Cn[t] + cp;"),
+    "bwd_decay_a_t_not_a_t1": ("cg = as[t] * g;", "cg = (t > 0 ? as[t - 1] : as[0]) * g;"),
+    "bwd_velocity_no_beta": ("cp = beta * p;", "cp = p;"),
+    "bwd_ddelta_no_exp_path": (" + a_dn * decay_term;", ";"),
+    "bwd_dA_without_delta": ("acc_a += dp[t] * decay_term;", "acc_a += decay_term;"),
+    "bwd_dB_without_alpha": ("dB[k * seqlen + t] += alpha * dp[t]", "dB[k * seqlen + t] += dp[t]"),
+    "bwd_dC_previous_state": ("dC[k * seqlen + t] += dy[t] * hs[t];",
+                              "dC[k * seqlen + t] += dy[t] * (t > 0 ? hs[t - 1] : 0.0);"),
+    "bwd_silu_grad_missing_term": ("dy[t] * ot * st * (1.0 + zt * (1.0 - st))",
+                                   "dy[t] * ot * st * (1.0 - st)"),
+    "bwd_softplus_grad_dropped": ("g_delta *= 1.0 / (1.0 + exp(-u));", ""),
+    "bwd_skip_grad_ungated": ("(Dv ? (double)Dv[d] * dy[t] : 0.0)",
+                              "(Dv ? (double)Dv[d] * (double)dout[c * seqlen + t] : 0.0)"),
+    "bwd_dhT_ignored": ("dhT ? dhT[c * dstate + n] : 0.0, dvT ? dvT[c * dstate + n] : 0.0,",
+                        "0.0, dvT ? dvT[c * dstate + n] : 0.0,"),
+}
+
+
+def _bwd_pins(lib):
+    """Finite-difference pins of tests/test_oracle_bwd_pins.py run against `lib`."""
+    from tests import test_oracle_bwd_pins as bp
+    return bp.fd_failures("momentum_h0v0", lib=lib) + bp.fd_failures("gated_softplus", lib=lib)
+
+
 def _gated_pins(lib):
     """Pins of tests/test_oracle_gated_pins.py run against `lib`."""
     from tests import test_oracle_gated_pins as gp
@@ -159,9 +188,11 @@ def test_real_oracle_passes_the_mutant_pins():
     assert _gated_pins(oracle.load()) == []
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SSD_MUTANTS) + sorted(GATED_MUTANTS))
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SSD_MUTANTS) + sorted(GATED_MUTANTS)
+                         + sorted(BWD_MUTANTS))
 def test_planted_mistake_is_caught(name, tmp_path):
-    old, new = MUTANTS.get(name) or SSD_MUTANTS.get(name) or GATED_MUTANTS[name]
+    old, new = (MUTANTS.get(name) or SSD_MUTANTS.get(name) or GATED_MUTANTS.get(name)
+                or BWD_MUTANTS[name])
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation anchor for {name} not found"
     mut_src = tmp_path / "mm_oracle.c"
@@ -171,5 +202,6 @@ def test_planted_mistake_is_caught(name, tmp_path):
     subprocess.run(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-shared",
                     "-fPIC", "-std=c11", "-o", str(so), str(mut_src), "-lm"], check=True)
     lib = oracle.load(str(so))
-    pins = _pins if name in MUTANTS else _ssd_pins if name in SSD_MUTANTS else _gated_pins
+    pins = (_pins if name in MUTANTS else _ssd_pins if name in SSD_MUTANTS
+            else _gated_pins if name in GATED_MUTANTS else _bwd_pins)
     assert pins(lib), f"no pin caught the planted mistake '{name}'"
