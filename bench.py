@@ -545,7 +545,7 @@ def main(argv=None):
         if args.gated:
             mm.mm_scan_fwd_gated(s["x"], s["delta"], s["A"], s["B"], s["C"], s["D"], s["z"],
                                  s["delta_bias"], 1, None, None, beta, alpha, s["y"], s["hT"], s["vT"],
-                                 stream)
+                                 None, stream)
         else:
             mm.mm_scan_fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha,
                            s["y"], s["hT"], s["vT"], stream)

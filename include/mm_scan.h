@@ -46,6 +46,9 @@ typedef enum {
 /* Storage type of the streamed tensors (x, delta, B, C, y). */
 typedef enum { MM_F32 = 0, MM_BF16 = 1 } mm_dtype;
 
+/* Steps between two checkpoints of the forward's state (see mm_scan_bwd). */
+#define MM_SCAN_CHUNK 64
+
 /* Sizes of one Mamba-1 scan call. */
 typedef struct {
     int64_t batch;   /* b: independent sequences                          */
@@ -135,6 +138,12 @@ mm_status mm_scan_fwd(const void *x, const void *delta, const float *A,
  * may overlap no input, z, D and delta_bias included), streaming property
  * and errors as mm_scan_fwd.  delta' is computed once per (batch, channel,
  * step) in fp32 from the loaded delta; the gate uses a fast exponential.
+ *
+ *   ckpt   (batch, dim, ceil(L / 64), 2, dstate) fp32, or NULL: for every
+ *          chunk k of MM_SCAN_CHUNK = 64 steps, (h, v) after its last step
+ *          (step min(64 k + 63, L - 1)); [.., 0, :] holds h and [.., 1, :]
+ *          holds v.  This is what mm_scan_bwd restarts from.  Size in bytes:
+ *          mm_scan_ckpt_size.  It may overlap no other argument.
  */
 mm_status mm_scan_fwd_gated(const void *x, const void *delta, const float *A,
                             const void *B, const void *C,
@@ -142,8 +151,59 @@ mm_status mm_scan_fwd_gated(const void *x, const void *delta, const float *A,
                             const float *delta_bias, int delta_softplus,
                             const float *h0, const float *v0,
                             float beta, float alpha,
-                            void *y, float *hT, float *vT,
+                            void *y, float *hT, float *vT, float *ckpt,
                             const mm_scan_dims *dims, void *stream);
+
+/* mm_scan_ckpt_size -- bytes of the checkpoint buffer of mm_scan_fwd_gated
+ * and mm_scan_bwd: batch * dim * ceil(seqlen / 64) * 2 * dstate * 4.
+ * Errors as the size checks of mm_scan_fwd. */
+mm_status mm_scan_ckpt_size(const mm_scan_dims *dims, size_t *bytes);
+
+/*
+ * mm_scan_bwd -- gradients of mm_scan_fwd ("Momentum Mamba: Enhanced State
+ * Space Models with Momentum", sections "Gradient Flow" and "Backward Pass:
+ * Reconstructed Forward + Reverse Scans").  The page's printed recursions
+ * use one symbol for both state gradients and omit a term; the ones used
+ * here follow from the recurrence.  Per (b, d, n), with G_t = dL/dh_t and
+ * P_t = dL/dv_t:
+ *
+ *   G_t = dy_t C_t[n] + a_{t+1} G_{t+1}      (G after the last step: dhT)
+ *   P_t = G_t + beta P_{t+1}                 (P after the last step: dvT)
+ *   dx_t     = alpha delta_t sum_n B_t[n] P_t[n]
+ *   ddelta_t = alpha x_t sum_n B_t[n] P_t[n] + sum_n A[d,n] a_t h_{t-1}[n] G_t[n]
+ *   dA[d,n]  = sum over b, t of delta_t a_t h_{t-1}[n] G_t[n]
+ *   dB_t[n]  = sum over d of alpha delta_t x_t P_t[n]   (per batch row)
+ *   dC_t[n]  = sum over d of dy_t h_t[n]                (per batch row)
+ *   dh0 = a_0 G_0,  dv0 = beta P_0,     a_t = exp(delta_t A[d,n])
+ *
+ * Inputs: x, delta, A, B, C, h0, v0, beta, alpha and dims exactly as given
+ * to the forward; ckpt as mm_scan_fwd_gated wrote it for those inputs (it
+ * may be NULL when seqlen <= 64); dy (batch, dim, L) io: the gradient
+ * reaching y; dhT, dvT (batch, dim, dstate) fp32: the gradients reaching
+ * hT, vT, or NULL for zero.
+ * Outputs (overwritten): dx, ddelta (batch, dim, L) io (rounded to nearest
+ * even for bf16); dA (dim, dstate), dB, dC (batch, dstate, L) fp32 (sums:
+ * the order of their additions is not fixed, so they can differ in the
+ * last bits between runs); dh0, dv0 (batch, dim, dstate) fp32 or NULL.
+ * No output may overlap an input or another output (MM_ERR_ALIAS); every
+ * pointer must be 16-byte aligned.
+ *
+ * Work: the kernel restarts every 64-step chunk from its checkpoint and
+ * rebuilds the states of each 8 steps once more on the way back, so it
+ * performs about two forward passes and one reverse pass of arithmetic.
+ *
+ * Errors: MM_ERR_NULL (a required pointer, or ckpt with seqlen > 64),
+ * MM_ERR_DIMS, MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE,
+ * MM_ERR_SCALAR, MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA.
+ */
+mm_status mm_scan_bwd(const void *x, const void *delta, const float *A,
+                      const void *B, const void *C,
+                      const float *h0, const float *v0, float beta, float alpha,
+                      const float *ckpt, const void *dy,
+                      const float *dhT, const float *dvT,
+                      void *dx, void *ddelta, float *dA, float *dB, float *dC,
+                      float *dh0, float *dv0,
+                      const mm_scan_dims *dims, void *stream);
 
 /* Sizes of one Mamba-2 SSD call. */
 typedef struct {

@@ -24,9 +24,10 @@ import threading
 
 __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
-    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_ssd_fwd", "mm_ssd_workspace_size", "mm_status_string",
-    "mm_last_error", "mm_scan_set_tile", "mm_version", "mm_device_status",
-    "scan_fwd", "ssd_fwd", "scan_fwd_host", "EXPORTED_SYMBOLS",
+    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_ssd_fwd",
+    "mm_ssd_workspace_size", "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
+    "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
+    "EXPORTED_SYMBOLS", "MM_SCAN_CHUNK",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +37,7 @@ _lib = None
 
 MM_F32 = 0
 MM_BF16 = 1
+MM_SCAN_CHUNK = 64      # steps between two checkpoints of the forward's state
 
 STATUS_NAMES = {
     0: "MM_OK", 1: "MM_ERR_NULL", 2: "MM_ERR_DIMS", 3: "MM_ERR_SCALAR", 4: "MM_ERR_DTYPE",
@@ -44,7 +46,8 @@ STATUS_NAMES = {
 }
 
 # Every function include/mm_scan.h declares.
-EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_ssd_workspace_size", "mm_ssd_fwd",
+EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd",
+                    "mm_ssd_workspace_size", "mm_ssd_fwd",
                     "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
 
@@ -80,7 +83,12 @@ def _declare(lib):
                                 ctypes.POINTER(ScanDims), vp]
     lib.mm_scan_fwd_gated.restype = ctypes.c_int
     lib.mm_scan_fwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, f, f,
-                                      vp, vp, vp, ctypes.POINTER(ScanDims), vp]
+                                      vp, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
+    lib.mm_scan_ckpt_size.restype = ctypes.c_int
+    lib.mm_scan_ckpt_size.argtypes = [ctypes.POINTER(ScanDims), ctypes.POINTER(ctypes.c_size_t)]
+    lib.mm_scan_bwd.restype = ctypes.c_int
+    lib.mm_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp,
+                                vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
     lib.mm_ssd_workspace_size.restype = ctypes.c_int
     lib.mm_ssd_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.POINTER(ctypes.c_size_t)]
     lib.mm_ssd_fwd.restype = ctypes.c_int
@@ -160,18 +168,46 @@ def mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
 
 
 def mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
-                      y, hT, vT, stream=None):
+                      y, hT, vT, ckpt=None, stream=None):
     """C entry point mm_scan_fwd_gated (marshalling only): mm_scan_fwd plus the
     optional D (dim,) fp32, z (batch, dim, L) in the storage type of x,
-    delta_bias (dim,) fp32 and the softplus switch."""
+    delta_bias (dim,) fp32, the softplus switch and the checkpoint output
+    ckpt (batch, dim, ceil(L / 64), 2, N) fp32."""
     batch, dim, L = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
     rc = load_library().mm_scan_fwd_gated(
         _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
         1 if delta_softplus else 0, _ptr(h0), _ptr(v0), float(beta), float(alpha), _ptr(y), _ptr(hT),
-        _ptr(vT), ctypes.byref(dims), _stream_handle(stream))
+        _ptr(vT), _ptr(ckpt), ctypes.byref(dims), _stream_handle(stream))
     _check(rc, "mm_scan_fwd_gated")
+
+
+def mm_scan_ckpt_size(batch, seqlen, dim, dstate, io=MM_F32) -> int:
+    """C entry point mm_scan_ckpt_size: bytes of the checkpoint buffer."""
+    dims = ScanDims(batch, seqlen, dim, dstate, io)
+    out = ctypes.c_size_t(0)
+    _check(load_library().mm_scan_ckpt_size(ctypes.byref(dims), ctypes.byref(out)), "mm_scan_ckpt_size")
+    return int(out.value)
+
+
+def mm_scan_bwd(x, delta, A, B, C, h0, v0, beta, alpha, ckpt, dy, dhT, dvT,
+                dx, ddelta, dA, dB, dC, dh0, dv0, stream=None):
+    """C entry point mm_scan_bwd on torch CUDA tensors (marshalling only).
+
+    Inputs as given to the forward, ckpt as the forward wrote it, dy (batch,
+    dim, L) in the storage type of x, dhT, dvT (batch, dim, N) fp32 or None.
+    Outputs: dx, ddelta like x; dA (dim, N), dB, dC (batch, N, L) fp32;
+    dh0, dv0 (batch, dim, N) fp32 or None.
+    """
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_bwd(
+        _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(v0), float(beta),
+        float(alpha), _ptr(ckpt), _ptr(dy), _ptr(dhT), _ptr(dvT), _ptr(dx), _ptr(ddelta), _ptr(dA),
+        _ptr(dB), _ptr(dC), _ptr(dh0), _ptr(dv0), ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_bwd")
 
 
 def mm_ssd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk) -> int:
@@ -239,8 +275,40 @@ def scan_fwd(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0,
         mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream)
     else:
         mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
-                          y, hT, vT, stream)
+                          y, hT, vT, None, stream)
     return y, hT, vT
+
+
+def scan_fwd_train(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, stream=None):
+    """Forward that also keeps the checkpoints the backward restarts from:
+    returns (y, hT, vT, ckpt), ckpt (batch, dim, ceil(L / 64), 2, N) fp32."""
+    import torch
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    y = torch.empty_like(x)
+    hT = torch.empty((batch, dim, N), device=x.device, dtype=torch.float32)
+    vT = torch.empty_like(hT)
+    ckpt = torch.empty((batch, dim, (L + MM_SCAN_CHUNK - 1) // MM_SCAN_CHUNK, 2, N), device=x.device,
+                       dtype=torch.float32)
+    mm_scan_fwd_gated(x, delta, A, B, C, None, None, None, False, h0, v0, beta, alpha, y, hT, vT,
+                      ckpt, stream)
+    return y, hT, vT, ckpt
+
+
+def scan_bwd(x, delta, A, B, C, ckpt, dy, h0=None, v0=None, dhT=None, dvT=None, beta=0.9,
+             alpha=1.0, stream=None):
+    """Allocate the gradients and run mm_scan_bwd; returns a dict with dx,
+    ddelta, dA, dB, dC, dh0, dv0."""
+    import torch
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    f32 = dict(device=x.device, dtype=torch.float32)
+    g = {"dx": torch.empty_like(x), "ddelta": torch.empty_like(x), "dA": torch.empty((dim, N), **f32),
+         "dB": torch.empty((batch, N, L), **f32), "dC": torch.empty((batch, N, L), **f32),
+         "dh0": torch.empty((batch, dim, N), **f32), "dv0": torch.empty((batch, dim, N), **f32)}
+    mm_scan_bwd(x, delta, A, B, C, h0, v0, beta, alpha, ckpt, dy, dhT, dvT, g["dx"], g["ddelta"],
+                g["dA"], g["dB"], g["dC"], g["dh0"], g["dv0"], stream)
+    return g
 
 
 def ssd_fwd(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, return_last_state=True,

@@ -74,6 +74,43 @@ mm_status from_cuda(cudaError_t e, const char* what) {
     return fail(MM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
 }
 
+// Checks shared by the scan calls (sizes, dtype, scalars) and the byte
+// sizes of their operands.
+struct ScanSizes {
+    int64_t esize;       // bytes of one io element
+    int64_t seq_bytes;   // (batch, dim, L) io
+    int64_t bc_bytes;    // (batch, dstate, L) io
+    int64_t bcf_bytes;   // (batch, dstate, L) fp32
+    int64_t a_bytes;     // (dim, dstate) fp32
+    int64_t st_bytes;    // (batch, dim, dstate) fp32
+    int64_t d_bytes;     // (dim) fp32
+    int64_t ck_bytes;    // (batch, dim, chunks, 2, dstate) fp32
+};
+
+mm_status check_scan_dims(const mm_scan_dims* dims, float beta, float alpha, ScanSizes* z) {
+    const int64_t bsz = dims->batch, L = dims->seqlen, D = dims->dim, N = dims->dstate;
+    if (bsz < 1 || L < 1 || D < 1 || N < 1)
+        return fail(MM_ERR_DIMS, "sizes must be >= 1 (batch=%lld seqlen=%lld dim=%lld dstate=%lld)",
+                    (long long)bsz, (long long)L, (long long)D, (long long)N);
+    if (N > 16) return fail(MM_ERR_UNSUPPORTED, "dstate=%lld > 16", (long long)N);
+    if (dims->io != MM_F32 && dims->io != MM_BF16)
+        return fail(MM_ERR_DTYPE, "io=%d is not MM_F32 or MM_BF16", (int)dims->io);
+    if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
+        return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
+    if (!std::isfinite(alpha) || alpha < 0.0f)
+        return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
+    z->esize = dims->io == MM_F32 ? 4 : 2;
+    const int64_t chunks = (L + MM_SCAN_CHUNK - 1) / MM_SCAN_CHUNK;
+    int64_t bd, bdl, bn, bnl, dn, bdn, bdc, bdc2;
+    if (!mul_ok(bsz, D, &bd) || !mul_ok(bd, L, &bdl) || !mul_ok(bdl, z->esize, &z->seq_bytes) ||
+        !mul_ok(bsz, N, &bn) || !mul_ok(bn, L, &bnl) || !mul_ok(bnl, z->esize, &z->bc_bytes) ||
+        !mul_ok(bnl, 4, &z->bcf_bytes) || !mul_ok(D, N, &dn) || !mul_ok(dn, 4, &z->a_bytes) ||
+        !mul_ok(bd, N, &bdn) || !mul_ok(bdn, 4, &z->st_bytes) || !mul_ok(D, 4, &z->d_bytes) ||
+        !mul_ok(bd, chunks, &bdc) || !mul_ok(bdc, 2 * N, &bdc2) || !mul_ok(bdc2, 4, &z->ck_bytes))
+        return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
+    return MM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -102,6 +139,7 @@ mm_status mm_device_status(void) {
     const cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return from_cuda(e, "mm_device_status: synchronize");
     const unsigned int w = mmscan::scan_read_and_clear_device_error() |
+                           mmscan::scan_bwd_read_and_clear_device_error() |
                            mmscan::ssd_read_and_clear_device_error();
     if (w) return fail(MM_ERR_DEVICE_TIMEOUT, "a device-side wait ran past its limit (word 0x%x)", w);
     return ok();
@@ -127,53 +165,43 @@ mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const vo
                       const void* C, const float* h0, const float* v0, float beta, float alpha,
                       void* y, float* hT, float* vT, const mm_scan_dims* dims, void* stream) {
     return mm_scan_fwd_gated(x, delta, A, B, C, nullptr, nullptr, nullptr, 0, h0, v0, beta, alpha,
-                             y, hT, vT, dims, stream);
+                             y, hT, vT, nullptr, dims, stream);
 }
 
 mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, const void* B,
                             const void* C, const float* Dskip, const void* z, const float* delta_bias,
                             int delta_softplus, const float* h0, const float* v0, float beta,
-                            float alpha, void* y, float* hT, float* vT, const mm_scan_dims* dims,
-                            void* stream) {
+                            float alpha, void* y, float* hT, float* vT, float* ckpt,
+                            const mm_scan_dims* dims, void* stream) {
     if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
     if (!x || !delta || !A || !B || !C || !y)
         return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
     const int64_t bsz = dims->batch, L = dims->seqlen, D = dims->dim, N = dims->dstate;
-    if (bsz < 1 || L < 1 || D < 1 || N < 1)
-        return fail(MM_ERR_DIMS, "sizes must be >= 1 (batch=%lld seqlen=%lld dim=%lld dstate=%lld)",
-                    (long long)bsz, (long long)L, (long long)D, (long long)N);
-    if (N > 16) return fail(MM_ERR_UNSUPPORTED, "dstate=%lld > 16", (long long)N);
-    if (dims->io != MM_F32 && dims->io != MM_BF16)
-        return fail(MM_ERR_DTYPE, "io=%d is not MM_F32 or MM_BF16", (int)dims->io);
-    if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
-        return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
-    if (!std::isfinite(alpha) || alpha < 0.0f)
-        return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
-    const int64_t esize = dims->io == MM_F32 ? 4 : 2;
-    int64_t bd, bdl, seq_bytes, bn, bnl, bc_bytes, dn, a_bytes, bdn, st_bytes;
-    if (!mul_ok(bsz, D, &bd) || !mul_ok(bd, L, &bdl) || !mul_ok(bdl, esize, &seq_bytes) ||
-        !mul_ok(bsz, N, &bn) || !mul_ok(bn, L, &bnl) || !mul_ok(bnl, esize, &bc_bytes) ||
-        !mul_ok(D, N, &dn) || !mul_ok(dn, 4, &a_bytes) || !mul_ok(bd, N, &bdn) ||
-        !mul_ok(bdn, 4, &st_bytes))
-        return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
-    const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT, Dskip, z, delta_bias};
+    const int64_t esize = zs.esize, seq_bytes = zs.seq_bytes, bc_bytes = zs.bc_bytes,
+                  a_bytes = zs.a_bytes, st_bytes = zs.st_bytes, d_bytes = zs.d_bytes;
+    const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT, Dskip, z, delta_bias, ckpt};
     const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "y", "hT", "vT", "D", "z",
-                           "delta_bias"};
-    for (int i = 0; i < 13; ++i)
+                           "delta_bias", "ckpt"};
+    for (int i = 0; i < 14; ++i)
         if (ptrs[i] && !aligned16(ptrs[i]))
             return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
-    int64_t d_bytes;
-    if (!mul_ok(D, 4, &d_bytes)) return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
 
     const Range rx = rng("x", x, seq_bytes), rd = rng("delta", delta, seq_bytes),
                 rA = rng("A", A, a_bytes), rB = rng("B", B, bc_bytes), rC = rng("C", C, bc_bytes),
                 rh0 = rng("h0", h0, st_bytes), rv0 = rng("v0", v0, st_bytes),
                 ry = rng("y", y, seq_bytes), rhT = rng("hT", hT, st_bytes),
                 rvT = rng("vT", vT, st_bytes), rD = rng("D", Dskip, d_bytes),
-                rz = rng("z", z, seq_bytes), rbias = rng("delta_bias", delta_bias, d_bytes);
+                rz = rng("z", z, seq_bytes), rbias = rng("delta_bias", delta_bias, d_bytes),
+                rck = rng("ckpt", ckpt, zs.ck_bytes);
     const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0, &rv0, &rD, &rz, &rbias};
-    for (const Range* in : inputs)
+    for (const Range* in : inputs) {
         if (overlap(ry, *in)) return fail(MM_ERR_ALIAS, "y overlaps %s", in->name);
+        if (overlap(rck, *in)) return fail(MM_ERR_ALIAS, "ckpt overlaps %s", in->name);
+    }
+    for (const Range* out : {&ry, &rhT, &rvT})
+        if (overlap(rck, *out)) return fail(MM_ERR_ALIAS, "ckpt overlaps %s", out->name);
     for (const Range* out : {&rhT, &rvT}) {
         for (const Range* in : inputs) {
             const bool same_state = (out == &rhT && in == &rh0) || (out == &rvT && in == &rv0);
@@ -194,11 +222,67 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.vec_ok = ((L * esize) % 16) == 0;
     a.Dskip = Dskip; a.z = z; a.dbias = delta_bias; a.softplus = delta_softplus ? 1 : 0;
     a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
+    a.ckpt = ckpt;
     const mmscan::ScanTileChoice t =
         mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load(),
                                  g_forced_ts.load());
     return from_cuda(mmscan::launch_scan_fwd(a, t, dims->io, static_cast<cudaStream_t>(stream)),
                      "mm_scan_fwd launch");
+}
+
+mm_status mm_scan_ckpt_size(const mm_scan_dims* dims, size_t* bytes) {
+    if (!dims || !bytes) return fail(MM_ERR_NULL, "dims and bytes are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, 0.0f, 1.0f, &zs)) return st;
+    *bytes = static_cast<size_t>(zs.ck_bytes);
+    return ok();
+}
+
+mm_status mm_scan_bwd(const void* x, const void* delta, const float* A, const void* B, const void* C,
+                      const float* h0, const float* v0, float beta, float alpha, const float* ckpt,
+                      const void* dy, const float* dhT, const float* dvT, void* dx, void* ddelta,
+                      float* dA, float* dB, float* dC, float* dh0, float* dv0,
+                      const mm_scan_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !dy || !dx || !ddelta || !dA || !dB || !dC)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C, dy, dx, ddelta, dA, dB and dC are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
+    const int64_t L = dims->seqlen;
+    if (!ckpt && L > MM_SCAN_CHUNK)
+        return fail(MM_ERR_NULL, "ckpt is required when seqlen > %d", MM_SCAN_CHUNK);
+    const void* ptrs[] = {x, delta, A, B, C, h0, v0, ckpt, dy, dhT, dvT, dx, ddelta, dA, dB, dC, dh0, dv0};
+    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "ckpt", "dy", "dhT", "dvT",
+                           "dx", "ddelta", "dA", "dB", "dC", "dh0", "dv0"};
+    for (int i = 0; i < 18; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    const Range in_r[] = {rng("x", x, zs.seq_bytes), rng("delta", delta, zs.seq_bytes),
+                          rng("A", A, zs.a_bytes), rng("B", B, zs.bc_bytes), rng("C", C, zs.bc_bytes),
+                          rng("h0", h0, zs.st_bytes), rng("v0", v0, zs.st_bytes),
+                          rng("ckpt", ckpt, zs.ck_bytes), rng("dy", dy, zs.seq_bytes),
+                          rng("dhT", dhT, zs.st_bytes), rng("dvT", dvT, zs.st_bytes)};
+    const Range out_r[] = {rng("dx", dx, zs.seq_bytes), rng("ddelta", ddelta, zs.seq_bytes),
+                           rng("dA", dA, zs.a_bytes), rng("dB", dB, zs.bcf_bytes),
+                           rng("dC", dC, zs.bcf_bytes), rng("dh0", dh0, zs.st_bytes),
+                           rng("dv0", dv0, zs.st_bytes)};
+    for (const Range& o : out_r) {
+        for (const Range& in : in_r)
+            if (overlap(o, in)) return fail(MM_ERR_ALIAS, "%s overlaps %s", o.name, in.name);
+        for (const Range& o2 : out_r)
+            if (&o2 != &o && overlap(o, o2)) return fail(MM_ERR_ALIAS, "%s overlaps %s", o.name, o2.name);
+    }
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+
+    mmscan::ScanBwdArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.h0 = h0; a.v0 = v0; a.ckpt = ckpt;
+    a.dout = dy; a.dhT = dhT; a.dvT = dvT;
+    a.dx = dx; a.ddelta = ddelta; a.dA = dA; a.dB = dB; a.dC = dC; a.dh0 = dh0; a.dv0 = dv0;
+    a.batch = dims->batch; a.seqlen = L; a.dim = dims->dim; a.dstate = (int)dims->dstate;
+    a.beta = beta; a.alpha = alpha;
+    a.vec_ok = ((L * zs.esize) % 16) == 0;
+    return from_cuda(mmscan::launch_scan_bwd(a, dims->io, static_cast<cudaStream_t>(stream)),
+                     "mm_scan_bwd launch");
 }
 
 mm_status mm_ssd_workspace_size(const mm_ssd_dims* dims, size_t* bytes) {

@@ -297,3 +297,95 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 }
 
 }  // namespace mmscan
+
+namespace mmscan {
+
+// ------------------------------------------------- scan helpers -----
+// Store `cnt` consecutive steps of one output row.
+template <typename IO>
+__device__ __forceinline__ void store_steps(IO* dst, const float* v, int cnt, bool vec) {
+    if constexpr (sizeof(IO) == 4) {
+        if (vec && cnt == 2) {
+            *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+            return;
+        }
+        if (vec && cnt == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+            return;
+        }
+    } else {
+        if (vec && cnt == 2) {
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v[0], v[1]);
+            return;
+        }
+        if (vec && cnt == 4) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+            return;
+        }
+    }
+}
+
+template <typename IO, int PER>
+__device__ __forceinline__ void store_steps_n(IO* dst, const float (&v)[PER], int cnt, bool vec) {
+    if (vec && cnt == PER && (PER == 2 || PER == 4)) {
+        store_steps<IO>(dst, v, PER, true);
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        if (i < cnt) store1(dst + i, v[i]);
+}
+
+// Sum, over the G consecutive lanes of a group, of K per-lane partials: a
+// butterfly that halves the values each lane carries at every stage (the lane
+// whose bit m is set keeps the upper half), so that group lane g ends with
+// the sums of entries [g K/G, (g+1) K/G) after log2 G exchanges of K/2, K/4,
+// ... values.  The exchanges stay in registers: no shared-memory traffic.
+template <int G, int K>
+__device__ __forceinline__ void butterfly_sum(const float (&v)[K], float (&out)[K / G], int g) {
+    static_assert((G & (G - 1)) == 0 && K % G == 0, "power-of-two group dividing K");
+    float cur[K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) cur[i] = v[i];
+#pragma unroll
+    for (int m = G / 2, n = K; m >= 1; m >>= 1, n >>= 1) {
+        const bool upper = (g & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float keep = upper ? cur[n / 2 + i] : cur[i];
+            const float send = upper ? cur[i] : cur[n / 2 + i];
+            cur[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < K / G; ++e) out[e] = cur[e];
+}
+
+__device__ __forceinline__ float2 shfl_up_f2(float2 v, int delta) {
+    return f2(__shfl_up_sync(0xffffffffu, v.x, delta), __shfl_up_sync(0xffffffffu, v.y, delta));
+}
+__device__ __forceinline__ float2 shfl_down_f2(float2 v, int delta) {
+    return f2(__shfl_down_sync(0xffffffffu, v.x, delta), __shfl_down_sync(0xffffffffu, v.y, delta));
+}
+
+// softplus(v) = ln(1 + e^v) = max(v, 0) + ln(1 + u) with u = e^-|v| in (0, 1].
+// ln(1 + u) = 2 atanh(s) for s = u / (2 + u) in (0, 1/3], summed as the odd
+// series s (1 + s^2/3 + s^4/5 + ... + s^14/15): every term is positive (no
+// cancellation) and the first one left out is below 2e-9 of the sum, so the
+// error is that of fp32 rounding and of the two MUFU operations.
+__device__ __forceinline__ float softplus_f32(float v) {
+    const float u = ex2_approx(-fabsf(v) * kLog2e);
+    const float s = __fdividef(u, 2.0f + u);
+    const float q = s * s;
+    float p = 1.0f / 15.0f;
+    p = fmaf(p, q, 1.0f / 13.0f);
+    p = fmaf(p, q, 1.0f / 11.0f);
+    p = fmaf(p, q, 1.0f / 9.0f);
+    p = fmaf(p, q, 1.0f / 7.0f);
+    p = fmaf(p, q, 1.0f / 5.0f);
+    p = fmaf(p, q, 1.0f / 3.0f);
+    p = fmaf(p, q, 1.0f);
+    return fmaxf(v, 0.0f) + 2.0f * s * p;
+}
+
+}  // namespace mmscan

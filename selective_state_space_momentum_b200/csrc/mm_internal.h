@@ -31,6 +31,34 @@ struct ScanArgs {
     const float* dbias;    // (dim) or null
     int softplus;          // delta' = softplus(delta + dbias)
     int ext;               // any of the four is present
+    float* ckpt;           // (batch, dim, ceil(L / 64), 2, dstate): (h, v) after each chunk, or null
+};
+
+// Arguments of one backward launch (device pointers; sizes as in mm_scan_dims).
+struct ScanBwdArgs {
+    const void* x;
+    const void* delta;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* h0;
+    const float* v0;
+    const float* ckpt;     // the forward's (h, v) after every 64-step chunk
+    const void* dout;      // gradient reaching y (io dtype)
+    const float* dhT;      // gradients reaching hT, vT, or null
+    const float* dvT;
+    void* dx;              // io dtype
+    void* ddelta;          // io dtype
+    float* dA;             // (dim, dstate), summed over the batch
+    float* dB;             // (batch, dstate, L), summed over dim
+    float* dC;
+    float* dh0;            // (batch, dim, dstate) or null
+    float* dv0;
+    int64_t batch, seqlen, dim;
+    int dstate;
+    int tiles_per_batch;   // filled by the launcher
+    float beta, alpha;
+    int vec_ok;            // rows of L elements are whole 16-byte pieces
 };
 
 struct ScanTileChoice {
@@ -44,8 +72,10 @@ bool scan_tile_supported(int spt, int warps, int time_lanes);
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
                                 int forced_spt, int forced_warps, int forced_ts);
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s);
+cudaError_t launch_scan_bwd(const ScanBwdArgs& a, int io, cudaStream_t s);
 // Read (and reset) the device error word of the scan / SSD kernels.
 unsigned int scan_read_and_clear_device_error();
+unsigned int scan_bwd_read_and_clear_device_error();
 unsigned int ssd_read_and_clear_device_error();
 
 // Arguments of one SSD call.

@@ -1,0 +1,547 @@
+// scan_bwd.cu -- sm_100a kernel for the backward of the Momentum Mamba selective scan.
+//
+// What it computes: the gradients of the forward in scan_fwd.cu ("Momentum
+// Mamba: Enhanced State Space Models with Momentum", "Gradient Flow" and
+// "Backward Pass: Reconstructed Forward + Reverse Scans").  The printed
+// recursions use one symbol for both state gradients and drop a term, so
+// they are derived from the recurrence: per (b, d, n), with G_t = dL/dh_t
+// and P_t = dL/dv_t (total derivatives),
+//     G_t = dy_t C_t[n] + a_{t+1} G_{t+1},    P_t = G_t + beta P_{t+1}
+// starting from dhT, dvT after the last step, and
+//     dx_t     = alpha delta_t sum_n B_t[n] P_t[n]
+//     ddelta_t = alpha x_t sum_n B_t[n] P_t[n] + sum_n A[d,n] a_t h_{t-1}[n] G_t[n]
+//     dA[d,n]  = sum_{b,t} delta_t a_t h_{t-1}[n] G_t[n]
+//     dB_t[n]  = sum_d alpha delta_t x_t P_t[n],     dC_t[n] = sum_d dy_t h_t[n]
+//     dh0 = a_0 G_0,    dv0 = beta P_0                 (a_t = exp(delta_t A[d,n]))
+//
+// Design (B200-first; the page's reverse block scans are prior art only):
+//  * Work split as in the forward: a CTA owns CH channels of one batch row,
+//    G = NP / 2 lanes per channel, two states per lane.  The CTA walks the
+//    chunks of 64 steps from the last to the first and carries (G, P) in
+//    registers, so the reverse recursion runs in time order and needs no
+//    carry recombination.
+//  * States.  The forward saved (h, v) after every chunk; a chunk starts from
+//    the previous chunk's checkpoint (h0, v0 for the first).  A first pass runs
+//    the chunk forward and keeps the state at the start of each group of 8
+//    steps in registers; the reverse pass rebuilds each group's states and
+//    exponentials from its start (a second forward over 8 steps) and walks
+//    them backwards.  The rebuilt states are those of the forward kernel bit
+//    for bit (same operations in the same order).  Nothing of size (L, D, N)
+//    is stored.
+//  * Reductions.  The sums over a channel's states (for dx, ddelta) use the
+//    forward's register butterfly.  dB and dC sum over channels: a butterfly
+//    across the channels of a warp, shared-memory atomics across the warps,
+//    then one vector atomic add per (4 steps, state) into global memory per
+//    chunk.  dA collects in registers over the whole sequence and is added
+//    once per lane.
+//  * Staging: x, delta, dy, B and C tiles by TMA (128-byte swizzle, no
+//    multicast), two chunks in flight; B and C transposed to [t][n] fp32 with
+//    alpha folded into B, as in the forward.
+#include <cuda.h>
+
+#include <atomic>
+
+#include "mm_common.cuh"
+#include "mm_internal.h"
+#include "mm_tma_host.h"
+
+namespace mmscan {
+
+// Device error word of this file's kernel (bounded waits that gave up).
+static __device__ unsigned int g_bwd_dev_err = 0;
+
+template <typename IO, int NP, int WARPS>
+struct BwdTile {
+    static constexpr int SPT = 2;                // states per lane
+    static constexpr int G = NP / SPT;           // lanes per channel
+    static constexpr int CPW = 32 / G;           // channels per warp
+    static constexpr int CH = WARPS * CPW;       // channels per CTA
+    static constexpr int NT = WARPS * 32;
+    static constexpr int EB = IOTraits<IO>::kBytes;
+    static constexpr int BOX_T = 128 / EB;       // steps in one 128-byte swizzled row
+    static constexpr int T = 64;                 // steps per chunk (the checkpoint interval)
+    static constexpr int NBOX = T / BOX_T;
+    static constexpr int STAGES = 2;
+    static constexpr int NPT = NP < 8 ? 8 : NP;  // B/C rows per box (whole swizzle atoms)
+    static constexpr int XBOX = CH * 128;
+    static constexpr int BBOX = NPT * 128;
+    static constexpr int OFF_X = 0;
+    static constexpr int OFF_D = NBOX * XBOX;
+    static constexpr int OFF_Y = 2 * NBOX * XBOX;     // dy, the gradient reaching y
+    static constexpr int OFF_B = 3 * NBOX * XBOX;
+    static constexpr int OFF_C = OFF_B + NBOX * BBOX;
+    static constexpr int STAGE_BYTES = OFF_C + NBOX * BBOX;
+    static constexpr int BP = NP + 4;            // row pitch (floats) of transposed B/C
+    static constexpr int BT_BYTES = T * BP * 4;
+    static constexpr int R = 8;                  // steps per group
+    static constexpr int NG = T / R;
+    static constexpr int PER = R / G;            // steps of a group whose sums a lane owns
+    static constexpr int RP = 2 * NP;            // dB and dC partials per step
+    static constexpr int OFF_BT = STAGES * STAGE_BYTES;   // B^T, then C^T
+    static constexpr int OFF_RED = OFF_BT + 2 * BT_BYTES;
+    static constexpr int RED_BYTES = T * RP * 4;
+    static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
+    static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
+    // 12 resident warps per SM (<= 168 registers a thread)
+    static constexpr int MIN_CTAS = 12 / WARPS > 0 ? 12 / WARPS : 1;
+
+    static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "lanes per channel");
+    static_assert(R % G == 0 && BOX_T % R == 0 && T % BOX_T == 0, "step grouping");
+    static_assert(CH % 8 == 0, "x tiles must be whole 1024-byte swizzle atoms");
+    static_assert(STAGE_BYTES % 1024 == 0 && OFF_BT % 16 == 0 && OFF_RED % 16 == 0, "alignment");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <typename IO, int NP, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, BwdTile<IO, NP, WARPS>::MIN_CTAS)
+scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
+                const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_B,
+                const __grid_constant__ CUtensorMap tm_C, const ScanBwdArgs p) {
+    using TL = BwdTile<IO, NP, WARPS>;
+    constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
+    constexpr int ST = TL::STAGES, EB = TL::EB, BP = TL::BP, NG = TL::NG, PER = TL::PER;
+    constexpr int RP = TL::RP;
+
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (base - raw_addr);
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int g = lane % G;
+    const int c = warp * CPW + lane / G;             // channel within the CTA
+    const int n0 = g * 2;                            // first of the lane's two states
+    const int64_t b = blockIdx.x / p.tiles_per_batch;
+    const int64_t d0 = (int64_t)(blockIdx.x % p.tiles_per_batch) * CH;
+    const int64_t d = d0 + c;
+    const bool active = d < p.dim;
+    const int64_t L = p.seqlen;
+    const int N = p.dstate;
+    const int64_t nchunks = (L + T - 1) / T;
+    const bool use_tma = p.vec_ok != 0;
+    const uint32_t bar0 = base + TL::OFF_BAR;
+    float* red = reinterpret_cast<float*>(smem + TL::OFF_RED);
+    float* Bt = reinterpret_cast<float*>(smem + TL::OFF_BT);
+    float* Ct = Bt + T * BP;
+
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, use_tma ? 1u : (uint32_t)NT);
+        fence_barrier_init();
+    }
+    for (int i = tid; i < T * RP; i += NT) red[i] = 0.0f;
+    __syncthreads();
+
+    // ---- per-lane constants and carries -------------------------------------
+    float A2v[2], Anv[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int n = n0 + e;
+        Anv[e] = (active && n < N) ? p.A[d * N + n] : 0.0f;
+        A2v[e] = Anv[e] * kLog2e;
+    }
+    const float2 A2 = f2(A2v[0], A2v[1]);        // exponent scale (log2 e A)
+    const float2 An = f2(Anv[0], Anv[1]);        // A itself, for ddelta
+    const float2 beta2 = f2(p.beta, p.beta);
+    const float alpha = p.alpha;
+    const int64_t srow = (b * p.dim + (active ? d : 0)) * N;   // this channel's state row
+    auto load_pair = [&](const float* src) {
+        float v[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            if (src && active && n0 + e < N) v[e] = src[n0 + e];
+        return f2(v[0], v[1]);
+    };
+    float2 cg = load_pair(p.dhT ? p.dhT + srow : nullptr);   // a_{t+1} G_{t+1}
+    float2 cp = load_pair(p.dvT ? p.dvT + srow : nullptr);   // beta P_{t+1}
+    float2 dA2 = f2(0.0f, 0.0f);
+
+    // ---- staging of one chunk into a stage buffer ----------------------------
+    auto issue = [&](int64_t k, int s) {
+        const int64_t t0 = k * T;
+        const uint32_t sb = base + s * TL::STAGE_BYTES;
+        const uint32_t bar = bar0 + 8 * s;
+        if (use_tma) {
+            if (tid == 0) {
+                mbar_expect_tx(bar, TL::STAGE_BYTES);
+#pragma unroll
+                for (int bx = 0; bx < TL::NBOX; ++bx) {
+                    const int tc = (int)(t0 + bx * TL::BOX_T);
+                    tma_load_3d(sb + TL::OFF_X + bx * TL::XBOX, &tm_x, bar, tc, (int)d0, (int)b);
+                    tma_load_3d(sb + TL::OFF_D + bx * TL::XBOX, &tm_d, bar, tc, (int)d0, (int)b);
+                    tma_load_3d(sb + TL::OFF_Y + bx * TL::XBOX, &tm_y, bar, tc, (int)d0, (int)b);
+                    tma_load_3d(sb + TL::OFF_B + bx * TL::BBOX, &tm_B, bar, tc, 0, (int)b);
+                    tma_load_3d(sb + TL::OFF_C + bx * TL::BBOX, &tm_C, bar, tc, 0, (int)b);
+                }
+            }
+            return;
+        }
+        // Element-wise fill of the same swizzled tiles (rows not 16-byte multiples).
+        const IO* srcs[3] = {static_cast<const IO*>(p.x), static_cast<const IO*>(p.delta),
+                             static_cast<const IO*>(p.dout)};
+        const IO* Bg = static_cast<const IO*>(p.B);
+        const IO* Cg = static_cast<const IO*>(p.C);
+        constexpr int ROWS = 3 * CH + 2 * TL::NPT;
+        for (int i = tid; i < ROWS * T; i += NT) {
+            const int r = i / T;
+            const int tau = i - r * T;
+            const int bx = tau / TL::BOX_T;
+            const int col = tau - bx * TL::BOX_T;
+            const int64_t t = t0 + tau;
+            const IO* src = nullptr;
+            uint32_t off;
+            if (r < 3 * CH) {
+                const int which = r / CH;
+                const int cc = r - which * CH;
+                off = which * TL::NBOX * TL::XBOX + bx * TL::XBOX + sw128(cc, col * EB);
+                if (d0 + cc < p.dim && t < L) src = srcs[which] + ((b * p.dim + d0 + cc) * L + t);
+            } else {
+                const int rr = r - 3 * CH;
+                const int n = rr < TL::NPT ? rr : rr - TL::NPT;
+                off = (rr < TL::NPT ? TL::OFF_B : TL::OFF_C) + bx * TL::BBOX + sw128(n, col * EB);
+                if (n < N && t < L) src = (rr < TL::NPT ? Bg : Cg) + ((b * N + n) * L + t);
+            }
+            if constexpr (EB == 4) {
+                cp_async_4(smem + s * TL::STAGE_BYTES + off, src ? src : srcs[0], src ? 4 : 0);
+            } else {
+                *reinterpret_cast<IO*>(smem + s * TL::STAGE_BYTES + off) = src ? *src : IO(0.0f);
+            }
+        }
+        if constexpr (EB == 4) cp_async_mbar_arrive(bar);
+        else mbar_arrive(bar);
+    };
+
+    // The i-th chunk processed (chunk nchunks - 1 - i) goes to stage i % ST.
+#pragma unroll
+    for (int i = 0; i < ST - 1; ++i)
+        if (i < nchunks) issue(nchunks - 1 - i, i);
+
+    IO* dxrow = static_cast<IO*>(p.dx) + (b * p.dim + (active ? d : 0)) * L;
+    IO* ddrow = static_cast<IO*>(p.ddelta) + (b * p.dim + (active ? d : 0)) * L;
+    const bool vec_out = use_tma;
+    const bool vec_red = (L % 4) == 0;
+
+    for (int64_t i = 0; i < nchunks; ++i) {
+        const int64_t k = nchunks - 1 - i;
+        const int s = (int)(i % ST);
+        const int64_t t0 = k * T;
+        const int nval = (int)((L - t0) < T ? (L - t0) : T);
+        // the chunk's start state: the previous chunk's checkpoint, or (h0, v0)
+        const float* hsrc = k > 0 ? p.ckpt + ((b * p.dim + (active ? d : 0)) * nchunks + (k - 1)) * 2 * N
+                                  : (p.h0 ? p.h0 + srow : nullptr);
+        const float* vsrc = k > 0 ? hsrc + N : (p.v0 ? p.v0 + srow : nullptr);
+        const float2 hst = load_pair(hsrc);
+        const float2 vst = load_pair(vsrc);
+        if (!mbar_wait(bar0 + 8 * s, (uint32_t)((i / ST) & 1), &g_bwd_dev_err)) return;
+        const unsigned char* sbuf = smem + s * TL::STAGE_BYTES;
+
+        // ---- transpose B, C to [t][n] fp32 in 4x4 blocks (alpha into B) ----
+        {
+            constexpr int NB4 = NP / 4 > 0 ? NP / 4 : 1;
+            constexpr int ITEMS = NB4 * (T / 4);
+            for (int it = tid; it < 2 * ITEMS; it += NT) {
+                const int which = it / ITEMS;
+                const int rem = it - which * ITEMS;
+                const int nb = (rem % NB4) * 4;
+                const int t4 = (rem / NB4) * 4;
+                const int bx = t4 / TL::BOX_T;
+                const int col = t4 - bx * TL::BOX_T;
+                const unsigned char* tile = sbuf + (which ? TL::OFF_C : TL::OFF_B) + bx * TL::BBOX;
+                float m[4][4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (nb + r < NP) {
+                        const float4 q = load4(reinterpret_cast<const IO*>(tile + sw128(nb + r, col * EB)));
+                        m[r][0] = q.x; m[r][1] = q.y; m[r][2] = q.z; m[r][3] = q.w;
+                    } else {
+                        m[r][0] = m[r][1] = m[r][2] = m[r][3] = 0.0f;
+                    }
+                }
+                const float sc = which ? 1.0f : alpha;
+                float* dst = (which ? Ct : Bt) + t4 * BP + nb;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if constexpr (NP >= 4) {
+                        *reinterpret_cast<float4*>(dst + j * BP) =
+                            make_float4(m[0][j] * sc, m[1][j] * sc, m[2][j] * sc, m[3][j] * sc);
+                    } else {
+                        dst[j * BP] = m[0][j] * sc;
+                        dst[j * BP + 1] = m[1][j] * sc;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        // Every thread is past the previous chunk: its stage is free.
+        if (i + ST - 1 < nchunks) issue(nchunks - 1 - (i + ST - 1), (int)((i + ST - 1) % ST));
+
+        // delta, x (and dy) of the R steps of group gi, this lane's channel
+        auto load_group = [&](int gi, float (&dl)[R], float (&xl)[R]) {
+            const int tau0 = gi * R;
+            const int bx = tau0 / TL::BOX_T;
+            const int col = tau0 - bx * TL::BOX_T;
+            const unsigned char* xt = sbuf + TL::OFF_X + bx * TL::XBOX;
+            const unsigned char* dt = sbuf + TL::OFF_D + bx * TL::XBOX;
+#pragma unroll
+            for (int j = 0; j < R; j += 4) {
+                const float4 dq = load4(reinterpret_cast<const IO*>(dt + sw128(c, (col + j) * EB)));
+                const float4 xq = load4(reinterpret_cast<const IO*>(xt + sw128(c, (col + j) * EB)));
+                dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
+                xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
+            }
+        };
+        auto load_dy = [&](int gi, float (&yl)[R]) {
+            const int tau0 = gi * R;
+            const int bx = tau0 / TL::BOX_T;
+            const int col = tau0 - bx * TL::BOX_T;
+            const unsigned char* yt = sbuf + TL::OFF_Y + bx * TL::XBOX;
+#pragma unroll
+            for (int j = 0; j < R; j += 4) {
+                const float4 q = load4(reinterpret_cast<const IO*>(yt + sw128(c, (col + j) * EB)));
+                yl[j] = q.x; yl[j + 1] = q.y; yl[j + 2] = q.z; yl[j + 3] = q.w;
+            }
+        };
+        // one forward step of the lane's two states (the forward kernel's operations)
+        auto fwd_step = [&](int tau, float dl, float u, float2& h, float2& v, float2& a) {
+            const float2 bq = *reinterpret_cast<const float2*>(Bt + tau * BP + n0);
+            const float2 r2 = __fmul2_rn(f2(dl, dl), A2);
+            a = f2(ex2_approx(r2.x), ex2_approx(r2.y));
+            const float2 w = __fmul2_rn(f2(u, u), bq);
+            v = __ffma2_rn(beta2, v, w);
+            h = __ffma2_rn(a, h, v);
+        };
+        // dB, dC partials of step tau: summed over the warp's channels by a
+        // butterfly, then over the warps by shared-memory atomics
+        auto chan_reduce = [&](int tau, float2 dBv, float2 dCv) {
+            const bool up1 = (lane & 16) != 0;
+            float k0 = up1 ? dCv.x : dBv.x, k1 = up1 ? dCv.y : dBv.y;
+            const float s0 = up1 ? dBv.x : dCv.x, s1 = up1 ? dBv.y : dCv.y;
+            k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+            k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+            const bool up2 = (lane & 8) != 0;
+            float kk = up2 ? k1 : k0;
+            const float ss = up2 ? k0 : k1;
+            kk += __shfl_xor_sync(0xffffffffu, ss, 8);
+#pragma unroll
+            for (int m = G; m < 8; m <<= 1) kk += __shfl_xor_sync(0xffffffffu, kk, m);
+            if ((lane & 7) < G) atomicAdd(red + tau * RP + (up1 ? NP : 0) + n0 + (up2 ? 1 : 0), kk);
+        };
+        // Group gi (first kmax steps valid) from its start state: rebuild the
+        // states and exponentials, then walk the steps backwards.
+        auto group_reverse = [&](int gi, int kmax, float2 h, float2 v) {
+            const int tau0 = gi * R;
+            float dl[R], xl[R], yl[R], u[R];
+            load_group(gi, dl, xl);
+            load_dy(gi, yl);
+#pragma unroll
+            for (int j = 0; j < R; ++j) u[j] = dl[j] * xl[j];
+            float2 ht[R], at[R];
+            const float2 hprev0 = h;
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                if (j < kmax) fwd_step(tau0 + j, dl[j], u[j], h, v, at[j]);
+                else at[j] = f2(1.0f, 1.0f);
+                ht[j] = h;
+            }
+            float sk[R], qk[R];
+#pragma unroll
+            for (int j = R - 1; j >= 0; --j) {
+                sk[j] = 0.0f;
+                qk[j] = 0.0f;
+                if (j < kmax) {
+                    const int tau = tau0 + j;
+                    const float2 bq = *reinterpret_cast<const float2*>(Bt + tau * BP + n0);
+                    const float2 cq = *reinterpret_cast<const float2*>(Ct + tau * BP + n0);
+                    const float2 Gt = __ffma2_rn(cq, f2(yl[j], yl[j]), cg);
+                    const float2 Pt = __fadd2_rn(Gt, cp);
+                    const float2 hp = j > 0 ? ht[j - 1] : hprev0;
+                    const float2 dt2 = __fmul2_rn(__fmul2_rn(at[j], hp), Gt);   // a_t h_{t-1} G_t
+                    const float2 s2 = __fmul2_rn(Pt, bq);                       // alpha B P
+                    const float2 q2 = __fmul2_rn(dt2, An);
+                    sk[j] = s2.x + s2.y;
+                    qk[j] = q2.x + q2.y;
+                    dA2 = __ffma2_rn(f2(dl[j], dl[j]), dt2, dA2);
+                    const float ua = u[j] * alpha;
+                    chan_reduce(tau, __fmul2_rn(Pt, f2(ua, ua)), __fmul2_rn(f2(yl[j], yl[j]), ht[j]));
+                    cg = __fmul2_rn(at[j], Gt);
+                    cp = __fmul2_rn(beta2, Pt);
+                }
+            }
+            // per-channel sums; lane g owns steps [g PER, (g + 1) PER) of the group
+            float so[PER], qo[PER];
+            butterfly_sum<G, R>(sk, so, g);
+            butterfly_sum<G, R>(qk, qo, g);
+            const int first = tau0 + g * PER;
+            const int cnt = nval - first < PER ? nval - first : PER;
+            float gx[PER], gd[PER];
+#pragma unroll
+            for (int e = 0; e < PER; ++e) {
+                const int st = first + e;
+                const int bxx = st / TL::BOX_T;
+                const int cc = st - bxx * TL::BOX_T;
+                const float de = load1(reinterpret_cast<const IO*>(sbuf + TL::OFF_D + bxx * TL::XBOX +
+                                                                    sw128(c, cc * EB)));
+                const float xe = load1(reinterpret_cast<const IO*>(sbuf + TL::OFF_X + bxx * TL::XBOX +
+                                                                    sw128(c, cc * EB)));
+                gx[e] = de * so[e];
+                gd[e] = __fmaf_rn(xe, so[e], qo[e]);
+            }
+            if (active && cnt > 0) {
+                store_steps_n<IO, PER>(dxrow + t0 + first, gx, cnt, vec_out);
+                store_steps_n<IO, PER>(ddrow + t0 + first, gd, cnt, vec_out);
+            }
+        };
+
+        if (nval == T) {
+            // pass 1: the chunk forward, keeping each group's start state
+            float2 hs[NG], vs[NG];
+            {
+                float2 h = hst, v = vst;
+#pragma unroll
+                for (int gi = 0; gi < NG; ++gi) {
+                    hs[gi] = h;
+                    vs[gi] = v;
+                    float dl[R], xl[R];
+                    load_group(gi, dl, xl);
+#pragma unroll
+                    for (int j = 0; j < R; ++j) {
+                        float2 a;
+                        fwd_step(gi * R + j, dl[j], dl[j] * xl[j], h, v, a);
+                    }
+                }
+            }
+            // pass 2: groups backwards
+#pragma unroll
+            for (int gi = NG - 1; gi >= 0; --gi) group_reverse(gi, R, hs[gi], vs[gi]);
+        } else {
+            // Ragged last chunk (processed first): each group's start state is
+            // rebuilt from the chunk's start.
+            const int ng = (nval + R - 1) / R;
+            for (int gi = ng - 1; gi >= 0; --gi) {
+                float2 h = hst, v = vst;
+                for (int gg = 0; gg < gi; ++gg) {
+                    float dl[R], xl[R];
+                    load_group(gg, dl, xl);
+#pragma unroll
+                    for (int j = 0; j < R; ++j) {
+                        float2 a;
+                        fwd_step(gg * R + j, dl[j], dl[j] * xl[j], h, v, a);
+                    }
+                }
+                const int kmax = nval - gi * R < R ? nval - gi * R : R;
+                group_reverse(gi, kmax, h, v);
+            }
+        }
+
+        // ---- dB, dC of the chunk into global memory ---------------------------
+        __syncthreads();
+        for (int it = tid; it < (T / 4) * RP; it += NT) {
+            const int slot = it % RP;
+            const int t4 = (it / RP) * 4;
+            float v4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                v4[e] = red[(t4 + e) * RP + slot];
+                red[(t4 + e) * RP + slot] = 0.0f;
+            }
+            const int which = slot / NP;
+            const int n = slot - which * NP;
+            if (n < N && t4 < nval) {
+                float* dst = (which ? p.dC : p.dB) + (b * N + n) * L + t0 + t4;
+                if (vec_red && t4 + 4 <= nval) {
+                    atomicAdd(reinterpret_cast<float4*>(dst), make_float4(v4[0], v4[1], v4[2], v4[3]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (t4 + e < nval) atomicAdd(dst + e, v4[e]);
+                }
+            }
+        }
+    }
+
+    // ---- gradients of the start state; dA ------------------------------------
+    if (active) {
+        const float gh[2] = {cg.x, cg.y}, gv[2] = {cp.x, cp.y}, ga[2] = {dA2.x, dA2.y};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int n = n0 + e;
+            if (n < N) {
+                if (p.dh0) p.dh0[srow + n] = gh[e];
+                if (p.dv0) p.dv0[srow + n] = gv[e];
+                atomicAdd(p.dA + d * N + n, ga[e]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------- launch -----
+namespace {
+
+template <typename IO, int NP, int WARPS>
+cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
+    using TL = BwdTile<IO, NP, WARPS>;
+    ScanBwdArgs a = a0;
+    a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
+    const int64_t grid = a.batch * a.tiles_per_batch;
+    if (grid > 0x7fffffffLL || a.dim > 0x7fffffffLL || a.batch > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    CUtensorMap mx, md, my, mB, mC;
+    memset(&mx, 0, sizeof(mx)); memset(&md, 0, sizeof(md)); memset(&my, 0, sizeof(my));
+    memset(&mB, 0, sizeof(mB)); memset(&mC, 0, sizeof(mC));
+    if (a.vec_ok) {
+        const bool bf = sizeof(IO) == 2;
+        const uint64_t L = (uint64_t)a.seqlen;
+        cudaError_t e;
+        if ((e = make_map_3d(&mx, a.x, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&md, a.delta, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&my, a.dout, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
+        if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
+    }
+    auto kern = scan_bwd_kernel<IO, NP, WARPS>;
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done.fetch_or(bit, std::memory_order_release);
+    }
+    kern<<<(unsigned)grid, TL::NT, TL::SMEM_BYTES, stream>>>(mx, md, my, mB, mC, a);
+    return cudaGetLastError();
+}
+
+template <typename IO>
+cudaError_t launch_bwd_io(const ScanBwdArgs& a, cudaStream_t s) {
+    const int64_t channels = a.batch * a.dim;
+    const int N = a.dstate;
+    if (N > 8) return channels >= 2048 ? launch_bwd_variant<IO, 16, 4>(a, s) : launch_bwd_variant<IO, 16, 2>(a, s);
+    if (N > 4) return launch_bwd_variant<IO, 8, 2>(a, s);
+    if (N > 2) return launch_bwd_variant<IO, 4, 2>(a, s);
+    return launch_bwd_variant<IO, 2, 2>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_scan_bwd(const ScanBwdArgs& a, int io, cudaStream_t s) {
+    // dA, dB and dC are sums that the kernel adds into: start them at zero.
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(a.dA, 0, (size_t)a.dim * a.dstate * 4, s)) != cudaSuccess) return e;
+    const size_t bc = (size_t)a.batch * a.dstate * a.seqlen * 4;
+    if ((e = cudaMemsetAsync(a.dB, 0, bc, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.dC, 0, bc, s)) != cudaSuccess) return e;
+    if (io == 0) return launch_bwd_io<float>(a, s);
+    return launch_bwd_io<bf16>(a, s);
+}
+
+unsigned int scan_bwd_read_and_clear_device_error() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_bwd_dev_err, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_bwd_dev_err, &z, sizeof(z));
+    return v;
+}
+
+}  // namespace mmscan

@@ -26,9 +26,11 @@
 //    exp(delta A) (A pre-scaled by log2 e), and packed f32x2 multiply / FMA
 //    for the write, the velocity, the hidden state and the read-out -- two
 //    states per instruction.  Nothing of size (L, D, N) is ever stored.
-//  * Read-out.  The G lanes of a channel add their partial C_t . h_t through
-//    a small per-warp buffer (no CTA barrier) and store y directly: the G
-//    lanes write G consecutive steps of their channel.
+//  * Read-out.  The G lanes of a channel add their partial C_t . h_t by a
+//    register butterfly (shuffles, no shared memory) and store y directly:
+//    the G lanes write consecutive steps of their channel.
+//  * Checkpoints (optional).  (h, v) after every chunk of 64 steps go to a
+//    (batch, dim, chunks, 2, N) buffer that the backward restarts from.
 //  * Final state.  (h, v) after the last step go to hT, vT.  The per-state
 //    operation sequence does not depend on where the sequence is cut into
 //    calls, so split calls reproduce hT, vT bit for bit.
@@ -39,6 +41,7 @@
 
 #include "mm_common.cuh"
 #include "mm_internal.h"
+#include "mm_tma_host.h"
 
 namespace mmscan {
 
@@ -94,93 +97,6 @@ struct ScanTile {
                   "time split: fp32 I/O, two groups per lane, 4 or 8 lanes per channel");
     static_assert(!EXT || TS == 1, "the selective_scan_fn extras run without the time split");
 };
-
-// Store `cnt` consecutive steps of one output row.
-template <typename IO>
-__device__ __forceinline__ void store_steps(IO* dst, const float* v, int cnt, bool vec) {
-    if constexpr (sizeof(IO) == 4) {
-        if (vec && cnt == 2) {
-            *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
-            return;
-        }
-        if (vec && cnt == 4) {
-            *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-            return;
-        }
-    } else {
-        if (vec && cnt == 2) {
-            *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v[0], v[1]);
-            return;
-        }
-        if (vec && cnt == 4) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
-            return;
-        }
-    }
-}
-
-template <typename IO, int PER>
-__device__ __forceinline__ void store_steps_n(IO* dst, const float (&v)[PER], int cnt, bool vec) {
-    if (vec && cnt == PER && (PER == 2 || PER == 4)) {
-        store_steps<IO>(dst, v, PER, true);
-        return;
-    }
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-        if (i < cnt) store1(dst + i, v[i]);
-}
-
-// Sum, over the G consecutive lanes of a group, of K per-lane partials: a
-// butterfly that halves the values each lane carries at every stage (the lane
-// whose bit m is set keeps the upper half), so that group lane g ends with
-// the sums of entries [g K/G, (g+1) K/G) after log2 G exchanges of K/2, K/4,
-// ... values.  The exchanges stay in registers: no shared-memory traffic.
-template <int G, int K>
-__device__ __forceinline__ void butterfly_sum(const float (&v)[K], float (&out)[K / G], int g) {
-    static_assert((G & (G - 1)) == 0 && K % G == 0, "power-of-two group dividing K");
-    float cur[K];
-#pragma unroll
-    for (int i = 0; i < K; ++i) cur[i] = v[i];
-#pragma unroll
-    for (int m = G / 2, n = K; m >= 1; m >>= 1, n >>= 1) {
-        const bool upper = (g & m) != 0;
-#pragma unroll
-        for (int i = 0; i < n / 2; ++i) {
-            const float keep = upper ? cur[n / 2 + i] : cur[i];
-            const float send = upper ? cur[i] : cur[n / 2 + i];
-            cur[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < K / G; ++e) out[e] = cur[e];
-}
-
-__device__ __forceinline__ float2 shfl_up_f2(float2 v, int delta) {
-    return f2(__shfl_up_sync(0xffffffffu, v.x, delta), __shfl_up_sync(0xffffffffu, v.y, delta));
-}
-__device__ __forceinline__ float2 shfl_down_f2(float2 v, int delta) {
-    return f2(__shfl_down_sync(0xffffffffu, v.x, delta), __shfl_down_sync(0xffffffffu, v.y, delta));
-}
-
-// softplus(v) = ln(1 + e^v) = max(v, 0) + ln(1 + u) with u = e^-|v| in (0, 1].
-// ln(1 + u) = 2 atanh(s) for s = u / (2 + u) in (0, 1/3], summed as the odd
-// series s (1 + s^2/3 + s^4/5 + ... + s^14/15): every term is positive (no
-// cancellation) and the first one left out is below 2e-9 of the sum, so the
-// error is that of fp32 rounding and of the two MUFU operations.
-__device__ __forceinline__ float softplus_f32(float v) {
-    const float u = ex2_approx(-fabsf(v) * kLog2e);
-    const float s = __fdividef(u, 2.0f + u);
-    const float q = s * s;
-    float p = 1.0f / 15.0f;
-    p = fmaf(p, q, 1.0f / 13.0f);
-    p = fmaf(p, q, 1.0f / 11.0f);
-    p = fmaf(p, q, 1.0f / 9.0f);
-    p = fmaf(p, q, 1.0f / 7.0f);
-    p = fmaf(p, q, 1.0f / 5.0f);
-    p = fmaf(p, q, 1.0f / 3.0f);
-    p = fmaf(p, q, 1.0f);
-    return fmaxf(v, 0.0f) + 2.0f * s * p;
-}
 
 template <typename IO, int NP, int SPT, int WARPS, int TS, bool EXT>
 __global__ void __launch_bounds__(WARPS * 32, ScanTile<IO, NP, SPT, WARPS, TS, EXT>::MIN_CTAS)
@@ -648,6 +564,21 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 ragged_chunk();
             }
         }
+        // ---- checkpoint: (h, v) after the chunk's last step, for the backward ----
+        if (p.ckpt && writer) {
+            float* cp = p.ckpt + ((b * p.dim + d) * nchunks + k) * 2 * N;
+#pragma unroll
+            for (int q = 0; q < NPAIR; ++q) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int n = g * SPT + 2 * q + e;
+                    if (n < N) {
+                        cp[n] = e ? hh[q].y : hh[q].x;
+                        cp[N + n] = e ? vv[q].y : vv[q].x;
+                    }
+                }
+            }
+        }
     }
 
     // ---- final states -------------------------------------------------------
@@ -669,41 +600,6 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
 // ------------------------------------------------------------- launch -----
 namespace {
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
-
-// 3-D tiled map over a (d2, d1, d0 = innermost) tensor, 128-byte swizzle.
-cudaError_t make_map_3d(CUtensorMap* m, const void* base, bool bf16_elems, uint64_t d0n, uint64_t d1n,
-                        uint64_t d2n, uint32_t box0, uint32_t box1) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    const uint64_t eb = bf16_elems ? 2 : 4;
-    const cuuint64_t dims[3] = {d0n, d1n, d2n};
-    const cuuint64_t strides[2] = {d0n * eb, d0n * d1n * eb};
-    const cuuint32_t box[3] = {box0, box1, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(m, bf16_elems ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
-                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
 
 template <typename IO, int NP, int SPT, int WARPS, int TS = 1, bool EXT = false>
 cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
@@ -835,8 +731,14 @@ ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int 
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s) {
-    if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, t.ts, s);
-    return launch_io<bf16>(a, t.np, t.spt, t.warps, t.ts, s);
+    // Checkpoints are laid out per 64-step chunk: the time split (32-step chunks) is not used.
+    const int ts = a.ckpt ? 1 : t.ts;
+    if (ts != t.ts && !scan_tile_supported(t.spt, t.warps, 1)) {
+        if (io == 0) return launch_io<float>(a, t.np, 2, 4, 1, s);
+        return launch_io<bf16>(a, t.np, 2, 4, 1, s);
+    }
+    if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, ts, s);
+    return launch_io<bf16>(a, t.np, t.spt, t.warps, ts, s);
 }
 
 unsigned int scan_read_and_clear_device_error() {

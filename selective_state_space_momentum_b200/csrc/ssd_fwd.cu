@@ -48,6 +48,7 @@
 
 #include "mm_common.cuh"
 #include "mm_internal.h"
+#include "mm_tma_host.h"
 
 namespace mmscan {
 
@@ -603,24 +604,6 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
 // ------------------------------------------------------------- launch -----
 namespace {
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
 
 // 4-D bf16 map (d0 innermost), box (box0, 1, 128, 1): 64 columns with the
 // 128-byte swizzle for the loads, 32 columns with the 64-byte swizzle for the y stores.

@@ -112,17 +112,56 @@ def test_gated_checks_its_extras(lib, monkeypatch):
     dims = D(L=64, dim=8)
     def call(**over):
         a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), D=None, z=None,
-                 bias=None, sp=0, h0=None, v0=None, y=_fake(5), hT=None, vT=None)
+                 bias=None, sp=0, h0=None, v0=None, y=_fake(5), hT=None, vT=None, ckpt=None)
         a.update(over)
         return lib.mm_scan_fwd_gated(a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"],
                                      a["bias"], a["sp"], a["h0"], a["v0"], 0.9, 1.0, a["y"], a["hT"],
-                                     a["vT"], ctypes.byref(dims), None)
+                                     a["vT"], a["ckpt"], ctypes.byref(dims), None)
     assert call(z=ctypes.c_void_p(A16 * 7 + 4)) == 5              # misaligned gate
     assert "z is not 16-byte aligned" in mm.mm_last_error()
     assert call(z=_fake(5)) == 9                                  # y on top of z
     assert call(D=_fake(5)) == 9                                  # y on top of D
+    assert call(ckpt=_fake(5)) == 9                               # checkpoints on top of y
+    assert call(ckpt=_fake(1)) == 9                               # ... or of an input
     monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
-    assert call(D=_fake(6), z=_fake(7), bias=_fake(8), sp=1) == 7  # passes every check
+    assert call(D=_fake(6), z=_fake(7), bias=_fake(8), sp=1, ckpt=_fake(9)) == 7  # passes every check
+
+
+def test_ckpt_size(lib):
+    dims = D(L=130, dim=8)          # 3 chunks of 64 steps
+    size = ctypes.c_size_t(0)
+    assert lib.mm_scan_ckpt_size(ctypes.byref(dims), ctypes.byref(size)) == 0
+    assert size.value == dims.batch * 8 * 3 * 2 * dims.dstate * 4
+    assert mm.mm_scan_ckpt_size(dims.batch, 130, 8, dims.dstate) == size.value
+    assert lib.mm_scan_ckpt_size(ctypes.byref(D(L=0, dim=8)), ctypes.byref(size)) == 2
+
+
+def test_bwd_checks_its_arguments(lib, monkeypatch):
+    dims = D(L=200, dim=8)
+    def call(**over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), h0=None, v0=None,
+                 ckpt=_fake(10), dy=_fake(11), dhT=None, dvT=None, dx=_fake(12), dd=_fake(13),
+                 dA=_fake(14), dB=_fake(15), dC=_fake(16), dh0=None, dv0=None, beta=0.9)
+        a.update(over)
+        return lib.mm_scan_bwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["h0"], a["v0"], a["beta"],
+                               1.0, a["ckpt"], a["dy"], a["dhT"], a["dvT"], a["dx"], a["dd"], a["dA"],
+                               a["dB"], a["dC"], a["dh0"], a["dv0"], ctypes.byref(dims), None)
+    assert call(dy=None) == 1
+    assert call(ckpt=None) == 1                                   # needed past 64 steps
+    assert "ckpt" in mm.mm_last_error()
+    assert call(beta=1.0) == 3
+    assert call(dB=ctypes.c_void_p(A16 * 15 + 8)) == 5
+    assert call(dx=_fake(0)) == 9                                 # gradient over an input
+    assert call(dC=_fake(15)) == 9                                # two gradients on one buffer
+    assert call(dh0=_fake(10)) == 9                               # over the checkpoints
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call() == 7                                            # passes every check
+    assert call(ckpt=None, **{}) == 1
+    short = D(L=64, dim=8)
+    rc = lib.mm_scan_bwd(_fake(0), _fake(1), _fake(2), _fake(3), _fake(4), None, None, 0.5, 1.0,
+                         None, _fake(11), None, None, _fake(12), _fake(13), _fake(14), _fake(15),
+                         _fake(16), None, None, ctypes.byref(short), None)
+    assert rc == 7                                                # one chunk: no checkpoint needed
 
 
 def test_set_tile(lib):
