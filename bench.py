@@ -57,6 +57,11 @@ ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
 DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
 IO_KEYS = ("x", "delta", "B", "C", "z")          # tensors in the workload's storage type
 GATED_EXTRAS = "D skip, z SiLU gate, delta_bias, softplus"
+FP32_LANES_PER_CLK_PER_SM = 128      # fp32 arithmetic lanes of one SM per clock
+# fp32 operations one state update needs in the backward (an FMA counts as one):
+# the forward rebuild (delta*A, w, v, h) and the reverse step (G, P, the two
+# carries, B.P, a h_{t-1} G (two), A-weighted sum, dA, dB, dC), plus one ex2.
+BWD_OPS_PER_UPDATE = 16
 
 
 def measured_traffic(kernel: str, workload: str):
@@ -94,6 +99,164 @@ def algorithmic_bytes(w: wl.ScanWorkload, gated: bool = False) -> int:
     extra = (bdl * eb + 2 * w.dim * 4) if gated else 0
     return 3 * bdl * eb + 2 * w.batch * w.dstate * w.seqlen * eb + w.dim * w.dstate * 4 \
         + 2 * w.batch * w.dim * w.dstate * 4 + extra
+
+
+def bwd_algorithmic_bytes(w: wl.ScanWorkload) -> int:
+    """Bytes the backward must move: x, delta, dy read and dx, ddelta written
+    once; B, C read and dB, dC (fp32) written once; the checkpoints read once;
+    A and dA."""
+    eb = 4 if w.io == "f32" else 2
+    bdl = w.batch * w.dim * w.seqlen
+    bnl = w.batch * w.dstate * w.seqlen
+    chunks = -(-w.seqlen // 16)
+    return 5 * bdl * eb + 2 * bnl * eb + 2 * bnl * 4 + w.batch * w.dim * chunks * 2 * w.dstate * 4 \
+        + 2 * w.dim * w.dstate * 4
+
+
+def bwd_cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0):
+    """The fp64 oracle's backward (as it stands) on the first D' channels of
+    batch row 0 (a whole backward of that slice: every gradient, dB and dC
+    summed over the slice), D' sized to about `budget_s` of CPU time."""
+    import oracle
+    inp = wl.scan_inputs(w)
+    rng = np.random.default_rng(5)
+    cores = oracle.num_threads()
+    wall_budget = budget_s / max(cores, 1)
+
+    def run(dd):
+        sl = {k: (v[:1, :dd] if k in ("x", "delta") else v[:1] if k in ("B", "C") else v[:dd])
+              for k, v in inp.items()}
+        dy = rng.standard_normal(sl["x"].shape).astype(np.float32)
+        t = time.perf_counter()
+        oracle.scan_bwd(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], dy, beta=beta, alpha=alpha)
+        return time.perf_counter() - t
+
+    probe = min(w.dim, 16)
+    per_chan = run(probe) / probe
+    dd = max(1, min(w.dim, int(wall_budget / max(per_chan, 1e-9))))
+    dt = run(dd)
+    return {"value": dd * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"backward of channels 0..{dd - 1} of batch row 0 (all gradients), beta={beta}, "
+                      f"alpha={alpha}, fp64, {dt:.2f} s wall on {cores} threads"}
+
+
+def run_scan_bwd(args, w, beta, alpha, rank, world):
+    """Time mm_scan_bwd (the backward kernel) on resident inputs, checkpoints
+    and output gradient; e2e adds the host copies of those in and of every
+    gradient out."""
+    import torch
+    import selective_state_space_momentum_b200 as mm
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))
+    iodt = torch.float32 if w.io == "f32" else torch.bfloat16
+    gen = torch.Generator().manual_seed(rank_seed(w.seed_index, rank) + 17)
+    host = {k: torch.from_numpy(v).to(iodt if k in IO_KEYS else torch.float32) for k, v in inp.items()}
+    host["dy"] = torch.randn(tuple(inp["x"].shape), generator=gen).to(iodt)
+    step_bytes = bwd_algorithmic_bytes(w)
+    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    sets = []
+    for _ in range(nsets):
+        s = {k: v.to(dev).contiguous() for k, v in host.items()}
+        _, _, _, s["ckpt"] = mm.scan_fwd_train(s["x"], s["delta"], s["A"], s["B"], s["C"], beta=beta,
+                                               alpha=alpha)
+        s["g"] = {"dx": torch.empty_like(s["x"]), "ddelta": torch.empty_like(s["x"]),
+                  "dA": torch.empty((w.dim, w.dstate), device=dev),
+                  "dB": torch.empty((w.batch, w.dstate, w.seqlen), device=dev),
+                  "dC": torch.empty((w.batch, w.dstate, w.seqlen), device=dev)}
+        sets.append(s)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def bwd(s):
+        g = s["g"]
+        mm.mm_scan_bwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha, s["ckpt"],
+                       s["dy"], None, None, g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], None, None,
+                       stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for i in range(args.warmup):
+        bwd(sets[i % nsets])
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            bwd(sets[i % nsets])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
+    value = whole_job_rate(w.updates, world, ms_step)
+
+    # ---- end to end: host copies in, the backward, every gradient out ------
+    e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
+    ck_host = sets[0]["ckpt"].cpu()
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    pinned["ckpt"] = ck_host.pin_memory()
+    out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in sets[0]["g"].items()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in out.values())
+
+    def e2e_step():
+        d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        g = mm.scan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["ckpt"], d["dy"], beta=beta,
+                        alpha=alpha, stream=stream)
+        for k in out:
+            out[k].copy_(g[k], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    barrier()
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        clocks = clk.summary()
+        sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
+        alu_peak = FP32_LANES_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
+        achieved = w.updates * BWD_OPS_PER_UPDATE / (ms_step * 1e-3)
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        hbm_achieved = step_bytes / (ms_step * 1e-3) / 1e9
+        line = {
+            "metric": "selective-scan backward state updates/s (B·L·D·N) and % of roofline, 1×B200",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.io, "data": "synthetic",
+            "config": {"workload": w.name, "pass": "backward", "batch": w.batch, "seq_len": w.seqlen,
+                       "dim": w.dim, "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
+                       "global_batch": w.batch * world, "parallelism": f"dp{world}",
+                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
+            "roofline": {"bound": "alu", "kernel": "scan_bwd_kernel",
+                         "achieved": achieved / 1e9, "peak": alu_peak / 1e9, "unit": "Gop/s",
+                         "frac": achieved / alu_peak, "traffic": None,
+                         "peak_source": f"128 fp32 lanes/clk/SM x 148 SMs x {sm_max:.0f} MHz; "
+                                        f"{BWD_OPS_PER_UPDATE} fp32 ops per state update",
+                         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": hbm_achieved / hbm_peak, "peak_source": peak_kind,
+                                 "algorithmic_bytes": step_bytes}},
+            "e2e": {"value": whole_job_rate(w.updates, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = bwd_cpu_baseline(w, beta, alpha)
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 # ------------------------------------------------------------ clocks -------
@@ -472,13 +635,19 @@ def main(argv=None):
                     help="wall seconds for the whole --impl reference run")
     ap.add_argument("--gated", action="store_true",
                     help="time mm_scan_fwd_gated with D, z, delta_bias and softplus (scan workloads)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward mm_scan_bwd (scan workloads)")
     ap.add_argument("--tile", default=None, help="force SPTxWARPS[xTIME_LANES], e.g. 4x2 or 4x2x2 (tuning)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[ALIASES.get(args.workload, args.workload)]
-    if args.gated and isinstance(w, wl.SSDWorkload):
-        ap.error("--gated applies to the scan workloads")
+    if (args.gated or args.backward) and isinstance(w, wl.SSDWorkload):
+        ap.error("--gated and --backward apply to the scan workloads")
+    if args.gated and args.backward:
+        ap.error("--backward times the plain scan's backward")
+    if args.backward and args.impl == "reference":
+        ap.error("--impl reference times the forward")
     if isinstance(w, wl.SSDWorkload):
         if args.impl == "reference":
             return run_reference(args, w)
@@ -514,6 +683,11 @@ def main(argv=None):
                                 device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
+    if args.backward:
+        rc = run_scan_bwd(args, w, beta, alpha, rank, world)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
     dev = torch.device("cuda", torch.cuda.current_device())
     if args.tile:
         parts = [int(v) for v in args.tile.split("x")]

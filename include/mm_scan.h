@@ -47,7 +47,7 @@ typedef enum {
 typedef enum { MM_F32 = 0, MM_BF16 = 1 } mm_dtype;
 
 /* Steps between two checkpoints of the forward's state (see mm_scan_bwd). */
-#define MM_SCAN_CHUNK 64
+#define MM_SCAN_CKPT_STEPS 16
 
 /* Sizes of one Mamba-1 scan call. */
 typedef struct {
@@ -139,11 +139,12 @@ mm_status mm_scan_fwd(const void *x, const void *delta, const float *A,
  * and errors as mm_scan_fwd.  delta' is computed once per (batch, channel,
  * step) in fp32 from the loaded delta; the gate uses a fast exponential.
  *
- *   ckpt   (batch, dim, ceil(L / 64), 2, dstate) fp32, or NULL: for every
- *          chunk k of MM_SCAN_CHUNK = 64 steps, (h, v) after its last step
- *          (step min(64 k + 63, L - 1)); [.., 0, :] holds h and [.., 1, :]
- *          holds v.  This is what mm_scan_bwd restarts from.  Size in bytes:
- *          mm_scan_ckpt_size.  It may overlap no other argument.
+ *   ckpt   (batch, dim, ceil(L / 16), 2, dstate) fp32, or NULL: for every
+ *          block i of MM_SCAN_CKPT_STEPS = 16 steps, (h, v) after its last
+ *          step (step min(16 i + 15, L - 1)); [.., 0, :] holds h and
+ *          [.., 1, :] holds v.  This is what mm_scan_bwd restarts from.  Size
+ *          in bytes: mm_scan_ckpt_size (L * batch * dim * dstate / 2 for L a
+ *          multiple of 16).  It may overlap no other argument.
  */
 mm_status mm_scan_fwd_gated(const void *x, const void *delta, const float *A,
                             const void *B, const void *C,
@@ -155,7 +156,7 @@ mm_status mm_scan_fwd_gated(const void *x, const void *delta, const float *A,
                             const mm_scan_dims *dims, void *stream);
 
 /* mm_scan_ckpt_size -- bytes of the checkpoint buffer of mm_scan_fwd_gated
- * and mm_scan_bwd: batch * dim * ceil(seqlen / 64) * 2 * dstate * 4.
+ * and mm_scan_bwd: batch * dim * ceil(seqlen / 16) * 2 * dstate * 4.
  * Errors as the size checks of mm_scan_fwd. */
 mm_status mm_scan_ckpt_size(const mm_scan_dims *dims, size_t *bytes);
 
@@ -178,7 +179,7 @@ mm_status mm_scan_ckpt_size(const mm_scan_dims *dims, size_t *bytes);
  *
  * Inputs: x, delta, A, B, C, h0, v0, beta, alpha and dims exactly as given
  * to the forward; ckpt as mm_scan_fwd_gated wrote it for those inputs (it
- * may be NULL when seqlen <= 64); dy (batch, dim, L) io: the gradient
+ * may be NULL when seqlen <= 16); dy (batch, dim, L) io: the gradient
  * reaching y; dhT, dvT (batch, dim, dstate) fp32: the gradients reaching
  * hT, vT, or NULL for zero.
  * Outputs (overwritten): dx, ddelta (batch, dim, L) io (rounded to nearest
@@ -188,11 +189,12 @@ mm_status mm_scan_ckpt_size(const mm_scan_dims *dims, size_t *bytes);
  * No output may overlap an input or another output (MM_ERR_ALIAS); every
  * pointer must be 16-byte aligned.
  *
- * Work: the kernel restarts every 64-step chunk from its checkpoint and
- * rebuilds the states of each 8 steps once more on the way back, so it
- * performs about two forward passes and one reverse pass of arithmetic.
+ * Work: the kernel restarts every 16-step block from its checkpoint,
+ * rebuilds the block's states once and walks them back (forming each
+ * exponential a second time there): one forward pass and one reverse pass
+ * of arithmetic.
  *
- * Errors: MM_ERR_NULL (a required pointer, or ckpt with seqlen > 64),
+ * Errors: MM_ERR_NULL (a required pointer, or ckpt with seqlen > 16),
  * MM_ERR_DIMS, MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE,
  * MM_ERR_SCALAR, MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA.
  */

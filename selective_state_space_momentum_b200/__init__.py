@@ -27,7 +27,7 @@ __all__ = [
     "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_ssd_fwd",
     "mm_ssd_workspace_size", "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
-    "EXPORTED_SYMBOLS", "MM_SCAN_CHUNK",
+    "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +37,7 @@ _lib = None
 
 MM_F32 = 0
 MM_BF16 = 1
-MM_SCAN_CHUNK = 64      # steps between two checkpoints of the forward's state
+MM_SCAN_CKPT_STEPS = 16     # steps between two checkpoints of the forward's state
 
 STATUS_NAMES = {
     0: "MM_OK", 1: "MM_ERR_NULL", 2: "MM_ERR_DIMS", 3: "MM_ERR_SCALAR", 4: "MM_ERR_DTYPE",
@@ -172,7 +172,7 @@ def mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v
     """C entry point mm_scan_fwd_gated (marshalling only): mm_scan_fwd plus the
     optional D (dim,) fp32, z (batch, dim, L) in the storage type of x,
     delta_bias (dim,) fp32, the softplus switch and the checkpoint output
-    ckpt (batch, dim, ceil(L / 64), 2, N) fp32."""
+    ckpt (batch, dim, ceil(L / 16), 2, N) fp32."""
     batch, dim, L = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
@@ -281,14 +281,14 @@ def scan_fwd(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0,
 
 def scan_fwd_train(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, stream=None):
     """Forward that also keeps the checkpoints the backward restarts from:
-    returns (y, hT, vT, ckpt), ckpt (batch, dim, ceil(L / 64), 2, N) fp32."""
+    returns (y, hT, vT, ckpt), ckpt (batch, dim, ceil(L / 16), 2, N) fp32."""
     import torch
     batch, dim, L = x.shape
     N = A.shape[1]
     y = torch.empty_like(x)
     hT = torch.empty((batch, dim, N), device=x.device, dtype=torch.float32)
     vT = torch.empty_like(hT)
-    ckpt = torch.empty((batch, dim, (L + MM_SCAN_CHUNK - 1) // MM_SCAN_CHUNK, 2, N), device=x.device,
+    ckpt = torch.empty((batch, dim, (L + MM_SCAN_CKPT_STEPS - 1) // MM_SCAN_CKPT_STEPS, 2, N), device=x.device,
                        dtype=torch.float32)
     mm_scan_fwd_gated(x, delta, A, B, C, None, None, None, False, h0, v0, beta, alpha, y, hT, vT,
                       ckpt, stream)

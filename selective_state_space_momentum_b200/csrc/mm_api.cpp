@@ -84,7 +84,7 @@ struct ScanSizes {
     int64_t a_bytes;     // (dim, dstate) fp32
     int64_t st_bytes;    // (batch, dim, dstate) fp32
     int64_t d_bytes;     // (dim) fp32
-    int64_t ck_bytes;    // (batch, dim, chunks, 2, dstate) fp32
+    int64_t ck_bytes;    // (batch, dim, ceil(L / 16), 2, dstate) fp32
 };
 
 mm_status check_scan_dims(const mm_scan_dims* dims, float beta, float alpha, ScanSizes* z) {
@@ -100,7 +100,7 @@ mm_status check_scan_dims(const mm_scan_dims* dims, float beta, float alpha, Sca
     if (!std::isfinite(alpha) || alpha < 0.0f)
         return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
     z->esize = dims->io == MM_F32 ? 4 : 2;
-    const int64_t chunks = (L + MM_SCAN_CHUNK - 1) / MM_SCAN_CHUNK;
+    const int64_t chunks = (L + MM_SCAN_CKPT_STEPS - 1) / MM_SCAN_CKPT_STEPS;
     int64_t bd, bdl, bn, bnl, dn, bdn, bdc, bdc2;
     if (!mul_ok(bsz, D, &bd) || !mul_ok(bd, L, &bdl) || !mul_ok(bdl, z->esize, &z->seq_bytes) ||
         !mul_ok(bsz, N, &bn) || !mul_ok(bn, L, &bnl) || !mul_ok(bnl, z->esize, &z->bc_bytes) ||
@@ -249,8 +249,8 @@ mm_status mm_scan_bwd(const void* x, const void* delta, const float* A, const vo
     ScanSizes zs;
     if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
     const int64_t L = dims->seqlen;
-    if (!ckpt && L > MM_SCAN_CHUNK)
-        return fail(MM_ERR_NULL, "ckpt is required when seqlen > %d", MM_SCAN_CHUNK);
+    if (!ckpt && L > MM_SCAN_CKPT_STEPS)
+        return fail(MM_ERR_NULL, "ckpt is required when seqlen > %d", MM_SCAN_CKPT_STEPS);
     const void* ptrs[] = {x, delta, A, B, C, h0, v0, ckpt, dy, dhT, dvT, dx, ddelta, dA, dB, dC, dh0, dv0};
     const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "ckpt", "dy", "dhT", "dvT",
                            "dx", "ddelta", "dA", "dB", "dC", "dh0", "dv0"};

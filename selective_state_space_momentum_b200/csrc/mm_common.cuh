@@ -10,6 +10,8 @@ namespace mmscan {
 
 // log2(e): exp(z) is evaluated as 2^(z * log2 e) on the MUFU unit.
 constexpr float kLog2e = 1.4426950408889634f;
+// Steps between two checkpoints of the scan state (forward writes, backward reads).
+constexpr int kCkptSteps = 16;
 
 using bf16 = __nv_bfloat16;
 

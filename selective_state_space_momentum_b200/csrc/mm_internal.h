@@ -31,7 +31,7 @@ struct ScanArgs {
     const float* dbias;    // (dim) or null
     int softplus;          // delta' = softplus(delta + dbias)
     int ext;               // any of the four is present
-    float* ckpt;           // (batch, dim, ceil(L / 64), 2, dstate): (h, v) after each chunk, or null
+    float* ckpt;           // (batch, dim, ceil(L / 16), 2, dstate): (h, v) after every 16 steps, or null
 };
 
 // Arguments of one backward launch (device pointers; sizes as in mm_scan_dims).
@@ -43,7 +43,7 @@ struct ScanBwdArgs {
     const void* C;
     const float* h0;
     const float* v0;
-    const float* ckpt;     // the forward's (h, v) after every 64-step chunk
+    const float* ckpt;     // the forward's (h, v) after every 16 steps
     const void* dout;      // gradient reaching y (io dtype)
     const float* dhT;      // gradients reaching hT, vT, or null
     const float* dvT;

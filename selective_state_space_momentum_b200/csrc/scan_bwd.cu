@@ -20,19 +20,18 @@
 //    chunks of 64 steps from the last to the first and carries (G, P) in
 //    registers, so the reverse recursion runs in time order and needs no
 //    carry recombination.
-//  * States.  The forward saved (h, v) after every chunk; a chunk starts from
-//    the previous chunk's checkpoint (h0, v0 for the first).  A first pass runs
-//    the chunk forward and keeps the state at the start of each group of 8
-//    steps in registers; the reverse pass rebuilds each group's states and
-//    exponentials from its start (a second forward over 8 steps) and walks
-//    them backwards.  The rebuilt states are those of the forward kernel bit
-//    for bit (same operations in the same order).  Nothing of size (L, D, N)
-//    is stored.
+//  * States.  The forward saved (h, v) after every 16 steps.  Each block of
+//    16 steps restarts from the checkpoint before it (h0, v0 for the first),
+//    rebuilds its 16 states and exponentials in registers and walks them
+//    backwards; the next block's checkpoint is loaded while a block runs.  The
+//    rebuilt states are those of the forward kernel bit for bit (same
+//    operations in the same order).  Nothing of size (L, D, N) is stored.
 //  * Reductions.  The sums over a channel's states (for dx, ddelta) use the
 //    forward's register butterfly.  dB and dC sum over channels: a butterfly
-//    across the channels of a warp, shared-memory atomics across the warps,
-//    then one vector atomic add per (4 steps, state) into global memory per
-//    chunk.  dA collects in registers over the whole sequence and is added
+//    across the channels of a warp (four steps at a time, so the exchanges
+//    are independent), shared-memory atomics across the warps into one of
+//    two buffers, then one vector atomic add per (4 steps, state) into global
+//    memory after each block.  dA collects in registers over the whole sequence and is added
 //    once per lane.
 //  * Staging: x, delta, dy, B and C tiles by TMA (128-byte swizzle, no
 //    multicast), two chunks in flight; B and C transposed to [t][n] fp32 with
@@ -40,6 +39,7 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "mm_common.cuh"
 #include "mm_internal.h"
@@ -73,20 +73,23 @@ struct BwdTile {
     static constexpr int STAGE_BYTES = OFF_C + NBOX * BBOX;
     static constexpr int BP = NP + 4;            // row pitch (floats) of transposed B/C
     static constexpr int BT_BYTES = T * BP * 4;
-    static constexpr int R = 8;                  // steps per group
-    static constexpr int NG = T / R;
+    static constexpr int KB = kCkptSteps;        // steps per block (the checkpoint interval)
+    static constexpr int R = 8;                  // steps per read-out group
     static constexpr int PER = R / G;            // steps of a group whose sums a lane owns
     static constexpr int RP = 2 * NP;            // dB and dC partials per step
     static constexpr int OFF_BT = STAGES * STAGE_BYTES;   // B^T, then C^T
     static constexpr int OFF_RED = OFF_BT + 2 * BT_BYTES;
-    static constexpr int RED_BYTES = T * RP * 4;
+    static constexpr int RED_BYTES = 2 * KB * RP * 4;   // two blocks' dB, dC partials
     static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
-    // 12 resident warps per SM (<= 168 registers a thread)
+    // 12 resident warps per SM (<= 168 registers a thread, no spills).  Four
+    // 4-warp CTAs would fit the shared memory, but at 128 registers the
+    // kernel spills and ran 33% slower on the 384-CTA fp32 grid.
     static constexpr int MIN_CTAS = 12 / WARPS > 0 ? 12 / WARPS : 1;
 
     static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "lanes per channel");
-    static_assert(R % G == 0 && BOX_T % R == 0 && T % BOX_T == 0, "step grouping");
+    static_assert(R % G == 0 && BOX_T % R == 0 && T % BOX_T == 0 && KB % R == 0 && T % KB == 0,
+                  "step grouping");
     static_assert(CH % 8 == 0, "x tiles must be whole 1024-byte swizzle atoms");
     static_assert(STAGE_BYTES % 1024 == 0 && OFF_BT % 16 == 0 && OFF_RED % 16 == 0, "alignment");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -99,7 +102,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_C, const ScanBwdArgs p) {
     using TL = BwdTile<IO, NP, WARPS>;
     constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
-    constexpr int ST = TL::STAGES, EB = TL::EB, BP = TL::BP, NG = TL::NG, PER = TL::PER;
+    constexpr int ST = TL::STAGES, EB = TL::EB, BP = TL::BP, PER = TL::PER, KB = TL::KB;
     constexpr int RP = TL::RP;
 
     extern __shared__ unsigned char smem_raw[];
@@ -130,7 +133,8 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, use_tma ? 1u : (uint32_t)NT);
         fence_barrier_init();
     }
-    for (int i = tid; i < T * RP; i += NT) red[i] = 0.0f;
+    for (int i = tid; i < 2 * KB * RP; i += NT) red[i] = 0.0f;
+    int nred = 0;                                    // blocks done: picks the partials buffer
     __syncthreads();
 
     // ---- per-lane constants and carries -------------------------------------
@@ -146,12 +150,19 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const float2 beta2 = f2(p.beta, p.beta);
     const float alpha = p.alpha;
     const int64_t srow = (b * p.dim + (active ? d : 0)) * N;   // this channel's state row
-    auto load_pair = [&](const float* src) {
+    auto load_pair = [&](const float* src, int64_t off = 0) {
         float v[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-            if (src && active && n0 + e < N) v[e] = src[n0 + e];
+            if (src && active && n0 + e < N) v[e] = src[off + n0 + e];
         return f2(v[0], v[1]);
+    };
+    // (h, v) where block gblk (of KB steps, counted over the whole sequence)
+    // starts: the checkpoint after block gblk - 1, or (h0, v0)
+    const int64_t ncks = (L + KB - 1) / KB;
+    auto start_state = [&](int64_t gblk, int which) {
+        if (gblk == 0) return load_pair(which ? p.v0 : p.h0, srow);
+        return load_pair(p.ckpt + ((b * p.dim + (active ? d : 0)) * ncks + gblk - 1) * 2 * N + which * N, 0);
     };
     float2 cg = load_pair(p.dhT ? p.dhT + srow : nullptr);   // a_{t+1} G_{t+1}
     float2 cp = load_pair(p.dvT ? p.dvT + srow : nullptr);   // beta P_{t+1}
@@ -227,12 +238,11 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const int s = (int)(i % ST);
         const int64_t t0 = k * T;
         const int nval = (int)((L - t0) < T ? (L - t0) : T);
-        // the chunk's start state: the previous chunk's checkpoint, or (h0, v0)
-        const float* hsrc = k > 0 ? p.ckpt + ((b * p.dim + (active ? d : 0)) * nchunks + (k - 1)) * 2 * N
-                                  : (p.h0 ? p.h0 + srow : nullptr);
-        const float* vsrc = k > 0 ? hsrc + N : (p.v0 ? p.v0 + srow : nullptr);
-        const float2 hst = load_pair(hsrc);
-        const float2 vst = load_pair(vsrc);
+        const int nblk = (nval + KB - 1) / KB;
+        // start state of the chunk's last block: loaded before the wait, and each
+        // block's predecessor is fetched while the block runs
+        float2 hn = start_state(k * (T / KB) + nblk - 1, 0);
+        float2 vn = start_state(k * (T / KB) + nblk - 1, 1);
         if (!mbar_wait(bar0 + 8 * s, (uint32_t)((i / ST) & 1), &g_bwd_dev_err)) return;
         const unsigned char* sbuf = smem + s * TL::STAGE_BYTES;
 
@@ -276,31 +286,16 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // Every thread is past the previous chunk: its stage is free.
         if (i + ST - 1 < nchunks) issue(nchunks - 1 - (i + ST - 1), (int)((i + ST - 1) % ST));
 
-        // delta, x (and dy) of the R steps of group gi, this lane's channel
-        auto load_group = [&](int gi, float (&dl)[R], float (&xl)[R]) {
-            const int tau0 = gi * R;
-            const int bx = tau0 / TL::BOX_T;
-            const int col = tau0 - bx * TL::BOX_T;
-            const unsigned char* xt = sbuf + TL::OFF_X + bx * TL::XBOX;
-            const unsigned char* dt = sbuf + TL::OFF_D + bx * TL::XBOX;
-#pragma unroll
-            for (int j = 0; j < R; j += 4) {
-                const float4 dq = load4(reinterpret_cast<const IO*>(dt + sw128(c, (col + j) * EB)));
-                const float4 xq = load4(reinterpret_cast<const IO*>(xt + sw128(c, (col + j) * EB)));
-                dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
-                xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
-            }
+        // delta, x or dy of the 4 steps from tau, this lane's channel
+        auto load4s = [&](int off, int tau) {
+            const int bx = tau / TL::BOX_T;
+            const int col = tau - bx * TL::BOX_T;
+            return load4(reinterpret_cast<const IO*>(sbuf + off + bx * TL::XBOX + sw128(c, col * EB)));
         };
-        auto load_dy = [&](int gi, float (&yl)[R]) {
-            const int tau0 = gi * R;
-            const int bx = tau0 / TL::BOX_T;
-            const int col = tau0 - bx * TL::BOX_T;
-            const unsigned char* yt = sbuf + TL::OFF_Y + bx * TL::XBOX;
-#pragma unroll
-            for (int j = 0; j < R; j += 4) {
-                const float4 q = load4(reinterpret_cast<const IO*>(yt + sw128(c, (col + j) * EB)));
-                yl[j] = q.x; yl[j + 1] = q.y; yl[j + 2] = q.z; yl[j + 3] = q.w;
-            }
+        auto load1s = [&](int off, int tau) {
+            const int bx = tau / TL::BOX_T;
+            const int col = tau - bx * TL::BOX_T;
+            return load1(reinterpret_cast<const IO*>(sbuf + off + bx * TL::XBOX + sw128(c, col * EB)));
         };
         // one forward step of the lane's two states (the forward kernel's operations)
         auto fwd_step = [&](int tau, float dl, float u, float2& h, float2& v, float2& a) {
@@ -311,150 +306,156 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             v = __ffma2_rn(beta2, v, w);
             h = __ffma2_rn(a, h, v);
         };
-        // dB, dC partials of step tau: summed over the warp's channels by a
-        // butterfly, then over the warps by shared-memory atomics
-        auto chan_reduce = [&](int tau, float2 dBv, float2 dCv) {
+        // dB, dC partials of 4 consecutive steps from tau: summed over the
+        // warp's channels by a butterfly (the lane keeps dB or dC, then one of
+        // its two states), then over the warps by shared-memory atomics
+        auto chan_reduce4 = [&](float* redb, int tau, const float2 (&dBv)[4], const float2 (&dCv)[4]) {
             const bool up1 = (lane & 16) != 0;
-            float k0 = up1 ? dCv.x : dBv.x, k1 = up1 ? dCv.y : dBv.y;
-            const float s0 = up1 ? dBv.x : dCv.x, s1 = up1 ? dBv.y : dCv.y;
-            k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-            k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
             const bool up2 = (lane & 8) != 0;
-            float kk = up2 ? k1 : k0;
-            const float ss = up2 ? k0 : k1;
-            kk += __shfl_xor_sync(0xffffffffu, ss, 8);
+            float r[4];
 #pragma unroll
-            for (int m = G; m < 8; m <<= 1) kk += __shfl_xor_sync(0xffffffffu, kk, m);
-            if ((lane & 7) < G) atomicAdd(red + tau * RP + (up1 ? NP : 0) + n0 + (up2 ? 1 : 0), kk);
+            for (int jj = 0; jj < 4; ++jj) {
+                float k0 = up1 ? dCv[jj].x : dBv[jj].x, k1 = up1 ? dCv[jj].y : dBv[jj].y;
+                const float s0 = up1 ? dBv[jj].x : dCv[jj].x, s1 = up1 ? dBv[jj].y : dCv[jj].y;
+                k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+                k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+                r[jj] = (up2 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, up2 ? k0 : k1, 8);
+            }
+#pragma unroll
+            for (int m = G; m < 8; m <<= 1) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) r[jj] += __shfl_xor_sync(0xffffffffu, r[jj], m);
+            }
+            if ((lane & 7) < G) {
+                float* dst = redb + tau * RP + (up1 ? NP : 0) + n0 + (up2 ? 1 : 0);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) atomicAdd(dst + jj * RP, r[jj]);
+            }
         };
-        // Group gi (first kmax steps valid) from its start state: rebuild the
-        // states and exponentials, then walk the steps backwards.
-        auto group_reverse = [&](int gi, int kmax, float2 h, float2 v) {
-            const int tau0 = gi * R;
-            float dl[R], xl[R], yl[R], u[R];
-            load_group(gi, dl, xl);
-            load_dy(gi, yl);
-#pragma unroll
-            for (int j = 0; j < R; ++j) u[j] = dl[j] * xl[j];
-            float2 ht[R], at[R];
+        // One block of KB steps (the first kmax valid) from its start state:
+        // rebuild its states, then walk it backwards (the exponentials are
+        // formed again there: two MUFU operations instead of 32 registers).
+        // kmax is a compile-time KB for whole blocks.
+        auto block = [&](int blk, auto kmax, float2 h, float2 v, float* redb) {
+            const int tb = blk * KB;
+            float2 ht[KB];
             const float2 hprev0 = h;
 #pragma unroll
-            for (int j = 0; j < R; ++j) {
-                if (j < kmax) fwd_step(tau0 + j, dl[j], u[j], h, v, at[j]);
-                else at[j] = f2(1.0f, 1.0f);
-                ht[j] = h;
-            }
-            float sk[R], qk[R];
+            for (int j4 = 0; j4 < KB; j4 += 4) {
+                if (j4 < kmax) {
+                    const float4 dq = load4s(TL::OFF_D, tb + j4);
+                    const float4 xq = load4s(TL::OFF_X, tb + j4);
+                    const float dl[4] = {dq.x, dq.y, dq.z, dq.w}, xl[4] = {xq.x, xq.y, xq.z, xq.w};
 #pragma unroll
-            for (int j = R - 1; j >= 0; --j) {
-                sk[j] = 0.0f;
-                qk[j] = 0.0f;
-                if (j < kmax) {
-                    const int tau = tau0 + j;
-                    const float2 bq = *reinterpret_cast<const float2*>(Bt + tau * BP + n0);
-                    const float2 cq = *reinterpret_cast<const float2*>(Ct + tau * BP + n0);
-                    const float2 Gt = __ffma2_rn(cq, f2(yl[j], yl[j]), cg);
-                    const float2 Pt = __fadd2_rn(Gt, cp);
-                    const float2 hp = j > 0 ? ht[j - 1] : hprev0;
-                    const float2 dt2 = __fmul2_rn(__fmul2_rn(at[j], hp), Gt);   // a_t h_{t-1} G_t
-                    const float2 s2 = __fmul2_rn(Pt, bq);                       // alpha B P
-                    const float2 q2 = __fmul2_rn(dt2, An);
-                    sk[j] = s2.x + s2.y;
-                    qk[j] = q2.x + q2.y;
-                    dA2 = __ffma2_rn(f2(dl[j], dl[j]), dt2, dA2);
-                    const float ua = u[j] * alpha;
-                    chan_reduce(tau, __fmul2_rn(Pt, f2(ua, ua)), __fmul2_rn(f2(yl[j], yl[j]), ht[j]));
-                    cg = __fmul2_rn(at[j], Gt);
-                    cp = __fmul2_rn(beta2, Pt);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        float2 a;
+                        if (j4 + jj < kmax) fwd_step(tb + j4 + jj, dl[jj], dl[jj] * xl[jj], h, v, a);
+                        ht[j4 + jj] = h;
+                    }
                 }
             }
-            // per-channel sums; lane g owns steps [g PER, (g + 1) PER) of the group
-            float so[PER], qo[PER];
-            butterfly_sum<G, R>(sk, so, g);
-            butterfly_sum<G, R>(qk, qo, g);
-            const int first = tau0 + g * PER;
-            const int cnt = nval - first < PER ? nval - first : PER;
-            float gx[PER], gd[PER];
 #pragma unroll
-            for (int e = 0; e < PER; ++e) {
-                const int st = first + e;
-                const int bxx = st / TL::BOX_T;
-                const int cc = st - bxx * TL::BOX_T;
-                const float de = load1(reinterpret_cast<const IO*>(sbuf + TL::OFF_D + bxx * TL::XBOX +
-                                                                    sw128(c, cc * EB)));
-                const float xe = load1(reinterpret_cast<const IO*>(sbuf + TL::OFF_X + bxx * TL::XBOX +
-                                                                    sw128(c, cc * EB)));
-                gx[e] = de * so[e];
-                gd[e] = __fmaf_rn(xe, so[e], qo[e]);
-            }
-            if (active && cnt > 0) {
-                store_steps_n<IO, PER>(dxrow + t0 + first, gx, cnt, vec_out);
-                store_steps_n<IO, PER>(ddrow + t0 + first, gd, cnt, vec_out);
+            for (int hf = KB / R - 1; hf >= 0; --hf) {
+                if (hf * R >= kmax) continue;
+                float sk[R], qk[R];
+#pragma unroll
+                for (int j4 = R - 4; j4 >= 0; j4 -= 4) {
+                    const int jb = hf * R + j4;              // first of these 4 steps in the block
+                    float2 dBv[4], dCv[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        sk[j4 + jj] = qk[j4 + jj] = 0.0f;
+                        dBv[jj] = dCv[jj] = f2(0.0f, 0.0f);
+                    }
+                    if (jb < kmax) {
+                        const float4 dq = load4s(TL::OFF_D, tb + jb);
+                        const float4 xq = load4s(TL::OFF_X, tb + jb);
+                        const float4 yq = load4s(TL::OFF_Y, tb + jb);
+                        const float dl[4] = {dq.x, dq.y, dq.z, dq.w}, xl[4] = {xq.x, xq.y, xq.z, xq.w};
+                        const float yl[4] = {yq.x, yq.y, yq.z, yq.w};
+#pragma unroll
+                        for (int jj = 3; jj >= 0; --jj) {
+                            const int j = jb + jj;
+                            if (j < kmax) {
+                                const int tau = tb + j;
+                                const float2 bq = *reinterpret_cast<const float2*>(Bt + tau * BP + n0);
+                                const float2 cq = *reinterpret_cast<const float2*>(Ct + tau * BP + n0);
+                                const float2 Gt = __ffma2_rn(cq, f2(yl[jj], yl[jj]), cg);
+                                const float2 Pt = __fadd2_rn(Gt, cp);
+                                const float2 hp = j > 0 ? ht[j > 0 ? j - 1 : 0] : hprev0;
+                                const float2 r2 = __fmul2_rn(f2(dl[jj], dl[jj]), A2);
+                                const float2 at = f2(ex2_approx(r2.x), ex2_approx(r2.y));
+                                const float2 dt2 = __fmul2_rn(__fmul2_rn(at, hp), Gt);      // a_t h_{t-1} G_t
+                                const float2 s2 = __fmul2_rn(Pt, bq);                       // alpha B P
+                                const float2 q2 = __fmul2_rn(dt2, An);
+                                sk[j4 + jj] = s2.x + s2.y;
+                                qk[j4 + jj] = q2.x + q2.y;
+                                dA2 = __ffma2_rn(f2(dl[jj], dl[jj]), dt2, dA2);
+                                const float ua = dl[jj] * xl[jj] * alpha;
+                                dBv[jj] = __fmul2_rn(Pt, f2(ua, ua));
+                                dCv[jj] = __fmul2_rn(f2(yl[jj], yl[jj]), ht[j]);
+                                cg = __fmul2_rn(at, Gt);
+                                cp = __fmul2_rn(beta2, Pt);
+                            }
+                        }
+                        chan_reduce4(redb, jb, dBv, dCv);
+                    }
+                }
+                // per-channel sums of these R steps; lane g owns PER of them
+                float so[PER], qo[PER];
+                butterfly_sum<G, R>(sk, so, g);
+                butterfly_sum<G, R>(qk, qo, g);
+                const int first = tb + hf * R + g * PER;
+                const int cnt = nval - first < PER ? nval - first : PER;
+                float gx[PER], gd[PER];
+#pragma unroll
+                for (int e = 0; e < PER; ++e) {
+                    gx[e] = load1s(TL::OFF_D, first + e) * so[e];
+                    gd[e] = __fmaf_rn(load1s(TL::OFF_X, first + e), so[e], qo[e]);
+                }
+                if (active && cnt > 0) {
+                    store_steps_n<IO, PER>(dxrow + t0 + first, gx, cnt, vec_out);
+                    store_steps_n<IO, PER>(ddrow + t0 + first, gd, cnt, vec_out);
+                }
             }
         };
 
-        if (nval == T) {
-            // pass 1: the chunk forward, keeping each group's start state
-            float2 hs[NG], vs[NG];
-            {
-                float2 h = hst, v = vst;
-#pragma unroll
-                for (int gi = 0; gi < NG; ++gi) {
-                    hs[gi] = h;
-                    vs[gi] = v;
-                    float dl[R], xl[R];
-                    load_group(gi, dl, xl);
-#pragma unroll
-                    for (int j = 0; j < R; ++j) {
-                        float2 a;
-                        fwd_step(gi * R + j, dl[j], dl[j] * xl[j], h, v, a);
-                    }
-                }
+#pragma unroll 1
+        for (int blk = nblk - 1; blk >= 0; --blk) {
+            const float2 h = hn, v = vn;
+            if (blk > 0) {
+                hn = start_state(k * (T / KB) + blk - 1, 0);
+                vn = start_state(k * (T / KB) + blk - 1, 1);
             }
-            // pass 2: groups backwards
-#pragma unroll
-            for (int gi = NG - 1; gi >= 0; --gi) group_reverse(gi, R, hs[gi], vs[gi]);
-        } else {
-            // Ragged last chunk (processed first): each group's start state is
-            // rebuilt from the chunk's start.
-            const int ng = (nval + R - 1) / R;
-            for (int gi = ng - 1; gi >= 0; --gi) {
-                float2 h = hst, v = vst;
-                for (int gg = 0; gg < gi; ++gg) {
-                    float dl[R], xl[R];
-                    load_group(gg, dl, xl);
-#pragma unroll
-                    for (int j = 0; j < R; ++j) {
-                        float2 a;
-                        fwd_step(gg * R + j, dl[j], dl[j] * xl[j], h, v, a);
-                    }
-                }
-                const int kmax = nval - gi * R < R ? nval - gi * R : R;
-                group_reverse(gi, kmax, h, v);
-            }
-        }
+            const int kmax = nval - blk * KB < KB ? nval - blk * KB : KB;
+            float* redb = red + (nred & 1) * (KB * RP);
+            if (kmax == KB) block(blk, std::integral_constant<int, KB>{}, h, v, redb);
+            else block(blk, kmax, h, v, redb);
+            ++nred;
 
-        // ---- dB, dC of the chunk into global memory ---------------------------
-        __syncthreads();
-        for (int it = tid; it < (T / 4) * RP; it += NT) {
-            const int slot = it % RP;
-            const int t4 = (it / RP) * 4;
-            float v4[4];
+            // ---- the block's dB, dC into global memory (the other buffer is
+            // the next block's; this one is next written two blocks later) ----
+            __syncthreads();
+            for (int it = tid; it < (KB / 4) * RP; it += NT) {
+                const int slot = it % RP;
+                const int t4 = (it / RP) * 4;
+                float v4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                v4[e] = red[(t4 + e) * RP + slot];
-                red[(t4 + e) * RP + slot] = 0.0f;
-            }
-            const int which = slot / NP;
-            const int n = slot - which * NP;
-            if (n < N && t4 < nval) {
-                float* dst = (which ? p.dC : p.dB) + (b * N + n) * L + t0 + t4;
-                if (vec_red && t4 + 4 <= nval) {
-                    atomicAdd(reinterpret_cast<float4*>(dst), make_float4(v4[0], v4[1], v4[2], v4[3]));
-                } else {
+                for (int e = 0; e < 4; ++e) {
+                    v4[e] = redb[(t4 + e) * RP + slot];
+                    redb[(t4 + e) * RP + slot] = 0.0f;
+                }
+                const int which = slot / NP;
+                const int n = slot - which * NP;
+                if (n < N && t4 < kmax) {
+                    float* dst = (which ? p.dC : p.dB) + (b * N + n) * L + t0 + blk * KB + t4;
+                    if (vec_red && t4 + 4 <= kmax) {
+                        atomicAdd(reinterpret_cast<float4*>(dst), make_float4(v4[0], v4[1], v4[2], v4[3]));
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (t4 + e < nval) atomicAdd(dst + e, v4[e]);
+                        for (int e = 0; e < 4; ++e)
+                            if (t4 + e < kmax) atomicAdd(dst + e, v4[e]);
+                    }
                 }
             }
         }

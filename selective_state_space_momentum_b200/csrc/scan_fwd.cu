@@ -29,8 +29,8 @@
 //  * Read-out.  The G lanes of a channel add their partial C_t . h_t by a
 //    register butterfly (shuffles, no shared memory) and store y directly:
 //    the G lanes write consecutive steps of their channel.
-//  * Checkpoints (optional).  (h, v) after every chunk of 64 steps go to a
-//    (batch, dim, chunks, 2, N) buffer that the backward restarts from.
+//  * Checkpoints (optional).  (h, v) after every 16 steps go to a
+//    (batch, dim, ceil(L / 16), 2, N) buffer that the backward restarts from.
 //  * Final state.  (h, v) after the last step go to hT, vT.  The per-state
 //    operation sequence does not depend on where the sequence is cut into
 //    calls, so split calls reproduce hT, vT bit for bit.
@@ -96,6 +96,7 @@ struct ScanTile {
     static_assert(TS == 1 || (TS == 2 && EB == 4 && T == 2 * 2 * R && (G == 4 || G == 8)),
                   "time split: fp32 I/O, two groups per lane, 4 or 8 lanes per channel");
     static_assert(!EXT || TS == 1, "the selective_scan_fn extras run without the time split");
+    static_assert(kCkptSteps % R == 0 && T % kCkptSteps == 0 || TS == 2, "checkpoints at group ends");
 };
 
 template <typename IO, int NP, int SPT, int WARPS, int TS, bool EXT>
@@ -129,6 +130,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int64_t L = p.seqlen;
     const int N = p.dstate;
     const int64_t nchunks = (L + T - 1) / T;
+    const int64_t ncks = (L + kCkptSteps - 1) / kCkptSteps;     // checkpoints per channel
     const bool use_tma = p.vec_ok != 0;
     const uint32_t bar0 = base + TL::OFF_BAR;
 
@@ -427,6 +429,24 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         };
 
         // The remaining nval < T steps of the sequence, one group at a time.
+        // (h, v) after steps 16 i + 15 and after the last step: where the
+        // backward restarts its 16-step blocks
+        auto save_ckpt = [&](int64_t idx) {
+            if (!p.ckpt || !writer) return;
+            float* cp = p.ckpt + ((b * p.dim + d) * ncks + idx) * 2 * N;
+#pragma unroll
+            for (int q = 0; q < NPAIR; ++q) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int n = g * SPT + 2 * q + e;
+                    if (n < N) {
+                        cp[n] = e ? hh[q].y : hh[q].x;
+                        cp[N + n] = e ? vv[q].y : vv[q].x;
+                    }
+                }
+            }
+        };
+
         auto ragged_chunk = [&]() {
             const int ngroups = (nval + R - 1) / R;
             for (int gi = 0; gi < ngroups; ++gi) {
@@ -457,6 +477,8 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     }
                 }
                 reduce_store(tau0, yk, zg);
+                const int end = tau0 + kmax;
+                if (end % kCkptSteps == 0 || end == nval) save_ckpt((t0 + end - 1) / kCkptSteps);
             }
         };
 
@@ -475,6 +497,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         if (gi + 1 < NG) prep(gi + 1, uA, aA, zA);
                         full_steps(gi, uB, aB, zB);
                     }
+                    if (((gi + 1) * R) % kCkptSteps == 0) save_ckpt((t0 + (gi + 1) * R) / kCkptSteps - 1);
                 }
             } else {
                 ragged_chunk();
@@ -562,21 +585,6 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     if (j_t) { vv[q] = vi; hh[q] = hi; }
                 }
                 ragged_chunk();
-            }
-        }
-        // ---- checkpoint: (h, v) after the chunk's last step, for the backward ----
-        if (p.ckpt && writer) {
-            float* cp = p.ckpt + ((b * p.dim + d) * nchunks + k) * 2 * N;
-#pragma unroll
-            for (int q = 0; q < NPAIR; ++q) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int n = g * SPT + 2 * q + e;
-                    if (n < N) {
-                        cp[n] = e ? hh[q].y : hh[q].x;
-                        cp[N + n] = e ? vv[q].y : vv[q].x;
-                    }
-                }
             }
         }
     }
@@ -731,7 +739,7 @@ ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int 
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s) {
-    // Checkpoints are laid out per 64-step chunk: the time split (32-step chunks) is not used.
+    // Checkpoints are written by the one-lane-along-time variants only.
     const int ts = a.ckpt ? 1 : t.ts;
     if (ts != t.ts && !scan_tile_supported(t.spt, t.warps, 1)) {
         if (io == 0) return launch_io<float>(a, t.np, 2, 4, 1, s);

@@ -128,10 +128,10 @@ def test_gated_checks_its_extras(lib, monkeypatch):
 
 
 def test_ckpt_size(lib):
-    dims = D(L=130, dim=8)          # 3 chunks of 64 steps
+    dims = D(L=130, dim=8)          # 9 blocks of 16 steps
     size = ctypes.c_size_t(0)
     assert lib.mm_scan_ckpt_size(ctypes.byref(dims), ctypes.byref(size)) == 0
-    assert size.value == dims.batch * 8 * 3 * 2 * dims.dstate * 4
+    assert size.value == dims.batch * 8 * 9 * 2 * dims.dstate * 4
     assert mm.mm_scan_ckpt_size(dims.batch, 130, 8, dims.dstate) == size.value
     assert lib.mm_scan_ckpt_size(ctypes.byref(D(L=0, dim=8)), ctypes.byref(size)) == 2
 
@@ -147,7 +147,7 @@ def test_bwd_checks_its_arguments(lib, monkeypatch):
                                1.0, a["ckpt"], a["dy"], a["dhT"], a["dvT"], a["dx"], a["dd"], a["dA"],
                                a["dB"], a["dC"], a["dh0"], a["dv0"], ctypes.byref(dims), None)
     assert call(dy=None) == 1
-    assert call(ckpt=None) == 1                                   # needed past 64 steps
+    assert call(ckpt=None) == 1                                   # needed past 16 steps
     assert "ckpt" in mm.mm_last_error()
     assert call(beta=1.0) == 3
     assert call(dB=ctypes.c_void_p(A16 * 15 + 8)) == 5
@@ -157,11 +157,11 @@ def test_bwd_checks_its_arguments(lib, monkeypatch):
     monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
     assert call() == 7                                            # passes every check
     assert call(ckpt=None, **{}) == 1
-    short = D(L=64, dim=8)
+    short = D(L=16, dim=8)
     rc = lib.mm_scan_bwd(_fake(0), _fake(1), _fake(2), _fake(3), _fake(4), None, None, 0.5, 1.0,
                          None, _fake(11), None, None, _fake(12), _fake(13), _fake(14), _fake(15),
                          _fake(16), None, None, ctypes.byref(short), None)
-    assert rc == 7                                                # one chunk: no checkpoint needed
+    assert rc == 7                                                # one block: no checkpoint needed
 
 
 def test_set_tile(lib):

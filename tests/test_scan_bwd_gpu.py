@@ -91,7 +91,7 @@ def test_bwd_matches_oracle(io, beta, alpha):
 @pytest.mark.parametrize("L", [1, 37, 64, 65, 129])
 def test_bwd_lengths_and_row_fallback(L):
     # L = 37 fp32 rows are not whole 16-byte pieces: element-wise staging;
-    # L = 1 and 64 need no checkpoint; 65 has a one-step last chunk
+    # L = 1 needs no checkpoint; 65 has a one-step last chunk and block
     w = wl.SCAN_MEDIUM
     inp, g = _problem(w, 1, L, 24)
     got, _ = _gpu(w, inp, g, 0.8, 1.5)
@@ -117,9 +117,9 @@ def test_checkpoints_are_the_states_after_each_chunk():
     w = wl.SCAN_MEDIUM
     inp, g = _problem(w, 2, 200, 24)
     _, (y, hT, vT, ckpt) = _gpu(w, inp, g, 0.9, 1.0)
-    ck = ckpt.cpu().numpy()                     # (batch, dim, 4, 2, N)
-    assert ck.shape == (2, 24, 4, 2, 16)
-    for k, end in enumerate([64, 128, 192, 200]):
+    ck = ckpt.cpu().numpy()                     # (batch, dim, 13, 2, N)
+    assert ck.shape == (2, 24, 13, 2, 16)
+    for k, end in enumerate(list(range(16, 200, 16)) + [200]):
         sub = {key: inp[key][..., :end] for key in ("x", "delta", "B", "C")}
         _, hr, vr = oracle.scan_seq(sub["x"], sub["delta"], inp["A"], sub["B"], sub["C"],
                                     h0=inp["h0"].astype(np.float64), v0=inp["v0"].astype(np.float64),
