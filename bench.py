@@ -52,8 +52,10 @@ L2_BYTES = 126e6
 
 WORKLOADS = {w.name: w for w in wl.SCAN_WORKLOADS}
 WORKLOADS[wl.SSD_MH.name] = wl.SSD_MH
+WORKLOADS[wl.DECODE.name] = wl.DECODE
 ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
-           "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name, "ssd": wl.SSD_MH.name}
+           "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name, "ssd": wl.SSD_MH.name,
+           "decode": wl.DECODE.name}
 DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
 IO_KEYS = ("x", "delta", "B", "C", "z")          # tensors in the workload's storage type
 GATED_EXTRAS = "D skip, z SiLU gate, delta_bias, softplus"
@@ -257,6 +259,141 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
             line["cpu_baseline"] = bwd_cpu_baseline(w, beta, alpha)
         print(json.dumps(line), flush=True)
     return 0
+
+
+def decode_bytes(w: wl.DecodeWorkload) -> int:
+    """Bytes one decode step must move: the cached h, v read and written
+    once; x, delta, z read and y written; B, C; A, D, delta_bias."""
+    eb = 4 if w.io == "f32" else 2
+    bd = w.batch * w.dim
+    return 4 * bd * w.dstate * 4 + 4 * bd * eb + 2 * w.batch * w.dstate * eb + w.dim * w.dstate * 4 \
+        + 2 * w.dim * 4
+
+
+def run_decode(args, w, rank, world):
+    """Time mm_scan_step (one decode step for every request) on resident
+    inputs and cached states; e2e adds the host copies of the step's inputs
+    (x, delta, z, B, C) and of y back: the states stay on the device."""
+    import torch
+    import selective_state_space_momentum_b200 as mm
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = wl.decode_inputs(w, seed=rank_seed(w.seed_index, rank))
+    iodt = torch.float32 if w.io == "f32" else torch.bfloat16
+    io_keys = ("x", "delta", "z", "B", "C")
+    host = {k: torch.from_numpy(v).to(iodt if k in io_keys else torch.float32) for k, v in inp.items()}
+    step_bytes = decode_bytes(w)
+    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    sets = []
+    for _ in range(nsets):
+        s = {k: v.to(dev).contiguous() for k, v in host.items()}
+        s["y"] = torch.empty_like(s["x"])
+        sets.append(s)
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        mm.mm_scan_step(s["x"], s["delta"], s["A"], s["B"], s["C"], s["D"], s["z"], s["delta_bias"], True,
+                        s["h"], s["v"], w.beta, w.alpha, s["y"], stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for i in range(args.warmup):
+        step(sets[i % nsets])
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(sets[i % nsets])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
+    value = whole_job_rate(w.updates, world, ms_step)
+
+    e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
+    pinned = {k: host[k].pin_memory() for k in io_keys}
+    yhost = torch.empty(tuple(inp["x"].shape), dtype=iodt, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = yhost.numel() * yhost.element_size()
+    s0 = sets[0]
+
+    def e2e_step():
+        d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        mm.mm_scan_step(d["x"], d["delta"], s0["A"], d["B"], d["C"], s0["D"], d["z"], s0["delta_bias"], True,
+                        s0["h"], s0["v"], w.beta, w.alpha, s0["y"], stream)
+        yhost.copy_(s0["y"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    barrier()
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        achieved = step_bytes / (ms_step * 1e-3) / 1e9
+        line = {
+            "metric": "decode-step state updates/s (B·D·N per step) and % of roofline, 1×B200",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.io, "data": "synthetic",
+            "config": {"workload": w.name, "pass": "decode step", "batch": w.batch, "seq_len": 1,
+                       "dim": w.dim, "dstate": w.dstate, "beta": w.beta, "alpha": w.alpha, "io": w.io,
+                       "extras": GATED_EXTRAS, "global_batch": w.batch * world,
+                       "parallelism": f"dp{world}",
+                       "l2": f"{nsets} rotating state sets ({nsets * step_bytes / 2e6:.0f} MB) > 126 MB L2"},
+            "roofline": {"bound": "hbm", "kernel": "scan_step_kernel", "achieved": achieved,
+                         "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                         "traffic": measured_traffic("scan_step_kernel", w.name),
+                         "peak_source": f"{peak_kind} copy bandwidth", "algorithmic_bytes": step_bytes},
+            "e2e": {"value": whole_job_rate(w.updates, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = decode_cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def decode_cpu_baseline(w: wl.DecodeWorkload, budget_s: float = 12.0):
+    """The fp64 oracle (one-step gated scan) on whole decode steps of the
+    workload, as many as fit the CPU-time budget (at least one)."""
+    import oracle
+    inp = wl.decode_inputs(w)
+    col = lambda a: a[..., None]
+    cores = oracle.num_threads()
+
+    def run():
+        oracle.scan_gated(col(inp["x"]), col(inp["delta"]), inp["A"], col(inp["B"]), col(inp["C"]),
+                          D=inp["D"], z=col(inp["z"]), delta_bias=inp["delta_bias"], delta_softplus=True,
+                          h0=inp["h"].astype(np.float64), v0=inp["v"].astype(np.float64),
+                          beta=w.beta, alpha=w.alpha)
+
+    t = time.perf_counter()
+    run()
+    one = time.perf_counter() - t
+    reps = max(1, min(20, int(budget_s / max(cores, 1) / max(one, 1e-9))))
+    t = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = time.perf_counter() - t
+    return {"value": reps * w.updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{reps} whole decode step(s) of {w.batch} requests, fp64, {dt:.2f} s wall on {cores} threads"}
 
 
 # ------------------------------------------------------------ clocks -------
@@ -642,8 +779,25 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[ALIASES.get(args.workload, args.workload)]
-    if (args.gated or args.backward) and isinstance(w, wl.SSDWorkload):
+    if (args.gated or args.backward) and not isinstance(w, wl.ScanWorkload):
         ap.error("--gated and --backward apply to the scan workloads")
+    if isinstance(w, wl.DecodeWorkload):
+        if args.impl == "reference":
+            ap.error("--impl reference times the forward scan")
+        import torch
+        rank, world, local = dist_env()
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            torch.cuda.set_device(0)
+        rc = run_decode(args, w, rank, world)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
     if args.gated and args.backward:
         ap.error("--backward times the plain scan's backward")
     if args.backward and args.impl == "reference":

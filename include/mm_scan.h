@@ -207,6 +207,37 @@ mm_status mm_scan_bwd(const void *x, const void *delta, const float *A,
                       float *dh0, float *dv0,
                       const mm_scan_dims *dims, void *stream);
 
+/*
+ * mm_scan_step -- one decode step on cached states, updated in place: the
+ * Mamba module's step() ("Momentum Mamba: Enhanced State Space Models with
+ * Momentum", section "Mamba Module": ssm_state and velocity_state carried
+ * from call to call) for the scan part of a layer.  It is mm_scan_fwd_gated
+ * with seqlen 1, (h0, v0) = (hT, vT) = (h, v):
+ *
+ *   delta' = softplus(delta + delta_bias)   (each part optional, as there)
+ *   v = beta v + alpha delta' B[n] x,   h = exp(delta' A[d,n]) h + v
+ *   y = (sum_n C[n] h + D[d] x) * z * sigmoid(z)
+ *
+ *   x, delta, z, y (batch, dim) io; B, C (batch, dstate) io; A (dim, dstate),
+ *   D, delta_bias (dim) fp32 (D, z, delta_bias may be NULL); h, v (batch,
+ *   dim, dstate) fp32, read and overwritten.  dims->seqlen must be 1.
+ *
+ * The per-state operations are those of mm_scan_fwd in the same order, so L
+ * steps leave (h, v) bit-identical to one mm_scan_fwd_gated call over the L
+ * steps from the same start (y agrees within rounding of the read-out).
+ * No output (h, v, y) may overlap an input or another output.
+ *
+ * Errors: MM_ERR_NULL, MM_ERR_DIMS (a size < 1 or seqlen != 1),
+ * MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE, MM_ERR_SCALAR,
+ * MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA.
+ */
+mm_status mm_scan_step(const void *x, const void *delta, const float *A,
+                       const void *B, const void *C,
+                       const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus,
+                       float *h, float *v, float beta, float alpha, void *y,
+                       const mm_scan_dims *dims, void *stream);
+
 /* Sizes of one Mamba-2 SSD call. */
 typedef struct {
     int64_t batch;    /* b                                                  */

@@ -24,7 +24,7 @@ import threading
 
 __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
-    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_ssd_fwd",
+    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_step", "mm_ssd_fwd",
     "mm_ssd_workspace_size", "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
@@ -46,7 +46,7 @@ STATUS_NAMES = {
 }
 
 # Every function include/mm_scan.h declares.
-EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd",
+EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_step",
                     "mm_ssd_workspace_size", "mm_ssd_fwd",
                     "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
@@ -86,6 +86,9 @@ def _declare(lib):
                                       vp, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
     lib.mm_scan_ckpt_size.restype = ctypes.c_int
     lib.mm_scan_ckpt_size.argtypes = [ctypes.POINTER(ScanDims), ctypes.POINTER(ctypes.c_size_t)]
+    lib.mm_scan_step.restype = ctypes.c_int
+    lib.mm_scan_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, f, f, vp,
+                                 ctypes.POINTER(ScanDims), vp]
     lib.mm_scan_bwd.restype = ctypes.c_int
     lib.mm_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp,
                                 vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
@@ -277,6 +280,24 @@ def scan_fwd(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0,
         mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
                           y, hT, vT, None, stream)
     return y, hT, vT
+
+
+def mm_scan_step(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h, v, beta, alpha, y,
+                 stream=None):
+    """C entry point mm_scan_step (marshalling only): one decode step.
+
+    x, delta, z, y (batch, dim) and B, C (batch, N) in one storage type; A
+    (dim, N), D, delta_bias (dim,) fp32; h, v (batch, dim, N) fp32, updated
+    in place.
+    """
+    batch, dim = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, 1, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_step(
+        _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if delta_softplus else 0, _ptr(h), _ptr(v), float(beta), float(alpha), _ptr(y),
+        ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_step")
 
 
 def scan_fwd_train(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, stream=None):

@@ -285,6 +285,46 @@ mm_status mm_scan_bwd(const void* x, const void* delta, const float* A, const vo
                      "mm_scan_bwd launch");
 }
 
+mm_status mm_scan_step(const void* x, const void* delta, const float* A, const void* B, const void* C,
+                       const float* Dskip, const void* z, const float* delta_bias, int delta_softplus,
+                       float* h, float* v, float beta, float alpha, void* y, const mm_scan_dims* dims,
+                       void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !h || !v || !y)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C, h, v and y are required");
+    if (dims->seqlen != 1) return fail(MM_ERR_DIMS, "a decode step has seqlen 1 (got %lld)",
+                                       (long long)dims->seqlen);
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
+    const void* ptrs[] = {x, delta, A, B, C, Dskip, z, delta_bias, h, v, y};
+    const char* names[] = {"x", "delta", "A", "B", "C", "D", "z", "delta_bias", "h", "v", "y"};
+    for (int i = 0; i < 11; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    const Range in_r[] = {rng("x", x, zs.seq_bytes), rng("delta", delta, zs.seq_bytes),
+                          rng("A", A, zs.a_bytes), rng("B", B, zs.bc_bytes), rng("C", C, zs.bc_bytes),
+                          rng("D", Dskip, zs.d_bytes), rng("z", z, zs.seq_bytes),
+                          rng("delta_bias", delta_bias, zs.d_bytes)};
+    const Range out_r[] = {rng("h", h, zs.st_bytes), rng("v", v, zs.st_bytes), rng("y", y, zs.seq_bytes)};
+    for (const Range& o : out_r) {
+        for (const Range& in : in_r)
+            if (overlap(o, in)) return fail(MM_ERR_ALIAS, "%s overlaps %s", o.name, in.name);
+        for (const Range& o2 : out_r)
+            if (&o2 != &o && overlap(o, o2)) return fail(MM_ERR_ALIAS, "%s overlaps %s", o.name, o2.name);
+    }
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+    mmscan::ScanStepArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C;
+    a.Dskip = Dskip; a.z = z; a.dbias = delta_bias; a.softplus = delta_softplus ? 1 : 0;
+    a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
+    a.h = h; a.v = v; a.y = y;
+    a.batch = dims->batch; a.dim = dims->dim; a.dstate = (int)dims->dstate;
+    a.vec = (dims->dstate % 4) == 0;
+    a.beta = beta; a.alpha = alpha;
+    return from_cuda(mmscan::launch_scan_step(a, dims->io, static_cast<cudaStream_t>(stream)),
+                     "mm_scan_step launch");
+}
+
 mm_status mm_ssd_workspace_size(const mm_ssd_dims* dims, size_t* bytes) {
     if (!dims || !bytes) return fail(MM_ERR_NULL, "dims and bytes are required");
     if (dims->batch < 1 || dims->seqlen < 1 || dims->nheads < 1 || dims->headdim < 1 ||

@@ -61,6 +61,27 @@ struct ScanBwdArgs {
     int vec_ok;            // rows of L elements are whole 16-byte pieces
 };
 
+// Arguments of one decode step (device pointers; states updated in place).
+struct ScanStepArgs {
+    const void* x;         // (batch, dim) io
+    const void* delta;     // (batch, dim) io
+    const float* A;        // (dim, dstate)
+    const void* B;         // (batch, dstate) io
+    const void* C;
+    const float* Dskip;    // (dim) or null
+    const void* z;         // (batch, dim) io, or null
+    const float* dbias;    // (dim) or null
+    int softplus;
+    int ext;               // any of the four extras is present
+    float* h;              // (batch, dim, dstate) fp32, read and written
+    float* v;
+    void* y;               // (batch, dim) io
+    int64_t batch, dim;
+    int dstate;
+    int vec;               // dstate is a multiple of 4: 16-byte state accesses
+    float beta, alpha;
+};
+
 struct ScanTileChoice {
     int np;      // states padded to a power of two (2, 4, 8, 16)
     int spt;     // states per lane (2 or 4)
@@ -73,6 +94,7 @@ ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int 
                                 int forced_spt, int forced_warps, int forced_ts);
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s);
 cudaError_t launch_scan_bwd(const ScanBwdArgs& a, int io, cudaStream_t s);
+cudaError_t launch_scan_step(const ScanStepArgs& a, int io, cudaStream_t s);
 // Read (and reset) the device error word of the scan / SSD kernels.
 unsigned int scan_read_and_clear_device_error();
 unsigned int scan_bwd_read_and_clear_device_error();

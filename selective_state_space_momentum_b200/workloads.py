@@ -131,6 +131,25 @@ class SSDWorkload:
         return self.batch * self.seqlen * self.nheads * self.headdim * self.dstate
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Single-token decode: one recurrence step for `batch` requests on their
+    cached states (the Mamba module's step()), with the selective_scan_fn
+    extras (delta bias and softplus, D skip, z gate) a Mamba layer applies."""
+    name: str
+    batch: int
+    dim: int
+    dstate: int
+    io: str = "bf16"                    # x, delta, z, B, C, y; the states are fp32
+    beta: float = 0.9
+    alpha: float = 1.0
+    seed_index: int = 5
+
+    @property
+    def updates(self) -> int:
+        return self.batch * self.dim * self.dstate
+
+
 SCAN_SMALL = ScanWorkload("scan_f32_b1_l256_d64_n16", 1, 256, 64, 16,
                           runs=((0.9, 1.0), (0.0, 1.0)), seed_index=0)
 SCAN_MEDIUM = ScanWorkload("scan_f32_b4_l2048_d1536_n16", 4, 2048, 1536, 16,
@@ -144,6 +163,8 @@ SCAN_LONG = ScanWorkload("scan_f32_b1_l131072_d2048_n16_stream", 1, 131072, 2048
                          runs=((0.99, 1.0),), split=65536, seed_index=3)
 SSD_MH = SSDWorkload("ssd_bf16_b4_l4096_h32_p64_n128_g1_q256", 4, 4096, 32, 64, 128, 1, 256,
                      seed_index=4)
+
+DECODE = DecodeWorkload("decode_bf16_b512_d2048_n16", 512, 2048, 16)
 
 SCAN_WORKLOADS = (SCAN_SMALL, SCAN_MEDIUM, SCAN_BF16, SCAN_LONG)
 
@@ -238,3 +259,36 @@ def ssd_inputs(w: SSDWorkload, *, batch: int | None = None, seqlen: int | None =
     B = bf16_round(_normal(rb, (bsz, L, G, N), 1.0 / math.sqrt(N)))
     C = bf16_round(_normal(rc, (bsz, L, G, N), 1.0 / math.sqrt(N)))
     return {"x": x, "delta": delta, "A": A, "B": B, "C": C}
+
+
+def decode_inputs(w: DecodeWorkload, *, batch: int | None = None, dim: int | None = None,
+                  dstate: int | None = None, seed: int | None = None):
+    """Draw one decode step's inputs and cached states.
+
+    Layouts: x, delta, z (batch, dim); B, C (batch, N); A (dim, N); D,
+    delta_bias (dim); h, v (batch, dim, N) fp32.  Laws as the scan workloads
+    and their extras: x, z ~ N(0, 1); a raw delta ~ N(0, 0.5) fed with
+    delta_bias = ln(expm1(dt)), dt log-uniform on [1e-3, 1e-1]; A = -(n + 1)
+    U(0.5, 2) per channel; B, C ~ N(0, 1/4); D ~ U(0.5, 1.5); the cached
+    states h ~ N(0, 1), v ~ N(0, 0.1).  bf16 tensors hold bf16-rounded values.
+    """
+    bsz = batch or w.batch
+    D = dim or w.dim
+    N = dstate or w.dstate
+    rx, rd, ra, rb, rc, rbias, rs, rz, rh, rv = _streams(
+        seed if seed is not None else seed_of(w.seed_index), 10)
+    x = _normal(rx, (bsz, D))
+    delta = _normal(rd, (bsz, D), 0.5)
+    A = ((ra.uniform(0.5, 2.0, size=D)[:, None]) * -(np.arange(N, dtype=np.float64) + 1.0)[None, :])
+    B = _normal(rb, (bsz, N), 0.25)
+    C = _normal(rc, (bsz, N), 0.25)
+    dt = _log_uniform(rbias, (D,), 1e-3, 1e-1).astype(np.float64)
+    bias = np.log(np.expm1(dt)).astype(np.float32)
+    Dskip = rs.uniform(0.5, 1.5, D).astype(np.float32)
+    z = _normal(rz, (bsz, D))
+    h = _normal(rh, (bsz, D, N))
+    v = _normal(rv, (bsz, D, N), 0.1)
+    if w.io == "bf16":
+        x, delta, B, C, z = (bf16_round(t) for t in (x, delta, B, C, z))
+    return {"x": x, "delta": delta, "A": np.ascontiguousarray(A.astype(np.float32)), "B": B, "C": C,
+            "D": Dskip, "z": z, "delta_bias": bias, "h": h, "v": v}

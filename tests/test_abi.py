@@ -164,6 +164,24 @@ def test_bwd_checks_its_arguments(lib, monkeypatch):
     assert rc == 7                                                # one block: no checkpoint needed
 
 
+def test_step_checks_its_arguments(lib, monkeypatch):
+    def call(L=1, **over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), D=None, z=None,
+                 bias=None, sp=0, h=_fake(5), v=_fake(6), y=_fake(7), beta=0.9)
+        a.update(over)
+        return lib.mm_scan_step(a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                                a["sp"], a["h"], a["v"], a["beta"], 1.0, a["y"],
+                                ctypes.byref(D(batch=4, L=L, dim=64)), None)
+    assert call(h=None) == 1
+    assert call(L=2) == 2                                         # a step is one time step
+    assert call(beta=-0.1) == 3
+    assert call(z=ctypes.c_void_p(A16 * 9 + 8)) == 5
+    assert call(y=_fake(0)) == 9                                  # output over an input
+    assert call(v=_fake(5)) == 9                                  # h and v on one buffer
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call(D=_fake(8), z=_fake(9), bias=_fake(10), sp=1) == 7
+
+
 def test_set_tile(lib):
     assert lib.mm_scan_set_tile(3, 2, 1) == 6
     assert lib.mm_scan_set_tile(4, 2, 3) == 6
