@@ -208,6 +208,37 @@ mm_status mm_scan_bwd(const void *x, const void *delta, const float *A,
                       const mm_scan_dims *dims, void *stream);
 
 /*
+ * mm_scan_bwd_gated -- gradients of mm_scan_fwd_gated: mm_scan_bwd through
+ * the extras, with dy now the gradient reaching the gated output.  With
+ * o_t = y_t + D x_t and s_t = sigmoid(z_t), delta'_t = softplus(delta_t +
+ * bias):
+ *
+ *   the scan's read-out receives dy_t z_t s_t (dy_t without the gate);
+ *   dx_t     += D dy_t z_t s_t                     (the skip)
+ *   dz_t      = dy_t o_t s_t (1 + z_t (1 - s_t))
+ *   dD        = sum over b, t of dy_t z_t s_t x_t
+ *   ddelta_t  = (ddelta'_t of mm_scan_bwd) * sigmoid(delta_t + bias)  (softplus;
+ *               else ddelta'_t),   ddelta_bias = sum over b, t of ddelta_t
+ *
+ * Inputs as given to mm_scan_fwd_gated (ckpt as it wrote it).  Extra
+ * outputs (overwritten; NULL: not formed): dD, ddelta_bias (dim) fp32,
+ * summed with atomics like dA; dz (batch, dim, L) io.  Aliasing, alignment
+ * and errors as mm_scan_bwd; with D, z, delta_bias NULL and delta_softplus
+ * 0 this is mm_scan_bwd.
+ */
+mm_status mm_scan_bwd_gated(const void *x, const void *delta, const float *A,
+                            const void *B, const void *C,
+                            const float *D, const void *z,
+                            const float *delta_bias, int delta_softplus,
+                            const float *h0, const float *v0, float beta, float alpha,
+                            const float *ckpt, const void *dy,
+                            const float *dhT, const float *dvT,
+                            void *dx, void *ddelta, float *dA, float *dB, float *dC,
+                            float *dD, void *dz, float *ddelta_bias,
+                            float *dh0, float *dv0,
+                            const mm_scan_dims *dims, void *stream);
+
+/*
  * mm_scan_step -- one decode step on cached states, updated in place: the
  * Mamba module's step() ("Momentum Mamba: Enhanced State Space Models with
  * Momentum", section "Mamba Module": ssm_state and velocity_state carried

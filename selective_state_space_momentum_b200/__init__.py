@@ -24,7 +24,8 @@ import threading
 
 __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
-    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_step", "mm_ssd_fwd",
+    "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_bwd_gated",
+    "mm_scan_step", "mm_ssd_fwd",
     "mm_ssd_workspace_size", "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
@@ -46,7 +47,8 @@ STATUS_NAMES = {
 }
 
 # Every function include/mm_scan.h declares.
-EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_step",
+EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd",
+                    "mm_scan_bwd_gated", "mm_scan_step",
                     "mm_ssd_workspace_size", "mm_ssd_fwd",
                     "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
@@ -89,6 +91,10 @@ def _declare(lib):
     lib.mm_scan_step.restype = ctypes.c_int
     lib.mm_scan_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, f, f, vp,
                                  ctypes.POINTER(ScanDims), vp]
+    lib.mm_scan_bwd_gated.restype = ctypes.c_int
+    lib.mm_scan_bwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, f, f, vp, vp,
+                                      vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                      ctypes.POINTER(ScanDims), vp]
     lib.mm_scan_bwd.restype = ctypes.c_int
     lib.mm_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp,
                                 vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
@@ -300,9 +306,27 @@ def mm_scan_step(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h, v, beta
     _check(rc, "mm_scan_step")
 
 
-def scan_fwd_train(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, stream=None):
+def mm_scan_bwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
+                      ckpt, dy, dhT, dvT, dx, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0, dv0,
+                      stream=None):
+    """C entry point mm_scan_bwd_gated (marshalling only): mm_scan_bwd through
+    D, z, delta_bias and softplus, with the extra outputs dD, dz, ddelta_bias."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_bwd_gated(
+        _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if delta_softplus else 0, _ptr(h0), _ptr(v0), float(beta), float(alpha), _ptr(ckpt), _ptr(dy),
+        _ptr(dhT), _ptr(dvT), _ptr(dx), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz),
+        _ptr(ddelta_bias), _ptr(dh0), _ptr(dv0), ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_bwd_gated")
+
+
+def scan_fwd_train(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, stream=None,
+                   D=None, z=None, delta_bias=None, delta_softplus=False):
     """Forward that also keeps the checkpoints the backward restarts from:
-    returns (y, hT, vT, ckpt), ckpt (batch, dim, ceil(L / 16), 2, N) fp32."""
+    returns (y, hT, vT, ckpt), ckpt (batch, dim, ceil(L / 16), 2, N) fp32.
+    D, z, delta_bias, delta_softplus as for scan_fwd."""
     import torch
     batch, dim, L = x.shape
     N = A.shape[1]
@@ -311,15 +335,16 @@ def scan_fwd_train(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, str
     vT = torch.empty_like(hT)
     ckpt = torch.empty((batch, dim, (L + MM_SCAN_CKPT_STEPS - 1) // MM_SCAN_CKPT_STEPS, 2, N), device=x.device,
                        dtype=torch.float32)
-    mm_scan_fwd_gated(x, delta, A, B, C, None, None, None, False, h0, v0, beta, alpha, y, hT, vT,
+    mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha, y, hT, vT,
                       ckpt, stream)
     return y, hT, vT, ckpt
 
 
 def scan_bwd(x, delta, A, B, C, ckpt, dy, h0=None, v0=None, dhT=None, dvT=None, beta=0.9,
-             alpha=1.0, stream=None):
-    """Allocate the gradients and run mm_scan_bwd; returns a dict with dx,
-    ddelta, dA, dB, dC, dh0, dv0."""
+             alpha=1.0, stream=None, D=None, z=None, delta_bias=None, delta_softplus=False):
+    """Allocate the gradients and run mm_scan_bwd (mm_scan_bwd_gated when any
+    of D, z, delta_bias, delta_softplus is given); returns a dict with dx,
+    ddelta, dA, dB, dC, dh0, dv0 and, with the extras, dD, dz, ddelta_bias."""
     import torch
     batch, dim, L = x.shape
     N = A.shape[1]
@@ -327,8 +352,16 @@ def scan_bwd(x, delta, A, B, C, ckpt, dy, h0=None, v0=None, dhT=None, dvT=None, 
     g = {"dx": torch.empty_like(x), "ddelta": torch.empty_like(x), "dA": torch.empty((dim, N), **f32),
          "dB": torch.empty((batch, N, L), **f32), "dC": torch.empty((batch, N, L), **f32),
          "dh0": torch.empty((batch, dim, N), **f32), "dv0": torch.empty((batch, dim, N), **f32)}
-    mm_scan_bwd(x, delta, A, B, C, h0, v0, beta, alpha, ckpt, dy, dhT, dvT, g["dx"], g["ddelta"],
-                g["dA"], g["dB"], g["dC"], g["dh0"], g["dv0"], stream)
+    if D is None and z is None and delta_bias is None and not delta_softplus:
+        mm_scan_bwd(x, delta, A, B, C, h0, v0, beta, alpha, ckpt, dy, dhT, dvT, g["dx"], g["ddelta"],
+                    g["dA"], g["dB"], g["dC"], g["dh0"], g["dv0"], stream)
+        return g
+    g["dD"] = torch.empty((dim,), **f32)
+    g["ddelta_bias"] = torch.empty((dim,), **f32)
+    g["dz"] = torch.empty_like(x) if z is not None else None
+    mm_scan_bwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha, ckpt, dy,
+                      dhT, dvT, g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"],
+                      g["ddelta_bias"], g["dh0"], g["dv0"], stream)
     return g
 
 

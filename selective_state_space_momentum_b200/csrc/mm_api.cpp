@@ -243,6 +243,18 @@ mm_status mm_scan_bwd(const void* x, const void* delta, const float* A, const vo
                       const void* dy, const float* dhT, const float* dvT, void* dx, void* ddelta,
                       float* dA, float* dB, float* dC, float* dh0, float* dv0,
                       const mm_scan_dims* dims, void* stream) {
+    return mm_scan_bwd_gated(x, delta, A, B, C, nullptr, nullptr, nullptr, 0, h0, v0, beta, alpha, ckpt,
+                             dy, dhT, dvT, dx, ddelta, dA, dB, dC, nullptr, nullptr, nullptr, dh0, dv0,
+                             dims, stream);
+}
+
+mm_status mm_scan_bwd_gated(const void* x, const void* delta, const float* A, const void* B,
+                            const void* C, const float* Dskip, const void* z, const float* delta_bias,
+                            int delta_softplus, const float* h0, const float* v0, float beta, float alpha,
+                            const float* ckpt, const void* dy, const float* dhT, const float* dvT,
+                            void* dx, void* ddelta, float* dA, float* dB, float* dC, float* dD,
+                            void* dz, float* ddelta_bias, float* dh0, float* dv0,
+                            const mm_scan_dims* dims, void* stream) {
     if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
     if (!x || !delta || !A || !B || !C || !dy || !dx || !ddelta || !dA || !dB || !dC)
         return fail(MM_ERR_NULL, "x, delta, A, B, C, dy, dx, ddelta, dA, dB and dC are required");
@@ -251,21 +263,26 @@ mm_status mm_scan_bwd(const void* x, const void* delta, const float* A, const vo
     const int64_t L = dims->seqlen;
     if (!ckpt && L > MM_SCAN_CKPT_STEPS)
         return fail(MM_ERR_NULL, "ckpt is required when seqlen > %d", MM_SCAN_CKPT_STEPS);
-    const void* ptrs[] = {x, delta, A, B, C, h0, v0, ckpt, dy, dhT, dvT, dx, ddelta, dA, dB, dC, dh0, dv0};
+    const void* ptrs[] = {x, delta, A, B, C, h0, v0, ckpt, dy, dhT, dvT, dx, ddelta, dA, dB, dC, dh0, dv0,
+                          Dskip, z, delta_bias, dD, dz, ddelta_bias};
     const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "ckpt", "dy", "dhT", "dvT",
-                           "dx", "ddelta", "dA", "dB", "dC", "dh0", "dv0"};
-    for (int i = 0; i < 18; ++i)
+                           "dx", "ddelta", "dA", "dB", "dC", "dh0", "dv0", "D", "z", "delta_bias",
+                           "dD", "dz", "ddelta_bias"};
+    for (int i = 0; i < 24; ++i)
         if (ptrs[i] && !aligned16(ptrs[i]))
             return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
     const Range in_r[] = {rng("x", x, zs.seq_bytes), rng("delta", delta, zs.seq_bytes),
                           rng("A", A, zs.a_bytes), rng("B", B, zs.bc_bytes), rng("C", C, zs.bc_bytes),
                           rng("h0", h0, zs.st_bytes), rng("v0", v0, zs.st_bytes),
                           rng("ckpt", ckpt, zs.ck_bytes), rng("dy", dy, zs.seq_bytes),
-                          rng("dhT", dhT, zs.st_bytes), rng("dvT", dvT, zs.st_bytes)};
+                          rng("dhT", dhT, zs.st_bytes), rng("dvT", dvT, zs.st_bytes),
+                          rng("D", Dskip, zs.d_bytes), rng("z", z, zs.seq_bytes),
+                          rng("delta_bias", delta_bias, zs.d_bytes)};
     const Range out_r[] = {rng("dx", dx, zs.seq_bytes), rng("ddelta", ddelta, zs.seq_bytes),
                            rng("dA", dA, zs.a_bytes), rng("dB", dB, zs.bcf_bytes),
                            rng("dC", dC, zs.bcf_bytes), rng("dh0", dh0, zs.st_bytes),
-                           rng("dv0", dv0, zs.st_bytes)};
+                           rng("dv0", dv0, zs.st_bytes), rng("dD", dD, zs.d_bytes),
+                           rng("dz", dz, zs.seq_bytes), rng("ddelta_bias", ddelta_bias, zs.d_bytes)};
     for (const Range& o : out_r) {
         for (const Range& in : in_r)
             if (overlap(o, in)) return fail(MM_ERR_ALIAS, "%s overlaps %s", o.name, in.name);
@@ -281,6 +298,11 @@ mm_status mm_scan_bwd(const void* x, const void* delta, const float* A, const vo
     a.batch = dims->batch; a.seqlen = L; a.dim = dims->dim; a.dstate = (int)dims->dstate;
     a.beta = beta; a.alpha = alpha;
     a.vec_ok = ((L * zs.esize) % 16) == 0;
+    a.Dskip = Dskip; a.z = z; a.dbias = delta_bias; a.softplus = delta_softplus ? 1 : 0;
+    a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
+    a.dD = a.ext ? dD : nullptr;
+    a.dz = z ? dz : nullptr;
+    a.ddbias = a.ext ? ddelta_bias : nullptr;
     return from_cuda(mmscan::launch_scan_bwd(a, dims->io, static_cast<cudaStream_t>(stream)),
                      "mm_scan_bwd launch");
 }

@@ -59,6 +59,15 @@ struct ScanBwdArgs {
     int tiles_per_batch;   // filled by the launcher
     float beta, alpha;
     int vec_ok;            // rows of L elements are whole 16-byte pieces
+    // selective_scan_fn extras (all absent for the plain scan's backward)
+    const float* Dskip;    // (dim) or null
+    const void* z;         // (batch, dim, L) io, or null
+    const float* dbias;    // (dim) or null
+    int softplus;
+    int ext;               // any of the four is present
+    float* dD;             // (dim), summed over batch and steps, or null
+    void* dz;              // (batch, dim, L) io, or null
+    float* ddbias;         // (dim), or null
 };
 
 // Arguments of one decode step (device pointers; states updated in place).

@@ -50,7 +50,7 @@ namespace mmscan {
 // Device error word of this file's kernel (bounded waits that gave up).
 static __device__ unsigned int g_bwd_dev_err = 0;
 
-template <typename IO, int NP, int WARPS>
+template <typename IO, int NP, int WARPS, bool EXT = false>
 struct BwdTile {
     static constexpr int SPT = 2;                // states per lane
     static constexpr int G = NP / SPT;           // lanes per channel
@@ -70,7 +70,8 @@ struct BwdTile {
     static constexpr int OFF_Y = 2 * NBOX * XBOX;     // dy, the gradient reaching y
     static constexpr int OFF_B = 3 * NBOX * XBOX;
     static constexpr int OFF_C = OFF_B + NBOX * BBOX;
-    static constexpr int STAGE_BYTES = OFF_C + NBOX * BBOX;
+    static constexpr int OFF_Z = OFF_C + NBOX * BBOX;       // the gate z (selective_scan_fn extras)
+    static constexpr int STAGE_BYTES = OFF_Z + (EXT ? NBOX * XBOX : 0);
     static constexpr int BP = NP + 4;            // row pitch (floats) of transposed B/C
     static constexpr int BT_BYTES = T * BP * 4;
     static constexpr int KB = kCkptSteps;        // steps per block (the checkpoint interval)
@@ -80,7 +81,13 @@ struct BwdTile {
     static constexpr int OFF_BT = STAGES * STAGE_BYTES;   // B^T, then C^T
     static constexpr int OFF_RED = OFF_BT + 2 * BT_BYTES;
     static constexpr int RED_BYTES = 2 * KB * RP * 4;   // two blocks' dB, dC partials
-    static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
+    // extras: delta' = softplus(delta + bias) and the gated dy = dy silu(z) of
+    // the chunk as fp32 in the fp32 box layout (32 steps x CH rows of 128 B)
+    static constexpr int XBOX_F32 = CH * 128;
+    static constexpr int EXB = EXT ? (T / 32) * XBOX_F32 : 0;
+    static constexpr int OFF_DP = OFF_RED + RED_BYTES;
+    static constexpr int OFF_GY = OFF_DP + EXB;
+    static constexpr int OFF_BAR = OFF_GY + EXB;
     static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
     // 12 resident warps per SM (<= 168 registers a thread, no spills).  Four
     // 4-warp CTAs would fit the shared memory, but at 128 registers the
@@ -95,12 +102,13 @@ struct BwdTile {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <typename IO, int NP, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, BwdTile<IO, NP, WARPS>::MIN_CTAS)
+template <typename IO, int NP, int WARPS, bool EXT>
+__global__ void __launch_bounds__(WARPS * 32, BwdTile<IO, NP, WARPS, EXT>::MIN_CTAS)
 scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_B,
-                const __grid_constant__ CUtensorMap tm_C, const ScanBwdArgs p) {
-    using TL = BwdTile<IO, NP, WARPS>;
+                const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_z,
+                const ScanBwdArgs p) {
+    using TL = BwdTile<IO, NP, WARPS, EXT>;
     constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
     constexpr int ST = TL::STAGES, EB = TL::EB, BP = TL::BP, PER = TL::PER, KB = TL::KB;
     constexpr int RP = TL::RP;
@@ -173,9 +181,10 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const int64_t t0 = k * T;
         const uint32_t sb = base + s * TL::STAGE_BYTES;
         const uint32_t bar = bar0 + 8 * s;
+        const bool load_z = EXT && p.z != nullptr;
         if (use_tma) {
             if (tid == 0) {
-                mbar_expect_tx(bar, TL::STAGE_BYTES);
+                mbar_expect_tx(bar, TL::STAGE_BYTES - (EXT && !load_z ? TL::NBOX * TL::XBOX : 0));
 #pragma unroll
                 for (int bx = 0; bx < TL::NBOX; ++bx) {
                     const int tc = (int)(t0 + bx * TL::BOX_T);
@@ -184,16 +193,18 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     tma_load_3d(sb + TL::OFF_Y + bx * TL::XBOX, &tm_y, bar, tc, (int)d0, (int)b);
                     tma_load_3d(sb + TL::OFF_B + bx * TL::BBOX, &tm_B, bar, tc, 0, (int)b);
                     tma_load_3d(sb + TL::OFF_C + bx * TL::BBOX, &tm_C, bar, tc, 0, (int)b);
+                    if (load_z) tma_load_3d(sb + TL::OFF_Z + bx * TL::XBOX, &tm_z, bar, tc, (int)d0, (int)b);
                 }
             }
             return;
         }
         // Element-wise fill of the same swizzled tiles (rows not 16-byte multiples).
-        const IO* srcs[3] = {static_cast<const IO*>(p.x), static_cast<const IO*>(p.delta),
-                             static_cast<const IO*>(p.dout)};
+        const IO* srcs[4] = {static_cast<const IO*>(p.x), static_cast<const IO*>(p.delta),
+                             static_cast<const IO*>(p.dout), static_cast<const IO*>(p.z)};
         const IO* Bg = static_cast<const IO*>(p.B);
         const IO* Cg = static_cast<const IO*>(p.C);
-        constexpr int ROWS = 3 * CH + 2 * TL::NPT;
+        constexpr int IOROWS = (EXT ? 4 : 3) * CH;
+        constexpr int ROWS = IOROWS + 2 * TL::NPT;
         for (int i = tid; i < ROWS * T; i += NT) {
             const int r = i / T;
             const int tau = i - r * T;
@@ -202,13 +213,13 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const int64_t t = t0 + tau;
             const IO* src = nullptr;
             uint32_t off;
-            if (r < 3 * CH) {
+            if (r < IOROWS) {
                 const int which = r / CH;
                 const int cc = r - which * CH;
-                off = which * TL::NBOX * TL::XBOX + bx * TL::XBOX + sw128(cc, col * EB);
-                if (d0 + cc < p.dim && t < L) src = srcs[which] + ((b * p.dim + d0 + cc) * L + t);
+                off = (which == 3 ? TL::OFF_Z : which * TL::NBOX * TL::XBOX) + bx * TL::XBOX + sw128(cc, col * EB);
+                if (srcs[which] && d0 + cc < p.dim && t < L) src = srcs[which] + ((b * p.dim + d0 + cc) * L + t);
             } else {
-                const int rr = r - 3 * CH;
+                const int rr = r - IOROWS;
                 const int n = rr < TL::NPT ? rr : rr - TL::NPT;
                 off = (rr < TL::NPT ? TL::OFF_B : TL::OFF_C) + bx * TL::BBOX + sw128(n, col * EB);
                 if (n < N && t < L) src = (rr < TL::NPT ? Bg : Cg) + ((b * N + n) * L + t);
@@ -230,6 +241,11 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     IO* dxrow = static_cast<IO*>(p.dx) + (b * p.dim + (active ? d : 0)) * L;
     IO* ddrow = static_cast<IO*>(p.ddelta) + (b * p.dim + (active ? d : 0)) * L;
+    // selective_scan_fn extras: skip weight, bias, and the per-channel sums dD, d bias
+    IO* dzrow = (EXT && p.dz) ? static_cast<IO*>(p.dz) + (b * p.dim + (active ? d : 0)) * L : nullptr;
+    const float skip_d = (EXT && p.Dskip && active) ? p.Dskip[d] : 0.0f;
+    const float dbias_d = (EXT && p.dbias && active) ? p.dbias[d] : 0.0f;
+    float acc_dD = 0.0f, acc_db = 0.0f;
     const bool vec_out = use_tma;
     const bool vec_red = (L % 4) == 0;
 
@@ -282,6 +298,34 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
         }
+        if constexpr (EXT) {
+            // delta' = softplus(delta + bias) and the gated dy = dy silu(z), once per
+            // (channel, step), four steps per item, into the fp32 buffers
+            for (int it = tid; it < CH * (T / 4); it += NT) {
+                const int cc = it / (T / 4);
+                const int t4 = (it - cc * (T / 4)) * 4;
+                const int bxs = t4 / TL::BOX_T;
+                const uint32_t so = bxs * TL::XBOX + sw128(cc, (t4 - bxs * TL::BOX_T) * EB);
+                const float4 dq = load4(reinterpret_cast<const IO*>(sbuf + TL::OFF_D + so));
+                const float4 yq = load4(reinterpret_cast<const IO*>(sbuf + TL::OFF_Y + so));
+                const float bv = (p.dbias && d0 + cc < p.dim) ? p.dbias[d0 + cc] : 0.0f;
+                float dv[4] = {dq.x + bv, dq.y + bv, dq.z + bv, dq.w + bv};
+                float gy[4] = {yq.x, yq.y, yq.z, yq.w};
+                if (p.softplus) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dv[e] = softplus_f32(dv[e]);
+                }
+                if (p.z) {
+                    const float4 zq = load4(reinterpret_cast<const IO*>(sbuf + TL::OFF_Z + so));
+                    const float zv[4] = {zq.x, zq.y, zq.z, zq.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) gy[e] *= __fdividef(zv[e], 1.0f + ex2_approx(-zv[e] * kLog2e));
+                }
+                const uint32_t fo = (t4 / 32) * TL::XBOX_F32 + sw128(cc, (t4 % 32) * 4);
+                *reinterpret_cast<float4*>(smem + TL::OFF_DP + fo) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+                *reinterpret_cast<float4*>(smem + TL::OFF_GY + fo) = make_float4(gy[0], gy[1], gy[2], gy[3]);
+            }
+        }
         __syncthreads();
         // Every thread is past the previous chunk: its stage is free.
         if (i + ST - 1 < nchunks) issue(nchunks - 1 - (i + ST - 1), (int)((i + ST - 1) % ST));
@@ -296,6 +340,25 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const int bx = tau / TL::BOX_T;
             const int col = tau - bx * TL::BOX_T;
             return load1(reinterpret_cast<const IO*>(sbuf + off + bx * TL::XBOX + sw128(c, col * EB)));
+        };
+        // delta' and the dy reaching the read-out (with the extras: the fp32 buffers)
+        auto ld_delta4 = [&](int tau) {
+            if constexpr (EXT)
+                return *reinterpret_cast<const float4*>(smem + TL::OFF_DP + (tau / 32) * TL::XBOX_F32 +
+                                                        sw128(c, (tau % 32) * 4));
+            else
+                return load4s(TL::OFF_D, tau);
+        };
+        auto ld_dy4 = [&](int tau) {
+            if constexpr (EXT)
+                return *reinterpret_cast<const float4*>(smem + TL::OFF_GY + (tau / 32) * TL::XBOX_F32 +
+                                                        sw128(c, (tau % 32) * 4));
+            else
+                return load4s(TL::OFF_Y, tau);
+        };
+        auto ld_f32 = [&](int off, int tau) {      // one value of an fp32 extras buffer
+            return *reinterpret_cast<const float*>(smem + off + (tau / 32) * TL::XBOX_F32 +
+                                                   sw128(c, (tau % 32) * 4));
         };
         // one forward step of the lane's two states (the forward kernel's operations)
         auto fwd_step = [&](int tau, float dl, float u, float2& h, float2& v, float2& a) {
@@ -343,7 +406,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
             for (int j4 = 0; j4 < KB; j4 += 4) {
                 if (j4 < kmax) {
-                    const float4 dq = load4s(TL::OFF_D, tb + j4);
+                    const float4 dq = ld_delta4(tb + j4);
                     const float4 xq = load4s(TL::OFF_X, tb + j4);
                     const float dl[4] = {dq.x, dq.y, dq.z, dq.w}, xl[4] = {xq.x, xq.y, xq.z, xq.w};
 #pragma unroll
@@ -357,7 +420,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
             for (int hf = KB / R - 1; hf >= 0; --hf) {
                 if (hf * R >= kmax) continue;
-                float sk[R], qk[R];
+                float sk[R], qk[R], yk[EXT ? R : 1];
 #pragma unroll
                 for (int j4 = R - 4; j4 >= 0; j4 -= 4) {
                     const int jb = hf * R + j4;              // first of these 4 steps in the block
@@ -365,12 +428,13 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         sk[j4 + jj] = qk[j4 + jj] = 0.0f;
+                        if constexpr (EXT) yk[j4 + jj] = 0.0f;
                         dBv[jj] = dCv[jj] = f2(0.0f, 0.0f);
                     }
                     if (jb < kmax) {
-                        const float4 dq = load4s(TL::OFF_D, tb + jb);
+                        const float4 dq = ld_delta4(tb + jb);
                         const float4 xq = load4s(TL::OFF_X, tb + jb);
-                        const float4 yq = load4s(TL::OFF_Y, tb + jb);
+                        const float4 yq = ld_dy4(tb + jb);
                         const float dl[4] = {dq.x, dq.y, dq.z, dq.w}, xl[4] = {xq.x, xq.y, xq.z, xq.w};
                         const float yl[4] = {yq.x, yq.y, yq.z, yq.w};
 #pragma unroll
@@ -394,6 +458,10 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                 const float ua = dl[jj] * xl[jj] * alpha;
                                 dBv[jj] = __fmul2_rn(Pt, f2(ua, ua));
                                 dCv[jj] = __fmul2_rn(f2(yl[jj], yl[jj]), ht[j]);
+                                if constexpr (EXT) {     // the read-out itself, for dz
+                                    const float2 cy = __fmul2_rn(cq, ht[j]);
+                                    yk[j4 + jj] = cy.x + cy.y;
+                                }
                                 cg = __fmul2_rn(at, Gt);
                                 cp = __fmul2_rn(beta2, Pt);
                             }
@@ -408,10 +476,40 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const int first = tb + hf * R + g * PER;
                 const int cnt = nval - first < PER ? nval - first : PER;
                 float gx[PER], gd[PER];
+                if constexpr (!EXT) {
 #pragma unroll
-                for (int e = 0; e < PER; ++e) {
-                    gx[e] = load1s(TL::OFF_D, first + e) * so[e];
-                    gd[e] = __fmaf_rn(load1s(TL::OFF_X, first + e), so[e], qo[e]);
+                    for (int e = 0; e < PER; ++e) {
+                        gx[e] = load1s(TL::OFF_D, first + e) * so[e];
+                        gd[e] = __fmaf_rn(load1s(TL::OFF_X, first + e), so[e], qo[e]);
+                    }
+                } else {
+                    float yo[PER], gz[PER];
+                    if (p.z) butterfly_sum<G, R>(yk, yo, g);
+#pragma unroll
+                    for (int e = 0; e < PER; ++e) {
+                        const int st = first + e;
+                        const bool valid = e < cnt;
+                        const float xe = load1s(TL::OFF_X, st);
+                        const float gye = ld_f32(TL::OFF_GY, st);
+                        gx[e] = __fmaf_rn(skip_d, gye, ld_f32(TL::OFF_DP, st) * so[e]);
+                        gd[e] = __fmaf_rn(xe, so[e], qo[e]);          // d delta'
+                        if (p.softplus) {                             // * sigmoid(delta + bias)
+                            const float uu = load1s(TL::OFF_D, st) + dbias_d;
+                            gd[e] *= __fdividef(1.0f, 1.0f + ex2_approx(-uu * kLog2e));
+                        }
+                        if (valid) {
+                            acc_dD = __fmaf_rn(gye, xe, acc_dD);
+                            acc_db += gd[e];
+                        }
+                        if (p.z) {          // dz = dy (y + D x) s (1 + z (1 - s)), s = sigmoid(z)
+                            const float zv = load1s(TL::OFF_Z, st);
+                            const float sg = __fdividef(1.0f, 1.0f + ex2_approx(-zv * kLog2e));
+                            const float o = __fmaf_rn(skip_d, xe, yo[e]);
+                            gz[e] = load1s(TL::OFF_Y, st) * o * sg * __fmaf_rn(zv, 1.0f - sg, 1.0f);
+                        }
+                    }
+                    if (p.z && p.dz && active && cnt > 0)
+                        store_steps_n<IO, PER>(dzrow + t0 + first, gz, cnt, vec_out);
                 }
                 if (active && cnt > 0) {
                     store_steps_n<IO, PER>(dxrow + t0 + first, gx, cnt, vec_out);
@@ -461,6 +559,19 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
     }
 
+    // ---- dD, d bias: this lane's steps, then the G lanes of the channel ----------
+    if constexpr (EXT) {
+#pragma unroll
+        for (int m = G / 2; m >= 1; m >>= 1) {
+            acc_dD += __shfl_xor_sync(0xffffffffu, acc_dD, m);
+            acc_db += __shfl_xor_sync(0xffffffffu, acc_db, m);
+        }
+        if (active && g == 0) {
+            if (p.dD) atomicAdd(p.dD + d, acc_dD);
+            if (p.ddbias) atomicAdd(p.ddbias + d, acc_db);
+        }
+    }
+
     // ---- gradients of the start state; dA ------------------------------------
     if (active) {
         const float gh[2] = {cg.x, cg.y}, gv[2] = {cp.x, cp.y}, ga[2] = {dA2.x, dA2.y};
@@ -479,17 +590,17 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 // ------------------------------------------------------------- launch -----
 namespace {
 
-template <typename IO, int NP, int WARPS>
+template <typename IO, int NP, int WARPS, bool EXT>
 cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
-    using TL = BwdTile<IO, NP, WARPS>;
+    using TL = BwdTile<IO, NP, WARPS, EXT>;
     ScanBwdArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t grid = a.batch * a.tiles_per_batch;
     if (grid > 0x7fffffffLL || a.dim > 0x7fffffffLL || a.batch > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
-    CUtensorMap mx, md, my, mB, mC;
+    CUtensorMap mx, md, my, mB, mC, mz;
     memset(&mx, 0, sizeof(mx)); memset(&md, 0, sizeof(md)); memset(&my, 0, sizeof(my));
-    memset(&mB, 0, sizeof(mB)); memset(&mC, 0, sizeof(mC));
+    memset(&mB, 0, sizeof(mB)); memset(&mC, 0, sizeof(mC)); memset(&mz, 0, sizeof(mz));
     if (a.vec_ok) {
         const bool bf = sizeof(IO) == 2;
         const uint64_t L = (uint64_t)a.seqlen;
@@ -499,8 +610,10 @@ cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
         if ((e = make_map_3d(&my, a.dout, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess) return e;
         if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
         if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
+        if (EXT && a.z && (e = make_map_3d(&mz, a.z, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess)
+            return e;
     }
-    auto kern = scan_bwd_kernel<IO, NP, WARPS>;
+    auto kern = scan_bwd_kernel<IO, NP, WARPS, EXT>;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -511,31 +624,34 @@ cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_done.fetch_or(bit, std::memory_order_release);
     }
-    kern<<<(unsigned)grid, TL::NT, TL::SMEM_BYTES, stream>>>(mx, md, my, mB, mC, a);
+    kern<<<(unsigned)grid, TL::NT, TL::SMEM_BYTES, stream>>>(mx, md, my, mB, mC, mz, a);
     return cudaGetLastError();
 }
 
-template <typename IO>
+template <typename IO, bool EXT>
 cudaError_t launch_bwd_io(const ScanBwdArgs& a, cudaStream_t s) {
     const int64_t channels = a.batch * a.dim;
     const int N = a.dstate;
-    if (N > 8) return channels >= 2048 ? launch_bwd_variant<IO, 16, 4>(a, s) : launch_bwd_variant<IO, 16, 2>(a, s);
-    if (N > 4) return launch_bwd_variant<IO, 8, 2>(a, s);
-    if (N > 2) return launch_bwd_variant<IO, 4, 2>(a, s);
-    return launch_bwd_variant<IO, 2, 2>(a, s);
+    if (N > 8)
+        return channels >= 2048 ? launch_bwd_variant<IO, 16, 4, EXT>(a, s) : launch_bwd_variant<IO, 16, 2, EXT>(a, s);
+    if (N > 4) return launch_bwd_variant<IO, 8, 2, EXT>(a, s);
+    if (N > 2) return launch_bwd_variant<IO, 4, 2, EXT>(a, s);
+    return launch_bwd_variant<IO, 2, 2, EXT>(a, s);
 }
 
 }  // namespace
 
 cudaError_t launch_scan_bwd(const ScanBwdArgs& a, int io, cudaStream_t s) {
-    // dA, dB and dC are sums that the kernel adds into: start them at zero.
+    // dA, dB, dC (and dD, d bias) are sums that the kernel adds into: start them at zero.
     cudaError_t e;
     if ((e = cudaMemsetAsync(a.dA, 0, (size_t)a.dim * a.dstate * 4, s)) != cudaSuccess) return e;
     const size_t bc = (size_t)a.batch * a.dstate * a.seqlen * 4;
     if ((e = cudaMemsetAsync(a.dB, 0, bc, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.dC, 0, bc, s)) != cudaSuccess) return e;
-    if (io == 0) return launch_bwd_io<float>(a, s);
-    return launch_bwd_io<bf16>(a, s);
+    if (a.dD && (e = cudaMemsetAsync(a.dD, 0, (size_t)a.dim * 4, s)) != cudaSuccess) return e;
+    if (a.ddbias && (e = cudaMemsetAsync(a.ddbias, 0, (size_t)a.dim * 4, s)) != cudaSuccess) return e;
+    if (a.ext) return io == 0 ? launch_bwd_io<float, true>(a, s) : launch_bwd_io<bf16, true>(a, s);
+    return io == 0 ? launch_bwd_io<float, false>(a, s) : launch_bwd_io<bf16, false>(a, s);
 }
 
 unsigned int scan_bwd_read_and_clear_device_error() {

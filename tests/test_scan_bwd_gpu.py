@@ -188,3 +188,55 @@ def test_bwd_full_size_sampled(io):
            "dC": got["dC"].reshape(-1, w.seqlen)[bn]}
     ref = dict(ref, dA=ref["dA"][ds])
     _compare(sub, ref, io, f"full {io}")
+
+
+GATED = [  # D, z, bias, softplus
+    (True, False, False, False), (False, True, False, False), (False, False, True, False),
+    (False, False, False, True), (False, False, True, True), (True, True, True, True),
+]
+
+
+def _gated(w, batch, L, dim, use_D, use_z, use_bias, softplus, beta=0.9, alpha=1.0, dstate=16):
+    inp, g = _problem(w, batch, L, dim, dstate=dstate)
+    ex = wl.scan_extras(w, batch=batch, seqlen=L, dim=dim)
+    if softplus:
+        inp["delta"] = ex["delta_raw"]
+        bias = ex["delta_bias"] if use_bias else None
+    else:
+        bias = np.linspace(1e-3, 5e-2, dim, dtype=np.float32) if use_bias else None
+    D = ex["D"] if use_D else None
+    z = ex["z"] if use_z else None
+    io = torch.float32 if w.io == "f32" else torch.bfloat16
+    dev = {k: _t(inp[k], io) for k in ("x", "delta", "B", "C")}
+    A, h0, v0 = _t(inp["A"]), _t(inp["h0"]), _t(inp["v0"])
+    kw = dict(D=_t(D), z=_t(z, io), delta_bias=_t(bias), delta_softplus=softplus)
+    _, _, _, ckpt = mm.scan_fwd_train(dev["x"], dev["delta"], A, dev["B"], dev["C"], h0=h0, v0=v0,
+                                      beta=beta, alpha=alpha, **kw)
+    gr = mm.scan_bwd(dev["x"], dev["delta"], A, dev["B"], dev["C"], ckpt, _t(g["dy"], io), h0=h0, v0=v0,
+                     dhT=_t(g["dhT"]), dvT=_t(g["dvT"]), beta=beta, alpha=alpha, **kw)
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    got = {k: v.float().cpu().numpy() for k, v in gr.items() if v is not None}
+    f64 = lambda a: np.asarray(a, np.float64)
+    ref = oracle.scan_bwd(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], g["dy"], D=D, z=z,
+                          delta_bias=bias, delta_softplus=softplus, h0=f64(inp["h0"]), v0=f64(inp["v0"]),
+                          dhT=f64(g["dhT"]), dvT=f64(g["dvT"]), beta=beta, alpha=alpha)
+    keys = GRADS + ("dD", "ddelta_bias") + (("dz",) if use_z else ())
+    _compare(got, ref, w.io, f"{w.io} D={use_D} z={use_z} bias={use_bias} softplus={softplus}", keys)
+
+
+@pytest.mark.parametrize("combo", GATED, ids=lambda c: "".join("DzbS"[i] if f else "-" for i, f in enumerate(c)))
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_gated_bwd_matches_oracle(io, combo):
+    w = wl.SCAN_BF16 if io == "bf16" else wl.SCAN_MEDIUM
+    _gated(w, 2, 200, 70, *combo)
+
+
+@pytest.mark.parametrize("L", [1, 37, 65])
+def test_gated_bwd_lengths_and_row_fallback(L):
+    _gated(wl.SCAN_MEDIUM, 1, L, 24, True, True, True, True, beta=0.5, alpha=2.0)
+
+
+@pytest.mark.parametrize("dstate", [4, 13])
+def test_gated_bwd_state_counts(dstate):
+    _gated(wl.SCAN_MEDIUM, 2, 100, 20, True, True, True, True, dstate=dstate)
