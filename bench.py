@@ -103,34 +103,41 @@ def algorithmic_bytes(w: wl.ScanWorkload, gated: bool = False) -> int:
         + 2 * w.batch * w.dim * w.dstate * 4 + extra
 
 
-def bwd_algorithmic_bytes(w: wl.ScanWorkload) -> int:
+def bwd_algorithmic_bytes(w: wl.ScanWorkload, gated: bool = False) -> int:
     """Bytes the backward must move: x, delta, dy read and dx, ddelta written
     once; B, C read and dB, dC (fp32) written once; the checkpoints read once;
-    A and dA."""
+    A and dA; with the extras also z read and dz written, D, bias, dD, d bias."""
     eb = 4 if w.io == "f32" else 2
     bdl = w.batch * w.dim * w.seqlen
     bnl = w.batch * w.dstate * w.seqlen
     chunks = -(-w.seqlen // 16)
+    extra = (2 * bdl * eb + 4 * w.dim * 4) if gated else 0
     return 5 * bdl * eb + 2 * bnl * eb + 2 * bnl * 4 + w.batch * w.dim * chunks * 2 * w.dstate * 4 \
-        + 2 * w.dim * w.dstate * 4
+        + 2 * w.dim * w.dstate * 4 + extra
 
 
-def bwd_cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0):
+def bwd_cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0,
+                     gated: bool = False):
     """The fp64 oracle's backward (as it stands) on the first D' channels of
     batch row 0 (a whole backward of that slice: every gradient, dB and dC
     summed over the slice), D' sized to about `budget_s` of CPU time."""
     import oracle
     inp = wl.scan_inputs(w)
+    if gated:
+        ex = wl.scan_extras(w)
+        inp["delta"] = ex["delta_raw"]
+        inp.update(z=ex["z"], D=ex["D"], delta_bias=ex["delta_bias"])
     rng = np.random.default_rng(5)
     cores = oracle.num_threads()
     wall_budget = budget_s / max(cores, 1)
 
     def run(dd):
-        sl = {k: (v[:1, :dd] if k in ("x", "delta") else v[:1] if k in ("B", "C") else v[:dd])
+        sl = {k: (v[:1, :dd] if k in ("x", "delta", "z") else v[:1] if k in ("B", "C") else v[:dd])
               for k, v in inp.items()}
         dy = rng.standard_normal(sl["x"].shape).astype(np.float32)
+        kw = dict(D=sl["D"], z=sl["z"], delta_bias=sl["delta_bias"], delta_softplus=True) if gated else {}
         t = time.perf_counter()
-        oracle.scan_bwd(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], dy, beta=beta, alpha=alpha)
+        oracle.scan_bwd(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], dy, beta=beta, alpha=alpha, **kw)
         return time.perf_counter() - t
 
     probe = min(w.dim, 16)
@@ -138,7 +145,8 @@ def bwd_cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: fl
     dd = max(1, min(w.dim, int(wall_budget / max(per_chan, 1e-9))))
     dt = run(dd)
     return {"value": dd * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"backward of channels 0..{dd - 1} of batch row 0 (all gradients), beta={beta}, "
+            "sample": f"backward of channels 0..{dd - 1} of batch row 0 (all gradients"
+                      f"{', D, z, delta_bias, softplus' if gated else ''}), beta={beta}, "
                       f"alpha={alpha}, fp64, {dt:.2f} s wall on {cores} threads"}
 
 
@@ -152,28 +160,44 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
     inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))
     iodt = torch.float32 if w.io == "f32" else torch.bfloat16
     gen = torch.Generator().manual_seed(rank_seed(w.seed_index, rank) + 17)
+    if args.gated:
+        ex = wl.scan_extras(w, seed=rank_seed(w.seed_index, rank))
+        inp["delta"] = ex["delta_raw"]
+        inp.update(z=ex["z"], D=ex["D"], delta_bias=ex["delta_bias"])
     host = {k: torch.from_numpy(v).to(iodt if k in IO_KEYS else torch.float32) for k, v in inp.items()}
     host["dy"] = torch.randn(tuple(inp["x"].shape), generator=gen).to(iodt)
-    step_bytes = bwd_algorithmic_bytes(w)
+    step_bytes = bwd_algorithmic_bytes(w, args.gated)
+    ext = dict(D=None, z=None, delta_bias=None, delta_softplus=False)
     nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
     sets = []
     for _ in range(nsets):
         s = {k: v.to(dev).contiguous() for k, v in host.items()}
+        if args.gated:
+            ext = dict(D=s["D"], z=s["z"], delta_bias=s["delta_bias"], delta_softplus=True)
         _, _, _, s["ckpt"] = mm.scan_fwd_train(s["x"], s["delta"], s["A"], s["B"], s["C"], beta=beta,
-                                               alpha=alpha)
+                                               alpha=alpha, **ext)
         s["g"] = {"dx": torch.empty_like(s["x"]), "ddelta": torch.empty_like(s["x"]),
                   "dA": torch.empty((w.dim, w.dstate), device=dev),
                   "dB": torch.empty((w.batch, w.dstate, w.seqlen), device=dev),
-                  "dC": torch.empty((w.batch, w.dstate, w.seqlen), device=dev)}
+                  "dC": torch.empty((w.batch, w.dstate, w.seqlen), device=dev),
+                  "dD": torch.empty((w.dim,), device=dev) if args.gated else None,
+                  "dz": torch.empty_like(s["x"]) if args.gated else None,
+                  "ddelta_bias": torch.empty((w.dim,), device=dev) if args.gated else None}
         sets.append(s)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
     def bwd(s):
         g = s["g"]
-        mm.mm_scan_bwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha, s["ckpt"],
-                       s["dy"], None, None, g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], None, None,
-                       stream)
+        if args.gated:
+            mm.mm_scan_bwd_gated(s["x"], s["delta"], s["A"], s["B"], s["C"], s["D"], s["z"], s["delta_bias"],
+                                 True, None, None, beta, alpha, s["ckpt"], s["dy"], None, None, g["dx"],
+                                 g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"],
+                                 None, None, stream)
+        else:
+            mm.mm_scan_bwd(s["x"], s["delta"], s["A"], s["B"], s["C"], None, None, beta, alpha, s["ckpt"],
+                           s["dy"], None, None, g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], None, None,
+                           stream)
 
     def barrier():
         if world > 1:
@@ -201,14 +225,16 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
     ck_host = sets[0]["ckpt"].cpu()
     pinned = {k: v.pin_memory() for k, v in host.items()}
     pinned["ckpt"] = ck_host.pin_memory()
-    out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in sets[0]["g"].items()}
+    out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in sets[0]["g"].items()
+           if v is not None}
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = sum(v.numel() * v.element_size() for v in out.values())
 
     def e2e_step():
         d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        ex = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"], delta_softplus=True) if args.gated else {}
         g = mm.scan_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["ckpt"], d["dy"], beta=beta,
-                        alpha=alpha, stream=stream)
+                        alpha=alpha, stream=stream, **ex)
         for k in out:
             out[k].copy_(g[k], non_blocking=True)
 
@@ -238,7 +264,8 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
             "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.io, "data": "synthetic",
-            "config": {"workload": w.name, "pass": "backward", "batch": w.batch, "seq_len": w.seqlen,
+            "config": {"workload": w.name, "pass": "backward", **({"extras": GATED_EXTRAS} if args.gated else {}),
+                       "batch": w.batch, "seq_len": w.seqlen,
                        "dim": w.dim, "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
                        "global_batch": w.batch * world, "parallelism": f"dp{world}",
                        "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
@@ -256,7 +283,7 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = bwd_cpu_baseline(w, beta, alpha)
+            line["cpu_baseline"] = bwd_cpu_baseline(w, beta, alpha, gated=args.gated)
         print(json.dumps(line), flush=True)
     return 0
 
@@ -798,8 +825,6 @@ def main(argv=None):
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc
-    if args.gated and args.backward:
-        ap.error("--backward times the plain scan's backward")
     if args.backward and args.impl == "reference":
         ap.error("--impl reference times the forward")
     if isinstance(w, wl.SSDWorkload):
