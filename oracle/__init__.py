@@ -81,6 +81,10 @@ def _declare(lib):
     lib.oracle_ssd_chunked.argtypes = [
         _f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64, _f64,
         _i64, _i64, _i64, _i64, _i64, _i64, _i64, _f64p, _f64p]
+    lib.oracle_ssd_chunked_momentum.restype = ctypes.c_int
+    lib.oracle_ssd_chunked_momentum.argtypes = [
+        _f32p, _f32p, _f32p, _f32p, _f32p, _f64p, _f64p, _f64, _f64,
+        _i64, _i64, _i64, _i64, _i64, _i64, _i64, _f64p, _f64p, _f64p]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     return lib
@@ -344,3 +348,33 @@ def ssd_chunked(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, lib=None):
 def num_threads(lib=None) -> int:
     """OpenMP threads the oracle's channel loops use."""
     return int((lib or load()).oracle_num_threads())
+
+
+def ssd_chunked_momentum(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, chunk=64, lib=None):
+    """The momentum recurrence in the SSD chunked form
+    (mm_oracle.c: oracle_ssd_chunked_momentum).
+
+    Momentum Mamba README, "Momentum Mamba Recurrence", in the form of
+    "Mamba-2 -- SSM = structured matrix multiply", "4-Step Algorithm": per
+    chunk the mask M_ij = sum_{k=j}^{i} exp(cs_i - cs_k) beta^(k-j) and two
+    carried states (h, v).  Layouts as :func:`ssd_seq`; returns fp64
+    (y (batch, L, H, P), hT, vT (batch, H, P, N)).
+    """
+    lib = lib or load()
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    xs, xp = _f32(x, "x")
+    ds, dp = _f32(delta, "delta")
+    As, Ap = _f32(A, "A")
+    Bs, Bp = _f32(B, "B")
+    Cs, Cp = _f32(C, "C")
+    h0s, h0p = _f64opt(h0, (batch, H, P, N), "h0")
+    v0s, v0p = _f64opt(v0, (batch, H, P, N), "v0")
+    y = np.empty((batch, L, H, P), np.float64)
+    hT = np.empty((batch, H, P, N), np.float64)
+    vT = np.empty((batch, H, P, N), np.float64)
+    rc = lib.oracle_ssd_chunked_momentum(xp, dp, Ap, Bp, Cp, h0p, v0p, float(beta), float(alpha),
+                                         batch, L, H, P, N, G, chunk, y.ctypes.data_as(_f64p),
+                                         hT.ctypes.data_as(_f64p), vT.ctypes.data_as(_f64p))
+    _check(rc, "oracle_ssd_chunked_momentum")
+    return y, hT, vT

@@ -736,6 +736,150 @@ int oracle_ssd_chunked(const float *x, const float *delta, const float *A,
     return err;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Mamba-2 SSD with momentum: the chunked algorithm for beta != 0.          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The [MM] momentum recurrence in the [SSD] chunked form.  Within a chunk of
+ * q steps that starts from the states (H0, V0) (P x N per head), with
+ * cs_i = sum_{t <= i} delta_t A_h and w_j[p, n] = alpha delta_j B_j[n] x_j[p],
+ * unrolling v_i = beta v_{i-1} + w_i and h_i = exp(delta_i A_h) h_{i-1} + v_i
+ * gives
+ *
+ *     v_i = beta^{i+1} V0 + sum_{j <= i} beta^{i-j} w_j
+ *     h_i = exp(cs_i) H0 + m_i V0 + sum_{j <= i} M_ij w_j
+ *     M_ij = sum_{k=j}^{i} exp(cs_i - cs_k) beta^{k-j}          (j <= i)
+ *     m_i  = sum_{k=0}^{i} exp(cs_i - cs_k) beta^{k+1}
+ *
+ * so the chunk's output and carried states are
+ *
+ *  1. intra-chunk   Y_diag[i, p] = sum_{j <= i} M_ij (C_i . B_j) alpha delta_j x_j[p]
+ *  2. carried in    Y_off[i, p]  = exp(cs_i) C_i . H0[p, :] + m_i C_i . V0[p, :]
+ *  3. carried out   H_end = h_{q-1},  V_end = beta^q V0 + sum_j beta^{q-1-j} w_j
+ *
+ * With beta = 0, M_ij reduces to exp(cs_i - cs_j) and m_i to 0: the 4-step
+ * algorithm of oracle_ssd_chunked.  M and m are written as their sums, not a
+ * closed form.  Same layouts as oracle_ssd_seq; v0 and vT as h0 and hT.
+ */
+int oracle_ssd_chunked_momentum(const float *x, const float *delta, const float *A,
+                                const float *Bm, const float *Cm, const double *h0,
+                                const double *v0, double beta, double alpha,
+                                int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                                int64_t dstate, int64_t ngroups, int64_t chunk,
+                                double *y, double *hT, double *vT)
+{
+    if (!x || !delta || !A || !Bm || !Cm || !y) return ORACLE_ERR_ARG;
+    if (batch < 1 || seqlen < 1 || nheads < 1 || headdim < 1 || dstate < 1 ||
+        ngroups < 1 || nheads % ngroups != 0 || chunk < 1)
+        return ORACLE_ERR_ARG;
+    const int64_t heads_per_group = nheads / ngroups;
+    const int64_t nchunks = (seqlen + chunk - 1) / chunk;
+    const int64_t PN = headdim * dstate;
+
+    int err = ORACLE_OK;
+    int64_t bh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (bh = 0; bh < batch * nheads; ++bh) {
+        const int64_t b = bh / nheads;
+        const int64_t hh = bh % nheads;
+        const int64_t g = hh / heads_per_group;
+        const double a_h = (double)A[hh];
+        double *H = (double *)malloc(sizeof(double) * (size_t)PN);
+        double *V = (double *)malloc(sizeof(double) * (size_t)PN);
+        double *Hn = (double *)malloc(sizeof(double) * (size_t)PN);
+        double *Vn = (double *)malloc(sizeof(double) * (size_t)PN);
+        double *cs = (double *)malloc(sizeof(double) * (size_t)chunk);
+        double *M = (double *)malloc(sizeof(double) * (size_t)chunk * (size_t)chunk);
+        double *mv = (double *)malloc(sizeof(double) * (size_t)chunk);
+        if (!H || !V || !Hn || !Vn || !cs || !M || !mv) {
+            free(H); free(V); free(Hn); free(Vn); free(cs); free(M); free(mv);
+#pragma omp atomic write
+            err = ORACLE_ERR_ALLOC;
+            continue;
+        }
+        for (int64_t k = 0; k < PN; ++k) {
+            H[k] = h0 ? h0[(b * nheads + hh) * PN + k] : 0.0;
+            V[k] = v0 ? v0[(b * nheads + hh) * PN + k] : 0.0;
+        }
+        for (int64_t c = 0; c < nchunks; ++c) {
+            const int64_t t0 = c * chunk;
+            const int64_t q = (t0 + chunk < seqlen) ? chunk : seqlen - t0;
+#define X_AT(t, p) ((double)x[((b * seqlen + (t)) * nheads + hh) * headdim + (p)])
+#define D_AT(t) ((double)delta[(b * seqlen + (t)) * nheads + hh])
+#define B_AT(t, n) ((double)Bm[((b * seqlen + (t)) * ngroups + g) * dstate + (n)])
+#define C_AT(t, n) ((double)Cm[((b * seqlen + (t)) * ngroups + g) * dstate + (n)])
+#define Y_AT(t, p) y[((b * seqlen + (t)) * nheads + hh) * headdim + (p)]
+            double acc = 0.0;
+            for (int64_t i = 0; i < q; ++i) {
+                acc += D_AT(t0 + i) * a_h;
+                cs[i] = acc;
+            }
+            /* the chunk's mask and carry weights, as their defining sums */
+            for (int64_t i = 0; i < q; ++i) {
+                for (int64_t j = 0; j <= i; ++j) {
+                    double sum = 0.0;
+                    for (int64_t k = j; k <= i; ++k) sum += exp(cs[i] - cs[k]) * pow(beta, (double)(k - j));
+                    M[i * chunk + j] = sum;
+                }
+                double sm = 0.0;
+                for (int64_t k = 0; k <= i; ++k) sm += exp(cs[i] - cs[k]) * pow(beta, (double)(k + 1));
+                mv[i] = sm;
+            }
+            /* steps 1 and 2: the chunk's outputs */
+            for (int64_t i = 0; i < q; ++i) {
+                for (int64_t p = 0; p < headdim; ++p) Y_AT(t0 + i, p) = 0.0;
+                for (int64_t j = 0; j <= i; ++j) {
+                    double cb = 0.0;
+                    for (int64_t n = 0; n < dstate; ++n) cb += C_AT(t0 + i, n) * B_AT(t0 + j, n);
+                    const double lij = M[i * chunk + j] * cb * alpha * D_AT(t0 + j);
+                    for (int64_t p = 0; p < headdim; ++p) Y_AT(t0 + i, p) += lij * X_AT(t0 + j, p);
+                }
+                const double ei = exp(cs[i]);
+                for (int64_t p = 0; p < headdim; ++p) {
+                    double ch = 0.0, cv = 0.0;
+                    for (int64_t n = 0; n < dstate; ++n) {
+                        ch += C_AT(t0 + i, n) * H[p * dstate + n];
+                        cv += C_AT(t0 + i, n) * V[p * dstate + n];
+                    }
+                    Y_AT(t0 + i, p) += ei * ch + mv[i] * cv;
+                }
+            }
+            /* step 3: the states carried out of the chunk */
+            const int64_t last = q - 1;
+            const double elast = exp(cs[last]);
+            const double bq = pow(beta, (double)q);
+            for (int64_t p = 0; p < headdim; ++p)
+                for (int64_t n = 0; n < dstate; ++n) {
+                    double hs = 0.0, vs = 0.0;
+                    for (int64_t j = 0; j < q; ++j) {
+                        const double wj = alpha * D_AT(t0 + j) * B_AT(t0 + j, n) * X_AT(t0 + j, p);
+                        hs += M[last * chunk + j] * wj;
+                        vs += pow(beta, (double)(last - j)) * wj;
+                    }
+                    const int64_t k = p * dstate + n;
+                    Hn[k] = elast * H[k] + mv[last] * V[k] + hs;
+                    Vn[k] = bq * V[k] + vs;
+                }
+            for (int64_t k = 0; k < PN; ++k) {
+                H[k] = Hn[k];
+                V[k] = Vn[k];
+            }
+#undef X_AT
+#undef D_AT
+#undef B_AT
+#undef C_AT
+#undef Y_AT
+        }
+        for (int64_t k = 0; k < PN; ++k) {
+            if (hT) hT[(b * nheads + hh) * PN + k] = H[k];
+            if (vT) vT[(b * nheads + hh) * PN + k] = V[k];
+        }
+        free(H); free(V); free(Hn); free(Vn); free(cs); free(M); free(mv);
+    }
+    return err;
+}
+
 /* Number of OpenMP threads the oracle's parallel loops use (1 without OpenMP). */
 int oracle_num_threads(void)
 {

@@ -95,6 +95,24 @@ BWD_MUTANTS = {
 }
 
 
+# Chunked momentum SSD: slips in the mask, the carry weights or the carried velocity.
+SSDM_MUTANTS = {
+    "ssdm_mask_without_beta": ("sum += exp(cs[i] - cs[k]) * pow(beta, (double)(k - j));",
+                               "sum += exp(cs[i] - cs[k]);"),
+    "ssdm_mask_beta_from_i": ("sum += exp(cs[i] - cs[k]) * pow(beta, (double)(k - j));",
+                              "sum += exp(cs[i] - cs[k]) * pow(beta, (double)(i - k));"),
+    "ssdm_carry_weight_power": ("sm += exp(cs[i] - cs[k]) * pow(beta, (double)(k + 1));",
+                                "sm += exp(cs[i] - cs[k]) * pow(beta, (double)k);"),
+    "ssdm_velocity_decay": ("const double bq = pow(beta, (double)q);", "const double bq = pow(beta, (double)(q - 1));"),
+    "ssdm_no_velocity_readout": ("Y_AT(t0 + i, p) += ei * ch + mv[i] * cv;", "Y_AT(t0 + i, p) += ei * ch;"),
+}
+
+
+def _ssdm_pins(lib):
+    from tests import test_oracle_ssd_momentum_pins as mp
+    return mp.chunked_failures(lib=lib)
+
+
 def _bwd_pins(lib):
     """Finite-difference pins of tests/test_oracle_bwd_pins.py run against `lib`."""
     from tests import test_oracle_bwd_pins as bp
@@ -189,10 +207,10 @@ def test_real_oracle_passes_the_mutant_pins():
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(SSD_MUTANTS) + sorted(GATED_MUTANTS)
-                         + sorted(BWD_MUTANTS))
+                         + sorted(BWD_MUTANTS) + sorted(SSDM_MUTANTS))
 def test_planted_mistake_is_caught(name, tmp_path):
     old, new = (MUTANTS.get(name) or SSD_MUTANTS.get(name) or GATED_MUTANTS.get(name)
-                or BWD_MUTANTS[name])
+                or BWD_MUTANTS.get(name) or SSDM_MUTANTS[name])
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation anchor for {name} not found"
     mut_src = tmp_path / "mm_oracle.c"
@@ -203,5 +221,6 @@ def test_planted_mistake_is_caught(name, tmp_path):
                     "-fPIC", "-std=c11", "-o", str(so), str(mut_src), "-lm"], check=True)
     lib = oracle.load(str(so))
     pins = (_pins if name in MUTANTS else _ssd_pins if name in SSD_MUTANTS
-            else _gated_pins if name in GATED_MUTANTS else _bwd_pins)
+            else _gated_pins if name in GATED_MUTANTS else _bwd_pins if name in BWD_MUTANTS
+            else _ssdm_pins)
     assert pins(lib), f"no pin caught the planted mistake '{name}'"
