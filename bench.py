@@ -53,9 +53,10 @@ L2_BYTES = 126e6
 WORKLOADS = {w.name: w for w in wl.SCAN_WORKLOADS}
 WORKLOADS[wl.SSD_MH.name] = wl.SSD_MH
 WORKLOADS[wl.DECODE.name] = wl.DECODE
+WORKLOADS[wl.SSD_MH_MOMENTUM.name] = wl.SSD_MH_MOMENTUM
 ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
            "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name, "ssd": wl.SSD_MH.name,
-           "decode": wl.DECODE.name}
+           "decode": wl.DECODE.name, "ssd_momentum": wl.SSD_MH_MOMENTUM.name}
 DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
 IO_KEYS = ("x", "delta", "B", "C", "z")          # tensors in the workload's storage type
 GATED_EXTRAS = "D skip, z SiLU gate, delta_bias, softplus"
@@ -640,6 +641,16 @@ def ssd_algorithmic_flops(w: wl.SSDWorkload) -> float:
     return w.batch * nchunk * (per_bc + w.nheads * per_head)
 
 
+def ssd_momentum_fmas(w: wl.SSDWorkload) -> float:
+    """Fused multiply-adds of the momentum chunked form with chunk Q: per
+    (batch, head, chunk) C.B^T (Q x Q x N), the causal half of the masked
+    product with X (Q x Q x P / 2), the read-out of both carried states
+    (2 x Q x P x N) and the update of both (2 x Q x P x N)."""
+    nchunk = math.ceil(w.seqlen / w.chunk)
+    Q, P, N = w.chunk, w.headdim, w.dstate
+    return w.batch * w.nheads * nchunk * (Q * Q * N + Q * Q * P / 2 + 4 * Q * P * N)
+
+
 def ssd_executed_flops(w: wl.SSDWorkload) -> float:
     """Tensor FLOPs the kernel issues: per head and 128-row block, C.B^T
     (128x128x128), M.X, B^T.Xhat and C.S^T (128x64x128 each)."""
@@ -672,10 +683,18 @@ def run_ssd(args, w, rank, world, local):
                                               w.ngroups, w.chunk), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    mom = w.beta != 0.0
+    for st in sets:
+        st["vT"] = torch.empty_like(st["hT"]) if mom else None
+
     def step(i):
         st = sets[i % nsets]
-        mm.mm_ssd_fwd(st["x"], st["delta"], st["A"], st["B"], st["C"], None, 0.0, w.alpha,
-                      st["y"], st["hT"], ws, w.chunk, stream)
+        if mom:
+            mm.mm_ssd_fwd_momentum(st["x"], st["delta"], st["A"], st["B"], st["C"], None, None, w.beta, w.alpha,
+                                   st["y"], st["hT"], st["vT"], stream)
+        else:
+            mm.mm_ssd_fwd(st["x"], st["delta"], st["A"], st["B"], st["C"], None, 0.0, w.alpha,
+                          st["y"], st["hT"], ws, w.chunk, stream)
 
     def barrier():
         if world > 1:
@@ -710,8 +729,12 @@ def run_ssd(args, w, rank, world, local):
 
     def e2e_step():
         d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
-        y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], alpha=w.alpha, chunk=w.chunk,
-                           workspace=ws)
+        if mom:
+            y, hT, _ = mm.ssd_fwd_momentum(d["x"], d["delta"], d["A"], d["B"], d["C"], beta=w.beta,
+                                           alpha=w.alpha)
+        else:
+            y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], alpha=w.alpha, chunk=w.chunk,
+                               workspace=ws)
         out_y.copy_(y, non_blocking=True)
         out_h.copy_(hT, non_blocking=True)
 
@@ -757,6 +780,18 @@ def run_ssd(args, w, rank, world, local):
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
         }
+        if mom:        # the CUDA-core chunked kernel: the fp32 FMA pipe is its roofline
+            sm_max = float(line["clocks"].get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
+            fma_peak = FP32_LANES_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
+            fmas = ssd_momentum_fmas(w)
+            line["roofline"] = {
+                "bound": "alu", "kernel": "ssd_mom_kernel", "achieved": fmas / (ms_step * 1e-3) / 1e9,
+                "peak": fma_peak / 1e9, "unit": "GFMA/s", "frac": fmas / (ms_step * 1e-3) / fma_peak,
+                "traffic": measured_traffic("ssd_mom_kernel", w.name),
+                "peak_source": f"128 fp32 lanes/clk/SM x 148 SMs x {sm_max:.0f} MHz",
+                "algorithmic_fmas": fmas,
+                "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
+                        "frac": hbm_achieved / hbm_peak, "algorithmic_bytes": step_bytes}}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = ssd_cpu_baseline(w)
         print(json.dumps(line), flush=True)
@@ -772,12 +807,12 @@ def ssd_cpu_baseline(w: wl.SSDWorkload, budget_s: float = 12.0):
     cores = oracle.num_threads()
     probe = np.arange(64, dtype=np.int64)
     t = time.perf_counter()
-    oracle.ssd_seq(**inp, beta=0.0, alpha=w.alpha, lane=probe)
+    oracle.ssd_seq(**inp, beta=w.beta, alpha=w.alpha, lane=probe)
     per = (time.perf_counter() - t) / len(probe)
     k = int(max(64, min(nl, budget_s / max(cores, 1) / max(per, 1e-9))))
     lanes = np.linspace(0, nl - 1, k).astype(np.int64)
     t = time.perf_counter()
-    oracle.ssd_seq(**inp, beta=0.0, alpha=w.alpha, lane=lanes)
+    oracle.ssd_seq(**inp, beta=w.beta, alpha=w.alpha, lane=lanes)
     dt = time.perf_counter() - t
     return {"value": k * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{k} of {nl} (batch, head, channel) lanes, fp64, {dt:.2f} s wall on {cores} threads"}

@@ -318,7 +318,8 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
  *   A      (H)               fp32   one decay rate per head
  *   B, C   (batch, L, G, N)  bf16
  *   h0     (batch, H, P, N)  fp32   initial state or NULL (zero)
- *   beta   must be 0 (momentum in chunked form is not built: MM_ERR_UNSUPPORTED)
+ *   beta   in [0, 1); beta != 0 runs mm_ssd_fwd_momentum with v0 = 0
+ *          (the final velocity is not returned)
  *   alpha  finite, >= 0
  *   y      (batch, L, H, P)  bf16   output (round to nearest-even)
  *   hT     (batch, H, P, N)  fp32   final state or NULL; may equal h0
@@ -336,6 +337,26 @@ mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
                      void *y, float *hT,
                      void *workspace, size_t workspace_bytes,
                      const mm_ssd_dims *dims, void *stream);
+
+/*
+ * mm_ssd_fwd_momentum -- the same multi-head scalar-A scan with the
+ * Momentum Mamba velocity ("Momentum Mamba Recurrence"):
+ *     v_t[p, n] = beta v_{t-1}[p, n] + alpha delta_t[h] B_t[g(h), n] x_t[h, p]
+ *     h_t[p, n] = exp(delta_t[h] A[h]) h_{t-1}[p, n] + v_t[p, n]
+ *     y_t[h, p] = sum_n C_t[g(h), n] h_t[p, n]
+ * in the chunked form momentum leads to (chunks of 64 steps; the mask is
+ * M_ij = sum_{k=j}^{i} exp(cs_i - cs_k) beta^(k-j), and the chunk carries
+ * both h and v).  Layouts as mm_ssd_fwd; v0, vT like h0, hT (NULL: zero /
+ * not written; vT may equal v0 and hT h0).  headdim <= 64, dstate <= 128;
+ * dims->chunk is not used (any value >= 1).  Runs on the CUDA cores, not
+ * the tensor cores.  Errors as mm_ssd_fwd (MM_ERR_UNSUPPORTED for headdim or
+ * dstate past those bounds).
+ */
+mm_status mm_ssd_fwd_momentum(const void *x, const float *delta, const float *A,
+                              const void *B, const void *C,
+                              const float *h0, const float *v0, float beta, float alpha,
+                              void *y, float *hT, float *vT,
+                              const mm_ssd_dims *dims, void *stream);
 
 /*
  * mm_device_status -- synchronise the current device, then report whether

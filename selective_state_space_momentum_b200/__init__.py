@@ -25,7 +25,7 @@ import threading
 __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
     "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_bwd_gated",
-    "mm_scan_step", "mm_ssd_fwd",
+    "mm_scan_step", "mm_ssd_fwd", "mm_ssd_fwd_momentum", "ssd_fwd_momentum",
     "mm_ssd_workspace_size", "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
@@ -48,7 +48,7 @@ STATUS_NAMES = {
 
 # Every function include/mm_scan.h declares.
 EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd",
-                    "mm_scan_bwd_gated", "mm_scan_step",
+                    "mm_scan_bwd_gated", "mm_scan_step", "mm_ssd_fwd_momentum",
                     "mm_ssd_workspace_size", "mm_ssd_fwd",
                     "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
@@ -103,6 +103,9 @@ def _declare(lib):
     lib.mm_ssd_fwd.restype = ctypes.c_int
     lib.mm_ssd_fwd.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, ctypes.c_size_t,
                                ctypes.POINTER(SSDDims), vp]
+    lib.mm_ssd_fwd_momentum.restype = ctypes.c_int
+    lib.mm_ssd_fwd_momentum.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp,
+                                        ctypes.POINTER(SSDDims), vp]
     lib.mm_status_string.restype = ctypes.c_char_p
     lib.mm_status_string.argtypes = [ctypes.c_int]
     lib.mm_last_error.restype = ctypes.c_char_p
@@ -244,6 +247,18 @@ def mm_ssd_fwd(x, delta, A, B, C, h0, beta, alpha, y, hT, workspace, chunk, stre
     _check(rc, "mm_ssd_fwd")
 
 
+def mm_ssd_fwd_momentum(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
+    """C entry point mm_ssd_fwd_momentum (marshalling only).  Layouts as
+    mm_ssd_fwd; v0, vT (batch, H, P, N) fp32 or None."""
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dims = SSDDims(batch, L, H, P, N, G, 64)
+    rc = load_library().mm_ssd_fwd_momentum(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
+                                            _ptr(v0), float(beta), float(alpha), _ptr(y), _ptr(hT),
+                                            _ptr(vT), ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_ssd_fwd_momentum")
+
+
 def mm_status_string(status: int) -> str:
     return load_library().mm_status_string(status).decode()
 
@@ -379,6 +394,18 @@ def ssd_fwd(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, return_last_state=
     hT = torch.empty((batch, H, P, N), device=x.device, dtype=torch.float32) if return_last_state else None
     mm_ssd_fwd(x, delta, A, B, C, h0, 0.0, alpha, y, hT, workspace, chunk, stream)
     return y, hT
+
+
+def ssd_fwd_momentum(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, stream=None):
+    """Allocate outputs and run mm_ssd_fwd_momentum; returns (y, hT, vT)."""
+    import torch
+    batch, L, H, P = x.shape
+    N = B.shape[3]
+    y = torch.empty_like(x)
+    hT = torch.empty((batch, H, P, N), device=x.device, dtype=torch.float32)
+    vT = torch.empty_like(hT)
+    mm_ssd_fwd_momentum(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream)
+    return y, hT, vT
 
 
 def scan_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, device="cuda",

@@ -375,8 +375,8 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
         return fail(MM_ERR_NULL, "a workspace of %zu bytes is required", need);
     if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
         return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
-    if (beta != 0.0f)
-        return fail(MM_ERR_UNSUPPORTED, "momentum (beta != 0) in the chunked SSD form is not built");
+    if (beta != 0.0f)       // momentum: the chunked form with two carried states
+        return mm_ssd_fwd_momentum(x, delta, A, B, C, h0, nullptr, beta, alpha, y, hT, nullptr, dims, stream);
     if (!std::isfinite(alpha) || alpha < 0.0f)
         return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
     if (workspace_bytes < need)
@@ -418,6 +418,58 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
     a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
     a.chunk = dims->chunk; a.alpha = alpha;
     return from_cuda(mmscan::launch_ssd_fwd(a, static_cast<cudaStream_t>(stream)), "mm_ssd_fwd launch");
+}
+
+mm_status mm_ssd_fwd_momentum(const void* x, const float* delta, const float* A, const void* B,
+                              const void* C, const float* h0, const float* v0, float beta, float alpha,
+                              void* y, float* hT, float* vT, const mm_ssd_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !y)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
+    const int64_t bsz = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
+                  N = dims->dstate, G = dims->ngroups;
+    if (bsz < 1 || L < 1 || H < 1 || P < 1 || N < 1 || G < 1 || dims->chunk < 1 || H % G != 0)
+        return fail(MM_ERR_DIMS, "sizes must be >= 1 and ngroups must divide nheads");
+    if (!mmscan::ssd_mom_shape_supported(P, N))
+        return fail(MM_ERR_UNSUPPORTED, "momentum SSD needs headdim <= 64 and dstate <= 128 (got %lld, %lld)",
+                    (long long)P, (long long)N);
+    if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
+        return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
+    if (!std::isfinite(alpha) || alpha < 0.0f)
+        return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
+    int64_t blh, xy_bytes, bl, d_bytes, blg, bc_elems, bc_bytes, st_elems, st_bytes;
+    if (!mul_ok(bsz * L, H, &blh) || !mul_ok(blh, P * 2, &xy_bytes) || !mul_ok(bsz, L, &bl) ||
+        !mul_ok(bl, H * 4, &d_bytes) || !mul_ok(bl, G, &blg) || !mul_ok(blg, N, &bc_elems) ||
+        !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz * H, P * N, &st_elems) ||
+        !mul_ok(st_elems, 4, &st_bytes))
+        return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
+    const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT};
+    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "y", "hT", "vT"};
+    for (int i = 0; i < 10; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    const Range rx = rng("x", x, xy_bytes), rd = rng("delta", delta, d_bytes), rA = rng("A", A, H * 4),
+                rB = rng("B", B, bc_bytes), rC = rng("C", C, bc_bytes), rh0 = rng("h0", h0, st_bytes),
+                rv0 = rng("v0", v0, st_bytes), ry = rng("y", y, xy_bytes), rhT = rng("hT", hT, st_bytes),
+                rvT = rng("vT", vT, st_bytes);
+    const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0, &rv0};
+    for (const Range* out : {&ry, &rhT, &rvT}) {
+        for (const Range* in : inputs) {
+            if (!overlap(*out, *in)) continue;
+            const bool same_state = (out == &rhT && in == &rh0) || (out == &rvT && in == &rv0);
+            if (same_state && out->lo == in->lo) continue;   // in-place streaming
+            return fail(MM_ERR_ALIAS, "%s overlaps %s", out->name, in->name);
+        }
+    }
+    if (overlap(ry, rhT) || overlap(ry, rvT) || overlap(rhT, rvT))
+        return fail(MM_ERR_ALIAS, "outputs overlap");
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+    mmscan::SSDMomArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.h0 = h0; a.v0 = v0;
+    a.y = y; a.hT = hT; a.vT = vT;
+    a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
+    a.beta = beta; a.alpha = alpha;
+    return from_cuda(mmscan::launch_ssd_mom(a, static_cast<cudaStream_t>(stream)), "mm_ssd_fwd_momentum launch");
 }
 
 }  // extern "C"

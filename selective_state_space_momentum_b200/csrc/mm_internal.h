@@ -125,6 +125,25 @@ struct SSDArgs {
     float alpha;
 };
 
+// Arguments of one momentum SSD call (the CUDA-core chunked kernel).
+struct SSDMomArgs {
+    const void* x;         // (batch, L, H, P) bf16
+    const float* delta;    // (batch, L, H)
+    const float* A;        // (H)
+    const void* B;         // (batch, L, G, N) bf16
+    const void* C;
+    const float* h0;       // (batch, H, P, N) fp32 or null
+    const float* v0;
+    void* y;               // (batch, L, H, P) bf16
+    float* hT;             // (batch, H, P, N) fp32 or null
+    float* vT;
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups;
+    float beta, alpha;
+};
+
+bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate);
+cudaError_t launch_ssd_mom(const SSDMomArgs& a, cudaStream_t s);
+
 size_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
                            int64_t dstate, int64_t chunk);
 bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk);

@@ -182,6 +182,24 @@ def test_step_checks_its_arguments(lib, monkeypatch):
     assert call(D=_fake(8), z=_fake(9), bias=_fake(10), sp=1) == 7
 
 
+def test_ssd_momentum_checks_its_arguments(lib, monkeypatch):
+    def call(P=64, N=128, H=4, G=2, beta=0.9, **over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), h0=None, v0=None,
+                 y=_fake(5), hT=None, vT=None)
+        a.update(over)
+        dims = mm.SSDDims(1, 128, H, P, N, G, 64)
+        return lib.mm_ssd_fwd_momentum(a["x"], a["delta"], a["A"], a["B"], a["C"], a["h0"], a["v0"], beta, 1.0,
+                                       a["y"], a["hT"], a["vT"], ctypes.byref(dims), None)
+    assert call(y=None) == 1
+    assert call(G=3) == 2                                         # groups must divide heads
+    assert call(P=128) == 6 and call(N=256) == 6                  # past the kernel's tile
+    assert call(beta=1.0) == 3
+    assert call(y=_fake(0)) == 9                                  # output over an input
+    assert call(vT=_fake(6), hT=_fake(6)) == 9                    # two outputs on one buffer
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call(h0=_fake(6), hT=_fake(6), v0=_fake(7), vT=_fake(7)) == 7   # in place: allowed
+
+
 def test_set_tile(lib):
     assert lib.mm_scan_set_tile(3, 2, 1) == 6
     assert lib.mm_scan_set_tile(4, 2, 3) == 6
@@ -209,7 +227,6 @@ def test_ssd_rejects_bad_arguments(lib, monkeypatch):
         return lib.mm_ssd_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["h0"], beta, alpha,
                               a["y"], a["hT"], a["w"], ws, ctypes.byref(dims), None)
     assert call(x=None) == 1
-    assert call(beta=0.5) == 6
     assert call(beta=1.5) == 3
     assert call(alpha=-2.0) == 3
     assert call(y=_fake(0)) == 9
@@ -218,3 +235,4 @@ def test_ssd_rejects_bad_arguments(lib, monkeypatch):
     monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
     assert call() == 7                                            # no workspace needed
     assert call(h0=_fake(6), hT=_fake(6)) == 7                   # in-place final state
+    assert call(beta=0.5) == 7                                    # momentum: the chunked momentum path

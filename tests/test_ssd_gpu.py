@@ -109,16 +109,6 @@ def test_in_place_state_and_determinism():
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
-def test_momentum_is_rejected():
-    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=128, nheads=1)
-    dev = _dev(inp)
-    y = torch.empty_like(dev["x"])
-    with pytest.raises(mm.MMError) as e:
-        mm.mm_ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], None, 0.5, 1.0, y, None,
-                      torch.empty(0, dtype=torch.uint8, device="cuda"), 256)
-    assert e.value.name == "MM_ERR_UNSUPPORTED"
-
-
 def test_repeated_runs_odd_block_counts_finish_without_device_timeout():
     """Several block counts (odd and even) run back to back; every call must
     complete its handshakes (mm_device_status raises on a bounded wait that
