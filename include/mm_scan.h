@@ -344,7 +344,7 @@ mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
  *     v_t[p, n] = beta v_{t-1}[p, n] + alpha delta_t[h] B_t[g(h), n] x_t[h, p]
  *     h_t[p, n] = exp(delta_t[h] A[h]) h_{t-1}[p, n] + v_t[p, n]
  *     y_t[h, p] = sum_n C_t[g(h), n] h_t[p, n]
- * in the chunked form momentum leads to (chunks of 64 steps; the mask is
+ * in the chunked form momentum leads to (chunks of 32 steps; the mask is
  * M_ij = sum_{k=j}^{i} exp(cs_i - cs_k) beta^(k-j), and the chunk carries
  * both h and v).  Layouts as mm_ssd_fwd; v0, vT like h0, hT (NULL: zero /
  * not written; vT may equal v0 and hT h0).  headdim <= 64, dstate <= 128;

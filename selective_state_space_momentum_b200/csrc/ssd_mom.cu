@@ -18,14 +18,16 @@
 //     H_end = E_{q-1} H0 + m_{q-1} V0 + sum_j M_{q-1,j} w_j
 //     V_end = beta^q V0 + sum_j beta^(q-1-j) w_j
 //
-// Design.  One CTA of 256 threads per (b, h) keeps H and V (P x N fp32) in
-// shared memory for the whole sequence and walks it in chunks of Q = 64
-// steps: the chunk's B, C (fp32, row pitch N + 1) and X^T are staged, 64
-// threads form the columns of M by the recursion above (one multiply-add a
-// step, no exponentials of differences, so nothing overflows) and one thread
-// the row weights E and m; C.B^T, the masked product with X and the two
-// carried-state read-outs run as 4 x 4 register-tiled products over shared
-// memory, and the state update is a rank-q sum per (p, n).  This form does
+// Design.  A CTA of 256 threads per (b, h, half of the channels) keeps its
+// H and V rows (fp32) in shared memory for the whole sequence and walks it
+// in chunks of Q = 32 steps (two CTAs per head, each with half of the head
+// channels; both form C.B^T): the chunk's B, C (fp32, row pitch N + 1) and
+// X^T are staged, Q threads form the columns of M by the recursion above
+// (one multiply-add a step, no exponentials of differences, so nothing
+// overflows) and one thread the row weights E and m; C.B^T, the masked
+// product with X and the two carried-state read-outs run as register-tiled
+// products over shared memory (a 16 x 16 thread grid), and the state update
+// is a rank-q sum per (p, n).  This form does
 // not use the tensor cores: the masked matrix is a product of the decay
 // mask and a beta-Toeplitz matrix, which the tcgen05 kernel (ssd_fwd.cu) of
 // the plain recurrence does not form.
@@ -37,26 +39,31 @@
 namespace mmscan {
 namespace ssdm {
 
-constexpr int Q = 64;              // steps per chunk
+constexpr int Q = 32;              // steps per chunk
+constexpr int PSPLIT = 2;          // CTAs per head, each with PMAX / PSPLIT head channels
 constexpr int PMAX = 64;           // head channels
+constexpr int PC = PMAX / PSPLIT;  // head channels of one CTA
 constexpr int NMAX = 128;          // states
-constexpr int NT = 256;            // threads: a 16 x 16 grid of 4 x 4 output tiles
+constexpr int NT = 256;            // threads: a 16 x 16 grid of register tiles
+constexpr int TQ = Q / 16;         // tile rows (steps i) and C.B^T columns (steps j) per thread
+constexpr int TP = PC / 16;        // tile columns (channels p) per thread
 constexpr int LDN = NMAX + 1;      // row pitch (floats) of the [*][n] arrays
 constexpr int LDQ = Q + 1;         // row pitch of the [*][j] arrays
-constexpr int OFF_H = 0;                        // H[p][n]
-constexpr int OFF_V = OFF_H + PMAX * LDN;       // V[p][n]
-constexpr int OFF_B = OFF_V + PMAX * LDN;       // B[j][n]
+constexpr int OFF_H = 0;                        // H[p][n], this CTA's channels
+constexpr int OFF_V = OFF_H + PC * LDN;         // V[p][n]
+constexpr int OFF_B = OFF_V + PC * LDN;         // B[j][n]
 constexpr int OFF_C = OFF_B + Q * LDN;          // C[i][n]
 constexpr int OFF_XT = OFF_C + Q * LDN;         // X^T[p][j]
-constexpr int OFF_L = OFF_XT + PMAX * LDQ;      // M, then the masked matrix L[i][j]
+constexpr int OFF_L = OFF_XT + PC * LDQ;        // M, then the masked matrix L[i][j]
 constexpr int OFF_VEC = OFF_L + Q * LDQ;        // per-step vectors, Q floats each
 constexpr int V_AD = 0, V_A = 1, V_E = 2, V_M = 3, V_WH = 4, V_WV = 5, V_SC = 6;
 constexpr int SMEM_BYTES = (OFF_VEC + 7 * Q) * 4;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(Q % 16 == 0 && PC % 16 == 0 && Q <= NT, "tiles");
 
 }  // namespace ssdm
 
-__global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p) {
+__global__ void __launch_bounds__(ssdm::NT, 2) ssd_mom_kernel(const SSDMomArgs p) {
     using namespace ssdm;
     extern __shared__ float sm[];
     float* Hs = sm + OFF_H;
@@ -75,8 +82,9 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
 
     const int tid = threadIdx.x;
     const int H = (int)p.nheads, P = (int)p.headdim, N = (int)p.dstate, G = (int)p.ngroups;
-    const int64_t b = blockIdx.x / H;
-    const int hh = blockIdx.x % H;
+    const int64_t b = blockIdx.x / (H * PSPLIT);
+    const int hh = (int)((blockIdx.x / PSPLIT) % H);
+    const int pbase = (int)(blockIdx.x % PSPLIT) * PC;   // this CTA's first head channel
     const int g = hh / (H / G);
     const int64_t L = p.seqlen;
     const float a2 = p.A[hh] * kLog2e;
@@ -85,12 +93,13 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
     const bf16* Bg = static_cast<const bf16*>(p.B);
     const bf16* Cg = static_cast<const bf16*>(p.C);
     bf16* yg = static_cast<bf16*>(p.y);
-    const int64_t srow = (b * H + hh) * P;     // first state row of this head
+    const int64_t srow = (b * H + hh) * P + pbase;     // first state row of this CTA
+    const int PL = P - pbase < PC ? P - pbase : PC;     // channels this CTA computes
 
-    for (int e = tid; e < PMAX * NMAX; e += NT) {
+    for (int e = tid; e < PC * NMAX; e += NT) {
         const int pp = e / NMAX, n = e - (e / NMAX) * NMAX;
         float hv = 0.0f, vv = 0.0f;
-        if (pp < P && n < N) {
+        if (pp < PL && n < N) {
             const int64_t si = (srow + pp) * N + n;
             if (p.h0) hv = p.h0[si];
             if (p.v0) vv = p.v0[si];
@@ -115,10 +124,10 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
             Bs[i * LDN + n] = bv;
             Cs[i * LDN + n] = cv;
         }
-        for (int e = tid; e < Q * PMAX; e += NT) {
-            const int i = e / PMAX, pp = e - (e / PMAX) * PMAX;
+        for (int e = tid; e < Q * PC; e += NT) {
+            const int i = e / PC, pp = e - (e / PC) * PC;
             float xv = 0.0f;
-            if (i < q && pp < P) xv = __bfloat162float(xg[((b * L + t0 + i) * H + hh) * P + pp]);
+            if (i < q && pp < PL) xv = __bfloat162float(xg[((b * L + t0 + i) * H + hh) * P + pbase + pp]);
             XT[pp * LDQ + i] = xv;
         }
         if (tid < Q) {
@@ -158,26 +167,26 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
         __syncthreads();
         // ---- L_ij = M_ij (C_i . B_j) alpha delta_j ----------------------------------
         {
-            float acc[4][4];
+            float acc[TQ][TQ];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < TQ; ++a)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
+                for (int c = 0; c < TQ; ++c) acc[a][c] = 0.0f;
             for (int n = 0; n < N; ++n) {
-                float cv[4], bv[4];
+                float cv[TQ], bv[TQ];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) cv[a] = Cs[(ti + 16 * a) * LDN + n];
+                for (int a = 0; a < TQ; ++a) cv[a] = Cs[(ti + 16 * a) * LDN + n];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) bv[c] = Bs[(tj + 16 * c) * LDN + n];
+                for (int c = 0; c < TQ; ++c) bv[c] = Bs[(tj + 16 * c) * LDN + n];
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
+                for (int a = 0; a < TQ; ++a)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[a][c] = __fmaf_rn(cv[a], bv[c], acc[a][c]);
+                    for (int c = 0; c < TQ; ++c) acc[a][c] = __fmaf_rn(cv[a], bv[c], acc[a][c]);
             }
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < TQ; ++a)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < TQ; ++c) {
                     const int i = ti + 16 * a, j = tj + 16 * c;
                     Ls[i * LDQ + j] *= acc[a][c] * vad[j];
                 }
@@ -185,49 +194,49 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
         __syncthreads();
         // ---- outputs: L X + E_i C_i.H0 + m_i C_i.V0 ----------------------------------
         {
-            float yd[4][4], yh[4][4], yv[4][4];
+            float yd[TQ][TP], yh[TQ][TP], yv[TQ][TP];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < TQ; ++a)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) yd[a][c] = yh[a][c] = yv[a][c] = 0.0f;
+                for (int c = 0; c < TP; ++c) yd[a][c] = yh[a][c] = yv[a][c] = 0.0f;
             for (int j = 0; j < q; ++j) {
-                float lv[4], xv[4];
+                float lv[TQ], xv[TP];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) lv[a] = Ls[(ti + 16 * a) * LDQ + j];
+                for (int a = 0; a < TQ; ++a) lv[a] = Ls[(ti + 16 * a) * LDQ + j];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) xv[c] = XT[(tj + 16 * c) * LDQ + j];
+                for (int c = 0; c < TP; ++c) xv[c] = XT[(tj + 16 * c) * LDQ + j];
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
+                for (int a = 0; a < TQ; ++a)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) yd[a][c] = __fmaf_rn(lv[a], xv[c], yd[a][c]);
+                    for (int c = 0; c < TP; ++c) yd[a][c] = __fmaf_rn(lv[a], xv[c], yd[a][c]);
             }
             for (int n = 0; n < N; ++n) {
-                float cv[4], hv[4], vv[4];
+                float cv[TQ], hv[TP], vv[TP];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) cv[a] = Cs[(ti + 16 * a) * LDN + n];
+                for (int a = 0; a < TQ; ++a) cv[a] = Cs[(ti + 16 * a) * LDN + n];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < TP; ++c) {
                     hv[c] = Hs[(tj + 16 * c) * LDN + n];
                     vv[c] = Vs[(tj + 16 * c) * LDN + n];
                 }
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
+                for (int a = 0; a < TQ; ++a)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < TP; ++c) {
                         yh[a][c] = __fmaf_rn(cv[a], hv[c], yh[a][c]);
                         yv[a][c] = __fmaf_rn(cv[a], vv[c], yv[a][c]);
                     }
             }
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
+            for (int a = 0; a < TQ; ++a) {
                 const int i = ti + 16 * a;
                 if (i >= q) continue;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < TP; ++c) {
                     const int pp = tj + 16 * c;
-                    if (pp >= P) continue;
+                    if (pp >= PL) continue;
                     const float out = yd[a][c] + vE[i] * yh[a][c] + vm[i] * yv[a][c];
-                    yg[((b * L + t0 + i) * H + hh) * P + pp] = __float2bfloat16_rn(out);
+                    yg[((b * L + t0 + i) * H + hh) * P + pbase + pp] = __float2bfloat16_rn(out);
                 }
             }
         }
@@ -235,7 +244,7 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
         // ---- the states carried out of the chunk -----------------------------------
         {
             const float eL = vE[q - 1], mL = vm[q - 1], bq = vsc[0];
-            for (int e = tid; e < P * N; e += NT) {
+            for (int e = tid; e < PL * N; e += NT) {
                 const int pp = e / N, n = e - (e / N) * N;
                 float sh = 0.0f, sv = 0.0f;
                 for (int j = 0; j < q; ++j) {
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(ssdm::NT, 1) ssd_mom_kernel(const SSDMomArgs p
         }
     }
     __syncthreads();
-    for (int e = tid; e < P * N; e += NT) {
+    for (int e = tid; e < PL * N; e += NT) {
         const int pp = e / N, n = e - (e / N) * N;
         const int64_t si = (srow + pp) * N + n;
         if (p.hT) p.hT[si] = Hs[pp * LDN + n];
@@ -270,7 +279,7 @@ cudaError_t launch_ssd_mom(const SSDMomArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    const int64_t grid = a.batch * a.nheads;
+    const int64_t grid = a.batch * a.nheads * ssdm::PSPLIT;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     ssd_mom_kernel<<<(unsigned)grid, ssdm::NT, ssdm::SMEM_BYTES, s>>>(a);
     return cudaGetLastError();

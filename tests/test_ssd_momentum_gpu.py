@@ -99,8 +99,8 @@ def test_ssd_fwd_with_beta_routes_to_momentum():
 
 
 def test_streaming_split_bit_identical():
-    """Two calls split at a multiple of 64 steps, carrying (hT, vT): the
-    same chunks, so the same final states bit for bit."""
+    """Two calls split at a multiple of the kernel's 32-step chunk, carrying
+    (hT, vT): the same chunks, so the same final states bit for bit."""
     inp, h0, v0 = _problem(batch=1, L=320, H=2, G=1, seed=7)
     d = _dev(inp)
     h0t, v0t = torch.from_numpy(h0).cuda(), torch.from_numpy(v0).cuda()
