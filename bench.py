@@ -679,7 +679,8 @@ def run_ssd(args, w, rank, world, local):
         st["y"] = torch.empty_like(st["x"])
         st["hT"] = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), device=dev)
         sets.append(st)
-    ws = torch.empty(mm.mm_ssd_workspace_size(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate,
+    ws = torch.empty(0 if w.beta != 0.0 else
+                     mm.mm_ssd_workspace_size(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate,
                                               w.ngroups, w.chunk), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

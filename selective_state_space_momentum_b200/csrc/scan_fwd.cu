@@ -99,7 +99,7 @@ struct ScanTile {
     static_assert(kCkptSteps % R == 0 && T % kCkptSteps == 0 || TS == 2, "checkpoints at group ends");
 };
 
-template <typename IO, int NP, int SPT, int WARPS, int TS, bool EXT>
+template <typename IO, int NP, int SPT, int WARPS, int TS, bool EXT, bool CK>
 __global__ void __launch_bounds__(WARPS * 32, ScanTile<IO, NP, SPT, WARPS, TS, EXT>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -431,8 +431,10 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // The remaining nval < T steps of the sequence, one group at a time.
         // (h, v) after steps 16 i + 15 and after the last step: where the
         // backward restarts its 16-step blocks
+        // (CK: a compile-time switch, so the kernels without checkpoints carry
+        // no trace of them in their unrolled groups)
         auto save_ckpt = [&](int64_t idx) {
-            if (!p.ckpt || !writer) return;
+            if (!writer) return;
             float* cp = p.ckpt + ((b * p.dim + d) * ncks + idx) * 2 * N;
 #pragma unroll
             for (int q = 0; q < NPAIR; ++q) {
@@ -477,8 +479,10 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     }
                 }
                 reduce_store(tau0, yk, zg);
-                const int end = tau0 + kmax;
-                if (end % kCkptSteps == 0 || end == nval) save_ckpt((t0 + end - 1) / kCkptSteps);
+                if constexpr (CK) {
+                    const int end = tau0 + kmax;
+                    if (end % kCkptSteps == 0 || end == nval) save_ckpt((t0 + end - 1) / kCkptSteps);
+                }
             }
         };
 
@@ -497,7 +501,8 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         if (gi + 1 < NG) prep(gi + 1, uA, aA, zA);
                         full_steps(gi, uB, aB, zB);
                     }
-                    if (((gi + 1) * R) % kCkptSteps == 0) save_ckpt((t0 + (gi + 1) * R) / kCkptSteps - 1);
+                    if constexpr (CK)
+                        if (((gi + 1) * R) % kCkptSteps == 0) save_ckpt((t0 + (gi + 1) * R) / kCkptSteps - 1);
                 }
             } else {
                 ragged_chunk();
@@ -609,7 +614,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 // ------------------------------------------------------------- launch -----
 namespace {
 
-template <typename IO, int NP, int SPT, int WARPS, int TS = 1, bool EXT = false>
+template <typename IO, int NP, int SPT, int WARPS, int TS = 1, bool EXT = false, bool CK = false>
 cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
     using TL = ScanTile<IO, NP, SPT, WARPS, TS, EXT>;
     ScanArgs a = a0;
@@ -629,7 +634,7 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
         if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
         if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::BOX_T, TL::NPT)) != cudaSuccess) return e;
     }
-    auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS, TS, EXT>;
+    auto kern = scan_fwd_kernel<IO, NP, SPT, WARPS, TS, EXT, CK>;
     // The dynamic shared-memory limit is raised once per device and variant.
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
@@ -647,8 +652,26 @@ cudaError_t launch_variant(const ScanArgs& a0, cudaStream_t stream) {
 
 // Variants that are built: (states per lane, warps per CTA) for 16 padded states,
 // and the natural choices for smaller state counts.
+template <typename IO, bool EXT>
+cudaError_t launch_ckpt(const ScanArgs& a, int np, int warps, cudaStream_t s) {
+    switch (np) {
+        case 16:
+            if (warps == 2) return launch_variant<IO, 16, 2, 2, 1, EXT, true>(a, s);
+            return launch_variant<IO, 16, 2, 4, 1, EXT, true>(a, s);
+        case 8: return launch_variant<IO, 8, 2, 2, 1, EXT, true>(a, s);
+        case 4: return launch_variant<IO, 4, 2, 2, 1, EXT, true>(a, s);
+        case 2: return launch_variant<IO, 2, 2, 1, 1, EXT, true>(a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 template <typename IO>
 cudaError_t launch_io(const ScanArgs& a, int np, int spt, int warps, int ts, cudaStream_t s) {
+    if (a.ckpt) {
+        // checkpoints: the automatic tiles (two states per lane, one lane along time)
+        const int w = (spt == 2 && warps == 2) ? 2 : 4;
+        return a.ext ? launch_ckpt<IO, true>(a, np, w, s) : launch_ckpt<IO, false>(a, np, w, s);
+    }
     if (a.ext) {
         // selective_scan_fn extras: built for the automatic tiles; a forced
         // tile outside them falls back to the automatic one.
@@ -739,14 +762,8 @@ ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int 
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s) {
-    // Checkpoints are written by the one-lane-along-time variants only.
-    const int ts = a.ckpt ? 1 : t.ts;
-    if (ts != t.ts && !scan_tile_supported(t.spt, t.warps, 1)) {
-        if (io == 0) return launch_io<float>(a, t.np, 2, 4, 1, s);
-        return launch_io<bf16>(a, t.np, 2, 4, 1, s);
-    }
-    if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, ts, s);
-    return launch_io<bf16>(a, t.np, t.spt, t.warps, ts, s);
+    if (io == 0) return launch_io<float>(a, t.np, t.spt, t.warps, t.ts, s);
+    return launch_io<bf16>(a, t.np, t.spt, t.warps, t.ts, s);
 }
 
 unsigned int scan_read_and_clear_device_error() {
