@@ -33,6 +33,8 @@
 // the plain recurrence does not form.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "mm_common.cuh"
 #include "mm_internal.h"
 
@@ -272,12 +274,16 @@ bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate) {
 }
 
 cudaError_t launch_ssd_mom(const SSDMomArgs& a, cudaStream_t s) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(ssd_mom_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ssdm::SMEM_BYTES);
+    // The dynamic shared-memory limit is raised once per device.
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(ssd_mom_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ssdm::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_done = true;
+        attr_done.fetch_or(bit, std::memory_order_release);
     }
     const int64_t grid = a.batch * a.nheads * ssdm::PSPLIT;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

@@ -164,6 +164,28 @@ def test_bwd_checks_its_arguments(lib, monkeypatch):
     assert rc == 7                                                # one block: no checkpoint needed
 
 
+def test_bwd_gated_checks_its_extras(lib, monkeypatch):
+    dims = D(L=200, dim=8)
+    def call(**over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), D=None, z=None, bias=None,
+                 sp=0, h0=None, v0=None, ckpt=_fake(10), dy=_fake(11), dhT=None, dvT=None, dx=_fake(12),
+                 dd=_fake(13), dA=_fake(14), dB=_fake(15), dC=_fake(16), dD=None, dz=None, db=None,
+                 dh0=None, dv0=None)
+        a.update(over)
+        return lib.mm_scan_bwd_gated(a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["bias"],
+                                     a["sp"], a["h0"], a["v0"], 0.9, 1.0, a["ckpt"], a["dy"], a["dhT"], a["dvT"],
+                                     a["dx"], a["dd"], a["dA"], a["dB"], a["dC"], a["dD"], a["dz"], a["db"],
+                                     a["dh0"], a["dv0"], ctypes.byref(dims), None)
+    assert call(z=ctypes.c_void_p(A16 * 17 + 4)) == 5            # misaligned gate
+    assert call(z=_fake(17), dz=_fake(17)) == 9                   # dz over z
+    assert call(D=_fake(18), dD=_fake(18)) == 9                   # dD over D
+    assert call(dD=_fake(12)) == 9                                # dD over dx
+    assert call(db=_fake(1)) == 9                                 # d bias over delta
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call(D=_fake(18), z=_fake(17), bias=_fake(19), sp=1, dD=_fake(20), dz=_fake(21),
+                db=_fake(22)) == 7                                # passes every check
+
+
 def test_step_checks_its_arguments(lib, monkeypatch):
     def call(L=1, **over):
         a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), D=None, z=None,
