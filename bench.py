@@ -145,7 +145,7 @@ def bwd_cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: fl
     per_chan = run(probe) / probe
     dd = max(1, min(w.dim, int(wall_budget / max(per_chan, 1e-9))))
     dt = run(dd)
-    return {"value": dd * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": dd * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu": cpu_model(),
             "sample": f"backward of channels 0..{dd - 1} of batch row 0 (all gradients"
                       f"{', D, z, delta_bias, softplus' if gated else ''}), beta={beta}, "
                       f"alpha={alpha}, fp64, {dt:.2f} s wall on {cores} threads"}
@@ -420,7 +420,7 @@ def decode_cpu_baseline(w: wl.DecodeWorkload, budget_s: float = 12.0):
     for _ in range(reps):
         run()
     dt = time.perf_counter() - t
-    return {"value": reps * w.updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": reps * w.updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu": cpu_model(),
             "sample": f"{reps} whole decode step(s) of {w.batch} requests, fp64, {dt:.2f} s wall on {cores} threads"}
 
 
@@ -519,6 +519,18 @@ def dist_env():
     return rank, world, local
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the baseline records."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float = 12.0,
                  gated: bool = False):
     """Time the fp64 oracle (as it stands) on whole passes over the workload,
@@ -554,7 +566,7 @@ def cpu_baseline(w: wl.ScanWorkload, beta: float, alpha: float, budget_s: float 
     for _ in range(passes):
         run_oracle(chan=chans)
     dt = time.perf_counter() - t
-    return {"value": updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": updates / dt, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu": cpu_model(),
             "sample": sample + f", beta={beta}, alpha={alpha}{', D, z, delta_bias, softplus' if gated else ''}, "
                       f"fp64, {dt:.2f} s wall on {cores} threads"}
 
@@ -618,7 +630,7 @@ def run_reference(args, w, beta=None, alpha=None):
         run(subset(args.warmup + i))
     dt = time.perf_counter() - t
     value = args.steps * k * per_unit_updates / dt
-    cb = {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+    cb = {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle", "cpu": cpu_model(),
           "sample": f"{k} of {n_units} {unit_name} per step (evenly spaced, rotating), fp64"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -815,7 +827,7 @@ def ssd_cpu_baseline(w: wl.SSDWorkload, budget_s: float = 12.0):
     t = time.perf_counter()
     oracle.ssd_seq(**inp, beta=w.beta, alpha=w.alpha, lane=lanes)
     dt = time.perf_counter() - t
-    return {"value": k * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": k * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu": cpu_model(),
             "sample": f"{k} of {nl} (batch, head, channel) lanes, fp64, {dt:.2f} s wall on {cores} threads"}
 
 
