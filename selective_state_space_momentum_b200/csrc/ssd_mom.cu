@@ -24,10 +24,12 @@
 // channels; both form C.B^T): the chunk's B, C (fp32, row pitch N + 1) and
 // X^T are staged, Q threads form the columns of M by the recursion above
 // (one multiply-add a step, no exponentials of differences, so nothing
-// overflows) and one thread the row weights E and m; C.B^T, the masked
-// product with X and the two carried-state read-outs run as register-tiled
-// products over shared memory (a 16 x 16 thread grid), and the state update
-// is a rank-q sum per (p, n).  This form does
+// overflows) and one thread the row weights E and m.  C.B^T and the two
+// carried-state read-outs (inner dimension N) and the masked product with X
+// (inner dimension q) are split over four groups of 64 threads, each a
+// quarter of the inner dimension in 4 x 4 register tiles, and the partial
+// sums meet in shared memory; the state update is a (p, n) product over the
+// q steps with X pre-weighted by the two carry weights, in 2 x 8 tiles.  This form does
 // not use the tensor cores: the masked matrix is a product of the decay
 // mask and a beta-Toeplitz matrix, which the tcgen05 kernel (ssd_fwd.cu) of
 // the plain recurrence does not form.
@@ -47,21 +49,25 @@ constexpr int PMAX = 64;           // head channels
 constexpr int PC = PMAX / PSPLIT;  // head channels of one CTA
 constexpr int NMAX = 128;          // states
 constexpr int NT = 256;            // threads: a 16 x 16 grid of register tiles
-constexpr int TQ = Q / 16;         // tile rows (steps i) and C.B^T columns (steps j) per thread
-constexpr int TP = PC / 16;        // tile columns (channels p) per thread
+constexpr int KQ = NMAX / 4;       // states per thread group in the split products
 constexpr int LDN = NMAX + 1;      // row pitch (floats) of the [*][n] arrays
 constexpr int LDQ = Q + 1;         // row pitch of the [*][j] arrays
+constexpr int YPP = 40;            // row pitch of a partial-sum tile (conflict-free 8 x 4 writes)
+constexpr int YPB = Q * YPP;       // floats of one group's partial-sum tile
 constexpr int OFF_H = 0;                        // H[p][n], this CTA's channels
 constexpr int OFF_V = OFF_H + PC * LDN;         // V[p][n]
 constexpr int OFF_B = OFF_V + PC * LDN;         // B[j][n]
 constexpr int OFF_C = OFF_B + Q * LDN;          // C[i][n]
 constexpr int OFF_XT = OFF_C + Q * LDN;         // X^T[p][j]
-constexpr int OFF_L = OFF_XT + PC * LDQ;        // M, then the masked matrix L[i][j]
-constexpr int OFF_VEC = OFF_L + Q * LDQ;        // per-step vectors, Q floats each
+constexpr int OFF_XH = OFF_XT + PC * LDQ;       // M_{q-1,j} alpha delta_j X^T[p][j]
+constexpr int OFF_XV = OFF_XH + PC * LDQ;       // beta^(q-1-j) alpha delta_j X^T[p][j]
+constexpr int OFF_L = OFF_XV + PC * LDQ;        // M, then the masked matrix L[i][j]
+constexpr int OFF_YP = OFF_L + Q * LDQ;         // four groups' partial sums
+constexpr int OFF_VEC = OFF_YP + 4 * YPB;       // per-step vectors, Q floats each
 constexpr int V_AD = 0, V_A = 1, V_E = 2, V_M = 3, V_WH = 4, V_WV = 5, V_SC = 6;
 constexpr int SMEM_BYTES = (OFF_VEC + 7 * Q) * 4;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-static_assert(Q % 16 == 0 && PC % 16 == 0 && Q <= NT, "tiles");
+static_assert(Q == 32 && PC == 32 && NT == 256 && NMAX % 4 == 0, "the 8 x 8 x 4 and 16 x 16 thread tilings");
 
 }  // namespace ssdm
 
@@ -74,6 +80,9 @@ __global__ void __launch_bounds__(ssdm::NT, 2) ssd_mom_kernel(const SSDMomArgs p
     float* Cs = sm + OFF_C;
     float* XT = sm + OFF_XT;
     float* Ls = sm + OFF_L;
+    float* XH = sm + OFF_XH;
+    float* XV = sm + OFF_XV;
+    float* YP = sm + OFF_YP;
     float* vad = sm + OFF_VEC + V_AD * Q;     // alpha delta_j
     float* va = sm + OFF_VEC + V_A * Q;       // a_i = exp(delta_i A_h)
     float* vE = sm + OFF_VEC + V_E * Q;       // E_i = a_0 ... a_i
@@ -109,7 +118,9 @@ __global__ void __launch_bounds__(ssdm::NT, 2) ssd_mom_kernel(const SSDMomArgs p
         Hs[pp * LDN + n] = hv;
         Vs[pp * LDN + n] = vv;
     }
-    const int ti = tid / 16, tj = tid % 16;    // output rows ti + 16 a, columns tj + 16 c
+    // split products: group gq (a quarter of the states, or of the steps j) and
+    // its 8 x 8 thread grid of 4 x 4 tiles, rows gi + 8 a, columns gj + 8 c
+    const int gq = tid / 64, gi = (tid % 64) / 8, gj = tid % 8;
 
     for (int64_t t0 = 0; t0 < L; t0 += Q) {
         const int q = (int)((L - t0) < Q ? (L - t0) : Q);
@@ -167,97 +178,138 @@ __global__ void __launch_bounds__(ssdm::NT, 2) ssd_mom_kernel(const SSDMomArgs p
             }
         }
         __syncthreads();
-        // ---- L_ij = M_ij (C_i . B_j) alpha delta_j ----------------------------------
+        // ---- L_ij = M_ij (C_i . B_j) alpha delta_j: four groups of 64 threads each
+        // take a quarter of the states (4 x 4 tiles), partial sums meet in YP ----
         {
-            float acc[TQ][TQ];
 #pragma unroll
-            for (int a = 0; a < TQ; ++a)
+            for (int r = 0; r < (PC * Q) / NT; ++r) {         // weighted X for the state update
+                const int e = tid + NT * r;
+                const int pp = e / Q, jj = e - (e / Q) * Q;
+                XH[pp * LDQ + jj] = vwH[jj] * XT[pp * LDQ + jj];
+                XV[pp * LDQ + jj] = vwV[jj] * XT[pp * LDQ + jj];
+            }
+            float acc[4][4];
 #pragma unroll
-                for (int c = 0; c < TQ; ++c) acc[a][c] = 0.0f;
-            for (int n = 0; n < N; ++n) {
-                float cv[TQ], bv[TQ];
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int a = 0; a < TQ; ++a) cv[a] = Cs[(ti + 16 * a) * LDN + n];
+                for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
+            for (int n = gq * KQ; n < gq * KQ + KQ; ++n) {
+                float cv[4], bv[4];
 #pragma unroll
-                for (int c = 0; c < TQ; ++c) bv[c] = Bs[(tj + 16 * c) * LDN + n];
+                for (int a = 0; a < 4; ++a) cv[a] = Cs[(gi + 8 * a) * LDN + n];
 #pragma unroll
-                for (int a = 0; a < TQ; ++a)
+                for (int c = 0; c < 4; ++c) bv[c] = Bs[(gj + 8 * c) * LDN + n];
 #pragma unroll
-                    for (int c = 0; c < TQ; ++c) acc[a][c] = __fmaf_rn(cv[a], bv[c], acc[a][c]);
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[a][c] = __fmaf_rn(cv[a], bv[c], acc[a][c]);
             }
 #pragma unroll
-            for (int a = 0; a < TQ; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int c = 0; c < TQ; ++c) {
-                    const int i = ti + 16 * a, j = tj + 16 * c;
-                    Ls[i * LDQ + j] *= acc[a][c] * vad[j];
-                }
+                for (int c = 0; c < 4; ++c) YP[gq * YPB + (gi + 8 * a) * YPP + gj + 8 * c] = acc[a][c];
         }
         __syncthreads();
-        // ---- outputs: L X + E_i C_i.H0 + m_i C_i.V0 ----------------------------------
+#pragma unroll
+        for (int r = 0; r < (Q * Q) / NT; ++r) {
+            const int e = tid + NT * r;
+            const int i = e / Q, jj = e - (e / Q) * Q;
+            const int o = i * YPP + jj;
+            const float cb = YP[o] + YP[YPB + o] + YP[2 * YPB + o] + YP[3 * YPB + o];
+            Ls[i * LDQ + jj] *= cb * vad[jj];                   // M is 0 above the diagonal and past q
+        }
+        __syncthreads();
+        // ---- outputs: L X + E_i C_i.H0 + m_i C_i.V0, split the same way ------------
         {
-            float yd[TQ][TP], yh[TQ][TP], yv[TQ][TP];
+            float yd[4][4], yh[4][4], yv[4][4];
 #pragma unroll
-            for (int a = 0; a < TQ; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int c = 0; c < TP; ++c) yd[a][c] = yh[a][c] = yv[a][c] = 0.0f;
-            for (int j = 0; j < q; ++j) {
-                float lv[TQ], xv[TP];
+                for (int c = 0; c < 4; ++c) yd[a][c] = yh[a][c] = yv[a][c] = 0.0f;
+            for (int jj = gq * (Q / 4); jj < gq * (Q / 4) + Q / 4; ++jj) {
+                float lv[4], xv[4];
 #pragma unroll
-                for (int a = 0; a < TQ; ++a) lv[a] = Ls[(ti + 16 * a) * LDQ + j];
+                for (int a = 0; a < 4; ++a) lv[a] = Ls[(gi + 8 * a) * LDQ + jj];
 #pragma unroll
-                for (int c = 0; c < TP; ++c) xv[c] = XT[(tj + 16 * c) * LDQ + j];
+                for (int c = 0; c < 4; ++c) xv[c] = XT[(gj + 8 * c) * LDQ + jj];
 #pragma unroll
-                for (int a = 0; a < TQ; ++a)
+                for (int a = 0; a < 4; ++a)
 #pragma unroll
-                    for (int c = 0; c < TP; ++c) yd[a][c] = __fmaf_rn(lv[a], xv[c], yd[a][c]);
+                    for (int c = 0; c < 4; ++c) yd[a][c] = __fmaf_rn(lv[a], xv[c], yd[a][c]);
             }
-            for (int n = 0; n < N; ++n) {
-                float cv[TQ], hv[TP], vv[TP];
+            for (int n = gq * KQ; n < gq * KQ + KQ; ++n) {
+                float cv[4], hv[4], vv[4];
 #pragma unroll
-                for (int a = 0; a < TQ; ++a) cv[a] = Cs[(ti + 16 * a) * LDN + n];
+                for (int a = 0; a < 4; ++a) cv[a] = Cs[(gi + 8 * a) * LDN + n];
 #pragma unroll
-                for (int c = 0; c < TP; ++c) {
-                    hv[c] = Hs[(tj + 16 * c) * LDN + n];
-                    vv[c] = Vs[(tj + 16 * c) * LDN + n];
+                for (int c = 0; c < 4; ++c) {
+                    hv[c] = Hs[(gj + 8 * c) * LDN + n];
+                    vv[c] = Vs[(gj + 8 * c) * LDN + n];
                 }
 #pragma unroll
-                for (int a = 0; a < TQ; ++a)
+                for (int a = 0; a < 4; ++a)
 #pragma unroll
-                    for (int c = 0; c < TP; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         yh[a][c] = __fmaf_rn(cv[a], hv[c], yh[a][c]);
                         yv[a][c] = __fmaf_rn(cv[a], vv[c], yv[a][c]);
                     }
             }
 #pragma unroll
-            for (int a = 0; a < TQ; ++a) {
-                const int i = ti + 16 * a;
-                if (i >= q) continue;
+            for (int a = 0; a < 4; ++a) {
+                const int i = gi + 8 * a;
 #pragma unroll
-                for (int c = 0; c < TP; ++c) {
-                    const int pp = tj + 16 * c;
-                    if (pp >= PL) continue;
-                    const float out = yd[a][c] + vE[i] * yh[a][c] + vm[i] * yv[a][c];
-                    yg[((b * L + t0 + i) * H + hh) * P + pbase + pp] = __float2bfloat16_rn(out);
-                }
+                for (int c = 0; c < 4; ++c)
+                    YP[gq * YPB + i * YPP + gj + 8 * c] = yd[a][c] + vE[i] * yh[a][c] + vm[i] * yv[a][c];
             }
         }
         __syncthreads();            // every read of the chunk's start state is done
-        // ---- the states carried out of the chunk -----------------------------------
-        {
-            const float eL = vE[q - 1], mL = vm[q - 1], bq = vsc[0];
-            for (int e = tid; e < PL * N; e += NT) {
-                const int pp = e / N, n = e - (e / N) * N;
-                float sh = 0.0f, sv = 0.0f;
-                for (int j = 0; j < q; ++j) {
-                    const float u = XT[pp * LDQ + j] * Bs[j * LDN + n];
-                    sh = __fmaf_rn(vwH[j], u, sh);
-                    sv = __fmaf_rn(vwV[j], u, sv);
-                }
-                const float h0v = Hs[pp * LDN + n], v0v = Vs[pp * LDN + n];
-                Hs[pp * LDN + n] = __fmaf_rn(eL, h0v, __fmaf_rn(mL, v0v, sh));
-                Vs[pp * LDN + n] = __fmaf_rn(bq, v0v, sv);
+        // ---- y, and the states carried out of the chunk ------------------------------
+#pragma unroll
+        for (int r = 0; r < (Q * PC) / NT; ++r) {
+            const int e = tid + NT * r;
+            const int i = e / PC, pp = e - (e / PC) * PC;
+            const int o = i * YPP + pp;
+            if (i < q && pp < PL) {
+                const float out = YP[o] + YP[YPB + o] + YP[2 * YPB + o] + YP[3 * YPB + o];
+                yg[((b * L + t0 + i) * H + hh) * P + pbase + pp] = __float2bfloat16_rn(out);
             }
+        }
+        {
+            // H <- E_{q-1} H + m_{q-1} V + (wH o X)^T B,  V <- beta^q V + (wV o X)^T B:
+            // 2 x 8 tiles, rows p = sp + 16 r, columns n = sn + 16 c
+            const int sp = tid / 16, sn = tid % 16;
+            float ah[2][8], av[2][8];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) ah[r][c] = av[r][c] = 0.0f;
+            for (int jj = 0; jj < q; ++jj) {
+                float xh[2], xv[2], bv[8];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    xh[r] = XH[(sp + 16 * r) * LDQ + jj];
+                    xv[r] = XV[(sp + 16 * r) * LDQ + jj];
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) bv[c] = Bs[jj * LDN + sn + 16 * c];
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        ah[r][c] = __fmaf_rn(xh[r], bv[c], ah[r][c]);
+                        av[r][c] = __fmaf_rn(xv[r], bv[c], av[r][c]);
+                    }
+            }
+            const float eL = vE[q - 1], mL = vm[q - 1], bq = vsc[0];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int o = (sp + 16 * r) * LDN + sn + 16 * c;
+                    const float h0v = Hs[o], v0v = Vs[o];
+                    Hs[o] = __fmaf_rn(eL, h0v, __fmaf_rn(mL, v0v, ah[r][c]));
+                    Vs[o] = __fmaf_rn(bq, v0v, av[r][c]);
+                }
         }
     }
     __syncthreads();
