@@ -589,7 +589,7 @@ def run_reference(args, w, beta=None, alpha=None):
         per_unit_updates = w.seqlen * w.dstate
 
         def run(sel):
-            oracle.ssd_seq(**inp, beta=0.0, alpha=w.alpha, lane=sel)
+            oracle.ssd_seq(**inp, beta=w.beta, alpha=w.alpha, lane=sel)
         config = {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads,
                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
                   "beta": w.beta, "alpha": w.alpha, "global_batch": w.batch, "parallelism": "dp1"}

@@ -1,0 +1,70 @@
+"""bench.py's command line and JSON contract, on the CPU.
+
+The reference arm (the fp64 oracle on the host cores) runs here; the GPU
+arms are exercised by the GPU runs.  Also the argument checks and the
+algorithmic byte counts the roofline divides by.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import bench
+from selective_state_space_momentum_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+REQUIRED = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+            "scaling", "vs_baseline", "dtype", "data", "config")
+
+
+def _bench(*args, timeout=300):
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True,
+                          text=True, timeout=timeout, cwd=ROOT, env=env)
+
+
+@pytest.mark.parametrize("workload", ["small", "ssd"])
+def test_reference_arm_prints_one_json_line(workload):
+    r = _bench("--impl", "reference", "--workload", workload, "--steps", "2", "--warmup", "3",
+               "--reference-budget", "2")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in REQUIRED:
+        assert k in d, k
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["cpu"]
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == bench.WORKLOADS[bench.ALIASES[workload]].name
+
+
+@pytest.mark.parametrize("args", [
+    ("--warmup", "2"),                                  # fewer than three warm-up steps
+    ("--workload", "ssd", "--gated"),                  # the extras belong to the scan
+    ("--workload", "ssd", "--backward"),
+    ("--backward", "--impl", "reference"),             # the reference arm times the forward
+    ("--workload", "decode", "--impl", "reference"),
+])
+def test_bad_arguments_are_refused(args):
+    r = _bench(*args, timeout=120)
+    assert r.returncode == 2, (args, r.stdout[-500:], r.stderr[-500:])
+
+
+def test_algorithmic_bytes_match_the_workload_definitions():
+    # x, delta, y once; B, C once; A; the final states (fp32 medium workload)
+    assert bench.algorithmic_bytes(wl.SCAN_MEDIUM) == 152_928_256
+    # bf16: half the streamed bytes
+    assert bench.algorithmic_bytes(wl.SCAN_BF16) == 3 * 8 * 2048 * 4096 * 2 + 2 * 8 * 16 * 4096 * 2 \
+        + 2048 * 16 * 4 + 2 * 8 * 2048 * 16 * 4
+    # decode: h and v read and written (4 D N fp32 a request) dominate
+    d = wl.DECODE
+    assert bench.decode_bytes(d) > 4 * d.batch * d.dim * d.dstate * 4
+    assert bench.decode_bytes(d) < 1.05 * 4 * d.batch * d.dim * d.dstate * 4
+    # the backward moves every forward stream plus dy, dx, ddelta and the checkpoints
+    assert bench.bwd_algorithmic_bytes(wl.SCAN_MEDIUM) > bench.algorithmic_bytes(wl.SCAN_MEDIUM)
