@@ -258,3 +258,21 @@ def test_ssd_rejects_bad_arguments(lib, monkeypatch):
     assert call() == 7                                            # no workspace needed
     assert call(h0=_fake(6), hT=_fake(6)) == 7                   # in-place final state
     assert call(beta=0.5) == 7                                    # momentum: the chunked momentum path
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++11")])
+def test_header_compiles_standalone(tmp_path, lang, std):
+    """include/mm_scan.h is a plain C header: it compiles on its own as C99
+    (pedantic) and as C++, with no CUDA or torch headers."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / ("t.c" if lang == "c" else "t.cpp")
+    src.write_text('#include "mm_scan.h"\n'
+                   "int main(void) { mm_scan_dims d = {1, 1, 1, 1, MM_F32}; (void)d; return (int)MM_OK; }\n")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-fsyntax-only",
+                        str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
