@@ -276,3 +276,23 @@ def test_header_compiles_standalone(tmp_path, lang, std):
     r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-fsyntax-only",
                         str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_plain_c_program_uses_the_abi(tmp_path):
+    """A C program (tests/c/abi_check.c) links libmmscan.so through the header
+    and gets the documented statuses back: the boundary needs no Python."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    lib = mm.library_path()
+    exe = tmp_path / "abi_check"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        os.path.join(here, "c", "abi_check.c"), lib, "-o", str(exe),
+                        "-Wl,-rpath," + os.path.dirname(lib)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and "abi ok" in run.stdout, run.stdout + run.stderr
