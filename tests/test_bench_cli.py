@@ -68,3 +68,23 @@ def test_algorithmic_bytes_match_the_workload_definitions():
     assert bench.decode_bytes(d) < 1.05 * 4 * d.batch * d.dim * d.dstate * 4
     # the backward moves every forward stream plus dy, dx, ddelta and the checkpoints
     assert bench.bwd_algorithmic_bytes(wl.SCAN_MEDIUM) > bench.algorithmic_bytes(wl.SCAN_MEDIUM)
+
+
+def test_reference_arm_under_torchrun_runs_on_rank_zero_only():
+    """Launched by torchrun with two ranks, rank 1 exits 0 at once with no
+    output and rank 0 alone prints the reference line."""
+    def run(rank):
+        env = dict(os.environ, OMP_NUM_THREADS="2", RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE="2",
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT="29555")
+        return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                               "--gpus", "2", "--workload", "small", "--steps", "2", "--warmup", "3",
+                               "--reference-budget", "2"], capture_output=True, text=True, timeout=300,
+                              cwd=ROOT, env=env)
+    r1 = run(1)
+    assert r1.returncode == 0 and r1.stdout.strip() == "", r1.stdout + r1.stderr[-1000:]
+    r0 = run(0)
+    assert r0.returncode == 0, r0.stderr[-2000:]
+    lines = [ln for ln in r0.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["cpu_baseline"]["kind"] == "oracle"
