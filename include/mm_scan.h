@@ -107,7 +107,8 @@ typedef struct {
  * carries its state across 32-step chunks.)
  *
  * Errors: MM_ERR_NULL (x, delta, A, B, C, y or dims NULL), MM_ERR_DIMS
- * (a size < 1), MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE,
+ * (a size < 1), MM_ERR_UNSUPPORTED (dstate > 16,
+ * seqlen > 2^30, batch or dim >= 2^31), MM_ERR_DTYPE,
  * MM_ERR_SCALAR, MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA (launch failure;
  * mm_last_error has CUDA's message).
  */
@@ -195,7 +196,8 @@ mm_status mm_scan_ckpt_size(const mm_scan_dims *dims, size_t *bytes);
  * of arithmetic.
  *
  * Errors: MM_ERR_NULL (a required pointer, or ckpt with seqlen > 16),
- * MM_ERR_DIMS, MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE,
+ * MM_ERR_DIMS, MM_ERR_UNSUPPORTED (dstate > 16,
+ * seqlen > 2^30, batch or dim >= 2^31), MM_ERR_DTYPE,
  * MM_ERR_SCALAR, MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA.
  */
 mm_status mm_scan_bwd(const void *x, const void *delta, const float *A,
@@ -259,7 +261,8 @@ mm_status mm_scan_bwd_gated(const void *x, const void *delta, const float *A,
  * No output (h, v, y) may overlap an input or another output.
  *
  * Errors: MM_ERR_NULL, MM_ERR_DIMS (a size < 1 or seqlen != 1),
- * MM_ERR_UNSUPPORTED (dstate > 16), MM_ERR_DTYPE, MM_ERR_SCALAR,
+ * MM_ERR_UNSUPPORTED (dstate > 16,
+ * seqlen > 2^30, batch or dim >= 2^31), MM_ERR_DTYPE, MM_ERR_SCALAR,
  * MM_ERR_ALIGN, MM_ERR_ALIAS, MM_ERR_CUDA.
  */
 mm_status mm_scan_step(const void *x, const void *delta, const float *A,
@@ -326,8 +329,8 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
  *   workspace, workspace_bytes      device scratch of at least
  *                                   mm_ssd_workspace_size() bytes (may be
  *                                   NULL when that size is 0)
- * Supported sizes: headdim 64, dstate 128, chunk 128 or 256, seqlen any
- * >= 1, H a multiple of G.  All of x, B, C must be 16-byte aligned.
+ * Supported sizes: headdim 64, dstate 128, chunk 128 or 256, seqlen from
+ * 1 to 2^30, batch * H < 2^31, H a multiple of G.  All of x, B, C must be 16-byte aligned.
  * Errors: as mm_scan_fwd, plus MM_ERR_DIMS for a workspace that is too
  * small.
  */
@@ -350,7 +353,7 @@ mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
  * not written; vT may equal v0 and hT h0).  headdim <= 64, dstate <= 128;
  * dims->chunk is not used (any value >= 1).  Runs on the CUDA cores, not
  * the tensor cores.  Errors as mm_ssd_fwd (MM_ERR_UNSUPPORTED for headdim or
- * dstate past those bounds).
+ * dstate past those bounds, seqlen > 2^30 or batch * H >= 2^31).
  */
 mm_status mm_ssd_fwd_momentum(const void *x, const float *delta, const float *A,
                               const void *B, const void *C,

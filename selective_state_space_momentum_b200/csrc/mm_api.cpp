@@ -46,6 +46,12 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
     return true;
 }
 
+// The kernels form time coordinates of the tiled copies, grid sizes and
+// channel numbers in 32 bits; requests beyond these bounds are refused
+// before launch.
+constexpr int64_t kMaxSeqlen = int64_t(1) << 30;
+constexpr int64_t kMaxIndex = 0x7fffffffLL;
+
 struct Range {
     const char* name;
     uintptr_t lo, hi;   // [lo, hi)
@@ -87,12 +93,25 @@ struct ScanSizes {
     int64_t ck_bytes;    // (batch, dim, ceil(L / 16), 2, dstate) fp32
 };
 
+// seqlen and batch * nheads (the grid) of the SSD calls within the 32-bit bounds.
+mm_status check_ssd_range(const mm_ssd_dims* dims) {
+    int64_t bh = 0;
+    if (dims->seqlen > kMaxSeqlen || !mul_ok(dims->batch, dims->nheads, &bh) || bh > kMaxIndex)
+        return fail(MM_ERR_UNSUPPORTED, "SSD seqlen=%lld batch=%lld nheads=%lld: seqlen must be <= 2^30 "
+                    "and batch * nheads < 2^31", (long long)dims->seqlen, (long long)dims->batch,
+                    (long long)dims->nheads);
+    return MM_OK;
+}
+
 mm_status check_scan_dims(const mm_scan_dims* dims, float beta, float alpha, ScanSizes* z) {
     const int64_t bsz = dims->batch, L = dims->seqlen, D = dims->dim, N = dims->dstate;
     if (bsz < 1 || L < 1 || D < 1 || N < 1)
         return fail(MM_ERR_DIMS, "sizes must be >= 1 (batch=%lld seqlen=%lld dim=%lld dstate=%lld)",
                     (long long)bsz, (long long)L, (long long)D, (long long)N);
     if (N > 16) return fail(MM_ERR_UNSUPPORTED, "dstate=%lld > 16", (long long)N);
+    if (L > kMaxSeqlen || bsz > kMaxIndex || D > kMaxIndex)
+        return fail(MM_ERR_UNSUPPORTED, "seqlen=%lld batch=%lld dim=%lld: seqlen must be <= 2^30 and "
+                    "batch, dim < 2^31", (long long)L, (long long)bsz, (long long)D);
     if (dims->io != MM_F32 && dims->io != MM_BF16)
         return fail(MM_ERR_DTYPE, "io=%d is not MM_F32 or MM_BF16", (int)dims->io);
     if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
@@ -353,6 +372,7 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims* dims, size_t* bytes) {
         dims->dstate < 1 || dims->ngroups < 1 || dims->chunk < 1 ||
         dims->nheads % dims->ngroups != 0)
         return fail(MM_ERR_DIMS, "invalid SSD sizes");
+    if (mm_status st = check_ssd_range(dims)) return st;
     if (!mmscan::ssd_shape_supported(dims->headdim, dims->dstate, dims->chunk))
         return fail(MM_ERR_UNSUPPORTED, "SSD with headdim=%lld dstate=%lld chunk=%lld is not built",
                     (long long)dims->headdim, (long long)dims->dstate, (long long)dims->chunk);
@@ -385,10 +405,11 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
     const int64_t bsz = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
                   N = dims->dstate, G = dims->ngroups;
     int64_t blh, xy_bytes, bl, d_bytes, blg, bc_elems, bc_bytes, st_elems, st_bytes;
-    if (!mul_ok(bsz * L, H, &blh) || !mul_ok(blh, P * 2, &xy_bytes) || !mul_ok(bsz, L, &bl) ||
+    int64_t bh, pn;
+    if (!mul_ok(bsz, L, &bl) || !mul_ok(bl, H, &blh) || !mul_ok(blh, P * 2, &xy_bytes) ||
         !mul_ok(bl, H * 4, &d_bytes) || !mul_ok(bl, G, &blg) || !mul_ok(blg, N, &bc_elems) ||
-        !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz * H, P * N, &st_elems) ||
-        !mul_ok(st_elems, 4, &st_bytes))
+        !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz, H, &bh) || !mul_ok(P, N, &pn) ||
+        !mul_ok(bh, pn, &st_elems) || !mul_ok(st_elems, 4, &st_bytes))
         return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
     const void* ptrs[] = {x, delta, A, B, C, h0, y, hT, workspace};
     const char* names[] = {"x", "delta", "A", "B", "C", "h0", "y", "hT", "workspace"};
@@ -430,6 +451,7 @@ mm_status mm_ssd_fwd_momentum(const void* x, const float* delta, const float* A,
                   N = dims->dstate, G = dims->ngroups;
     if (bsz < 1 || L < 1 || H < 1 || P < 1 || N < 1 || G < 1 || dims->chunk < 1 || H % G != 0)
         return fail(MM_ERR_DIMS, "sizes must be >= 1 and ngroups must divide nheads");
+    if (mm_status st = check_ssd_range(dims)) return st;
     if (!mmscan::ssd_mom_shape_supported(P, N))
         return fail(MM_ERR_UNSUPPORTED, "momentum SSD needs headdim <= 64 and dstate <= 128 (got %lld, %lld)",
                     (long long)P, (long long)N);
@@ -438,10 +460,11 @@ mm_status mm_ssd_fwd_momentum(const void* x, const float* delta, const float* A,
     if (!std::isfinite(alpha) || alpha < 0.0f)
         return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
     int64_t blh, xy_bytes, bl, d_bytes, blg, bc_elems, bc_bytes, st_elems, st_bytes;
-    if (!mul_ok(bsz * L, H, &blh) || !mul_ok(blh, P * 2, &xy_bytes) || !mul_ok(bsz, L, &bl) ||
+    int64_t bh, pn;
+    if (!mul_ok(bsz, L, &bl) || !mul_ok(bl, H, &blh) || !mul_ok(blh, P * 2, &xy_bytes) ||
         !mul_ok(bl, H * 4, &d_bytes) || !mul_ok(bl, G, &blg) || !mul_ok(blg, N, &bc_elems) ||
-        !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz * H, P * N, &st_elems) ||
-        !mul_ok(st_elems, 4, &st_bytes))
+        !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz, H, &bh) || !mul_ok(P, N, &pn) ||
+        !mul_ok(bh, pn, &st_elems) || !mul_ok(st_elems, 4, &st_bytes))
         return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
     const void* ptrs[] = {x, delta, A, B, C, h0, v0, y, hT, vT};
     const char* names[] = {"x", "delta", "A", "B", "C", "h0", "v0", "y", "hT", "vT"};

@@ -296,3 +296,21 @@ def test_plain_c_program_uses_the_abi(tmp_path):
     assert r.returncode == 0, r.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and "abi ok" in run.stdout, run.stdout + run.stderr
+
+
+def test_sizes_past_the_32_bit_index_range_are_refused(lib):
+    """The kernels index time coordinates, grids and channels in 32 bits:
+    seqlen past 2^30, and batch, dim or batch * heads from 2^31, are refused
+    on the host with MM_ERR_UNSUPPORTED (and 64-bit byte-count overflow
+    with MM_ERR_DIMS) before anything is launched."""
+    assert _scan(lib, D(L=(1 << 30) + 1)) == 6
+    assert _scan(lib, D(batch=1 << 31)) == 6
+    assert _scan(lib, D(dim=1 << 31)) == 6
+    assert _scan(lib, D(batch=(1 << 31) - 1, dim=(1 << 31) - 1, L=1 << 30)) == 2   # bytes overflow
+    size = ctypes.c_size_t(0)
+    for dims in (mm.SSDDims(1, (1 << 30) + 1, 4, 64, 128, 1, 256), mm.SSDDims(1 << 29, 64, 4, 64, 128, 1, 256),
+                 mm.SSDDims(1 << 40, 64, 1 << 40, 64, 128, 1, 256)):
+        assert lib.mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == 6
+        st = lib.mm_ssd_fwd_momentum(_fake(0), _fake(1), _fake(2), _fake(3), _fake(4), None, None, 0.9, 1.0,
+                                     _fake(5), None, None, ctypes.byref(dims), None)
+        assert st == 6
