@@ -18,6 +18,9 @@ final state.  Inputs are synthetic and seeded (see workloads.py).
 * cpu_baseline: the fp64 oracle on the host cores (rank 0, N = 1), on a
   bounded sample of the same workload.
 * --impl reference: the oracle alone as the reference arm.
+* --batch, --seqlen: the named workload resized (same value laws and seed;
+  the workload name gains the new sizes), to see how a kernel's time
+  depends on the shape at a fixed amount of work.
 
 Multi-GPU (launched by torchrun): one process per GPU, each scanning its own
 batch; there is no collective on the data path, only a barrier and a max of
@@ -26,6 +29,7 @@ the per-rank times (weak scaling).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -83,6 +87,22 @@ def measured_traffic(kernel: str, workload: str):
         return float(rec["dram_bytes_per_launch"])
     except (OSError, ValueError, KeyError):
         return None
+
+
+def resized_workload(w, batch=None, seqlen=None):
+    """The workload with another batch and/or sequence length, same value
+    laws and seed, under a name that says so (so no committed ncu counters
+    of the original apply to it)."""
+    if isinstance(w, wl.DecodeWorkload) and seqlen is not None:
+        raise ValueError("a decode step has no sequence length")
+    b = w.batch if batch is None else batch
+    if b < 1 or (seqlen is not None and seqlen < 1):
+        raise ValueError("--batch and --seqlen must be >= 1")
+    if isinstance(w, wl.DecodeWorkload):
+        return dataclasses.replace(w, batch=b, name=f"{w.name}_as_b{b}")
+    L = w.seqlen if seqlen is None else seqlen
+    extra = {"split": 0} if isinstance(w, wl.ScanWorkload) else {}
+    return dataclasses.replace(w, batch=b, seqlen=L, name=f"{w.name}_as_b{b}_l{L}", **extra)
 
 
 def measured_peaks():
@@ -850,10 +870,19 @@ def main(argv=None):
     ap.add_argument("--backward", action="store_true",
                     help="time the backward mm_scan_bwd (scan workloads)")
     ap.add_argument("--tile", default=None, help="force SPTxWARPS[xTIME_LANES], e.g. 4x2 or 4x2x2 (tuning)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (exploration; renames the workload)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the workload's sequence length (scan and SSD workloads)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[ALIASES.get(args.workload, args.workload)]
+    if args.batch is not None or args.seqlen is not None:
+        try:
+            w = resized_workload(w, args.batch, args.seqlen)
+        except ValueError as e:
+            ap.error(str(e))
     if (args.gated or args.backward) and not isinstance(w, wl.ScanWorkload):
         ap.error("--gated and --backward apply to the scan workloads")
     if isinstance(w, wl.DecodeWorkload):

@@ -88,3 +88,27 @@ def test_reference_arm_under_torchrun_runs_on_rank_zero_only():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_resized_workloads_keep_their_laws_and_change_their_name():
+    w = bench.resized_workload(wl.SSD_MH, batch=16, seqlen=1024)
+    assert (w.batch, w.seqlen, w.nheads, w.seed_index) == (16, 1024, wl.SSD_MH.nheads, wl.SSD_MH.seed_index)
+    assert w.name == wl.SSD_MH.name + "_as_b16_l1024"
+    s = bench.resized_workload(wl.SCAN_LONG, seqlen=8192)
+    assert (s.batch, s.seqlen, s.split) == (1, 8192, 0)
+    assert bench.measured_traffic("scan_fwd_kernel", s.name) is None     # no counters for another shape
+    assert bench.resized_workload(wl.DECODE, batch=8).batch == 8
+    with pytest.raises(ValueError):
+        bench.resized_workload(wl.DECODE, seqlen=4)
+    with pytest.raises(ValueError):
+        bench.resized_workload(wl.SCAN_SMALL, batch=0)
+
+
+def test_reference_arm_on_a_resized_workload():
+    r = _bench("--impl", "reference", "--workload", "small", "--batch", "2", "--seqlen", "64",
+               "--steps", "2", "--warmup", "3", "--reference-budget", "1")
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["config"]["workload"] == wl.SCAN_SMALL.name + "_as_b2_l64"
+    assert d["config"]["batch"] == 2 and d["config"]["seq_len"] == 64
+    assert _bench("--workload", "decode", "--seqlen", "4", timeout=120).returncode == 2
