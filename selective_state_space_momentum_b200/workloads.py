@@ -21,7 +21,7 @@ and returned as the fp32 numbers they represent (``bf16_bits`` gives the
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import numpy as np
 

@@ -9,7 +9,6 @@ whole-job throughput.
 import os
 import socket
 
-import numpy as np
 import pytest
 
 torch = pytest.importorskip("torch")
