@@ -199,3 +199,56 @@ def test_ssd_momentum_chunked_equals_sequential(shape, beta, alpha, chunk):
     ys, hs, vs = oracle.ssd_seq(**inp, h0=h0, v0=v0, beta=beta, alpha=alpha)
     assert _close(yc.transpose(0, 2, 3, 1).reshape(-1, L), ys, 1e-10)
     assert _close(hc.reshape(-1, N), hs, 1e-10) and _close(vc.reshape(-1, N), vs, 1e-10)
+
+
+bwd_shapes = st.tuples(st.integers(0, 2**31 - 1), st.integers(1, 2), st.integers(1, 3), st.integers(1, 20),
+                       st.integers(1, 6))
+
+
+@SETTINGS
+@given(bwd_shapes, st.floats(0.0, 0.95), st.floats(0.1, 2.0), st.booleans(), st.booleans())
+def test_backward_matches_directional_differences(shape, beta, alpha, extras, states):
+    """The backward oracle's gradient of a random linear functional of
+    (out, hT, vT) against a central difference of the forward along a random
+    direction, one input array at a time, for random shapes and scalars
+    (with and without D, z, delta_bias + softplus, h0 and v0)."""
+    seed, batch, dim, L, N = shape
+    rng = np.random.default_rng(seed)
+    f32 = np.float32
+    p = {"x": rng.standard_normal((batch, dim, L)).astype(f32),
+         "delta": (rng.uniform(0.02, 0.3, (batch, dim, L)) if not extras
+                   else rng.standard_normal((batch, dim, L)) * 0.5).astype(f32),
+         "A": (-rng.uniform(0.2, 2.0, (dim, N))).astype(f32),
+         "B": rng.standard_normal((batch, N, L)).astype(f32),
+         "C": rng.standard_normal((batch, N, L)).astype(f32)}
+    if extras:
+        p.update(D=rng.uniform(0.5, 1.5, dim).astype(f32), z=rng.standard_normal((batch, dim, L)).astype(f32),
+                 delta_bias=rng.uniform(-3.0, -1.0, dim).astype(f32))
+    if states:
+        p.update(h0=rng.standard_normal((batch, dim, N)), v0=rng.standard_normal((batch, dim, N)))
+    dout = rng.standard_normal((batch, dim, L)).astype(f32)
+    dhT = rng.standard_normal((batch, dim, N))
+    dvT = rng.standard_normal((batch, dim, N))
+
+    def loss(q):
+        out, hT, vT = oracle.scan_gated(q["x"], q["delta"], q["A"], q["B"], q["C"], D=q.get("D"), z=q.get("z"),
+                                        delta_bias=q.get("delta_bias"), delta_softplus=extras, h0=q.get("h0"),
+                                        v0=q.get("v0"), beta=beta, alpha=alpha)
+        return (float(np.sum(dout.astype(np.float64).reshape(out.shape) * out))
+                + float(np.sum(dhT.reshape(hT.shape) * hT)) + float(np.sum(dvT.reshape(vT.shape) * vT)))
+
+    gr = oracle.scan_bwd(p["x"], p["delta"], p["A"], p["B"], p["C"], dout, D=p.get("D"), z=p.get("z"),
+                         delta_bias=p.get("delta_bias"), delta_softplus=extras, h0=p.get("h0"), v0=p.get("v0"),
+                         dhT=dhT, dvT=dvT, beta=beta, alpha=alpha)
+    grad_of = {"x": "dx", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD", "z": "dz",
+               "delta_bias": "ddelta_bias", "h0": "dh0", "v0": "dv0"}
+    for name, arr in p.items():
+        r = rng.standard_normal(arr.shape)
+        eps = 1e-4 if arr.dtype == f32 else 1e-6    # curvature error ~2e-5 of the difference at most
+        up = (arr + eps * r).astype(arr.dtype)
+        dn = (arr - eps * r).astype(arr.dtype)
+        step = up.astype(np.float64) - dn.astype(np.float64)     # the move the dtype actually made
+        lhs = loss(dict(p, **{name: up})) - loss(dict(p, **{name: dn}))
+        rhs = float(np.sum(gr[grad_of[name]].reshape(arr.shape) * step))
+        scale = max(abs(lhs), abs(rhs))
+        assert abs(lhs - rhs) <= 2e-4 * scale + 1e-9, (name, lhs, rhs)
