@@ -314,3 +314,31 @@ def test_sizes_past_the_32_bit_index_range_are_refused(lib):
         st = lib.mm_ssd_fwd_momentum(_fake(0), _fake(1), _fake(2), _fake(3), _fake(4), None, None, 0.9, 1.0,
                                      _fake(5), None, None, ctypes.byref(dims), None)
         assert st == 6
+
+
+def test_host_checks_under_sanitizers(tmp_path):
+    """mm_api.cpp built with AddressSanitizer and UndefinedBehaviorSanitizer
+    against a stand-in runtime and stub launchers (tests/c/api_checks_sanitized.cpp):
+    every entry point, with sizes at and past every limit and non-finite
+    scalars, returns a documented status without undefined behaviour, and
+    the in-range calls reach their launchers."""
+    import shutil
+    import subprocess
+    cxx = shutil.which("g++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    csrc = os.path.join(root, "selective_state_space_momentum_b200", "csrc")
+    exe = tmp_path / "api_checks"
+    r = subprocess.run([cxx, "-std=c++17", "-O1", "-g", "-fsanitize=address,undefined", "-fno-omit-frame-pointer",
+                        "-fno-sanitize-recover=undefined", "-Wall", "-Werror",
+                        "-I", os.path.join(here, "c", "stub_cuda"), "-I", os.path.join(root, "include"), "-I", csrc,
+                        os.path.join(here, "c", "api_checks_sanitized.cpp"), os.path.join(csrc, "mm_api.cpp"),
+                        "-o", str(exe)], capture_output=True, text=True)
+    if r.returncode != 0 and "sanitize" in r.stderr and "cannot find" in r.stderr:
+        pytest.skip("sanitizer runtimes not available")
+    assert r.returncode == 0, r.stderr[-3000:]
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300,
+                         env=dict(os.environ, ASAN_OPTIONS="detect_leaks=0"))
+    assert run.returncode == 0 and "api checks ok" in run.stdout, (run.stdout + run.stderr)[-3000:]
