@@ -26,6 +26,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(PKG, "_build")
 LIB_PATH = os.path.join(PKG, "libmmscan.so")
+PROBE_SRC = os.path.join(PKG, "probe", "pipe_peaks.cu")
+PROBE_LIB = os.path.join(PKG, "libmmprobe.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -75,8 +77,34 @@ def _compile(src: str, hdr: str, extra: list[str], verbose: bool) -> str:
     return obj
 
 
+def _link(objs: list[str], out: str, verbose: bool, force: bool) -> None:
+    stamp = hashlib.sha256("|".join(objs).encode()).hexdigest()[:16]
+    stamp_path = os.path.join(BUILD_DIR, os.path.basename(out) + ".stamp")
+    if (not force and os.path.exists(out) and os.path.exists(stamp_path)
+            and open(stamp_path).read() == stamp):
+        return
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lpthread", "-ldl", "-lrt"]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
+    os.replace(tmp, out)
+    with open(stamp_path, "w") as f:
+        f.write(stamp)
+
+
+def build_probe(force: bool = False, verbose: bool = False) -> str:
+    """Compile libmmprobe.so (the pipe-throughput probes the benchmark uses); return its path."""
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    obj = _compile(PROBE_SRC, "", [], verbose)
+    _link([obj], PROBE_LIB, verbose, force)
+    return PROBE_LIB
+
+
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile and link libmmscan.so; return its path."""
+    """Compile and link libmmscan.so (and libmmprobe.so); return libmmscan's path."""
     extra = list(extra or [])
     os.makedirs(BUILD_DIR, exist_ok=True)
     if force:
@@ -87,21 +115,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     srcs = _sources()
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(lambda s: _compile(s, hdr, extra, verbose), srcs))
-    stamp = hashlib.sha256("|".join(objs).encode()).hexdigest()[:16]
-    stamp_path = os.path.join(BUILD_DIR, "libmmscan.stamp")
-    if (not force and os.path.exists(LIB_PATH) and os.path.exists(stamp_path)
-            and open(stamp_path).read() == stamp):
-        return LIB_PATH
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lpthread", "-ldl", "-lrt"]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-    os.replace(tmp, LIB_PATH)
-    with open(stamp_path, "w") as f:
-        f.write(stamp)
+    _link(objs, LIB_PATH, verbose, force)
+    build_probe(force=force, verbose=verbose)
     return LIB_PATH
 
 
