@@ -3,9 +3,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 A step is one mm_scan_fwd call over one batch of the named workload (default:
-fp32, batch 4, L 2048, D 1536, N 16, beta 0.9, alpha 1.0), i.e. every step of
-the scan: staging, discretisation, velocity and hidden recurrences, read-out,
-final state.  Inputs are synthetic and seeded (see workloads.py).
+the long streaming workload, fp32, batch 1, L 131072, D 2048, N 16,
+beta 0.99, alpha 1.0 -- the largest scan configuration that one GPU holds),
+i.e. every step of the scan: staging, discretisation, velocity and hidden
+recurrences, read-out, final state.  Inputs are synthetic and seeded (see
+workloads.py).
 
 * value: state updates/s (batch * L * D * N per step, summed over ranks) with
   inputs resident in HBM, timed with CUDA events on the launching stream over
@@ -13,8 +15,10 @@ final state.  Inputs are synthetic and seeded (see workloads.py).
   bytes a step reads were evicted from the 126 MB L2 by the steps before it.
 * e2e: the same metric through the public host-memory call: every step copies
   the inputs from pinned host memory, scans, and copies y, hT, vT back.
-* roofline: the scan kernel is bound by its exponentials (one MUFU ex2 per
-  state update, 16 per clock per SM); peak = 16 * 148 SMs * max SM clock.
+* roofline: the slower of the exponentials (one MUFU ex2 per state update)
+  at the MUFU rate measured by libmmprobe (ex2 per clock per SM, scaled to
+  148 SMs at the max SM clock) and the algorithmic bytes at the measured HBM
+  copy bandwidth; for N = 16 the exponentials bind.
 * cpu_baseline: the fp64 oracle on the host cores (rank 0, N = 1), on a
   bounded sample of the same workload.
 * --impl reference: the oracle alone as the reference arm.
@@ -61,7 +65,7 @@ WORKLOADS[wl.SSD_MH_MOMENTUM.name] = wl.SSD_MH_MOMENTUM
 ALIASES = {"small": wl.SCAN_SMALL.name, "medium": wl.SCAN_MEDIUM.name,
            "bf16": wl.SCAN_BF16.name, "long": wl.SCAN_LONG.name, "ssd": wl.SSD_MH.name,
            "decode": wl.DECODE.name, "ssd_momentum": wl.SSD_MH_MOMENTUM.name}
-DEFAULT_WORKLOAD = wl.SCAN_MEDIUM.name
+DEFAULT_WORKLOAD = wl.SCAN_LONG.name
 IO_KEYS = ("x", "delta", "B", "C", "z")          # tensors in the workload's storage type
 GATED_EXTRAS = "D skip, z SiLU gate, delta_bias, softplus"
 FP32_LANES_PER_CLK_PER_SM = 128      # fp32 arithmetic lanes of one SM per clock
@@ -112,6 +116,49 @@ def measured_peaks():
             return json.load(f), "measured"
     except (OSError, ValueError):
         return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": FALLBACK_SM_MAX_MHZ}, "fallback"
+
+
+def rotating_sets(step_bytes: int) -> int:
+    """Input sets the timed steps rotate through, so that a step's bytes were
+    evicted from L2 by the steps before it."""
+    return min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+
+
+def l2_note(step_bytes: int, what: str = "input") -> str:
+    n = rotating_sets(step_bytes)
+    return f"{n} rotating {what} sets ({n * step_bytes / 1e6:.0f} MB) > 126 MB L2"
+
+
+def scan_config(w, beta, alpha, world, gated=False):
+    """The `config` of a scan forward line; the reference arm prints the same dict."""
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
+            "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
+            "global_batch": w.batch * world, "parallelism": f"dp{world}",
+            "l2": l2_note(algorithmic_bytes(w, gated)),
+            **({"extras": GATED_EXTRAS} if gated else {})}
+
+
+def ssd_config(w, world):
+    """The `config` of an SSD line; the reference arm prints the same dict."""
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads,
+            "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
+            "beta": w.beta, "alpha": w.alpha, "global_batch": w.batch * world,
+            "parallelism": f"dp{world}", "l2": l2_note(ssd_bytes(w))}
+
+
+def mufu_peak_now(sm_max_mhz: float):
+    """The MUFU ex2 rate measured now by libmmprobe (ex2 per clock per SM, at
+    the clock sampled during the probe), scaled to the max SM clock; falls back
+    to the 16 per clock per SM of the unit counts if the probe is missing."""
+    try:
+        from selective_state_space_momentum_b200 import peaks as pk
+        r = pk.measure(("ex2",), target_ms=20.0, reps=3)["ex2"]
+        per = float(r["ops_per_clk_per_sm"])
+        return (per * B200_SMS * sm_max_mhz * 1e6,
+                f"measured {per:.2f} ex2/clk/SM (libmmprobe, {r['sm_mhz']:.0f} MHz) x 148 SMs x {sm_max_mhz:.0f} MHz")
+    except Exception as e:  # the probe library is built with the kernels; say so if it is absent
+        return (MUFU_EX2_PER_CLK_PER_SM * B200_SMS * sm_max_mhz * 1e6,
+                f"unit count 16 ex2/clk/SM x 148 SMs x {sm_max_mhz:.0f} MHz (probe unavailable: {e})")
 
 
 def algorithmic_bytes(w: wl.ScanWorkload, gated: bool = False) -> int:
@@ -189,7 +236,7 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
     host["dy"] = torch.randn(tuple(inp["x"].shape), generator=gen).to(iodt)
     step_bytes = bwd_algorithmic_bytes(w, args.gated)
     ext = dict(D=None, z=None, delta_bias=None, delta_softplus=False)
-    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    nsets = rotating_sets(step_bytes)
     sets = []
     for _ in range(nsets):
         s = {k: v.to(dev).contiguous() for k, v in host.items()}
@@ -330,7 +377,7 @@ def run_decode(args, w, rank, world):
     io_keys = ("x", "delta", "z", "B", "C")
     host = {k: torch.from_numpy(v).to(iodt if k in io_keys else torch.float32) for k, v in inp.items()}
     step_bytes = decode_bytes(w)
-    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    nsets = rotating_sets(step_bytes)
     sets = []
     for _ in range(nsets):
         s = {k: v.to(dev).contiguous() for k, v in host.items()}
@@ -610,9 +657,7 @@ def run_reference(args, w, beta=None, alpha=None):
 
         def run(sel):
             oracle.ssd_seq(**inp, beta=w.beta, alpha=w.alpha, lane=sel)
-        config = {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads,
-                  "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
-                  "beta": w.beta, "alpha": w.alpha, "global_batch": w.batch, "parallelism": "dp1"}
+        config = ssd_config(w, args.gpus)
         unit_name = "(batch, head, channel) lanes"
     else:
         inp = wl.scan_inputs(w)
@@ -627,11 +672,7 @@ def run_reference(args, w, beta=None, alpha=None):
                 oracle.scan_gated(inp["x"], ex["delta_raw"], inp["A"], inp["B"], inp["C"], D=ex["D"],
                                   z=ex["z"], delta_bias=ex["delta_bias"], delta_softplus=True,
                                   beta=beta, alpha=alpha, chan=sel)
-        config = {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
-                  "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
-                  "global_batch": w.batch, "parallelism": "dp1"}
-        if args.gated:
-            config["extras"] = GATED_EXTRAS
+        config = scan_config(w, beta, alpha, args.gpus, args.gated)
         unit_name = "channels"
     probe = np.arange(min(n_units, 64), dtype=np.int64)
     t = time.perf_counter()
@@ -704,16 +745,13 @@ def run_ssd(args, w, rank, world, local):
     host = {k: torch.from_numpy(v) for k, v in inp.items()}
     bf = {"x", "B", "C"}
     step_bytes = ssd_bytes(w)
-    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    nsets = rotating_sets(step_bytes)
     sets = []
     for _ in range(nsets):
         st = {k: host[k].to(dev).to(torch.bfloat16 if k in bf else torch.float32).contiguous() for k in host}
         st["y"] = torch.empty_like(st["x"])
         st["hT"] = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), device=dev)
         sets.append(st)
-    ws = torch.empty(0 if w.beta != 0.0 else
-                     mm.mm_ssd_workspace_size(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate,
-                                              w.ngroups, w.chunk), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     mom = w.beta != 0.0
@@ -727,7 +765,7 @@ def run_ssd(args, w, rank, world, local):
                                    st["y"], st["hT"], st["vT"], stream)
         else:
             mm.mm_ssd_fwd(st["x"], st["delta"], st["A"], st["B"], st["C"], None, 0.0, w.alpha,
-                          st["y"], st["hT"], ws, w.chunk, stream)
+                          st["y"], st["hT"], w.chunk, stream)
 
     def barrier():
         if world > 1:
@@ -766,8 +804,7 @@ def run_ssd(args, w, rank, world, local):
             y, hT, _ = mm.ssd_fwd_momentum(d["x"], d["delta"], d["A"], d["B"], d["C"], beta=w.beta,
                                            alpha=w.alpha)
         else:
-            y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], alpha=w.alpha, chunk=w.chunk,
-                               workspace=ws)
+            y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], alpha=w.alpha, chunk=w.chunk)
         out_y.copy_(y, non_blocking=True)
         out_h.copy_(hT, non_blocking=True)
 
@@ -795,11 +832,7 @@ def run_ssd(args, w, rank, world, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "nheads": w.nheads,
-                       "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
-                       "beta": w.beta, "alpha": w.alpha, "global_batch": w.batch * world,
-                       "parallelism": f"dp{world}",
-                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
+            "config": ssd_config(w, world),
             "roofline": {"bound": "tensor", "kernel": "ssd_fwd_kernel", "achieved": achieved,
                          "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved / tf_peak,
                          "traffic": measured_traffic("ssd_fwd_kernel", w.name),
@@ -870,6 +903,10 @@ def main(argv=None):
     ap.add_argument("--backward", action="store_true",
                     help="time the backward mm_scan_bwd (scan workloads)")
     ap.add_argument("--tile", default=None, help="force SPTxWARPS[xTIME_LANES], e.g. 4x2 or 4x2x2 (tuning)")
+    ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2],
+                    help="scan path: 0 automatic, 1 register-resident, 2 sequence-split (tuning)")
+    ap.add_argument("--seg-len", type=int, default=0,
+                    help="segment length of the sequence-split path (power of two; 0 automatic)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (exploration; renames the workload)")
     ap.add_argument("--seqlen", type=int, default=None,
@@ -948,6 +985,8 @@ def main(argv=None):
     if args.tile:
         parts = [int(v) for v in args.tile.split("x")]
         mm.mm_scan_set_tile(parts[0], parts[1], parts[2] if len(parts) > 2 else 1)
+    if args.path or args.seg_len:
+        mm.mm_scan_set_path(args.path or 2, args.seg_len)
 
     # Each rank scans its own batch (seed offset by rank): weak scaling.
     inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))
@@ -959,7 +998,7 @@ def main(argv=None):
     host = {k: torch.from_numpy(v) for k, v in inp.items()}
     step_bytes = algorithmic_bytes(w, args.gated)
     # enough input sets that a step's bytes were evicted by the steps before it
-    nsets = min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+    nsets = rotating_sets(step_bytes)
     sets = []
     for _ in range(nsets):
         s = {k: host[k].to(dev).to(iodt if k in IO_KEYS else torch.float32).contiguous()
@@ -1033,10 +1072,27 @@ def main(argv=None):
         peaks, peak_kind = measured_peaks()
         clocks = clk.summary()
         sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
-        mufu_peak = MUFU_EX2_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
+        mufu_peak, mufu_source = mufu_peak_now(sm_max)
         achieved = updates / (ms_step * 1e-3)      # one ex2 per update, per launch
         hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
         hbm_achieved = step_bytes / (ms_step * 1e-3) / 1e9
+        # the roofline is the slower of the exponentials on MUFU and the bytes on HBM
+        t_mufu = updates / mufu_peak
+        t_hbm = step_bytes / (hbm_peak * 1e9)
+        kernel = ("scan_seg_kernel" if not args.gated and
+                  mm.mm_scan_segment_len(w.batch, w.seqlen, w.dim, w.dstate, 0 if w.io == "f32" else 1) > 0
+                  else "scan_fwd_kernel")
+        if t_mufu >= t_hbm:
+            roof = {"bound": "alu", "kernel": kernel, "achieved": achieved / 1e9, "peak": mufu_peak / 1e9,
+                    "unit": "Gex2/s", "frac": t_mufu / (ms_step * 1e-3), "peak_source": mufu_source}
+        else:
+            roof = {"bound": "hbm", "kernel": kernel, "achieved": hbm_achieved, "peak": hbm_peak,
+                    "unit": "GB/s", "frac": t_hbm / (ms_step * 1e-3), "peak_source": f"{peak_kind} copy bandwidth"}
+        roof["traffic"] = None if args.gated else measured_traffic(kernel, w.name)
+        roof["hbm"] = {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_achieved / hbm_peak,
+                       "peak_source": peak_kind, "algorithmic_bytes": step_bytes}
+        roof["mufu"] = {"achieved": achieved / 1e9, "peak": mufu_peak / 1e9, "unit": "Gex2/s",
+                        "frac": achieved / mufu_peak, "peak_source": mufu_source}
         cb = None
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w, beta, alpha, gated=args.gated)
@@ -1044,19 +1100,8 @@ def main(argv=None):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "dim": w.dim,
-                       "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
-                       "global_batch": w.batch * world, "parallelism": f"dp{world}",
-                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2",
-                       **({"extras": GATED_EXTRAS} if args.gated else {})},
-            "roofline": {"bound": "alu", "kernel": "scan_fwd_kernel",
-                         "achieved": achieved / 1e9, "peak": mufu_peak / 1e9, "unit": "Gex2/s",
-                         "frac": achieved / mufu_peak,
-                         "traffic": None if args.gated else measured_traffic("scan_fwd_kernel", w.name),
-                         "peak_source": f"16 ex2/clk/SM x 148 SMs x {sm_max:.0f} MHz",
-                         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
-                                 "frac": hbm_achieved / hbm_peak, "peak_source": peak_kind,
-                                 "algorithmic_bytes": step_bytes}},
+            "config": scan_config(w, beta, alpha, world, args.gated),
+            "roofline": roof,
             "e2e": {"value": whole_job_rate(updates, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,

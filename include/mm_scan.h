@@ -98,13 +98,28 @@ typedef struct {
  * one); no other overlap between outputs and inputs is allowed
  * (MM_ERR_ALIAS).
  *
+ * Two execution paths, chosen from (batch * dim, dstate, io) only, never
+ * from L:
+ *   - register-resident: every (channel, state) lane walks the whole
+ *     sequence in time order with its state in registers;
+ *   - sequence-split (few channels, dstate 9..16, fp32, rows of a whole
+ *     number of 16-byte pieces): the sequence is cut into segments of S
+ *     steps (S a power of two, mm_scan_segment_len) at absolute multiples of
+ *     S, each run from a zero state on its own CTA, and joined by folding
+ *     each segment's 2x2 affine carry map onto the concrete carry in segment
+ *     order ("Forward Pass: Two-Stage Parallel Scan" of the same page, with
+ *     the chunk carry [[beta^S, 0], [Q, P]] per lane); y gets the response to
+ *     each segment's carry-in until that response is below 2^-25 of its start
+ *     (when A <= 0 and delta >= 0), else over the whole segment.
+ *
  * Streaming: for a fixed (batch, dim, dstate, io), calling with the first
- * L1 steps (L1 a multiple of 64) and then with the remaining steps,
- * passing (hT, vT) of the first call as (h0, v0) of the second, gives final
- * states bit-identical to one call over all steps, and the same y within
- * rounding of the read-out.  (With one lane along time per state group the
- * steps are applied in order and any L1 gives the same; the time split
- * carries its state across 32-step chunks.)
+ * L1 steps and then with the remaining steps, passing (hT, vT) of the first
+ * call as (h0, v0) of the second, gives final states bit-identical to one
+ * call over all steps, and the same y within rounding, when L1 is a
+ * multiple of mm_scan_segment_len() (sequence-split path), of 32
+ * (register-resident time split, mm_scan_set_tile with two time lanes), or
+ * any L1 (register-resident path with one time lane, which applies the
+ * steps in order).
  *
  * Errors: MM_ERR_NULL (x, delta, A, B, C, y or dims NULL), MM_ERR_DIMS
  * (a size < 1), MM_ERR_UNSUPPORTED (dstate > 16,
@@ -284,16 +299,6 @@ typedef struct {
 } mm_ssd_dims;
 
 /*
- * mm_ssd_workspace_size -- bytes of device workspace mm_ssd_fwd needs for
- * these sizes (written to *bytes).  This build needs none (0): the state
- * never leaves the SM.  When the size is non-zero the caller allocates a
- * 256-byte aligned device buffer of at least that size and passes it to
- * every call with the same sizes; nothing is kept in it between calls.
- * Errors: MM_ERR_NULL, MM_ERR_DIMS, MM_ERR_UNSUPPORTED as for mm_ssd_fwd.
- */
-mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
-
-/*
  * mm_ssd_fwd -- Mamba-2 scalar-A multi-head scan through the chunked (SSD)
  * algorithm ("Mamba-2 -- SSM = structured matrix multiply", sections
  * "4-Step Algorithm" and "Multi-Head Expansion"; first-order
@@ -326,19 +331,15 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims *dims, size_t *bytes);
  *   alpha  finite, >= 0
  *   y      (batch, L, H, P)  bf16   output (round to nearest-even)
  *   hT     (batch, H, P, N)  fp32   final state or NULL; may equal h0
- *   workspace, workspace_bytes      device scratch of at least
- *                                   mm_ssd_workspace_size() bytes (may be
- *                                   NULL when that size is 0)
  * Supported sizes: headdim 64, dstate 128, chunk 128 or 256, seqlen from
  * 1 to 2^30, batch * H < 2^31, H a multiple of G.  All of x, B, C must be 16-byte aligned.
- * Errors: as mm_scan_fwd, plus MM_ERR_DIMS for a workspace that is too
- * small.
+ * Errors: as mm_scan_fwd; MM_ERR_DIMS for sizes < 1 or H not a multiple
+ * of G; MM_ERR_UNSUPPORTED for other headdim, dstate or chunk values.
  */
 mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
                      const void *B, const void *C, const float *h0,
                      float beta, float alpha,
                      void *y, float *hT,
-                     void *workspace, size_t workspace_bytes,
                      const mm_ssd_dims *dims, void *stream);
 
 /*
@@ -386,6 +387,25 @@ const char *mm_last_error(void);
  * Returns MM_ERR_UNSUPPORTED for a combination that is not built.
  */
 mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_lanes);
+
+/*
+ * Tuning and test knob: force the scan path -- 0 automatic, 1 the
+ * register-resident kernel, 2 the sequence-split kernel (used where it
+ * applies: no extras, no checkpoints, dstate <= 16, rows of a whole number of
+ * 16-byte pieces) -- and its segment length (0: automatic; else a power of
+ * two in [32, 2^30]).  Process-wide, not thread-safe with concurrent calls.
+ * MM_ERR_UNSUPPORTED for other values.
+ */
+mm_status mm_scan_set_path(int path, int64_t seg_len);
+
+/*
+ * mm_scan_segment_len -- the segment length S the scan uses for these sizes
+ * (*seg_len = 0 when the call runs on the register-resident path).  A
+ * streaming caller that splits a sequence at multiples of S gets final
+ * states bit-identical to one call (see mm_scan_fwd).  Errors as
+ * mm_scan_fwd's size checks; MM_ERR_NULL for a NULL argument.
+ */
+mm_status mm_scan_segment_len(const mm_scan_dims *dims, int64_t *seg_len);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mm_version(void);

@@ -26,7 +26,8 @@ __all__ = [
     "MMError", "MM_F32", "MM_BF16", "load_library", "library_path",
     "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_bwd_gated",
     "mm_scan_step", "mm_ssd_fwd", "mm_ssd_fwd_momentum", "ssd_fwd_momentum",
-    "mm_ssd_workspace_size", "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
+    "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
+    "mm_scan_set_path", "mm_scan_segment_len",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
 ]
@@ -49,9 +50,10 @@ STATUS_NAMES = {
 # Every function include/mm_scan.h declares.
 EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd",
                     "mm_scan_bwd_gated", "mm_scan_step", "mm_ssd_fwd_momentum",
-                    "mm_ssd_workspace_size", "mm_ssd_fwd",
+                    "mm_ssd_fwd",
                     "mm_device_status",
-                    "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version")
+                    "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
+                    "mm_scan_set_path", "mm_scan_segment_len")
 
 
 class MMError(RuntimeError):
@@ -98,11 +100,8 @@ def _declare(lib):
     lib.mm_scan_bwd.restype = ctypes.c_int
     lib.mm_scan_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp,
                                 vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
-    lib.mm_ssd_workspace_size.restype = ctypes.c_int
-    lib.mm_ssd_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.POINTER(ctypes.c_size_t)]
     lib.mm_ssd_fwd.restype = ctypes.c_int
-    lib.mm_ssd_fwd.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, ctypes.c_size_t,
-                               ctypes.POINTER(SSDDims), vp]
+    lib.mm_ssd_fwd.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp, ctypes.POINTER(SSDDims), vp]
     lib.mm_ssd_fwd_momentum.restype = ctypes.c_int
     lib.mm_ssd_fwd_momentum.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp,
                                         ctypes.POINTER(SSDDims), vp]
@@ -112,6 +111,10 @@ def _declare(lib):
     lib.mm_last_error.argtypes = []
     lib.mm_scan_set_tile.restype = ctypes.c_int
     lib.mm_scan_set_tile.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.mm_scan_set_path.restype = ctypes.c_int
+    lib.mm_scan_set_path.argtypes = [ctypes.c_int, ctypes.c_int64]
+    lib.mm_scan_segment_len.restype = ctypes.c_int
+    lib.mm_scan_segment_len.argtypes = [ctypes.POINTER(ScanDims), ctypes.POINTER(ctypes.c_int64)]
     lib.mm_version.restype = ctypes.c_int
     lib.mm_version.argtypes = []
     lib.mm_device_status.restype = ctypes.c_int
@@ -163,6 +166,98 @@ def _io_code(dtype) -> int:
     raise TypeError(f"unsupported storage type {dtype}; use float32 or bfloat16")
 
 
+# Argument checks of the C-named calls.  The library sizes every operand
+# from the sizes it is given and reads raw device pointers, so a tensor on the
+# host, on another device, of another type or shape, or a strided view would
+# be read wrongly or past its end; each call checks its tensors here first
+# (TypeError for a wrong type, ValueError for the rest).
+def _require(name, t, shape, dtypes, device, optional=False):
+    import torch
+    if t is None:
+        if optional:
+            return
+        raise TypeError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}; expected {' or '.join(str(d) for d in dtypes)}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (call .contiguous() on views)")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, x on {device}")
+
+
+def _lead(x, ndim, name="x"):
+    """Check the tensor that fixes the call's sizes, device and storage type."""
+    import torch
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(x).__name__}")
+    if x.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(x.shape)}")
+    _io_code(x.dtype)
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (call .contiguous() on views)")
+    return x.device, x.dtype
+
+
+def _on_cuda(device):
+    if device.type != "cuda":
+        raise ValueError(f"the operands must be CUDA tensors (got device {device})")
+
+
+def _require_scan(x, A, tensors, seq_dims=3):
+    """x (batch, dim, L) -- or (batch, dim) for a decode step -- and A (dim, N)
+    fix the sizes; `tensors` is a list of (name, tensor, kind, optional) with
+    kind one of io (like x), io_bc (batch, N[, L]) in x's type, state
+    (batch, dim, N) fp32, a (dim, N) fp32, vec (dim,) fp32, bc32 (batch, N, L)
+    fp32, ckpt (batch, dim, ceil(L / 16), 2, N) fp32."""
+    import torch
+    load_library()            # no library: fail first, whatever the arguments
+    dev, io = _lead(x, seq_dims)
+    if not isinstance(A, torch.Tensor) or A.dim() != 2:
+        raise ValueError("A must be a 2-D (dim, dstate) tensor")
+    batch, dim = x.shape[0], x.shape[1]
+    N = A.shape[1]
+    _require("A", A, (dim, N), (torch.float32,), dev)
+    f32 = (torch.float32,)
+    tail = tuple(x.shape[2:])
+    shapes = {"io": (tuple(x.shape), (io,)),
+              "io_bc": ((batch, N) + tail, (io,)),
+              "state": ((batch, dim, N), f32),
+              "a": ((dim, N), f32),
+              "vec": ((dim,), f32),
+              "bc32": ((batch, N) + tail, f32)}
+    if tail:
+        shapes["ckpt"] = ((batch, dim, (tail[0] + MM_SCAN_CKPT_STEPS - 1) // MM_SCAN_CKPT_STEPS, 2, N), f32)
+    for name, t, kind, optional in tensors:
+        shape, dts = shapes[kind]
+        _require(name, t, shape, dts, dev, optional)
+    _on_cuda(dev)
+
+
+def _require_ssd(x, delta, A, B, C, y, states=()):
+    import torch
+    load_library()
+    dev, io = _lead(x, 4)
+    if io != torch.bfloat16:
+        raise TypeError("the SSD path takes bf16 x, B, C and y")
+    batch, L, H, P = x.shape
+    if not isinstance(B, torch.Tensor) or B.dim() != 4:
+        raise ValueError("B must be a 4-D (batch, L, G, N) tensor")
+    G, N = B.shape[2], B.shape[3]
+    bf, f32 = (torch.bfloat16,), (torch.float32,)
+    _require("delta", delta, (batch, L, H), f32, dev)
+    _require("A", A, (H,), f32, dev)
+    _require("B", B, (batch, L, G, N), bf, dev)
+    _require("C", C, (batch, L, G, N), bf, dev)
+    _require("y", y, (batch, L, H, P), bf, dev)
+    for name, t in states:
+        _require(name, t, (batch, H, P, N), f32, dev, optional=True)
+    _on_cuda(dev)
+
+
 def mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
     """C entry point mm_scan_fwd on torch CUDA tensors (marshalling only).
 
@@ -170,6 +265,9 @@ def mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
     h0, v0, hT, vT (batch, dim, N) fp32 or None.  x, delta, B, C, y share one
     storage type (fp32 or bf16).  Raises MMError on a non-OK status.
     """
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("h0", h0, "state", True), ("v0", v0, "state", True), ("y", y, "io", False),
+                         ("hT", hT, "state", True), ("vT", vT, "state", True)])
     batch, dim, L = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
@@ -185,6 +283,10 @@ def mm_scan_fwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v
     optional D (dim,) fp32, z (batch, dim, L) in the storage type of x,
     delta_bias (dim,) fp32, the softplus switch and the checkpoint output
     ckpt (batch, dim, ceil(L / 16), 2, N) fp32."""
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("D", D, "vec", True), ("z", z, "io", True), ("delta_bias", delta_bias, "vec", True),
+                         ("h0", h0, "state", True), ("v0", v0, "state", True), ("y", y, "io", False),
+                         ("hT", hT, "state", True), ("vT", vT, "state", True), ("ckpt", ckpt, "ckpt", True)])
     batch, dim, L = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
@@ -212,6 +314,12 @@ def mm_scan_bwd(x, delta, A, B, C, h0, v0, beta, alpha, ckpt, dy, dhT, dvT,
     Outputs: dx, ddelta like x; dA (dim, N), dB, dC (batch, N, L) fp32;
     dh0, dv0 (batch, dim, N) fp32 or None.
     """
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("h0", h0, "state", True), ("v0", v0, "state", True), ("ckpt", ckpt, "ckpt", True),
+                         ("dy", dy, "io", False), ("dhT", dhT, "state", True), ("dvT", dvT, "state", True),
+                         ("dx", dx, "io", False), ("ddelta", ddelta, "io", False), ("dA", dA, "a", False),
+                         ("dB", dB, "bc32", False), ("dC", dC, "bc32", False), ("dh0", dh0, "state", True),
+                         ("dv0", dv0, "state", True)])
     batch, dim, L = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
@@ -222,27 +330,18 @@ def mm_scan_bwd(x, delta, A, B, C, h0, v0, beta, alpha, ckpt, dy, dhT, dvT,
     _check(rc, "mm_scan_bwd")
 
 
-def mm_ssd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk) -> int:
-    dims = SSDDims(batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
-    out = ctypes.c_size_t(0)
-    _check(load_library().mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(out)),
-           "mm_ssd_workspace_size")
-    return int(out.value)
-
-
-def mm_ssd_fwd(x, delta, A, B, C, h0, beta, alpha, y, hT, workspace, chunk, stream=None):
+def mm_ssd_fwd(x, delta, A, B, C, h0, beta, alpha, y, hT, chunk, stream=None):
     """C entry point mm_ssd_fwd on torch CUDA tensors (marshalling only).
 
     x, y (batch, L, H, P) bf16; delta (batch, L, H) fp32; A (H) fp32;
-    B, C (batch, L, G, N) bf16; h0, hT (batch, H, P, N) fp32 or None;
-    workspace: a uint8 CUDA tensor of mm_ssd_workspace_size() bytes.
+    B, C (batch, L, G, N) bf16; h0, hT (batch, H, P, N) fp32 or None.
     """
+    _require_ssd(x, delta, A, B, C, y, states=(("h0", h0), ("hT", hT)))
     batch, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     dims = SSDDims(batch, L, H, P, N, G, chunk)
     rc = load_library().mm_ssd_fwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
-                                   float(beta), float(alpha), _ptr(y), _ptr(hT), _ptr(workspace),
-                                   workspace.numel() * workspace.element_size(),
+                                   float(beta), float(alpha), _ptr(y), _ptr(hT),
                                    ctypes.byref(dims), _stream_handle(stream))
     _check(rc, "mm_ssd_fwd")
 
@@ -250,6 +349,7 @@ def mm_ssd_fwd(x, delta, A, B, C, h0, beta, alpha, y, hT, workspace, chunk, stre
 def mm_ssd_fwd_momentum(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
     """C entry point mm_ssd_fwd_momentum (marshalling only).  Layouts as
     mm_ssd_fwd; v0, vT (batch, H, P, N) fp32 or None."""
+    _require_ssd(x, delta, A, B, C, y, states=(("h0", h0), ("v0", v0), ("hT", hT), ("vT", vT)))
     batch, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     dims = SSDDims(batch, L, H, P, N, G, 64)
@@ -270,6 +370,21 @@ def mm_last_error() -> str:
 def mm_scan_set_tile(states_per_thread: int, warps_per_block: int, time_lanes: int = 1):
     _check(load_library().mm_scan_set_tile(states_per_thread, warps_per_block, time_lanes),
            "mm_scan_set_tile")
+
+
+def mm_scan_set_path(path: int, seg_len: int = 0):
+    """Force the scan path (0 automatic, 1 register-resident, 2 sequence-split)
+    and the segment length (0 automatic)."""
+    _check(load_library().mm_scan_set_path(int(path), int(seg_len)), "mm_scan_set_path")
+
+
+def mm_scan_segment_len(batch, seqlen, dim, dstate, io=MM_F32) -> int:
+    """C entry point mm_scan_segment_len: the segment length of the
+    sequence-split path for these sizes (0 on the register-resident path)."""
+    dims = ScanDims(batch, seqlen, dim, dstate, io)
+    out = ctypes.c_int64(0)
+    _check(load_library().mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(out)), "mm_scan_segment_len")
+    return int(out.value)
 
 
 def mm_version() -> int:
@@ -311,6 +426,10 @@ def mm_scan_step(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h, v, beta
     (dim, N), D, delta_bias (dim,) fp32; h, v (batch, dim, N) fp32, updated
     in place.
     """
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("D", D, "vec", True), ("z", z, "io", True), ("delta_bias", delta_bias, "vec", True),
+                         ("h", h, "state", False), ("v", v, "state", False), ("y", y, "io", False)],
+                  seq_dims=2)
     batch, dim = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, 1, dim, N, _io_code(x.dtype))
@@ -326,6 +445,14 @@ def mm_scan_bwd_gated(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v
                       stream=None):
     """C entry point mm_scan_bwd_gated (marshalling only): mm_scan_bwd through
     D, z, delta_bias and softplus, with the extra outputs dD, dz, ddelta_bias."""
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("D", D, "vec", True), ("z", z, "io", True), ("delta_bias", delta_bias, "vec", True),
+                         ("h0", h0, "state", True), ("v0", v0, "state", True), ("ckpt", ckpt, "ckpt", True),
+                         ("dy", dy, "io", False), ("dhT", dhT, "state", True), ("dvT", dvT, "state", True),
+                         ("dx", dx, "io", False), ("ddelta", ddelta, "io", False), ("dA", dA, "a", False),
+                         ("dB", dB, "bc32", False), ("dC", dC, "bc32", False), ("dD", dD, "vec", True),
+                         ("dz", dz, "io", True), ("ddelta_bias", ddelta_bias, "vec", True),
+                         ("dh0", dh0, "state", True), ("dv0", dv0, "state", True)])
     batch, dim, L = x.shape
     N = A.shape[1]
     dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
@@ -380,19 +507,14 @@ def scan_bwd(x, delta, A, B, C, ckpt, dy, h0=None, v0=None, dhT=None, dvT=None, 
     return g
 
 
-def ssd_fwd(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, return_last_state=True,
-            workspace=None, stream=None):
-    """Allocate outputs (and workspace if not given) and run mm_ssd_fwd;
-    returns (y, hT)."""
+def ssd_fwd(x, delta, A, B, C, h0=None, alpha=1.0, chunk=256, return_last_state=True, stream=None):
+    """Allocate outputs and run mm_ssd_fwd; returns (y, hT)."""
     import torch
     batch, L, H, P = x.shape
-    G, N = B.shape[2], B.shape[3]
-    need = mm_ssd_workspace_size(batch, L, H, P, N, G, chunk)
-    if workspace is None or workspace.numel() * workspace.element_size() < need:
-        workspace = torch.empty(need, device=x.device, dtype=torch.uint8)
+    N = B.shape[3]
     y = torch.empty_like(x)
     hT = torch.empty((batch, H, P, N), device=x.device, dtype=torch.float32) if return_last_state else None
-    mm_ssd_fwd(x, delta, A, B, C, h0, 0.0, alpha, y, hT, workspace, chunk, stream)
+    mm_ssd_fwd(x, delta, A, B, C, h0, 0.0, alpha, y, hT, chunk, stream)
     return y, hT
 
 

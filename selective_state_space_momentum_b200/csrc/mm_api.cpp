@@ -35,6 +35,30 @@ mm_status ok() {
 std::atomic<int> g_forced_spt{0};
 std::atomic<int> g_forced_warps{0};
 std::atomic<int> g_forced_ts{1};
+// Scan path: 0 automatic, 1 the register-resident kernel, 2 the sequence-split
+// kernel; and its segment length (0: automatic).
+std::atomic<int> g_forced_path{0};
+std::atomic<int64_t> g_forced_seg_len{0};
+
+// The automatic path choice depends on (batch * dim, dstate, io) only, never
+// on L, so calls that split one sequence take the same path.  The
+// sequence-split kernel pads the states to 16, so it serves dstate > 8; it
+// pays off when there are few channels (the register-resident kernel then
+// cannot fill the GPU).
+bool seg_auto(int64_t batch, int64_t dim, int64_t dstate, int io) {
+    return dstate > 8 && io == MM_F32 && batch * dim <= 4096;
+}
+
+// Segment length of the sequence-split path for these sizes, or 0 when the
+// call runs on the register-resident kernel.
+int64_t seg_len_for(int64_t batch, int64_t dim, int64_t dstate, int io, bool vec_ok) {
+    const int path = g_forced_path.load();
+    if (!vec_ok || dstate > 16) return 0;
+    if (path == 1) return 0;
+    if (path == 0 && !seg_auto(batch, dim, dstate, io)) return 0;
+    const int64_t forced = g_forced_seg_len.load();
+    return forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -158,6 +182,7 @@ mm_status mm_device_status(void) {
     const cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return from_cuda(e, "mm_device_status: synchronize");
     const unsigned int w = mmscan::scan_read_and_clear_device_error() |
+                           mmscan::scan_seg_read_and_clear_device_error() |
                            mmscan::scan_bwd_read_and_clear_device_error() |
                            mmscan::ssd_read_and_clear_device_error();
     if (w) return fail(MM_ERR_DEVICE_TIMEOUT, "a device-side wait ran past its limit (word 0x%x)", w);
@@ -177,6 +202,26 @@ mm_status mm_scan_set_tile(int spt, int warps, int time_lanes) {
     g_forced_spt = spt;
     g_forced_warps = warps;
     g_forced_ts = time_lanes;
+    return ok();
+}
+
+mm_status mm_scan_set_path(int path, int64_t seg_len) {
+    if (path < 0 || path > 2)
+        return fail(MM_ERR_UNSUPPORTED, "scan path %d is not 0 (automatic), 1 or 2", path);
+    if (seg_len != 0 && (seg_len < 32 || seg_len > (int64_t(1) << 30) || (seg_len & (seg_len - 1)) != 0))
+        return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not 0 or a power of two in [32, 2^30]",
+                    (long long)seg_len);
+    g_forced_path = path;
+    g_forced_seg_len = seg_len;
+    return ok();
+}
+
+mm_status mm_scan_segment_len(const mm_scan_dims* dims, int64_t* seg_len) {
+    if (!dims || !seg_len) return fail(MM_ERR_NULL, "dims and seg_len are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, 0.0f, 1.0f, &zs)) return st;
+    *seg_len = seg_len_for(dims->batch, dims->dim, dims->dstate, dims->io,
+                           ((dims->seqlen * zs.esize) % 16) == 0);
     return ok();
 }
 
@@ -242,6 +287,12 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.Dskip = Dskip; a.z = z; a.dbias = delta_bias; a.softplus = delta_softplus ? 1 : 0;
     a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
     a.ckpt = ckpt;
+    if (!a.ext && !ckpt) {
+        const int64_t seg = seg_len_for(bsz, D, N, dims->io, a.vec_ok != 0);
+        if (seg > 0)
+            return from_cuda(mmscan::launch_scan_seg(a, dims->io, seg, static_cast<cudaStream_t>(stream)),
+                             "mm_scan_fwd launch");
+    }
     const mmscan::ScanTileChoice t =
         mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load(),
                                  g_forced_ts.load());
@@ -366,8 +417,12 @@ mm_status mm_scan_step(const void* x, const void* delta, const float* A, const v
                      "mm_scan_step launch");
 }
 
-mm_status mm_ssd_workspace_size(const mm_ssd_dims* dims, size_t* bytes) {
-    if (!dims || !bytes) return fail(MM_ERR_NULL, "dims and bytes are required");
+mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const void* B,
+                     const void* C, const float* h0, float beta, float alpha, void* y, float* hT,
+                     const mm_ssd_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !y)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
     if (dims->batch < 1 || dims->seqlen < 1 || dims->nheads < 1 || dims->headdim < 1 ||
         dims->dstate < 1 || dims->ngroups < 1 || dims->chunk < 1 ||
         dims->nheads % dims->ngroups != 0)
@@ -376,32 +431,12 @@ mm_status mm_ssd_workspace_size(const mm_ssd_dims* dims, size_t* bytes) {
     if (!mmscan::ssd_shape_supported(dims->headdim, dims->dstate, dims->chunk))
         return fail(MM_ERR_UNSUPPORTED, "SSD with headdim=%lld dstate=%lld chunk=%lld is not built",
                     (long long)dims->headdim, (long long)dims->dstate, (long long)dims->chunk);
-    *bytes = mmscan::ssd_workspace_bytes(dims->batch, dims->seqlen, dims->nheads, dims->headdim,
-                                         dims->dstate, dims->chunk);
-    return ok();
-}
-
-mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const void* B,
-                     const void* C, const float* h0, float beta, float alpha, void* y, float* hT,
-                     void* workspace, size_t workspace_bytes, const mm_ssd_dims* dims,
-                     void* stream) {
-    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
-    if (!x || !delta || !A || !B || !C || !y)
-        return fail(MM_ERR_NULL, "x, delta, A, B, C and y are required");
-    size_t need = 0;
-    mm_status st = mm_ssd_workspace_size(dims, &need);
-    if (st != MM_OK) return st;
-    if (need > 0 && !workspace)
-        return fail(MM_ERR_NULL, "a workspace of %zu bytes is required", need);
     if (!std::isfinite(beta) || beta < 0.0f || beta >= 1.0f)
         return fail(MM_ERR_SCALAR, "beta=%g is outside [0, 1)", (double)beta);
     if (beta != 0.0f)       // momentum: the chunked form with two carried states
         return mm_ssd_fwd_momentum(x, delta, A, B, C, h0, nullptr, beta, alpha, y, hT, nullptr, dims, stream);
     if (!std::isfinite(alpha) || alpha < 0.0f)
         return fail(MM_ERR_SCALAR, "alpha=%g must be finite and >= 0", (double)alpha);
-    if (workspace_bytes < need)
-        return fail(MM_ERR_DIMS, "workspace of %zu bytes is smaller than the %zu needed",
-                    workspace_bytes, need);
     const int64_t bsz = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
                   N = dims->dstate, G = dims->ngroups;
     int64_t blh, xy_bytes, bl, d_bytes, blg, bc_elems, bc_bytes, st_elems, st_bytes;
@@ -411,31 +446,28 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
         !mul_ok(bc_elems, 2, &bc_bytes) || !mul_ok(bsz, H, &bh) || !mul_ok(P, N, &pn) ||
         !mul_ok(bh, pn, &st_elems) || !mul_ok(st_elems, 4, &st_bytes))
         return fail(MM_ERR_DIMS, "sizes overflow 64-bit byte counts");
-    const void* ptrs[] = {x, delta, A, B, C, h0, y, hT, workspace};
-    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "y", "hT", "workspace"};
-    for (int i = 0; i < 9; ++i)
+    const void* ptrs[] = {x, delta, A, B, C, h0, y, hT};
+    const char* names[] = {"x", "delta", "A", "B", "C", "h0", "y", "hT"};
+    for (int i = 0; i < 8; ++i)
         if (ptrs[i] && !aligned16(ptrs[i]))
             return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
     const Range rx = rng("x", x, xy_bytes), rd = rng("delta", delta, d_bytes),
                 rA = rng("A", A, H * 4), rB = rng("B", B, bc_bytes), rC = rng("C", C, bc_bytes),
                 rh0 = rng("h0", h0, st_bytes), ry = rng("y", y, xy_bytes),
-                rhT = rng("hT", hT, st_bytes),
-                rw = rng("workspace", workspace, (int64_t)workspace_bytes);
+                rhT = rng("hT", hT, st_bytes);
     const Range* inputs[] = {&rx, &rd, &rA, &rB, &rC, &rh0};
-    for (const Range* out : {&ry, &rhT, &rw}) {
+    for (const Range* out : {&ry, &rhT}) {
         for (const Range* in : inputs) {
             if (!overlap(*out, *in)) continue;
             if (out == &rhT && in == &rh0 && out->lo == in->lo) continue;
             return fail(MM_ERR_ALIAS, "%s overlaps %s", out->name, in->name);
         }
     }
-    if (overlap(ry, rhT) || overlap(ry, rw) || overlap(rhT, rw))
-        return fail(MM_ERR_ALIAS, "outputs and workspace overlap");
+    if (overlap(ry, rhT)) return fail(MM_ERR_ALIAS, "y overlaps hT");
     if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
 
     mmscan::SSDArgs a{};
     a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.h0 = h0; a.y = y; a.hT = hT;
-    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
     a.chunk = dims->chunk; a.alpha = alpha;
     return from_cuda(mmscan::launch_ssd_fwd(a, static_cast<cudaStream_t>(stream)), "mm_ssd_fwd launch");

@@ -98,6 +98,15 @@ struct ScanTileChoice {
     int ts;      // lanes along time per state group (1, or 2 for the time split)
 };
 
+// Sequence-split scan (scan_seg.cu): segments of a power-of-two length at
+// absolute multiples of it, one per CTA of a cluster of at most
+// kSegMaxCluster CTAs, joined through their 2x2 affine carry maps.
+constexpr int kSegMaxCluster = 8;
+constexpr int64_t kSegMinLen = 16384;
+int64_t scan_seg_default_len(int64_t batch, int64_t dim);
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s);
+unsigned int scan_seg_read_and_clear_device_error();
+
 bool scan_tile_supported(int spt, int warps, int time_lanes);
 ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int io,
                                 int forced_spt, int forced_warps, int forced_ts);
@@ -119,8 +128,6 @@ struct SSDArgs {
     const float* h0;
     void* y;
     float* hT;
-    void* workspace;
-    size_t workspace_bytes;
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
     float alpha;
 };
@@ -144,8 +151,6 @@ struct SSDMomArgs {
 bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate);
 cudaError_t launch_ssd_mom(const SSDMomArgs& a, cudaStream_t s);
 
-size_t ssd_workspace_bytes(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
-                           int64_t dstate, int64_t chunk);
 bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk);
 cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t s);
 

@@ -259,11 +259,13 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // block's predecessor is fetched while the block runs
         float2 hn = start_state(k * (T / KB) + nblk - 1, 0);
         float2 vn = start_state(k * (T / KB) + nblk - 1, 1);
-        if (!mbar_wait(bar0 + 8 * s, (uint32_t)((i / ST) & 1), &g_bwd_dev_err)) return;
+        // Every thread waits; the outcome is made uniform at the barrier below, so
+        // that a wait that gave up makes the whole CTA leave together.
+        const bool waited = mbar_wait(bar0 + 8 * s, (uint32_t)((i / ST) & 1), &g_bwd_dev_err);
         const unsigned char* sbuf = smem + s * TL::STAGE_BYTES;
 
         // ---- transpose B, C to [t][n] fp32 in 4x4 blocks (alpha into B) ----
-        {
+        if (waited) {
             constexpr int NB4 = NP / 4 > 0 ? NP / 4 : 1;
             constexpr int ITEMS = NB4 * (T / 4);
             for (int it = tid; it < 2 * ITEMS; it += NT) {
@@ -301,7 +303,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         if constexpr (EXT) {
             // delta' = softplus(delta + bias) and the gated dy = dy silu(z), once per
             // (channel, step), four steps per item, into the fp32 buffers
-            for (int it = tid; it < CH * (T / 4); it += NT) {
+            for (int it = waited ? tid : CH * (T / 4); it < CH * (T / 4); it += NT) {
                 const int cc = it / (T / 4);
                 const int t4 = (it - cc * (T / 4)) * 4;
                 const int bxs = t4 / TL::BOX_T;
@@ -326,7 +328,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 *reinterpret_cast<float4*>(smem + TL::OFF_GY + fo) = make_float4(gy[0], gy[1], gy[2], gy[3]);
             }
         }
-        __syncthreads();
+        if (!__syncthreads_and(waited)) return;
         // Every thread is past the previous chunk: its stage is free.
         if (i + ST - 1 < nchunks) issue(nchunks - 1 - (i + ST - 1), (int)((i + ST - 1) % ST));
 

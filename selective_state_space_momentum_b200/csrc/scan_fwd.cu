@@ -238,13 +238,15 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const int s = (int)(k % ST);
         const int64_t t0 = k * T;
         const int nval = (int)((L - t0) < T ? (L - t0) : T);
-        if (!mbar_wait(bar0 + 8 * s, (uint32_t)((k / ST) & 1), &g_scan_dev_err)) return;
+        // Every thread waits; the outcome is made uniform at the barrier below, so
+        // that a wait that gave up makes the whole CTA leave together.
+        const bool waited = mbar_wait(bar0 + 8 * s, (uint32_t)((k / ST) & 1), &g_scan_dev_err);
         const unsigned char* sbuf = smem + s * TL::STAGE_BYTES;
         float* Bt = reinterpret_cast<float*>(smem + TL::OFF_BT + (int)(k & 1) * TL::BT_BYTES);
         float* Ct = reinterpret_cast<float*>(smem + TL::OFF_BT + (2 + (int)(k & 1)) * TL::BT_BYTES);
 
         // ---- transpose B, C to [t][n] fp32 in 4x4 blocks (alpha into B) ----
-        {
+        if (waited) {
             constexpr int NB4 = NP / 4 > 0 ? NP / 4 : 1;
             constexpr int ITEMS = NB4 * (T / 4);
             for (int i = tid; i < 2 * ITEMS; i += NT) {
@@ -282,7 +284,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         if constexpr (EXT) {
             // delta' = softplus(delta + bias) once per (channel, step) of the chunk,
             // four steps per item, as fp32 in the fp32 box layout.
-            if (p.dbias || p.softplus) {
+            if (waited && (p.dbias || p.softplus)) {
                 unsigned char* dp = (EB == 4) ? smem + s * TL::STAGE_BYTES + TL::OFF_D
                                               : smem + TL::OFF_DP + (int)(k & 1) * TL::DP_BYTES;
                 for (int i = tid; i < CH * (T / 4); i += NT) {
@@ -303,7 +305,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
         }
-        __syncthreads();
+        if (!__syncthreads_and(waited)) return;
         // Every thread is past compute(k-1): its stage and B^T/C^T buffers are free.
         if (k + ST - 1 < nchunks) issue(k + ST - 1, (int)((k + ST - 1) % ST));
 

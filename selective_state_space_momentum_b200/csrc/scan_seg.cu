@@ -1,0 +1,682 @@
+// scan_seg.cu -- sm_100a Momentum Mamba forward scan with the sequence cut
+// into segments that run on the CTAs of a thread-block cluster.
+//
+// What it computes ("Momentum Mamba: Enhanced State Space Models with
+// Momentum", "Momentum Mamba Recurrence" and "Discretization Note"), per
+// batch row b, channel d, state n:
+//     v_t = beta v_{t-1} + alpha delta_t B_t[n] x_t
+//     h_t = exp(delta_t A[d,n]) h_{t-1} + v_t
+//     y_t = sum_n C_t[n] h_t[n]
+//
+// Why segments.  A sequence with few channels (one row of 2048 channels, say)
+// gives too few independent (channel, state) lanes to keep 148 SMs busy when
+// each lane walks the whole sequence.  The recurrence is affine in its start
+// state, so the sequence is cut into segments of S steps (S a power of two,
+// fixed for a given (batch * dim, dstate, io), never derived from L) that run
+// side by side, each from a zero state, and are joined afterwards; this is the
+// "Forward Pass: Two-Stage Parallel Scan" of the same page (chunk scans, then
+// a running prefix of the chunk carries) with the chunk carry kept as a 2x2
+// affine map per lane:
+//   * Main pass (one CTA per segment).  From v = h = 0 the CTA runs the
+//     segment, stores its read-out y0_t, and keeps, per lane, the zero-start
+//     end state (zv, zh), the response of h at the end to a unit velocity at
+//     the start, Q = sum_j beta^(j+1) prod_{s>j} a_s (one extra FMA per
+//     update: q_t = a_t q_{t-1} + beta^(t+1)), and P = prod_s a_s, formed as
+//     2^(A log2e * sum_s delta_s).  The segment maps a start state (v, h) to
+//         v' = beta^S v + zv,   h' = P h + Q v + zh.
+//   * Carry fold.  The CTAs of a cluster hold consecutive segments of the
+//     same channels.  After a cluster barrier each CTA reads the maps of the
+//     segments before its own from the other CTAs' shared memory
+//     (distributed shared memory, no global scratch) and folds them in
+//     segment order onto the concrete carry, starting from (h0, v0).  Every
+//     CTA folds the same maps in the same order, so the carries -- and hT, vT,
+//     which are the carry after the last segment -- do not depend on how the
+//     cluster or the call is cut: two calls split at a multiple of S give hT,
+//     vT bit-identical to one call.
+//   * Correction.  The true state inside segment k is the zero-start state
+//     plus the response to the carry-in (v_in, h_in):  r_v <- beta r_v,
+//     r_h <- a_t r_h + r_v, added to y as C_t . r_h.  The response decays; it
+//     is run until the bound |r_h| + beta/(1-beta) |r_v| -- which caps every
+//     later |r_h| while every a_t <= 1 (A <= 0 and delta >= 0 over the
+//     segment, checked) -- falls below 2^-25 of its start value for every lane
+//     of the CTA, or to the segment's end.  The y it leaves out is below fp32
+//     rounding of the state.
+//   * Sequences longer than cluster-size * S: the cluster walks rounds of
+//     consecutive segments, each round folding onto the previous one's carry.
+//
+// Lanes.  One warp owns 16 channels of one batch row: lane = 4 p + g holds
+// channels 2p, 2p+1 and states 4g .. 4g+3 (v, h and q in fp32 registers), so
+// each B_t / C_t value read from shared memory serves two channels and each
+// delta_t / x_t value four states.  The four lanes of a channel pair add
+// their read-outs with a register butterfly and store whole 32-byte pieces
+// of y.  Staging: one thread issues TMA tile loads (no multicast) of x, delta
+// (box 128 bytes of steps x 16 channels) and B, C (x 16 states) into 128-byte
+// swizzled tiles; B, C are then transposed to [t][n] fp32 (alpha folded into
+// B) so that a lane reads its four states of a step with one vector load.
+#include <cuda.h>
+
+#include <atomic>
+
+#include "mm_common.cuh"
+#include "mm_internal.h"
+#include "mm_tma_host.h"
+
+namespace mmscan {
+
+// Device error word of this file's kernel (bounded waits that gave up).
+static __device__ unsigned int g_seg_dev_err = 0;
+
+// 2^-25: the correction stops once every lane's response bound fell by this factor.
+constexpr float kCorrTol = 2.98023223876953125e-8f;
+
+template <typename IO, int W, int ST>
+struct SegTile {
+    static constexpr int NP = 16;                // states, padded
+    static constexpr int G = 4;                  // lanes per channel pair (4 states each)
+    static constexpr int CPW = 16;               // channels per warp
+    static constexpr int CH = W * CPW;           // channels per CTA
+    static constexpr int NT = W * 32;
+    static constexpr int EB = IOTraits<IO>::kBytes;
+    static constexpr int T = 128 / EB;           // steps per chunk: one 128-byte swizzled row
+    static constexpr int XBOX = CH * 128;        // one x (or delta) tile
+    static constexpr int BBOX = NP * 128;        // one B (or C) tile
+    static constexpr int OFF_X = 0, OFF_D = XBOX, OFF_B = 2 * XBOX, OFF_C = 2 * XBOX + BBOX;
+    static constexpr int STAGE_BYTES = 2 * XBOX + 2 * BBOX;
+    static constexpr int MAIN_TX = STAGE_BYTES;  // main pass: x, delta, B, C
+    static constexpr int CORR_TX = XBOX + BBOX;  // correction: delta, C
+    static constexpr int BT_BYTES = T * NP * 4;  // one transposed [t][n] fp32 matrix
+    static constexpr int OFF_BT = ST * STAGE_BYTES;
+    static constexpr int OFF_CT = OFF_BT + BT_BYTES;
+    // The segment maps (8 float4 per thread) are published in the B^T/C^T area.
+    static constexpr int AGG_BYTES = NT * 8 * 16;
+    // The concrete carry (v, h) of each lane's 8 states between folds.
+    static constexpr int OFF_CARRY = OFF_BT + 2 * BT_BYTES;
+    static constexpr int CARRY_BYTES = NT * 16 * 4;
+    static constexpr int OFF_BAR = OFF_CARRY + CARRY_BYTES;
+    static constexpr int SMEM_BYTES = OFF_BAR + ST * 8 + 1024;    // + alignment slack
+    static_assert(AGG_BYTES <= 2 * BT_BYTES, "segment maps fit the transposed area");
+    static_assert(STAGE_BYTES % 1024 == 0, "tiles stay 1024-byte aligned");
+    static_assert(T % 8 == 0, "8-step groups");
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float4 dsmem_ld4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+    return v;
+}
+
+// beta^n by binary powering: the same value wherever a segment's length is n.
+__device__ __forceinline__ float pow_steps(float beta, int64_t n) {
+    float r = 1.0f, b = beta;
+    while (n > 0) {
+        if (n & 1) r *= b;
+        b *= b;
+        n >>= 1;
+    }
+    return r;
+}
+
+template <typename IO, int W, int ST>
+__global__ void __launch_bounds__(W * 32)
+scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
+                const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+                const ScanArgs p, const int64_t seg_len, const int csize) {
+    using TL = SegTile<IO, W, ST>;
+    constexpr int NT = TL::NT, T = TL::T, CH = TL::CH, EB = TL::EB, G = TL::G;
+
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (base - raw_addr);
+    float* Bt = reinterpret_cast<float*>(smem + TL::OFF_BT);
+    float* Ct = reinterpret_cast<float*>(smem + TL::OFF_CT);
+    float4* agg = reinterpret_cast<float4*>(smem + TL::OFF_BT);
+    const uint32_t agg_addr = base + TL::OFF_BT;
+    const uint32_t bar0 = base + TL::OFF_BAR;
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int g = lane & (G - 1);                 // state group: states 4g .. 4g+3
+    const int pr = lane >> 2;                     // channel pair within the warp
+    const int rank = (int)cluster_ctarank();      // segment within the round
+    const int64_t cl = blockIdx.x / csize;        // (batch row, channel tile)
+    const int64_t b = cl / p.tiles_per_batch;
+    const int64_t d0 = (cl % p.tiles_per_batch) * CH;
+    const int cc0 = warp * TL::CPW + 2 * pr;      // first channel of the pair, within the CTA
+    const int64_t L = p.seqlen;
+    const int N = p.dstate;
+    const float beta = p.beta;
+    const int64_t nseg = (L + seg_len - 1) / seg_len;
+    const int64_t rounds = (nseg + csize - 1) / csize;
+
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, 1u);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // ---- per-lane constants ---------------------------------------------------
+    bool act[2];
+    int64_t dch[2];
+    float Al[2][4];               // A[d, 4g + e] log2 e
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        dch[c] = d0 + cc0 + c;
+        act[c] = dch[c] < p.dim;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int n = 4 * g + e;
+            Al[c][e] = (act[c] && n < N) ? p.A[dch[c] * N + n] * kLog2e : 0.0f;
+        }
+    }
+    bool a_nonpos = true;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a_nonpos = a_nonpos && (Al[c][e] <= 0.0f);
+    a_nonpos = __syncthreads_and(a_nonpos) != 0;
+
+    // The concrete carry entering the current round, per lane (c, e): starts at
+    // (h0, v0); kept in shared memory between folds ([c][e][v/h][thread]).
+    float* carry_s = reinterpret_cast<float*>(smem + TL::OFF_CARRY);
+    auto carry_at = [&](int c, int e, int which) -> float& { return carry_s[((c * 4 + e) * 2 + which) * NT + tid]; };
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int n = 4 * g + e;
+            float v = 0.0f, h = 0.0f;
+            if (act[c] && n < N) {
+                const int64_t si = (b * p.dim + dch[c]) * N + n;
+                if (p.h0) h = p.h0[si];
+                if (p.v0) v = p.v0[si];
+            }
+            carry_at(c, e, 0) = v;
+            carry_at(c, e, 1) = h;
+        }
+
+    // ---- TMA staging --------------------------------------------------------------
+    // Chunks are consumed in the order they are issued; `issued` / `consumed`
+    // count them over the whole kernel and give each its stage and phase.
+    int64_t issued = 0, consumed = 0;
+    bool dead = false;            // a bounded wait gave up: skip the work, keep the barriers
+    auto issue = [&](int64_t t0, bool main_pass) {
+        const int s = (int)(issued % ST);
+        if (tid == 0) {
+            const uint32_t sb = base + s * TL::STAGE_BYTES;
+            const uint32_t bar = bar0 + 8 * s;
+            mbar_expect_tx(bar, main_pass ? TL::MAIN_TX : TL::CORR_TX);
+            const int tc = (int)t0;
+            tma_load_3d(sb + TL::OFF_D, &tm_d, bar, tc, (int)d0, (int)b);
+            tma_load_3d(sb + TL::OFF_C, &tm_C, bar, tc, 0, (int)b);
+            if (main_pass) {
+                tma_load_3d(sb + TL::OFF_X, &tm_x, bar, tc, (int)d0, (int)b);
+                tma_load_3d(sb + TL::OFF_B, &tm_B, bar, tc, 0, (int)b);
+            }
+        }
+        ++issued;
+    };
+    // Wait for the oldest issued chunk; the outcome is made uniform over the CTA.
+    auto wait_next = [&]() -> const unsigned char* {
+        const int s = (int)(consumed % ST);
+        const uint32_t par = (uint32_t)((consumed / ST) & 1);
+        bool ok = mbar_wait(bar0 + 8 * s, par, &g_seg_dev_err);
+        ok = __syncthreads_and(ok) != 0;
+        ++consumed;
+        if (!ok) dead = true;
+        return smem + s * TL::STAGE_BYTES;
+    };
+    // Drain chunks issued but not consumed (the correction may stop early).
+    auto drain = [&]() {
+        while (!dead && consumed < issued) (void)wait_next();
+    };
+
+    // B, C of a staged chunk to [t][n] fp32 (alpha into B); `withB` false: C only.
+    auto transpose = [&](const unsigned char* sbuf, bool withB) {
+        const int items = withB ? 2 * 4 * (T / 4) : 4 * (T / 4);
+        for (int i = tid; i < items; i += NT) {
+            const int which = withB ? (i / (4 * (T / 4))) : 1;     // 0 = B, 1 = C
+            const int rem = i % (4 * (T / 4));
+            const int n0 = (rem & 3) * 4;
+            const int t4 = (rem >> 2) * 4;
+            const unsigned char* tile = sbuf + (which ? TL::OFF_C : TL::OFF_B);
+            float m[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float4 q = load4(reinterpret_cast<const IO*>(tile + sw128(n0 + r, t4 * EB)));
+                m[r][0] = q.x; m[r][1] = q.y; m[r][2] = q.z; m[r][3] = q.w;
+            }
+            const float sc = which ? 1.0f : p.alpha;
+            float* dst = (which ? Ct : Bt) + t4 * TL::NP + n0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<float4*>(dst + j * TL::NP) =
+                    make_float4(m[0][j] * sc, m[1][j] * sc, m[2][j] * sc, m[3][j] * sc);
+        }
+    };
+
+    // delta, x of the two channels for 4 steps from a staged tile.
+    auto load_dx = [&](const unsigned char* sbuf, int off, int tau, float (&v)[2][4]) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const float4 q = load4(reinterpret_cast<const IO*>(sbuf + off + sw128(cc0 + c, tau * EB)));
+            v[c][0] = q.x; v[c][1] = q.y; v[c][2] = q.z; v[c][3] = q.w;
+        }
+    };
+
+    // The lane's output after the butterfly: channel cc0 + (g >> 1), steps 4 (g & 1) .. + 3 of a group.
+    const bool oact = (g >> 1) ? act[1] : act[0];
+    const int64_t odch = (g >> 1) ? dch[1] : dch[0];
+    IO* const orow = static_cast<IO*>(p.y) + (b * p.dim + (oact ? odch : 0)) * L;
+    const int ostep = (g & 1) * 4;
+
+    const float2 beta2 = f2(beta, beta);
+    const float kappa = beta / (1.0f - beta);
+
+    // Four steps of the two channels: delta (and, on the main pass, the input
+    // delta * x) and the exponentials 2^(delta A log2 e) of the four states.
+    struct Quad {
+        float u[2][4];
+        float a[2][4][4];          // [channel][state][step]
+    };
+    // Main pass state of the segment (zero start) and its running sums.
+    float2 vv[2][2], hh[2][2], qq[2][2];
+    float2 bp2;                   // beta^(t+1)
+    float2 dacc[2];               // sum of delta over the current chunk, (even, odd) steps
+    uint32_t dbits;               // OR of delta's bit patterns over the segment
+    auto prep = [&](const unsigned char* sbuf, int tau, Quad& Q, bool main_pass) {
+        float dl[2][4];
+        load_dx(sbuf, TL::OFF_D, tau, dl);
+        if (main_pass) {
+            float xl[2][4];
+            load_dx(sbuf, TL::OFF_X, tau, xl);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+#pragma unroll
+                for (int j2 = 0; j2 < 4; j2 += 2) {
+                    const float2 uu = __fmul2_rn(f2(dl[c][j2], dl[c][j2 + 1]), f2(xl[c][j2], xl[c][j2 + 1]));
+                    Q.u[c][j2] = uu.x;
+                    Q.u[c][j2 + 1] = uu.y;
+                }
+                dbits |= __float_as_uint(dl[c][0]) | __float_as_uint(dl[c][1]) |
+                         __float_as_uint(dl[c][2]) | __float_as_uint(dl[c][3]);
+                // steps past the end of the sequence are zero-filled by TMA: no effect on the sum
+                dacc[c] = __fadd2_rn(dacc[c], __fadd2_rn(f2(dl[c][0], dl[c][1]), f2(dl[c][2], dl[c][3])));
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j2 = 0; j2 < 4; j2 += 2)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 ex = __fmul2_rn(f2(dl[c][j2], dl[c][j2 + 1]), f2(Al[c][e], Al[c][e]));
+                    Q.a[c][e][j2] = ex2_approx(ex.x);
+                    Q.a[c][e][j2 + 1] = ex2_approx(ex.y);
+                }
+    };
+
+    // The four steps of Q from chunk step tau; partial read-outs into yk[c][j0 + j].
+    // `ragged`: steps at or past nval leave the state alone (the last chunk).
+    auto main_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int step = tau + j;
+            const bool valid = !ragged || step < nval;
+            const float4 b4 = *reinterpret_cast<const float4*>(Bt + step * TL::NP + 4 * g);
+            const float4 c4 = *reinterpret_cast<const float4*>(Ct + step * TL::NP + 4 * g);
+            const float2 bq[2] = {f2(b4.x, b4.y), f2(b4.z, b4.w)};
+            const float2 cq[2] = {f2(c4.x, c4.y), f2(c4.z, c4.w)};
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float2 uu = f2(Q.u[c][j], Q.u[c][j]);
+                float2 yy;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float2 aa = f2(Q.a[c][2 * q][j], Q.a[c][2 * q + 1][j]);
+                    const float2 w = __fmul2_rn(uu, bq[q]);
+                    const float2 vn = __ffma2_rn(beta2, vv[c][q], w);
+                    const float2 hn = __ffma2_rn(aa, hh[c][q], vn);
+                    const float2 qn = __ffma2_rn(aa, qq[c][q], bp2);
+                    if (valid) { vv[c][q] = vn; hh[c][q] = hn; qq[c][q] = qn; }
+                    yy = q == 0 ? __fmul2_rn(cq[0], hh[c][0]) : __ffma2_rn(cq[1], hh[c][1], yy);
+                }
+                yk[c][j0 + j] = yy.x + yy.y;
+            }
+            if (valid) bp2 = __fmul2_rn(bp2, beta2);
+        }
+    };
+
+    // Add the four lanes' partials of an 8-step group and store (or add to) y.
+    auto flush = [&](const float (&yk)[2][8], int64_t t0, int first8, int nval, bool add) {
+        float out[4];
+        butterfly_sum<G, 16>(*reinterpret_cast<const float(*)[16]>(&yk[0][0]), out, g);
+        const int first = first8 + ostep;
+        const int cnt = nval - first < 4 ? nval - first : 4;
+        if (!oact || cnt <= 0) return;
+        IO* yp = orow + t0 + first;
+        if (add) {
+            if (cnt == 4) {
+                const float4 q4 = load4(static_cast<const IO*>(yp));
+                out[0] += q4.x; out[1] += q4.y; out[2] += q4.z; out[3] += q4.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (e < cnt) out[e] += load1(static_cast<const IO*>(yp + e));
+            }
+        }
+        store_steps_n<IO, 4>(yp, out, cnt, true);
+    };
+
+    // Correction state: the response to the carry-in.
+    float2 rvv[2][2], rhh[2][2];
+    auto corr_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int step = tau + j;
+            const bool valid = !ragged || step < nval;
+            const float4 c4 = *reinterpret_cast<const float4*>(Ct + step * TL::NP + 4 * g);
+            const float2 cq[2] = {f2(c4.x, c4.y), f2(c4.z, c4.w)};
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float2 yy;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float2 aa = f2(Q.a[c][2 * q][j], Q.a[c][2 * q + 1][j]);
+                    const float2 vn = __fmul2_rn(beta2, rvv[c][q]);
+                    const float2 hn = __ffma2_rn(aa, rhh[c][q], vn);
+                    if (valid) { rvv[c][q] = vn; rhh[c][q] = hn; }
+                    yy = q == 0 ? __fmul2_rn(cq[0], rhh[c][0]) : __ffma2_rn(cq[1], rhh[c][1], yy);
+                }
+                yk[c][j0 + j] = yy.x + yy.y;
+            }
+        }
+    };
+
+    // One staged chunk: full chunks run unpredicated with each group's loads and
+    // exponentials issued one group ahead; the last chunk of the sequence is ragged.
+    auto run_chunk = [&](const unsigned char* sbuf, int64_t t0, int nval, bool main_pass) {
+        float yk[2][8] = {};
+        if (nval == T) {
+            Quad Q0, Q1;
+            prep(sbuf, 0, Q0, main_pass);
+#pragma unroll 1
+            for (int g8 = 0; g8 < T; g8 += 8) {
+                prep(sbuf, g8 + 4, Q1, main_pass);
+                if (main_pass) main_steps(Q0, g8, 0, yk, false, T);
+                else corr_steps(Q0, g8, 0, yk, false, T);
+                if (g8 + 8 < T) prep(sbuf, g8 + 8, Q0, main_pass);
+                if (main_pass) main_steps(Q1, g8 + 4, 4, yk, false, T);
+                else corr_steps(Q1, g8 + 4, 4, yk, false, T);
+                flush(yk, t0, g8, T, !main_pass);
+            }
+        } else {
+#pragma unroll 1
+            for (int g8 = 0; g8 < nval; g8 += 8) {
+                Quad Q;
+                prep(sbuf, g8, Q, main_pass);
+                if (main_pass) main_steps(Q, g8, 0, yk, true, nval);
+                else corr_steps(Q, g8, 0, yk, true, nval);
+                if (g8 + 4 < nval) {
+                    prep(sbuf, g8 + 4, Q, main_pass);
+                    if (main_pass) main_steps(Q, g8 + 4, 4, yk, true, nval);
+                    else corr_steps(Q, g8 + 4, 4, yk, true, nval);
+                }
+                flush(yk, t0, g8, nval, !main_pass);
+            }
+        }
+    };
+
+    for (int64_t r = 0; r < rounds; ++r) {
+        const int64_t k = r * csize + rank;                       // this CTA's segment
+        const int64_t s0 = k * seg_len;
+        const int64_t slen = s0 < L ? (L - s0 < seg_len ? L - s0 : seg_len) : 0;
+        const int64_t nch = (slen + T - 1) / T;
+
+        // ================= main pass: the segment from a zero state ==============
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) vv[c][q] = hh[c][q] = qq[c][q] = f2(0.0f, 0.0f);
+        bp2 = beta2;
+        float dsum[2] = {0.0f, 0.0f};                             // sum of delta over the segment
+        dbits = 0;
+        if (!dead && nch > 0) {
+            for (int64_t j = 0; j < ST && j < nch; ++j) issue(s0 + j * T, true);
+            for (int64_t kc = 0; kc < nch; ++kc) {
+                const unsigned char* sbuf = wait_next();
+                if (dead) break;
+                const int64_t t0 = s0 + kc * T;
+                const int nval = (int)(slen - kc * T < T ? slen - kc * T : T);
+                transpose(sbuf, true);
+                __syncthreads();
+                dacc[0] = dacc[1] = f2(0.0f, 0.0f);
+                run_chunk(sbuf, t0, nval, true);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) dsum[c] += dacc[c].x + dacc[c].y;
+                __syncthreads();          // every lane is done with this stage and B^T, C^T
+                const int64_t nx = kc + ST;
+                if (nx < nch) issue(s0 + nx * T, true);
+            }
+            drain();
+        }
+
+        // ================= publish this segment's map; fold the carries ===========
+        const bool seg_nonneg = __syncthreads_and((dbits & 0x80000000u) == 0u) != 0;
+        if (!dead) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float P0 = ex2_approx(Al[c][2 * q] * dsum[c]);
+                    const float P1 = ex2_approx(Al[c][2 * q + 1] * dsum[c]);
+                    const int i0 = (c * 2 + q) * 2;
+                    agg[i0 * NT + tid] = make_float4(vv[c][q].x, vv[c][q].y, hh[c][q].x, hh[c][q].y);
+                    agg[(i0 + 1) * NT + tid] = make_float4(qq[c][q].x, qq[c][q].y, P0, P1);
+                }
+        }
+        cluster_sync_all();               // every segment's map is published
+        float cv[2][4], ch[2][4];         // the concrete carry, folded segment by segment
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { cv[c][e] = carry_at(c, e, 0); ch[c][e] = carry_at(c, e, 1); }
+        float rv[2][4], rh[2][4];         // this segment's carry-in
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { rv[c][e] = 0.0f; rh[c][e] = 0.0f; }
+        for (int jr = 0; jr < csize; ++jr) {
+            if (jr == rank) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { rv[c][e] = cv[c][e]; rh[c][e] = ch[c][e]; }
+            }
+            const int64_t kj = r * csize + jr;
+            const int64_t sj = kj * seg_len;
+            const int64_t lj = sj < L ? (L - sj < seg_len ? L - sj : seg_len) : 0;
+            if (lj <= 0 || dead) continue;
+            const float bS = pow_steps(beta, lj);
+            const uint32_t ra = dsmem_map(agg_addr, (uint32_t)jr);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int i0 = (c * 2 + q) * 2;
+                    const float4 zvh = dsmem_ld4(ra + (uint32_t)((i0 * NT + tid) * 16));
+                    const float4 qp = dsmem_ld4(ra + (uint32_t)(((i0 + 1) * NT + tid) * 16));
+                    const float zv[2] = {zvh.x, zvh.y}, zh[2] = {zvh.z, zvh.w};
+                    const float Qm[2] = {qp.x, qp.y}, Pm[2] = {qp.z, qp.w};
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int e = 2 * q + e2;
+                        const float hn = fmaf(Pm[e2], ch[c][e], fmaf(Qm[e2], cv[c][e], zh[e2]));
+                        cv[c][e] = fmaf(bS, cv[c][e], zv[e2]);
+                        ch[c][e] = hn;
+                    }
+                }
+        }
+        cluster_sync_all();               // every CTA has read the maps: the area is free again
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { carry_at(c, e, 0) = cv[c][e]; carry_at(c, e, 1) = ch[c][e]; }
+
+        // ================= correction: the response to the carry-in ==============
+        bool any = false;
+        float bnd0[2][4];
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                bnd0[c][e] = fabsf(rh[c][e]) + kappa * fabsf(rv[c][e]);
+                any = any || rv[c][e] != 0.0f || rh[c][e] != 0.0f;
+            }
+        any = __syncthreads_or(any) != 0;
+        const bool can_stop = a_nonpos && seg_nonneg;
+        if (!dead && any && nch > 0) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    rvv[c][q] = f2(rv[c][2 * q], rv[c][2 * q + 1]);
+                    rhh[c][q] = f2(rh[c][2 * q], rh[c][2 * q + 1]);
+                }
+            for (int64_t j = 0; j < ST && j < nch; ++j) issue(s0 + j * T, false);
+            for (int64_t kc = 0; kc < nch; ++kc) {
+                const unsigned char* sbuf = wait_next();
+                if (dead) break;
+                const int64_t t0 = s0 + kc * T;
+                const int nval = (int)(slen - kc * T < T ? slen - kc * T : T);
+                transpose(sbuf, false);
+                __syncthreads();
+                run_chunk(sbuf, t0, nval, false);
+                // Stop once every lane's response bound has fallen below 2^-25 of its start.
+                bool small = can_stop;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const float b0 = fabsf(rhh[c][q].x) + kappa * fabsf(rvv[c][q].x);
+                        const float b1 = fabsf(rhh[c][q].y) + kappa * fabsf(rvv[c][q].y);
+                        small = small && b0 <= kCorrTol * bnd0[c][2 * q] && b1 <= kCorrTol * bnd0[c][2 * q + 1];
+                    }
+                const bool stop = __syncthreads_and(small) != 0;   // also: every lane is done with this stage
+                if (stop) break;
+                const int64_t nx = kc + ST;
+                if (nx < nch) issue(s0 + nx * T, false);
+            }
+            drain();
+        }
+    }
+
+    // ---- final states: the carry after the last segment -----------------------
+    if (rank == 0 && !dead) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int n = 4 * g + e;
+                if (act[c] && n < N) {
+                    const int64_t si = (b * p.dim + dch[c]) * N + n;
+                    if (p.hT) p.hT[si] = carry_at(c, e, 1);
+                    if (p.vT) p.vT[si] = carry_at(c, e, 0);
+                }
+            }
+    }
+}
+
+// ------------------------------------------------------------- launch -----
+namespace {
+
+constexpr int kSegWarps = 1;
+constexpr int kSegStages = 2;
+
+template <typename IO>
+cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream) {
+    using TL = SegTile<IO, kSegWarps, kSegStages>;
+    ScanArgs a = a0;
+    a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
+    const int64_t nseg = (a.seqlen + seg_len - 1) / seg_len;
+    const int csize = (int)(nseg < kSegMaxCluster ? nseg : kSegMaxCluster);
+    const int64_t grid = (int64_t)csize * a.batch * a.tiles_per_batch;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    CUtensorMap mx, md, mB, mC;
+    const bool bf = sizeof(IO) == 2;
+    const uint64_t L = (uint64_t)a.seqlen;
+    cudaError_t e;
+    if ((e = make_map_3d(&mx, a.x, bf, L, a.dim, a.batch, TL::T, TL::CH)) != cudaSuccess) return e;
+    if ((e = make_map_3d(&md, a.delta, bf, L, a.dim, a.batch, TL::T, TL::CH)) != cudaSuccess) return e;
+    if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
+    if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
+    auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages>;
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM_BYTES)) !=
+            cudaSuccess)
+            return e;
+        attr_done.fetch_or(bit, std::memory_order_release);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(TL::NT, 1, 1);
+    cfg.dynamicSmemBytes = TL::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize);
+}
+
+}  // namespace
+
+int64_t scan_seg_default_len(int64_t batch, int64_t dim) {
+    // About 2^25 channel-steps per round of segments: 16384 steps for 2048
+    // channels (eight segments of a 131072-step sequence), longer for fewer
+    // channels, never shorter than 16384 so that the correction -- a few
+    // thousand steps at beta = 0.99 -- stays a small part of a segment.
+    const int64_t ch = batch * dim;
+    int64_t s = kSegMinLen;
+    while (s < (int64_t(1) << 30) && s * ch < (int64_t(1) << 25)) s <<= 1;
+    return s;
+}
+
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s) {
+    if (io == 0) return launch_seg<float>(a, seg_len, s);
+    return launch_seg<bf16>(a, seg_len, s);
+}
+
+unsigned int scan_seg_read_and_clear_device_error() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_seg_dev_err, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_seg_dev_err, &z, sizeof(z));
+    return v;
+}
+
+}  // namespace mmscan

@@ -628,7 +628,6 @@ bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk) {
     return headdim == ssd::P && dstate == ssd::NS && (chunk == 128 || chunk == 256);
 }
 
-size_t ssd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t) { return 0; }
 
 cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t stream) {
     if (a.batch * a.nheads > 0x7fffffffLL || a.seqlen > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

@@ -41,6 +41,9 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs&, int, cudaStream_t) { ++g_launche
 cudaError_t launch_scan_step(const ScanStepArgs&, int, cudaStream_t) { ++g_launches; return cudaSuccess; }
 cudaError_t launch_ssd_fwd(const SSDArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
 cudaError_t launch_ssd_mom(const SSDMomArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
+int64_t scan_seg_default_len(int64_t, int64_t) { return 16384; }
+cudaError_t launch_scan_seg(const ScanArgs&, int, int64_t, cudaStream_t) { ++g_launches; return cudaSuccess; }
+unsigned int scan_seg_read_and_clear_device_error() { return 0; }
 unsigned int scan_read_and_clear_device_error() { return 0; }
 unsigned int scan_bwd_read_and_clear_device_error() { return 0; }
 unsigned int ssd_read_and_clear_device_error() { return 0; }
@@ -50,7 +53,6 @@ bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk) {
 bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate) {
     return headdim >= 1 && headdim <= 64 && dstate >= 1 && dstate <= 128;
 }
-size_t ssd_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t) { return 0; }
 }  // namespace mmscan
 
 // ---- the driver ---------------------------------------------------------------
@@ -93,13 +95,13 @@ void scan_calls(const mm_scan_dims& d, float beta, float alpha) {
                                ffake(6), beta, alpha, fake(7), &one, nullptr), "mm_scan_step");
     size_t bytes = 0;
     expect_status(mm_scan_ckpt_size(&d, &bytes), "mm_scan_ckpt_size");
+    int64_t seg = 0;
+    expect_status(mm_scan_segment_len(&d, &seg), "mm_scan_segment_len");
 }
 
 void ssd_calls(const mm_ssd_dims& d, float beta, float alpha) {
-    size_t bytes = 0;
-    expect_status(mm_ssd_workspace_size(&d, &bytes), "mm_ssd_workspace_size");
     expect_status(mm_ssd_fwd(fake(0), ffake(1), ffake(2), fake(3), fake(4), ffake(5), beta, alpha, fake(6), ffake(7),
-                             fake(8), 1u << 20, &d, nullptr), "mm_ssd_fwd");
+                             &d, nullptr), "mm_ssd_fwd");
     expect_status(mm_ssd_fwd_momentum(fake(0), ffake(1), ffake(2), fake(3), fake(4), ffake(5), ffake(9), beta, alpha,
                                       fake(6), ffake(7), ffake(10), &d, nullptr), "mm_ssd_fwd_momentum");
 }
@@ -141,7 +143,7 @@ int main() {
         ++g_bad;
     }
     const mm_ssd_dims sok = {1, 256, 2, 64, 128, 1, 256};
-    if (mm_ssd_fwd(fake(0), ffake(1), ffake(2), fake(3), fake(4), nullptr, 0.0f, 1.0f, fake(6), nullptr, nullptr, 0,
+    if (mm_ssd_fwd(fake(0), ffake(1), ffake(2), fake(3), fake(4), nullptr, 0.0f, 1.0f, fake(6), nullptr,
                    &sok, nullptr) != MM_OK || g_launches != before + 2) {
         std::printf("an in-range SSD call did not launch\n");
         ++g_bad;

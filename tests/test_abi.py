@@ -231,31 +231,46 @@ def test_set_tile(lib):
     assert lib.mm_scan_set_tile(0, 0, 0) == 0
 
 
+def test_set_path_and_segment_length_query(lib):
+    assert lib.mm_scan_set_path(3, 0) == 6
+    assert lib.mm_scan_set_path(2, 48) == 6                       # not a power of two
+    assert lib.mm_scan_set_path(2, 16) == 6                       # below 32
+    seg = ctypes.c_int64(-1)
+    dims = mm.ScanDims(1, 131072, 2048, 16, 0)
+    assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 16384
+    assert lib.mm_scan_set_path(2, 256) == 0
+    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg)) == 0
+    assert seg.value == 256                                       # forced onto the sequence-split path
+    assert lib.mm_scan_set_path(1, 0) == 0
+    assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 0
+    assert lib.mm_scan_set_path(0, 0) == 0
+    unaligned = mm.ScanDims(1, 131071, 2048, 16, 0)               # rows not whole 16-byte pieces
+    assert lib.mm_scan_segment_len(ctypes.byref(unaligned), ctypes.byref(seg)) == 0 and seg.value == 0
+    assert lib.mm_scan_segment_len(None, ctypes.byref(seg)) == 1
+    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(0, 1, 1, 1, 0)), ctypes.byref(seg)) == 2
+
+
 def test_ssd_rejects_bad_arguments(lib, monkeypatch):
     dims = mm.SSDDims(1, 512, 4, 64, 128, 1, 256)
-    size = ctypes.c_size_t(123)
-    assert lib.mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == 0
-    assert size.value == 0                                        # the state stays on chip
-    bad = mm.SSDDims(1, 512, 4, 64, 128, 3, 256)                  # H % G != 0
-    assert lib.mm_ssd_workspace_size(ctypes.byref(bad), ctypes.byref(size)) == 2
-    for odd in (mm.SSDDims(1, 512, 4, 48, 128, 1, 256), mm.SSDDims(1, 512, 4, 64, 64, 1, 256),
-                mm.SSDDims(1, 512, 4, 64, 128, 1, 64)):
-        assert lib.mm_ssd_workspace_size(ctypes.byref(odd), ctypes.byref(size)) == 6
 
-    def call(beta=0.0, alpha=1.0, ws=0, **over):
+    def call(beta=0.0, alpha=1.0, d=None, **over):
         a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), h0=None,
-                 y=_fake(5), hT=None, w=None)
+                 y=_fake(5), hT=None)
         a.update(over)
         return lib.mm_ssd_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], a["h0"], beta, alpha,
-                              a["y"], a["hT"], a["w"], ws, ctypes.byref(dims), None)
+                              a["y"], a["hT"], ctypes.byref(d or dims), None)
     assert call(x=None) == 1
     assert call(beta=1.5) == 3
     assert call(alpha=-2.0) == 3
     assert call(y=_fake(0)) == 9
     assert call(hT=_fake(3)) == 9
     assert call(B=ctypes.c_void_p(A16 * 4 + 8)) == 5
+    assert call(d=mm.SSDDims(1, 512, 4, 64, 128, 3, 256)) == 2                # H % G != 0
+    for odd in (mm.SSDDims(1, 512, 4, 48, 128, 1, 256), mm.SSDDims(1, 512, 4, 64, 64, 1, 256),
+                mm.SSDDims(1, 512, 4, 64, 128, 1, 64)):
+        assert call(d=odd) == 6
     monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
-    assert call() == 7                                            # no workspace needed
+    assert call() == 7
     assert call(h0=_fake(6), hT=_fake(6)) == 7                   # in-place final state
     assert call(beta=0.5) == 7                                    # momentum: the chunked momentum path
 
@@ -307,10 +322,10 @@ def test_sizes_past_the_32_bit_index_range_are_refused(lib):
     assert _scan(lib, D(batch=1 << 31)) == 6
     assert _scan(lib, D(dim=1 << 31)) == 6
     assert _scan(lib, D(batch=(1 << 31) - 1, dim=(1 << 31) - 1, L=1 << 30)) == 2   # bytes overflow
-    size = ctypes.c_size_t(0)
     for dims in (mm.SSDDims(1, (1 << 30) + 1, 4, 64, 128, 1, 256), mm.SSDDims(1 << 29, 64, 4, 64, 128, 1, 256),
                  mm.SSDDims(1 << 40, 64, 1 << 40, 64, 128, 1, 256)):
-        assert lib.mm_ssd_workspace_size(ctypes.byref(dims), ctypes.byref(size)) == 6
+        assert lib.mm_ssd_fwd(_fake(0), _fake(1), _fake(2), _fake(3), _fake(4), None, 0.0, 1.0, _fake(5), None,
+                              ctypes.byref(dims), None) == 6
         st = lib.mm_ssd_fwd_momentum(_fake(0), _fake(1), _fake(2), _fake(3), _fake(4), None, None, 0.9, 1.0,
                                      _fake(5), None, None, ctypes.byref(dims), None)
         assert st == 6

@@ -131,9 +131,14 @@ def test_checkpoints_are_the_states_after_each_chunk():
     # the last checkpoint is the final state itself, and keeping checkpoints changes nothing
     assert np.array_equal(ck[:, :, -1, 0, :], hT.cpu().numpy())
     assert np.array_equal(ck[:, :, -1, 1, :], vT.cpu().numpy())
+    # (the forward that keeps checkpoints is the register-resident kernel; compare with that path)
     dev = {k: _t(inp[k]) for k in ("x", "delta", "A", "B", "C", "h0", "v0")}
-    y2, h2, v2 = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=dev["h0"],
-                             v0=dev["v0"], beta=0.9, alpha=1.0)
+    mm.mm_scan_set_path(1, 0)
+    try:
+        y2, h2, v2 = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=dev["h0"],
+                                 v0=dev["v0"], beta=0.9, alpha=1.0)
+    finally:
+        mm.mm_scan_set_path(0, 0)
     assert torch.equal(y2, y) and torch.equal(h2, hT) and torch.equal(v2, vT)
 
 

@@ -145,7 +145,16 @@ def test_long_workload_streaming_split_bit_identical():
     ysplit = torch.cat([y1, y2], dim=-1).cpu().numpy()
     scale = np.abs(one[0]).max()
     assert np.abs(ysplit - one[0]).max() <= F32_TOL * scale
-    _sampled_compare(inp, "f32", beta, alpha, got=one, k=12, what="long one-shot")
+    # 64 sampled channels (the first and the last included) against the oracle
+    _sampled_compare(inp, "f32", beta, alpha, got=one, k=64, what="long one-shot")
+    # and the state handed over at the split point
+    N = inp["A"].shape[1]
+    chan = _sample_channels(inp["x"].shape[0] * inp["x"].shape[1], 64)
+    inp1 = {k: (np.ascontiguousarray(v[..., :half]) if k in ("x", "delta", "B", "C") else v)
+            for k, v in inp.items()}
+    _, hr1, vr1 = oracle.scan_seq(**inp1, beta=beta, alpha=alpha, chan=chan)
+    _max_abs_ok(h1.cpu().numpy().reshape(-1, N)[chan], hr1, "long split-point hT")
+    _max_abs_ok(v1.cpu().numpy().reshape(-1, N)[chan], vr1, "long split-point vT")
 
 
 # -------------------------------------------------------- edge cases -----
@@ -191,9 +200,10 @@ def test_every_tile_variant_matches(io):
     w = wl.SCAN_BF16 if io == "bf16" else wl.SCAN_MEDIUM
     inp = wl.scan_inputs(w, batch=2, seqlen=200, dim=70)
     dev = _dev(inp, io)
-    base = _run(dev, 0.9, 1.0)
+    mm.mm_scan_set_path(1, 0)          # the tiles are those of the register-resident kernel
     yr, hr, vr = oracle.scan_seq(**inp, beta=0.9, alpha=1.0)
     try:
+        base = _run(dev, 0.9, 1.0)
         for spt, warps in ((2, 2), (2, 4), (2, 8), (4, 1), (4, 2), (4, 4)):
                 mm.mm_scan_set_tile(spt, warps, 1)
                 got = _run(dev, 0.9, 1.0)
@@ -203,6 +213,7 @@ def test_every_tile_variant_matches(io):
                 assert np.array_equal(got[1], base[1]) and np.array_equal(got[2], base[2])
     finally:
         mm.mm_scan_set_tile(0, 0, 1)
+        mm.mm_scan_set_path(0, 0)
 
 
 TIME_SPLIT_TILES = ((4, 2), (4, 4), (2, 4), (2, 8))
@@ -222,6 +233,7 @@ def test_time_split_variants_match_and_agree_on_state():
     yr, hr, vr = oracle.scan_seq(**inp, h0=h0.astype(np.float64), v0=v0.astype(np.float64),
                                  beta=0.9, alpha=1.0)
     first = None
+    mm.mm_scan_set_path(1, 0)
     try:
         for spt, warps in TIME_SPLIT_TILES:
             mm.mm_scan_set_tile(spt, warps, 2)
@@ -233,36 +245,55 @@ def test_time_split_variants_match_and_agree_on_state():
             assert np.array_equal(got[1], first[1]) and np.array_equal(got[2], first[2])
     finally:
         mm.mm_scan_set_tile(0, 0, 1)
+        mm.mm_scan_set_path(0, 0)
 
 
 @pytest.mark.parametrize("L", [1, 31, 32, 33, 64, 65, 130])
 @pytest.mark.parametrize("beta", [0.0, 0.9])
 def test_time_split_lengths(L, beta):
     inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=1, seqlen=L, dim=24)
+    mm.mm_scan_set_path(1, 0)
     try:
         mm.mm_scan_set_tile(4, 2, 2)
         _full_compare(inp, "f32", beta, 1.0, what=f"time split L={L} beta={beta}")
     finally:
         mm.mm_scan_set_tile(0, 0, 1)
+        mm.mm_scan_set_path(0, 0)
+
+
+def _split_streaming_bit_identical(halves):
+    inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=2, seqlen=448, dim=40)
+    dev = _dev(inp, "f32")
+    one = _run(dev, 0.99, 1.0)
+    for half in halves:
+        d1 = {k: (v[..., :half].contiguous() if k in ("x", "delta", "B", "C") else v) for k, v in dev.items()}
+        d2 = {k: (v[..., half:].contiguous() if k in ("x", "delta", "B", "C") else v) for k, v in dev.items()}
+        y1, h1, v1 = mm.scan_fwd(d1["x"], d1["delta"], d1["A"], d1["B"], d1["C"], beta=0.99, alpha=1.0)
+        y2, h2, v2 = mm.scan_fwd(d2["x"], d2["delta"], d2["A"], d2["B"], d2["C"], h0=h1, v0=v1,
+                                 beta=0.99, alpha=1.0)
+        torch.cuda.synchronize()
+        assert np.array_equal(h2.cpu().numpy(), one[1]), f"hT differs (split at {half})"
+        assert np.array_equal(v2.cpu().numpy(), one[2]), f"vT differs (split at {half})"
+
+
+def test_register_path_streaming_any_split_bit_identical():
+    # one time lane per state group applies the steps in order: any split point
+    mm.mm_scan_set_path(1, 0)
+    try:
+        _split_streaming_bit_identical((100, 1, 257, 444))
+    finally:
+        mm.mm_scan_set_path(0, 0)
 
 
 def test_time_split_streaming_bit_identical():
-    inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=2, seqlen=448, dim=40)
-    dev = _dev(inp, "f32")
+    # the time split carries its state across 32-step chunks: splits at multiples of 32
+    mm.mm_scan_set_path(1, 0)
     try:
         mm.mm_scan_set_tile(4, 2, 2)
-        one = _run(dev, 0.99, 1.0)
-        for half in (64, 192, 384):
-            d1 = {k: (v[..., :half].contiguous() if k in ("x", "delta", "B", "C") else v) for k, v in dev.items()}
-            d2 = {k: (v[..., half:].contiguous() if k in ("x", "delta", "B", "C") else v) for k, v in dev.items()}
-            y1, h1, v1 = mm.scan_fwd(d1["x"], d1["delta"], d1["A"], d1["B"], d1["C"], beta=0.99, alpha=1.0)
-            y2, h2, v2 = mm.scan_fwd(d2["x"], d2["delta"], d2["A"], d2["B"], d2["C"], h0=h1, v0=v1,
-                                     beta=0.99, alpha=1.0)
-            torch.cuda.synchronize()
-            assert np.array_equal(h2.cpu().numpy(), one[1]), f"hT differs (split at {half})"
-            assert np.array_equal(v2.cpu().numpy(), one[2]), f"vT differs (split at {half})"
+        _split_streaming_bit_identical((64, 192, 384, 32, 416))
     finally:
         mm.mm_scan_set_tile(0, 0, 1)
+        mm.mm_scan_set_path(0, 0)
 
 
 def test_in_place_streaming_state_and_optional_outputs():

@@ -1,0 +1,188 @@
+"""GPU parity of the sequence-split scan path against the fp64 oracle.
+
+The sequence-split kernel cuts the sequence into segments of a power-of-two
+length S that run side by side from a zero state and are joined by folding
+each segment's 2x2 affine carry map ("Momentum Mamba: Enhanced State Space
+Models with Momentum", "Forward Pass: Two-Stage Parallel Scan").  These tests
+force that path (mm_scan_set_path) with short segments so that small inputs
+cross many segments, several rounds of a cluster and ragged ends, and compare
+the whole output with the oracle at the scan's tolerances:
+  * fp32 I/O: max |y - y_ref| <= 1e-4 * max |y_ref| (also hT, vT);
+  * bf16 I/O: ||y - y_ref||_2 / ||y_ref||_2 <= 1e-2;
+  * streaming: hT, vT bit-identical between one call and two calls split at
+    a multiple of S.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import selective_state_space_momentum_b200 as mm
+from selective_state_space_momentum_b200 import workloads as wl
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-4
+BF16_TOL = 1e-2
+
+
+@pytest.fixture
+def seg_path():
+    """Force the sequence-split path with a given segment length; restore after."""
+    def force(seg_len):
+        mm.mm_scan_set_path(2, seg_len)
+    yield force
+    mm.mm_scan_set_path(0, 0)
+
+
+def _inputs(batch, L, D, N, seed, io="f32", law=wl.SCAN_MEDIUM):
+    inp = wl.scan_inputs(law, batch=batch, seqlen=L, dim=D, dstate=N, seed=seed)
+    if io == "bf16":
+        for k in ("x", "delta", "B", "C"):
+            inp[k] = wl.bf16_round(inp[k])
+    return inp
+
+
+def _dev(inp, io):
+    dt = torch.float32 if io == "f32" else torch.bfloat16
+    out = {k: torch.from_numpy(inp[k]).cuda().to(dt).contiguous() for k in ("x", "delta", "B", "C")}
+    out["A"] = torch.from_numpy(inp["A"]).cuda().contiguous()
+    return out
+
+
+def _states(rng, batch, D, N, scale):
+    h0 = (rng.standard_normal((batch, D, N)) * scale).astype(np.float32)
+    v0 = (rng.standard_normal((batch, D, N)) * scale * 0.3).astype(np.float32)
+    return h0, v0
+
+
+def _run(dev, beta, alpha, h0=None, v0=None):
+    th0 = None if h0 is None else torch.from_numpy(h0).cuda()
+    tv0 = None if v0 is None else torch.from_numpy(v0).cuda()
+    y, hT, vT = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=th0, v0=tv0,
+                            beta=beta, alpha=alpha)
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    return y.float().cpu().numpy(), hT.cpu().numpy(), vT.cpu().numpy()
+
+
+def _check(io, got, inp, beta, alpha, h0=None, v0=None, what=""):
+    y, hT, vT = got
+    L = inp["x"].shape[2]
+    N = inp["A"].shape[1]
+    h0r = None if h0 is None else h0.astype(np.float64)
+    v0r = None if v0 is None else v0.astype(np.float64)
+    yr, hr, vr = oracle.scan_seq(**inp, h0=h0r, v0=v0r, beta=beta, alpha=alpha)
+    y = y.reshape(-1, L)
+    if io == "f32":
+        err = np.abs(y - yr).max()
+        assert err <= F32_TOL * np.abs(yr).max(), f"{what}: y max abs err {err:.3e} vs {np.abs(yr).max():.3e}"
+    else:
+        r = np.linalg.norm(y - yr) / np.linalg.norm(yr)
+        assert r <= BF16_TOL, f"{what}: y relative L2 {r:.3e}"
+    for got_s, ref_s, name in ((hT.reshape(-1, N), hr, "hT"), (vT.reshape(-1, N), vr, "vT")):
+        err = np.abs(got_s - ref_s).max()
+        scale = np.abs(ref_s).max()
+        assert err <= F32_TOL * scale, f"{what}: {name} max abs err {err:.3e} vs {scale:.3e}"
+
+
+@pytest.mark.parametrize("L,seg", [(256, 32), (1000, 64), (4096, 128), (4133 // 4 * 4, 256), (96, 128)])
+@pytest.mark.parametrize("beta,alpha", [(0.9, 1.0), (0.0, 1.0), (0.99, 0.5)])
+def test_segments_rounds_and_ragged_ends(seg_path, L, seg, beta, alpha):
+    # up to 32 segments: several rounds of an 8-CTA cluster, a ragged last chunk
+    seg_path(seg)
+    inp = _inputs(2, L, 40, 16, seed=7 + L)
+    _check("f32", _run(_dev(inp, "f32"), beta, alpha), inp, beta, alpha, what=f"L={L} S={seg}")
+
+
+@pytest.mark.parametrize("N", [9, 12, 16])
+def test_state_counts_and_initial_state(seg_path, N):
+    seg_path(64)
+    rng = np.random.default_rng(N)
+    inp = _inputs(1, 640, 33, N, seed=100 + N)
+    h0, v0 = _states(rng, 1, 33, N, 2.0)
+    _check("f32", _run(_dev(inp, "f32"), 0.9, 1.0, h0, v0), inp, 0.9, 1.0, h0, v0, what=f"N={N} with h0, v0")
+
+
+def test_bf16_io(seg_path):
+    seg_path(128)
+    inp = _inputs(2, 1024, 48, 16, seed=5, io="bf16", law=wl.SCAN_BF16)
+    rng = np.random.default_rng(3)
+    h0, v0 = _states(rng, 2, 48, 16, 1.0)
+    _check("bf16", _run(_dev(inp, "bf16"), 0.9, 1.0, h0, v0), inp, 0.9, 1.0, h0, v0, what="bf16")
+
+
+def test_slow_decay_runs_the_whole_correction(seg_path):
+    # beta = 0.999 and tiny steps: the carry's response outlives every segment
+    seg_path(64)
+    inp = _inputs(1, 512, 16, 16, seed=11)
+    inp["delta"] = (inp["delta"] * 1e-2).astype(np.float32)
+    rng = np.random.default_rng(1)
+    h0, v0 = _states(rng, 1, 16, 16, 1.0)
+    _check("f32", _run(_dev(inp, "f32"), 0.999, 1.0, h0, v0), inp, 0.999, 1.0, h0, v0, what="slow decay")
+
+
+def test_growing_modes_are_not_cut_short(seg_path):
+    # A > 0 on some lanes: the response grows, so the correction must run to each segment's end
+    seg_path(64)
+    inp = _inputs(1, 384, 16, 16, seed=12)
+    inp["A"][:, 0] = 0.5
+    inp["delta"] = (inp["delta"] * 0.1).astype(np.float32)
+    _check("f32", _run(_dev(inp, "f32"), 0.5, 1.0), inp, 0.5, 1.0, what="A > 0")
+
+
+@pytest.mark.parametrize("seg", [64, 256])
+def test_streaming_split_at_segment_multiples_is_bit_identical(seg_path, seg):
+    seg_path(seg)
+    L, L1 = 2048, 4 * seg
+    inp = _inputs(2, L, 48, 16, seed=21)
+    dev = _dev(inp, "f32")
+    rng = np.random.default_rng(2)
+    h0, v0 = _states(rng, 2, 48, 16, 1.0)
+    th0, tv0 = torch.from_numpy(h0).cuda(), torch.from_numpy(v0).cuda()
+    y, hT, vT = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=th0, v0=tv0, beta=0.99)
+    parts = []
+    h, v = th0, tv0
+    for lo, hi in ((0, L1), (L1, L)):
+        sl = {k: dev[k][..., lo:hi].contiguous() for k in ("x", "delta", "B", "C")}
+        yp, h, v = mm.scan_fwd(sl["x"], sl["delta"], dev["A"], sl["B"], sl["C"], h0=h, v0=v, beta=0.99)
+        parts.append(yp)
+    torch.cuda.synchronize()
+    assert torch.equal(h, hT) and torch.equal(v, vT), "final states differ between one call and two"
+    y2 = torch.cat(parts, dim=-1)
+    assert torch.equal(y2, y), "y differs between one call and two calls split at a segment multiple"
+
+
+def test_segmented_and_register_paths_agree(seg_path):
+    inp = _inputs(1, 2048, 64, 16, seed=31)
+    dev = _dev(inp, "f32")
+    mm.mm_scan_set_path(1, 0)
+    y1, h1, v1 = _run(dev, 0.9, 1.0)
+    seg_path(256)
+    y2, h2, v2 = _run(dev, 0.9, 1.0)
+    scale = np.abs(y1).max()
+    assert np.abs(y1 - y2).max() <= 2 * F32_TOL * scale
+    assert np.abs(h1 - h2).max() <= 2 * F32_TOL * np.abs(h1).max()
+
+
+def test_in_place_streaming_state(seg_path):
+    # hT may be h0 and vT may be v0
+    seg_path(64)
+    inp = _inputs(1, 512, 32, 16, seed=41)
+    dev = _dev(inp, "f32")
+    rng = np.random.default_rng(4)
+    h0, v0 = _states(rng, 1, 32, 16, 1.0)
+    h = torch.from_numpy(h0).cuda()
+    v = torch.from_numpy(v0).cuda()
+    y = torch.empty_like(dev["x"])
+    mm.mm_scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h, v, 0.9, 1.0, y, h, v)
+    torch.cuda.synchronize()
+    _check("f32", (y.cpu().numpy(), h.cpu().numpy(), v.cpu().numpy()), inp, 0.9, 1.0, h0, v0, what="in place")
+
+
+def test_segment_length_query():
+    # the automatic choice: the long workload's 2048 channels get 16384-step segments
+    assert mm.mm_scan_segment_len(1, 131072, 2048, 16) == 16384
+    assert mm.mm_scan_segment_len(1, 131072, 1024, 16) == 32768
+    assert mm.mm_scan_segment_len(4, 2048, 1536, 16) == 0          # register-resident path
+    assert mm.mm_scan_segment_len(1, 131072, 2048, 8) == 0          # dstate <= 8

@@ -100,8 +100,7 @@ def test_in_place_state_and_determinism():
     h0 = rng.standard_normal((1, 2, 64, 128)).astype(np.float32)
     st = torch.from_numpy(h0).cuda()
     y = torch.empty_like(dev["x"])
-    mm.mm_ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], st, 0.0, 1.0, y, st,
-                  torch.empty(0, dtype=torch.uint8, device="cuda"), 256)
+    mm.mm_ssd_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], st, 0.0, 1.0, y, st, 256)
     torch.cuda.synchronize()
     _compare(inp, y.float().cpu().numpy(), st.cpu().numpy(), h0=h0, what="in place")
     a = _run(dev)

@@ -87,10 +87,9 @@ def test_ssd_fwd_with_beta_routes_to_momentum():
     h0t = torch.from_numpy(h0).cuda()
     y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], h0=h0t, alpha=1.0, chunk=256)
     ym, hm, _ = mm.ssd_fwd_momentum(d["x"], d["delta"], d["A"], d["B"], d["C"], h0=h0t, beta=0.0)
-    ws = torch.empty(0, device="cuda", dtype=torch.uint8)
     y2 = torch.empty_like(d["x"])
     h2 = torch.empty_like(hT)
-    mm.mm_ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], h0t, 0.7, 1.0, y2, h2, ws, 256)
+    mm.mm_ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], h0t, 0.7, 1.0, y2, h2, 256)
     torch.cuda.synchronize()
     ref = oracle.ssd_chunked_momentum(**inp, h0=h0.astype(np.float64), beta=0.7, alpha=1.0, chunk=64)
     rel = np.linalg.norm(y2.float().cpu().numpy() - ref[0].reshape(y2.shape)) / np.linalg.norm(ref[0])
