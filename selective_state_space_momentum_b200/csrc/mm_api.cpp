@@ -99,6 +99,17 @@ bool inject_launch_failure() {
     return v && std::strcmp(v, "launch") == 0;
 }
 
+// Test hook for the device-side give-up path: with MMSCAN_FAULT_INJECT=stall
+// the kernels that stage their inputs through bounded waits (the two forward
+// scans, the backward, the SSD kernel) are launched with their producer told
+// to issue nothing.  Nothing is then in flight; every wait runs out after its
+// limit, the kernel returns, and mm_device_status reports
+// MM_ERR_DEVICE_TIMEOUT.  The outputs of such a call are not written.
+int inject_stall() {
+    const char* v = std::getenv("MMSCAN_FAULT_INJECT");
+    return (v && std::strcmp(v, "stall") == 0) ? 1 : 0;
+}
+
 mm_status from_cuda(cudaError_t e, const char* what) {
     if (e == cudaSuccess) return ok();
     return fail(MM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
@@ -287,6 +298,7 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.Dskip = Dskip; a.z = z; a.dbias = delta_bias; a.softplus = delta_softplus ? 1 : 0;
     a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
     a.ckpt = ckpt;
+    a.stall = inject_stall();
     if (!a.ext && !ckpt) {
         const int64_t seg = seg_len_for(bsz, D, N, dims->io, a.vec_ok != 0);
         if (seg > 0)
@@ -373,6 +385,7 @@ mm_status mm_scan_bwd_gated(const void* x, const void* delta, const float* A, co
     a.dD = a.ext ? dD : nullptr;
     a.dz = z ? dz : nullptr;
     a.ddbias = a.ext ? ddelta_bias : nullptr;
+    a.stall = inject_stall();
     return from_cuda(mmscan::launch_scan_bwd(a, dims->io, static_cast<cudaStream_t>(stream)),
                      "mm_scan_bwd launch");
 }
@@ -470,6 +483,7 @@ mm_status mm_ssd_fwd(const void* x, const float* delta, const float* A, const vo
     a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.h0 = h0; a.y = y; a.hT = hT;
     a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
     a.chunk = dims->chunk; a.alpha = alpha;
+    a.stall = inject_stall();
     return from_cuda(mmscan::launch_ssd_fwd(a, static_cast<cudaStream_t>(stream)), "mm_ssd_fwd launch");
 }
 

@@ -32,6 +32,7 @@ struct ScanArgs {
     int softplus;          // delta' = softplus(delta + dbias)
     int ext;               // any of the four is present
     float* ckpt;           // (batch, dim, ceil(L / 16), 2, dstate): (h, v) after every 16 steps, or null
+    int stall;             // test only: stage no input, so that the bounded waits run out
 };
 
 // Arguments of one backward launch (device pointers; sizes as in mm_scan_dims).
@@ -68,6 +69,7 @@ struct ScanBwdArgs {
     float* dD;             // (dim), summed over batch and steps, or null
     void* dz;              // (batch, dim, L) io, or null
     float* ddbias;         // (dim), or null
+    int stall;             // test only: stage no input, so that the bounded waits run out
 };
 
 // Arguments of one decode step (device pointers; states updated in place).
@@ -130,6 +132,7 @@ struct SSDArgs {
     float* hT;
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
     float alpha;
+    int stall;             // test only: stage no input, so that the bounded waits run out
 };
 
 // Arguments of one momentum SSD call (the CUDA-core chunked kernel).

@@ -178,6 +178,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     // ---- staging of one chunk into a stage buffer ----------------------------
     auto issue = [&](int64_t k, int s) {
+        if (p.stall) return;      // test only: nothing staged, the waits run out
         const int64_t t0 = k * T;
         const uint32_t sb = base + s * TL::STAGE_BYTES;
         const uint32_t bar = bar0 + 8 * s;

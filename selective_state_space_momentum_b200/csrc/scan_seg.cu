@@ -85,8 +85,7 @@ struct SegTile {
     static constexpr int MAIN_TX = STAGE_BYTES;  // main pass: x, delta, B, C
     static constexpr int CORR_TX = XBOX + BBOX;  // correction: delta, C
     static constexpr int BT_BYTES = T * NP * 4;  // one transposed [t][n] fp32 matrix
-    static constexpr int OFF_BT = ST * STAGE_BYTES;
-    static constexpr int OFF_CT = OFF_BT + BT_BYTES;
+    static constexpr int OFF_BT = ST * STAGE_BYTES;  // B^T and C^T interleaved, [t][32] fp32
     // The segment maps (8 float4 per thread) are published in the B^T/C^T area.
     static constexpr int AGG_BYTES = NT * 8 * 16;
     // The concrete carry (v, h) of each lane's 8 states between folds.
@@ -145,8 +144,7 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     unsigned char* smem = smem_raw + (base - raw_addr);
-    float* Bt = reinterpret_cast<float*>(smem + TL::OFF_BT);
-    float* Ct = reinterpret_cast<float*>(smem + TL::OFF_CT);
+    float* BCt = reinterpret_cast<float*>(smem + TL::OFF_BT);     // [t][32]: B^T | C^T, swizzled
     float4* agg = reinterpret_cast<float4*>(smem + TL::OFF_BT);
     const uint32_t agg_addr = base + TL::OFF_BT;
     const uint32_t bar0 = base + TL::OFF_BAR;
@@ -220,7 +218,7 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     bool dead = false;            // a bounded wait gave up: skip the work, keep the barriers
     auto issue = [&](int64_t t0, bool main_pass) {
         const int s = (int)(issued % ST);
-        if (tid == 0) {
+        if (tid == 0 && !p.stall) {   // (stall: test only, nothing staged, the waits run out)
             const uint32_t sb = base + s * TL::STAGE_BYTES;
             const uint32_t bar = bar0 + 8 * s;
             mbar_expect_tx(bar, main_pass ? TL::MAIN_TX : TL::CORR_TX);
@@ -249,14 +247,21 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         while (!dead && consumed < issued) (void)wait_next();
     };
 
-    // B, C of a staged chunk to [t][n] fp32 (alpha into B); `withB` false: C only.
+    // B, C of a staged chunk into one [t][32] fp32 area (alpha folded into B):
+    // row t holds B_t[0..15] in 16-byte chunks 0-3 and C_t[0..15] in chunks 4-7,
+    // chunk c stored at position c ^ ((t >> 2) & 7).  An item moves a 4 x 4
+    // block (4 states, 4 steps); the 8 lanes of a quarter warp take 8
+    // consecutive 4-step blocks of one (matrix, state block), so that both the
+    // swizzled tile reads and the [t] row writes hit 8 distinct bank groups.
+    // `withB` false: C only (the correction pass).
     auto transpose = [&](const unsigned char* sbuf, bool withB) {
-        const int items = withB ? 2 * 4 * (T / 4) : 4 * (T / 4);
+        const int items = (withB ? 8 : 4) * (T / 4);
         for (int i = tid; i < items; i += NT) {
-            const int which = withB ? (i / (4 * (T / 4))) : 1;     // 0 = B, 1 = C
-            const int rem = i % (4 * (T / 4));
-            const int n0 = (rem & 3) * 4;
-            const int t4 = (rem >> 2) * 4;
+            const int combo = withB ? ((i >> 3) & 7) : 4 + ((i >> 3) & 3);   // matrix * 4 + state block
+            const int tb = (i & 7) | ((withB ? (i >> 6) : (i >> 5)) << 3);    // 4-step block
+            const int which = combo >> 2;                                      // 0 = B, 1 = C
+            const int n0 = (combo & 3) * 4;
+            const int t4 = tb * 4;
             const unsigned char* tile = sbuf + (which ? TL::OFF_C : TL::OFF_B);
             float m[4][4];
 #pragma unroll
@@ -265,10 +270,10 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 m[r][0] = q.x; m[r][1] = q.y; m[r][2] = q.z; m[r][3] = q.w;
             }
             const float sc = which ? 1.0f : p.alpha;
-            float* dst = (which ? Ct : Bt) + t4 * TL::NP + n0;
+            float* dst = BCt + t4 * 32 + ((combo ^ (tb & 7)) * 4);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<float4*>(dst + j * TL::NP) =
+                *reinterpret_cast<float4*>(dst + j * 32) =
                     make_float4(m[0][j] * sc, m[1][j] * sc, m[2][j] * sc, m[3][j] * sc);
         }
     };
@@ -291,8 +296,8 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const float2 beta2 = f2(beta, beta);
     const float kappa = beta / (1.0f - beta);
 
-    // Four steps of the two channels: delta (and, on the main pass, the input
-    // delta * x) and the exponentials 2^(delta A log2 e) of the four states.
+    // Four steps of the two channels: the input delta * x (main pass) and the
+    // exponentials 2^(delta A log2 e) of the four states.
     struct Quad {
         float u[2][4];
         float a[2][4][4];          // [channel][state][step]
@@ -302,8 +307,10 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     float2 bp2;                   // beta^(t+1)
     float2 dacc[2];               // sum of delta over the current chunk, (even, odd) steps
     uint32_t dbits;               // OR of delta's bit patterns over the segment
-    auto prep = [&](const unsigned char* sbuf, int tau, Quad& Q, bool main_pass) {
-        float dl[2][4];
+
+    // Loads of a group: delta into dl; on the main pass x, u = delta * x, and
+    // the segment's delta sums.
+    auto prep_load = [&](const unsigned char* sbuf, int tau, float (&dl)[2][4], Quad& Q, bool main_pass) {
         load_dx(sbuf, TL::OFF_D, tau, dl);
         if (main_pass) {
             float xl[2][4];
@@ -322,27 +329,32 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 dacc[c] = __fadd2_rn(dacc[c], __fadd2_rn(f2(dl[c][0], dl[c][1]), f2(dl[c][2], dl[c][3])));
             }
         }
+    };
+    // Eight of a group's exponentials: channel c, steps 2 jp and 2 jp + 1.
+    auto prep_exp = [&](const float (&dl)[2][4], Quad& Q, int c, int jp) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int j2 = 0; j2 < 4; j2 += 2)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 ex = __fmul2_rn(f2(dl[c][j2], dl[c][j2 + 1]), f2(Al[c][e], Al[c][e]));
-                    Q.a[c][e][j2] = ex2_approx(ex.x);
-                    Q.a[c][e][j2 + 1] = ex2_approx(ex.y);
-                }
+        for (int e = 0; e < 4; ++e) {
+            const float2 ex = __fmul2_rn(f2(dl[c][2 * jp], dl[c][2 * jp + 1]), f2(Al[c][e], Al[c][e]));
+            Q.a[c][e][2 * jp] = ex2_approx(ex.x);
+            Q.a[c][e][2 * jp + 1] = ex2_approx(ex.y);
+        }
     };
 
     // The four steps of Q from chunk step tau; partial read-outs into yk[c][j0 + j].
+    // With `nxt`, step j also forms eight exponentials of the next group, so that
+    // the MUFU work is spread between the FMAs instead of issued in bursts.
     // `ragged`: steps at or past nval leave the state alone (the last chunk).
-    auto main_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval) {
+    auto main_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval,
+                          const float (&dln)[2][4], Quad& Qn, bool nxt) {
+        const int sw = (tau >> 2) & 7;                 // row swizzle of the 4 steps
+        const int bo = (g ^ sw) * 4, co = ((4 + g) ^ sw) * 4;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+            if (nxt) prep_exp(dln, Qn, j & 1, j >> 1);
             const int step = tau + j;
             const bool valid = !ragged || step < nval;
-            const float4 b4 = *reinterpret_cast<const float4*>(Bt + step * TL::NP + 4 * g);
-            const float4 c4 = *reinterpret_cast<const float4*>(Ct + step * TL::NP + 4 * g);
+            const float4 b4 = *reinterpret_cast<const float4*>(BCt + step * 32 + bo);
+            const float4 c4 = *reinterpret_cast<const float4*>(BCt + step * 32 + co);
             const float2 bq[2] = {f2(b4.x, b4.y), f2(b4.z, b4.w)};
             const float2 cq[2] = {f2(c4.x, c4.y), f2(c4.z, c4.w)};
 #pragma unroll
@@ -365,35 +377,49 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
     };
 
-    // Add the four lanes' partials of an 8-step group and store (or add to) y.
-    auto flush = [&](const float (&yk)[2][8], int64_t t0, int first8, int nval, bool add) {
+    // Add the four lanes' partials of an 8-step group and store y (main pass),
+    // or add them to the y stored by the main pass, read ahead into yold.
+    auto flush = [&](const float (&yk)[2][8], int64_t t0, int first8, int nval, bool add, const float (&yold)[4]) {
         float out[4];
         butterfly_sum<G, 16>(*reinterpret_cast<const float(*)[16]>(&yk[0][0]), out, g);
         const int first = first8 + ostep;
         const int cnt = nval - first < 4 ? nval - first : 4;
         if (!oact || cnt <= 0) return;
-        IO* yp = orow + t0 + first;
         if (add) {
-            if (cnt == 4) {
-                const float4 q4 = load4(static_cast<const IO*>(yp));
-                out[0] += q4.x; out[1] += q4.y; out[2] += q4.z; out[3] += q4.w;
-            } else {
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (e < cnt) out[e] += load1(static_cast<const IO*>(yp + e));
-            }
+            for (int e = 0; e < 4; ++e) out[e] += yold[e];
         }
-        store_steps_n<IO, 4>(yp, out, cnt, true);
+        store_steps_n<IO, 4>(orow + t0 + first, out, cnt, true);
+    };
+    // The main pass's y of the lane's four outputs of the 8-step group at first8.
+    auto load_yold = [&](int64_t t0, int first8, int nval, float (&yold)[4]) {
+        const int first = first8 + ostep;
+        const int cnt = nval - first < 4 ? nval - first : 4;
+        yold[0] = yold[1] = yold[2] = yold[3] = 0.0f;
+        if (!oact || cnt <= 0) return;
+        const IO* yp = orow + t0 + first;
+        if (cnt == 4) {
+            const float4 q4 = load4(yp);
+            yold[0] = q4.x; yold[1] = q4.y; yold[2] = q4.z; yold[3] = q4.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (e < cnt) yold[e] = load1(yp + e);
+        }
     };
 
     // Correction state: the response to the carry-in.
     float2 rvv[2][2], rhh[2][2];
-    auto corr_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval) {
+    auto corr_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval,
+                          const float (&dln)[2][4], Quad& Qn, bool nxt) {
+        const int sw = (tau >> 2) & 7;
+        const int co = ((4 + g) ^ sw) * 4;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+            if (nxt) prep_exp(dln, Qn, j & 1, j >> 1);
             const int step = tau + j;
             const bool valid = !ragged || step < nval;
-            const float4 c4 = *reinterpret_cast<const float4*>(Ct + step * TL::NP + 4 * g);
+            const float4 c4 = *reinterpret_cast<const float4*>(BCt + step * 32 + co);
             const float2 cq[2] = {f2(c4.x, c4.y), f2(c4.z, c4.w)};
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -410,37 +436,63 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
         }
     };
+    auto steps = [&](bool main_pass, const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval,
+                     const float (&dln)[2][4], Quad& Qn, bool nxt) {
+        if (main_pass) main_steps(Q, tau, j0, yk, ragged, nval, dln, Qn, nxt);
+        else corr_steps(Q, tau, j0, yk, ragged, nval, dln, Qn, nxt);
+    };
 
-    // One staged chunk: full chunks run unpredicated with each group's loads and
-    // exponentials issued one group ahead; the last chunk of the sequence is ragged.
+    // One staged chunk.  Full chunks run unpredicated, each group's loads and
+    // exponentials formed during the group before; the last chunk of the
+    // sequence is ragged.  The correction reads the main pass's y one group ahead.
     auto run_chunk = [&](const unsigned char* sbuf, int64_t t0, int nval, bool main_pass) {
         float yk[2][8] = {};
+        float dl[2][4];
+        float yold[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ynext[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (nval == T) {
             Quad Q0, Q1;
-            prep(sbuf, 0, Q0, main_pass);
+            prep_load(sbuf, 0, dl, Q0, main_pass);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int jp = 0; jp < 2; ++jp) prep_exp(dl, Q0, c, jp);
+            if (!main_pass) load_yold(t0, 0, T, yold);
 #pragma unroll 1
             for (int g8 = 0; g8 < T; g8 += 8) {
-                prep(sbuf, g8 + 4, Q1, main_pass);
-                if (main_pass) main_steps(Q0, g8, 0, yk, false, T);
-                else corr_steps(Q0, g8, 0, yk, false, T);
-                if (g8 + 8 < T) prep(sbuf, g8 + 8, Q0, main_pass);
-                if (main_pass) main_steps(Q1, g8 + 4, 4, yk, false, T);
-                else corr_steps(Q1, g8 + 4, 4, yk, false, T);
-                flush(yk, t0, g8, T, !main_pass);
+                const bool more = g8 + 8 < T;
+                if (!main_pass && more) load_yold(t0, g8 + 8, T, ynext);
+                prep_load(sbuf, g8 + 4, dl, Q1, main_pass);
+                steps(main_pass, Q0, g8, 0, yk, false, T, dl, Q1, true);
+                if (more) {
+                    prep_load(sbuf, g8 + 8, dl, Q0, main_pass);
+                    steps(main_pass, Q1, g8 + 4, 4, yk, false, T, dl, Q0, true);
+                } else {
+                    steps(main_pass, Q1, g8 + 4, 4, yk, false, T, dl, Q0, false);
+                }
+                flush(yk, t0, g8, T, !main_pass, yold);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) yold[e] = ynext[e];
             }
         } else {
 #pragma unroll 1
             for (int g8 = 0; g8 < nval; g8 += 8) {
                 Quad Q;
-                prep(sbuf, g8, Q, main_pass);
-                if (main_pass) main_steps(Q, g8, 0, yk, true, nval);
-                else corr_steps(Q, g8, 0, yk, true, nval);
+                if (!main_pass) load_yold(t0, g8, nval, yold);
+                prep_load(sbuf, g8, dl, Q, main_pass);
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int jp = 0; jp < 2; ++jp) prep_exp(dl, Q, c, jp);
+                steps(main_pass, Q, g8, 0, yk, true, nval, dl, Q, false);
                 if (g8 + 4 < nval) {
-                    prep(sbuf, g8 + 4, Q, main_pass);
-                    if (main_pass) main_steps(Q, g8 + 4, 4, yk, true, nval);
-                    else corr_steps(Q, g8 + 4, 4, yk, true, nval);
+                    prep_load(sbuf, g8 + 4, dl, Q, main_pass);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+#pragma unroll
+                        for (int jp = 0; jp < 2; ++jp) prep_exp(dl, Q, c, jp);
+                    steps(main_pass, Q, g8 + 4, 4, yk, true, nval, dl, Q, false);
                 }
-                flush(yk, t0, g8, nval, !main_pass);
+                flush(yk, t0, g8, nval, !main_pass, yold);
             }
         }
     };
@@ -644,13 +696,18 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream)
     cfg.blockDim = dim3(TL::NT, 1, 1);
     cfg.dynamicSmemBytes = TL::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Load-balancing placement spreads the clusters' one-warp CTAs over all 148
+    // SMs (6-8 each for the long workload); the default placement filled 142
+    // SMs to 7-8 and left 6 without any.
+    attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize);
 }
 

@@ -116,6 +116,7 @@ struct SSDKArgs {
     int64_t batch, seqlen, nheads, ngroups;
     int nblocks;
     float alpha;
+    int stall;
 };
 
 __global__ void __launch_bounds__(ssd::NTHREADS, 1)
@@ -177,7 +178,8 @@ ssd_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
     if (warp == W_PROD) {
         // ------------------------------------------------------ producer ----
-        if (lane == 0) {
+        // (stall: test only, nothing staged, every other role's wait runs out)
+        if (lane == 0 && !p.stall) {
             for (int u = 0; u < nblk; ++u) {
                 cur_blk = u;
                 const int s = u & 1;
@@ -643,6 +645,7 @@ cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t stream) {
     k.batch = a.batch; k.seqlen = a.seqlen; k.nheads = a.nheads; k.ngroups = a.ngroups;
     k.nblocks = (int)((a.seqlen + ssd::UB - 1) / ssd::UB);
     k.alpha = a.alpha;
+    k.stall = a.stall;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
