@@ -91,7 +91,10 @@ struct SegTile {
     // The concrete carry (v, h) of each lane's 8 states between folds.
     static constexpr int OFF_CARRY = OFF_BT + 2 * BT_BYTES;
     static constexpr int CARRY_BYTES = NT * 16 * 4;
-    static constexpr int OFF_BAR = OFF_CARRY + CARRY_BYTES;
+    // Scaled form: alpha beta^-(tau+1) and beta^(tau+1) for the steps tau of a chunk.
+    static constexpr int OFF_TAB = OFF_CARRY + CARRY_BYTES;
+    static constexpr int TAB_BYTES = 2 * T * 4;
+    static constexpr int OFF_BAR = OFF_TAB + TAB_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + ST * 8 + 1024;    // + alignment slack
     static_assert(AGG_BYTES <= 2 * BT_BYTES, "segment maps fit the transposed area");
     static_assert(STAGE_BYTES % 1024 == 0, "tiles stay 1024-byte aligned");
@@ -132,7 +135,17 @@ __device__ __forceinline__ float pow_steps(float beta, int64_t n) {
     return r;
 }
 
-template <typename IO, int W, int ST>
+// Scaled form (SC, used for beta >= 1/2).  Within a chunk of T steps the
+// states are carried as v~ = v / beta^(tau+1), h~ = h / beta^(tau+1) (tau the
+// step within the chunk), which turns the two recurrences into
+//     v~_tau = v~_{tau-1} + u_tau B~_tau,       B~_tau = alpha beta^-(tau+1) B_tau
+//     h~_tau = a~_tau h~_{tau-1} + v~_tau,      a~_tau = 2^(delta A log2 e - log2 beta)
+//     y_tau  = sum_n C~_tau h~_tau,             C~_tau = beta^(tau+1) C_tau
+// with B~ and C~ formed once per chunk by the transpose: one FMA per state
+// for the velocity instead of a multiply and an FMA.  At the end of the chunk
+// the states are multiplied back by beta^T.  The factors stay within 2^+-32
+// (2^+-64 for bf16 chunks of 64 steps) for beta >= 1/2.
+template <typename IO, int W, int ST, bool SC>
 __global__ void __launch_bounds__(W * 32)
 scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -146,6 +159,8 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     unsigned char* smem = smem_raw + (base - raw_addr);
     float* BCt = reinterpret_cast<float*>(smem + TL::OFF_BT);     // [t][32]: B^T | C^T, swizzled
     float4* agg = reinterpret_cast<float4*>(smem + TL::OFF_BT);
+    float* tab_ib = reinterpret_cast<float*>(smem + TL::OFF_TAB);  // alpha beta^-(tau+1)
+    float* tab_cb = tab_ib + T;                                      // beta^(tau+1)
     const uint32_t agg_addr = base + TL::OFF_BT;
     const uint32_t bar0 = base + TL::OFF_BAR;
 
@@ -169,15 +184,30 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, 1u);
         fence_barrier_init();
     }
+    if constexpr (SC) {
+        for (int t = tid; t < T; t += NT) {
+            const float cb = pow_steps(beta, t + 1);
+            tab_cb[t] = cb;
+            tab_ib[t] = __fdiv_rn(p.alpha, cb);
+        }
+    }
     __syncthreads();
 
     // ---- per-lane constants ---------------------------------------------------
+    // The lane's two channels, in an order of its own: lanes 4p+2, 4p+3 take
+    // the pair's channels the other way round, so that the first step of the
+    // read-out butterfly (lanes g and g^2) exchanges the same register set on
+    // every lane and needs no selects.
     bool act[2];
     int64_t dch[2];
+    int lch[2];                   // channel within the CTA
+    uint32_t dxo[2];              // its row in a swizzled x / delta tile: row * 128 + (row & 7) * 16
     float Al[2][4];               // A[d, 4g + e] log2 e
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-        dch[c] = d0 + cc0 + c;
+        lch[c] = cc0 + (c ^ (g >> 1));
+        dxo[c] = (uint32_t)lch[c] * 128u + (((uint32_t)lch[c] & 7u) << 4);
+        dch[c] = d0 + lch[c];
         act[c] = dch[c] < p.dim;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -191,6 +221,8 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
         for (int e = 0; e < 4; ++e) a_nonpos = a_nonpos && (Al[c][e] <= 0.0f);
     a_nonpos = __syncthreads_and(a_nonpos) != 0;
+    // -log2(beta), added to every exponent of the scaled form
+    const float nl2b = SC ? -log2f(beta) : 0.0f;
 
     // The concrete carry entering the current round, per lane (c, e): starts at
     // (h0, v0); kept in shared memory between folds ([c][e][v/h][thread]).
@@ -247,9 +279,10 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         while (!dead && consumed < issued) (void)wait_next();
     };
 
-    // B, C of a staged chunk into one [t][32] fp32 area (alpha folded into B):
-    // row t holds B_t[0..15] in 16-byte chunks 0-3 and C_t[0..15] in chunks 4-7,
-    // chunk c stored at position c ^ ((t >> 2) & 7).  An item moves a 4 x 4
+    // B, C of a staged chunk into one [t][32] fp32 area: row t holds B_t[0..15]
+    // in 16-byte chunks 0-3 and C_t[0..15] in chunks 4-7, chunk c stored at
+    // position c ^ ((t >> 2) & 7); B carries alpha (and beta^-(tau+1) in the
+    // scaled form), C beta^(tau+1) in the scaled form.  An item moves a 4 x 4
     // block (4 states, 4 steps); the 8 lanes of a quarter warp take 8
     // consecutive 4-step blocks of one (matrix, state block), so that both the
     // swizzled tile reads and the [t] row writes hit 8 distinct bank groups.
@@ -269,27 +302,53 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const float4 q = load4(reinterpret_cast<const IO*>(tile + sw128(n0 + r, t4 * EB)));
                 m[r][0] = q.x; m[r][1] = q.y; m[r][2] = q.z; m[r][3] = q.w;
             }
-            const float sc = which ? 1.0f : p.alpha;
+            float sc[4];
+            if constexpr (SC) {
+                const float4 f = *reinterpret_cast<const float4*>((which ? tab_cb : tab_ib) + t4);
+                sc[0] = f.x; sc[1] = f.y; sc[2] = f.z; sc[3] = f.w;
+            } else {
+                sc[0] = sc[1] = sc[2] = sc[3] = which ? 1.0f : p.alpha;
+            }
             float* dst = BCt + t4 * 32 + ((combo ^ (tb & 7)) * 4);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 *reinterpret_cast<float4*>(dst + j * 32) =
-                    make_float4(m[0][j] * sc, m[1][j] * sc, m[2][j] * sc, m[3][j] * sc);
+                    make_float4(m[0][j] * sc[j], m[1][j] * sc[j], m[2][j] * sc[j], m[3][j] * sc[j]);
         }
     };
 
+    // Sum and sign bits of delta per channel: thread pair (2 c, 2 c + 1) of a
+    // warp takes channel c of the warp's 16, each half of the chunk's steps.
+    float dpart = 0.0f;            // this thread's sum over the current segment
+    uint32_t dbits = 0;            // OR of the bit patterns it saw (sign bit: some delta < 0)
+    auto delta_sums = [&](const unsigned char* sbuf) {
+        const int ch = tid >> 1;
+        const int h0s = (tid & 1) * (T / 2);
+        float s2 = 0.0f;
+#pragma unroll
+        for (int k = 0; k < T / 2; k += 4) {
+            const float4 q = load4(reinterpret_cast<const IO*>(sbuf + TL::OFF_D + sw128(ch, (h0s + k) * EB)));
+            s2 += (q.x + q.y) + (q.z + q.w);
+            dbits |= __float_as_uint(q.x) | __float_as_uint(q.y) | __float_as_uint(q.z) | __float_as_uint(q.w);
+        }
+        dpart += s2;               // steps past the end of the sequence are zero-filled by TMA
+    };
+
     // delta, x of the two channels for 4 steps from a staged tile.
+    // (the 128-byte swizzle puts 16-byte chunk k of row r at chunk k ^ (r & 7):
+    // with the row's own bits precomputed in dxo, one XOR finds any chunk)
     auto load_dx = [&](const unsigned char* sbuf, int off, int tau, float (&v)[2][4]) {
+        const uint32_t kb = (uint32_t)(tau * EB);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            const float4 q = load4(reinterpret_cast<const IO*>(sbuf + off + sw128(cc0 + c, tau * EB)));
+            const float4 q = load4(reinterpret_cast<const IO*>(sbuf + off + ((dxo[c] ^ (kb & ~15u)) + (kb & 15u))));
             v[c][0] = q.x; v[c][1] = q.y; v[c][2] = q.z; v[c][3] = q.w;
         }
     };
 
-    // The lane's output after the butterfly: channel cc0 + (g >> 1), steps 4 (g & 1) .. + 3 of a group.
-    const bool oact = (g >> 1) ? act[1] : act[0];
-    const int64_t odch = (g >> 1) ? dch[1] : dch[0];
+    // The lane's output after the butterfly: its first channel, steps 4 (g & 1) .. + 3 of a group.
+    const bool oact = act[0];
+    const int64_t odch = dch[0];
     IO* const orow = static_cast<IO*>(p.y) + (b * p.dim + (oact ? odch : 0)) * L;
     const int ostep = (g & 1) * 4;
 
@@ -297,44 +356,37 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const float kappa = beta / (1.0f - beta);
 
     // Four steps of the two channels: the input delta * x (main pass) and the
-    // exponentials 2^(delta A log2 e) of the four states.
+    // exponentials of the four states (a, or a / beta in the scaled form).
     struct Quad {
         float u[2][4];
         float a[2][4][4];          // [channel][state][step]
     };
-    // Main pass state of the segment (zero start) and its running sums.
+    // Main pass state of the segment (zero start).
     float2 vv[2][2], hh[2][2], qq[2][2];
-    float2 bp2;                   // beta^(t+1)
-    float2 dacc[2];               // sum of delta over the current chunk, (even, odd) steps
-    uint32_t dbits;               // OR of delta's bit patterns over the segment
+    float2 bp2;                   // forcing of q: beta^(t+1) (plain form) or beta^(chunk start) (scaled form)
 
-    // Loads of a group: delta into dl; on the main pass x, u = delta * x, and
-    // the segment's delta sums.
     auto prep_load = [&](const unsigned char* sbuf, int tau, float (&dl)[2][4], Quad& Q, bool main_pass) {
         load_dx(sbuf, TL::OFF_D, tau, dl);
         if (main_pass) {
             float xl[2][4];
             load_dx(sbuf, TL::OFF_X, tau, xl);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int j2 = 0; j2 < 4; j2 += 2) {
                     const float2 uu = __fmul2_rn(f2(dl[c][j2], dl[c][j2 + 1]), f2(xl[c][j2], xl[c][j2 + 1]));
                     Q.u[c][j2] = uu.x;
                     Q.u[c][j2 + 1] = uu.y;
                 }
-                dbits |= __float_as_uint(dl[c][0]) | __float_as_uint(dl[c][1]) |
-                         __float_as_uint(dl[c][2]) | __float_as_uint(dl[c][3]);
-                // steps past the end of the sequence are zero-filled by TMA: no effect on the sum
-                dacc[c] = __fadd2_rn(dacc[c], __fadd2_rn(f2(dl[c][0], dl[c][1]), f2(dl[c][2], dl[c][3])));
-            }
         }
     };
     // Eight of a group's exponentials: channel c, steps 2 jp and 2 jp + 1.
     auto prep_exp = [&](const float (&dl)[2][4], Quad& Q, int c, int jp) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 ex = __fmul2_rn(f2(dl[c][2 * jp], dl[c][2 * jp + 1]), f2(Al[c][e], Al[c][e]));
+            const float2 dd = f2(dl[c][2 * jp], dl[c][2 * jp + 1]);
+            const float2 ex = SC ? __ffma2_rn(dd, f2(Al[c][e], Al[c][e]), f2(nl2b, nl2b))
+                                 : __fmul2_rn(dd, f2(Al[c][e], Al[c][e]));
             Q.a[c][e][2 * jp] = ex2_approx(ex.x);
             Q.a[c][e][2 * jp + 1] = ex2_approx(ex.y);
         }
@@ -364,8 +416,8 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const float2 aa = f2(Q.a[c][2 * q][j], Q.a[c][2 * q + 1][j]);
-                    const float2 w = __fmul2_rn(uu, bq[q]);
-                    const float2 vn = __ffma2_rn(beta2, vv[c][q], w);
+                    const float2 vn = SC ? __ffma2_rn(uu, bq[q], vv[c][q])
+                                         : __ffma2_rn(beta2, vv[c][q], __fmul2_rn(uu, bq[q]));
                     const float2 hn = __ffma2_rn(aa, hh[c][q], vn);
                     const float2 qn = __ffma2_rn(aa, qq[c][q], bp2);
                     if (valid) { vv[c][q] = vn; hh[c][q] = hn; qq[c][q] = qn; }
@@ -373,15 +425,27 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 yk[c][j0 + j] = yy.x + yy.y;
             }
-            if (valid) bp2 = __fmul2_rn(bp2, beta2);
+            if (!SC && valid) bp2 = __fmul2_rn(bp2, beta2);
         }
     };
 
     // Add the four lanes' partials of an 8-step group and store y (main pass),
     // or add them to the y stored by the main pass, read ahead into yold.
     auto flush = [&](const float (&yk)[2][8], int64_t t0, int first8, int nval, bool add, const float (&yold)[4]) {
+        // lanes g, g^2 hold the pair's channels in opposite order: keep the first,
+        // add the partner's second (the same channel); then lanes g, g^1 split the
+        // eight steps in halves
+        float s1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s1[i] = yk[0][i] + __shfl_xor_sync(0xffffffffu, yk[1][i], 2);
         float out[4];
-        butterfly_sum<G, 16>(*reinterpret_cast<const float(*)[16]>(&yk[0][0]), out, g);
+        const bool up = (g & 1) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float keep = up ? s1[4 + i] : s1[i];
+            const float send = up ? s1[i] : s1[4 + i];
+            out[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        }
         const int first = first8 + ostep;
         const int cnt = nval - first < 4 ? nval - first : 4;
         if (!oact || cnt <= 0) return;
@@ -408,7 +472,8 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
     };
 
-    // Correction state: the response to the carry-in.
+    // Correction state: the response to the carry-in (in the scaled form the
+    // velocity part v~ stays constant within a chunk).
     float2 rvv[2][2], rhh[2][2];
     auto corr_steps = [&](const Quad& Q, int tau, int j0, float (&yk)[2][8], bool ragged, int nval,
                           const float (&dln)[2][4], Quad& Qn, bool nxt) {
@@ -427,7 +492,7 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const float2 aa = f2(Q.a[c][2 * q][j], Q.a[c][2 * q + 1][j]);
-                    const float2 vn = __fmul2_rn(beta2, rvv[c][q]);
+                    const float2 vn = SC ? rvv[c][q] : __fmul2_rn(beta2, rvv[c][q]);
                     const float2 hn = __ffma2_rn(aa, rhh[c][q], vn);
                     if (valid) { rvv[c][q] = vn; rhh[c][q] = hn; }
                     yy = q == 0 ? __fmul2_rn(cq[0], rhh[c][0]) : __ffma2_rn(cq[1], rhh[c][1], yy);
@@ -495,6 +560,25 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 flush(yk, t0, g8, nval, !main_pass, yold);
             }
         }
+        if constexpr (SC) {
+            // back from the scaled variables: multiply by beta^(steps of the chunk)
+            const float s = tab_cb[nval - 1];
+            const float2 s2 = f2(s, s);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    if (main_pass) {
+                        vv[c][q] = __fmul2_rn(vv[c][q], s2);
+                        hh[c][q] = __fmul2_rn(hh[c][q], s2);
+                        qq[c][q] = __fmul2_rn(qq[c][q], s2);
+                    } else {
+                        rvv[c][q] = __fmul2_rn(rvv[c][q], s2);
+                        rhh[c][q] = __fmul2_rn(rhh[c][q], s2);
+                    }
+                }
+            if (main_pass) bp2 = __fmul2_rn(bp2, s2);
+        }
     };
 
     for (int64_t r = 0; r < rounds; ++r) {
@@ -508,8 +592,8 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int q = 0; q < 2; ++q) vv[c][q] = hh[c][q] = qq[c][q] = f2(0.0f, 0.0f);
-        bp2 = beta2;
-        float dsum[2] = {0.0f, 0.0f};                             // sum of delta over the segment
+        bp2 = SC ? f2(1.0f, 1.0f) : beta2;
+        dpart = 0.0f;
         dbits = 0;
         if (!dead && nch > 0) {
             for (int64_t j = 0; j < ST && j < nch; ++j) issue(s0 + j * T, true);
@@ -519,11 +603,9 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const int64_t t0 = s0 + kc * T;
                 const int nval = (int)(slen - kc * T < T ? slen - kc * T : T);
                 transpose(sbuf, true);
+                delta_sums(sbuf);
                 __syncthreads();
-                dacc[0] = dacc[1] = f2(0.0f, 0.0f);
                 run_chunk(sbuf, t0, nval, true);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) dsum[c] += dacc[c].x + dacc[c].y;
                 __syncthreads();          // every lane is done with this stage and B^T, C^T
                 const int64_t nx = kc + ST;
                 if (nx < nch) issue(s0 + nx * T, true);
@@ -533,6 +615,11 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
         // ================= publish this segment's map; fold the carries ===========
         const bool seg_nonneg = __syncthreads_and((dbits & 0x80000000u) == 0u) != 0;
+        // the channel's delta sum: its two threads' halves, then to the pair's lanes
+        const float dch_sum = dpart + __shfl_xor_sync(0xffffffffu, dpart, 1);
+        float dsum[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) dsum[c] = __shfl_sync(0xffffffffu, dch_sum, 2 * (lch[c] & 15));
         if (!dead) {
 #pragma unroll
             for (int c = 0; c < 2; ++c)
@@ -663,7 +750,7 @@ namespace {
 constexpr int kSegWarps = 1;
 constexpr int kSegStages = 2;
 
-template <typename IO>
+template <typename IO, bool SC>
 cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream) {
     using TL = SegTile<IO, kSegWarps, kSegStages>;
     ScanArgs a = a0;
@@ -680,7 +767,7 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream)
     if ((e = make_map_3d(&md, a.delta, bf, L, a.dim, a.batch, TL::T, TL::CH)) != cudaSuccess) return e;
     if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
     if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
-    auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages>;
+    auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages, SC>;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -725,8 +812,10 @@ int64_t scan_seg_default_len(int64_t batch, int64_t dim) {
 }
 
 cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s) {
-    if (io == 0) return launch_seg<float>(a, seg_len, s);
-    return launch_seg<bf16>(a, seg_len, s);
+    // The scaled form needs beta^-T within range: beta >= 1/2 (see the kernel).
+    const bool scaled = a.beta >= 0.5f;
+    if (io == 0) return scaled ? launch_seg<float, true>(a, seg_len, s) : launch_seg<float, false>(a, seg_len, s);
+    return scaled ? launch_seg<bf16, true>(a, seg_len, s) : launch_seg<bf16, false>(a, seg_len, s);
 }
 
 unsigned int scan_seg_read_and_clear_device_error() {

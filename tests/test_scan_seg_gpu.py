@@ -87,8 +87,9 @@ def _check(io, got, inp, beta, alpha, h0=None, v0=None, what=""):
 
 
 @pytest.mark.parametrize("L,seg", [(256, 32), (1000, 64), (4096, 128), (4133 // 4 * 4, 256), (96, 128)])
-@pytest.mark.parametrize("beta,alpha", [(0.9, 1.0), (0.0, 1.0), (0.99, 0.5)])
+@pytest.mark.parametrize("beta,alpha", [(0.9, 1.0), (0.0, 1.0), (0.99, 0.5), (0.3, 2.0), (0.5, 1.0)])
 def test_segments_rounds_and_ragged_ends(seg_path, L, seg, beta, alpha):
+    # beta >= 1/2 runs the scaled form of the recurrence, smaller beta the plain one
     # up to 32 segments: several rounds of an 8-CTA cluster, a ragged last chunk
     seg_path(seg)
     inp = _inputs(2, L, 40, 16, seed=7 + L)
