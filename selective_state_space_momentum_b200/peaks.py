@@ -19,7 +19,7 @@ import time
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 PROBE_LIB = os.path.join(_PKG, "libmmprobe.so")
-KINDS = {"ex2": 0, "ffma": 1, "ffma2": 2}
+KINDS = {"ex2": 0, "ffma": 1, "ffma2": 2, "ex2_lowocc": 3, "ex2_ffma2x3_lowocc": 4}
 SMS = 148
 
 
@@ -123,11 +123,44 @@ def measure(kinds=("ex2", "ffma", "ffma2"), target_ms: float = 25.0, reps: int =
     return res
 
 
-def main():
+def occupancy_sweep(warps_per_sm=(2, 4, 6, 8, 16), iters: int = 20000) -> dict:
+    """MUFU ex2 per clock per SM with one-warp blocks at the given warps per
+    SM, alone and with 3 dependent packed FMAs after each ex2 (8 chains per
+    thread; the rate is taken at the max SM clock)."""
     import torch
+    lib = _load()
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    out = torch.empty(sms * 16 * 32, device="cuda", dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+    res = {}
+    with _Clock(torch.cuda.current_device()) as clk:
+        for kind in ("ex2_lowocc", "ex2_ffma2x3_lowocc"):
+            for w in warps_per_sm:
+                blocks = sms * w
+                lib.mmprobe_launch(KINDS[kind], out.data_ptr(), blocks, 32, 100, stream.cuda_stream)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                rc = lib.mmprobe_launch(KINDS[kind], out.data_ptr(), blocks, 32, iters, stream.cuda_stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if rc != 0:
+                    raise RuntimeError(f"probe {kind}: CUDA error {rc}")
+                ms = e0.elapsed_time(e1)
+                ex2 = float(blocks) * 32 * iters * 8
+                res[f"{kind}/{w}"] = ex2 / (ms * 1e-3) / sms
+    mhz = clk.mhz()
+    return {k: v / (mhz * 1e6) for k, v in res.items()} | {"sm_mhz": mhz}
+
+
+def main():
+    import argparse
+    import torch
+    ap = argparse.ArgumentParser(description="measured pipe rates of this GPU")
+    ap.add_argument("--occupancy", action="store_true", help="MUFU rate against warps per SM")
+    args = ap.parse_args()
     if not torch.cuda.is_available():
         raise SystemExit("no CUDA device")
-    print(json.dumps(measure(), indent=1))
+    print(json.dumps(occupancy_sweep() if args.occupancy else measure(), indent=1))
 
 
 if __name__ == "__main__":
