@@ -98,12 +98,12 @@ typedef struct {
  * one); no other overlap between outputs and inputs is allowed
  * (MM_ERR_ALIAS).
  *
- * Two execution paths, chosen from (batch * dim, dstate, io) only, never
- * from L:
+ * Two execution paths, chosen from (batch * dim, dstate, io) and from
+ * whether L exceeds one segment of the sequence-split path:
  *   - register-resident: every (channel, state) lane walks the whole
  *     sequence in time order with its state in registers;
  *   - sequence-split (few channels, dstate 9..16, fp32, rows of a whole
- *     number of 16-byte pieces): the sequence is cut into segments of S
+ *     number of 16-byte pieces, L > S): the sequence is cut into segments of S
  *     steps (S a power of two, mm_scan_segment_len) at absolute multiples of
  *     S, each run from a zero state on its own CTA, and joined by folding
  *     each segment's 2x2 affine carry map onto the concrete carry in segment
@@ -115,11 +115,13 @@ typedef struct {
  * Streaming: for a fixed (batch, dim, dstate, io), calling with the first
  * L1 steps and then with the remaining steps, passing (hT, vT) of the first
  * call as (h0, v0) of the second, gives final states bit-identical to one
- * call over all steps, and the same y within rounding, when L1 is a
- * multiple of mm_scan_segment_len() (sequence-split path), of 32
- * (register-resident time split, mm_scan_set_tile with two time lanes), or
- * any L1 (register-resident path with one time lane, which applies the
- * steps in order).
+ * call over all steps, and the same y within rounding, when all three calls
+ * take the same path and L1 is a multiple of S (sequence-split path: S is
+ * the mm_scan_segment_len() of the calls), of 32 (register-resident time
+ * split, mm_scan_set_tile with two time lanes), or any L1 (register-resident
+ * path with one time lane, which applies the steps in order).  The path of
+ * each call is what mm_scan_segment_len() reports for its sizes (0: the
+ * register-resident path); mm_scan_set_path pins it.
  *
  * Errors: MM_ERR_NULL (x, delta, A, B, C, y or dims NULL), MM_ERR_DIMS
  * (a size < 1), MM_ERR_UNSUPPORTED (dstate > 16,
@@ -400,9 +402,11 @@ mm_status mm_scan_set_path(int path, int64_t seg_len);
 
 /*
  * mm_scan_segment_len -- the segment length S the scan uses for these sizes
- * (*seg_len = 0 when the call runs on the register-resident path).  A
- * streaming caller that splits a sequence at multiples of S gets final
- * states bit-identical to one call (see mm_scan_fwd).  Errors as
+ * (*seg_len = 0 when the call runs on the register-resident path, which the
+ * automatic choice takes whenever seqlen <= S).  S itself depends on
+ * (batch * dim) only.  A streaming caller that splits a sequence at
+ * multiples of S, into calls that all take the sequence-split path, gets
+ * final states bit-identical to one call (see mm_scan_fwd).  Errors as
  * mm_scan_fwd's size checks; MM_ERR_NULL for a NULL argument.
  */
 mm_status mm_scan_segment_len(const mm_scan_dims *dims, int64_t *seg_len);

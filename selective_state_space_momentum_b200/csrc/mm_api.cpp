@@ -40,24 +40,28 @@ std::atomic<int> g_forced_ts{1};
 std::atomic<int> g_forced_path{0};
 std::atomic<int64_t> g_forced_seg_len{0};
 
-// The automatic path choice depends on (batch * dim, dstate, io) only, never
-// on L, so calls that split one sequence take the same path.  The
-// sequence-split kernel pads the states to 16, so it serves dstate > 8; it
-// pays off when there are few channels (the register-resident kernel then
-// cannot fill the GPU).
+// The automatic path choice depends on (batch * dim, dstate, io) and on
+// whether the sequence is longer than one segment.  The sequence-split
+// kernel pads the states to 16, so it serves dstate > 8; it pays off when
+// there are few channels (the register-resident kernel then cannot fill the
+// GPU) and the sequence spans more than one segment (a single segment
+// leaves nothing to split).
 bool seg_auto(int64_t batch, int64_t dim, int64_t dstate, int io) {
     return dstate > 8 && io == MM_F32 && batch * dim <= 4096;
 }
 
 // Segment length of the sequence-split path for these sizes, or 0 when the
-// call runs on the register-resident kernel.
-int64_t seg_len_for(int64_t batch, int64_t dim, int64_t dstate, int io, bool vec_ok) {
+// call runs on the register-resident kernel.  The length itself depends on
+// (batch * dim) only, never on L.
+int64_t seg_len_for(int64_t batch, int64_t L, int64_t dim, int64_t dstate, int io, bool vec_ok) {
     const int path = g_forced_path.load();
     if (!vec_ok || dstate > 16) return 0;
     if (path == 1) return 0;
     if (path == 0 && !seg_auto(batch, dim, dstate, io)) return 0;
     const int64_t forced = g_forced_seg_len.load();
-    return forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
+    const int64_t S = forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
+    if (path == 0 && L <= S) return 0;
+    return S;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -231,7 +235,7 @@ mm_status mm_scan_segment_len(const mm_scan_dims* dims, int64_t* seg_len) {
     if (!dims || !seg_len) return fail(MM_ERR_NULL, "dims and seg_len are required");
     ScanSizes zs;
     if (mm_status st = check_scan_dims(dims, 0.0f, 1.0f, &zs)) return st;
-    *seg_len = seg_len_for(dims->batch, dims->dim, dims->dstate, dims->io,
+    *seg_len = seg_len_for(dims->batch, dims->seqlen, dims->dim, dims->dstate, dims->io,
                            ((dims->seqlen * zs.esize) % 16) == 0);
     return ok();
 }
@@ -300,7 +304,7 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.ckpt = ckpt;
     a.stall = inject_stall();
     if (!a.ext && !ckpt) {
-        const int64_t seg = seg_len_for(bsz, D, N, dims->io, a.vec_ok != 0);
+        const int64_t seg = seg_len_for(bsz, L, D, N, dims->io, a.vec_ok != 0);
         if (seg > 0)
             return from_cuda(mmscan::launch_scan_seg(a, dims->io, seg, static_cast<cudaStream_t>(stream)),
                              "mm_scan_fwd launch");

@@ -238,6 +238,10 @@ def test_set_path_and_segment_length_query(lib):
     seg = ctypes.c_int64(-1)
     dims = mm.ScanDims(1, 131072, 2048, 16, 0)
     assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 16384
+    one_segment = mm.ScanDims(1, 16384, 2048, 16, 0)               # L <= S: the register-resident path
+    assert lib.mm_scan_segment_len(ctypes.byref(one_segment), ctypes.byref(seg)) == 0 and seg.value == 0
+    just_over = mm.ScanDims(1, 16388, 2048, 16, 0)
+    assert lib.mm_scan_segment_len(ctypes.byref(just_over), ctypes.byref(seg)) == 0 and seg.value == 16384
     assert lib.mm_scan_set_path(2, 256) == 0
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg)) == 0
     assert seg.value == 256                                       # forced onto the sequence-split path

@@ -187,3 +187,5 @@ def test_segment_length_query():
     assert mm.mm_scan_segment_len(1, 131072, 1024, 16) == 32768
     assert mm.mm_scan_segment_len(4, 2048, 1536, 16) == 0          # register-resident path
     assert mm.mm_scan_segment_len(1, 131072, 2048, 8) == 0          # dstate <= 8
+    assert mm.mm_scan_segment_len(1, 256, 64, 16) == 0              # one segment: nothing to split
+    assert mm.mm_scan_segment_len(1, 16384, 2048, 16) == 0
