@@ -31,9 +31,12 @@
 //    the G lanes write consecutive steps of their channel.
 //  * Checkpoints (optional).  (h, v) after every 16 steps go to a
 //    (batch, dim, ceil(L / 16), 2, N) buffer that the backward restarts from.
-//  * Final state.  (h, v) after the last step go to hT, vT.  The per-state
-//    operation sequence does not depend on where the sequence is cut into
-//    calls, so split calls reproduce hT, vT bit for bit.
+//  * Final state.  (h, v) after the last step go to hT, vT.  With one time
+//    lane (TS = 1) the per-state operation sequence does not depend on where
+//    the sequence is cut into calls, so split calls reproduce hT, vT bit for
+//    bit at any split.  The time split (TS = 2) runs a full 32-step chunk as
+//    a zero-start second half plus a carry correction but a ragged chunk in
+//    order, so its splits reproduce hT, vT only at multiples of 32 steps.
 #include <cuda.h>
 
 #include <atomic>
