@@ -8,8 +8,12 @@
  * - Pointers named as device buffers must be CUDA device (or managed) memory
  *   of the current device; the caller allocates and owns every buffer.  The
  *   library allocates no memory and keeps no state between calls except a
- *   per-thread copy of the last error message (mm_last_error).
- * - Every base pointer must be 16-byte aligned (MM_ERR_ALIGN otherwise).
+ *   per-thread copy of the last error message (mm_last_error), the
+ *   process-wide tuning switches (mm_scan_set_tile, mm_scan_set_path) and
+ *   the per-thread side streams of the *_host entry points, which take host
+ *   buffers and a device workspace.
+ * - Every base pointer of a device buffer must be 16-byte aligned
+ *   (MM_ERR_ALIGN otherwise).
  *   Tensors are dense and contiguous in the stated layout, last index
  *   fastest.
  * - All argument checks run on the host before anything is launched; a call
@@ -363,6 +367,82 @@ mm_status mm_ssd_fwd_momentum(const void *x, const float *delta, const float *A,
                               const float *h0, const float *v0, float beta, float alpha,
                               void *y, float *hT, float *vT,
                               const mm_ssd_dims *dims, void *stream);
+
+/*
+ * Host-buffer entry points.
+ *
+ * mm_scan_fwd_host and mm_ssd_fwd_host compute exactly what mm_scan_fwd_gated
+ * and mm_ssd_fwd / mm_ssd_fwd_momentum compute, on tensors in HOST memory
+ * (same layouts and arguments; every tensor argument is a host pointer).
+ * The call streams the sequence through a device workspace in time chunks
+ * of `chunk_steps` steps (0: automatic -- about 1/32 of the streamed bytes
+ * per chunk, at least 8 MB and 2 KB host rows, a multiple of 32 steps for
+ * the scan and of dims->chunk for the SSD).  Chunk i's inputs are copied in
+ * on a stream of the call, its device call runs on `stream`, and its
+ * outputs are copied out on another stream of the call, through a ring of
+ * three workspace slots, so that with page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister) both directions of the host link and
+ * the kernels overlap.  Pageable host memory works too, without overlap.
+ * The carried states stay in the workspace between chunks, so the result
+ * is the device call's streaming result for that split (see mm_scan_fwd):
+ * with a chunk length that is a multiple of S on the sequence-split path,
+ * or on the register-resident path with one time lane, identical to the
+ * device entry point on the same sizes.
+ *
+ * Ordering: the call's copies start after the work queued on `stream`
+ * before the call, and work queued on `stream` after the call starts after
+ * the last copy-out; synchronise `stream` before reading the outputs.  The
+ * call returns once everything is queued (with pageable output buffers the
+ * copies themselves may block the host).
+ *
+ * workspace: device memory of at least the bytes the matching
+ * *_workspace_size query returns for the same dims and chunk_steps, 16-byte
+ * aligned, owned by the caller, not used by anything else until the call's
+ * work on `stream` has completed.  The library allocates no memory.  A call
+ * of more than one chunk runs its copies on two streams of its own, with
+ * eleven events; they are created on first use and kept for the calling
+ * host thread and device until the thread exits.  A call of one chunk runs
+ * everything on `stream`.
+ *
+ * Errors: those of the device entry point on the same sizes and scalars
+ * (checked before anything is queued), and MM_ERR_NULL (workspace NULL),
+ * MM_ERR_ALIGN (workspace), MM_ERR_DIMS (workspace too small, chunk_steps
+ * < 0), MM_ERR_UNSUPPORTED (a tensor argument in device memory, or the
+ * workspace not in device memory), MM_ERR_ALIAS (host output ranges that
+ * overlap an input or each other, except hT == h0 and vT == v0).  An error
+ * from CUDA after work was queued (MM_ERR_CUDA) leaves the outputs
+ * unspecified; the streams are still joined.
+ */
+
+/* Device workspace bytes of mm_scan_fwd_host for these sizes, with room for
+ * the gate z when with_z != 0. */
+mm_status mm_scan_fwd_host_workspace_size(const mm_scan_dims *dims, int with_z,
+                                          int64_t chunk_steps, size_t *bytes);
+
+/* mm_scan_fwd_gated over host tensors (D, z, delta_bias, h0, v0, hT, vT
+ * optional as there; no checkpoints). */
+mm_status mm_scan_fwd_host(const void *x, const void *delta, const float *A,
+                           const void *B, const void *C,
+                           const float *D, const void *z, const float *delta_bias,
+                           int delta_softplus,
+                           const float *h0, const float *v0, float beta, float alpha,
+                           void *y, float *hT, float *vT,
+                           void *workspace, size_t workspace_bytes, int64_t chunk_steps,
+                           const mm_scan_dims *dims, void *stream);
+
+/* Device workspace bytes of mm_ssd_fwd_host for these sizes; momentum != 0
+ * adds the carried velocity. */
+mm_status mm_ssd_fwd_host_workspace_size(const mm_ssd_dims *dims, int momentum,
+                                         int64_t chunk_steps, size_t *bytes);
+
+/* The SSD scan over host tensors: mm_ssd_fwd when beta == 0 and v0, vT are
+ * NULL, else mm_ssd_fwd_momentum (whose workspace needs momentum != 0). */
+mm_status mm_ssd_fwd_host(const void *x, const float *delta, const float *A,
+                          const void *B, const void *C,
+                          const float *h0, const float *v0, float beta, float alpha,
+                          void *y, float *hT, float *vT,
+                          void *workspace, size_t workspace_bytes, int64_t chunk_steps,
+                          const mm_ssd_dims *dims, void *stream);
 
 /*
  * mm_device_status -- synchronise the current device, then report whether

@@ -28,7 +28,10 @@ __all__ = [
     "mm_scan_step", "mm_ssd_fwd", "mm_ssd_fwd_momentum", "ssd_fwd_momentum",
     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
     "mm_scan_set_path", "mm_scan_segment_len",
+    "mm_scan_fwd_host", "mm_scan_fwd_host_workspace_size", "mm_ssd_fwd_host",
+    "mm_ssd_fwd_host_workspace_size",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
+    "ssd_fwd_host",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
 ]
 
@@ -53,7 +56,9 @@ EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm
                     "mm_ssd_fwd",
                     "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
-                    "mm_scan_set_path", "mm_scan_segment_len")
+                    "mm_scan_set_path", "mm_scan_segment_len",
+                    "mm_scan_fwd_host_workspace_size", "mm_scan_fwd_host",
+                    "mm_ssd_fwd_host_workspace_size", "mm_ssd_fwd_host")
 
 
 class MMError(RuntimeError):
@@ -105,6 +110,19 @@ def _declare(lib):
     lib.mm_ssd_fwd_momentum.restype = ctypes.c_int
     lib.mm_ssd_fwd_momentum.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp,
                                         ctypes.POINTER(SSDDims), vp]
+    i64, sz = ctypes.c_int64, ctypes.c_size_t
+    lib.mm_scan_fwd_host_workspace_size.restype = ctypes.c_int
+    lib.mm_scan_fwd_host_workspace_size.argtypes = [ctypes.POINTER(ScanDims), ctypes.c_int, i64,
+                                                    ctypes.POINTER(sz)]
+    lib.mm_scan_fwd_host.restype = ctypes.c_int
+    lib.mm_scan_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, f, f, vp, vp, vp,
+                                     vp, sz, i64, ctypes.POINTER(ScanDims), vp]
+    lib.mm_ssd_fwd_host_workspace_size.restype = ctypes.c_int
+    lib.mm_ssd_fwd_host_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int, i64,
+                                                   ctypes.POINTER(sz)]
+    lib.mm_ssd_fwd_host.restype = ctypes.c_int
+    lib.mm_ssd_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp, sz, i64,
+                                    ctypes.POINTER(SSDDims), vp]
     lib.mm_status_string.restype = ctypes.c_char_p
     lib.mm_status_string.argtypes = [ctypes.c_int]
     lib.mm_last_error.restype = ctypes.c_char_p
@@ -207,7 +225,19 @@ def _on_cuda(device):
         raise ValueError(f"the operands must be CUDA tensors (got device {device})")
 
 
-def _require_scan(x, A, tensors, seq_dims=3):
+def _on_host(device):
+    if device.type != "cpu":
+        raise ValueError(f"the host entry points take CPU tensors (got device {device})")
+
+
+def _require_workspace(ws):
+    import torch
+    if not isinstance(ws, torch.Tensor) or ws.device.type != "cuda" or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ws.numel() * ws.element_size()
+
+
+def _require_scan(x, A, tensors, seq_dims=3, host=False):
     """x (batch, dim, L) -- or (batch, dim) for a decode step -- and A (dim, N)
     fix the sizes; `tensors` is a list of (name, tensor, kind, optional) with
     kind one of io (like x), io_bc (batch, N[, L]) in x's type, state
@@ -234,10 +264,10 @@ def _require_scan(x, A, tensors, seq_dims=3):
     for name, t, kind, optional in tensors:
         shape, dts = shapes[kind]
         _require(name, t, shape, dts, dev, optional)
-    _on_cuda(dev)
+    (_on_host if host else _on_cuda)(dev)
 
 
-def _require_ssd(x, delta, A, B, C, y, states=()):
+def _require_ssd(x, delta, A, B, C, y, states=(), host=False):
     import torch
     load_library()
     dev, io = _lead(x, 4)
@@ -255,7 +285,7 @@ def _require_ssd(x, delta, A, B, C, y, states=()):
     _require("y", y, (batch, L, H, P), bf, dev)
     for name, t in states:
         _require(name, t, (batch, H, P, N), f32, dev, optional=True)
-    _on_cuda(dev)
+    (_on_host if host else _on_cuda)(dev)
 
 
 def mm_scan_fwd(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
@@ -357,6 +387,66 @@ def mm_ssd_fwd_momentum(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, strea
                                             _ptr(v0), float(beta), float(alpha), _ptr(y), _ptr(hT),
                                             _ptr(vT), ctypes.byref(dims), _stream_handle(stream))
     _check(rc, "mm_ssd_fwd_momentum")
+
+
+def mm_scan_fwd_host_workspace_size(batch, seqlen, dim, dstate, io=MM_F32, with_z=False, chunk_steps=0) -> int:
+    """C entry point mm_scan_fwd_host_workspace_size: device bytes the host
+    entry needs for these sizes."""
+    dims = ScanDims(batch, seqlen, dim, dstate, io)
+    out = ctypes.c_size_t(0)
+    _check(load_library().mm_scan_fwd_host_workspace_size(ctypes.byref(dims), 1 if with_z else 0,
+                                                          int(chunk_steps), ctypes.byref(out)),
+           "mm_scan_fwd_host_workspace_size")
+    return int(out.value)
+
+
+def mm_scan_fwd_host(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
+                     y, hT, vT, workspace, chunk_steps=0, stream=None):
+    """C entry point mm_scan_fwd_host (marshalling only): mm_scan_fwd_gated
+    on CPU tensors (page-locked for overlap) through a CUDA workspace tensor
+    of at least mm_scan_fwd_host_workspace_size bytes.  Queues the work on
+    ``stream`` and returns; synchronise before reading y, hT, vT."""
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("D", D, "vec", True), ("z", z, "io", True), ("delta_bias", delta_bias, "vec", True),
+                         ("h0", h0, "state", True), ("v0", v0, "state", True), ("y", y, "io", False),
+                         ("hT", hT, "state", True), ("vT", vT, "state", True)], host=True)
+    nbytes = _require_workspace(workspace)
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_fwd_host(
+        _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if delta_softplus else 0, _ptr(h0), _ptr(v0), float(beta), float(alpha), _ptr(y), _ptr(hT),
+        _ptr(vT), _ptr(workspace), nbytes, int(chunk_steps), ctypes.byref(dims),
+        _stream_handle(stream))
+    _check(rc, "mm_scan_fwd_host")
+
+
+def mm_ssd_fwd_host_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups=1, chunk=256,
+                                   momentum=False, chunk_steps=0) -> int:
+    """C entry point mm_ssd_fwd_host_workspace_size."""
+    dims = SSDDims(batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
+    out = ctypes.c_size_t(0)
+    _check(load_library().mm_ssd_fwd_host_workspace_size(ctypes.byref(dims), 1 if momentum else 0,
+                                                         int(chunk_steps), ctypes.byref(out)),
+           "mm_ssd_fwd_host_workspace_size")
+    return int(out.value)
+
+
+def mm_ssd_fwd_host(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, workspace, chunk=256,
+                    chunk_steps=0, stream=None):
+    """C entry point mm_ssd_fwd_host (marshalling only): the SSD scan on CPU
+    tensors (layouts as mm_ssd_fwd) through a CUDA workspace tensor."""
+    _require_ssd(x, delta, A, B, C, y, states=(("h0", h0), ("v0", v0), ("hT", hT), ("vT", vT)), host=True)
+    nbytes = _require_workspace(workspace)
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dims = SSDDims(batch, L, H, P, N, G, chunk)
+    rc = load_library().mm_ssd_fwd_host(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(v0),
+                                        float(beta), float(alpha), _ptr(y), _ptr(hT), _ptr(vT),
+                                        _ptr(workspace), nbytes, int(chunk_steps), ctypes.byref(dims),
+                                        _stream_handle(stream))
+    _check(rc, "mm_ssd_fwd_host")
 
 
 def mm_status_string(status: int) -> str:
@@ -530,28 +620,73 @@ def ssd_fwd_momentum(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, s
     return y, hT, vT
 
 
-def scan_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, device="cuda",
-                  out=None, stream=None, D=None, z=None, delta_bias=None, delta_softplus=False):
-    """End-to-end scan of host (CPU, ideally pinned) tensors.
+_ws_cache = {}
 
-    Copies the inputs to the device, runs mm_scan_fwd (mm_scan_fwd_gated when
-    any of D, z, delta_bias, delta_softplus is given), and copies y, hT and
-    vT back into ``out`` (a dict of host tensors, allocated if None).
-    Returns that dict after synchronising the stream.
-    """
+
+def _cached_workspace(device, nbytes):
+    """A device workspace of at least ``nbytes`` per device, kept between
+    calls (calls on one stream may share it; calls that may run at the same
+    time on different streams must pass workspaces of their own)."""
     import torch
-    s = stream or torch.cuda.current_stream(device)
-    with torch.cuda.stream(s):
-        dev = [t.to(device, non_blocking=True) if t is not None else None
-               for t in (x, delta, A, B, C, h0, v0, D, z, delta_bias)]
-        y, hT, vT = scan_fwd(*dev[:5], h0=dev[5], v0=dev[6], beta=beta, alpha=alpha, stream=s,
-                             D=dev[7], z=dev[8], delta_bias=dev[9], delta_softplus=delta_softplus)
+    dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    with _lock:
+        ws = _ws_cache.get(dev.index)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+            _ws_cache[dev.index] = ws
+    return ws
+
+
+def scan_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.9, alpha=1.0, device="cuda",
+                  out=None, stream=None, D=None, z=None, delta_bias=None, delta_softplus=False,
+                  chunk_steps=0, workspace=None):
+    """End-to-end scan of host (CPU, ideally page-locked) tensors through
+    mm_scan_fwd_host: the sequence is streamed through the device in time
+    chunks with copy-in, kernels and copy-out overlapped.  Results go to
+    ``out`` (a dict of host tensors y, hT, vT; page-locked ones are allocated
+    if None), returned after the stream has been synchronised."""
+    import torch
+    with torch.cuda.device(torch.device(device)):
+        s = stream or torch.cuda.current_stream()
+        batch, dim, L = x.shape
+        N = A.shape[1]
         if out is None:
-            out = {"y": torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
-                   "hT": torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True),
-                   "vT": torch.empty(vT.shape, dtype=vT.dtype, pin_memory=True)}
-        out["y"].copy_(y, non_blocking=True)
-        out["hT"].copy_(hT, non_blocking=True)
-        out["vT"].copy_(vT, non_blocking=True)
-    s.synchronize()
+            out = {"y": torch.empty(x.shape, dtype=x.dtype, pin_memory=True),
+                   "hT": torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=True),
+                   "vT": torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=True)}
+        if workspace is None:
+            need = mm_scan_fwd_host_workspace_size(batch, L, dim, N, _io_code(x.dtype), z is not None,
+                                                   chunk_steps)
+            workspace = _cached_workspace(device, need)
+        mm_scan_fwd_host(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, v0, beta, alpha,
+                         out["y"], out.get("hT"), out.get("vT"), workspace, chunk_steps, s)
+        s.synchronize()
+    return out
+
+
+def ssd_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.0, alpha=1.0, chunk=256, device="cuda",
+                 out=None, stream=None, chunk_steps=0, workspace=None):
+    """End-to-end SSD scan of host tensors through mm_ssd_fwd_host (the
+    momentum form when beta > 0 or v0 is given).  Results go to ``out`` (y,
+    hT and, with momentum, vT; page-locked ones allocated if None),
+    returned after the stream has been synchronised."""
+    import torch
+    momentum = beta != 0.0 or v0 is not None
+    with torch.cuda.device(torch.device(device)):
+        s = stream or torch.cuda.current_stream()
+        batch, L, H, P = x.shape
+        G, N = B.shape[2], B.shape[3]
+        if out is None:
+            out = {"y": torch.empty(x.shape, dtype=x.dtype, pin_memory=True),
+                   "hT": torch.empty((batch, H, P, N), dtype=torch.float32, pin_memory=True)}
+            if momentum:
+                out["vT"] = torch.empty((batch, H, P, N), dtype=torch.float32, pin_memory=True)
+        if workspace is None:
+            need = mm_ssd_fwd_host_workspace_size(batch, L, H, P, N, G, chunk, momentum, chunk_steps)
+            workspace = _cached_workspace(device, need)
+        mm_ssd_fwd_host(x, delta, A, B, C, h0, v0, beta, alpha, out["y"], out.get("hT"), out.get("vT"),
+                        workspace, chunk, chunk_steps, s)
+        s.synchronize()
     return out

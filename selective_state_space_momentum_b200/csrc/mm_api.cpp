@@ -171,6 +171,22 @@ mm_status check_scan_dims(const mm_scan_dims* dims, float beta, float alpha, Sca
 
 }  // namespace
 
+namespace mmscan {
+
+mm_status report(mm_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+mm_status report_ok() { return ok(); }
+
+}  // namespace mmscan
+
 extern "C" {
 
 const char* mm_status_string(mm_status s) {

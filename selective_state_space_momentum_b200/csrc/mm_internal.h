@@ -6,7 +6,18 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "mm_scan.h"
+
 namespace mmscan {
+
+// Record the calling thread's last error message (mm_last_error) and return
+// `st`; report_ok clears the message and returns MM_OK.
+mm_status report(mm_status st, const char* fmt, ...);
+mm_status report_ok();
+
+// Release the side streams and events the host-buffer entry points keep for
+// the calling thread (created again on the next call that needs them).
+void host_pipeline_release();
 
 // Arguments of one scan launch (device pointers; sizes as in mm_scan_dims).
 struct ScanArgs {

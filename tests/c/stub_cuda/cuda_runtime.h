@@ -21,6 +21,16 @@ cudaError_t cudaStreamWaitEvent(cudaStream_t s, cudaEvent_t e, unsigned flags);
 cudaError_t cudaMemcpyAsync(void* dst, const void* src, size_t n, cudaMemcpyKind k, cudaStream_t s);
 cudaError_t cudaMemcpy2DAsync(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width,
                               size_t height, cudaMemcpyKind k, cudaStream_t s);
+enum cudaMemoryType { cudaMemoryTypeUnregistered = 0, cudaMemoryTypeHost = 1, cudaMemoryTypeDevice = 2,
+                      cudaMemoryTypeManaged = 3 };
+struct cudaPointerAttributes {
+    enum cudaMemoryType type;
+    int device;
+    void* devicePointer;
+    void* hostPointer;
+};
+cudaError_t cudaPointerGetAttributes(cudaPointerAttributes* attr, const void* ptr);
+cudaError_t cudaGetDevice(int* device);
 cudaError_t cudaDeviceSynchronize(void);
 const char* cudaGetErrorString(cudaError_t e);
 const char* cudaGetErrorName(cudaError_t e);

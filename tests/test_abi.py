@@ -361,3 +361,34 @@ def test_host_checks_under_sanitizers(tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300,
                          env=dict(os.environ, ASAN_OPTIONS="detect_leaks=0"))
     assert run.returncode == 0 and "api checks ok" in run.stdout, (run.stdout + run.stderr)[-3000:]
+
+
+def test_host_pipeline_under_sanitizers(tmp_path):
+    """mm_host.cpp (the host-buffer entry points) and mm_api.cpp built with
+    AddressSanitizer and UndefinedBehaviorSanitizer against a stand-in
+    runtime whose streams are queues run in adversarial orders, with CPU
+    stand-ins for the kernels (tests/c/host_pipeline_sanitized.cpp): every
+    chunked call reproduces one device call byte for byte under 24
+    schedules, every copy and kernel operand stays inside its buffer, the
+    argument checks answer before anything is queued, and dropping any one
+    of the pipeline's waits makes some schedule fail."""
+    import shutil
+    import subprocess
+    cxx = shutil.which("g++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    csrc = os.path.join(root, "selective_state_space_momentum_b200", "csrc")
+    exe = tmp_path / "host_pipeline"
+    r = subprocess.run([cxx, "-std=c++17", "-O1", "-g", "-fsanitize=address,undefined", "-fno-omit-frame-pointer",
+                        "-fno-sanitize-recover=undefined", "-Wall", "-Werror",
+                        "-I", os.path.join(here, "c", "stub_cuda"), "-I", os.path.join(root, "include"), "-I", csrc,
+                        os.path.join(here, "c", "host_pipeline_sanitized.cpp"), os.path.join(csrc, "mm_api.cpp"),
+                        os.path.join(csrc, "mm_host.cpp"), "-o", str(exe)], capture_output=True, text=True)
+    if r.returncode != 0 and "sanitize" in r.stderr and "cannot find" in r.stderr:
+        pytest.skip("sanitizer runtimes not available")
+    assert r.returncode == 0, r.stderr[-3000:]
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300,
+                         env=dict(os.environ, ASAN_OPTIONS="detect_leaks=0"))
+    assert run.returncode == 0 and "host pipeline ok" in run.stdout, (run.stdout + run.stderr)[-3000:]
