@@ -13,8 +13,10 @@ workloads.py).
   inputs resident in HBM, timed with CUDA events on the launching stream over
   exactly K steps between barriers; several input sets rotate so that the
   bytes a step reads were evicted from the 126 MB L2 by the steps before it.
-* e2e: the same metric through the public host-memory call: every step copies
-  the inputs from pinned host memory, scans, and copies y, hT, vT back.
+* e2e: the same metric through the public host-memory call (mm_scan_fwd_host,
+  mm_ssd_fwd_host): every step streams the inputs from pinned host memory
+  through the device in time chunks, scans, and copies y, hT, vT back, with
+  copy-in, kernels and copy-out overlapped (--host-chunk sets the chunk).
 * roofline: the slower of the exponentials (one MUFU ex2 per state update)
   at the MUFU rate measured by libmmprobe (ex2 per clock per SM, scaled to
   148 SMs at the max SM clock) and the algorithmic bytes at the measured HBM
@@ -124,9 +126,49 @@ def rotating_sets(step_bytes: int) -> int:
     return min(4, max(2, math.ceil(2 * L2_BYTES / step_bytes) + 1))
 
 
+def needs_flush(step_bytes: int) -> bool:
+    """True when the rotating input sets together are too small to evict a
+    step's bytes from L2: the steps are then timed one by one with L2 flushed
+    in between."""
+    return rotating_sets(step_bytes) * step_bytes < 2 * L2_BYTES
+
+
+FLUSH_BYTES = 512 << 20
+
+
 def l2_note(step_bytes: int, what: str = "input") -> str:
     n = rotating_sets(step_bytes)
+    if needs_flush(step_bytes):
+        return (f"{n} rotating {what} sets ({n * step_bytes / 1e6:.1f} MB) fit in L2: each step timed alone "
+                f"between CUDA events, L2 flushed before it by writing {FLUSH_BYTES >> 20} MB")
     return f"{n} rotating {what} sets ({n * step_bytes / 1e6:.0f} MB) > 126 MB L2"
+
+
+def timed_ms(step, steps: int, stream, step_bytes: int) -> float:
+    """Device milliseconds of `steps` calls of step(i) on `stream` (CUDA
+    events on that stream).  Inputs larger than L2 in rotation: one event pair
+    around all steps.  Otherwise each step is timed alone, after a write of
+    FLUSH_BYTES that evicts L2 (and keeps the GPU busy while the host queues
+    the step); the sum of the per-step times is returned."""
+    import torch
+    if not needs_flush(step_bytes):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=stream.device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.fill_(i & 0xff)
+            evs[i][0].record(stream)
+            step(i)
+            evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs)
 
 
 def scan_config(w, beta, alpha, world, gated=False):
@@ -276,16 +318,11 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
-        ev0.record(stream)
-        for i in range(args.steps):
-            bwd(sets[i % nsets])
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        ms_timed = timed_ms(lambda i: bwd(sets[i % nsets]), args.steps, stream, step_bytes)
     barrier()
     torch.cuda.synchronize()
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
+    ms_step = max_over_ranks(ms_timed, dev) / args.steps
     value = whole_job_rate(w.updates, world, ms_step)
 
     # ---- end to end: host copies in, the backward, every gradient out ------
@@ -336,7 +373,7 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
                        "batch": w.batch, "seq_len": w.seqlen,
                        "dim": w.dim, "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
                        "global_batch": w.batch * world, "parallelism": f"dp{world}",
-                       "l2": f"{nsets} rotating input sets ({nsets * step_bytes / 1e6:.0f} MB) > 126 MB L2"},
+                       "l2": l2_note(step_bytes)},
             "roofline": {"bound": "alu", "kernel": "scan_bwd_kernel",
                          "achieved": achieved / 1e9, "peak": alu_peak / 1e9, "unit": "Gop/s",
                          "frac": achieved / alu_peak, "traffic": None,
@@ -398,16 +435,11 @@ def run_decode(args, w, rank, world):
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(sets[i % nsets])
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        ms_timed = timed_ms(lambda i: step(sets[i % nsets]), args.steps, stream, step_bytes)
     barrier()
     torch.cuda.synchronize()
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dev) / args.steps
+    ms_step = max_over_ranks(ms_timed, dev) / args.steps
     value = whole_job_rate(w.updates, world, ms_step)
 
     e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
@@ -777,16 +809,11 @@ def run_ssd(args, w, rank, world, local):
     mm.mm_device_status()
     barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if world == 1 else local) as clk:
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        ms_timed = timed_ms(step, args.steps, stream, step_bytes)
     mm.mm_device_status()
     barrier()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    ms_total = max_over_ranks(ms_timed, dev)
     ms_step = ms_total / args.steps
     value = whole_job_rate(w.updates, world, ms_step)
 
@@ -799,14 +826,10 @@ def run_ssd(args, w, rank, world, local):
     e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
 
     def e2e_step():
-        d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
-        if mom:
-            y, hT, _ = mm.ssd_fwd_momentum(d["x"], d["delta"], d["A"], d["B"], d["C"], beta=w.beta,
-                                           alpha=w.alpha)
-        else:
-            y, hT = mm.ssd_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], alpha=w.alpha, chunk=w.chunk)
-        out_y.copy_(y, non_blocking=True)
-        out_h.copy_(hT, non_blocking=True)
+        # mm_ssd_fwd_host: copy-in, the chunk's device call and copy-out overlapped
+        mm.ssd_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
+                        beta=w.beta if mom else 0.0, alpha=w.alpha, chunk=w.chunk,
+                        out={"y": out_y, "hT": out_h}, stream=stream, chunk_steps=args.host_chunk)
 
     for _ in range(2):
         e2e_step()
@@ -895,6 +918,8 @@ def main(argv=None):
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--host-chunk", type=int, default=0,
+                    help="time steps per chunk of the host-buffer call in the e2e leg (0: automatic)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget", type=float, default=60.0,
                     help="wall seconds for the whole --impl reference run")
@@ -1028,16 +1053,11 @@ def main(argv=None):
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if world == 1 else local) as clk:
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        ms_timed = timed_ms(step, args.steps, stream, step_bytes)
     barrier()
     torch.cuda.synchronize()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    ms_total = max_over_ranks(ms_timed, dev)
     ms_step = ms_total / args.steps
     updates = w.updates
     value = whole_job_rate(updates, world, ms_step)
@@ -1055,14 +1075,14 @@ def main(argv=None):
     d2h = sum(v.numel() * v.element_size() for v in out.values())
     for _ in range(2):
         mm.scan_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
-                         beta=beta, alpha=alpha, out=out, **extras)
+                         beta=beta, alpha=alpha, out=out, stream=stream, chunk_steps=args.host_chunk, **extras)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         mm.scan_fwd_host(pinned["x"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"],
-                         beta=beta, alpha=alpha, out=out, stream=stream, **extras)
+                         beta=beta, alpha=alpha, out=out, stream=stream, chunk_steps=args.host_chunk, **extras)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
