@@ -354,13 +354,16 @@ mm_status mm_ssd_fwd(const void *x, const float *delta, const float *A,
  *     v_t[p, n] = beta v_{t-1}[p, n] + alpha delta_t[h] B_t[g(h), n] x_t[h, p]
  *     h_t[p, n] = exp(delta_t[h] A[h]) h_{t-1}[p, n] + v_t[p, n]
  *     y_t[h, p] = sum_n C_t[g(h), n] h_t[p, n]
- * in the chunked form momentum leads to (chunks of 32 steps; the mask is
- * M_ij = sum_{k=j}^{i} exp(cs_i - cs_k) beta^(k-j), and the chunk carries
+ * in the chunked form momentum leads to (the mask is
+ * M_ij = sum_{k=j}^{i} exp(cs_i - cs_k) beta^(k-j), and each chunk carries
  * both h and v).  Layouts as mm_ssd_fwd; v0, vT like h0, hT (NULL: zero /
  * not written; vT may equal v0 and hT h0).  headdim <= 64, dstate <= 128;
- * dims->chunk is not used (any value >= 1).  Runs on the CUDA cores, not
- * the tensor cores.  Errors as mm_ssd_fwd (MM_ERR_UNSUPPORTED for headdim or
- * dstate past those bounds, seqlen > 2^30 or batch * H >= 2^31).
+ * dims->chunk is not used (any value >= 1).  headdim 64 with dstate 128
+ * runs on the tensor cores (tcgen05, blocks of 128 steps); other sizes on
+ * the CUDA cores (chunks of 32 steps).  Streaming calls split at a multiple
+ * of that block or chunk length reproduce y and the states bit for bit.
+ * Errors as mm_ssd_fwd (MM_ERR_UNSUPPORTED for headdim or dstate past those
+ * bounds, seqlen > 2^30 or batch * H >= 2^31).
  */
 mm_status mm_ssd_fwd_momentum(const void *x, const float *delta, const float *A,
                               const void *B, const void *C,

@@ -215,7 +215,8 @@ mm_status mm_device_status(void) {
     const unsigned int w = mmscan::scan_read_and_clear_device_error() |
                            mmscan::scan_seg_read_and_clear_device_error() |
                            mmscan::scan_bwd_read_and_clear_device_error() |
-                           mmscan::ssd_read_and_clear_device_error();
+                           mmscan::ssd_read_and_clear_device_error() |
+                           mmscan::ssd_mom_tc_read_and_clear_device_error();
     if (w) return fail(MM_ERR_DEVICE_TIMEOUT, "a device-side wait ran past its limit (word 0x%x)", w);
     return ok();
 }
@@ -558,6 +559,10 @@ mm_status mm_ssd_fwd_momentum(const void* x, const float* delta, const float* A,
     a.y = y; a.hT = hT; a.vT = vT;
     a.batch = bsz; a.seqlen = L; a.nheads = H; a.headdim = P; a.dstate = N; a.ngroups = G;
     a.beta = beta; a.alpha = alpha;
+    a.stall = inject_stall();
+    if (mmscan::ssd_mom_tc_shape_supported(P, N))
+        return from_cuda(mmscan::launch_ssd_mom_tc(a, static_cast<cudaStream_t>(stream)),
+                         "mm_ssd_fwd_momentum launch");
     return from_cuda(mmscan::launch_ssd_mom(a, static_cast<cudaStream_t>(stream)), "mm_ssd_fwd_momentum launch");
 }
 

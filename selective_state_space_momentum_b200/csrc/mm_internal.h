@@ -160,10 +160,15 @@ struct SSDMomArgs {
     float* vT;
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups;
     float beta, alpha;
+    int stall;             // test only (tensor-core kernel): stage no input, so that the bounded waits run out
 };
 
 bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate);
 cudaError_t launch_ssd_mom(const SSDMomArgs& a, cudaStream_t s);
+// The tensor-core form (ssd_mom_tc.cu) for headdim 64, dstate 128.
+bool ssd_mom_tc_shape_supported(int64_t headdim, int64_t dstate);
+cudaError_t launch_ssd_mom_tc(const SSDMomArgs& a, cudaStream_t s);
+unsigned int ssd_mom_tc_read_and_clear_device_error();
 
 bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk);
 cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t s);

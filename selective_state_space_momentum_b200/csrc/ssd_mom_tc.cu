@@ -1,0 +1,626 @@
+// ssd_mom_tc.cu -- the multi-head scalar-A scan with the Momentum Mamba
+// velocity, in the chunked (SSD) form, on sm_100a tensor cores (tcgen05 / TMEM).
+//
+// What it computes ("Momentum Mamba: Enhanced State Space Models with
+// Momentum", "Momentum Mamba Recurrence", in the multi-head layout of
+// "Mamba-2 -- SSM = structured matrix multiply", "Multi-Head Expansion"), for
+// batch row b, head h (group g = h / (H/G)), head channel p, state n:
+//     v_t[p, n] = beta v_{t-1}[p, n] + alpha delta_t B_t[n] x_t[p]
+//     h_t[p, n] = exp(delta_t A_h) h_{t-1}[p, n] + v_t[p, n]
+//     y_t[p]    = sum_n C_t[n] h_t[p, n]
+// through the chunked form of the "4-Step Algorithm" of the Mamba-2 page.
+// Per block of 128 rows with carried states (H, V) from the block before and
+// in-block cumulative log2-decay cs_i:
+//     y_i  = sum_{j<=i} M_ij (C_i . B_j) alpha delta_j x_j + 2^cs_i C_i.H + q_i C_i.V
+//     M_ij = sum_{k=j}^{i} 2^(cs_i - cs_k) beta^(k-j)     (q_i = beta M_i0)
+//     H'   = 2^cs_l H + q_l V + sum_j M_lj alpha delta_j B_j x_j^T
+//     V'   = beta^(l+1) V + sum_j beta^(l-j) alpha delta_j B_j x_j^T
+// with l the block's last row inside the sequence.  Every factor is a sum of
+// positive terms no larger than 1 / (1 - beta) while A <= 0, so nothing
+// cancels and nothing overflows.
+//
+// Tensor-core steps of a block (bf16 operands, fp32 accumulators in TMEM):
+//   CB  = C . B^T (128 x 128, K = N = 128)
+//   the mask warps form P_ij = M_ij alpha delta_j CB_ij (j <= i) in registers,
+//       M by the row recurrence R <- 2^(cs_i - cs_j) + beta R from the
+//       diagonal down to column 0, and write P back to TMEM as bf16 pairs
+//   Y_diag = P . X (A operand from TMEM)
+//   Y_A = C . H^T, Y_V = C . V^T (H, V as bf16 operands in shared memory)
+//   s_V = B^T . (w_V o X), s_H = B^T . (w_H o X), w_V = beta^(l-j) alpha delta,
+//       w_H = M_lj alpha delta
+// and y = Y_diag + 2^cs_i Y_A + q_i Y_V, stored as bf16, while the state
+// warps update (H, V) in fp32 registers.
+//
+// Roles (14 warps): warps 0-3 (mask warpgroup) scale X into w_V o X and,
+// once Y_diag has read X, into w_H o X in place, and form P; warps 4-7 and
+// 8-11 (state warpgroups, head channels 0-31 and 32-63) carry H and V and
+// write y; warps 4-7 also run the block's scans (cs, the suffix recurrence
+// for M_lj) one block ahead; warp 12 issues the TMA loads (no multicast)
+// into a 2-deep ring; warp 13 issues every tcgen05.mma.  Every wait is an
+// mbarrier wait bounded by kWaitLimitNs; on give-up the kernel records the
+// fact, every role leaves its loop (each group together), TMEM is freed and
+// the kernel returns.
+#include <cuda.h>
+
+#include <atomic>
+
+#include "mm_common.cuh"
+#include "mm_internal.h"
+#include "mm_tma_host.h"
+
+namespace mmscan {
+
+static __device__ unsigned int g_ssdm_dev_err = 0;
+
+namespace ssdmt {
+constexpr int P = 64;                  // head dimension
+constexpr int NS = 128;                // states
+constexpr int UB = 128;                // rows per block
+constexpr int NG = 128;                // threads of one warpgroup
+constexpr int NTHREADS = 3 * NG + 64;  // mask warpgroup, two state warpgroups, producer warp, MMA warp
+constexpr int W_PROD = 12, W_MMA = 13;
+static_assert(NTHREADS == 32 * (W_MMA + 1), "roles cover every warp");
+constexpr int X_TILE = UB * P * 2;          // 16 KB: [128 rows][64 p] bf16, 128-byte swizzle
+constexpr int BC_SLAB = UB * 64 * 2;        // 16 KB: [128 rows][64 states]
+constexpr int BC_TILE = 2 * BC_SLAB;        // 32 KB
+constexpr int SLOT = X_TILE + 2 * BC_TILE;  // 80 KB: X, B, C of one block
+constexpr int OFF_XV = 2 * SLOT;            // w_V o X
+constexpr int S_TILE = NS * P * 2;          // 16 KB: [128 rows n][64 p] bf16, swizzled
+constexpr int OFF_SH = OFF_XV + X_TILE;
+constexpr int OFF_SV = OFF_SH + S_TILE;
+constexpr int OFF_CS = OFF_SV + S_TILE;     // cs[2][128] (log2 units)
+constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha delta [2][128]
+constexpr int OFF_WV = OFF_DA + 2 * UB * 4; // w_V [2][128]
+constexpr int OFF_WH = OFF_WV + 2 * UB * 4; // w_H [2][128]
+constexpr int OFF_E = OFF_WH + 2 * UB * 4;  // 2^cs_i [2][128]
+constexpr int OFF_Q = OFF_E + 2 * UB * 4;   // q_i [2][128], written by the mask warps
+constexpr int OFF_BLK = OFF_Q + 2 * UB * 4; // per buffer: 2^cs_l, q_l, beta^(l+1), pad
+constexpr int OFF_RED = OFF_BLK + 2 * 16;   // scan partials
+constexpr int OFF_BAR = OFF_RED + 128;
+constexpr int NBAR = 24;
+constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
+constexpr int OFF_ABORT = OFF_TSLOT + 8;
+constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(SLOT % 1024 == 0 && OFF_XV % 1024 == 0 && OFF_SH % 1024 == 0 && OFF_SV % 1024 == 0,
+              "swizzled tiles are 1024-byte aligned");
+// TMEM columns (512): per block buffer k the fp32 C.B^T at 128k, which becomes
+// P (bf16 pairs) in its upper 64 columns and Y_diag in its lower 64; the
+// carried-state read-outs Y_A, Y_V; the block states s_H, s_V.
+__device__ __forceinline__ uint32_t tm_cb(int k) { return (uint32_t)k * 128u; }
+constexpr uint32_t TM_YA = 256, TM_YV = 320, TM_SH = 384, TM_SV = 448;
+constexpr uint32_t TM_COLS = 512;
+enum {
+    B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_SCAL = 10, B_TFREE = 12,  // pairs
+    B_XV = 14, B_XH = 15, B_STATE = 16, B_STFREE = 17, B_SFREE = 18, B_SREADY = 19, B_YOFREE = 20
+};
+constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
+constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . (w o X), both MN-major
+constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // P(tmem) . X
+constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 1);   // C . S^T
+}  // namespace ssdmt
+
+struct SSDMTArgs {
+    const float* delta;
+    const float* A;
+    const float* h0;
+    const float* v0;
+    bf16* y;
+    float* hT;
+    float* vT;
+    int64_t batch, seqlen, nheads, ngroups;
+    int nblocks;
+    float alpha, beta, lb;   // lb = log2(beta), or -1000 for beta = 0
+    int stall;
+};
+
+// 16 consecutive 32-bit TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// 14 warps on the SM's four schedulers: 4 warps x 32 lanes x 128 registers
+// fill one scheduler's register file, so 128 is the most a thread may take.
+__global__ void __maxnreg__(128)
+ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
+                  const __grid_constant__ CUtensorMap tm_C, const SSDMTArgs p) {
+    using namespace ssdmt;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (base - raw_addr);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t b = blockIdx.x / p.nheads;
+    const int64_t h = blockIdx.x % p.nheads;
+    const int64_t g = h / (p.nheads / p.ngroups);
+    const int64_t L = p.seqlen;
+    const int nblk = p.nblocks;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    auto bar = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
+    auto fsm = [&](int off, int k) { return reinterpret_cast<float*>(smem + off) + k * UB; };
+
+    if (tid == 0) {
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(bar(B_FULL + k), 1);
+            mbar_init(bar(B_EMPTY + k), 1);
+            mbar_init(bar(B_CB + k), 1);
+            mbar_init(bar(B_M + k), NG);
+            mbar_init(bar(B_Y + k), 1);
+            mbar_init(bar(B_SCAL + k), NG);
+            mbar_init(bar(B_TFREE + k), 2 * NG);
+        }
+        mbar_init(bar(B_XV), NG);
+        mbar_init(bar(B_XH), NG);
+        mbar_init(bar(B_STATE), 1);
+        mbar_init(bar(B_STFREE), 2 * NG);
+        mbar_init(bar(B_SFREE), 1);
+        mbar_init(bar(B_SREADY), 2 * NG);
+        mbar_init(bar(B_YOFREE), 2 * NG);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(base + OFF_TSLOT, TM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT);
+
+    auto wait = [&](int i, uint32_t parity) -> bool {
+        if (*abort_flag) return false;
+        if (!mbar_wait(bar(i), parity, &g_ssdm_dev_err)) {
+            *abort_flag = 1;
+            return false;
+        }
+        return true;
+    };
+
+    if (warp == W_PROD) {
+        // ------------------------------------------------------ producer ----
+        // (stall: test only, nothing staged, every other role's wait runs out)
+        if (lane == 0 && !p.stall) {
+            for (int u = 0; u < nblk; ++u) {
+                const int s = u & 1;
+                if (!wait(B_EMPTY + s, (uint32_t)(((u >> 1) + 1) & 1))) break;
+                const uint32_t slot = base + s * SLOT;
+                const uint32_t fb = bar(B_FULL + s);
+                mbar_expect_tx(fb, SLOT);
+                const int t0 = u * UB;
+                tma_load_4d(slot, &tm_x, fb, 0, (int)h, t0, (int)b);
+                tma_load_4d(slot + X_TILE, &tm_B, fb, 0, (int)g, t0, (int)b);
+                tma_load_4d(slot + X_TILE + BC_SLAB, &tm_B, fb, 64, (int)g, t0, (int)b);
+                tma_load_4d(slot + X_TILE + BC_TILE, &tm_C, fb, 0, (int)g, t0, (int)b);
+                tma_load_4d(slot + X_TILE + BC_TILE + BC_SLAB, &tm_C, fb, 64, (int)g, t0, (int)b);
+            }
+        }
+    } else if (warp == W_MMA) {
+        // ----------------------------------------------------------- MMA ----
+        // Per block u: the carried-state read-outs Y_A, Y_V (they need the
+        // states after block u-1), Y_diag (needs P), s_V, s_H (the scaled X
+        // copies), then C.B^T of block u+1 so the mask warps can start on it.
+        if (lane == 0) {
+            auto issue_cb = [&](int v) -> bool {
+                const int k = v & 1;
+                const uint32_t slot = base + k * SLOT;
+                const uint32_t bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
+                if (!wait(B_FULL + k, (uint32_t)((v >> 1) & 1))) return false;
+                if (!wait(B_TFREE + k, (uint32_t)(((v >> 1) + 1) & 1))) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
+                    umma_ss(tmem + tm_cb(k), umma_desc_sw128(cs + koff, 16, 1024),
+                            umma_desc_sw128(bs + koff, 16, 1024), ID_CB, ks > 0);
+                }
+                umma_commit(bar(B_CB + k));
+                return true;
+            };
+            bool live = nblk > 0 && issue_cb(0);
+            for (int u = 0; u < nblk && live; ++u) {
+                const int k = u & 1;
+                const uint32_t slot = base + k * SLOT;
+                const uint32_t xs = slot, bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
+                // Y_A = C . H^T, Y_V = C . V^T with the states after block u-1
+                if (!(live = wait(B_SREADY, (uint32_t)(u & 1)))) break;
+                if (!(live = wait(B_YOFREE, (uint32_t)((u + 1) & 1)))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
+                    umma_ss(tmem + TM_YA, umma_desc_sw128(cs + koff, 16, 1024),
+                            umma_desc_sw128(base + OFF_SH + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
+                }
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
+                    umma_ss(tmem + TM_YV, umma_desc_sw128(cs + koff, 16, 1024),
+                            umma_desc_sw128(base + OFF_SV + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
+                }
+                umma_commit(bar(B_SFREE));
+                // Y_diag = P(tmem) . X
+                if (!(live = wait(B_M + k, (uint32_t)((u >> 1) & 1)))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ts(tmem + tm_cb(k), tmem + tm_cb(k) + 64 + ks * 8,
+                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
+                umma_commit(bar(B_Y + k));
+                // s_V = B^T . (w_V o X) once the mask warps have scaled it, and the
+                // state warps have read the previous block's s_H, s_V
+                if (!(live = wait(B_XV, (uint32_t)(u & 1)))) break;
+                if (!(live = wait(B_STFREE, (uint32_t)((u + 1) & 1)))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ss(tmem + TM_SV, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
+                            umma_desc_sw128(base + OFF_XV + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
+                // s_H = B^T . (w_H o X), X scaled in place after Y_diag read it
+                if (!(live = wait(B_XH, (uint32_t)(u & 1)))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ss(tmem + TM_SH, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
+                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
+                umma_commit(bar(B_STATE));
+                umma_commit(bar(B_EMPTY + k));
+                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
+            }
+            // Drain: the last commit must land before the CTA may exit.
+            if (nblk > 0 && !*abort_flag) {
+                const int u = nblk - 1;
+                wait(B_EMPTY + (u & 1), (uint32_t)((u >> 1) & 1));
+            }
+        }
+    } else if (warp < 4) {
+        // ------------------------------------- mask warpgroup (warps 0-3) ----
+        const int i = tid;                          // TMEM lane = row i of the block
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float beta = p.beta;
+        // Waits are made uniform over the warpgroup (all leave the loop together),
+        // since the named barriers need every one of its threads.
+        auto gwait = [&](int bi, uint32_t par) { return named_bar_and(1, NG, wait(bi, par)); };
+        // Rows of X this warp scales: the warps with fewer mask batches take more.
+        const int r0 = warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116;
+        const int r1 = warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128;
+        auto scale_rows = [&](const unsigned char* src, unsigned char* dst, const float* w) {
+            const int units = (r1 - r0) * 8;
+            for (int e = lane; e < units; e += 32) {
+                const int r = r0 + (e >> 3);
+                const int pc = ((e & 7) ^ (r & 7)) << 4;        // swizzled 16-byte chunk
+                const float wr = w[r];
+                const uint4 q = *reinterpret_cast<const uint4*>(src + r * 128 + pc);
+                uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w4[c] = pack_bf16x2(bf16_lo(w4[c]) * wr, bf16_hi(w4[c]) * wr);
+                *reinterpret_cast<uint4*>(dst + r * 128 + pc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+        };
+        bool ok = true;
+        for (int u = 0; u < nblk && ok; ++u) {
+            const int k = u & 1;
+            unsigned char* xs = smem + k * SLOT;
+            // (a) block u's scalars are published
+            if (!(ok = gwait(B_SCAL + k, (uint32_t)((u >> 1) & 1)))) break;
+            // (b) w_V o X into its own tile: s_V of block u-1 must be done with it
+            if (u >= 1 && !(ok = gwait(B_STATE, (uint32_t)((u - 1) & 1)))) break;
+            if (!(ok = gwait(B_FULL + k, (uint32_t)((u >> 1) & 1)))) break;
+            scale_rows(xs, smem + OFF_XV, fsm(OFF_WV, k));
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_XV));
+            // (c) P = M o CB o alpha delta_j (j <= i): one batch of 32 columns at a
+            //     time from the diagonal batch down to batch 0, the recurrence
+            //     R <- 2^(cs_i - cs_j) + beta R running across batches.  Packed
+            //     batch cb goes to columns 64 + 16 cb, inside fp32 batches 2 and 3,
+            //     which this warp has read by then (or never reads).
+            const bool lok = __all_sync(0xffffffffu, wait(B_CB + k, (uint32_t)((u >> 1) & 1)));
+            tc_fence_after();
+            if (lok) {
+                const float* cs_sm = fsm(OFF_CS, k);
+                const float* da_sm = fsm(OFF_DA, k);
+                const float csi = cs_sm[i];
+                float R = 0.0f;
+#pragma unroll 1
+                for (int cb = warp; cb >= 0; --cb) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e4 = 7; e4 >= 0; --e4) {
+                        const float4 c4 = *reinterpret_cast<const float4*>(cs_sm + cb * 32 + 4 * e4);
+                        const float4 d4 = *reinterpret_cast<const float4*>(da_sm + cb * 32 + 4 * e4);
+                        const float csj[4] = {c4.x, c4.y, c4.z, c4.w};
+                        const float daj[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float m[4];
+#pragma unroll
+                        for (int jj = 3; jj >= 0; --jj) {
+                            const int j = cb * 32 + 4 * e4 + jj;
+                            const float lij = j <= i ? ex2_approx(csi - csj[jj]) : 0.0f;
+                            R = fmaf(beta, R, lij);
+                            m[jj] = R * (daj[jj] * __uint_as_float(r[4 * e4 + jj]));
+                        }
+                        pk[2 * e4] = pack_bf16x2(m[0], m[1]);
+                        pk[2 * e4 + 1] = pack_bf16x2(m[2], m[3]);
+                    }
+                    tmem_st16(tmem + lane_base + tm_cb(k) + 64 + cb * 16, pk);
+                }
+#pragma unroll 1
+                for (int cb = warp + 1; cb < 4; ++cb) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    tmem_st16(tmem + lane_base + tm_cb(k) + 64 + cb * 16, pk);
+                }
+                fsm(OFF_Q, k)[i] = beta * R;                 // q_i = beta M_i0
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            if (lok) mbar_arrive(bar(B_M + k));
+            // (d) w_H o X in place, after Y_diag has read X
+            if (!(ok = named_bar_and(1, NG, lok) && gwait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
+            scale_rows(xs, xs, fsm(OFF_WH, k));
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_XH));
+        }
+    } else if (warp < 12) {
+        // ------------------------- state warpgroups (warps 4-7 and 8-11) ----
+        const int sg = (warp - 4) >> 2;             // head channels 32 sg .. 32 sg + 31
+        const int t = tid - NG - sg * NG;           // TMEM lane: state n (update) and row i (output)
+        const int wq = (warp - 4) & 3;
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        const int pc0 = sg * 32;
+        float H[32], V[32];                         // state row n = t, channels pc0 .. pc0 + 31
+        {
+            const int64_t sbase = ((b * p.nheads + h) * P + pc0) * NS + t;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                H[q] = p.h0 ? p.h0[sbase + (int64_t)q * NS] : 0.0f;
+                V[q] = p.v0 ? p.v0[sbase + (int64_t)q * NS] : 0.0f;
+            }
+        }
+        // This thread's 32 channels of state row t as bf16 operands (MN-major, swizzled).
+        auto write_S = [&]() {
+            unsigned char* rh = smem + OFF_SH + t * 128;
+            unsigned char* rv = smem + OFF_SV + t * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int chunk = sg * 4 + c;
+                uint32_t wh[4], wv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    wh[e] = pack_bf16x2(H[c * 8 + 2 * e], H[c * 8 + 2 * e + 1]);
+                    wv[e] = pack_bf16x2(V[c * 8 + 2 * e], V[c * 8 + 2 * e + 1]);
+                }
+                const int off = (chunk ^ (t & 7)) << 4;
+                *reinterpret_cast<uint4*>(rh + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                *reinterpret_cast<uint4*>(rv + off) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_SREADY));
+        };
+        // Block v's scalars (first state warpgroup only; row t of the block):
+        // cs (inclusive prefix of delta A log2 e), alpha delta, 2^cs, w_V, w_H
+        // (the suffix recurrence r_j = 2^(cs_l - cs_j) + beta r_{j+1} gives
+        // M_lj), and per block 2^cs_l, q_l = beta M_l0, beta^(l+1).
+        const float a_h = p.A[h] * kLog2e;
+        const float beta = p.beta, lb = p.lb;
+        float* red = reinterpret_cast<float*>(smem + OFF_RED);
+        auto load_dt = [&](int v) -> float {
+            const int64_t tv = (int64_t)v * UB + t;
+            return tv < L ? p.delta[((b * L + tv) * p.nheads) + h] : 0.0f;
+        };
+        auto scan_block = [&](int v, float dt) {
+            const int kv = v & 1;
+            const int64_t left = L - (int64_t)v * UB;
+            const int last = left >= UB ? UB - 1 : (int)left - 1;
+            float cs = dt * a_h;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, cs, off);
+                if (lane >= off) cs += o;
+            }
+            if (lane == 31) red[wq] = cs;
+            named_bar_sync(2, NG);
+            float prefix = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (w < wq) prefix += red[w];
+            cs += prefix;
+            fsm(OFF_CS, kv)[t] = cs;
+            named_bar_sync(2, NG);                  // every cs_t in place (red reusable)
+            const float cs_l = fsm(OFF_CS, kv)[last];
+            const float da = p.alpha * dt;
+            // suffix recurrence over the rows j <= l, in-warp then across warps
+            float r = t <= last ? ex2_approx(cs_l - cs) : 0.0f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_down_sync(0xffffffffu, r, off);
+                if (lane + off < 32) r = fmaf(ex2_approx((float)off * lb), o, r);
+            }
+            if (lane == 0) red[4 + wq] = r;         // r at row 32 wq, this warp's rows only
+            named_bar_sync(2, NG);
+            float carry = 0.0f;                     // global r at row 32 (wq + 1)
+            for (int w = 3; w > wq; --w) carry = fmaf(ex2_approx(32.0f * lb), carry, red[4 + w]);
+            if (wq < 3) r = fmaf(ex2_approx((float)(32 - lane) * lb), carry, r);
+            fsm(OFF_DA, kv)[t] = da;
+            fsm(OFF_E, kv)[t] = ex2_approx(cs);
+            fsm(OFF_WV, kv)[t] = t <= last ? ex2_approx((float)(last - t) * lb) * da : 0.0f;
+            fsm(OFF_WH, kv)[t] = r * da;
+            if (t == 0) {
+                float* blk = reinterpret_cast<float*>(smem + OFF_BLK) + kv * 4;
+                blk[0] = ex2_approx(cs_l);
+                blk[1] = beta * r;                  // q_l = beta M_l0
+                blk[2] = ex2_approx((float)(last + 1) * lb);
+            }
+            mbar_arrive(bar(B_SCAL + kv));
+        };
+        auto swait = [&](int bi, uint32_t par) { return __all_sync(0xffffffffu, wait(bi, par)); };
+        float dt_next = 0.0f;
+        if (sg == 0) {
+            dt_next = nblk > 1 ? load_dt(1) : 0.0f;
+            if (nblk > 0) scan_block(0, load_dt(0));
+        }
+        write_S();                                  // the states before block 0
+        bool ok = true;
+        for (int u = 0; u < nblk; ++u) {
+            // Both state warpgroups leave together; and the second has finished
+            // block u-1 (its scalars and the q_i of that buffer) before the first
+            // overwrites the buffer with block u+1's.
+            ok = named_bar_and(3, 2 * NG, ok);
+            if (!ok) break;
+            const int k = u & 1;
+            const int64_t t0 = (int64_t)u * UB;
+            if (sg == 0 && u + 1 < nblk) {
+                const float dt1 = dt_next;
+                if (u + 2 < nblk) dt_next = load_dt(u + 2);
+                // the mask warps read buffer (u+1)&1 up to their in-place scaling of block u-1
+                ok = named_bar_and(2, NG, u == 0 || wait(B_XH, (uint32_t)((u - 1) & 1)));
+                if (ok) scan_block(u + 1, dt1);
+            }
+            // (d) H <- 2^cs_l H + q_l V + s_H, V <- beta^(l+1) V + s_V
+            ok = ok && swait(B_SCAL + k, (uint32_t)((u >> 1) & 1)) && swait(B_STATE, (uint32_t)(u & 1));
+            if (!ok) continue;
+            tc_fence_after();
+            {
+                const float* blk = reinterpret_cast<const float*>(smem + OFF_BLK) + k * 4;
+                const float gam = blk[0], ql = blk[1], bnv = blk[2];
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t sh[16], sv[16];
+                    tmem_ld16(tmem + lane_base + TM_SH + pc0 + hc * 16, sh);
+                    tmem_ld16(tmem + lane_base + TM_SV + pc0 + hc * 16, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int c = hc * 16 + q;
+                        const float hn = fmaf(gam, H[c], fmaf(ql, V[c], __uint_as_float(sh[q])));
+                        V[c] = fmaf(bnv, V[c], __uint_as_float(sv[q]));
+                        H[c] = hn;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_STFREE));
+            // publish the states after block u once Y_A(u), Y_V(u) have read the old ones
+            if (!(ok = swait(B_SFREE, (uint32_t)(u & 1)))) continue;
+            write_S();
+            // (e) y = Y_diag + 2^cs_i Y_A + q_i Y_V, bf16, row t of block u
+            if (!(ok = swait(B_M + k, (uint32_t)((u >> 1) & 1)) && swait(B_Y + k, (uint32_t)((u >> 1) & 1))))
+                continue;
+            tc_fence_after();
+            {
+                const float et = fsm(OFF_E, k)[t], qt = fsm(OFF_Q, k)[t];
+                const bool live_row = t0 + t < L;
+                bf16* yrow = p.y + ((b * L + t0 + t) * p.nheads + h) * P + pc0;
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t rd[16], ra[16], rv[16];
+                    tmem_ld16(tmem + lane_base + tm_cb(k) + pc0 + hc * 16, rd);
+                    tmem_ld16(tmem + lane_base + TM_YA + pc0 + hc * 16, ra);
+                    tmem_ld16(tmem + lane_base + TM_YV + pc0 + hc * 16, rv);
+                    tmem_wait_ld();
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float y0 = fmaf(qt, __uint_as_float(rv[2 * e]),
+                                              fmaf(et, __uint_as_float(ra[2 * e]), __uint_as_float(rd[2 * e])));
+                        const float y1 = fmaf(qt, __uint_as_float(rv[2 * e + 1]),
+                                              fmaf(et, __uint_as_float(ra[2 * e + 1]), __uint_as_float(rd[2 * e + 1])));
+                        w[e] = pack_bf16x2(y0, y1);
+                    }
+                    if (live_row) {
+                        uint4* dst = reinterpret_cast<uint4*>(yrow + hc * 16);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_TFREE + k));
+            mbar_arrive(bar(B_YOFREE));
+        }
+        if (ok && (p.hT || p.vT)) {
+            const int64_t sbase = ((b * p.nheads + h) * P + pc0) * NS + t;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                if (p.hT) p.hT[sbase + (int64_t)q * NS] = H[q];
+                if (p.vT) p.vT[sbase + (int64_t)q * NS] = V[q];
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+// ------------------------------------------------------------- launch -----
+namespace {
+
+// 4-D bf16 map (d0 innermost), box (64, 1, 128, 1) with the 128-byte swizzle.
+cudaError_t map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool ssd_mom_tc_shape_supported(int64_t headdim, int64_t dstate) {
+    return headdim == ssdmt::P && dstate == ssdmt::NS;
+}
+
+cudaError_t launch_ssd_mom_tc(const SSDMomArgs& a, cudaStream_t stream) {
+    if (a.batch * a.nheads > 0x7fffffffLL || a.seqlen > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    CUtensorMap mx, mB, mC;
+    cudaError_t e;
+    if ((e = map_4d(&mx, a.x, ssdmt::P, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
+    if ((e = map_4d(&mB, a.B, ssdmt::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
+    if ((e = map_4d(&mC, a.C, ssdmt::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
+    SSDMTArgs k{};
+    k.delta = a.delta; k.A = a.A; k.h0 = a.h0; k.v0 = a.v0;
+    k.y = static_cast<bf16*>(a.y); k.hT = a.hT; k.vT = a.vT;
+    k.batch = a.batch; k.seqlen = a.seqlen; k.nheads = a.nheads; k.ngroups = a.ngroups;
+    k.nblocks = (int)((a.seqlen + ssdmt::UB - 1) / ssdmt::UB);
+    k.alpha = a.alpha;
+    k.beta = a.beta;
+    k.lb = a.beta > 0.0f ? log2f(a.beta) : -1000.0f;
+    k.stall = a.stall;
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(ssd_mom_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 ssdmt::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done.fetch_or(bit, std::memory_order_release);
+    }
+    ssd_mom_tc_kernel<<<(unsigned)(a.batch * a.nheads), ssdmt::NTHREADS, ssdmt::SMEM_BYTES, stream>>>(mx, mB, mC, k);
+    return cudaGetLastError();
+}
+
+unsigned int ssd_mom_tc_read_and_clear_device_error() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_ssdm_dev_err, sizeof(v)) != cudaSuccess) return 0;
+    if (v) cudaMemcpyToSymbol(g_ssdm_dev_err, &z, sizeof(z));
+    return v;
+}
+
+}  // namespace mmscan

@@ -50,6 +50,9 @@ unsigned int ssd_read_and_clear_device_error() { return 0; }
 bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk) {
     return headdim == 64 && dstate == 128 && (chunk == 128 || chunk == 256);
 }
+bool ssd_mom_tc_shape_supported(int64_t headdim, int64_t dstate) { return headdim == 64 && dstate == 128; }
+cudaError_t launch_ssd_mom_tc(const SSDMomArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
+unsigned int ssd_mom_tc_read_and_clear_device_error() { return 0; }
 bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate) {
     return headdim >= 1 && headdim <= 64 && dstate >= 1 && dstate <= 128;
 }

@@ -390,6 +390,9 @@ bool ssd_shape_supported(int64_t headdim, int64_t dstate, int64_t chunk) {
     return headdim >= 1 && dstate >= 1 && chunk >= 1;
 }
 bool ssd_mom_shape_supported(int64_t headdim, int64_t dstate) { return headdim >= 1 && dstate >= 1; }
+bool ssd_mom_tc_shape_supported(int64_t, int64_t) { return false; }
+cudaError_t launch_ssd_mom_tc(const SSDMomArgs& a, cudaStream_t s) { return launch_ssd_mom(a, s); }
+unsigned int ssd_mom_tc_read_and_clear_device_error() { return 0; }
 }  // namespace mmscan
 
 // ---- the driver ---------------------------------------------------------------

@@ -9,7 +9,7 @@ all -- a flag that nothing sets, the allowed way to make a wait run out: no
 copy is in flight, no GPU fault is provoked -- and each test then checks the
 status and that a normal call right after still matches the fp64 oracle.
 One test per kernel family: the register-resident scan, the sequence-split
-scan, the backward, the SSD kernel.
+scan, the backward, the SSD kernel, the tensor-core momentum SSD kernel.
 """
 import numpy as np
 import pytest
@@ -94,3 +94,25 @@ def test_ssd_wait_runs_out(monkeypatch):
     yg = yg.transpose(0, 2, 3, 1).reshape(Bsz * H * P, L)
     rel = np.linalg.norm(yg - yr) / np.linalg.norm(yr)
     assert rel <= 1e-2, f"SSD after a timeout: relative L2 {rel:.3e}"
+
+
+def test_momentum_ssd_wait_runs_out(monkeypatch):
+    inp = wl.ssd_inputs(wl.SSD_MH, batch=1, seqlen=256, nheads=2)
+    dev = {"x": torch.from_numpy(inp["x"]).cuda().to(torch.bfloat16).contiguous(),
+           "delta": torch.from_numpy(inp["delta"]).cuda().contiguous(),
+           "A": torch.from_numpy(inp["A"]).cuda().contiguous(),
+           "B": torch.from_numpy(inp["B"]).cuda().to(torch.bfloat16).contiguous(),
+           "C": torch.from_numpy(inp["C"]).cuda().to(torch.bfloat16).contiguous()}
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "stall")
+    mm.ssd_fwd_momentum(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], beta=0.9)
+    monkeypatch.delenv("MMSCAN_FAULT_INJECT")
+    _expect_timeout()
+    y, hT, vT = mm.ssd_fwd_momentum(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], beta=0.9)
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    yr, hr, _ = oracle.ssd_seq(**inp, beta=0.9, alpha=1.0)
+    yg = y.float().cpu().numpy()
+    Bsz, L, H, P = inp["x"].shape
+    yg = yg.transpose(0, 2, 3, 1).reshape(Bsz * H * P, L)
+    rel = np.linalg.norm(yg - yr) / np.linalg.norm(yr)
+    assert rel <= 1e-2, f"momentum SSD after a timeout: relative L2 {rel:.3e}"
