@@ -746,14 +746,24 @@ def ssd_algorithmic_flops(w: wl.SSDWorkload) -> float:
     return w.batch * nchunk * (per_bc + w.nheads * per_head)
 
 
-def ssd_momentum_fmas(w: wl.SSDWorkload) -> float:
-    """Fused multiply-adds of the momentum chunked form with chunk Q: per
-    (batch, head, chunk) C.B^T (Q x Q x N), the causal half of the masked
-    product with X (Q x Q x P / 2), the read-out of both carried states
-    (2 x Q x P x N) and the update of both (2 x Q x P x N)."""
+def ssd_momentum_flops(w: wl.SSDWorkload) -> float:
+    """Tensor FLOPs of the momentum chunked form with chunk Q, full squares:
+    C.B^T once per (batch, chunk) (groups share it), then per head the masked
+    product with X, the read-out of both carried states (h and v) and both
+    chunk states."""
     nchunk = math.ceil(w.seqlen / w.chunk)
     Q, P, N = w.chunk, w.headdim, w.dstate
-    return w.batch * w.nheads * nchunk * (Q * Q * N + Q * Q * P / 2 + 4 * Q * P * N)
+    per_bc = 2 * Q * Q * N * w.ngroups
+    per_head = 2 * Q * Q * P + 4 * (2 * Q * N * P)
+    return w.batch * nchunk * (per_bc + w.nheads * per_head)
+
+
+def ssd_momentum_executed_flops(w: wl.SSDWorkload) -> float:
+    """Tensor FLOPs the momentum kernel issues: per head and 128-row block,
+    C.B^T (128x128x128), P.X, C.H^T, C.V^T, B^T.(w_H o X), B^T.(w_V o X)
+    (128x64x128 each)."""
+    nblk = math.ceil(w.seqlen / 128)
+    return w.batch * w.nheads * nblk * (2 * 128 * 128 * 128 + 5 * 2 * 128 * 128 * 64)
 
 
 def ssd_executed_flops(w: wl.SSDWorkload) -> float:
@@ -869,18 +879,15 @@ def run_ssd(args, w, rank, world, local):
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
         }
-        if mom:        # the CUDA-core chunked kernel: the fp32 FMA pipe is its roofline
-            sm_max = float(line["clocks"].get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
-            fma_peak = FP32_LANES_PER_CLK_PER_SM * B200_SMS * sm_max * 1e6
-            fmas = ssd_momentum_fmas(w)
-            line["roofline"] = {
-                "bound": "alu", "kernel": "ssd_mom_kernel", "achieved": fmas / (ms_step * 1e-3) / 1e9,
-                "peak": fma_peak / 1e9, "unit": "GFMA/s", "frac": fmas / (ms_step * 1e-3) / fma_peak,
-                "traffic": measured_traffic("ssd_mom_kernel", w.name),
-                "peak_source": f"128 fp32 lanes/clk/SM x 148 SMs x {sm_max:.0f} MHz",
-                "algorithmic_fmas": fmas,
-                "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
-                        "frac": hbm_achieved / hbm_peak, "algorithmic_bytes": step_bytes}}
+        if mom:        # the tensor-core momentum kernel: useful FLOPs of the momentum chunked form
+            alg = ssd_momentum_flops(w)
+            exe = ssd_momentum_executed_flops(w)
+            achieved = alg / (ms_step * 1e-3) / 1e12
+            line["roofline"].update({
+                "kernel": "ssd_mom_tc_kernel", "achieved": achieved, "frac": achieved / tf_peak,
+                "traffic": measured_traffic("ssd_mom_tc_kernel", w.name),
+                "algorithmic_flops": alg, "executed_flops": exe,
+                "executed_tflops": exe / (ms_step * 1e-3) / 1e12})
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = ssd_cpu_baseline(w)
         print(json.dumps(line), flush=True)

@@ -164,7 +164,9 @@ SCAN_LONG = ScanWorkload("scan_f32_b1_l131072_d2048_n16_stream", 1, 131072, 2048
 SSD_MH = SSDWorkload("ssd_bf16_b4_l4096_h32_p64_n128_g1_q256", 4, 4096, 32, 64, 128, 1, 256,
                      seed_index=4)
 # the same shapes and inputs with the momentum velocity (beta = 0.9)
-SSD_MH_MOMENTUM = SSDWorkload("ssd_momentum_bf16_b4_l4096_h32_p64_n128_g1", 4, 4096, 32, 64, 128, 1, 32,
+# chunk: the 128-step block of the tensor-core momentum kernel (the momentum
+# call takes no chunk argument; this is the Q of the FLOP count)
+SSD_MH_MOMENTUM = SSDWorkload("ssd_momentum_bf16_b4_l4096_h32_p64_n128_g1", 4, 4096, 32, 64, 128, 1, 128,
                               beta=0.9, seed_index=4)
 
 DECODE = DecodeWorkload("decode_bf16_b512_d2048_n16", 512, 2048, 16)
