@@ -28,13 +28,15 @@
 //   Y_A = C . H^T, Y_V = C . V^T (H, V as bf16 operands in shared memory)
 //   s_V = B^T . (w_V o X), s_H = B^T . (w_H o X), w_V = beta^(l-j) alpha delta,
 //       w_H = M_lj alpha delta
-// and y = Y_diag + 2^cs_i Y_A + q_i Y_V, stored as bf16, while the state
-// warps update (H, V) in fp32 registers.
+// and y = Y_diag + 2^cs_i Y_A + q_i Y_V, stored as bf16.  H and V stay in
+// TMEM as fp32 accumulators: per block the state warps publish them as the
+// bf16 read-out operands, rescale them in place (H <- 2^cs_l H + q_l V,
+// V <- beta^(l+1) V) and the block-state products accumulate onto them.
 //
 // Roles (14 warps): warps 0-3 (mask warpgroup) scale X into w_V o X and,
 // once Y_diag has read X, into w_H o X in place, and form P; warps 4-7 and
-// 8-11 (state warpgroups, head channels 0-31 and 32-63) carry H and V and
-// write y; warps 4-7 also run the block's scans (cs, the suffix recurrence
+// 8-11 (state warpgroups, head channels 0-31 and 32-63) publish and rescale
+// H and V and write y; warps 4-7 also run the block's scans (cs, the suffix recurrence
 // for M_lj) one block ahead; warp 12 issues the TMA loads (no multicast)
 // into a 2-deep ring; warp 13 issues every tcgen05.mma.  Every wait is an
 // mbarrier wait bounded by kWaitLimitNs; on give-up the kernel records the
@@ -86,13 +88,14 @@ static_assert(SLOT % 1024 == 0 && OFF_XV % 1024 == 0 && OFF_SH % 1024 == 0 && OF
               "swizzled tiles are 1024-byte aligned");
 // TMEM columns (512): per block buffer k the fp32 C.B^T at 128k, which becomes
 // P (bf16 pairs) in its upper 64 columns and Y_diag in its lower 64; the
-// carried-state read-outs Y_A, Y_V; the block states s_H, s_V.
+// carried-state read-outs Y_A, Y_V; the carried states H, V themselves
+// (lane n, column p), onto which the block-state products accumulate.
 __device__ __forceinline__ uint32_t tm_cb(int k) { return (uint32_t)k * 128u; }
-constexpr uint32_t TM_YA = 256, TM_YV = 320, TM_SH = 384, TM_SV = 448;
+constexpr uint32_t TM_YA = 256, TM_YV = 320, TM_H = 384, TM_V = 448;
 constexpr uint32_t TM_COLS = 512;
 enum {
     B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_SCAL = 10, B_TFREE = 12,  // pairs
-    B_XV = 14, B_XH = 15, B_STATE = 16, B_STFREE = 17, B_SFREE = 18, B_SREADY = 19, B_YOFREE = 20
+    B_XV = 14, B_XH = 15, B_STATE = 16, B_SCALED = 17, B_SFREE = 18, B_SREADY = 19, B_YOFREE = 20
 };
 constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
 constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . (w o X), both MN-major
@@ -127,7 +130,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 // fill one scheduler's register file, so 128 is the most a thread may take.
 __global__ void __maxnreg__(128)
 ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
-                  const __grid_constant__ CUtensorMap tm_C, const SSDMTArgs p) {
+                  const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_y,
+                  const SSDMTArgs p) {
     using namespace ssdmt;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -159,7 +163,7 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         mbar_init(bar(B_XV), NG);
         mbar_init(bar(B_XH), NG);
         mbar_init(bar(B_STATE), 1);
-        mbar_init(bar(B_STFREE), 2 * NG);
+        mbar_init(bar(B_SCALED), 2 * NG);
         mbar_init(bar(B_SFREE), 1);
         mbar_init(bar(B_SREADY), 2 * NG);
         mbar_init(bar(B_YOFREE), 2 * NG);
@@ -202,8 +206,8 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     } else if (warp == W_MMA) {
         // ----------------------------------------------------------- MMA ----
         // Per block u: the carried-state read-outs Y_A, Y_V (they need the
-        // states after block u-1), Y_diag (needs P), s_V, s_H (the scaled X
-        // copies), then C.B^T of block u+1 so the mask warps can start on it.
+        // states after block u-1), Y_diag (needs P), C.B^T of block u+1, then
+        // the block-state products onto the rescaled H, V.
         if (lane == 0) {
             auto issue_cb = [&](int v) -> bool {
                 const int k = v & 1;
@@ -251,25 +255,27 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     umma_ts(tmem + tm_cb(k), tmem + tm_cb(k) + 64 + ks * 8,
                             umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
                 umma_commit(bar(B_Y + k));
-                // s_V = B^T . (w_V o X) once the mask warps have scaled it, and the
-                // state warps have read the previous block's s_H, s_V
+                // C.B^T of block u+1 next, so the mask warps can start on it while
+                // this block's X is scaled for the state products
+                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
+                // V += B^T . (w_V o X) once the mask warps have scaled X and the
+                // state warps have rescaled V for this block (likewise H below)
                 if (!(live = wait(B_XV, (uint32_t)(u & 1)))) break;
-                if (!(live = wait(B_STFREE, (uint32_t)((u + 1) & 1)))) break;
+                if (!(live = wait(B_SCALED, (uint32_t)(u & 1)))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_ss(tmem + TM_SV, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
-                            umma_desc_sw128(base + OFF_XV + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
-                // s_H = B^T . (w_H o X), X scaled in place after Y_diag read it
+                    umma_ss(tmem + TM_V, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
+                            umma_desc_sw128(base + OFF_XV + ks * 2048, X_TILE, 1024), ID_ST, 1);
+                // H += B^T . (w_H o X), X scaled in place after Y_diag read it
                 if (!(live = wait(B_XH, (uint32_t)(u & 1)))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_ss(tmem + TM_SH, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
-                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_ST, ks > 0);
+                    umma_ss(tmem + TM_H, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
+                            umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_ST, 1);
                 umma_commit(bar(B_STATE));
                 umma_commit(bar(B_EMPTY + k));
-                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
             }
             // Drain: the last commit must land before the CTA may exit.
             if (nblk > 0 && !*abort_flag) {
@@ -282,17 +288,16 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         const int i = tid;                          // TMEM lane = row i of the block
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const float beta = p.beta;
-        // Waits are made uniform over the warpgroup (all leave the loop together),
-        // since the named barriers need every one of its threads.
-        auto gwait = [&](int bi, uint32_t par) { return named_bar_and(1, NG, wait(bi, par)); };
-        // Rows of X this warp scales: the warps with fewer mask batches take more.
-        const int r0 = warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116;
-        const int r1 = warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128;
-        auto scale_rows = [&](const unsigned char* src, unsigned char* dst, const float* w) {
+        // Waits are warp-uniform (the TMEM accesses are warp-collective) and
+        // the warps agree once per block at a named barrier, so that all of
+        // them leave the loop together when any wait has given up.
+        auto wwait = [&](int bi, uint32_t par) { return __all_sync(0xffffffffu, wait(bi, par)); };
+        // Scale rows [r0, r1) of an X tile by the per-row weights w (16-byte chunks, swizzled).
+        auto scale_rows = [&](const unsigned char* src, unsigned char* dst, const float* w, int r0, int r1) {
             const int units = (r1 - r0) * 8;
             for (int e = lane; e < units; e += 32) {
                 const int r = r0 + (e >> 3);
-                const int pc = ((e & 7) ^ (r & 7)) << 4;        // swizzled 16-byte chunk
+                const int pc = ((e & 7) ^ (r & 7)) << 4;
                 const float wr = w[r];
                 const uint4 q = *reinterpret_cast<const uint4*>(src + r * 128 + pc);
                 uint32_t w4[4] = {q.x, q.y, q.z, q.w};
@@ -301,26 +306,24 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 *reinterpret_cast<uint4*>(dst + r * 128 + pc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
         };
+        // w_V o X comes right after each warp's share of P: the warps with fewer
+        // mask batches are free first and take more of its rows.
+        const int v0r = warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116;
+        const int v1r = warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128;
         bool ok = true;
-        for (int u = 0; u < nblk && ok; ++u) {
+        for (int u = 0; u < nblk; ++u) {
+            ok = named_bar_and(1, NG, ok);
+            if (!ok) break;
             const int k = u & 1;
             unsigned char* xs = smem + k * SLOT;
-            // (a) block u's scalars are published
-            if (!(ok = gwait(B_SCAL + k, (uint32_t)((u >> 1) & 1)))) break;
-            // (b) w_V o X into its own tile: s_V of block u-1 must be done with it
-            if (u >= 1 && !(ok = gwait(B_STATE, (uint32_t)((u - 1) & 1)))) break;
-            if (!(ok = gwait(B_FULL + k, (uint32_t)((u >> 1) & 1)))) break;
-            scale_rows(xs, smem + OFF_XV, fsm(OFF_WV, k));
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_XV));
             // (c) P = M o CB o alpha delta_j (j <= i): one batch of 32 columns at a
             //     time from the diagonal batch down to batch 0, the recurrence
             //     R <- 2^(cs_i - cs_j) + beta R running across batches.  Packed
             //     batch cb goes to columns 64 + 16 cb, inside fp32 batches 2 and 3,
             //     which this warp has read by then (or never reads).
-            const bool lok = __all_sync(0xffffffffu, wait(B_CB + k, (uint32_t)((u >> 1) & 1)));
+            bool good = wwait(B_SCAL + k, (uint32_t)((u >> 1) & 1)) && wwait(B_CB + k, (uint32_t)((u >> 1) & 1));
             tc_fence_after();
-            if (lok) {
+            if (good) {
                 const float* cs_sm = fsm(OFF_CS, k);
                 const float* da_sm = fsm(OFF_DA, k);
                 const float csi = cs_sm[i];
@@ -361,12 +364,24 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 tmem_wait_st();
             }
             tc_fence_before();
-            if (lok) mbar_arrive(bar(B_M + k));
-            // (d) w_H o X in place, after Y_diag has read X
-            if (!(ok = named_bar_and(1, NG, lok) && gwait(B_Y + k, (uint32_t)((u >> 1) & 1)))) break;
-            scale_rows(xs, xs, fsm(OFF_WH, k));
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_XH));
+            if (good) mbar_arrive(bar(B_M + k));
+            // (b) w_V o X into its own tile: raw X has landed and s_V of block u-1
+            //     is done with the tile
+            good = good && wwait(B_FULL + k, (uint32_t)((u >> 1) & 1)) &&
+                   (u == 0 || wwait(B_STATE, (uint32_t)((u - 1) & 1)));
+            if (good) {
+                scale_rows(xs, smem + OFF_XV, fsm(OFF_WV, k), v0r, v1r);
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_XV));
+            }
+            // (d) w_H o X in place, after Y_diag has read X (32 rows per warp)
+            good = good && wwait(B_Y + k, (uint32_t)((u >> 1) & 1));
+            if (good) {
+                scale_rows(xs, xs, fsm(OFF_WH, k), warp * 32, warp * 32 + 32);
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_XH));
+            }
+            ok = good;
         }
     } else if (warp < 12) {
         // ------------------------- state warpgroups (warps 4-7 and 8-11) ----
@@ -375,34 +390,38 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         const int wq = (warp - 4) & 3;
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const int pc0 = sg * 32;
-        float H[32], V[32];                         // state row n = t, channels pc0 .. pc0 + 31
-        {
-            const int64_t sbase = ((b * p.nheads + h) * P + pc0) * NS + t;
+        const int64_t sbase = ((b * p.nheads + h) * P + pc0) * NS + t;   // h0[b, h, pc0, t]
+        // The initial states into TMEM: lane t = state n, this warpgroup's 32 channels.
+#pragma unroll 1
+        for (int hc = 0; hc < 2; ++hc) {
+            uint32_t wh[16], wv[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                H[q] = p.h0 ? p.h0[sbase + (int64_t)q * NS] : 0.0f;
-                V[q] = p.v0 ? p.v0[sbase + (int64_t)q * NS] : 0.0f;
+            for (int q = 0; q < 16; ++q) {
+                const int64_t o = sbase + (int64_t)(hc * 16 + q) * NS;
+                wh[q] = __float_as_uint(p.h0 ? p.h0[o] : 0.0f);
+                wv[q] = __float_as_uint(p.v0 ? p.v0[o] : 0.0f);
             }
+            tmem_st16(tmem + lane_base + TM_H + pc0 + hc * 16, wh);
+            tmem_st16(tmem + lane_base + TM_V + pc0 + hc * 16, wv);
         }
-        // This thread's 32 channels of state row t as bf16 operands (MN-major, swizzled).
-        auto write_S = [&]() {
-            unsigned char* rh = smem + OFF_SH + t * 128;
-            unsigned char* rv = smem + OFF_SV + t * 128;
+        tmem_wait_st();
+        // 16 channels (pc0 + 16 hc ..) of state row t as bf16 operands (MN-major, swizzled).
+        auto write_S16 = [&](int hc, const uint32_t (&rh)[16], const uint32_t (&rv)[16]) {
+            unsigned char* sh = smem + OFF_SH + t * 128;
+            unsigned char* sv = smem + OFF_SV + t * 128;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int chunk = sg * 4 + c;
+            for (int c = 0; c < 2; ++c) {
+                const int chunk = sg * 4 + hc * 2 + c;
                 uint32_t wh[4], wv[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    wh[e] = pack_bf16x2(H[c * 8 + 2 * e], H[c * 8 + 2 * e + 1]);
-                    wv[e] = pack_bf16x2(V[c * 8 + 2 * e], V[c * 8 + 2 * e + 1]);
+                    wh[e] = pack_bf16x2(__uint_as_float(rh[c * 8 + 2 * e]), __uint_as_float(rh[c * 8 + 2 * e + 1]));
+                    wv[e] = pack_bf16x2(__uint_as_float(rv[c * 8 + 2 * e]), __uint_as_float(rv[c * 8 + 2 * e + 1]));
                 }
                 const int off = (chunk ^ (t & 7)) << 4;
-                *reinterpret_cast<uint4*>(rh + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                *reinterpret_cast<uint4*>(rv + off) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                *reinterpret_cast<uint4*>(sh + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                *reinterpret_cast<uint4*>(sv + off) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_SREADY));
         };
         // Block v's scalars (first state warpgroup only; row t of the block):
         // cs (inclusive prefix of delta A log2 e), alpha delta, 2^cs, w_V, w_H
@@ -466,12 +485,12 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
             dt_next = nblk > 1 ? load_dt(1) : 0.0f;
             if (nblk > 0) scan_block(0, load_dt(0));
         }
-        write_S();                                  // the states before block 0
         bool ok = true;
         for (int u = 0; u < nblk; ++u) {
-            // Both state warpgroups leave together; and the second has finished
+            // Both state warpgroups leave together; the second has finished
             // block u-1 (its scalars and the q_i of that buffer) before the first
-            // overwrites the buffer with block u+1's.
+            // overwrites the buffer with block u+1's; and the y store of block
+            // u-1 has read its stage (the H operand tile) before it is rewritten.
             ok = named_bar_and(3, 2 * NG, ok);
             if (!ok) break;
             const int k = u & 1;
@@ -483,42 +502,49 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 ok = named_bar_and(2, NG, u == 0 || wait(B_XH, (uint32_t)((u - 1) & 1)));
                 if (ok) scan_block(u + 1, dt1);
             }
-            // (d) H <- 2^cs_l H + q_l V + s_H, V <- beta^(l+1) V + s_V
-            ok = ok && swait(B_SCAL + k, (uint32_t)((u >> 1) & 1)) && swait(B_STATE, (uint32_t)(u & 1));
-            if (!ok) continue;
-            tc_fence_after();
-            {
+            // (d) the states after block u-1: publish them as the bf16 operands of
+            //     Y_A(u), Y_V(u) (once Y_A(u-1), Y_V(u-1) have read the previous
+            //     ones), then rescale them in place for block u:
+            //     H <- 2^cs_l H + q_l V, V <- beta^(l+1) V
+            bool good = ok && swait(B_SCAL + k, (uint32_t)((u >> 1) & 1));
+            if (u >= 1)
+                good = good && swait(B_STATE, (uint32_t)((u - 1) & 1)) && swait(B_SFREE, (uint32_t)((u - 1) & 1));
+            if (good) {
+                tc_fence_after();
                 const float* blk = reinterpret_cast<const float*>(smem + OFF_BLK) + k * 4;
                 const float gam = blk[0], ql = blk[1], bnv = blk[2];
-#pragma unroll
+#pragma unroll 1
                 for (int hc = 0; hc < 2; ++hc) {
-                    uint32_t sh[16], sv[16];
-                    tmem_ld16(tmem + lane_base + TM_SH + pc0 + hc * 16, sh);
-                    tmem_ld16(tmem + lane_base + TM_SV + pc0 + hc * 16, sv);
+                    uint32_t rh[16], rv[16];
+                    tmem_ld16(tmem + lane_base + TM_H + pc0 + hc * 16, rh);
+                    tmem_ld16(tmem + lane_base + TM_V + pc0 + hc * 16, rv);
                     tmem_wait_ld();
+                    write_S16(hc, rh, rv);
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
-                        const int c = hc * 16 + q;
-                        const float hn = fmaf(gam, H[c], fmaf(ql, V[c], __uint_as_float(sh[q])));
-                        V[c] = fmaf(bnv, V[c], __uint_as_float(sv[q]));
-                        H[c] = hn;
+                        const float hv = __uint_as_float(rh[q]), vv = __uint_as_float(rv[q]);
+                        rh[q] = __float_as_uint(fmaf(gam, hv, ql * vv));
+                        rv[q] = __float_as_uint(bnv * vv);
                     }
+                    tmem_st16(tmem + lane_base + TM_H + pc0 + hc * 16, rh);
+                    tmem_st16(tmem + lane_base + TM_V + pc0 + hc * 16, rv);
                 }
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar(B_SREADY));
+                mbar_arrive(bar(B_SCALED));
             }
-            tc_fence_before();
-            mbar_arrive(bar(B_STFREE));
-            // publish the states after block u once Y_A(u), Y_V(u) have read the old ones
-            if (!(ok = swait(B_SFREE, (uint32_t)(u & 1)))) continue;
-            write_S();
-            // (e) y = Y_diag + 2^cs_i Y_A + q_i Y_V, bf16, row t of block u
-            if (!(ok = swait(B_M + k, (uint32_t)((u >> 1) & 1)) && swait(B_Y + k, (uint32_t)((u >> 1) & 1))))
-                continue;
-            tc_fence_after();
-            {
+            // (e) y = Y_diag + 2^cs_i Y_A + q_i Y_V, bf16, row t of block u, staged
+            //     in the H operand tile (Y_A(u), Y_V(u) are done with it: they
+            //     completed before Y_diag) in the y map's swizzled layout and
+            //     written by one TMA store per block; rows past L are clipped
+            good = good && swait(B_M + k, (uint32_t)((u >> 1) & 1)) && swait(B_Y + k, (uint32_t)((u >> 1) & 1));
+            if (good) {
+                tc_fence_after();
                 const float et = fsm(OFF_E, k)[t], qt = fsm(OFF_Q, k)[t];
-                const bool live_row = t0 + t < L;
-                bf16* yrow = p.y + ((b * L + t0 + t) * p.nheads + h) * P + pc0;
-#pragma unroll
+                unsigned char* yst = smem + OFF_SH + t * 128;
+#pragma unroll 1
                 for (int hc = 0; hc < 2; ++hc) {
                     uint32_t rd[16], ra[16], rv[16];
                     tmem_ld16(tmem + lane_base + tm_cb(k) + pc0 + hc * 16, rd);
@@ -534,23 +560,42 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                                               fmaf(et, __uint_as_float(ra[2 * e + 1]), __uint_as_float(rd[2 * e + 1])));
                         w[e] = pack_bf16x2(y0, y1);
                     }
-                    if (live_row) {
-                        uint4* dst = reinterpret_cast<uint4*>(yrow + hc * 16);
-                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const int chunk = sg * 4 + hc * 2 + c;
+                        *reinterpret_cast<uint4*>(yst + ((chunk ^ (t & 7)) << 4)) =
+                            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(bar(B_TFREE + k));
+                mbar_arrive(bar(B_YOFREE));
+                fence_proxy_async_smem();
             }
-            tc_fence_before();
-            mbar_arrive(bar(B_TFREE + k));
-            mbar_arrive(bar(B_YOFREE));
+            good = named_bar_and(4, 2 * NG, good);      // every row of the stage written
+            if (good && tid == NG) {
+                tma_store_4d(&tm_y, base + OFF_SH, 0, (int)h, (int)t0, (int)b);
+                bulk_commit_group();
+                bulk_wait_read_all();                    // the stage is free again
+            }
+            ok = good;
         }
-        if (ok && (p.hT || p.vT)) {
-            const int64_t sbase = ((b * p.nheads + h) * P + pc0) * NS + t;
+        if (tid == NG) bulk_wait_all();                  // y stores complete before the CTA exits
+        // the final states once the last block's products have landed
+        if (ok && nblk > 0 && (p.hT || p.vT) && swait(B_STATE, (uint32_t)((nblk - 1) & 1))) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int hc = 0; hc < 2; ++hc) {
+                uint32_t rh[16], rv[16];
+                tmem_ld16(tmem + lane_base + TM_H + pc0 + hc * 16, rh);
+                tmem_ld16(tmem + lane_base + TM_V + pc0 + hc * 16, rv);
+                tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                if (p.hT) p.hT[sbase + (int64_t)q * NS] = H[q];
-                if (p.vT) p.vT[sbase + (int64_t)q * NS] = V[q];
+                for (int q = 0; q < 16; ++q) {
+                    const int64_t o = sbase + (int64_t)(hc * 16 + q) * NS;
+                    if (p.hT) p.hT[o] = __uint_as_float(rh[q]);
+                    if (p.vT) p.vT[o] = __uint_as_float(rv[q]);
+                }
             }
         }
     }
@@ -566,7 +611,8 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
 // ------------------------------------------------------------- launch -----
 namespace {
 
-// 4-D bf16 map (d0 innermost), box (64, 1, 128, 1) with the 128-byte swizzle.
+// 4-D bf16 map (d0 innermost), box (64, 1, 128, 1) with the 128-byte swizzle
+// (the loads of x, B, C and the stores of y).
 cudaError_t map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -588,9 +634,10 @@ bool ssd_mom_tc_shape_supported(int64_t headdim, int64_t dstate) {
 
 cudaError_t launch_ssd_mom_tc(const SSDMomArgs& a, cudaStream_t stream) {
     if (a.batch * a.nheads > 0x7fffffffLL || a.seqlen > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    CUtensorMap mx, mB, mC;
+    CUtensorMap mx, mB, mC, my;
     cudaError_t e;
     if ((e = map_4d(&mx, a.x, ssdmt::P, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
+    if ((e = map_4d(&my, a.y, ssdmt::P, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = map_4d(&mB, a.B, ssdmt::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = map_4d(&mC, a.C, ssdmt::NS, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
     SSDMTArgs k{};
@@ -612,7 +659,7 @@ cudaError_t launch_ssd_mom_tc(const SSDMomArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_done.fetch_or(bit, std::memory_order_release);
     }
-    ssd_mom_tc_kernel<<<(unsigned)(a.batch * a.nheads), ssdmt::NTHREADS, ssdmt::SMEM_BYTES, stream>>>(mx, mB, mC, k);
+    ssd_mom_tc_kernel<<<(unsigned)(a.batch * a.nheads), ssdmt::NTHREADS, ssdmt::SMEM_BYTES, stream>>>(mx, mB, mC, my, k);
     return cudaGetLastError();
 }
 
