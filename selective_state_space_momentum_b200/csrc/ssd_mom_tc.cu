@@ -74,10 +74,11 @@ constexpr int OFF_CS = OFF_SV + S_TILE;     // cs[2][128] (log2 units)
 constexpr int OFF_DA = OFF_CS + 2 * UB * 4; // alpha delta [2][128]
 constexpr int OFF_WV = OFF_DA + 2 * UB * 4; // w_V [2][128]
 constexpr int OFF_WH = OFF_WV + 2 * UB * 4; // w_H [2][128]
-constexpr int OFF_E = OFF_WH + 2 * UB * 4;  // 2^cs_i [2][128]
-constexpr int OFF_Q = OFF_E + 2 * UB * 4;   // q_i [2][128], written by the mask warps
-constexpr int OFF_BLK = OFF_Q + 2 * UB * 4; // per buffer: 2^cs_l, q_l, beta^(l+1), pad
-constexpr int OFF_RED = OFF_BLK + 2 * 16;   // scan partials
+constexpr int OFF_CF = OFF_WH + 2 * UB * 4; // column factors 2^(ref - cs_j) [2][128]
+constexpr int OFF_Q = OFF_CF + 2 * UB * 4;  // q_i [2][128], written by the mask warps
+constexpr int OFF_BLK = OFF_Q + 2 * UB * 4; // per buffer: 2^cs_l, q_l, beta^(l+1), ref
+constexpr int OFF_MODE = OFF_BLK + 2 * 16;  // per buffer: 1 = factored block
+constexpr int OFF_RED = OFF_MODE + 16;      // scan partials
 constexpr int OFF_BAR = OFF_RED + 128;
 constexpr int NBAR = 24;
 constexpr int OFF_TSLOT = OFF_BAR + NBAR * 8;
@@ -93,6 +94,7 @@ static_assert(SLOT % 1024 == 0 && OFF_XV % 1024 == 0 && OFF_SH % 1024 == 0 && OF
 __device__ __forceinline__ uint32_t tm_cb(int k) { return (uint32_t)k * 128u; }
 constexpr uint32_t TM_YA = 256, TM_YV = 320, TM_H = 384, TM_V = 448;
 constexpr uint32_t TM_COLS = 512;
+static_assert(OFF_SV == OFF_SH + S_TILE && TM_YV == TM_YA + 64, "one read-out product spans both state tiles");
 enum {
     B_FULL = 0, B_EMPTY = 2, B_CB = 4, B_M = 6, B_Y = 8, B_SCAL = 10, B_TFREE = 12,  // pairs
     B_XV = 14, B_XH = 15, B_STATE = 16, B_SCALED = 17, B_SFREE = 18, B_SREADY = 19, B_YOFREE = 20
@@ -100,7 +102,12 @@ enum {
 constexpr uint32_t ID_CB = umma_idesc_bf16(128, 128, 0, 0);  // C . B^T
 constexpr uint32_t ID_ST = umma_idesc_bf16(128, 64, 1, 1);   // B^T . (w o X), both MN-major
 constexpr uint32_t ID_YD = umma_idesc_bf16(128, 64, 0, 1);   // P(tmem) . X
-constexpr uint32_t ID_YO = umma_idesc_bf16(128, 64, 0, 1);   // C . S^T
+constexpr uint32_t ID_YO = umma_idesc_bf16(128, 128, 0, 1);  // C . [H | V]^T (both states, N = 128)
+// A block is factored when every |cs_i - ref| (ref = cs_l / 2) stays within
+// this many powers of two: 2^(cs_i - cs_j) = 2^(cs_i - ref) 2^(ref - cs_j)
+// then splits into a row factor applied to Y_diag and column factors the mask
+// recurrence sums, far from the fp32 range limits.
+constexpr float FACTOR_RANGE = 60.0f;
 }  // namespace ssdmt
 
 struct SSDMTArgs {
@@ -124,6 +131,33 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+// One batch of 32 columns of row i of P, from column 32 cb + 31 down to 32 cb:
+// R <- l_ij + beta R with l_ij = 2^(ref - cs_j) (FAC: the column factor, the
+// row factor 2^(cs_i - ref) is applied to Y_diag) or 2^(cs_i - cs_j), zero
+// above the diagonal (DIAG: the batch that holds it); P_ij = R alpha delta_j
+// CB_ij, packed to bf16 pairs.  v holds cf_j (FAC) or cs_j, da alpha delta_j.
+template <bool FAC, bool DIAG>
+__device__ __forceinline__ void mom_mask_batch(const uint32_t (&r)[32], uint32_t (&pk)[16], float& R, int cb, int i,
+                                               float csi, float beta, const float* v, const float* da) {
+#pragma unroll
+    for (int e4 = 7; e4 >= 0; --e4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(v + cb * 32 + 4 * e4);
+        const float4 d4 = *reinterpret_cast<const float4*>(da + cb * 32 + 4 * e4);
+        const float vj[4] = {c4.x, c4.y, c4.z, c4.w};
+        const float dj[4] = {d4.x, d4.y, d4.z, d4.w};
+        float m[4];
+#pragma unroll
+        for (int jj = 3; jj >= 0; --jj) {
+            float l = FAC ? vj[jj] : ex2_approx(csi - vj[jj]);
+            if (DIAG) l = cb * 32 + 4 * e4 + jj <= i ? l : 0.0f;
+            R = fmaf(beta, R, l);
+            m[jj] = R * (dj[jj] * __uint_as_float(r[4 * e4 + jj]));
+        }
+        pk[2 * e4] = pack_bf16x2(m[0], m[1]);
+        pk[2 * e4 + 1] = pack_bf16x2(m[2], m[3]);
+    }
 }
 
 // 14 warps on the SM's four schedulers: 4 warps x 32 lanes x 128 registers
@@ -206,8 +240,9 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     } else if (warp == W_MMA) {
         // ----------------------------------------------------------- MMA ----
         // Per block u: the carried-state read-outs Y_A, Y_V (they need the
-        // states after block u-1), Y_diag (needs P), C.B^T of block u+1, then
-        // the block-state products onto the rescaled H, V.
+        // states after block u-1), Y_diag (needs P), V's block-state product
+        // onto the rescaled V, C.B^T of block u+1, then H's block-state product
+        // (its scaled X is formed in place after Y_diag).
         if (lane == 0) {
             auto issue_cb = [&](int v) -> bool {
                 const int k = v & 1;
@@ -230,7 +265,9 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 const int k = u & 1;
                 const uint32_t slot = base + k * SLOT;
                 const uint32_t xs = slot, bs = slot + X_TILE, cs = slot + X_TILE + BC_TILE;
-                // Y_A = C . H^T, Y_V = C . V^T with the states after block u-1
+                // Y_A = C . H^T and Y_V = C . V^T in one product with N = 128 (the H
+                // and V operand tiles are adjacent: two 64-column groups), with the
+                // states after block u-1
                 if (!(live = wait(B_SREADY, (uint32_t)(u & 1)))) break;
                 if (!(live = wait(B_YOFREE, (uint32_t)((u + 1) & 1)))) break;
                 tc_fence_after();
@@ -239,12 +276,6 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
                     umma_ss(tmem + TM_YA, umma_desc_sw128(cs + koff, 16, 1024),
                             umma_desc_sw128(base + OFF_SH + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
-                }
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t koff = (ks >> 2) * BC_SLAB + (ks & 3) * 32;
-                    umma_ss(tmem + TM_YV, umma_desc_sw128(cs + koff, 16, 1024),
-                            umma_desc_sw128(base + OFF_SV + ks * 2048, S_TILE, 1024), ID_YO, ks > 0);
                 }
                 umma_commit(bar(B_SFREE));
                 // Y_diag = P(tmem) . X
@@ -255,11 +286,8 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     umma_ts(tmem + tm_cb(k), tmem + tm_cb(k) + 64 + ks * 8,
                             umma_desc_sw128(xs + ks * 2048, X_TILE, 1024), ID_YD, ks > 0);
                 umma_commit(bar(B_Y + k));
-                // C.B^T of block u+1 next, so the mask warps can start on it while
-                // this block's X is scaled for the state products
-                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
                 // V += B^T . (w_V o X) once the mask warps have scaled X and the
-                // state warps have rescaled V for this block (likewise H below)
+                // state warps have rescaled V for this block
                 if (!(live = wait(B_XV, (uint32_t)(u & 1)))) break;
                 if (!(live = wait(B_SCALED, (uint32_t)(u & 1)))) break;
                 tc_fence_after();
@@ -267,7 +295,9 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 for (int ks = 0; ks < 8; ++ks)
                     umma_ss(tmem + TM_V, umma_desc_sw128(bs + ks * 2048, BC_SLAB, 1024),
                             umma_desc_sw128(base + OFF_XV + ks * 2048, X_TILE, 1024), ID_ST, 1);
-                // H += B^T . (w_H o X), X scaled in place after Y_diag read it
+                // C.B^T of block u+1, while the mask warps scale X in place for H
+                if (u + 1 < nblk && !(live = issue_cb(u + 1))) break;
+                // H += B^T . (w_H o X), X scaled in place once Y_diag has read it
                 if (!(live = wait(B_XH, (uint32_t)(u & 1)))) break;
                 tc_fence_after();
 #pragma unroll
@@ -292,40 +322,58 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         // the warps agree once per block at a named barrier, so that all of
         // them leave the loop together when any wait has given up.
         auto wwait = [&](int bi, uint32_t par) { return __all_sync(0xffffffffu, wait(bi, par)); };
-        // Scale rows [r0, r1) of an X tile by the per-row weights w (16-byte chunks, swizzled).
+        // Scale rows [r0, r1) of an X tile by the per-row weights w (16-byte chunks,
+        // swizzled), four chunks per lane in flight.
         auto scale_rows = [&](const unsigned char* src, unsigned char* dst, const float* w, int r0, int r1) {
             const int units = (r1 - r0) * 8;
-            for (int e = lane; e < units; e += 32) {
-                const int r = r0 + (e >> 3);
-                const int pc = ((e & 7) ^ (r & 7)) << 4;
-                const float wr = w[r];
-                const uint4 q = *reinterpret_cast<const uint4*>(src + r * 128 + pc);
-                uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+            for (int e0 = lane; e0 < units; e0 += 128) {
+                uint4 q[4];
+                float wr[4];
+                int off[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) w4[c] = pack_bf16x2(bf16_lo(w4[c]) * wr, bf16_hi(w4[c]) * wr);
-                *reinterpret_cast<uint4*>(dst + r * 128 + pc) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                for (int c = 0; c < 4; ++c) {
+                    const int e = e0 + 32 * c;
+                    const int r = r0 + (e >> 3);
+                    off[c] = r * 128 + (((e & 7) ^ (r & 7)) << 4);
+                    if (e < units) {
+                        wr[c] = w[r];
+                        q[c] = *reinterpret_cast<const uint4*>(src + off[c]);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (e0 + 32 * c >= units) continue;
+                    uint32_t w4[4] = {q[c].x, q[c].y, q[c].z, q[c].w};
+#pragma unroll
+                    for (int h2 = 0; h2 < 4; ++h2)
+                        w4[h2] = pack_bf16x2(bf16_lo(w4[h2]) * wr[c], bf16_hi(w4[h2]) * wr[c]);
+                    *reinterpret_cast<uint4*>(dst + off[c]) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
             }
         };
         // w_V o X comes right after each warp's share of P: the warps with fewer
         // mask batches are free first and take more of its rows.
         const int v0r = warp == 0 ? 0 : warp == 1 ? 52 : warp == 2 ? 92 : 116;
         const int v1r = warp == 0 ? 52 : warp == 1 ? 92 : warp == 2 ? 116 : 128;
+        unsigned char* xv = smem + OFF_XV;
         bool ok = true;
         for (int u = 0; u < nblk; ++u) {
             ok = named_bar_and(1, NG, ok);
             if (!ok) break;
             const int k = u & 1;
-            unsigned char* xs = smem + k * SLOT;
+            const unsigned char* xs = smem + k * SLOT;
             // (c) P = M o CB o alpha delta_j (j <= i): one batch of 32 columns at a
             //     time from the diagonal batch down to batch 0, the recurrence
-            //     R <- 2^(cs_i - cs_j) + beta R running across batches.  Packed
-            //     batch cb goes to columns 64 + 16 cb, inside fp32 batches 2 and 3,
-            //     which this warp has read by then (or never reads).
+            //     running across batches.  Packed batch cb goes to columns
+            //     64 + 16 cb, inside fp32 batches 2 and 3, which this warp has read
+            //     by then (or never reads).
             bool good = wwait(B_SCAL + k, (uint32_t)((u >> 1) & 1)) && wwait(B_CB + k, (uint32_t)((u >> 1) & 1));
             tc_fence_after();
             if (good) {
+                const bool fac = reinterpret_cast<volatile const int*>(smem + OFF_MODE)[k] != 0;
                 const float* cs_sm = fsm(OFF_CS, k);
                 const float* da_sm = fsm(OFF_DA, k);
+                const float* v_sm = fac ? fsm(OFF_CF, k) : cs_sm;
                 const float csi = cs_sm[i];
                 float R = 0.0f;
 #pragma unroll 1
@@ -334,22 +382,12 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     tmem_ld32(tmem + lane_base + tm_cb(k) + cb * 32, r);
                     tmem_wait_ld();
                     uint32_t pk[16];
-#pragma unroll
-                    for (int e4 = 7; e4 >= 0; --e4) {
-                        const float4 c4 = *reinterpret_cast<const float4*>(cs_sm + cb * 32 + 4 * e4);
-                        const float4 d4 = *reinterpret_cast<const float4*>(da_sm + cb * 32 + 4 * e4);
-                        const float csj[4] = {c4.x, c4.y, c4.z, c4.w};
-                        const float daj[4] = {d4.x, d4.y, d4.z, d4.w};
-                        float m[4];
-#pragma unroll
-                        for (int jj = 3; jj >= 0; --jj) {
-                            const int j = cb * 32 + 4 * e4 + jj;
-                            const float lij = j <= i ? ex2_approx(csi - csj[jj]) : 0.0f;
-                            R = fmaf(beta, R, lij);
-                            m[jj] = R * (daj[jj] * __uint_as_float(r[4 * e4 + jj]));
-                        }
-                        pk[2 * e4] = pack_bf16x2(m[0], m[1]);
-                        pk[2 * e4 + 1] = pack_bf16x2(m[2], m[3]);
+                    if (fac) {
+                        if (cb == warp) mom_mask_batch<true, true>(r, pk, R, cb, i, csi, beta, v_sm, da_sm);
+                        else mom_mask_batch<true, false>(r, pk, R, cb, i, csi, beta, v_sm, da_sm);
+                    } else {
+                        if (cb == warp) mom_mask_batch<false, true>(r, pk, R, cb, i, csi, beta, v_sm, da_sm);
+                        else mom_mask_batch<false, false>(r, pk, R, cb, i, csi, beta, v_sm, da_sm);
                     }
                     tmem_st16(tmem + lane_base + tm_cb(k) + 64 + cb * 16, pk);
                 }
@@ -360,24 +398,26 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
                     tmem_st16(tmem + lane_base + tm_cb(k) + 64 + cb * 16, pk);
                 }
-                fsm(OFF_Q, k)[i] = beta * R;                 // q_i = beta M_i0
+                // q_i = beta M_i0 (a factored block's R carries M / 2^(cs_i - ref))
+                const float ref = (reinterpret_cast<const float*>(smem + OFF_BLK) + k * 4)[3];
+                fsm(OFF_Q, k)[i] = beta * (fac ? ex2_approx(csi - ref) * R : R);
                 tmem_wait_st();
             }
             tc_fence_before();
             if (good) mbar_arrive(bar(B_M + k));
             // (b) w_V o X into its own tile: raw X has landed and s_V of block u-1
-            //     is done with the tile
+            //     has read the tile's previous contents
             good = good && wwait(B_FULL + k, (uint32_t)((u >> 1) & 1)) &&
                    (u == 0 || wwait(B_STATE, (uint32_t)((u - 1) & 1)));
             if (good) {
-                scale_rows(xs, smem + OFF_XV, fsm(OFF_WV, k), v0r, v1r);
+                scale_rows(xs, xv, fsm(OFF_WV, k), v0r, v1r);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_XV));
             }
-            // (d) w_H o X in place, after Y_diag has read X (32 rows per warp)
+            // (d) w_H o X in place once Y_diag has read X (32 rows per warp)
             good = good && wwait(B_Y + k, (uint32_t)((u >> 1) & 1));
             if (good) {
-                scale_rows(xs, xs, fsm(OFF_WH, k), warp * 32, warp * 32 + 32);
+                scale_rows(xs, const_cast<unsigned char*>(xs), fsm(OFF_WH, k), warp * 32, warp * 32 + 32);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_XH));
             }
@@ -467,8 +507,11 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
             float carry = 0.0f;                     // global r at row 32 (wq + 1)
             for (int w = 3; w > wq; --w) carry = fmaf(ex2_approx(32.0f * lb), carry, red[4 + w]);
             if (wq < 3) r = fmaf(ex2_approx((float)(32 - lane) * lb), carry, r);
+            // factored (see FACTOR_RANGE) when every row is within range of ref = cs_l / 2
+            const float ref = 0.5f * cs_l;
+            const bool fac = named_bar_and(2, NG, fabsf(cs - ref) <= FACTOR_RANGE);
             fsm(OFF_DA, kv)[t] = da;
-            fsm(OFF_E, kv)[t] = ex2_approx(cs);
+            fsm(OFF_CF, kv)[t] = fac ? ex2_approx(ref - cs) : 0.0f;
             fsm(OFF_WV, kv)[t] = t <= last ? ex2_approx((float)(last - t) * lb) * da : 0.0f;
             fsm(OFF_WH, kv)[t] = r * da;
             if (t == 0) {
@@ -476,6 +519,8 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 blk[0] = ex2_approx(cs_l);
                 blk[1] = beta * r;                  // q_l = beta M_l0
                 blk[2] = ex2_approx((float)(last + 1) * lb);
+                blk[3] = ref;
+                reinterpret_cast<volatile int*>(smem + OFF_MODE)[kv] = fac ? 1 : 0;
             }
             mbar_arrive(bar(B_SCAL + kv));
         };
@@ -542,7 +587,11 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
             good = good && swait(B_M + k, (uint32_t)((u >> 1) & 1)) && swait(B_Y + k, (uint32_t)((u >> 1) & 1));
             if (good) {
                 tc_fence_after();
-                const float et = fsm(OFF_E, k)[t], qt = fsm(OFF_Q, k)[t];
+                // y_i = rf_i Y_diag + 2^cs_i Y_A + q_i Y_V; rf_i = 2^(cs_i - ref) on a factored block
+                const float csi = fsm(OFF_CS, k)[t], qt = fsm(OFF_Q, k)[t];
+                const bool fac = reinterpret_cast<volatile const int*>(smem + OFF_MODE)[k] != 0;
+                const float ref = (reinterpret_cast<const float*>(smem + OFF_BLK) + k * 4)[3];
+                const float et = ex2_approx(csi), rf = fac ? ex2_approx(csi - ref) : 1.0f;
                 unsigned char* yst = smem + OFF_SH + t * 128;
 #pragma unroll 1
                 for (int hc = 0; hc < 2; ++hc) {
@@ -555,9 +604,10 @@ ssd_mom_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float y0 = fmaf(qt, __uint_as_float(rv[2 * e]),
-                                              fmaf(et, __uint_as_float(ra[2 * e]), __uint_as_float(rd[2 * e])));
+                                              fmaf(et, __uint_as_float(ra[2 * e]), rf * __uint_as_float(rd[2 * e])));
                         const float y1 = fmaf(qt, __uint_as_float(rv[2 * e + 1]),
-                                              fmaf(et, __uint_as_float(ra[2 * e + 1]), __uint_as_float(rd[2 * e + 1])));
+                                              fmaf(et, __uint_as_float(ra[2 * e + 1]),
+                                                   rf * __uint_as_float(rd[2 * e + 1])));
                         w[e] = pack_bf16x2(y0, y1);
                     }
 #pragma unroll
