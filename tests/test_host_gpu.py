@@ -8,9 +8,8 @@ mm_scan_fwd: final states bit-identical, y within rounding), and match the
 fp64 oracle at the device path's tolerances:
   * scan fp32: max |err| <= 1e-4 max |ref| (y, hT, vT); bf16 y relative L2
     <= 1e-2;
-  * SSD (tensor-core kernel, bf16 operands): y and hT relative L2 <= 1e-2;
-    momentum SSD (CUDA cores): y relative L2 <= 1e-2, fp32 states max |err|
-    <= 1e-4 max |ref|.
+  * SSD and momentum SSD (tensor-core kernels at headdim 64, dstate 128:
+    bf16 operands): y and the states relative L2 <= 1e-2.
 """
 import ctypes
 
@@ -168,8 +167,10 @@ def test_ssd_host_plain_and_momentum():
     y = out["y"].float().numpy()
     rel = np.linalg.norm(y - yr.reshape(y.shape)) / np.linalg.norm(yr)
     assert rel <= BF16_TOL, f"momentum SSD host y relative L2 {rel:.3e}"
-    _max_ok(out["hT"].numpy(), hr.reshape(out["hT"].shape), "momentum SSD host hT")
-    _max_ok(out["vT"].numpy(), vr.reshape(out["vT"].shape), "momentum SSD host vT")
+    for name, ref in (("hT", hr), ("vT", vr)):      # tensor-core form: bf16 state products
+        got = out[name].numpy()
+        rel = np.linalg.norm(got - ref.reshape(got.shape)) / np.linalg.norm(ref)
+        assert rel <= BF16_TOL, f"momentum SSD host {name} relative L2 {rel:.3e}"
 
 
 def test_host_entry_rejects_device_tensors_and_small_workspaces():
