@@ -84,13 +84,16 @@ def measured_traffic(kernel: str, workload: str):
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f).get(kernel)
-        if not rec or rec.get("workload") != workload:
-            return None
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest()[:16] != rec["source_sha256_16"]:
-                return None
-        return float(rec["dram_bytes_per_launch"])
+            recs = json.load(f).get(kernel)
+        recs = recs if isinstance(recs, list) else [recs] if recs else []
+        for rec in recs:
+            if rec.get("workload") != workload:
+                continue
+            with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest()[:16] != rec["source_sha256_16"]:
+                    return None
+            return float(rec["dram_bytes_per_launch"])
+        return None
     except (OSError, ValueError, KeyError):
         return None
 
