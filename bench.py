@@ -30,7 +30,10 @@ workloads.py).
 
 Multi-GPU (launched by torchrun): one process per GPU, each scanning its own
 batch; there is no collective on the data path, only a barrier and a max of
-the per-rank times (weak scaling).
+the per-rank times (weak scaling).  With --split-l the ranks instead share
+one sequence (strong scaling): each scans its piece of the time axis
+(mm_scan_fwd_split_maps), the ranks all-gather their segment-map records
+over NCCL, and each folds them into its piece (mm_scan_fwd_split_correct).
 """
 from __future__ import annotations
 
@@ -593,6 +596,150 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ helpers ------
+def split_seg_len(w: wl.ScanWorkload, world: int, forced: int = 0) -> int:
+    """Segment length of the sequence split over `world` ranks: the
+    sequence-split path's own length for the workload, halved until every
+    rank holds at least eight segments (one round of a full cluster), never
+    below one staged chunk."""
+    import selective_state_space_momentum_b200 as mm
+    if forced:
+        return forced
+    mm.mm_scan_set_path(2, 0)
+    try:
+        S = mm.mm_scan_segment_len(w.batch, w.seqlen, w.dim, w.dstate, 0 if w.io == "f32" else 1)
+    finally:
+        mm.mm_scan_set_path(0, 0)
+    chunk = 32 if w.io == "f32" else 64
+    while S > chunk and -(-w.seqlen // S) < 8 * world:
+        S //= 2
+    return S
+
+
+def run_scan_split(args, w, beta, alpha, rank, world):
+    """One sequence shared by the ranks along time (strong scaling): a step is
+    the split's first launch on every rank's piece, the all-gather of the
+    segment records (NCCL), and the second launch."""
+    import torch
+    import torch.distributed as dist
+    import selective_state_space_momentum_b200 as mm
+    dev = torch.device("cuda", torch.cuda.current_device())
+    S = split_seg_len(w, world, args.seg_len)
+    pieces = mm.split_pieces(w.seqlen, world, S)
+    first, n = pieces[rank]
+    io = mm.MM_F32 if w.io == "f32" else mm.MM_BF16
+    iodt = torch.float32 if w.io == "f32" else torch.bfloat16
+    per = pieces[0][1] // S if world > 1 else -(-w.seqlen // S)
+    rec = mm.mm_scan_split_maps_size(w.batch, n, w.dim, w.dstate, 1, io)
+    # every rank draws the whole sequence from one seed and keeps its piece
+    inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, 0))
+    host = {k: torch.from_numpy(np.ascontiguousarray(v[..., first:first + n]) if k in IO_KEYS else v)
+            for k, v in inp.items()}
+    del inp
+    piece_bytes = algorithmic_bytes(w) * n // w.seqlen
+    nsets = rotating_sets(piece_bytes)
+    sets = []
+    for _ in range(nsets):
+        s = {k: host[k].to(dev).to(iodt if k in IO_KEYS else torch.float32).contiguous() for k in host}
+        s["y"] = torch.empty_like(s["x"])
+        s["hT"] = torch.empty((w.batch, w.dim, w.dstate), device=dev)
+        s["vT"] = torch.empty_like(s["hT"])
+        s["maps"] = torch.empty(per * rec, dtype=torch.uint8, device=dev)
+        s["all"] = torch.empty(world * per * rec, dtype=torch.uint8, device=dev) if world > 1 else s["maps"]
+        sets.append(s)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % nsets]
+        mm.mm_scan_fwd_split_maps(s["x"], s["delta"], s["A"], s["B"], s["C"], beta, alpha, s["y"], s["maps"], S,
+                                  stream)
+        if world > 1:
+            dist.all_gather_into_tensor(s["all"], s["maps"])
+        mm.mm_scan_fwd_split_correct(s["delta"], s["A"], s["C"], None, None, beta, alpha, s["y"], s["hT"],
+                                     s["vT"], s["all"], S, first, w.seqlen, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        ms_timed = timed_ms(step, args.steps, stream, piece_bytes)
+    barrier()
+    torch.cuda.synchronize()
+    ms_step = max_over_ranks(ms_timed, dev) / args.steps
+    updates = w.updates                        # the whole sequence, shared by the ranks
+    value = updates / (ms_step * 1e-3)
+
+    # ---- end to end: the piece from pinned host memory, the results back ----
+    e2e_steps = args.e2e_steps or max(3, min(20, args.steps))
+    pinned = {k: v.to(iodt if k in IO_KEYS else torch.float32).pin_memory() for k, v in host.items()}
+    out = {"y": torch.empty(tuple(pinned["x"].shape), dtype=iodt, pin_memory=True),
+           "hT": torch.empty((w.batch, w.dim, w.dstate), pin_memory=True),
+           "vT": torch.empty((w.batch, w.dim, w.dstate), pin_memory=True)}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for v in out.values())
+
+    def e2e_step():
+        d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        y, hT, vT = mm.scan_fwd_split(d["x"], d["delta"], d["A"], d["B"], d["C"], S, w.seqlen, beta=beta,
+                                      alpha=alpha)
+        out["y"].copy_(y, non_blocking=True)
+        out["hT"].copy_(hT, non_blocking=True)
+        out["vT"].copy_(vT, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    barrier()
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        clocks = clk.summary()
+        sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
+        mufu_peak, mufu_source = mufu_peak_now(sm_max)
+        # the roofline of one rank's share: its exponentials (its piece, once in the
+        # first launch) on its GPU's MUFU pipes
+        share = updates * n / w.seqlen
+        t_mufu = share / mufu_peak
+        roof = {"bound": "alu", "kernel": "scan_seg_kernel", "achieved": share / (ms_step * 1e-3) / 1e9,
+                "peak": mufu_peak / 1e9, "unit": "Gex2/s", "frac": t_mufu / (ms_step * 1e-3),
+                "peak_source": mufu_source, "traffic": None,
+                "note": "rank 0's piece; the step includes the record exchange and the carry-in corrections"}
+        cb = None
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(w, beta, alpha)
+        cfg = scan_config(w, beta, alpha, 1)
+        cfg.update(global_batch=w.batch, parallelism=f"sp{world}", l2=l2_note(piece_bytes, "piece"),
+                   split={"seg_len": S, "pieces": [list(p) for p in pieces], "exchange": "NCCL all-gather"
+                          if world > 1 else "none (one rank)"})
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
+            "config": cfg, "roofline": roof,
+            "e2e": {"value": updates / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+        }
+        if cb is not None:
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def rank_seed(index: int, rank: int) -> int:
     """Each rank draws its own batch (weak scaling): a distinct, fixed seed."""
     return wl.seed_of(index) + 1000 * rank
@@ -946,6 +1093,8 @@ def main(argv=None):
                     help="override the workload's batch (exploration; renames the workload)")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="override the workload's sequence length (scan and SSD workloads)")
+    ap.add_argument("--split-l", action="store_true",
+                    help="scan workloads: the ranks share one sequence, split along time (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1013,6 +1162,13 @@ def main(argv=None):
         torch.cuda.set_device(0)
     if args.backward:
         rc = run_scan_bwd(args, w, beta, alpha, rank, world)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
+    if args.split_l:
+        if args.gated:
+            ap.error("--split-l times the plain forward")
+        rc = run_scan_split(args, w, beta, alpha, rank, world)
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc

@@ -478,7 +478,8 @@ mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_
  * register-resident kernel, 2 the sequence-split kernel (used where it
  * applies: no extras, no checkpoints, dstate <= 16, rows of a whole number of
  * 16-byte pieces) -- and its segment length (0: automatic; else a power of
- * two in [32, 2^30]).  Process-wide, not thread-safe with concurrent calls.
+ * two in [32, 2^30]; bf16 calls use at least 64, one staged chunk of the
+ * kernel).  Process-wide, not thread-safe with concurrent calls.
  * MM_ERR_UNSUPPORTED for other values.
  */
 mm_status mm_scan_set_path(int path, int64_t seg_len);
@@ -493,6 +494,85 @@ mm_status mm_scan_set_path(int path, int64_t seg_len);
  * mm_scan_fwd's size checks; MM_ERR_NULL for a NULL argument.
  */
 mm_status mm_scan_segment_len(const mm_scan_dims *dims, int64_t *seg_len);
+
+/*
+ * The sequence split across devices.  "Forward Pass: Two-Stage Parallel
+ * Scan" of "Momentum Mamba: Enhanced State Space Models with Momentum" joins
+ * chunks of the sequence by their 2x2 affine carry maps; here the chunks are
+ * segments of S steps (S a power of two) and the sequence of seqlen_total
+ * steps is cut into pieces at multiples of S, one per device (rank), every
+ * piece but the last a whole number of segments.  A rank holds its piece --
+ * steps [seq_first, seq_first + seqlen) of every (batch row, channel) in the
+ * usual layouts, with seqlen = dims->seqlen -- and runs:
+ *   1. mm_scan_fwd_split_maps: the main pass of the piece's segments, each
+ *      from a zero state; y gets that zero-start read-out and `maps` one
+ *      record per segment (the lanes' carry maps (beta^S, Q, P, z_v, z_h)
+ *      and whether the segment's delta had no negative value);
+ *   2. an exchange of the records (an all-gather in piece order, by the
+ *      caller: NCCL over NVLink on GPUs), so that one buffer holds the record
+ *      of every segment of the sequence in order;
+ *   3. mm_scan_fwd_split_correct: each segment's carry-in, the fold of all
+ *      earlier segments' maps onto (h0, v0) in order, and its response added
+ *      to y (over the whole segment, or until it has fallen below 2^-25 of
+ *      its start when A <= 0 and delta >= 0); hT, vT = the fold of every
+ *      segment (each rank writes them).
+ * y, hT and vT then equal, bit for bit, one mm_scan_fwd over the whole
+ * sequence on the sequence-split path with the same S
+ * (mm_scan_set_path(2, S)).
+ *
+ * mm_scan_split_maps_size -- *bytes = the size of `segments` records for
+ * dims' (batch, dim).  A piece's buffer holds ceil(seqlen / S) records, the
+ * gathered buffer ceil(seqlen_total / S); record j starts at j times the
+ * size of one.  Errors as mm_scan_fwd's size checks; MM_ERR_DIMS for
+ * segments outside [0, 2^30]; MM_ERR_NULL.
+ */
+mm_status mm_scan_split_maps_size(const mm_scan_dims *dims, int64_t segments, size_t *bytes);
+
+/*
+ * mm_scan_fwd_split_maps -- launch 1 of the split (see above) on `stream`.
+ *   x, delta (batch, dim, seqlen) io; A (dim, dstate) fp32;
+ *   B, C (batch, dstate, seqlen) io: the piece, device memory, read only;
+ *   y    (batch, dim, seqlen) io, written: the zero-start read-out;
+ *   maps device memory of mm_scan_split_maps_size(dims, ceil(seqlen / S))
+ *        bytes, written; the caller owns every buffer.
+ *   seg_len S: a power of two in [32, 2^30] for fp32 I/O, [64, 2^30] for
+ *        bf16 (a segment is a whole number of the kernel's staged chunks).
+ * Errors: MM_ERR_NULL, MM_ERR_DIMS, MM_ERR_DTYPE, MM_ERR_SCALAR as
+ * mm_scan_fwd; MM_ERR_UNSUPPORTED (dstate > 16, S outside its range, rows
+ * of seqlen elements not a whole number of 16-byte pieces); MM_ERR_ALIGN
+ * (a pointer not 16-byte aligned); MM_ERR_ALIAS (y or maps overlapping an
+ * input or each other); MM_ERR_CUDA.  A record is written only by a CTA
+ * that finished its segment: after mm_device_status reports
+ * MM_ERR_DEVICE_TIMEOUT the records are not to be used.
+ */
+mm_status mm_scan_fwd_split_maps(const void *x, const void *delta, const float *A,
+                                 const void *B, const void *C, float beta, float alpha,
+                                 void *y, void *maps, int64_t seg_len,
+                                 const mm_scan_dims *dims, void *stream);
+
+/*
+ * mm_scan_fwd_split_correct -- launch 3 of the split on `stream`.
+ *   delta, A, C   the piece, as for launch 1 (read only);
+ *   h0, v0        (batch, dim, dstate) fp32 state at step 0 of the whole
+ *                 sequence, or NULL for zero;
+ *   y             launch 1's output for this piece, read and updated;
+ *   hT, vT        (batch, dim, dstate) fp32, the states after the last step
+ *                 of the whole sequence, or NULL;
+ *   maps_all      the gathered records of all ceil(seqlen_total / S)
+ *                 segments, device memory, read only;
+ *   seq_first     the piece's first step: a multiple of S;
+ *   seqlen_total  steps of the whole sequence (<= 2^30); a piece that ends
+ *                 before it holds whole segments.
+ * beta, alpha and S as in launch 1.  Errors as launch 1, and
+ * MM_ERR_UNSUPPORTED for a piece outside the sequence or not on segment
+ * boundaries; MM_ERR_ALIAS for y, hT or vT overlapping an input (h0, v0
+ * and maps_all included) or each other.
+ */
+mm_status mm_scan_fwd_split_correct(const void *delta, const float *A, const void *C,
+                                    const float *h0, const float *v0, float beta, float alpha,
+                                    void *y, float *hT, float *vT, const void *maps_all,
+                                    int64_t seg_len, int64_t seq_first, int64_t seqlen_total,
+                                    const mm_scan_dims *dims, void *stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mm_version(void);

@@ -15,6 +15,9 @@ Convenience wrappers allocate outputs:
 * :func:`ssd_fwd` -- ``(y, last_state)`` of the multi-head scalar-A form.
 * :func:`scan_fwd_host` -- end-to-end call on host arrays (copies in, scan,
   copies out) for callers whose data lives in host memory.
+* :func:`scan_fwd_split` -- one sequence cut into pieces over the ranks of a
+  process group: each rank scans its piece, the ranks exchange their segment
+  maps (all-gather), and each folds them into its piece's carry-in.
 """
 from __future__ import annotations
 
@@ -30,8 +33,9 @@ __all__ = [
     "mm_scan_set_path", "mm_scan_segment_len",
     "mm_scan_fwd_host", "mm_scan_fwd_host_workspace_size", "mm_ssd_fwd_host",
     "mm_ssd_fwd_host_workspace_size",
+    "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
     "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
-    "ssd_fwd_host",
+    "ssd_fwd_host", "split_pieces", "scan_fwd_split",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
 ]
 
@@ -58,7 +62,8 @@ EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
                     "mm_scan_set_path", "mm_scan_segment_len",
                     "mm_scan_fwd_host_workspace_size", "mm_scan_fwd_host",
-                    "mm_ssd_fwd_host_workspace_size", "mm_ssd_fwd_host")
+                    "mm_ssd_fwd_host_workspace_size", "mm_ssd_fwd_host",
+                    "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct")
 
 
 class MMError(RuntimeError):
@@ -123,6 +128,13 @@ def _declare(lib):
     lib.mm_ssd_fwd_host.restype = ctypes.c_int
     lib.mm_ssd_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp, sz, i64,
                                     ctypes.POINTER(SSDDims), vp]
+    lib.mm_scan_split_maps_size.restype = ctypes.c_int
+    lib.mm_scan_split_maps_size.argtypes = [ctypes.POINTER(ScanDims), i64, ctypes.POINTER(sz)]
+    lib.mm_scan_fwd_split_maps.restype = ctypes.c_int
+    lib.mm_scan_fwd_split_maps.argtypes = [vp, vp, vp, vp, vp, f, f, vp, vp, i64, ctypes.POINTER(ScanDims), vp]
+    lib.mm_scan_fwd_split_correct.restype = ctypes.c_int
+    lib.mm_scan_fwd_split_correct.argtypes = [vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp, i64, i64, i64,
+                                              ctypes.POINTER(ScanDims), vp]
     lib.mm_status_string.restype = ctypes.c_char_p
     lib.mm_status_string.argtypes = [ctypes.c_int]
     lib.mm_last_error.restype = ctypes.c_char_p
@@ -477,6 +489,66 @@ def mm_scan_segment_len(batch, seqlen, dim, dstate, io=MM_F32) -> int:
     return int(out.value)
 
 
+def mm_scan_split_maps_size(batch, seqlen, dim, dstate, segments, io=MM_F32) -> int:
+    """C entry point mm_scan_split_maps_size: bytes of `segments` segment-map
+    records of a split scan over (batch, dim)."""
+    dims = ScanDims(batch, seqlen, dim, dstate, io)
+    out = ctypes.c_size_t(0)
+    _check(load_library().mm_scan_split_maps_size(ctypes.byref(dims), int(segments), ctypes.byref(out)),
+           "mm_scan_split_maps_size")
+    return int(out.value)
+
+
+def _require_maps(name, maps, nbytes, device):
+    import torch
+    if not isinstance(maps, torch.Tensor) or maps.dtype != torch.uint8 or not maps.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous uint8 tensor")
+    if maps.device != device:
+        raise ValueError(f"{name} is on {maps.device}, x on {device}")
+    if maps.numel() < nbytes:
+        raise ValueError(f"{name} holds {maps.numel()} bytes; the call needs {nbytes}")
+
+
+def mm_scan_fwd_split_maps(x, delta, A, B, C, beta, alpha, y, maps, seg_len, stream=None):
+    """C entry point mm_scan_fwd_split_maps (marshalling only): the main pass
+    of this rank's piece x, delta, B, C (shapes as mm_scan_fwd); y gets the
+    zero-start read-out, `maps` (uint8, at least mm_scan_split_maps_size(...,
+    ceil(L / seg_len)) bytes) the piece's segment records."""
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("y", y, "io", False)])
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    if seg_len >= 1:
+        need = mm_scan_split_maps_size(batch, L, dim, N, -(-L // int(seg_len)), dims.io)
+        _require_maps("maps", maps, need, x.device)
+    rc = load_library().mm_scan_fwd_split_maps(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), float(beta),
+                                               float(alpha), _ptr(y), _ptr(maps), int(seg_len),
+                                               ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_fwd_split_maps")
+
+
+def mm_scan_fwd_split_correct(delta, A, C, h0, v0, beta, alpha, y, hT, vT, maps_all, seg_len, seq_first,
+                              seqlen_total, stream=None):
+    """C entry point mm_scan_fwd_split_correct (marshalling only): fold the
+    whole sequence's records `maps_all` into this piece's carry-ins, add their
+    response to y (mm_scan_fwd_split_maps' output) and write the final
+    states of the whole sequence to hT, vT (or None)."""
+    _require_scan(delta, A, [("C", C, "io_bc", False), ("h0", h0, "state", True), ("v0", v0, "state", True),
+                             ("y", y, "io", False), ("hT", hT, "state", True), ("vT", vT, "state", True)])
+    batch, dim, L = delta.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(delta.dtype))
+    if seg_len >= 1:
+        need = mm_scan_split_maps_size(batch, L, dim, N, -(-int(seqlen_total) // int(seg_len)), dims.io)
+        _require_maps("maps_all", maps_all, need, delta.device)
+    rc = load_library().mm_scan_fwd_split_correct(_ptr(delta), _ptr(A), _ptr(C), _ptr(h0), _ptr(v0),
+                                                  float(beta), float(alpha), _ptr(y), _ptr(hT), _ptr(vT),
+                                                  _ptr(maps_all), int(seg_len), int(seq_first),
+                                                  int(seqlen_total), ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_fwd_split_correct")
+
+
 def mm_version() -> int:
     return int(load_library().mm_version())
 
@@ -690,3 +762,85 @@ def ssd_fwd_host(x, delta, A, B, C, h0=None, v0=None, beta=0.0, alpha=1.0, chunk
                         workspace, chunk, chunk_steps, s)
         s.synchronize()
     return out
+
+
+# ------------------------------------------------- sequence split ---------
+def split_pieces(seqlen_total: int, world: int, seg_len: int):
+    """The pieces of a sequence of ``seqlen_total`` steps over ``world`` ranks:
+    a list of (first step, steps), rank order.  Every piece but the last holds
+    the same whole number of segments of ``seg_len`` steps; the last holds
+    the rest.  Raises ValueError when a rank would get no step."""
+    if seqlen_total < 1 or world < 1 or seg_len < 1:
+        raise ValueError("seqlen_total, world and seg_len must be >= 1")
+    nseg = -(-seqlen_total // seg_len)
+    per = -(-nseg // world)
+    pieces = []
+    for r in range(world):
+        lo = min(r * per * seg_len, seqlen_total)
+        hi = min((r + 1) * per * seg_len, seqlen_total)
+        if hi <= lo:
+            raise ValueError(f"{seqlen_total} steps in segments of {seg_len} leave rank {r} of {world} "
+                             "without a piece")
+        pieces.append((lo, hi - lo))
+    return pieces
+
+
+def _all_gather_bytes(local, world, group):
+    """Concatenate every rank's byte buffer in rank order.  NCCL gathers in
+    device memory; a backend without CUDA support (gloo) goes through host
+    memory."""
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return local
+    out = torch.empty(world * local.numel(), dtype=torch.uint8, device=local.device)
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(out, local, group=group)
+        return out
+    parts = [torch.empty(local.numel(), dtype=torch.uint8) for _ in range(world)]
+    dist.all_gather(parts, local.cpu(), group=group)
+    out.copy_(torch.cat(parts))
+    return out
+
+
+def scan_fwd_split(x, delta, A, B, C, seg_len, seqlen_total, h0=None, v0=None, beta=0.9, alpha=1.0,
+                   group=None, stream=None):
+    """This rank's part of one scan whose sequence is cut over the ranks of
+    ``group`` (a torch.distributed process group; None: the default group,
+    or a single rank without one).  x, delta, B, C are this rank's piece,
+    ``split_pieces(seqlen_total, world, seg_len)[rank]``; h0, v0 the state
+    at step 0 of the whole sequence.  Returns (y of the piece, hT, vT of the
+    whole sequence), equal bit for bit to one mm_scan_fwd over the whole
+    sequence on the sequence-split path with segment length ``seg_len``."""
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        rank, world = dist.get_rank(group), dist.get_world_size(group)
+    else:
+        rank, world = 0, 1
+    first, steps = split_pieces(int(seqlen_total), world, int(seg_len))[rank]
+    if x.dim() != 3 or x.shape[2] != steps:
+        raise ValueError(f"rank {rank} holds steps [{first}, {first + steps}): x must be (batch, dim, {steps})")
+    batch, dim, _ = x.shape
+    N = A.shape[1]
+    io = _io_code(x.dtype)
+    per = split_pieces(int(seqlen_total), world, int(seg_len))[0][1] // int(seg_len) if world > 1 else \
+        -(-steps // int(seg_len))
+    rec = mm_scan_split_maps_size(batch, steps, dim, N, 1, io)
+    local = torch.empty(per * rec, dtype=torch.uint8, device=x.device)
+    y = torch.empty_like(x)
+    mm_scan_fwd_split_maps(x, delta, A, B, C, beta, alpha, y, local, seg_len, stream)
+    if world > 1:
+        # the collective runs on torch's current stream: order it after the launch
+        if stream is not None:
+            torch.cuda.current_stream(x.device).wait_stream(stream)
+        gathered = _all_gather_bytes(local, world, group)
+        if stream is not None:
+            stream.wait_stream(torch.cuda.current_stream(x.device))
+    else:
+        gathered = local
+    hT = torch.empty((batch, dim, N), device=x.device, dtype=torch.float32)
+    vT = torch.empty_like(hT)
+    mm_scan_fwd_split_correct(delta, A, C, h0, v0, beta, alpha, y, hT, vT, gathered, seg_len, first,
+                              seqlen_total, stream)
+    return y, hT, vT

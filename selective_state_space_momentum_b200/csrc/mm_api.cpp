@@ -59,7 +59,10 @@ int64_t seg_len_for(int64_t batch, int64_t L, int64_t dim, int64_t dstate, int i
     if (path == 1) return 0;
     if (path == 0 && !seg_auto(batch, dim, dstate, io)) return 0;
     const int64_t forced = g_forced_seg_len.load();
-    const int64_t S = forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
+    int64_t S = forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
+    // a segment is a whole number of staged chunks (64 steps for bf16)
+    const int64_t chunk = mmscan::scan_seg_chunk_steps(io == MM_F32 ? 0 : 1);
+    if (S < chunk) S = chunk;
     if (path == 0 && L <= S) return 0;
     return S;
 }
@@ -169,6 +172,39 @@ mm_status check_scan_dims(const mm_scan_dims* dims, float beta, float alpha, Sca
     return MM_OK;
 }
 
+// Bytes of `segments` segment records of a split scan over (batch, dim);
+// false when the count overflows 64 bits.
+bool split_record_bytes(int64_t batch, int64_t dim, int64_t segments, int64_t* out) {
+    const int64_t ch = mmscan::scan_seg_tile_channels();
+    const int64_t tiles = dim / ch + (dim % ch != 0);
+    int64_t per_seg = 0;
+    return mul_ok(batch, tiles, &per_seg) && mul_ok(per_seg, mmscan::scan_seg_tile_record_bytes(), &per_seg) &&
+           mul_ok(per_seg, segments, out);
+}
+
+// The checks the two launches of a split scan share: the segment length, the
+// row rule of the tiled copies, and the piece's place in the whole sequence.
+mm_status check_split(const mm_scan_dims* dims, const ScanSizes& zs, int64_t seg_len, int64_t seq_first,
+                      int64_t seqlen_total) {
+    const int64_t chunk = mmscan::scan_seg_chunk_steps(dims->io == MM_F32 ? 0 : 1);
+    if (seg_len < chunk || seg_len > kMaxSeqlen || (seg_len & (seg_len - 1)) != 0)
+        return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not a power of two in [%lld, 2^30]",
+                    (long long)seg_len, (long long)chunk);
+    if ((dims->seqlen * zs.esize) % 16 != 0)
+        return fail(MM_ERR_UNSUPPORTED, "rows of seqlen=%lld elements are not a whole number of 16-byte pieces",
+                    (long long)dims->seqlen);
+    if (seqlen_total < 1 || seqlen_total > kMaxSeqlen)
+        return fail(MM_ERR_UNSUPPORTED, "seqlen_total=%lld is outside [1, 2^30]", (long long)seqlen_total);
+    if (seq_first < 0 || seq_first % seg_len != 0 || seq_first + dims->seqlen > seqlen_total)
+        return fail(MM_ERR_UNSUPPORTED, "piece [%lld, %lld) does not start at a multiple of %lld within %lld steps",
+                    (long long)seq_first, (long long)(seq_first + dims->seqlen), (long long)seg_len,
+                    (long long)seqlen_total);
+    if (seq_first + dims->seqlen < seqlen_total && dims->seqlen % seg_len != 0)
+        return fail(MM_ERR_UNSUPPORTED, "a piece before the last must hold whole segments (seqlen=%lld, S=%lld)",
+                    (long long)dims->seqlen, (long long)seg_len);
+    return MM_OK;
+}
+
 }  // namespace
 
 namespace mmscan {
@@ -255,6 +291,96 @@ mm_status mm_scan_segment_len(const mm_scan_dims* dims, int64_t* seg_len) {
     *seg_len = seg_len_for(dims->batch, dims->seqlen, dims->dim, dims->dstate, dims->io,
                            ((dims->seqlen * zs.esize) % 16) == 0);
     return ok();
+}
+
+mm_status mm_scan_split_maps_size(const mm_scan_dims* dims, int64_t segments, size_t* bytes) {
+    if (!dims || !bytes) return fail(MM_ERR_NULL, "dims and bytes are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, 0.0f, 1.0f, &zs)) return st;
+    if (segments < 0 || segments > kMaxSeqlen)
+        return fail(MM_ERR_DIMS, "segments=%lld is outside [0, 2^30]", (long long)segments);
+    int64_t total = 0;
+    if (!split_record_bytes(dims->batch, dims->dim, segments, &total))
+        return fail(MM_ERR_DIMS, "record bytes overflow 64 bits");
+    *bytes = static_cast<size_t>(total);
+    return ok();
+}
+
+mm_status mm_scan_fwd_split_maps(const void* x, const void* delta, const float* A, const void* B,
+                                 const void* C, float beta, float alpha, void* y, void* maps,
+                                 int64_t seg_len, const mm_scan_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !y || !maps)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C, y and maps are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
+    // a piece is checked as the last one of a sequence that ends with it
+    if (mm_status st = check_split(dims, zs, seg_len, 0, dims->seqlen)) return st;
+    const void* ptrs[] = {x, delta, A, B, C, y, maps};
+    const char* names[] = {"x", "delta", "A", "B", "C", "y", "maps"};
+    for (int i = 0; i < 7; ++i)
+        if (!aligned16(ptrs[i])) return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    int64_t maps_bytes = 0;
+    if (!split_record_bytes(dims->batch, dims->dim, (dims->seqlen + seg_len - 1) / seg_len, &maps_bytes))
+        return fail(MM_ERR_DIMS, "record bytes overflow 64 bits");
+    const Range ry = rng("y", y, zs.seq_bytes), rm = rng("maps", maps, maps_bytes);
+    const Range ins[] = {rng("x", x, zs.seq_bytes), rng("delta", delta, zs.seq_bytes), rng("A", A, zs.a_bytes),
+                         rng("B", B, zs.bc_bytes), rng("C", C, zs.bc_bytes)};
+    for (const Range& in : ins) {
+        if (overlap(ry, in)) return fail(MM_ERR_ALIAS, "y overlaps %s", in.name);
+        if (overlap(rm, in)) return fail(MM_ERR_ALIAS, "maps overlaps %s", in.name);
+    }
+    if (overlap(rm, ry)) return fail(MM_ERR_ALIAS, "maps overlaps y");
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+    mmscan::ScanArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.y = y;
+    a.batch = dims->batch; a.seqlen = dims->seqlen; a.dim = dims->dim; a.dstate = (int)dims->dstate;
+    a.beta = beta; a.alpha = alpha;
+    a.vec_ok = 1;
+    a.stall = inject_stall();
+    return from_cuda(mmscan::launch_scan_seg_split(a, dims->io, seg_len, 1, maps, 0, dims->seqlen,
+                                                   static_cast<cudaStream_t>(stream)),
+                     "mm_scan_fwd_split_maps launch");
+}
+
+mm_status mm_scan_fwd_split_correct(const void* delta, const float* A, const void* C, const float* h0,
+                                    const float* v0, float beta, float alpha, void* y, float* hT, float* vT,
+                                    const void* maps_all, int64_t seg_len, int64_t seq_first,
+                                    int64_t seqlen_total, const mm_scan_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!delta || !A || !C || !y || !maps_all)
+        return fail(MM_ERR_NULL, "delta, A, C, y and maps_all are required");
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
+    if (mm_status st = check_split(dims, zs, seg_len, seq_first, seqlen_total)) return st;
+    const void* ptrs[] = {delta, A, C, h0, v0, y, hT, vT, maps_all};
+    const char* names[] = {"delta", "A", "C", "h0", "v0", "y", "hT", "vT", "maps_all"};
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    int64_t maps_bytes = 0;
+    if (!split_record_bytes(dims->batch, dims->dim, (seqlen_total + seg_len - 1) / seg_len, &maps_bytes))
+        return fail(MM_ERR_DIMS, "record bytes overflow 64 bits");
+    const Range ry = rng("y", y, zs.seq_bytes), rhT = rng("hT", hT, zs.st_bytes), rvT = rng("vT", vT, zs.st_bytes);
+    const Range ins[] = {rng("delta", delta, zs.seq_bytes), rng("A", A, zs.a_bytes), rng("C", C, zs.bc_bytes),
+                         rng("h0", h0, zs.st_bytes), rng("v0", v0, zs.st_bytes),
+                         rng("maps_all", maps_all, maps_bytes)};
+    for (const Range* out : {&ry, &rhT, &rvT})
+        for (const Range& in : ins)
+            if (overlap(*out, in)) return fail(MM_ERR_ALIAS, "%s overlaps %s", out->name, in.name);
+    if (overlap(rhT, ry) || overlap(rvT, ry) || overlap(rhT, rvT))
+        return fail(MM_ERR_ALIAS, "hT, vT and y overlap");
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+    mmscan::ScanArgs a{};
+    a.x = nullptr; a.delta = delta; a.A = A; a.B = nullptr; a.C = C; a.h0 = h0; a.v0 = v0;
+    a.y = y; a.hT = hT; a.vT = vT;
+    a.batch = dims->batch; a.seqlen = dims->seqlen; a.dim = dims->dim; a.dstate = (int)dims->dstate;
+    a.beta = beta; a.alpha = alpha;
+    a.vec_ok = 1;
+    a.stall = inject_stall();
+    return from_cuda(mmscan::launch_scan_seg_split(a, dims->io, seg_len, 2, const_cast<void*>(maps_all),
+                                                   seq_first / seg_len, seqlen_total,
+                                                   static_cast<cudaStream_t>(stream)),
+                     "mm_scan_fwd_split_correct launch");
 }
 
 mm_status mm_scan_fwd(const void* x, const void* delta, const float* A, const void* B,

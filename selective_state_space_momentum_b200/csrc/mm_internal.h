@@ -118,6 +118,18 @@ constexpr int kSegMaxCluster = 8;
 constexpr int64_t kSegMinLen = 16384;
 int64_t scan_seg_default_len(int64_t batch, int64_t dim);
 cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s);
+// Steps of one staged chunk of the sequence-split kernel (32 fp32, 64 bf16).
+int64_t scan_seg_chunk_steps(int io);
+// The sequence split over several calls: the channels of one CTA's tile and
+// the bytes of one tile's record of one segment (a segment's records: one
+// per (batch row, channel tile), in that order), and the two launches --
+// mode 1 the main pass with the maps to `maps`, mode 2 the fold of the whole
+// sequence's maps and the correction (seg_first: global index of the call's
+// first segment).
+int64_t scan_seg_tile_channels();
+int64_t scan_seg_tile_record_bytes();
+cudaError_t launch_scan_seg_split(const ScanArgs& a, int io, int64_t seg_len, int mode, void* maps,
+                                  int64_t seg_first, int64_t seqlen_total, cudaStream_t s);
 unsigned int scan_seg_read_and_clear_device_error();
 
 bool scan_tile_supported(int spt, int warps, int time_lanes);

@@ -135,6 +135,25 @@ __device__ __forceinline__ float pow_steps(float beta, int64_t n) {
     return r;
 }
 
+// The sequence split over several calls (ranks), in two launches around an
+// exchange of segment maps:
+//   MODE 1: the main pass of this call's segments only; y gets the zero-start
+//     read-out and each segment's map goes to `maps` (record k for the call's
+//     segment k) instead of being folded;
+//   MODE 2: with the maps of every segment of the whole sequence (all calls'
+//     records in segment order), fold segments 0 .. K-1 onto (h0, v0) for this
+//     call's segment K (global index seg_first + k), add the response to y,
+//     and write hT, vT as the fold of all nseg_total segments.
+// A record holds, per (batch row, channel tile) cluster, the 8 float4 maps of
+// each of the NT lanes and one float4 whose x is 1 when the segment's delta
+// had no negative value; MODE 0 is the fused kernel above.
+struct SegSplit {
+    float4* maps;             // MODE 1: this call's records; MODE 2: every segment's records (read only)
+    int64_t seg_first;        // MODE 2: global index of this call's first segment
+    int64_t nseg_total;       // MODE 2: segments of the whole sequence
+    int64_t L_total;          // MODE 2: steps of the whole sequence
+};
+
 // Scaled form (SC, used for beta >= 1/2).  Within a chunk of T steps the
 // states are carried as v~ = v / beta^(tau+1), h~ = h / beta^(tau+1) (tau the
 // step within the chunk), which turns the two recurrences into
@@ -145,11 +164,11 @@ __device__ __forceinline__ float pow_steps(float beta, int64_t n) {
 // for the velocity instead of a multiply and an FMA.  At the end of the chunk
 // the states are multiplied back by beta^T.  The factors stay within 2^+-32
 // (2^+-64 for bf16 chunks of 64 steps) for beta >= 1/2.
-template <typename IO, int W, int ST, bool SC>
+template <typename IO, int W, int ST, bool SC, int MODE>
 __global__ void __launch_bounds__(W * 32)
 scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
-                const ScanArgs p, const int64_t seg_len, const int csize) {
+                const ScanArgs p, const int64_t seg_len, const int csize, const SegSplit sp) {
     using TL = SegTile<IO, W, ST>;
     constexpr int NT = TL::NT, T = TL::T, CH = TL::CH, EB = TL::EB, G = TL::G;
 
@@ -179,6 +198,9 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const float beta = p.beta;
     const int64_t nseg = (L + seg_len - 1) / seg_len;
     const int64_t rounds = (nseg + csize - 1) / csize;
+    // records of the split launches: (segment, cluster) -> 8 * NT + 1 float4
+    const int64_t ncl = (int64_t)gridDim.x / csize;
+    constexpr int REC = 8 * NT + 1;
 
     if (tid == 0) {
         for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, 1u);
@@ -581,6 +603,50 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
     };
 
+    // One segment map (zv, zh | Q, P of the lane's two states c, 2q .. 2q+1)
+    // applied to a concrete carry (v, h): the same operations in every mode, so
+    // that the split launches reproduce the fused kernel bit for bit.
+    auto apply_map = [&](float (&cv)[2][4], float (&ch)[2][4], float4 zvh, float4 qp, int c, int q, float bS) {
+        const float zv[2] = {zvh.x, zvh.y}, zh[2] = {zvh.z, zvh.w};
+        const float Qm[2] = {qp.x, qp.y}, Pm[2] = {qp.z, qp.w};
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+            const int e = 2 * q + e2;
+            const float hn = fmaf(Pm[e2], ch[c][e], fmaf(Qm[e2], cv[c][e], zh[e2]));
+            cv[c][e] = fmaf(bS, cv[c][e], zv[e2]);
+            ch[c][e] = hn;
+        }
+    };
+    // Split launches: the records of segments 0 .. nfold-1 of the whole sequence
+    // folded in order onto the carry; each record is read one segment ahead.
+    auto fold_records = [&](float (&cv)[2][4], float (&ch)[2][4], int64_t nfold) {
+        const float4* rec0 = sp.maps + (int64_t)(blockIdx.x / csize) * REC + tid;
+        const int64_t seg_stride = ncl * REC;
+        float4 cur[8], nxt[8];
+        if (nfold > 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cur[i] = rec0[i * NT];
+        }
+        for (int64_t j = 0; j < nfold; ++j) {
+            if (j + 1 < nfold) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) nxt[i] = rec0[(j + 1) * seg_stride + i * NT];
+            }
+            const int64_t sj = j * seg_len;
+            const int64_t lj = sp.L_total - sj < seg_len ? sp.L_total - sj : seg_len;
+            const float bS = pow_steps(beta, lj);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int i0 = (c * 2 + q) * 2;
+                    apply_map(cv, ch, cur[i0], cur[i0 + 1], c, q, bS);
+                }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+        }
+    };
+
     for (int64_t r = 0; r < rounds; ++r) {
         const int64_t k = r * csize + rank;                       // this CTA's segment
         const int64_t s0 = k * seg_len;
@@ -595,7 +661,7 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         bp2 = SC ? f2(1.0f, 1.0f) : beta2;
         dpart = 0.0f;
         dbits = 0;
-        if (!dead && nch > 0) {
+        if (MODE != 2 && !dead && nch > 0) {
             for (int64_t j = 0; j < ST && j < nch; ++j) issue(s0 + j * T, true);
             for (int64_t kc = 0; kc < nch; ++kc) {
                 const unsigned char* sbuf = wait_next();
@@ -614,25 +680,45 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
 
         // ================= publish this segment's map; fold the carries ===========
-        const bool seg_nonneg = __syncthreads_and((dbits & 0x80000000u) == 0u) != 0;
+        bool seg_nonneg = __syncthreads_and((dbits & 0x80000000u) == 0u) != 0;
         // the channel's delta sum: its two threads' halves, then to the pair's lanes
         const float dch_sum = dpart + __shfl_xor_sync(0xffffffffu, dpart, 1);
         float dsum[2];
 #pragma unroll
         for (int c = 0; c < 2; ++c) dsum[c] = __shfl_sync(0xffffffffu, dch_sum, 2 * (lch[c] & 15));
-        if (!dead) {
+        if constexpr (MODE == 1) {
+            // the split's first launch: this segment's map and delta-sign flag to its record
+            if (!dead && slen > 0) {
+                float4* rec = sp.maps + (k * ncl + (int64_t)(blockIdx.x / csize)) * REC;
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const float P0 = ex2_approx(Al[c][2 * q] * dsum[c]);
-                    const float P1 = ex2_approx(Al[c][2 * q + 1] * dsum[c]);
-                    const int i0 = (c * 2 + q) * 2;
-                    agg[i0 * NT + tid] = make_float4(vv[c][q].x, vv[c][q].y, hh[c][q].x, hh[c][q].y);
-                    agg[(i0 + 1) * NT + tid] = make_float4(qq[c][q].x, qq[c][q].y, P0, P1);
-                }
+                    for (int q = 0; q < 2; ++q) {
+                        const float P0 = ex2_approx(Al[c][2 * q] * dsum[c]);
+                        const float P1 = ex2_approx(Al[c][2 * q + 1] * dsum[c]);
+                        const int i0 = (c * 2 + q) * 2;
+                        rec[i0 * NT + tid] = make_float4(vv[c][q].x, vv[c][q].y, hh[c][q].x, hh[c][q].y);
+                        rec[(i0 + 1) * NT + tid] = make_float4(qq[c][q].x, qq[c][q].y, P0, P1);
+                    }
+                if (tid == 0) rec[8 * NT] = make_float4(seg_nonneg ? 1.0f : 0.0f, 0.0f, 0.0f, 0.0f);
+            }
+            continue;                     // no fold and no correction in this launch
         }
-        cluster_sync_all();               // every segment's map is published
+        if constexpr (MODE == 0) {
+            if (!dead) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const float P0 = ex2_approx(Al[c][2 * q] * dsum[c]);
+                        const float P1 = ex2_approx(Al[c][2 * q + 1] * dsum[c]);
+                        const int i0 = (c * 2 + q) * 2;
+                        agg[i0 * NT + tid] = make_float4(vv[c][q].x, vv[c][q].y, hh[c][q].x, hh[c][q].y);
+                        agg[(i0 + 1) * NT + tid] = make_float4(qq[c][q].x, qq[c][q].y, P0, P1);
+                    }
+            }
+            cluster_sync_all();           // every segment's map is published
+        }
         float cv[2][4], ch[2][4];         // the concrete carry, folded segment by segment
 #pragma unroll
         for (int c = 0; c < 2; ++c)
@@ -643,7 +729,19 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int e = 0; e < 4; ++e) { rv[c][e] = 0.0f; rh[c][e] = 0.0f; }
-        for (int jr = 0; jr < csize; ++jr) {
+        if constexpr (MODE == 2) {
+            // the carry-in of global segment kg: every earlier segment's map, in order, onto (h0, v0)
+            const int64_t kg = sp.seg_first + k;
+            if (!dead && slen > 0) {
+                fold_records(cv, ch, kg);
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { rv[c][e] = cv[c][e]; rh[c][e] = ch[c][e]; }
+                seg_nonneg = sp.maps[(kg * ncl + (int64_t)(blockIdx.x / csize)) * REC + 8 * NT].x != 0.0f;
+            }
+        }
+        for (int jr = 0; MODE == 0 && jr < csize; ++jr) {
             if (jr == rank) {
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
@@ -661,24 +759,17 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int i0 = (c * 2 + q) * 2;
-                    const float4 zvh = dsmem_ld4(ra + (uint32_t)((i0 * NT + tid) * 16));
-                    const float4 qp = dsmem_ld4(ra + (uint32_t)(((i0 + 1) * NT + tid) * 16));
-                    const float zv[2] = {zvh.x, zvh.y}, zh[2] = {zvh.z, zvh.w};
-                    const float Qm[2] = {qp.x, qp.y}, Pm[2] = {qp.z, qp.w};
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const int e = 2 * q + e2;
-                        const float hn = fmaf(Pm[e2], ch[c][e], fmaf(Qm[e2], cv[c][e], zh[e2]));
-                        cv[c][e] = fmaf(bS, cv[c][e], zv[e2]);
-                        ch[c][e] = hn;
-                    }
+                    apply_map(cv, ch, dsmem_ld4(ra + (uint32_t)((i0 * NT + tid) * 16)),
+                              dsmem_ld4(ra + (uint32_t)(((i0 + 1) * NT + tid) * 16)), c, q, bS);
                 }
         }
-        cluster_sync_all();               // every CTA has read the maps: the area is free again
+        if constexpr (MODE == 0) {
+            cluster_sync_all();           // every CTA has read the maps: the area is free again
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) { carry_at(c, e, 0) = cv[c][e]; carry_at(c, e, 1) = ch[c][e]; }
+                for (int e = 0; e < 4; ++e) { carry_at(c, e, 0) = cv[c][e]; carry_at(c, e, 1) = ch[c][e]; }
+        }
 
         // ================= correction: the response to the carry-in ==============
         bool any = false;
@@ -729,7 +820,22 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
 
     // ---- final states: the carry after the last segment -----------------------
-    if (rank == 0 && !dead) {
+    if constexpr (MODE == 2) {
+        // every segment of the whole sequence folded onto (h0, v0), as above
+        if (rank == 0 && !dead) {
+            float cv[2][4], ch[2][4];
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { cv[c][e] = carry_at(c, e, 0); ch[c][e] = carry_at(c, e, 1); }
+            fold_records(cv, ch, sp.nseg_total);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { carry_at(c, e, 0) = cv[c][e]; carry_at(c, e, 1) = ch[c][e]; }
+        }
+    }
+    if (MODE != 1 && rank == 0 && !dead) {
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -750,8 +856,8 @@ namespace {
 constexpr int kSegWarps = 1;
 constexpr int kSegStages = 2;
 
-template <typename IO, bool SC>
-cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream) {
+template <typename IO, bool SC, int MODE>
+cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, cudaStream_t stream) {
     using TL = SegTile<IO, kSegWarps, kSegStages>;
     ScanArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
@@ -763,11 +869,15 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream)
     const bool bf = sizeof(IO) == 2;
     const uint64_t L = (uint64_t)a.seqlen;
     cudaError_t e;
-    if ((e = make_map_3d(&mx, a.x, bf, L, a.dim, a.batch, TL::T, TL::CH)) != cudaSuccess) return e;
+    // (the correction launch of a split reads no x and no B: its maps for them
+    // describe delta and C and are never used)
+    const void* xs = MODE == 2 ? a.delta : a.x;
+    const void* Bs = MODE == 2 ? a.C : a.B;
+    if ((e = make_map_3d(&mx, xs, bf, L, a.dim, a.batch, TL::T, TL::CH)) != cudaSuccess) return e;
     if ((e = make_map_3d(&md, a.delta, bf, L, a.dim, a.batch, TL::T, TL::CH)) != cudaSuccess) return e;
-    if ((e = make_map_3d(&mB, a.B, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
+    if ((e = make_map_3d(&mB, Bs, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
     if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
-    auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages, SC>;
+    auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages, SC, MODE>;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -795,7 +905,16 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, cudaStream_t stream)
     attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize);
+    return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize, sp);
+}
+
+template <int MODE>
+cudaError_t launch_seg_mode(const ScanArgs& a, int io, int64_t seg_len, const SegSplit& sp, cudaStream_t s) {
+    // The scaled form needs beta^-T within range: beta >= 1/2 (see the kernel).
+    const bool scaled = a.beta >= 0.5f;
+    if (io == 0)
+        return scaled ? launch_seg<float, true, MODE>(a, seg_len, sp, s) : launch_seg<float, false, MODE>(a, seg_len, sp, s);
+    return scaled ? launch_seg<bf16, true, MODE>(a, seg_len, sp, s) : launch_seg<bf16, false, MODE>(a, seg_len, sp, s);
 }
 
 }  // namespace
@@ -812,10 +931,32 @@ int64_t scan_seg_default_len(int64_t batch, int64_t dim) {
 }
 
 cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s) {
-    // The scaled form needs beta^-T within range: beta >= 1/2 (see the kernel).
-    const bool scaled = a.beta >= 0.5f;
-    if (io == 0) return scaled ? launch_seg<float, true>(a, seg_len, s) : launch_seg<float, false>(a, seg_len, s);
-    return scaled ? launch_seg<bf16, true>(a, seg_len, s) : launch_seg<bf16, false>(a, seg_len, s);
+    return launch_seg_mode<0>(a, io, seg_len, SegSplit{}, s);
+}
+
+int64_t scan_seg_chunk_steps(int io) {
+    return io == 0 ? SegTile<float, kSegWarps, kSegStages>::T : SegTile<bf16, kSegWarps, kSegStages>::T;
+}
+
+int64_t scan_seg_tile_channels() { return SegTile<float, kSegWarps, kSegStages>::CH; }
+
+int64_t scan_seg_tile_record_bytes() {
+    using TL = SegTile<float, kSegWarps, kSegStages>;
+    static_assert(SegTile<bf16, kSegWarps, kSegStages>::CH == TL::CH && SegTile<bf16, kSegWarps, kSegStages>::NT == TL::NT,
+                  "one record layout for both element types");
+    return (int64_t)(8 * TL::NT + 1) * 16;
+}
+
+cudaError_t launch_scan_seg_split(const ScanArgs& a, int io, int64_t seg_len, int mode, void* maps,
+                                  int64_t seg_first, int64_t seqlen_total, cudaStream_t s) {
+    SegSplit sp{};
+    sp.maps = static_cast<float4*>(maps);
+    sp.seg_first = seg_first;
+    sp.L_total = seqlen_total;
+    sp.nseg_total = (seqlen_total + seg_len - 1) / seg_len;
+    if (mode == 1) return launch_seg_mode<1>(a, io, seg_len, sp, s);
+    if (mode == 2) return launch_seg_mode<2>(a, io, seg_len, sp, s);
+    return cudaErrorInvalidValue;
 }
 
 unsigned int scan_seg_read_and_clear_device_error() {

@@ -43,6 +43,13 @@ cudaError_t launch_ssd_fwd(const SSDArgs&, cudaStream_t) { ++g_launches; return 
 cudaError_t launch_ssd_mom(const SSDMomArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
 int64_t scan_seg_default_len(int64_t, int64_t) { return 16384; }
 cudaError_t launch_scan_seg(const ScanArgs&, int, int64_t, cudaStream_t) { ++g_launches; return cudaSuccess; }
+int64_t scan_seg_chunk_steps(int io) { return io == 0 ? 32 : 64; }
+int64_t scan_seg_tile_channels() { return 16; }
+int64_t scan_seg_tile_record_bytes() { return 257 * 16; }
+cudaError_t launch_scan_seg_split(const ScanArgs&, int, int64_t, int, void*, int64_t, int64_t, cudaStream_t) {
+    ++g_launches;
+    return cudaSuccess;
+}
 unsigned int scan_seg_read_and_clear_device_error() { return 0; }
 unsigned int scan_read_and_clear_device_error() { return 0; }
 unsigned int scan_bwd_read_and_clear_device_error() { return 0; }
@@ -100,6 +107,19 @@ void scan_calls(const mm_scan_dims& d, float beta, float alpha) {
     expect_status(mm_scan_ckpt_size(&d, &bytes), "mm_scan_ckpt_size");
     int64_t seg = 0;
     expect_status(mm_scan_segment_len(&d, &seg), "mm_scan_segment_len");
+    // the split launches, with their segment length and the piece's place at extremes
+    for (int64_t S : {int64_t(-1), int64_t(0), int64_t(32), int64_t(64), int64_t(1) << 30, int64_t(1) << 62})
+        for (int64_t first : {int64_t(-64), int64_t(0), int64_t(64), int64_t(1) << 30, int64_t(1) << 62})
+            for (int64_t total : {int64_t(0), int64_t(64), d.seqlen, int64_t(1) << 30, std::numeric_limits<int64_t>::max()}) {
+                expect_status(mm_scan_fwd_split_correct(fake(1), ffake(2), fake(4), ffake(5), ffake(6), beta, alpha,
+                                                        fake(7), ffake(8), ffake(9), fake(10), S, first, total, &d,
+                                                        nullptr), "mm_scan_fwd_split_correct");
+            }
+    for (int64_t S : {int64_t(-1), int64_t(32), int64_t(64), int64_t(1) << 30, int64_t(1) << 62})
+        expect_status(mm_scan_fwd_split_maps(fake(0), fake(1), ffake(2), fake(3), fake(4), beta, alpha, fake(7),
+                                             fake(10), S, &d, nullptr), "mm_scan_fwd_split_maps");
+    for (int64_t n : {int64_t(-1), int64_t(0), int64_t(1), int64_t(1) << 30, int64_t(1) << 31})
+        expect_status(mm_scan_split_maps_size(&d, n, &bytes), "mm_scan_split_maps_size");
 }
 
 void ssd_calls(const mm_ssd_dims& d, float beta, float alpha) {
@@ -149,6 +169,15 @@ int main() {
     if (mm_ssd_fwd(fake(0), ffake(1), ffake(2), fake(3), fake(4), nullptr, 0.0f, 1.0f, fake(6), nullptr,
                    &sok, nullptr) != MM_OK || g_launches != before + 2) {
         std::printf("an in-range SSD call did not launch\n");
+        ++g_bad;
+    }
+    const mm_scan_dims piece = {2, 128, 8, 16, MM_F32};
+    if (mm_scan_fwd_split_maps(fake(0), fake(1), ffake(2), fake(3), fake(4), 0.9f, 1.0f, fake(7), fake(10), 64,
+                               &piece, nullptr) != MM_OK ||
+        mm_scan_fwd_split_correct(fake(1), ffake(2), fake(4), nullptr, nullptr, 0.9f, 1.0f, fake(7), ffake(8),
+                                  nullptr, fake(10), 64, 128, 300, &piece, nullptr) != MM_OK ||
+        g_launches != before + 4) {
+        std::printf("an in-range split call did not launch\n");
         ++g_bad;
     }
     expect_status(mm_device_status(), "mm_device_status");

@@ -245,6 +245,11 @@ def test_set_path_and_segment_length_query(lib):
     assert lib.mm_scan_set_path(2, 256) == 0
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg)) == 0
     assert seg.value == 256                                       # forced onto the sequence-split path
+    assert lib.mm_scan_set_path(2, 32) == 0
+    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 2048, 64, 16, 1)), ctypes.byref(seg)) == 0
+    assert seg.value == 64                                        # bf16: at least one 64-step chunk
+    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 2048, 64, 16, 0)), ctypes.byref(seg)) == 0
+    assert seg.value == 32
     assert lib.mm_scan_set_path(1, 0) == 0
     assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 0
     assert lib.mm_scan_set_path(0, 0) == 0
@@ -252,6 +257,49 @@ def test_set_path_and_segment_length_query(lib):
     assert lib.mm_scan_segment_len(ctypes.byref(unaligned), ctypes.byref(seg)) == 0 and seg.value == 0
     assert lib.mm_scan_segment_len(None, ctypes.byref(seg)) == 1
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(0, 1, 1, 1, 0)), ctypes.byref(seg)) == 2
+
+
+def test_split_sizes_and_checks(lib, monkeypatch):
+    """The sequence split's host checks: record sizes, the segment length, the
+    piece's place in the whole sequence, and aliasing."""
+    size = ctypes.c_size_t(0)
+    # one record per (batch row, 16-channel tile) of a segment: 8 float4 maps of 32 lanes and a flag
+    assert lib.mm_scan_split_maps_size(ctypes.byref(D(batch=2, dim=40)), 3, ctypes.byref(size)) == 0
+    assert size.value == 3 * 2 * 3 * 257 * 16
+    assert lib.mm_scan_split_maps_size(ctypes.byref(D()), -1, ctypes.byref(size)) == 2
+    assert lib.mm_scan_split_maps_size(None, 1, ctypes.byref(size)) == 1
+
+    def maps(S=64, d=None, **over):
+        a = dict(x=_fake(0), delta=_fake(1), A=_fake(2), B=_fake(3), C=_fake(4), y=_fake(5), maps=_fake(6))
+        a.update(over)
+        dims = d if d is not None else D(L=128)
+        return lib.mm_scan_fwd_split_maps(a["x"], a["delta"], a["A"], a["B"], a["C"], 0.9, 1.0, a["y"], a["maps"],
+                                          S, ctypes.byref(dims), None)
+
+    def correct(S=64, first=0, total=128, d=None, **over):
+        a = dict(delta=_fake(1), A=_fake(2), C=_fake(4), h0=None, v0=None, y=_fake(5), hT=_fake(7), vT=None,
+                 maps=_fake(6))
+        a.update(over)
+        dims = d if d is not None else D(L=128)
+        return lib.mm_scan_fwd_split_correct(a["delta"], a["A"], a["C"], a["h0"], a["v0"], 0.9, 1.0, a["y"],
+                                             a["hT"], a["vT"], a["maps"], S, first, total, ctypes.byref(dims), None)
+
+    assert maps(S=48) == 6 and maps(S=16) == 6                    # not a power of two >= one chunk
+    assert maps(S=32, d=D(L=128, io=1)) == 6                      # bf16: a chunk is 64 steps
+    assert maps(d=D(L=129)) == 6                                  # rows not whole 16-byte pieces
+    assert maps(maps=None) == 1
+    assert maps(maps=ctypes.c_void_p(A16 * 7 + 8)) == 5
+    assert maps(maps=_fake(1)) == 9                               # records on top of delta
+    assert maps(y=_fake(6)) == 9                                  # y on top of the records
+    assert correct(first=32) == 6                                 # piece not at a segment boundary
+    assert correct(first=64, total=128) == 6                      # piece past the end
+    assert correct(first=0, total=300, d=D(L=96)) == 6            # an inner piece of a partial segment
+    assert correct(total=0) == 6
+    assert correct(hT=_fake(6)) == 9                              # hT on top of the records
+    assert correct(h0=_fake(7), hT=_fake(7)) == 9                 # no in-place state here
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert maps() == 7                                            # in range: reaches the launch step
+    assert correct(first=128, total=300) == 7                     # the last piece may be partial
 
 
 def test_ssd_rejects_bad_arguments(lib, monkeypatch):

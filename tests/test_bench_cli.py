@@ -112,3 +112,20 @@ def test_reference_arm_on_a_resized_workload():
     assert d["config"]["workload"] == wl.SCAN_SMALL.name + "_as_b2_l64"
     assert d["config"]["batch"] == 2 and d["config"]["seq_len"] == 64
     assert _bench("--workload", "decode", "--seqlen", "4", timeout=120).returncode == 2
+
+
+def test_split_segment_length_gives_every_rank_a_full_round():
+    # the long workload: 16384-step segments on one rank (eight of them); over eight
+    # ranks, halved until each rank holds eight segments
+    import selective_state_space_momentum_b200 as mm
+    from selective_state_space_momentum_b200 import build as mmbuild
+    mmbuild.build()
+    w = wl.SCAN_LONG
+    assert bench.split_seg_len(w, 1) == 16384
+    assert bench.split_seg_len(w, 2) == 8192
+    assert bench.split_seg_len(w, 8) == 2048
+    assert bench.split_seg_len(w, 8, forced=4096) == 4096
+    for world in (1, 2, 4, 8):
+        S = bench.split_seg_len(w, world)
+        pieces = mm.split_pieces(w.seqlen, world, S)
+        assert all(n // S >= 8 for _, n in pieces)

@@ -9,7 +9,8 @@ all -- a flag that nothing sets, the allowed way to make a wait run out: no
 copy is in flight, no GPU fault is provoked -- and each test then checks the
 status and that a normal call right after still matches the fp64 oracle.
 One test per kernel family: the register-resident scan, the sequence-split
-scan, the backward, the SSD kernel, the tensor-core momentum SSD kernel.
+scan (fused, and both launches of its split across ranks), the backward,
+the SSD kernel, the tensor-core momentum SSD kernel.
 """
 import numpy as np
 import pytest
@@ -59,6 +60,28 @@ def test_forward_scan_wait_runs_out(monkeypatch, path, seg):
         _scan_check(dev, inp)
     finally:
         mm.mm_scan_set_path(0, 0)
+
+
+def test_split_scan_waits_run_out(monkeypatch):
+    # both launches of the scan split across ranks (one rank here)
+    inp = wl.scan_inputs(wl.SCAN_MEDIUM, batch=2, seqlen=512, dim=48)
+    dev = _scan_dev(inp)
+    S, (batch, dim, L), N = 64, dev["x"].shape, dev["A"].shape[1]
+    maps = torch.empty(mm.mm_scan_split_maps_size(batch, L, dim, N, L // S), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(dev["x"])
+    h0 = torch.ones((batch, dim, N), device="cuda")
+    hT, vT = torch.empty_like(h0), torch.empty_like(h0)
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "stall")
+    mm.mm_scan_fwd_split_maps(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], 0.9, 1.0, y, maps, S)
+    monkeypatch.delenv("MMSCAN_FAULT_INJECT")
+    _expect_timeout()
+    mm.mm_scan_fwd_split_maps(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], 0.9, 1.0, y, maps, S)
+    mm.mm_device_status()
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "stall")
+    mm.mm_scan_fwd_split_correct(dev["delta"], dev["A"], dev["C"], h0, None, 0.9, 1.0, y, hT, vT, maps, S, 0, L)
+    monkeypatch.delenv("MMSCAN_FAULT_INJECT")
+    _expect_timeout()
+    _scan_check(dev, inp)
 
 
 def test_backward_wait_runs_out(monkeypatch):
