@@ -574,6 +574,45 @@ mm_status mm_scan_fwd_split_correct(const void *delta, const float *A, const voi
                                     int64_t seg_len, int64_t seq_first, int64_t seqlen_total,
                                     const mm_scan_dims *dims, void *stream);
 
+/*
+ * mm_scan_fwd_noalloc -- mm_scan_fwd for callers that cannot allocate device
+ * memory.  (An addition of this library: the paper has no counterpart.)
+ *
+ * Who needs it: code that runs where every device allocation belongs to a
+ * host framework (a plugin, a serving runtime's custom-op slot), a process
+ * whose device memory was reserved once at start-up, or a path that must
+ * not pay cudaMalloc's device-wide synchronisation.  The scan's two-launch
+ * sequence split (mm_scan_fwd_split_maps, then mm_scan_fwd_split_correct,
+ * on this one device) passes segment records between its launches; here
+ * they live in a fixed 8 MiB array inside the library, reserved on every GPU
+ * that loads the library until the process exits.  Nothing is allocated:
+ * no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Arguments, layouts and results as mm_scan_fwd (the caller owns and passes
+ * every input and output); y, hT, vT equal those of one call of the
+ * sequence-split path with this entry's segment length S, the path's own
+ * length for (batch * dim), at least one staged chunk (32 fp32 / 64 bf16
+ * steps).  Limits: the records of ceil(seqlen / S) segments
+ * (mm_scan_split_maps_size) must fit in 8 MiB, else MM_ERR_UNSUPPORTED
+ * with the bytes needed; rows of seqlen elements must be a whole number of
+ * 16-byte pieces and dstate <= 16 (MM_ERR_UNSUPPORTED); hT, vT may not be
+ * h0, v0 (MM_ERR_ALIAS).  Other errors as mm_scan_fwd.
+ *
+ * The first call on a device looks up the array's address on that device
+ * (cudaGetSymbolAddress, that device current); make that first call before
+ * any stream capture.  Every call shares the one array and leaves its
+ * records there: nothing in it has to start at zero (each call writes every
+ * record it reads before reading it), but calls whose work overlaps on the
+ * GPU -- on two streams, or from two host threads -- race on it and must be
+ * ordered by the caller.
+ */
+mm_status mm_scan_fwd_noalloc(const void *x, const void *delta, const float *A,
+                              const void *B, const void *C,
+                              const float *h0, const float *v0,
+                              float beta, float alpha,
+                              void *y, float *hT, float *vT,
+                              const mm_scan_dims *dims, void *stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mm_version(void);
 

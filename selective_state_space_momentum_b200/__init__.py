@@ -34,7 +34,7 @@ __all__ = [
     "mm_scan_fwd_host", "mm_scan_fwd_host_workspace_size", "mm_ssd_fwd_host",
     "mm_ssd_fwd_host_workspace_size",
     "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
-    "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
+    "mm_scan_fwd_noalloc", "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
     "ssd_fwd_host", "split_pieces", "scan_fwd_split",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
 ]
@@ -63,7 +63,8 @@ EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm
                     "mm_scan_set_path", "mm_scan_segment_len",
                     "mm_scan_fwd_host_workspace_size", "mm_scan_fwd_host",
                     "mm_ssd_fwd_host_workspace_size", "mm_ssd_fwd_host",
-                    "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct")
+                    "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
+                    "mm_scan_fwd_noalloc")
 
 
 class MMError(RuntimeError):
@@ -135,6 +136,8 @@ def _declare(lib):
     lib.mm_scan_fwd_split_correct.restype = ctypes.c_int
     lib.mm_scan_fwd_split_correct.argtypes = [vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp, i64, i64, i64,
                                               ctypes.POINTER(ScanDims), vp]
+    lib.mm_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.mm_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
     lib.mm_status_string.restype = ctypes.c_char_p
     lib.mm_status_string.argtypes = [ctypes.c_int]
     lib.mm_last_error.restype = ctypes.c_char_p
@@ -547,6 +550,23 @@ def mm_scan_fwd_split_correct(delta, A, C, h0, v0, beta, alpha, y, hT, vT, maps_
                                                   _ptr(maps_all), int(seg_len), int(seq_first),
                                                   int(seqlen_total), ctypes.byref(dims), _stream_handle(stream))
     _check(rc, "mm_scan_fwd_split_correct")
+
+
+def mm_scan_fwd_noalloc(x, delta, A, B, C, h0, v0, beta, alpha, y, hT, vT, stream=None):
+    """C entry point mm_scan_fwd_noalloc (marshalling only): mm_scan_fwd for
+    callers that cannot allocate device memory; the records between its two
+    launches live in the library's fixed 8 MiB device array.  Shapes as
+    mm_scan_fwd; hT, vT may not be h0, v0."""
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("h0", h0, "state", True), ("v0", v0, "state", True), ("y", y, "io", False),
+                         ("hT", hT, "state", True), ("vT", vT, "state", True)])
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_fwd_noalloc(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(v0),
+                                            float(beta), float(alpha), _ptr(y), _ptr(hT), _ptr(vT),
+                                            ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_fwd_noalloc")
 
 
 def mm_version() -> int:
