@@ -7,11 +7,13 @@
  * ---------------------------------------
  * - Pointers named as device buffers must be CUDA device (or managed) memory
  *   of the current device; the caller allocates and owns every buffer.  The
- *   library allocates no memory and keeps no state between calls except a
- *   per-thread copy of the last error message (mm_last_error), the
- *   process-wide tuning switches (mm_scan_set_tile, mm_scan_set_path) and
- *   the per-thread side streams of the *_host entry points, which take host
- *   buffers and a device workspace.
+ *   library's only device memory of its own is the stream-ordered record
+ *   memory of mm_scan_fwd's sequence-split path (a pool per device, see
+ *   mm_scan_fwd) and the fixed array of mm_scan_fwd_noalloc; it keeps no
+ *   other state between calls except a per-thread copy of the last error
+ *   message (mm_last_error), the process-wide tuning switches
+ *   (mm_scan_set_tile, mm_scan_set_path) and the per-thread side streams of
+ *   the *_host entry points, which take host buffers and a device workspace.
  * - Every base pointer of a device buffer must be 16-byte aligned
  *   (MM_ERR_ALIGN otherwise).
  *   Tensors are dense and contiguous in the stated layout, last index
@@ -114,7 +116,18 @@ typedef struct {
  *     order ("Forward Pass: Two-Stage Parallel Scan" of the same page, with
  *     the chunk carry [[beta^S, 0], [Q, P]] per lane); y gets the response to
  *     each segment's carry-in until that response is below 2^-25 of its start
- *     (when A <= 0 and delta >= 0), else over the whole segment.
+ *     (when A <= 0 and delta >= 0), else over the whole segment.  It runs as
+ *     two launches on `stream` -- the segments' main passes, their maps
+ *     written to records, then the folds and corrections -- with the records
+ *     (ceil(L / S) * batch * ceil(dim / 16) * 4112 bytes, 4.2 MB for one row
+ *     of 2048 channels and 131072 steps) in stream-ordered memory from a
+ *     pool the library creates per device on first use and keeps (up to
+ *     64 MiB reserved between calls; cudaMallocFromPoolAsync, cudaFreeAsync
+ *     on `stream`).  When that memory cannot be had (or records would pass
+ *     1 GiB), and for in-place streaming (hT = h0 or vT = v0), it runs as one
+ *     launch whose segments exchange their maps through distributed shared
+ *     memory; both forms give bit-identical results.  mm_scan_fwd_noalloc
+ *     allocates nothing.
  *
  * Streaming: for a fixed (batch, dim, dstate, io), calling with the first
  * L1 steps and then with the remaining steps, passing (hT, vT) of the first
@@ -401,7 +414,8 @@ mm_status mm_ssd_fwd_momentum(const void *x, const float *delta, const float *A,
  * workspace: device memory of at least the bytes the matching
  * *_workspace_size query returns for the same dims and chunk_steps, 16-byte
  * aligned, owned by the caller, not used by anything else until the call's
- * work on `stream` has completed.  The library allocates no memory.  A call
+ * work on `stream` has completed.  The chunks' scans are mm_scan_fwd calls
+ * (with their record memory on the sequence-split path).  A call
  * of more than one chunk runs its copies on two streams of its own, with
  * eleven events; they are created on first use and kept for the calling
  * host thread and device until the thread exits.  A call of one chunk runs
@@ -477,7 +491,8 @@ mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_
  * Tuning and test knob: force the scan path -- 0 automatic, 1 the
  * register-resident kernel, 2 the sequence-split kernel (used where it
  * applies: no extras, no checkpoints, dstate <= 16, rows of a whole number of
- * 16-byte pieces) -- and its segment length (0: automatic; else a power of
+ * 16-byte pieces), 3 the same as one fused launch (no records, see
+ * mm_scan_fwd) -- and its segment length (0: automatic; else a power of
  * two in [32, 2^30]; bf16 calls use at least 64, one staged chunk of the
  * kernel).  Process-wide, not thread-safe with concurrent calls.
  * MM_ERR_UNSUPPORTED for other values.

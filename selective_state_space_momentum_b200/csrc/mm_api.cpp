@@ -57,7 +57,7 @@ int64_t seg_len_for(int64_t batch, int64_t L, int64_t dim, int64_t dstate, int i
     const int path = g_forced_path.load();
     if (!vec_ok || dstate > 16) return 0;
     if (path == 1) return 0;
-    if (path == 0 && !seg_auto(batch, dim, dstate, io)) return 0;
+    if (path == 0 && !seg_auto(batch, dim, dstate, io)) return 0;       // 2, 3: forced
     const int64_t forced = g_forced_seg_len.load();
     int64_t S = forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
     // a segment is a whole number of staged chunks (64 steps for bf16)
@@ -111,7 +111,7 @@ bool inject_launch_failure() {
 // scans, the backward, the SSD kernel) are launched with their producer told
 // to issue nothing.  Nothing is then in flight; every wait runs out after its
 // limit, the kernel returns, and mm_device_status reports
-// MM_ERR_DEVICE_TIMEOUT.  The outputs of such a call are not written.
+// MM_ERR_DEVICE_TIMEOUT.  The outputs of such a call are undefined.
 int inject_stall() {
     const char* v = std::getenv("MMSCAN_FAULT_INJECT");
     return (v && std::strcmp(v, "stall") == 0) ? 1 : 0;
@@ -274,8 +274,8 @@ mm_status mm_scan_set_tile(int spt, int warps, int time_lanes) {
 }
 
 mm_status mm_scan_set_path(int path, int64_t seg_len) {
-    if (path < 0 || path > 2)
-        return fail(MM_ERR_UNSUPPORTED, "scan path %d is not 0 (automatic), 1 or 2", path);
+    if (path < 0 || path > 3)
+        return fail(MM_ERR_UNSUPPORTED, "scan path %d is not 0 (automatic), 1, 2 or 3", path);
     if (seg_len != 0 && (seg_len < 32 || seg_len > (int64_t(1) << 30) || (seg_len & (seg_len - 1)) != 0))
         return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not 0 or a power of two in [32, 2^30]",
                     (long long)seg_len);
@@ -448,9 +448,13 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.stall = inject_stall();
     if (!a.ext && !ckpt) {
         const int64_t seg = seg_len_for(bsz, L, D, N, dims->io, a.vec_ok != 0);
-        if (seg > 0)
-            return from_cuda(mmscan::launch_scan_seg(a, dims->io, seg, static_cast<cudaStream_t>(stream)),
+        if (seg > 0) {
+            // in-place streaming (hT = h0 or vT = v0) needs the fused launch, whose CTAs
+            // all read the initial state before any writes the final one
+            const bool fused = g_forced_path.load() == 3 || (hT && hT == h0) || (vT && vT == v0);
+            return from_cuda(mmscan::launch_scan_seg(a, dims->io, seg, fused, static_cast<cudaStream_t>(stream)),
                              "mm_scan_fwd launch");
+        }
     }
     const mmscan::ScanTileChoice t =
         mmscan::choose_scan_tile(bsz, D, N, dims->io, g_forced_spt.load(), g_forced_warps.load(),

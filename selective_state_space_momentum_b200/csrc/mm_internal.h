@@ -117,7 +117,11 @@ struct ScanTileChoice {
 constexpr int kSegMaxCluster = 8;
 constexpr int64_t kSegMinLen = 16384;
 int64_t scan_seg_default_len(int64_t batch, int64_t dim);
-cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s);
+// The sequence-split path of mm_scan_fwd: by default two launches (the main
+// passes with their segment maps to records in stream-ordered memory from a
+// library pool, then the fold and correction); `fused`, or records that
+// cannot be had, run the single fused launch.
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, bool fused, cudaStream_t s);
 // Steps of one staged chunk of the sequence-split kernel (32 fp32, 64 bf16).
 int64_t scan_seg_chunk_steps(int io);
 // The sequence split over several calls: the channels of one CTA's tile and

@@ -56,6 +56,7 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "mm_common.cuh"
 #include "mm_internal.h"
@@ -188,7 +189,9 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int warp = tid >> 5;
     const int g = lane & (G - 1);                 // state group: states 4g .. 4g+3
     const int pr = lane >> 2;                     // channel pair within the warp
-    const int rank = (int)cluster_ctarank();      // segment within the round
+    // segment within the round (the split launches run without clusters: the
+    // same mapping from the block index)
+    const int rank = MODE == 0 ? (int)cluster_ctarank() : (int)(blockIdx.x % (unsigned)csize);
     const int64_t cl = blockIdx.x / csize;        // (batch row, channel tile)
     const int64_t b = cl / p.tiles_per_batch;
     const int64_t d0 = (cl % p.tiles_per_batch) * CH;
@@ -904,7 +907,8 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, 
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
     attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    // the split launches share nothing between CTAs: plain grids, placed freely
+    cfg.numAttrs = MODE == 0 ? 2 : 0;
     return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize, sp);
 }
 
@@ -930,7 +934,75 @@ int64_t scan_seg_default_len(int64_t batch, int64_t dim) {
     return s;
 }
 
-cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, cudaStream_t s) {
+namespace {
+
+// Stream-ordered memory for the segment records of the two-launch form: one
+// pool per device, created on first use, keeping up to kPoolKeepBytes
+// reserved between calls so that a call after a synchronisation does not go
+// back to the driver for its records.
+constexpr int kPoolDevices = 64;
+constexpr uint64_t kPoolKeepBytes = uint64_t(64) << 20;
+constexpr int64_t kMaxRecordBytes = int64_t(1) << 30;   // larger record sets run the fused launch
+std::mutex g_pool_mutex;
+cudaMemPool_t g_pool[kPoolDevices] = {};
+bool g_pool_unavailable[kPoolDevices] = {};
+
+cudaMemPool_t records_pool() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kPoolDevices) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_pool_mutex);
+    if (g_pool[dev] || g_pool_unavailable[dev]) return g_pool[dev];
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+        (void)cudaGetLastError();
+        g_pool_unavailable[dev] = true;
+        return nullptr;
+    }
+    uint64_t keep = kPoolKeepBytes;
+    (void)cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pool[dev] = pool;
+    return pool;
+}
+
+// Bytes of the records of every segment of the call, or -1 beyond kMaxRecordBytes.
+int64_t call_record_bytes(const ScanArgs& a, int64_t seg_len) {
+    const int64_t nseg = (a.seqlen + seg_len - 1) / seg_len;
+    constexpr int CH = SegTile<float, kSegWarps, kSegStages>::CH;
+    const int64_t tiles = (a.dim + CH - 1) / CH;
+    const double b = (double)nseg * (double)a.batch * (double)tiles * (double)scan_seg_tile_record_bytes();
+    return b > (double)kMaxRecordBytes ? -1 : (int64_t)b;
+}
+
+}  // namespace
+
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, bool fused, cudaStream_t s) {
+    if (!fused) {
+        // The two-launch form: main passes with their maps to records in
+        // stream-ordered memory, then the fold and correction.  Compiled
+        // apart, the main pass runs 6% faster than inside the fused kernel.
+        const int64_t bytes = call_record_bytes(a, seg_len);
+        cudaMemPool_t pool = bytes > 0 ? records_pool() : nullptr;
+        void* rec = nullptr;
+        if (pool && cudaMallocFromPoolAsync(&rec, (size_t)bytes, pool, s) == cudaSuccess) {
+            SegSplit sp{};
+            sp.maps = static_cast<float4*>(rec);
+            sp.seg_first = 0;
+            sp.L_total = a.seqlen;
+            sp.nseg_total = (a.seqlen + seg_len - 1) / seg_len;
+            cudaError_t e = launch_seg_mode<1>(a, io, seg_len, sp, s);
+            if (e == cudaSuccess) e = launch_seg_mode<2>(a, io, seg_len, sp, s);
+            const cudaError_t ef = cudaFreeAsync(rec, s);
+            return e != cudaSuccess ? e : ef;
+        }
+        (void)cudaGetLastError();   // no records: the fused launch needs none
+    }
     return launch_seg_mode<0>(a, io, seg_len, SegSplit{}, s);
 }
 

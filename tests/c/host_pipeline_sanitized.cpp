@@ -358,7 +358,7 @@ cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice&, int io, cu
     enqueue(s, [a, io] { scan_cpu(a, io); });
     return cudaSuccess;
 }
-cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t, cudaStream_t s) {
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t, bool, cudaStream_t s) {
     ++g_launches;
     enqueue(s, [a, io] { scan_cpu(a, io); });
     return cudaSuccess;

@@ -232,7 +232,12 @@ def test_set_tile(lib):
 
 
 def test_set_path_and_segment_length_query(lib):
-    assert lib.mm_scan_set_path(3, 0) == 6
+    assert lib.mm_scan_set_path(4, 0) == 6
+    assert lib.mm_scan_set_path(3, 0) == 0                        # the sequence split as one fused launch
+    seg3 = ctypes.c_int64(-1)
+    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg3)) == 0
+    assert seg3.value == 16384                                    # forced onto the sequence-split path
+    assert lib.mm_scan_set_path(0, 0) == 0
     assert lib.mm_scan_set_path(2, 48) == 6                       # not a power of two
     assert lib.mm_scan_set_path(2, 16) == 6                       # below 32
     seg = ctypes.c_int64(-1)

@@ -6,7 +6,10 @@ each segment's 2x2 affine carry map ("Momentum Mamba: Enhanced State Space
 Models with Momentum", "Forward Pass: Two-Stage Parallel Scan").  These tests
 force that path (mm_scan_set_path) with short segments so that small inputs
 cross many segments, several rounds of a cluster and ragged ends, and compare
-the whole output with the oracle at the scan's tolerances:
+the whole output with the oracle at the scan's tolerances.  The path runs as
+two launches (segment maps passed through stream-ordered records) or, forced
+with path 3 and for in-place streaming, as one fused launch (maps through
+distributed shared memory); the two forms must agree bit for bit.
   * fp32 I/O: max |y - y_ref| <= 1e-4 * max |y_ref| (also hT, vT);
   * bf16 I/O: ||y - y_ref||_2 / ||y_ref||_2 <= 1e-2;
   * streaming: hT, vT bit-identical between one call and two calls split at
@@ -28,9 +31,10 @@ BF16_TOL = 1e-2
 
 @pytest.fixture
 def seg_path():
-    """Force the sequence-split path with a given segment length; restore after."""
-    def force(seg_len):
-        mm.mm_scan_set_path(2, seg_len)
+    """Force the sequence-split path (2: two launches, 3: one fused launch)
+    with a given segment length; restore after."""
+    def force(seg_len, path=2):
+        mm.mm_scan_set_path(path, seg_len)
     yield force
     mm.mm_scan_set_path(0, 0)
 
@@ -86,12 +90,13 @@ def _check(io, got, inp, beta, alpha, h0=None, v0=None, what=""):
         assert err <= F32_TOL * scale, f"{what}: {name} max abs err {err:.3e} vs {scale:.3e}"
 
 
+@pytest.mark.parametrize("path", [2, 3], ids=["two-launch", "fused"])
 @pytest.mark.parametrize("L,seg", [(256, 32), (1000, 64), (4096, 128), (4133 // 4 * 4, 256), (96, 128)])
 @pytest.mark.parametrize("beta,alpha", [(0.9, 1.0), (0.0, 1.0), (0.99, 0.5), (0.3, 2.0), (0.5, 1.0)])
-def test_segments_rounds_and_ragged_ends(seg_path, L, seg, beta, alpha):
+def test_segments_rounds_and_ragged_ends(seg_path, L, seg, beta, alpha, path):
     # beta >= 1/2 runs the scaled form of the recurrence, smaller beta the plain one
     # up to 32 segments: several rounds of an 8-CTA cluster, a ragged last chunk
-    seg_path(seg)
+    seg_path(seg, path)
     inp = _inputs(2, L, 40, 16, seed=7 + L)
     _check("f32", _run(_dev(inp, "f32"), beta, alpha), inp, beta, alpha, what=f"L={L} S={seg}")
 
@@ -189,3 +194,21 @@ def test_segment_length_query():
     assert mm.mm_scan_segment_len(1, 131072, 2048, 8) == 0          # dstate <= 8
     assert mm.mm_scan_segment_len(1, 256, 64, 16) == 0              # one segment: nothing to split
     assert mm.mm_scan_segment_len(1, 16384, 2048, 16) == 0
+
+
+@pytest.mark.parametrize("L,seg,beta,io", [(4096, 128, 0.99, "f32"), (1000, 64, 0.3, "f32"),
+                                           (2048, 256, 0.9, "bf16"), (8192, 64, 0.999, "f32")])
+def test_two_launch_and_fused_forms_are_bit_identical(seg_path, L, seg, beta, io):
+    law = wl.SCAN_MEDIUM if io == "f32" else wl.SCAN_BF16
+    inp = _inputs(2, L, 40, 16, seed=L + seg, io=io, law=law)
+    dev = _dev(inp, io)
+    rng = np.random.default_rng(L)
+    h0, v0 = (torch.from_numpy(a).cuda() for a in _states(rng, 2, 40, 16, 1.0))
+    out = {}
+    for path in (2, 3):
+        seg_path(seg, path)
+        out[path] = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=h0, v0=v0, beta=beta)
+        torch.cuda.synchronize()
+        mm.mm_device_status()
+    for a, b, name in zip(out[2], out[3], ("y", "hT", "vT")):
+        assert torch.equal(a, b), f"{name} differs between the two-launch and the fused form"
