@@ -118,6 +118,12 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t addr, uint32_t rank) {
     return r;
 }
 
+__device__ __forceinline__ float dsmem_ld1(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float4 dsmem_ld4(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -620,22 +626,33 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             ch[c][e] = hn;
         }
     };
-    // Split launches: the records of segments 0 .. nfold-1 of the whole sequence
-    // folded in order onto the carry; each record is read one segment ahead.
-    auto fold_records = [&](float (&cv)[2][4], float (&ch)[2][4], int64_t nfold) {
-        const float4* rec0 = sp.maps + (int64_t)(blockIdx.x / csize) * REC + tid;
+    // Split launches: the records of segments j0 .. j1-1 of the whole sequence
+    // folded in order onto the carry.  Records stream through a ring of
+    // kFoldRing slots in the (then idle) staging area, kFoldRing - 1 ahead of
+    // the one applied: the fold's time is its FMA chain, not one L2 round trip
+    // per segment.  Each lane copies and reads only its own 8 float4 of a
+    // record, so no barrier is needed.
+    constexpr int kFoldRing = 4;
+    static_assert(kFoldRing * 8 * NT * 16 <= ST * TL::STAGE_BYTES, "the fold ring fits the staging area");
+    auto fold_records = [&](float (&cv)[2][4], float (&ch)[2][4], int64_t j0, int64_t j1) {
+        const int64_t nfold = j1 > j0 ? j1 - j0 : 0;
+        const float4* rec0 = sp.maps + (j0 * ncl + (int64_t)(blockIdx.x / csize)) * REC + tid;
         const int64_t seg_stride = ncl * REC;
-        float4 cur[8], nxt[8];
-        if (nfold > 0) {
+        float4* ring = reinterpret_cast<float4*>(smem) + tid;        // [slot][8][NT]
+        auto fetch = [&](int64_t j) {
+            if (j < nfold) {
+                const int slot = (int)(j % kFoldRing);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) cur[i] = rec0[i * NT];
-        }
-        for (int64_t j = 0; j < nfold; ++j) {
-            if (j + 1 < nfold) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) nxt[i] = rec0[(j + 1) * seg_stride + i * NT];
+                for (int i = 0; i < 8; ++i) cp_async_16(ring + (slot * 8 + i) * NT, rec0 + j * seg_stride + i * NT, 16);
             }
-            const int64_t sj = j * seg_len;
+            cp_async_commit();            // one group per record index, empty past the end
+        };
+        for (int64_t j = 0; j < kFoldRing - 1; ++j) fetch(j);
+        for (int64_t j = 0; j < nfold; ++j) {
+            fetch(j + kFoldRing - 1);
+            cp_async_wait<kFoldRing - 1>();   // record j's group has landed
+            const float4* cur = ring + (int)(j % kFoldRing) * 8 * NT;
+            const int64_t sj = (j0 + j) * seg_len;
             const int64_t lj = sp.L_total - sj < seg_len ? sp.L_total - sj : seg_len;
             const float bS = pow_steps(beta, lj);
 #pragma unroll
@@ -643,12 +660,53 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int i0 = (c * 2 + q) * 2;
-                    apply_map(cv, ch, cur[i0], cur[i0 + 1], c, q, bS);
+                    apply_map(cv, ch, cur[i0 * NT], cur[(i0 + 1) * NT], c, q, bS);
                 }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
         }
+        cp_async_wait<0>();
+        // the correction's tiled copies overwrite the ring next (behind a CTA barrier)
+        fence_proxy_async_smem();
     };
+
+    // The carry entering the segment rounds: (h0, v0) folded through the
+    // earlier pieces' records.  In a piece after the first, one CTA of each
+    // cluster (the channel tile's CTAs) folds them and the others copy the
+    // result from its shared memory, instead of every CTA reading every
+    // earlier record.
+    auto load_carry = [&](float (&cv)[2][4], float (&ch)[2][4]) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { cv[c][e] = carry_at(c, e, 0); ch[c][e] = carry_at(c, e, 1); }
+    };
+    auto store_carry = [&](const float (&cv)[2][4], const float (&ch)[2][4]) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { carry_at(c, e, 0) = cv[c][e]; carry_at(c, e, 1) = ch[c][e]; }
+    };
+    if constexpr (MODE == 2) {
+        if (sp.seg_first > 0) {           // launched in clusters of the tile's csize CTAs
+            if (rank == 0) {
+                float cv[2][4], ch[2][4];
+                load_carry(cv, ch);
+                fold_records(cv, ch, 0, sp.seg_first);
+                store_carry(cv, ch);
+            }
+            cluster_sync_all();
+            if (rank != 0) {
+                const uint32_t src = dsmem_map(base + TL::OFF_CARRY, 0u);
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+#pragma unroll
+                        for (int w2 = 0; w2 < 2; ++w2)
+                            carry_at(c, e, w2) = dsmem_ld1(src + (uint32_t)(((((c * 4 + e) * 2 + w2) * NT) + tid) * 4));
+            }
+            cluster_sync_all();           // rank 0's area has been read before any CTA goes on
+        }
+    }
 
     for (int64_t r = 0; r < rounds; ++r) {
         const int64_t k = r * csize + rank;                       // this CTA's segment
@@ -733,10 +791,12 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
             for (int e = 0; e < 4; ++e) { rv[c][e] = 0.0f; rh[c][e] = 0.0f; }
         if constexpr (MODE == 2) {
-            // the carry-in of global segment kg: every earlier segment's map, in order, onto (h0, v0)
+            // the carry-in of global segment kg: the carry at the round's start (every
+            // earlier segment's map, in order, onto (h0, v0)) through the round's
+            // segments before it
             const int64_t kg = sp.seg_first + k;
             if (!dead && slen > 0) {
-                fold_records(cv, ch, kg);
+                fold_records(cv, ch, sp.seg_first + r * csize, kg);
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -820,22 +880,28 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             drain();
         }
+        if constexpr (MODE == 2) {
+            // the carry at the next round's start: the round's segments of this piece
+            const int64_t j0 = sp.seg_first + r * csize;
+            const int64_t jend = sp.seg_first + nseg < j0 + csize ? sp.seg_first + nseg : j0 + csize;
+            if (!dead && r + 1 < rounds) {
+                float cv[2][4], ch[2][4];
+                load_carry(cv, ch);
+                fold_records(cv, ch, j0, jend);
+                store_carry(cv, ch);
+            }
+        }
     }
 
     // ---- final states: the carry after the last segment -----------------------
     if constexpr (MODE == 2) {
-        // every segment of the whole sequence folded onto (h0, v0), as above
+        // every segment of the whole sequence folded onto (h0, v0): from the carry
+        // at the last round's start, through the rest
         if (rank == 0 && !dead) {
             float cv[2][4], ch[2][4];
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) { cv[c][e] = carry_at(c, e, 0); ch[c][e] = carry_at(c, e, 1); }
-            fold_records(cv, ch, sp.nseg_total);
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) { carry_at(c, e, 0) = cv[c][e]; carry_at(c, e, 1) = ch[c][e]; }
+            load_carry(cv, ch);
+            fold_records(cv, ch, sp.seg_first + (rounds - 1) * csize, sp.nseg_total);
+            store_carry(cv, ch);
         }
     }
     if (MODE != 1 && rank == 0 && !dead) {
@@ -907,8 +973,10 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, 
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
     attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
     cfg.attrs = attr;
-    // the split launches share nothing between CTAs: plain grids, placed freely
-    cfg.numAttrs = MODE == 0 ? 2 : 0;
+    // the split launches run as plain grids, placed freely, except the second
+    // launch of a piece after the first, whose tiles share one fold of the
+    // earlier pieces' records in a cluster
+    cfg.numAttrs = (MODE == 0 || (MODE == 2 && sp.seg_first > 0)) ? 2 : 0;
     return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize, sp);
 }
 
