@@ -124,9 +124,10 @@ typedef struct {
  *     pool the library creates per device on first use and keeps (up to
  *     64 MiB reserved between calls; cudaMallocFromPoolAsync, cudaFreeAsync
  *     on `stream`).  When that memory cannot be had (or records would pass
- *     1 GiB), and for in-place streaming (hT = h0 or vT = v0), it runs as one
- *     launch whose segments exchange their maps through distributed shared
- *     memory; both forms give bit-identical results.  mm_scan_fwd_noalloc
+ *     1 GiB), for in-place streaming (hT = h0 or vT = v0), and while `stream`
+ *     is being captured into a CUDA graph (nothing is allocated then), it
+ *     runs as one launch whose segments exchange their maps through
+ *     distributed shared memory; both forms give bit-identical results.  mm_scan_fwd_noalloc
  *     allocates nothing.
  *
  * Streaming: for a fixed (batch, dim, dstate, io), calling with the first

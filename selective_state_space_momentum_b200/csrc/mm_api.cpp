@@ -117,6 +117,14 @@ int inject_stall() {
     return (v && std::strcmp(v, "stall") == 0) ? 1 : 0;
 }
 
+// Test hook for the sequence-split path's fallback: with
+// MMSCAN_FAULT_INJECT=records its request for record memory asks for more
+// than any device holds, fails, and the call runs the fused launch.
+int inject_records_denied() {
+    const char* v = std::getenv("MMSCAN_FAULT_INJECT");
+    return (v && std::strcmp(v, "records") == 0) ? 1 : 0;
+}
+
 mm_status from_cuda(cudaError_t e, const char* what) {
     if (e == cudaSuccess) return ok();
     return fail(MM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
@@ -446,6 +454,7 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.ext = (Dskip || z || delta_bias || delta_softplus) ? 1 : 0;
     a.ckpt = ckpt;
     a.stall = inject_stall();
+    a.deny_records = inject_records_denied();
     if (!a.ext && !ckpt) {
         const int64_t seg = seg_len_for(bsz, L, D, N, dims->io, a.vec_ok != 0);
         if (seg > 0) {

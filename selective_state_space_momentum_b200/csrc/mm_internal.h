@@ -44,6 +44,7 @@ struct ScanArgs {
     int ext;               // any of the four is present
     float* ckpt;           // (batch, dim, ceil(L / 16), 2, dstate): (h, v) after every 16 steps, or null
     int stall;             // test only: stage no input, so that the bounded waits run out
+    int deny_records;      // test only: the sequence-split path's record memory request fails
 };
 
 // Arguments of one backward launch (device pointers; sizes as in mm_scan_dims).

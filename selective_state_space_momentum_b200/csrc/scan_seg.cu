@@ -947,14 +947,21 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, 
     if ((e = make_map_3d(&mB, Bs, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
     if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
     auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages, SC, MODE>;
+    // The shared-memory attribute of all three modes is set on the first launch
+    // of any on a device: a later call that switches to the fused launch (under
+    // graph capture, say) then makes no such call.
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_done.load(std::memory_order_acquire) & bit)) {
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM_BYTES)) !=
-            cudaSuccess)
-            return e;
+        const void* kerns[3] = {reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 0>),
+                                reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 1>),
+                                reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 2>)};
+        for (const void* k : kerns)
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM_BYTES)) !=
+                cudaSuccess)
+                return e;
         attr_done.fetch_or(bit, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
@@ -1051,14 +1058,22 @@ int64_t call_record_bytes(const ScanArgs& a, int64_t seg_len) {
 }  // namespace
 
 cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, bool fused, cudaStream_t s) {
-    if (!fused) {
+    // A stream being captured into a graph gets the fused launch: no pool is
+    // created and nothing is allocated while the capture is open.
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) {
+        (void)cudaGetLastError();
+        capture = cudaStreamCaptureStatusActive;
+    }
+    if (!fused && capture == cudaStreamCaptureStatusNone) {
         // The two-launch form: main passes with their maps to records in
         // stream-ordered memory, then the fold and correction.  Compiled
         // apart, the main pass runs 6% faster than inside the fused kernel.
         const int64_t bytes = call_record_bytes(a, seg_len);
         cudaMemPool_t pool = bytes > 0 ? records_pool() : nullptr;
         void* rec = nullptr;
-        if (pool && cudaMallocFromPoolAsync(&rec, (size_t)bytes, pool, s) == cudaSuccess) {
+        const size_t request = a.deny_records ? (size_t(1) << 62) : (size_t)bytes;
+        if (pool && cudaMallocFromPoolAsync(&rec, request, pool, s) == cudaSuccess) {
             SegSplit sp{};
             sp.maps = static_cast<float4*>(rec);
             sp.seg_first = 0;

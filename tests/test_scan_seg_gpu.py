@@ -212,3 +212,47 @@ def test_two_launch_and_fused_forms_are_bit_identical(seg_path, L, seg, beta, io
         mm.mm_device_status()
     for a, b, name in zip(out[2], out[3], ("y", "hT", "vT")):
         assert torch.equal(a, b), f"{name} differs between the two-launch and the fused form"
+
+
+def test_graph_capture_runs_the_fused_launch_and_replays(seg_path):
+    # a call captured into a CUDA graph allocates nothing: it records the fused launch,
+    # whose replay gives what the eager two-launch call gave
+    seg_path(128)
+    inp = _inputs(1, 2048, 32, 16, seed=61)
+    dev = _dev(inp, "f32")
+    rng = np.random.default_rng(6)
+    h0, v0 = (torch.from_numpy(a).cuda() for a in _states(rng, 1, 32, 16, 1.0))
+    y_ref, h_ref, v_ref = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0=h0, v0=v0, beta=0.95)
+    torch.cuda.synchronize()
+    y, hT, vT = torch.empty_like(y_ref), torch.empty_like(h_ref), torch.empty_like(v_ref)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        mm.mm_scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], h0, v0, 0.95, 1.0, y, hT, vT)
+    for _ in range(2):
+        y.zero_()
+        hT.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        mm.mm_device_status()
+        assert torch.equal(y, y_ref) and torch.equal(hT, h_ref) and torch.equal(vT, v_ref)
+    del g
+
+
+def test_record_memory_refused_runs_the_fused_launch(seg_path, monkeypatch):
+    # the request for record memory fails (test hook): the call runs the fused launch,
+    # bit-identical to it, and leaves no CUDA error behind for the next call to find
+    inp = _inputs(2, 3000, 40, 16, seed=71)
+    dev = _dev(inp, "f32")
+    seg_path(256, 3)
+    fused = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], beta=0.97)
+    seg_path(256, 2)
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "records")
+    got = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], beta=0.97)
+    monkeypatch.delenv("MMSCAN_FAULT_INJECT")
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    assert all(torch.equal(a, b) for a, b in zip(got, fused))
+    again = mm.scan_fwd(dev["x"], dev["delta"], dev["A"], dev["B"], dev["C"], beta=0.97)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(again, fused))
+    _check("f32", tuple(t.cpu().numpy() for t in got), inp, 0.97, 1.0, what="fallback")
