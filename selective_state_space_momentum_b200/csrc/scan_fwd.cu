@@ -238,6 +238,25 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     IO* yrow = static_cast<IO*>(p.y) + (b * p.dim + (active ? d : 0)) * L;
     const bool vec_out = use_tma;
 
+    // The gate z of the outputs a lane stores, read from global memory one chunk
+    // ahead into registers (ZC values a chunk): the reads of chunk k + 1 are in
+    // flight while chunk k runs, so the gate never waits on DRAM.
+    // (tiles with few lanes per channel apply many gates each: they read them in
+    // the group before, as the ragged chunk does, rather than hold a chunk's worth)
+    constexpr bool ZPRE = EXT && (TL::T / TL::R) * ZN <= 16;
+    constexpr int ZC = ZPRE ? (TL::T / TL::R) * ZN : 1;
+    float znext[ZC];
+    auto load_gates = [&](int64_t kz) {
+        if constexpr (ZPRE) {
+#pragma unroll
+            for (int i = 0; i < ZC; ++i) {
+                const int64_t tz = kz * T + (i / ZN) * TL::R + g * ZN + (i % ZN);
+                znext[i] = (zrow && active && tz < L) ? load1(zrow + tz) : 0.0f;
+            }
+        }
+    };
+    if (nchunks > 0) load_gates(0);
+
     for (int64_t k = 0; k < nchunks; ++k) {
         const int s = (int)(k % ST);
         const int64_t t0 = k * T;
@@ -312,6 +331,10 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         if (!__syncthreads_and(waited)) return;
         // Every thread is past compute(k-1): its stage and B^T/C^T buffers are free.
         if (k + ST - 1 < nchunks) issue(k + ST - 1, (int)((k + ST - 1) % ST));
+        float zcur[ZC];
+#pragma unroll
+        for (int i = 0; i < ZC; ++i) zcur[i] = znext[i];
+        if (ZPRE && k + 1 < nchunks) load_gates(k + 1);
 
         // ---- the recurrence over this chunk, R steps at a time -------------
         const float* Bg = Bt + g * SPT;
@@ -320,7 +343,9 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // Loads, delta*x and exponentials of the R steps of group gi.
         const bool dprime_bf16 = EXT && EB == 2 && (p.dbias || p.softplus);
         const unsigned char* dpb = smem + TL::OFF_DP + (int)(k & 1) * TL::DP_BYTES;
-        auto prep = [&](int gi, float (&u)[R], float (&a)[R][SPT], float (&zg)[ZN]) {
+        // (`full`: a full chunk, whose groups are unrolled, takes its gates from the
+        // registers read a chunk ahead; the ragged last chunk reads them here)
+        auto prep = [&](int gi, float (&u)[R], float (&a)[R][SPT], float (&zg)[ZN], bool full) {
             const int tau0 = gi * R;
             const int bx = tau0 / TL::BOX_T;
             const int col = tau0 - bx * TL::BOX_T;
@@ -339,11 +364,16 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 dl[j] = dq.x; dl[j + 1] = dq.y; dl[j + 2] = dq.z; dl[j + 3] = dq.w;
                 xl[j] = xq.x; xl[j + 1] = xq.y; xl[j + 2] = xq.z; xl[j + 3] = xq.w;
             }
-            if constexpr (EXT) {      // the gate of this lane's outputs, one group ahead
+            if constexpr (EXT) {      // the gate of this lane's outputs
+                if (ZPRE && full) {
 #pragma unroll
-                for (int e = 0; e < ZN; ++e) {
-                    const int64_t tz = t0 + tau0 + g * ZN + e;
-                    zg[e] = (zrow && active && tz < L) ? load1(zrow + tz) : 0.0f;
+                    for (int e = 0; e < ZN; ++e) zg[e] = zcur[(gi * ZN + e) % ZC];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < ZN; ++e) {
+                        const int64_t tz = t0 + tau0 + g * ZN + e;
+                        zg[e] = (zrow && active && tz < L) ? load1(zrow + tz) : 0.0f;
+                    }
                 }
             }
 #pragma unroll
@@ -461,7 +491,7 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const int tau0 = gi * R;
                 const int kmax = nval - tau0 < R ? nval - tau0 : R;
                 float u[R], a[R][SPT], yk[R], zg[ZN];
-                prep(gi, u, a, zg);
+                prep(gi, u, a, zg, false);
                 if (kmax == R) {
                     group_steps(gi, u, a, yk);
                 } else {
@@ -497,14 +527,14 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // Full chunk: groups unrolled, each group's exponentials issued one group ahead.
                 constexpr int NG = T / R;
                 float uA[R], uB[R], aA[R][SPT], aB[R][SPT], zA[ZN], zB[ZN];
-                prep(0, uA, aA, zA);
+                prep(0, uA, aA, zA, true);
 #pragma unroll
                 for (int gi = 0; gi < NG; ++gi) {
                     if ((gi & 1) == 0) {
-                        if (gi + 1 < NG) prep(gi + 1, uB, aB, zB);
+                        if (gi + 1 < NG) prep(gi + 1, uB, aB, zB, true);
                         full_steps(gi, uA, aA, zA);
                     } else {
-                        if (gi + 1 < NG) prep(gi + 1, uA, aA, zA);
+                        if (gi + 1 < NG) prep(gi + 1, uA, aA, zA, true);
                         full_steps(gi, uB, aB, zB);
                     }
                     if constexpr (CK)
@@ -526,8 +556,8 @@ scan_fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 constexpr int HALF = T / 2;
                 const int gi0 = 2 * j_t;
                 float uA[R], uB[R], aA[R][SPT], aB[R][SPT], yk[HALF], zd[ZN];
-                prep(gi0, uA, aA, zd);
-                prep(gi0 + 1, uB, aB, zd);
+                prep(gi0, uA, aA, zd, true);
+                prep(gi0 + 1, uB, aB, zd, true);
                 {
                     float y8[R];
                     group_steps(gi0, uA, aA, y8);
