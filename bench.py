@@ -710,14 +710,22 @@ def run_scan_split(args, w, beta, alpha, rank, world):
         clocks = clk.summary()
         sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or FALLBACK_SM_MAX_MHZ)
         mufu_peak, mufu_source = mufu_peak_now(sm_max)
-        # the roofline of one rank's share: its exponentials (its piece, once in the
-        # first launch) on its GPU's MUFU pipes
+        # the roofline of one rank's share: the slower of its exponentials (its piece,
+        # once in the first launch) on its GPU's MUFU pipes and its piece's bytes on HBM
         share = updates * n / w.seqlen
         t_mufu = share / mufu_peak
-        roof = {"bound": "alu", "kernel": "scan_seg_kernel", "achieved": share / (ms_step * 1e-3) / 1e9,
-                "peak": mufu_peak / 1e9, "unit": "Gex2/s", "frac": t_mufu / (ms_step * 1e-3),
-                "peak_source": mufu_source, "traffic": None,
-                "note": "rank 0's piece; the step includes the record exchange and the carry-in corrections"}
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        t_hbm = piece_bytes / (hbm_peak * 1e9)
+        note = "rank 0's piece; the step includes the record exchange and the carry-in corrections"
+        if t_mufu >= t_hbm:
+            roof = {"bound": "alu", "kernel": "scan_seg_kernel", "achieved": share / (ms_step * 1e-3) / 1e9,
+                    "peak": mufu_peak / 1e9, "unit": "Gex2/s", "frac": t_mufu / (ms_step * 1e-3),
+                    "peak_source": mufu_source, "traffic": None, "note": note}
+        else:
+            roof = {"bound": "hbm", "kernel": "scan_seg_kernel",
+                    "achieved": piece_bytes / (ms_step * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": t_hbm / (ms_step * 1e-3), "peak_source": f"{peak_kind} copy bandwidth",
+                    "traffic": None, "note": note}
         cb = None
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(w, beta, alpha)
