@@ -158,6 +158,16 @@ def timed_ms(step, steps: int, stream, step_bytes: int) -> float:
     FLUSH_BYTES that evicts L2 (and keeps the GPU busy while the host queues
     the step); the sum of the per-step times is returned."""
     import torch
+    # an NVTX range marks the timed steps for a profiler's timeline (ncu --nvtx)
+    torch.cuda.nvtx.range_push(f"timed {steps} steps")
+    try:
+        return _timed_ms(step, steps, stream, step_bytes)
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
+def _timed_ms(step, steps: int, stream, step_bytes: int) -> float:
+    import torch
     if not needs_flush(step_bytes):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
