@@ -658,9 +658,19 @@ def run_scan_split(args, w, beta, alpha, rank, world):
         s["all"] = torch.empty(world * per * rec, dtype=torch.uint8, device=dev) if world > 1 else s["maps"]
         sets.append(s)
     stream = torch.cuda.current_stream()
+    peers = (mm.SplitPeers(w.batch, w.dim, w.dstate, w.seqlen, S, io=io, device=dev)
+             if args.exchange == "peers" else None)
 
     def step(i):
         s = sets[i % nsets]
+        if peers is not None:
+            dests, local = peers.next()
+            mm.mm_scan_fwd_split_maps_peers(s["x"], s["delta"], s["A"], s["B"], s["C"], beta, alpha, s["y"],
+                                            dests, S, first, w.seqlen, stream)
+            peers.barrier()
+            mm.mm_scan_fwd_split_correct(s["delta"], s["A"], s["C"], None, None, beta, alpha, s["y"], s["hT"],
+                                         s["vT"], local, S, first, w.seqlen, stream)
+            return
         mm.mm_scan_fwd_split_maps(s["x"], s["delta"], s["A"], s["B"], s["C"], beta, alpha, s["y"], s["maps"], S,
                                   stream)
         if world > 1:
@@ -696,8 +706,12 @@ def run_scan_split(args, w, beta, alpha, rank, world):
 
     def e2e_step():
         d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
-        y, hT, vT = mm.scan_fwd_split(d["x"], d["delta"], d["A"], d["B"], d["C"], S, w.seqlen, beta=beta,
-                                      alpha=alpha)
+        if peers is not None:
+            y, hT, vT = mm.scan_fwd_split_peers(d["x"], d["delta"], d["A"], d["B"], d["C"], S, w.seqlen, peers,
+                                                beta=beta, alpha=alpha)
+        else:
+            y, hT, vT = mm.scan_fwd_split(d["x"], d["delta"], d["A"], d["B"], d["C"], S, w.seqlen, beta=beta,
+                                          alpha=alpha)
         out["y"].copy_(y, non_blocking=True)
         out["hT"].copy_(hT, non_blocking=True)
         out["vT"].copy_(vT, non_blocking=True)
@@ -741,8 +755,11 @@ def run_scan_split(args, w, beta, alpha, rank, world):
             cb = cpu_baseline(w, beta, alpha)
         cfg = scan_config(w, beta, alpha, 1)
         cfg.update(global_batch=w.batch, parallelism=f"sp{world}", l2=l2_note(piece_bytes, "piece"),
-                   split={"seg_len": S, "pieces": [list(p) for p in pieces], "exchange": "NCCL all-gather"
-                          if world > 1 else "none (one rank)"})
+                   split={"seg_len": S, "pieces": [list(p) for p in pieces],
+                          "exchange": ("none (one rank)" if world == 1 else
+                                       "records stored by the first launch into every rank's buffer (CUDA IPC "
+                                       "peer memory), NCCL all-reduce as the barrier"
+                                       if args.exchange == "peers" else "NCCL all-gather")})
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -756,6 +773,11 @@ def run_scan_split(args, w, beta, alpha, rank, world):
         if cb is not None:
             line["cpu_baseline"] = cb
         print(json.dumps(line), flush=True)
+    if peers is not None:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()            # every rank is done with the others' buffers
+        peers.close()
     return 0
 
 
@@ -1115,6 +1137,9 @@ def main(argv=None):
                     help="override the workload's sequence length (scan and SSD workloads)")
     ap.add_argument("--split-l", action="store_true",
                     help="scan workloads: the ranks share one sequence, split along time (strong scaling)")
+    ap.add_argument("--exchange", default="gather", choices=["gather", "peers"],
+                    help="--split-l: records all-gathered by NCCL, or stored by the first launch straight into "
+                         "every rank's buffer (CUDA IPC peer memory) with a barrier")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

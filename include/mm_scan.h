@@ -567,6 +567,53 @@ mm_status mm_scan_fwd_split_maps(const void *x, const void *delta, const float *
                                  const mm_scan_dims *dims, void *stream);
 
 /*
+ * mm_scan_fwd_split_maps_peers -- launch 1 of the split with the exchange
+ * folded into it: instead of into a buffer of the piece's own records, each
+ * segment's record is stored, at its global index seq_first / S + k, into
+ * every one of `ndest` buffers of the whole sequence's records -- the
+ * buffers launch 3 reads on each rank, reached as peer memory (CUDA IPC,
+ * mm_ipc_open_handle; over NVLink between GPUs).  After every rank's launch
+ * has completed (a stream-ordered barrier across the ranks, e.g. an NCCL
+ * all-reduce of one value), launch 3 runs on the local buffer; no gather of
+ * records is needed.  The kernel fences its stores at system scope before it
+ * completes.
+ *   x, delta, A, B, C, y, seg_len, dims: as mm_scan_fwd_split_maps;
+ *   dests      device memory: an array of ndest device pointers (8-byte
+ *              aligned), each to a 16-byte-aligned buffer of
+ *              mm_scan_split_maps_size(dims, ceil(seqlen_total / S)) bytes;
+ *   ndest      1 .. MM_SPLIT_MAX_RANKS;
+ *   seq_first, seqlen_total: the piece's place, as mm_scan_fwd_split_correct.
+ * Errors: as mm_scan_fwd_split_maps and mm_scan_fwd_split_correct's piece
+ * checks; MM_ERR_UNSUPPORTED for ndest out of range; MM_ERR_ALIGN for dests.
+ * The pointers in dests are not checked (device memory): each must be a
+ * buffer as stated.
+ */
+#define MM_SPLIT_MAX_RANKS 64
+mm_status mm_scan_fwd_split_maps_peers(const void *x, const void *delta, const float *A,
+                                       const void *B, const void *C, float beta, float alpha,
+                                       void *y, void *const *dests, int ndest,
+                                       int64_t seq_first, int64_t seg_len, int64_t seqlen_total,
+                                       const mm_scan_dims *dims, void *stream);
+
+/*
+ * CUDA IPC for the records buffers of the split (wrappers of
+ * cudaIpcGetMemHandle, cudaIpcOpenMemHandle with lazy peer access, and
+ * cudaIpcCloseMemHandle; the pages have no counterpart).  A handle names the
+ * whole allocation (cudaMalloc memory) that holds dev_ptr -- an allocator may
+ * hand out pieces of a larger one -- so mm_ipc_get_handle also returns dev_ptr's byte offset in
+ * it; the caller exchanges handle (MM_IPC_HANDLE_BYTES opaque bytes) and
+ * offset, mm_ipc_open_handle in another process returns the mapped
+ * allocation plus the offset, and mm_ipc_close_handle takes that pointer and
+ * the same offset.  A handle opens only in another process than the one that
+ * made it.  Errors: MM_ERR_NULL, MM_ERR_DIMS (negative offset), MM_ERR_CUDA
+ * (with CUDA's message in mm_last_error).
+ */
+#define MM_IPC_HANDLE_BYTES 64
+mm_status mm_ipc_get_handle(const void *dev_ptr, void *handle, int64_t *offset);
+mm_status mm_ipc_open_handle(const void *handle, int64_t offset, void **dev_ptr);
+mm_status mm_ipc_close_handle(void *dev_ptr, int64_t offset);
+
+/*
  * mm_scan_fwd_split_correct -- launch 3 of the split on `stream`.
  *   delta, A, C   the piece, as for launch 1 (read only);
  *   h0, v0        (batch, dim, dstate) fp32 state at step 0 of the whole

@@ -34,8 +34,9 @@ __all__ = [
     "mm_scan_fwd_host", "mm_scan_fwd_host_workspace_size", "mm_ssd_fwd_host",
     "mm_ssd_fwd_host_workspace_size",
     "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
-    "mm_scan_fwd_noalloc", "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
-    "ssd_fwd_host", "split_pieces", "scan_fwd_split",
+    "mm_scan_fwd_noalloc", "mm_scan_fwd_split_maps_peers", "mm_ipc_get_handle", "mm_ipc_open_handle",
+    "mm_ipc_close_handle", "SplitPeers", "mm_device_status", "scan_fwd", "scan_fwd_train", "scan_bwd", "ssd_fwd", "scan_fwd_host",
+    "ssd_fwd_host", "split_pieces", "scan_fwd_split", "scan_fwd_split_peers",
     "EXPORTED_SYMBOLS", "MM_SCAN_CKPT_STEPS",
 ]
 
@@ -64,7 +65,8 @@ EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm
                     "mm_scan_fwd_host_workspace_size", "mm_scan_fwd_host",
                     "mm_ssd_fwd_host_workspace_size", "mm_ssd_fwd_host",
                     "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
-                    "mm_scan_fwd_noalloc")
+                    "mm_scan_fwd_noalloc", "mm_scan_fwd_split_maps_peers", "mm_ipc_get_handle",
+                    "mm_ipc_open_handle", "mm_ipc_close_handle")
 
 
 class MMError(RuntimeError):
@@ -136,6 +138,15 @@ def _declare(lib):
     lib.mm_scan_fwd_split_correct.restype = ctypes.c_int
     lib.mm_scan_fwd_split_correct.argtypes = [vp, vp, vp, vp, vp, f, f, vp, vp, vp, vp, i64, i64, i64,
                                               ctypes.POINTER(ScanDims), vp]
+    lib.mm_scan_fwd_split_maps_peers.restype = ctypes.c_int
+    lib.mm_scan_fwd_split_maps_peers.argtypes = [vp, vp, vp, vp, vp, f, f, vp, vp, ctypes.c_int, i64, i64, i64,
+                                                 ctypes.POINTER(ScanDims), vp]
+    lib.mm_ipc_get_handle.restype = ctypes.c_int
+    lib.mm_ipc_get_handle.argtypes = [vp, vp, ctypes.POINTER(i64)]
+    lib.mm_ipc_open_handle.restype = ctypes.c_int
+    lib.mm_ipc_open_handle.argtypes = [vp, i64, ctypes.POINTER(ctypes.c_void_p)]
+    lib.mm_ipc_close_handle.restype = ctypes.c_int
+    lib.mm_ipc_close_handle.argtypes = [vp, i64]
     lib.mm_scan_fwd_noalloc.restype = ctypes.c_int
     lib.mm_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, f, f, vp, vp, vp, ctypes.POINTER(ScanDims), vp]
     lib.mm_status_string.restype = ctypes.c_char_p
@@ -531,6 +542,54 @@ def mm_scan_fwd_split_maps(x, delta, A, B, C, beta, alpha, y, maps, seg_len, str
     _check(rc, "mm_scan_fwd_split_maps")
 
 
+def mm_scan_fwd_split_maps_peers(x, delta, A, B, C, beta, alpha, y, dests, seg_len, seq_first, seqlen_total,
+                                 stream=None):
+    """C entry point mm_scan_fwd_split_maps_peers (marshalling only): the
+    split's first launch storing each segment record straight into every
+    buffer whose device pointer the int64 CUDA tensor `dests` holds."""
+    import torch
+    _require_scan(x, A, [("delta", delta, "io", False), ("B", B, "io_bc", False), ("C", C, "io_bc", False),
+                         ("y", y, "io", False)])
+    if not isinstance(dests, torch.Tensor) or dests.dtype != torch.int64 or dests.dim() != 1 or \
+            not dests.is_contiguous() or dests.device != x.device:
+        raise TypeError("dests must be a contiguous 1-D int64 tensor of device pointers on x's device")
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dims = ScanDims(batch, L, dim, N, _io_code(x.dtype))
+    rc = load_library().mm_scan_fwd_split_maps_peers(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), float(beta),
+                                                     float(alpha), _ptr(y), _ptr(dests), int(dests.numel()),
+                                                     int(seq_first), int(seg_len), int(seqlen_total),
+                                                     ctypes.byref(dims), _stream_handle(stream))
+    _check(rc, "mm_scan_fwd_split_maps_peers")
+
+
+MM_IPC_HANDLE_BYTES = 64
+
+
+def mm_ipc_get_handle(t):
+    """C entry point mm_ipc_get_handle: (handle bytes, byte offset) of a CUDA
+    tensor's memory within the allocation that holds it."""
+    buf = ctypes.create_string_buffer(MM_IPC_HANDLE_BYTES)
+    off = ctypes.c_int64(0)
+    _check(load_library().mm_ipc_get_handle(ctypes.c_void_p(t.data_ptr()), buf, ctypes.byref(off)),
+           "mm_ipc_get_handle")
+    return buf.raw, int(off.value)
+
+
+def mm_ipc_open_handle(handle: bytes, offset: int) -> int:
+    """C entry point mm_ipc_open_handle: a device pointer to another process's memory."""
+    if len(handle) != MM_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle is {MM_IPC_HANDLE_BYTES} bytes")
+    out = ctypes.c_void_p(0)
+    _check(load_library().mm_ipc_open_handle(ctypes.create_string_buffer(handle, MM_IPC_HANDLE_BYTES),
+                                             int(offset), ctypes.byref(out)), "mm_ipc_open_handle")
+    return int(out.value)
+
+
+def mm_ipc_close_handle(ptr: int, offset: int):
+    _check(load_library().mm_ipc_close_handle(ctypes.c_void_p(ptr), int(offset)), "mm_ipc_close_handle")
+
+
 def mm_scan_fwd_split_correct(delta, A, C, h0, v0, beta, alpha, y, hT, vT, maps_all, seg_len, seq_first,
                               seqlen_total, stream=None):
     """C entry point mm_scan_fwd_split_correct (marshalling only): fold the
@@ -862,5 +921,98 @@ def scan_fwd_split(x, delta, A, B, C, seg_len, seqlen_total, h0=None, v0=None, b
     hT = torch.empty((batch, dim, N), device=x.device, dtype=torch.float32)
     vT = torch.empty_like(hT)
     mm_scan_fwd_split_correct(delta, A, C, h0, v0, beta, alpha, y, hT, vT, gathered, seg_len, first,
+                              seqlen_total, stream)
+    return y, hT, vT
+
+
+class SplitPeers:
+    """The records buffers of a split whose exchange is done by the first
+    launch itself: every rank holds buffers of the whole sequence's records,
+    and every rank's first launch stores its records into all ranks' buffers
+    through peer pointers (CUDA IPC).  Two sets alternate from call to call:
+    a rank's next first launch writes into the set no rank can still be
+    reading (every rank passed the barrier of the call in between).
+    Collective over ``group``: every rank builds it with the same sizes and
+    makes the same calls.  ``close()`` releases the peer mappings."""
+
+    def __init__(self, batch, dim, dstate, seqlen_total, seg_len, io=MM_F32, group=None, device=None):
+        import torch
+        import torch.distributed as dist
+        self.group = group
+        if dist.is_available() and dist.is_initialized():
+            self.rank, self.world = dist.get_rank(group), dist.get_world_size(group)
+        else:
+            self.rank, self.world = 0, 1
+        device = device or torch.device("cuda", torch.cuda.current_device())
+        nseg = -(-int(seqlen_total) // int(seg_len))
+        self.nbytes = mm_scan_split_maps_size(batch, int(seqlen_total), dim, dstate, nseg, io)
+        self.locals = [torch.empty(self.nbytes, dtype=torch.uint8, device=device) for _ in range(2)]
+        self._opened = []
+        self.dests = []
+        for buf in self.locals:
+            ptrs = [0] * self.world
+            ptrs[self.rank] = buf.data_ptr()
+            if self.world > 1:
+                handles = [None] * self.world
+                dist.all_gather_object(handles, mm_ipc_get_handle(buf), group=group)
+                for r, (h, off) in enumerate(handles):
+                    if r != self.rank:
+                        ptrs[r] = mm_ipc_open_handle(h, off)
+                        self._opened.append((ptrs[r], off))
+            self.dests.append(torch.tensor(ptrs, dtype=torch.int64, device=device))
+        self._turn = 0
+
+    def next(self):
+        """(device array of every rank's buffer, this rank's buffer) of the next call."""
+        k = self._turn
+        self._turn ^= 1
+        return self.dests[k], self.locals[k]
+
+    def barrier(self, stream=None):
+        """Every rank's first launch has completed (stream-ordered for NCCL, on
+        the host for a backend without CUDA support)."""
+        import torch
+        import torch.distributed as dist
+        if self.world == 1:
+            return
+        dev = self.locals[0].device
+        if dist.get_backend(self.group) == "nccl":
+            # the collective runs on torch's current stream: order it after `stream`'s launch
+            cur = torch.cuda.current_stream(dev)
+            if stream is not None:
+                cur.wait_stream(stream)
+            flag = torch.zeros(1, device=dev)
+            dist.all_reduce(flag, group=self.group)
+            if stream is not None:
+                stream.wait_stream(cur)
+        else:
+            torch.cuda.synchronize(dev)
+            dist.barrier(group=self.group)
+
+    def close(self):
+        for p, off in self._opened:
+            mm_ipc_close_handle(p, off)
+        self._opened = []
+
+
+def scan_fwd_split_peers(x, delta, A, B, C, seg_len, seqlen_total, peers, h0=None, v0=None, beta=0.9, alpha=1.0,
+                         stream=None):
+    """scan_fwd_split with the exchange folded into the first launch: each
+    rank's records go straight into every rank's buffer (``peers``, a
+    SplitPeers built for these sizes), a barrier, then the second launch on
+    the local buffer.  Same results as scan_fwd_split, bit for bit."""
+    import torch
+    first, steps = split_pieces(int(seqlen_total), peers.world, int(seg_len))[peers.rank]
+    if x.dim() != 3 or x.shape[2] != steps:
+        raise ValueError(f"rank {peers.rank} holds steps [{first}, {first + steps}): x must be (batch, dim, {steps})")
+    batch, dim, _ = x.shape
+    N = A.shape[1]
+    y = torch.empty_like(x)
+    dests, local = peers.next()
+    mm_scan_fwd_split_maps_peers(x, delta, A, B, C, beta, alpha, y, dests, seg_len, first, seqlen_total, stream)
+    peers.barrier(stream)
+    hT = torch.empty((batch, dim, N), device=x.device, dtype=torch.float32)
+    vT = torch.empty_like(hT)
+    mm_scan_fwd_split_correct(delta, A, C, h0, v0, beta, alpha, y, hT, vT, local, seg_len, first,
                               seqlen_total, stream)
     return y, hT, vT

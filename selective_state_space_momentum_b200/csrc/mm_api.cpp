@@ -203,9 +203,9 @@ mm_status check_split(const mm_scan_dims* dims, const ScanSizes& zs, int64_t seg
                     (long long)dims->seqlen);
     if (seqlen_total < 1 || seqlen_total > kMaxSeqlen)
         return fail(MM_ERR_UNSUPPORTED, "seqlen_total=%lld is outside [1, 2^30]", (long long)seqlen_total);
-    if (seq_first < 0 || seq_first % seg_len != 0 || seq_first + dims->seqlen > seqlen_total)
-        return fail(MM_ERR_UNSUPPORTED, "piece [%lld, %lld) does not start at a multiple of %lld within %lld steps",
-                    (long long)seq_first, (long long)(seq_first + dims->seqlen), (long long)seg_len,
+    if (seq_first < 0 || seq_first % seg_len != 0 || seq_first > seqlen_total - dims->seqlen)
+        return fail(MM_ERR_UNSUPPORTED, "a piece of %lld steps at step %lld does not start at a multiple of %lld "
+                    "within %lld steps", (long long)dims->seqlen, (long long)seq_first, (long long)seg_len,
                     (long long)seqlen_total);
     if (seq_first + dims->seqlen < seqlen_total && dims->seqlen % seg_len != 0)
         return fail(MM_ERR_UNSUPPORTED, "a piece before the last must hold whole segments (seqlen=%lld, S=%lld)",
@@ -346,9 +346,43 @@ mm_status mm_scan_fwd_split_maps(const void* x, const void* delta, const float* 
     a.beta = beta; a.alpha = alpha;
     a.vec_ok = 1;
     a.stall = inject_stall();
-    return from_cuda(mmscan::launch_scan_seg_split(a, dims->io, seg_len, 1, maps, 0, dims->seqlen,
+    return from_cuda(mmscan::launch_scan_seg_split(a, dims->io, seg_len, 1, maps, 0, dims->seqlen, nullptr, 0,
                                                    static_cast<cudaStream_t>(stream)),
                      "mm_scan_fwd_split_maps launch");
+}
+
+mm_status mm_scan_fwd_split_maps_peers(const void* x, const void* delta, const float* A, const void* B,
+                                       const void* C, float beta, float alpha, void* y, void* const* dests,
+                                       int ndest, int64_t seq_first, int64_t seg_len, int64_t seqlen_total,
+                                       const mm_scan_dims* dims, void* stream) {
+    if (!dims) return fail(MM_ERR_NULL, "dims is NULL");
+    if (!x || !delta || !A || !B || !C || !y || !dests)
+        return fail(MM_ERR_NULL, "x, delta, A, B, C, y and dests are required");
+    if (ndest < 1 || ndest > MM_SPLIT_MAX_RANKS)
+        return fail(MM_ERR_UNSUPPORTED, "ndest=%d is outside [1, %d]", ndest, MM_SPLIT_MAX_RANKS);
+    ScanSizes zs;
+    if (mm_status st = check_scan_dims(dims, beta, alpha, &zs)) return st;
+    if (mm_status st = check_split(dims, zs, seg_len, seq_first, seqlen_total)) return st;
+    const void* ptrs[] = {x, delta, A, B, C, y};
+    const char* names[] = {"x", "delta", "A", "B", "C", "y"};
+    for (int i = 0; i < 6; ++i)
+        if (!aligned16(ptrs[i])) return fail(MM_ERR_ALIGN, "%s is not 16-byte aligned", names[i]);
+    if ((reinterpret_cast<uintptr_t>(dests) & 7u) != 0) return fail(MM_ERR_ALIGN, "dests is not 8-byte aligned");
+    const Range ry = rng("y", y, zs.seq_bytes);
+    const Range ins[] = {rng("x", x, zs.seq_bytes), rng("delta", delta, zs.seq_bytes), rng("A", A, zs.a_bytes),
+                         rng("B", B, zs.bc_bytes), rng("C", C, zs.bc_bytes)};
+    for (const Range& in : ins)
+        if (overlap(ry, in)) return fail(MM_ERR_ALIAS, "y overlaps %s", in.name);
+    if (inject_launch_failure()) return fail(MM_ERR_CUDA, "injected launch failure (MMSCAN_FAULT_INJECT)");
+    mmscan::ScanArgs a{};
+    a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.y = y;
+    a.batch = dims->batch; a.seqlen = dims->seqlen; a.dim = dims->dim; a.dstate = (int)dims->dstate;
+    a.beta = beta; a.alpha = alpha;
+    a.vec_ok = 1;
+    a.stall = inject_stall();
+    return from_cuda(mmscan::launch_scan_seg_split(a, dims->io, seg_len, 1, nullptr, seq_first / seg_len,
+                                                   seqlen_total, dests, ndest, static_cast<cudaStream_t>(stream)),
+                     "mm_scan_fwd_split_maps_peers launch");
 }
 
 mm_status mm_scan_fwd_split_correct(const void* delta, const float* A, const void* C, const float* h0,
@@ -386,7 +420,7 @@ mm_status mm_scan_fwd_split_correct(const void* delta, const float* A, const voi
     a.vec_ok = 1;
     a.stall = inject_stall();
     return from_cuda(mmscan::launch_scan_seg_split(a, dims->io, seg_len, 2, const_cast<void*>(maps_all),
-                                                   seq_first / seg_len, seqlen_total,
+                                                   seq_first / seg_len, seqlen_total, nullptr, 0,
                                                    static_cast<cudaStream_t>(stream)),
                      "mm_scan_fwd_split_correct launch");
 }

@@ -133,8 +133,11 @@ int64_t scan_seg_chunk_steps(int io);
 // first segment).
 int64_t scan_seg_tile_channels();
 int64_t scan_seg_tile_record_bytes();
+// (mode 1 with ndest > 0: the records go to the ndest buffers whose device
+// pointers `dests` (a device array) holds, at their global index)
 cudaError_t launch_scan_seg_split(const ScanArgs& a, int io, int64_t seg_len, int mode, void* maps,
-                                  int64_t seg_first, int64_t seqlen_total, cudaStream_t s);
+                                  int64_t seg_first, int64_t seqlen_total, void* const* dests, int ndest,
+                                  cudaStream_t s);
 unsigned int scan_seg_read_and_clear_device_error();
 
 bool scan_tile_supported(int spt, int warps, int time_lanes);

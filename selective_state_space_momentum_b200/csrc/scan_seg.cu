@@ -156,9 +156,14 @@ __device__ __forceinline__ float pow_steps(float beta, int64_t n) {
 // had no negative value; MODE 0 is the fused kernel above.
 struct SegSplit {
     float4* maps;             // MODE 1: this call's records; MODE 2: every segment's records (read only)
-    int64_t seg_first;        // MODE 2: global index of this call's first segment
+    int64_t seg_first;        // global index of this call's first segment
     int64_t nseg_total;       // MODE 2: segments of the whole sequence
     int64_t L_total;          // MODE 2: steps of the whole sequence
+    // MODE 1 with ndest > 0: each record goes, at its global index, straight into
+    // every rank's buffer of the whole sequence's records (device pointers, peer
+    // memory over NVLink included) instead of into `maps`
+    float4* const* dests;
+    int ndest;
 };
 
 // Scaled form (SC, used for beta >= 1/2).  Within a chunk of T steps the
@@ -750,7 +755,7 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         if constexpr (MODE == 1) {
             // the split's first launch: this segment's map and delta-sign flag to its record
             if (!dead && slen > 0) {
-                float4* rec = sp.maps + (k * ncl + (int64_t)(blockIdx.x / csize)) * REC;
+                float4 m[8];
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -758,10 +763,21 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         const float P0 = ex2_approx(Al[c][2 * q] * dsum[c]);
                         const float P1 = ex2_approx(Al[c][2 * q + 1] * dsum[c]);
                         const int i0 = (c * 2 + q) * 2;
-                        rec[i0 * NT + tid] = make_float4(vv[c][q].x, vv[c][q].y, hh[c][q].x, hh[c][q].y);
-                        rec[(i0 + 1) * NT + tid] = make_float4(qq[c][q].x, qq[c][q].y, P0, P1);
+                        m[i0] = make_float4(vv[c][q].x, vv[c][q].y, hh[c][q].x, hh[c][q].y);
+                        m[i0 + 1] = make_float4(qq[c][q].x, qq[c][q].y, P0, P1);
                     }
-                if (tid == 0) rec[8 * NT] = make_float4(seg_nonneg ? 1.0f : 0.0f, 0.0f, 0.0f, 0.0f);
+                const float4 flag = make_float4(seg_nonneg ? 1.0f : 0.0f, 0.0f, 0.0f, 0.0f);
+                const int64_t cli = (int64_t)(blockIdx.x / csize);
+                auto put = [&](float4* rec) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) rec[i * NT + tid] = m[i];
+                    if (tid == 0) rec[8 * NT] = flag;
+                };
+                if (sp.ndest > 0) {
+                    for (int r = 0; r < sp.ndest; ++r) put(sp.dests[r] + ((sp.seg_first + k) * ncl + cli) * REC);
+                } else {
+                    put(sp.maps + (k * ncl + cli) * REC);
+                }
             }
             continue;                     // no fold and no correction in this launch
         }
@@ -903,6 +919,11 @@ scan_seg_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             fold_records(cv, ch, sp.seg_first + (rounds - 1) * csize, sp.nseg_total);
             store_carry(cv, ch);
         }
+    }
+    if constexpr (MODE == 1) {
+        // records written into other ranks' memory are visible there before the
+        // kernel is seen complete
+        if (sp.ndest > 0) __threadfence_system();
     }
     if (MODE != 1 && rank == 0 && !dead) {
 #pragma unroll
@@ -1103,9 +1124,12 @@ int64_t scan_seg_tile_record_bytes() {
 }
 
 cudaError_t launch_scan_seg_split(const ScanArgs& a, int io, int64_t seg_len, int mode, void* maps,
-                                  int64_t seg_first, int64_t seqlen_total, cudaStream_t s) {
+                                  int64_t seg_first, int64_t seqlen_total, void* const* dests, int ndest,
+                                  cudaStream_t s) {
     SegSplit sp{};
     sp.maps = static_cast<float4*>(maps);
+    sp.dests = reinterpret_cast<float4* const*>(dests);
+    sp.ndest = ndest;
     sp.seg_first = seg_first;
     sp.L_total = seqlen_total;
     sp.nseg_total = (seqlen_total + seg_len - 1) / seg_len;

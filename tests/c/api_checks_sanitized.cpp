@@ -46,7 +46,8 @@ cudaError_t launch_scan_seg(const ScanArgs&, int, int64_t, bool, cudaStream_t) {
 int64_t scan_seg_chunk_steps(int io) { return io == 0 ? 32 : 64; }
 int64_t scan_seg_tile_channels() { return 16; }
 int64_t scan_seg_tile_record_bytes() { return 257 * 16; }
-cudaError_t launch_scan_seg_split(const ScanArgs&, int, int64_t, int, void*, int64_t, int64_t, cudaStream_t) {
+cudaError_t launch_scan_seg_split(const ScanArgs&, int, int64_t, int, void*, int64_t, int64_t, void* const*, int,
+                                  cudaStream_t) {
     ++g_launches;
     return cudaSuccess;
 }
@@ -109,15 +110,25 @@ void scan_calls(const mm_scan_dims& d, float beta, float alpha) {
     expect_status(mm_scan_segment_len(&d, &seg), "mm_scan_segment_len");
     // the split launches, with their segment length and the piece's place at extremes
     for (int64_t S : {int64_t(-1), int64_t(0), int64_t(32), int64_t(64), int64_t(1) << 30, int64_t(1) << 62})
-        for (int64_t first : {int64_t(-64), int64_t(0), int64_t(64), int64_t(1) << 30, int64_t(1) << 62})
+        for (int64_t first : {int64_t(-64), int64_t(0), int64_t(64), int64_t(1) << 30, int64_t(1) << 62,
+                              std::numeric_limits<int64_t>::max() - 1})
             for (int64_t total : {int64_t(0), int64_t(64), d.seqlen, int64_t(1) << 30, std::numeric_limits<int64_t>::max()}) {
                 expect_status(mm_scan_fwd_split_correct(fake(1), ffake(2), fake(4), ffake(5), ffake(6), beta, alpha,
                                                         fake(7), ffake(8), ffake(9), fake(10), S, first, total, &d,
                                                         nullptr), "mm_scan_fwd_split_correct");
             }
-    for (int64_t S : {int64_t(-1), int64_t(32), int64_t(64), int64_t(1) << 30, int64_t(1) << 62})
+    for (int64_t S : {int64_t(-1), int64_t(32), int64_t(64), int64_t(1) << 30, int64_t(1) << 62}) {
         expect_status(mm_scan_fwd_split_maps(fake(0), fake(1), ffake(2), fake(3), fake(4), beta, alpha, fake(7),
                                              fake(10), S, &d, nullptr), "mm_scan_fwd_split_maps");
+        for (int nd : {0, 1, 65})
+            for (int64_t first : {int64_t(0), int64_t(1) << 40})
+                expect_status(mm_scan_fwd_split_maps_peers(fake(0), fake(1), ffake(2), fake(3), fake(4), beta, alpha,
+                                                           fake(7), reinterpret_cast<void* const*>(fake(11)), nd,
+                                                           first, S,
+                                                           d.seqlen > INT64_MAX - first ? INT64_MAX : first + d.seqlen,
+                                                           &d, nullptr),
+                              "mm_scan_fwd_split_maps_peers");
+    }
     for (int64_t n : {int64_t(-1), int64_t(0), int64_t(1), int64_t(1) << 30, int64_t(1) << 31})
         expect_status(mm_scan_split_maps_size(&d, n, &bytes), "mm_scan_split_maps_size");
 }

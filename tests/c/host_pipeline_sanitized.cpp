@@ -385,7 +385,8 @@ cudaError_t launch_ssd_mom(const SSDMomArgs& a, cudaStream_t s) {
 int64_t scan_seg_chunk_steps(int io) { return io == 0 ? 32 : 64; }
 int64_t scan_seg_tile_channels() { return 16; }
 int64_t scan_seg_tile_record_bytes() { return 257 * 16; }
-cudaError_t launch_scan_seg_split(const ScanArgs&, int, int64_t, int, void*, int64_t, int64_t, cudaStream_t) {
+cudaError_t launch_scan_seg_split(const ScanArgs&, int, int64_t, int, void*, int64_t, int64_t, void* const*, int,
+                                  cudaStream_t) {
     return cudaErrorInvalidValue;
 }
 unsigned int scan_seg_read_and_clear_device_error() { return 0; }

@@ -307,6 +307,27 @@ def test_split_sizes_and_checks(lib, monkeypatch):
     assert correct(first=128, total=300) == 7                     # the last piece may be partial
 
 
+def test_peer_split_and_ipc_checks(lib, monkeypatch):
+    dims = D(L=128)
+    call = lambda nd, first=0, total=128, dests=_fake(9): lib.mm_scan_fwd_split_maps_peers(
+        _fake(0), _fake(1), _fake(2), _fake(3), _fake(4), 0.9, 1.0, _fake(5), dests, nd, first, 64, total,
+        ctypes.byref(dims), None)
+    assert call(0) == 6 and call(65) == 6                         # 1 .. MM_SPLIT_MAX_RANKS destinations
+    assert call(2, dests=None) == 1
+    assert call(2, dests=ctypes.c_void_p(A16 * 10 + 4)) == 5      # the pointer array is 8-byte aligned
+    assert call(2, first=32, total=256) == 6                      # piece off a segment boundary
+    monkeypatch.setenv("MMSCAN_FAULT_INJECT", "launch")
+    assert call(2, first=128, total=256) == 7                     # in range: reaches the launch step
+    monkeypatch.delenv("MMSCAN_FAULT_INJECT")
+    off = ctypes.c_int64(0)
+    ptr = ctypes.c_void_p(0)
+    handle = ctypes.create_string_buffer(64)
+    assert lib.mm_ipc_get_handle(None, handle, ctypes.byref(off)) == 1
+    assert lib.mm_ipc_open_handle(None, 0, ctypes.byref(ptr)) == 1
+    assert lib.mm_ipc_open_handle(handle, -16, ctypes.byref(ptr)) == 2
+    assert lib.mm_ipc_close_handle(None, 0) == 1
+
+
 def test_ssd_rejects_bad_arguments(lib, monkeypatch):
     dims = mm.SSDDims(1, 512, 4, 64, 128, 1, 256)
 

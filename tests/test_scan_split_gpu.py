@@ -17,8 +17,14 @@ with the same segment length, and match the fp64 oracle at the scan's
 tolerances:
   * fp32 I/O: max |y - y_ref| <= 1e-4 * max |y_ref| (also hT, vT);
   * bf16 I/O: ||y - y_ref||_2 / ||y_ref||_2 <= 1e-2, states at fp32 bound.
-A last test runs the wrapper scan_fwd_split in two processes joined by a
-gloo group (records exchanged through host memory), each on its own piece.
+The exchange can also be folded into the first launch
+(mm_scan_fwd_split_maps_peers): each piece's records are stored straight
+into every rank's buffer of the whole sequence's records.  That form is
+emulated the same way, each emulated rank with a buffer of its own.  The
+last tests run the wrappers scan_fwd_split (records gathered through host
+memory) and scan_fwd_split_peers (records stored into the other process's
+buffer through CUDA IPC) in two processes on this GPU joined by a gloo group,
+each on its own piece.
 """
 import os
 import socket
@@ -176,13 +182,59 @@ def test_split_records_are_what_the_first_launch_wrote():
     assert torch.equal(y[..., 256:], y2)           # the zero-start read-out of the same segments
 
 
+def _emulate_peers(dev, h0, v0, beta, alpha, S, world):
+    """The split with the exchange in the first launch: every emulated rank
+    stores its records into every rank's own buffer, then corrects from its
+    own buffer."""
+    batch, dim, L = dev["x"].shape
+    N = dev["A"].shape[1]
+    io = mm.MM_F32 if dev["x"].dtype == torch.float32 else mm.MM_BF16
+    pieces = mm.split_pieces(L, world, S)
+    nbytes = mm.mm_scan_split_maps_size(batch, L, dim, N, -(-L // S), io)
+    bufs = [torch.full((nbytes,), 0xff, dtype=torch.uint8, device="cuda") for _ in range(world)]
+    dests = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device="cuda")
+    sl = [{k: dev[k][..., f:f + n].contiguous() for k in ("x", "delta", "B", "C")} for f, n in pieces]
+    ys = []
+    for (first, _), p in zip(pieces, sl):
+        y = torch.empty_like(p["x"])
+        mm.mm_scan_fwd_split_maps_peers(p["x"], p["delta"], dev["A"], p["B"], p["C"], beta, alpha, y, dests, S,
+                                        first, L)
+        ys.append(y)
+    torch.cuda.synchronize()
+    for b in bufs[1:]:
+        assert torch.equal(b, bufs[0]), "the ranks' record buffers differ"
+    states = []
+    for r, ((first, _), p, y) in enumerate(zip(pieces, sl, ys)):
+        hT = torch.empty((batch, dim, N), device="cuda")
+        vT = torch.empty_like(hT)
+        mm.mm_scan_fwd_split_correct(p["delta"], dev["A"], p["C"], h0, v0, beta, alpha, y, hT, vT, bufs[r], S,
+                                     first, L)
+        states.append((hT, vT))
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    return torch.cat(ys, dim=-1), states
+
+
+@pytest.mark.parametrize("L,S,world,io", [(1024, 64, 2, "f32"), (1000, 64, 3, "f32"), (2048, 128, 4, "bf16"),
+                                          (768, 256, 1, "f32")])
+def test_records_stored_into_every_rank_buffer(L, S, world, io):
+    inp = _inputs(2, L, 40, 16, seed=L * 3 + world, io=io)
+    dev = _dev(inp, io)
+    h0, v0 = (torch.from_numpy(a).cuda() for a in _states(2, 40, 16, seed=world + 10))
+    y, states = _emulate_peers(dev, h0, v0, 0.95, 1.0, S, world)
+    y1, h1, v1 = _one_call(dev, h0, v0, 0.95, 1.0, S)
+    assert torch.equal(y, y1), "y of the peer-exchange split differs from one call"
+    for hT, vT in states:
+        assert torch.equal(hT, h1) and torch.equal(vT, v1)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, exchange="gather"):
     import datetime
 
     import torch.distributed as dist
@@ -196,8 +248,18 @@ def _worker(rank, world, port, q):
         h0, v0 = (torch.from_numpy(a).cuda() for a in _states(2, 48, 16, seed=78))
         first, n = mm.split_pieces(L, world, S)[rank]
         p = {k: dev[k][..., first:first + n].contiguous() for k in ("x", "delta", "B", "C")}
-        y, hT, vT = mm.scan_fwd_split(p["x"], p["delta"], dev["A"], p["B"], p["C"], S, L, h0=h0, v0=v0,
-                                      beta=0.95, alpha=1.0)
+        if exchange == "peers":
+            peers = mm.SplitPeers(2, 48, 16, L, S)
+            runs = [mm.scan_fwd_split_peers(p["x"], p["delta"], dev["A"], p["B"], p["C"], S, L, peers, h0=h0,
+                                            v0=v0, beta=0.95, alpha=1.0) for _ in range(3)]   # both buffer sets
+            torch.cuda.synchronize()
+            dist.barrier()            # the other rank has read its records before the mapping goes
+            peers.close()
+            y, hT, vT = runs[-1]
+            assert all(torch.equal(a, b) for r in runs[:-1] for a, b in zip(r, runs[-1]))
+        else:
+            y, hT, vT = mm.scan_fwd_split(p["x"], p["delta"], dev["A"], p["B"], p["C"], S, L, h0=h0, v0=v0,
+                                          beta=0.95, alpha=1.0)
         torch.cuda.synchronize()
         mm.mm_device_status()
         y1, h1, v1 = _one_call(dev, h0, v0, 0.95, 1.0, S)
@@ -215,11 +277,12 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_split_one_sequence():
+@pytest.mark.parametrize("exchange", ["gather", "peers"])
+def test_two_gloo_ranks_split_one_sequence(exchange):
     ctx = torch.multiprocessing.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, exchange)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
