@@ -256,3 +256,29 @@ def test_record_memory_refused_runs_the_fused_launch(seg_path, monkeypatch):
     torch.cuda.synchronize()
     assert all(torch.equal(a, b) for a, b in zip(again, fused))
     _check("f32", tuple(t.cpu().numpy() for t in got), inp, 0.97, 1.0, what="fallback")
+
+
+def test_concurrent_calls_on_two_streams_keep_their_own_records(seg_path):
+    # the two-launch form's records come from stream-ordered memory: calls on two
+    # streams at once each get their own, and give what they give one at a time
+    seg_path(128)
+    a = _dev(_inputs(1, 4096, 48, 16, seed=81), "f32")
+    b = _dev(_inputs(1, 4096, 48, 16, seed=82), "f32")
+    ref_a = mm.scan_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], beta=0.97)
+    ref_b = mm.scan_fwd(b["x"], b["delta"], b["A"], b["B"], b["C"], beta=0.97)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    s1.wait_stream(torch.cuda.current_stream())
+    s2.wait_stream(torch.cuda.current_stream())
+    outs = []
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            ga = mm.scan_fwd(a["x"], a["delta"], a["A"], a["B"], a["C"], beta=0.97, stream=s1)
+        with torch.cuda.stream(s2):
+            gb = mm.scan_fwd(b["x"], b["delta"], b["A"], b["B"], b["C"], beta=0.97, stream=s2)
+        outs.append((ga, gb))
+    torch.cuda.synchronize()
+    mm.mm_device_status()
+    for ga, gb in outs:
+        assert all(torch.equal(p, q) for p, q in zip(ga, ref_a))
+        assert all(torch.equal(p, q) for p, q in zip(gb, ref_b))
