@@ -293,3 +293,23 @@ def test_two_gloo_ranks_split_one_sequence(exchange):
     for d in res:
         assert d["same_y"] and d["same_states"], d
         assert d["y_err"] <= F32_TOL and d["h_err"] <= F32_TOL, d
+
+
+def test_long_workload_over_eight_emulated_ranks():
+    # the long streaming workload (B1 L131072 D2048 N16, beta 0.99) cut over eight ranks
+    # with 2048-step segments, as bench.py --split-l at eight GPUs cuts it: bit-identical
+    # to one call with the same segments, and a channel sample within the oracle's tolerance
+    w = wl.SCAN_LONG
+    inp = wl.scan_inputs(w, seed=wl.seed_of(w.seed_index))
+    dev = {k: torch.from_numpy(inp[k]).cuda().contiguous() for k in ("x", "delta", "B", "C", "A")}
+    y, states = _emulate(dev, None, None, 0.99, 1.0, 2048, 8)
+    y1, h1, v1 = _one_call(dev, None, None, 0.99, 1.0, 2048)
+    assert torch.equal(y, y1), "y of the eight-rank split differs from one call"
+    assert all(torch.equal(h, h1) and torch.equal(v, v1) for h, v in states)
+    rng = np.random.default_rng(8)
+    chan = np.sort(rng.choice(w.dim, 24, replace=False))
+    yr, hr, vr = oracle.scan_seq(**inp, beta=0.99, alpha=1.0, chan=chan)
+    yg = y.cpu().numpy().reshape(-1, w.seqlen)[chan]
+    assert np.abs(yg - yr).max() <= F32_TOL * np.abs(yr).max()
+    hg = states[0][0].cpu().numpy().reshape(-1, w.dstate)[chan]
+    assert np.abs(hg - hr).max() <= F32_TOL * np.abs(hr).max()
