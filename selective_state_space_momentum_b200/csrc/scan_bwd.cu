@@ -29,8 +29,10 @@
 //  * Reductions.  The sums over a channel's states (for dx, ddelta) use the
 //    forward's register butterfly.  dB and dC sum over channels: a butterfly
 //    across the channels of a warp (four steps at a time, so the exchanges
-//    are independent), shared-memory atomics across the warps into one of
-//    two buffers, then one vector atomic add per (4 steps, state) into global
+//    are independent) into the warp's own slice of one of two buffers, the
+//    slices summed when a block is flushed (tiles whose CTAs would then not fit
+//    at full occupancy add into one slice with shared-memory atomics), then one
+//    vector atomic add per (4 steps, state) into global
 //    memory after each block.  dA collects in registers over the whole sequence and is added
 //    once per lane.
 //  * Staging: x, delta, dy, B and C tiles by TMA (128-byte swizzle, no
@@ -80,19 +82,26 @@ struct BwdTile {
     static constexpr int RP = 2 * NP;            // dB and dC partials per step
     static constexpr int OFF_BT = STAGES * STAGE_BYTES;   // B^T, then C^T
     static constexpr int OFF_RED = OFF_BT + 2 * BT_BYTES;
-    static constexpr int RED_BYTES = 2 * KB * RP * 4;   // two blocks' dB, dC partials
     // extras: delta' = softplus(delta + bias) and the gated dy = dy silu(z) of
     // the chunk as fp32 in the fp32 box layout (32 steps x CH rows of 128 B)
     static constexpr int XBOX_F32 = CH * 128;
     static constexpr int EXB = EXT ? (T / 32) * XBOX_F32 : 0;
-    static constexpr int OFF_DP = OFF_RED + RED_BYTES;
-    static constexpr int OFF_GY = OFF_DP + EXB;
-    static constexpr int OFF_BAR = OFF_GY + EXB;
-    static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
     // 12 resident warps per SM (<= 168 registers a thread, no spills).  Four
     // 4-warp CTAs would fit the shared memory, but at 128 registers the
     // kernel spills and ran 33% slower on the 384-CTA fp32 grid.
     static constexpr int MIN_CTAS = 12 / WARPS > 0 ? 12 / WARPS : 1;
+    // Two blocks' dB, dC partials: one slice per warp, summed when a block is
+    // flushed, where MIN_CTAS CTAs of that size still fit an SM; else one
+    // slice that the warps add into with shared-memory atomics.
+    static constexpr int smem_with(int red_warps) {
+        return OFF_RED + 2 * red_warps * KB * RP * 4 + 2 * EXB + STAGES * 8 + 1024;
+    }
+    static constexpr int RED_WARPS = MIN_CTAS * (smem_with(WARPS) + 1024) <= 228 * 1024 ? WARPS : 1;
+    static constexpr int RED_BYTES = 2 * RED_WARPS * KB * RP * 4;
+    static constexpr int OFF_DP = OFF_RED + RED_BYTES;
+    static constexpr int OFF_GY = OFF_DP + EXB;
+    static constexpr int OFF_BAR = OFF_GY + EXB;
+    static constexpr int SMEM_BYTES = OFF_BAR + STAGES * 8 + 1024;   // + alignment slack
 
     static_assert(G >= 1 && G <= 8 && (G & (G - 1)) == 0, "lanes per channel");
     static_assert(R % G == 0 && BOX_T % R == 0 && T % BOX_T == 0 && KB % R == 0 && T % KB == 0,
@@ -141,7 +150,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int s = 0; s < ST; ++s) mbar_init(bar0 + 8 * s, use_tma ? 1u : (uint32_t)NT);
         fence_barrier_init();
     }
-    for (int i = tid; i < 2 * KB * RP; i += NT) red[i] = 0.0f;
+    for (int i = tid; i < 2 * TL::RED_WARPS * KB * RP; i += NT) red[i] = 0.0f;
     int nred = 0;                                    // blocks done: picks the partials buffer
     __syncthreads();
 
@@ -374,7 +383,9 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         };
         // dB, dC partials of 4 consecutive steps from tau: summed over the
         // warp's channels by a butterfly (the lane keeps dB or dC, then one of
-        // its two states), then over the warps by shared-memory atomics
+        // its two states) and stored into the warp's slice (each slot of a step
+        // has one writer in the warp; shared-memory atomics across the warps
+        // had cost a fifth of the kernel's time)
         auto chan_reduce4 = [&](float* redb, int tau, const float2 (&dBv)[4], const float2 (&dCv)[4]) {
             const bool up1 = (lane & 16) != 0;
             const bool up2 = (lane & 8) != 0;
@@ -395,7 +406,10 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if ((lane & 7) < G) {
                 float* dst = redb + tau * RP + (up1 ? NP : 0) + n0 + (up2 ? 1 : 0);
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) atomicAdd(dst + jj * RP, r[jj]);
+                for (int jj = 0; jj < 4; ++jj) {
+                    if constexpr (TL::RED_WARPS > 1) dst[jj * RP] = r[jj];
+                    else atomicAdd(dst + jj * RP, r[jj]);
+                }
             }
         };
         // One block of KB steps (the first kmax valid) from its start state:
@@ -469,7 +483,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                 cp = __fmul2_rn(beta2, Pt);
                             }
                         }
-                        chan_reduce4(redb, jb, dBv, dCv);
+                        chan_reduce4(redb + (TL::RED_WARPS > 1 ? warp : 0) * (KB * RP), jb, dBv, dCv);
                     }
                 }
                 // per-channel sums of these R steps; lane g owns PER of them
@@ -529,7 +543,7 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 vn = start_state(k * (T / KB) + blk - 1, 1);
             }
             const int kmax = nval - blk * KB < KB ? nval - blk * KB : KB;
-            float* redb = red + (nred & 1) * (KB * RP);
+            float* redb = red + (nred & 1) * (TL::RED_WARPS * KB * RP);
             if (kmax == KB) block(blk, std::integral_constant<int, KB>{}, h, v, redb);
             else block(blk, kmax, h, v, redb);
             ++nred;
@@ -540,11 +554,17 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             for (int it = tid; it < (KB / 4) * RP; it += NT) {
                 const int slot = it % RP;
                 const int t4 = (it / RP) * 4;
+                // the warps' slices in a fixed order (entries of steps past kmax
+                // are stale and never used); one slice of atomic sums is zeroed
+                // for its next block
                 float v4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    v4[e] = redb[(t4 + e) * RP + slot];
-                    redb[(t4 + e) * RP + slot] = 0.0f;
+                    float acc = redb[(t4 + e) * RP + slot];
+#pragma unroll
+                    for (int w = 1; w < TL::RED_WARPS; ++w) acc += redb[w * (KB * RP) + (t4 + e) * RP + slot];
+                    if constexpr (TL::RED_WARPS == 1) redb[(t4 + e) * RP + slot] = 0.0f;
+                    v4[e] = acc;
                 }
                 const int which = slot / NP;
                 const int n = slot - which * NP;
