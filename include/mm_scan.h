@@ -121,7 +121,7 @@ typedef struct {
  *     (when A <= 0 and delta >= 0), else over the whole segment.  It runs as
  *     two launches on `stream` -- the segments' main passes, their maps
  *     written to records, then the folds and corrections -- with the records
- *     (ceil(L / S) * batch * ceil(dim / 16) * 4112 bytes, 4.2 MB for one row
+ *     (ceil(L / S) * batch * ceil(dim / 16) * 4112 bytes, 4.7 MB for one row
  *     of 2048 channels and 131072 steps) in stream-ordered memory from a
  *     pool the library creates per device on first use and keeps (up to
  *     64 MiB reserved between calls; cudaMallocFromPoolAsync, cudaFreeAsync
