@@ -608,16 +608,18 @@ class ClockSampler:
 
 # ------------------------------------------------------------ helpers ------
 def split_seg_len(w: wl.ScanWorkload, world: int, forced: int = 0) -> int:
-    """Segment length of the sequence split over `world` ranks (the split
-    entry points take a power of two): the largest power of two, at most
-    16384 for up to 2048 channels (2^25 channel-steps) and doubling below
-    that, at which every rank holds at least eight segments (one round of a
-    full cluster), never below one staged chunk."""
+    """Segment length of the sequence split over `world` ranks: the
+    sequence-split path's own length for the workload, halved until every
+    rank holds at least eight segments (one round of a full cluster), never
+    below one staged chunk."""
+    import selective_state_space_momentum_b200 as mm
     if forced:
         return forced
-    S = 16384
-    while S < (1 << 30) and S * w.batch * w.dim < (1 << 25):
-        S *= 2
+    mm.mm_scan_set_path(2, 0)
+    try:
+        S = mm.mm_scan_segment_len(w.batch, w.seqlen, w.dim, w.dstate, 0 if w.io == "f32" else 1)
+    finally:
+        mm.mm_scan_set_path(0, 0)
     chunk = 32 if w.io == "f32" else 64
     while S > chunk and -(-w.seqlen // S) < 8 * world:
         S //= 2

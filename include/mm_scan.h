@@ -109,11 +109,9 @@ typedef struct {
  *   - register-resident: every (channel, state) lane walks the whole
  *     sequence in time order with its state in registers;
  *   - sequence-split (few channels, dstate 9..16, fp32, rows of a whole
- *     number of 16-byte pieces, L > 16384): the sequence is cut into segments of S
- *     steps (mm_scan_segment_len: by default L cut into as many parts as fill
- *     two one-warp CTAs per warp scheduler, rounded up to whole chunks of the
- *     kernel) at absolute multiples of S, each run from a zero state on its
- *     own CTA, and joined by folding
+ *     number of 16-byte pieces, L > S): the sequence is cut into segments of S
+ *     steps (S a power of two, mm_scan_segment_len) at absolute multiples of
+ *     S, each run from a zero state on its own CTA, and joined by folding
  *     each segment's 2x2 affine carry map onto the concrete carry in segment
  *     order ("Forward Pass: Two-Stage Parallel Scan" of the same page, with
  *     the chunk carry [[beta^S, 0], [Q, P]] per lane); y gets the response to
@@ -121,7 +119,7 @@ typedef struct {
  *     (when A <= 0 and delta >= 0), else over the whole segment.  It runs as
  *     two launches on `stream` -- the segments' main passes, their maps
  *     written to records, then the folds and corrections -- with the records
- *     (ceil(L / S) * batch * ceil(dim / 16) * 4112 bytes, 4.7 MB for one row
+ *     (ceil(L / S) * batch * ceil(dim / 16) * 4112 bytes, 4.2 MB for one row
  *     of 2048 channels and 131072 steps) in stream-ordered memory from a
  *     pool the library creates per device on first use and keeps (up to
  *     64 MiB reserved between calls; cudaMallocFromPoolAsync, cudaFreeAsync
@@ -129,19 +127,15 @@ typedef struct {
  *     1 GiB), for in-place streaming (hT = h0 or vT = v0), and while `stream`
  *     is being captured into a CUDA graph (nothing is allocated then), it
  *     runs as one launch whose segments exchange their maps through
- *     distributed shared memory (a cluster of up to 8 CTAs per channel tile;
- *     with the automatic length its segments are at least ceil(L / 8) steps,
- *     whole chunks, so that one round covers the sequence); both forms give
- *     bit-identical results at one S.  mm_scan_fwd_noalloc
+ *     distributed shared memory; both forms give bit-identical results.  mm_scan_fwd_noalloc
  *     allocates nothing.
  *
  * Streaming: for a fixed (batch, dim, dstate, io), calling with the first
  * L1 steps and then with the remaining steps, passing (hT, vT) of the first
  * call as (h0, v0) of the second, gives final states bit-identical to one
  * call over all steps, and the same y within rounding, when all three calls
- * take the same path and L1 is a multiple of S (sequence-split path: all
- * three calls with one S, pinned by mm_scan_set_path(2, S) since the
- * automatic S depends on seqlen), of 32 (register-resident time
+ * take the same path and L1 is a multiple of S (sequence-split path: S is
+ * the mm_scan_segment_len() of the calls), of 32 (register-resident time
  * split, mm_scan_set_tile with two time lanes), or any L1 (register-resident
  * path with one time lane, which applies the steps in order).  The path of
  * each call is what mm_scan_segment_len() reports for its sizes (0: the
@@ -499,9 +493,9 @@ mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_
  * register-resident kernel, 2 the sequence-split kernel (used where it
  * applies: no extras, no checkpoints, dstate <= 16, rows of a whole number of
  * 16-byte pieces), 3 the same as one fused launch (no records, see
- * mm_scan_fwd) -- and its segment length (0: automatic; else a multiple of
- * 32 in [32, 2^30]; bf16 calls round it up to a multiple of 64, one staged
- * chunk of the kernel).  Process-wide, not thread-safe with concurrent calls.
+ * mm_scan_fwd) -- and its segment length (0: automatic; else a power of
+ * two in [32, 2^30]; bf16 calls use at least 64, one staged chunk of the
+ * kernel).  Process-wide, not thread-safe with concurrent calls.
  * MM_ERR_UNSUPPORTED for other values.
  */
 mm_status mm_scan_set_path(int path, int64_t seg_len);
@@ -509,15 +503,10 @@ mm_status mm_scan_set_path(int path, int64_t seg_len);
 /*
  * mm_scan_segment_len -- the segment length S the scan uses for these sizes
  * (*seg_len = 0 when the call runs on the register-resident path, which the
- * automatic choice takes whenever seqlen <= 16384 or seqlen <= S).  The
- * automatic S depends on (batch * dim), seqlen and the current device's SM
- * count (148 assumed when no device answers): seqlen cut into
- * floor(8 * SMs / (batch * ceil(dim / 16))) parts, at least 1024 steps,
- * rounded up to a whole staged chunk (32 steps, 64 for bf16) -- 14592 for
- * one row of 2048 channels and 131072 steps on 148 SMs.  A streaming caller
- * that pins S with mm_scan_set_path and splits a sequence at multiples of it,
- * into calls that all take the sequence-split path, gets final states
- * bit-identical to one call (see mm_scan_fwd).  Errors as
+ * automatic choice takes whenever seqlen <= S).  S itself depends on
+ * (batch * dim) only.  A streaming caller that splits a sequence at
+ * multiples of S, into calls that all take the sequence-split path, gets
+ * final states bit-identical to one call (see mm_scan_fwd).  Errors as
  * mm_scan_fwd's size checks; MM_ERR_NULL for a NULL argument.
  */
 mm_status mm_scan_segment_len(const mm_scan_dims *dims, int64_t *seg_len);

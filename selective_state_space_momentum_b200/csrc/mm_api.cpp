@@ -51,34 +51,19 @@ bool seg_auto(int64_t batch, int64_t dim, int64_t dstate, int io) {
 }
 
 // Segment length of the sequence-split path for these sizes, or 0 when the
-// call runs on the register-resident kernel.  The automatic length depends on
-// (batch * dim), L and the device's SM count; a forced one on nothing.
-// *fused_len: the length the single fused launch uses instead -- a forced
-// length as it is; the automatic one raised so that one round of a cluster of
-// kSegMaxCluster CTAs covers the sequence (more segments than that would walk
-// rounds, each CTA running several segments one after another).
-int64_t seg_len_for(int64_t batch, int64_t L, int64_t dim, int64_t dstate, int io, bool vec_ok,
-                    int64_t* fused_len = nullptr) {
-    if (fused_len) *fused_len = 0;
+// call runs on the register-resident kernel.  The length itself depends on
+// (batch * dim) only, never on L.
+int64_t seg_len_for(int64_t batch, int64_t L, int64_t dim, int64_t dstate, int io, bool vec_ok) {
     const int path = g_forced_path.load();
     if (!vec_ok || dstate > 16) return 0;
     if (path == 1) return 0;
     if (path == 0 && !seg_auto(batch, dim, dstate, io)) return 0;       // 2, 3: forced
     const int64_t forced = g_forced_seg_len.load();
-    int64_t S = forced > 0 ? forced : mmscan::scan_seg_fill_len(batch, dim, L);
+    int64_t S = forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
     // a segment is a whole number of staged chunks (64 steps for bf16)
     const int64_t chunk = mmscan::scan_seg_chunk_steps(io == MM_F32 ? 0 : 1);
-    S = (S + chunk - 1) / chunk * chunk;
-    if (path == 0 && (L <= mmscan::kSegMinLen || L <= S)) return 0;
-    if (fused_len) {
-        int64_t Sf = S;
-        if (forced <= 0) {
-            const int64_t one_round = (L + mmscan::kSegMaxCluster - 1) / mmscan::kSegMaxCluster;
-            Sf = (one_round + chunk - 1) / chunk * chunk;
-            if (Sf < S) Sf = S;
-        }
-        *fused_len = Sf;
-    }
+    if (S < chunk) S = chunk;
+    if (path == 0 && L <= S) return 0;
     return S;
 }
 
@@ -299,8 +284,8 @@ mm_status mm_scan_set_tile(int spt, int warps, int time_lanes) {
 mm_status mm_scan_set_path(int path, int64_t seg_len) {
     if (path < 0 || path > 3)
         return fail(MM_ERR_UNSUPPORTED, "scan path %d is not 0 (automatic), 1, 2 or 3", path);
-    if (seg_len != 0 && (seg_len < 32 || seg_len > (int64_t(1) << 30) || seg_len % 32 != 0))
-        return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not 0 or a multiple of 32 in [32, 2^30]",
+    if (seg_len != 0 && (seg_len < 32 || seg_len > (int64_t(1) << 30) || (seg_len & (seg_len - 1)) != 0))
+        return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not 0 or a power of two in [32, 2^30]",
                     (long long)seg_len);
     g_forced_path = path;
     g_forced_seg_len = seg_len;
@@ -505,14 +490,12 @@ mm_status mm_scan_fwd_gated(const void* x, const void* delta, const float* A, co
     a.stall = inject_stall();
     a.deny_records = inject_records_denied();
     if (!a.ext && !ckpt) {
-        int64_t seg_fused = 0;
-        const int64_t seg = seg_len_for(bsz, L, D, N, dims->io, a.vec_ok != 0, &seg_fused);
+        const int64_t seg = seg_len_for(bsz, L, D, N, dims->io, a.vec_ok != 0);
         if (seg > 0) {
             // in-place streaming (hT = h0 or vT = v0) needs the fused launch, whose CTAs
             // all read the initial state before any writes the final one
             const bool fused = g_forced_path.load() == 3 || (hT && hT == h0) || (vT && vT == v0);
-            return from_cuda(mmscan::launch_scan_seg(a, dims->io, seg, seg_fused, fused,
-                                                     static_cast<cudaStream_t>(stream)),
+            return from_cuda(mmscan::launch_scan_seg(a, dims->io, seg, fused, static_cast<cudaStream_t>(stream)),
                              "mm_scan_fwd launch");
         }
     }

@@ -112,31 +112,17 @@ struct ScanTileChoice {
     int ts;      // lanes along time per state group (1, or 2 for the time split)
 };
 
-// Sequence-split scan (scan_seg.cu): segments of S steps (a whole number of
-// staged chunks) at absolute multiples of S, joined through their 2x2 affine
-// carry maps.  The fused launch runs the segments of a channel tile as one
-// cluster of at most kSegMaxCluster CTAs; the two-launch form runs them as a
-// plain grid of up to kSegMaxRound segments per channel tile at a time.
-// Longer sequences walk rounds.
+// Sequence-split scan (scan_seg.cu): segments of a power-of-two length at
+// absolute multiples of it, one per CTA of a cluster of at most
+// kSegMaxCluster CTAs, joined through their 2x2 affine carry maps.
 constexpr int kSegMaxCluster = 8;
-constexpr int kSegMaxRound = 256;
-// The automatic choice splits only sequences longer than kSegMinLen, into
-// segments of at least kSegFloorLen steps.
 constexpr int64_t kSegMinLen = 16384;
-constexpr int64_t kSegFloorLen = 1024;
-// A power-of-two length from (batch * dim) alone: about 2^25 channel-steps per
-// round of segments, never below kSegMinLen (the fixed-scratch entry point's).
 int64_t scan_seg_default_len(int64_t batch, int64_t dim);
-// The automatic length: the segments of every channel tile together fill two
-// one-warp CTAs per warp scheduler of the current device.
-int64_t scan_seg_fill_len(int64_t batch, int64_t dim, int64_t seqlen);
 // The sequence-split path of mm_scan_fwd: by default two launches (the main
 // passes with their segment maps to records in stream-ordered memory from a
-// library pool, then the fold and correction) over segments of seg_len steps;
-// `fused`, or records that cannot be had, run the single fused launch over
-// segments of fused_seg_len steps.
-cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, int64_t fused_seg_len, bool fused,
-                            cudaStream_t s);
+// library pool, then the fold and correction); `fused`, or records that
+// cannot be had, run the single fused launch.
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, bool fused, cudaStream_t s);
 // Steps of one staged chunk of the sequence-split kernel (32 fp32, 64 bf16).
 int64_t scan_seg_chunk_steps(int io);
 // The sequence split over several calls: the channels of one CTA's tile and

@@ -946,47 +946,19 @@ namespace {
 constexpr int kSegWarps = 1;
 constexpr int kSegStages = 2;
 
-// The shared-memory attribute of all three modes is set on the first launch
-// of any on a device: a later call that switches to the fused launch (under
-// graph capture, say) then makes no such call.
-template <typename IO, bool SC>
-cudaError_t prepare_seg_kernels(int dev) {
-    using TL = SegTile<IO, kSegWarps, kSegStages>;
-    static std::atomic<uint64_t> done{0};
-    const uint64_t bit = 1ull << (dev & 63);
-    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
-    const void* kerns[3] = {reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 0>),
-                            reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 1>),
-                            reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 2>)};
-    for (const void* k : kerns) {
-        const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-    }
-    done.fetch_or(bit, std::memory_order_release);
-    return cudaSuccess;
-}
-
 template <typename IO, bool SC, int MODE>
 cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, cudaStream_t stream) {
     using TL = SegTile<IO, kSegWarps, kSegStages>;
     ScanArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t nseg = (a.seqlen + seg_len - 1) / seg_len;
-    // A launch in clusters holds at most kSegMaxCluster segments of a channel
-    // tile at a time; a plain grid (the CTAs share nothing) holds up to
-    // kSegMaxRound, so that the segment count can be chosen to fill the GPU.
-    const bool clustered = MODE == 0 || (MODE == 2 && sp.seg_first > 0);
-    cudaError_t e;
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = prepare_seg_kernels<IO, SC>(dev)) != cudaSuccess) return e;
-    const int64_t cap = clustered ? kSegMaxCluster : kSegMaxRound;
-    const int csize = (int)(nseg < cap ? nseg : cap);
+    const int csize = (int)(nseg < kSegMaxCluster ? nseg : kSegMaxCluster);
     const int64_t grid = (int64_t)csize * a.batch * a.tiles_per_batch;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     CUtensorMap mx, md, mB, mC;
     const bool bf = sizeof(IO) == 2;
     const uint64_t L = (uint64_t)a.seqlen;
+    cudaError_t e;
     // (the correction launch of a split reads no x and no B: its maps for them
     // describe delta and C and are never used)
     const void* xs = MODE == 2 ? a.delta : a.x;
@@ -996,6 +968,23 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, 
     if ((e = make_map_3d(&mB, Bs, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
     if ((e = make_map_3d(&mC, a.C, bf, L, a.dstate, a.batch, TL::T, TL::NP)) != cudaSuccess) return e;
     auto kern = scan_seg_kernel<IO, kSegWarps, kSegStages, SC, MODE>;
+    // The shared-memory attribute of all three modes is set on the first launch
+    // of any on a device: a later call that switches to the fused launch (under
+    // graph capture, say) then makes no such call.
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load(std::memory_order_acquire) & bit)) {
+        const void* kerns[3] = {reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 0>),
+                                reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 1>),
+                                reinterpret_cast<const void*>(scan_seg_kernel<IO, kSegWarps, kSegStages, SC, 2>)};
+        for (const void* k : kerns)
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, TL::SMEM_BYTES)) !=
+                cudaSuccess)
+                return e;
+        attr_done.fetch_or(bit, std::memory_order_release);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(TL::NT, 1, 1);
@@ -1015,7 +1004,7 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, 
     // the split launches run as plain grids, placed freely, except the second
     // launch of a piece after the first, whose tiles share one fold of the
     // earlier pieces' records in a cluster
-    cfg.numAttrs = clustered ? 2 : 0;
+    cfg.numAttrs = (MODE == 0 || (MODE == 2 && sp.seg_first > 0)) ? 2 : 0;
     return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize, sp);
 }
 
@@ -1039,45 +1028,6 @@ int64_t scan_seg_default_len(int64_t batch, int64_t dim) {
     int64_t s = kSegMinLen;
     while (s < (int64_t(1) << 30) && s * ch < (int64_t(1) << 25)) s <<= 1;
     return s;
-}
-
-namespace {
-
-// SMs of the current device (148 on B200; that count when no device answers,
-// as on a host without a GPU).
-int device_sms() {
-    static std::atomic<int> sms_of[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-        (void)cudaGetLastError();
-        return 148;
-    }
-    int n = sms_of[dev].load(std::memory_order_relaxed);
-    if (n > 0) return n;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-        (void)cudaGetLastError();
-        return 148;
-    }
-    sms_of[dev].store(n, std::memory_order_relaxed);
-    return n;
-}
-
-}  // namespace
-
-int64_t scan_seg_fill_len(int64_t batch, int64_t dim, int64_t seqlen) {
-    // The main pass of a one-warp CTA is bound by issue latency: a scheduler
-    // with two warps finishes them in less than twice one warp's time, but one
-    // with three takes longer than the rest, and the launch lasts as long as
-    // its most loaded scheduler.  So the segments of all channel tiles fill two
-    // warps on each of the SM's four schedulers, 8 CTAs per SM, and no more:
-    // for one row of 2048 channels (128 tiles) on 148 SMs, nine segments (1152
-    // CTAs) of 14592 steps.  Never shorter than kSegFloorLen.
-    constexpr int CH = SegTile<float, kSegWarps, kSegStages>::CH;
-    const int64_t tiles = batch * ((dim + CH - 1) / CH);
-    int64_t nseg = tiles > 0 ? (int64_t)8 * device_sms() / tiles : 1;
-    if (nseg < 1) nseg = 1;
-    int64_t S = (seqlen + nseg - 1) / nseg;
-    return S < kSegFloorLen ? kSegFloorLen : S;
 }
 
 namespace {
@@ -1128,8 +1078,7 @@ int64_t call_record_bytes(const ScanArgs& a, int64_t seg_len) {
 
 }  // namespace
 
-cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, int64_t fused_seg_len, bool fused,
-                            cudaStream_t s) {
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, bool fused, cudaStream_t s) {
     // A stream being captured into a graph gets the fused launch: no pool is
     // created and nothing is allocated while the capture is open.
     cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
@@ -1158,7 +1107,7 @@ cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t seg_len, int64_t 
         }
         (void)cudaGetLastError();   // no records: the fused launch needs none
     }
-    return launch_seg_mode<0>(a, io, fused_seg_len, SegSplit{}, s);
+    return launch_seg_mode<0>(a, io, seg_len, SegSplit{}, s);
 }
 
 int64_t scan_seg_chunk_steps(int io) {

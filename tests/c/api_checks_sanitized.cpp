@@ -42,8 +42,7 @@ cudaError_t launch_scan_step(const ScanStepArgs&, int, cudaStream_t) { ++g_launc
 cudaError_t launch_ssd_fwd(const SSDArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
 cudaError_t launch_ssd_mom(const SSDMomArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
 int64_t scan_seg_default_len(int64_t, int64_t) { return 16384; }
-int64_t scan_seg_fill_len(int64_t, int64_t, int64_t) { return 16384; }
-cudaError_t launch_scan_seg(const ScanArgs&, int, int64_t, int64_t, bool, cudaStream_t) { ++g_launches; return cudaSuccess; }
+cudaError_t launch_scan_seg(const ScanArgs&, int, int64_t, bool, cudaStream_t) { ++g_launches; return cudaSuccess; }
 int64_t scan_seg_chunk_steps(int io) { return io == 0 ? 32 : 64; }
 int64_t scan_seg_tile_channels() { return 16; }
 int64_t scan_seg_tile_record_bytes() { return 257 * 16; }

@@ -358,13 +358,12 @@ cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice&, int io, cu
     enqueue(s, [a, io] { scan_cpu(a, io); });
     return cudaSuccess;
 }
-cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t, int64_t, bool, cudaStream_t s) {
+cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t, bool, cudaStream_t s) {
     ++g_launches;
     enqueue(s, [a, io] { scan_cpu(a, io); });
     return cudaSuccess;
 }
 int64_t scan_seg_default_len(int64_t, int64_t) { return 64; }
-int64_t scan_seg_fill_len(int64_t, int64_t, int64_t) { return 64; }
 cudaError_t launch_scan_bwd(const ScanBwdArgs&, int, cudaStream_t) { return cudaErrorInvalidValue; }
 cudaError_t launch_scan_step(const ScanStepArgs&, int, cudaStream_t) { return cudaErrorInvalidValue; }
 cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t s) {

@@ -236,33 +236,17 @@ def test_set_path_and_segment_length_query(lib):
     assert lib.mm_scan_set_path(3, 0) == 0                        # the sequence split as one fused launch
     seg3 = ctypes.c_int64(-1)
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg3)) == 0
-    # forced onto the sequence-split path: 384 channel tiles fill 8 CTAs on each
-    # of 148 SMs (no device here answers) with three segments, below the floor
-    assert seg3.value == 1024
+    assert seg3.value == 16384                                    # forced onto the sequence-split path
     assert lib.mm_scan_set_path(0, 0) == 0
-    assert lib.mm_scan_set_path(2, 48) == 6                       # not a multiple of 32
+    assert lib.mm_scan_set_path(2, 48) == 6                       # not a power of two
     assert lib.mm_scan_set_path(2, 16) == 6                       # below 32
-    assert lib.mm_scan_set_path(2, (1 << 30) + 32) == 6           # above 2^30
     seg = ctypes.c_int64(-1)
-    # one row of 2048 channels (128 tiles): nine segments of ceil(131072 / 9)
-    # steps rounded up to a whole 32-step chunk
     dims = mm.ScanDims(1, 131072, 2048, 16, 0)
-    assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 14592
-    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 131072, 1024, 16, 0)), ctypes.byref(seg)) == 0
-    assert seg.value == 7296                                      # 64 tiles: eighteen segments
-    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 131072, 16, 16, 0)), ctypes.byref(seg)) == 0
-    assert seg.value == 1024                                      # one tile: the floor, 128 segments
-    one_segment = mm.ScanDims(1, 16384, 2048, 16, 0)               # L <= 16384: the register-resident path
+    assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 16384
+    one_segment = mm.ScanDims(1, 16384, 2048, 16, 0)               # L <= S: the register-resident path
     assert lib.mm_scan_segment_len(ctypes.byref(one_segment), ctypes.byref(seg)) == 0 and seg.value == 0
     just_over = mm.ScanDims(1, 16388, 2048, 16, 0)
-    assert lib.mm_scan_segment_len(ctypes.byref(just_over), ctypes.byref(seg)) == 0 and seg.value == 1824
-    assert lib.mm_scan_set_path(2, 14592) == 0                    # any whole number of 32-step chunks
-    assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 14592
-    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 131072, 2048, 16, 1)), ctypes.byref(seg)) == 0
-    assert seg.value == 14592                                     # already a whole 64-step chunk for bf16
-    assert lib.mm_scan_set_path(2, 96) == 0
-    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 2048, 64, 16, 1)), ctypes.byref(seg)) == 0
-    assert seg.value == 128                                       # bf16: rounded up to whole 64-step chunks
+    assert lib.mm_scan_segment_len(ctypes.byref(just_over), ctypes.byref(seg)) == 0 and seg.value == 16384
     assert lib.mm_scan_set_path(2, 256) == 0
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg)) == 0
     assert seg.value == 256                                       # forced onto the sequence-split path

@@ -39,7 +39,7 @@ def _close(got, ref, what):
 @pytest.mark.gpu
 def test_no_alloc_scan_matches_mm_scan_fwd_on_two_calls_in_a_row():
     mm.mm_scan_set_path(0, 0)                 # mm_scan_fwd on its automatic path
-    batch, L, D, N = 1, 32768, 2048, 16       # the entry point: 2048 channels in two 16384-step segments
+    batch, L, D, N = 1, 32768, 2048, 16       # 2048 channels: 16384-step segments, two of them
     for call, seed in enumerate((101, 202)):
         inp = wl.scan_inputs(wl.SCAN_LONG, batch=batch, seqlen=L, dim=D, dstate=N, seed=seed)
         dev = {k: torch.from_numpy(v).cuda().contiguous() for k, v in inp.items()}
