@@ -12,7 +12,8 @@
  *   mm_scan_fwd) and the fixed array of mm_scan_fwd_noalloc; it keeps no
  *   other state between calls except a per-thread copy of the last error
  *   message (mm_last_error), the process-wide tuning switches
- *   (mm_scan_set_tile, mm_scan_set_path) and the per-thread side streams of
+ *   (mm_scan_set_tile, mm_scan_set_path, mm_scan_set_deterministic) and the
+ *   per-thread side streams of
  *   the *_host entry points, which take host buffers and a device workspace.
  * - Every base pointer of a device buffer must be 16-byte aligned
  *   (MM_ERR_ALIGN otherwise).
@@ -220,8 +221,10 @@ mm_status mm_scan_ckpt_size(const mm_scan_dims *dims, size_t *bytes);
  * hT, vT, or NULL for zero.
  * Outputs (overwritten): dx, ddelta (batch, dim, L) io (rounded to nearest
  * even for bf16); dA (dim, dstate), dB, dC (batch, dstate, L) fp32 (sums:
- * the order of their additions is not fixed, so they can differ in the
- * last bits between runs); dh0, dv0 (batch, dim, dstate) fp32 or NULL.
+ * by default added atomically across CTAs, in no fixed order, so they can
+ * differ in the last bits between runs; after mm_scan_set_deterministic(1)
+ * summed in a fixed order and bit-identical between runs); dh0, dv0
+ * (batch, dim, dstate) fp32 or NULL.
  * No output may overlap an input or another output (MM_ERR_ALIAS); every
  * pointer must be 16-byte aligned.
  *
@@ -499,6 +502,27 @@ mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_
  * MM_ERR_UNSUPPORTED for other values.
  */
 mm_status mm_scan_set_path(int path, int64_t seg_len);
+
+/*
+ * mm_scan_set_deterministic -- 1: mm_scan_bwd and mm_scan_bwd_gated give
+ * run-to-run bit-identical dA, dB, dC, dD and ddelta_bias (every other output
+ * already is).  Each CTA then writes its channel tile's partial sums to a
+ * workspace instead of adding them atomically, and a second kernel adds the
+ * partials in a fixed order: dB, dC over the channel tiles of each batch row
+ * in tile order, dA, dD, ddelta_bias over the batch rows in row order.  The
+ * workspace, (tiles * 2 * batch * dstate * seqlen + batch * dim * (dstate +
+ * 2)) * 4 bytes with tiles = ceil(dim / channels per CTA) (dstate 9..16:
+ * 16 when batch * dim >= 2048, else 8; dstate 5..8: 16; 3..4: 32; 1..2: 64;
+ * 101 MB for batch 4, dim 1536, dstate 16, L 2048), is allocated and freed
+ * on the call's stream from a pool the library creates per device on first
+ * use (cudaMallocFromPoolAsync / cudaFreeAsync; up to 2 GiB kept reserved
+ * between calls); a call on a stream being captured into a graph returns
+ * MM_ERR_UNSUPPORTED.  The sums
+ * may differ from the default's in the last bits.  0 (the default): atomic
+ * sums.  Process-wide, not thread-safe with concurrent calls.
+ * MM_ERR_UNSUPPORTED for other values.
+ */
+mm_status mm_scan_set_deterministic(int on);
 
 /*
  * mm_scan_segment_len -- the segment length S the scan uses for these sizes

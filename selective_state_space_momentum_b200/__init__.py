@@ -30,7 +30,7 @@ __all__ = [
     "mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm_scan_bwd", "mm_scan_bwd_gated",
     "mm_scan_step", "mm_ssd_fwd", "mm_ssd_fwd_momentum", "ssd_fwd_momentum",
     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
-    "mm_scan_set_path", "mm_scan_segment_len",
+    "mm_scan_set_path", "mm_scan_segment_len", "mm_scan_set_deterministic",
     "mm_scan_fwd_host", "mm_scan_fwd_host_workspace_size", "mm_ssd_fwd_host",
     "mm_ssd_fwd_host_workspace_size",
     "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
@@ -61,7 +61,7 @@ EXPORTED_SYMBOLS = ("mm_scan_fwd", "mm_scan_fwd_gated", "mm_scan_ckpt_size", "mm
                     "mm_ssd_fwd",
                     "mm_device_status",
                     "mm_status_string", "mm_last_error", "mm_scan_set_tile", "mm_version",
-                    "mm_scan_set_path", "mm_scan_segment_len",
+                    "mm_scan_set_path", "mm_scan_segment_len", "mm_scan_set_deterministic",
                     "mm_scan_fwd_host_workspace_size", "mm_scan_fwd_host",
                     "mm_ssd_fwd_host_workspace_size", "mm_ssd_fwd_host",
                     "mm_scan_split_maps_size", "mm_scan_fwd_split_maps", "mm_scan_fwd_split_correct",
@@ -157,6 +157,8 @@ def _declare(lib):
     lib.mm_scan_set_tile.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.mm_scan_set_path.restype = ctypes.c_int
     lib.mm_scan_set_path.argtypes = [ctypes.c_int, ctypes.c_int64]
+    lib.mm_scan_set_deterministic.restype = ctypes.c_int
+    lib.mm_scan_set_deterministic.argtypes = [ctypes.c_int]
     lib.mm_scan_segment_len.restype = ctypes.c_int
     lib.mm_scan_segment_len.argtypes = [ctypes.POINTER(ScanDims), ctypes.POINTER(ctypes.c_int64)]
     lib.mm_version.restype = ctypes.c_int
@@ -492,6 +494,13 @@ def mm_scan_set_path(path: int, seg_len: int = 0):
     """Force the scan path (0 automatic, 1 register-resident, 2 sequence-split)
     and the segment length (0 automatic)."""
     _check(load_library().mm_scan_set_path(int(path), int(seg_len)), "mm_scan_set_path")
+
+
+def mm_scan_set_deterministic(on: bool):
+    """C entry point mm_scan_set_deterministic: the backward's parameter
+    gradients (dA, dB, dC, dD, d bias) summed in a fixed order, bit-identical
+    between runs (True), or added atomically (False, the default)."""
+    _check(load_library().mm_scan_set_deterministic(1 if on else 0), "mm_scan_set_deterministic")
 
 
 def mm_scan_segment_len(batch, seqlen, dim, dstate, io=MM_F32) -> int:

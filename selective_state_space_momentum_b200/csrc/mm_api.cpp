@@ -38,6 +38,7 @@ std::atomic<int> g_forced_ts{1};
 // Scan path: 0 automatic, 1 the register-resident kernel, 2 the sequence-split
 // kernel; and its segment length (0: automatic).
 std::atomic<int> g_forced_path{0};
+std::atomic<int> g_deterministic{0};
 std::atomic<int64_t> g_forced_seg_len{0};
 
 // The automatic path choice depends on (batch * dim, dstate, io) and on
@@ -289,6 +290,12 @@ mm_status mm_scan_set_path(int path, int64_t seg_len) {
                     (long long)seg_len);
     g_forced_path = path;
     g_forced_seg_len = seg_len;
+    return ok();
+}
+
+mm_status mm_scan_set_deterministic(int on) {
+    if (on != 0 && on != 1) return fail(MM_ERR_UNSUPPORTED, "deterministic switch %d is not 0 or 1", on);
+    g_deterministic = on;
     return ok();
 }
 
@@ -580,6 +587,16 @@ mm_status mm_scan_bwd_gated(const void* x, const void* delta, const float* A, co
     a.dz = z ? dz : nullptr;
     a.ddbias = a.ext ? ddelta_bias : nullptr;
     a.stall = inject_stall();
+    a.det = g_deterministic.load();
+    if (a.det) {
+        // the deterministic form allocates its workspace on the stream: not while
+        // the stream is being captured into a graph
+        if (mmscan::stream_capturing(static_cast<cudaStream_t>(stream)))
+            return fail(MM_ERR_UNSUPPORTED, "the deterministic backward allocates its workspace on the stream; "
+                                            "it does not run while the stream is being captured");
+        if (mmscan::scan_bwd_det_workspace_bytes(a.batch, a.dim, a.dstate, L) < 0)
+            return fail(MM_ERR_UNSUPPORTED, "the deterministic backward's workspace overflows 64 bits");
+    }
     return from_cuda(mmscan::launch_scan_bwd(a, dims->io, static_cast<cudaStream_t>(stream)),
                      "mm_scan_bwd launch");
 }

@@ -82,6 +82,13 @@ struct ScanBwdArgs {
     void* dz;              // (batch, dim, L) io, or null
     float* ddbias;         // (dim), or null
     int stall;             // test only: stage no input, so that the bounded waits run out
+    // The deterministic form (mm_scan_set_deterministic): per-tile partials of
+    // dB, dC and per-row partials of dA, dD, d bias in a workspace (filled by
+    // the launcher), summed in a fixed order by a second kernel.
+    int det;
+    float* ws_bc;          // [tile][dB, dC][batch][dstate][L]
+    float* ws_a;           // [batch][dim][dstate]
+    float* ws_d;           // [dD, d bias][batch][dim]
 };
 
 // Arguments of one decode step (device pointers; states updated in place).
@@ -145,6 +152,10 @@ ScanTileChoice choose_scan_tile(int64_t batch, int64_t dim, int64_t dstate, int 
                                 int forced_spt, int forced_warps, int forced_ts);
 cudaError_t launch_scan_fwd(const ScanArgs& a, const ScanTileChoice& t, int io, cudaStream_t s);
 cudaError_t launch_scan_bwd(const ScanBwdArgs& a, int io, cudaStream_t s);
+// Bytes of the deterministic backward's workspace (-1 past 2^63).
+int64_t scan_bwd_det_workspace_bytes(int64_t batch, int64_t dim, int dstate, int64_t seqlen);
+// Whether `s` is being captured into a CUDA graph (false when that cannot be told).
+bool stream_capturing(cudaStream_t s);
 cudaError_t launch_scan_step(const ScanStepArgs& a, int io, cudaStream_t s);
 // Read (and reset) the device error word of the scan / SSD kernels.
 unsigned int scan_read_and_clear_device_error();

@@ -41,6 +41,7 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <mutex>
 #include <type_traits>
 
 #include "mm_common.cuh"
@@ -52,7 +53,7 @@ namespace mmscan {
 // Device error word of this file's kernel (bounded waits that gave up).
 static __device__ unsigned int g_bwd_dev_err = 0;
 
-template <typename IO, int NP, int WARPS, bool EXT = false>
+template <typename IO, int NP, int WARPS, bool EXT = false, bool DET = false>
 struct BwdTile {
     static constexpr int SPT = 2;                // states per lane
     static constexpr int G = NP / SPT;           // lanes per channel
@@ -91,12 +92,13 @@ struct BwdTile {
     // kernel spills and ran 33% slower on the 384-CTA fp32 grid.
     static constexpr int MIN_CTAS = 12 / WARPS > 0 ? 12 / WARPS : 1;
     // Two blocks' dB, dC partials: one slice per warp, summed when a block is
-    // flushed, where MIN_CTAS CTAs of that size still fit an SM; else one
-    // slice that the warps add into with shared-memory atomics.
+    // flushed, where MIN_CTAS CTAs of that size still fit an SM (always in the
+    // deterministic form, whose sums must not depend on the warps' timing);
+    // else one slice that the warps add into with shared-memory atomics.
     static constexpr int smem_with(int red_warps) {
         return OFF_RED + 2 * red_warps * KB * RP * 4 + 2 * EXB + STAGES * 8 + 1024;
     }
-    static constexpr int RED_WARPS = MIN_CTAS * (smem_with(WARPS) + 1024) <= 228 * 1024 ? WARPS : 1;
+    static constexpr int RED_WARPS = DET || MIN_CTAS * (smem_with(WARPS) + 1024) <= 228 * 1024 ? WARPS : 1;
     static constexpr int RED_BYTES = 2 * RED_WARPS * KB * RP * 4;
     static constexpr int OFF_DP = OFF_RED + RED_BYTES;
     static constexpr int OFF_GY = OFF_DP + EXB;
@@ -111,13 +113,13 @@ struct BwdTile {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <typename IO, int NP, int WARPS, bool EXT>
-__global__ void __launch_bounds__(WARPS * 32, BwdTile<IO, NP, WARPS, EXT>::MIN_CTAS)
+template <typename IO, int NP, int WARPS, bool EXT, bool DET>
+__global__ void __launch_bounds__(WARPS * 32, BwdTile<IO, NP, WARPS, EXT, DET>::MIN_CTAS)
 scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_d,
                 const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_B,
                 const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_z,
                 const ScanBwdArgs p) {
-    using TL = BwdTile<IO, NP, WARPS, EXT>;
+    using TL = BwdTile<IO, NP, WARPS, EXT, DET>;
     constexpr int G = TL::G, CPW = TL::CPW, CH = TL::CH, NT = TL::NT, T = TL::T, R = TL::R;
     constexpr int ST = TL::STAGES, EB = TL::EB, BP = TL::BP, PER = TL::PER, KB = TL::KB;
     constexpr int RP = TL::RP;
@@ -568,7 +570,19 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 const int which = slot / NP;
                 const int n = slot - which * NP;
-                if (n < N && t4 < kmax) {
+                if (DET && n < N && t4 < kmax) {
+                    // the deterministic form: this channel tile's partial, stored once
+                    // per element, summed over the tiles in order by the reduce kernel
+                    const int64_t tile = blockIdx.x % p.tiles_per_batch;
+                    float* dst = p.ws_bc + ((tile * 2 + which) * p.batch + b) * N * L + n * L + t0 + blk * KB + t4;
+                    if (vec_red && t4 + 4 <= kmax) {
+                        *reinterpret_cast<float4*>(dst) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (t4 + e < kmax) dst[e] = v4[e];
+                    }
+                } else if (n < N && t4 < kmax) {
                     float* dst = (which ? p.dC : p.dB) + (b * N + n) * L + t0 + blk * KB + t4;
                     if (vec_red && t4 + 4 <= kmax) {
                         atomicAdd(reinterpret_cast<float4*>(dst), make_float4(v4[0], v4[1], v4[2], v4[3]));
@@ -590,8 +604,13 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             acc_db += __shfl_xor_sync(0xffffffffu, acc_db, m);
         }
         if (active && g == 0) {
-            if (p.dD) atomicAdd(p.dD + d, acc_dD);
-            if (p.ddbias) atomicAdd(p.ddbias + d, acc_db);
+            if constexpr (DET) {
+                if (p.dD) p.ws_d[b * p.dim + d] = acc_dD;
+                if (p.ddbias) p.ws_d[(p.batch + b) * p.dim + d] = acc_db;
+            } else {
+                if (p.dD) atomicAdd(p.dD + d, acc_dD);
+                if (p.ddbias) atomicAdd(p.ddbias + d, acc_db);
+            }
         }
     }
 
@@ -604,7 +623,8 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (n < N) {
                 if (p.dh0) p.dh0[srow + n] = gh[e];
                 if (p.dv0) p.dv0[srow + n] = gv[e];
-                atomicAdd(p.dA + d * N + n, ga[e]);
+                if constexpr (DET) p.ws_a[(b * p.dim + d) * N + n] = ga[e];
+                else atomicAdd(p.dA + d * N + n, ga[e]);
             }
         }
     }
@@ -613,9 +633,9 @@ scan_bwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 // ------------------------------------------------------------- launch -----
 namespace {
 
-template <typename IO, int NP, int WARPS, bool EXT>
+template <typename IO, int NP, int WARPS, bool EXT, bool DET>
 cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
-    using TL = BwdTile<IO, NP, WARPS, EXT>;
+    using TL = BwdTile<IO, NP, WARPS, EXT, DET>;
     ScanBwdArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t grid = a.batch * a.tiles_per_batch;
@@ -636,7 +656,7 @@ cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
         if (EXT && a.z && (e = make_map_3d(&mz, a.z, bf, L, a.dim, a.batch, TL::BOX_T, TL::CH)) != cudaSuccess)
             return e;
     }
-    auto kern = scan_bwd_kernel<IO, NP, WARPS, EXT>;
+    auto kern = scan_bwd_kernel<IO, NP, WARPS, EXT, DET>;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -651,30 +671,157 @@ cudaError_t launch_bwd_variant(const ScanBwdArgs& a0, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <typename IO, bool EXT>
+template <typename IO, bool EXT, bool DET>
 cudaError_t launch_bwd_io(const ScanBwdArgs& a, cudaStream_t s) {
     const int64_t channels = a.batch * a.dim;
     const int N = a.dstate;
     if (N > 8)
-        return channels >= 2048 ? launch_bwd_variant<IO, 16, 4, EXT>(a, s) : launch_bwd_variant<IO, 16, 2, EXT>(a, s);
-    if (N > 4) return launch_bwd_variant<IO, 8, 2, EXT>(a, s);
-    if (N > 2) return launch_bwd_variant<IO, 4, 2, EXT>(a, s);
-    return launch_bwd_variant<IO, 2, 2, EXT>(a, s);
+        return channels >= 2048 ? launch_bwd_variant<IO, 16, 4, EXT, DET>(a, s)
+                                : launch_bwd_variant<IO, 16, 2, EXT, DET>(a, s);
+    if (N > 4) return launch_bwd_variant<IO, 8, 2, EXT, DET>(a, s);
+    if (N > 2) return launch_bwd_variant<IO, 4, 2, EXT, DET>(a, s);
+    return launch_bwd_variant<IO, 2, 2, EXT, DET>(a, s);
+}
+
+// Channels of one CTA of the backward for these sizes (the tile launch_bwd_io picks).
+int bwd_tile_channels(int64_t batch, int64_t dim, int N) {
+    if (N > 8)
+        return batch * dim >= 2048 ? BwdTile<float, 16, 4>::CH : BwdTile<float, 16, 2>::CH;
+    if (N > 4) return BwdTile<float, 8, 2>::CH;
+    if (N > 2) return BwdTile<float, 4, 2>::CH;
+    return BwdTile<float, 2, 2>::CH;
+}
+
+// The deterministic form's sums: each output element adds its partials in a
+// fixed order -- dB, dC over the channel tiles of the batch row (tile 0
+// first), dA, dD and d bias over the batch rows (row 0 first) -- and is
+// written, not added to.
+__global__ void __launch_bounds__(256) bwd_det_reduce_kernel(const ScanBwdArgs p) {
+    const int64_t nbc = p.batch * p.dstate * p.seqlen;     // elements of dB (and of dC)
+    const int64_t na = p.dim * p.dstate;
+    const int64_t total = 2 * nbc + na + 2 * p.dim;
+    const int64_t tiles = p.tiles_per_batch;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < 2 * nbc) {
+            // partials laid out [tile][dB or dC][batch][state][step]
+            float acc = 0.0f;
+#pragma unroll 8
+            for (int64_t k = 0; k < tiles; ++k) acc += p.ws_bc[k * 2 * nbc + i];
+            if (i < nbc) p.dB[i] = acc;
+            else p.dC[i - nbc] = acc;
+        } else if (i < 2 * nbc + na) {
+            const int64_t j = i - 2 * nbc;                   // (channel, state)
+            float acc = 0.0f;
+            for (int64_t r = 0; r < p.batch; ++r) acc += p.ws_a[r * na + j];
+            p.dA[j] = acc;
+        } else {
+            const int64_t j = i - 2 * nbc - na;              // [dD or d bias][channel]
+            const int which = j >= p.dim ? 1 : 0;
+            const int64_t d = j - which * p.dim;
+            float* dst = which ? p.ddbias : p.dD;
+            if (!dst) continue;
+            float acc = 0.0f;
+            for (int64_t r = 0; r < p.batch; ++r) acc += p.ws_d[(which * p.batch + r) * p.dim + d];
+            dst[d] = acc;
+        }
+    }
 }
 
 }  // namespace
 
-cudaError_t launch_scan_bwd(const ScanBwdArgs& a, int io, cudaStream_t s) {
-    // dA, dB, dC (and dD, d bias) are sums that the kernel adds into: start them at zero.
+namespace {
+
+// Stream-ordered memory for the deterministic form's workspace: one pool per
+// device, created on first use, keeping up to kDetKeepBytes reserved between
+// calls (a workspace given back to the driver at every synchronisation had
+// to be mapped again by the next call, which cost more than the backward).
+constexpr int kDetPoolDevices = 64;
+constexpr uint64_t kDetKeepBytes = uint64_t(2) << 30;
+std::mutex g_det_pool_mutex;
+cudaMemPool_t g_det_pool[kDetPoolDevices] = {};
+
+cudaMemPool_t det_pool() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDetPoolDevices) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_det_pool_mutex);
+    if (g_det_pool[dev]) return g_det_pool[dev];
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    uint64_t keep = kDetKeepBytes;
+    (void)cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_det_pool[dev] = pool;
+    return pool;
+}
+
+}  // namespace
+
+bool stream_capturing(cudaStream_t s) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    return cap != cudaStreamCaptureStatusNone;
+}
+
+int64_t scan_bwd_det_workspace_bytes(int64_t batch, int64_t dim, int dstate, int64_t seqlen) {
+    const int64_t tiles = (dim + bwd_tile_channels(batch, dim, dstate) - 1) / bwd_tile_channels(batch, dim, dstate);
+    const double floats = (double)tiles * 2.0 * batch * dstate * seqlen + (double)batch * dim * dstate +
+                          2.0 * batch * dim;
+    if (floats * 4.0 > 9.0e18) return -1;
+    return (int64_t)floats * 4;
+}
+
+cudaError_t launch_scan_bwd(const ScanBwdArgs& a0, int io, cudaStream_t s) {
     cudaError_t e;
+    if (a0.det) {
+        // Per-tile partials into a workspace in stream-ordered memory, then the
+        // fixed-order sums; nothing is added atomically.
+        const int64_t bytes = scan_bwd_det_workspace_bytes(a0.batch, a0.dim, a0.dstate, a0.seqlen);
+        if (bytes < 0) return cudaErrorInvalidValue;
+        void* ws = nullptr;
+        cudaMemPool_t pool = det_pool();
+        if (!pool) return cudaErrorMemoryAllocation;
+        if ((e = cudaMallocFromPoolAsync(&ws, (size_t)bytes, pool, s)) != cudaSuccess) return e;
+        ScanBwdArgs a = a0;
+        a.tiles_per_batch = (int)((a.dim + bwd_tile_channels(a.batch, a.dim, a.dstate) - 1) /
+                                  bwd_tile_channels(a.batch, a.dim, a.dstate));
+        a.ws_bc = static_cast<float*>(ws);
+        a.ws_a = a.ws_bc + (int64_t)a.tiles_per_batch * 2 * a.batch * a.dstate * a.seqlen;
+        a.ws_d = a.ws_a + a.batch * a.dim * a.dstate;
+        e = a.ext ? (io == 0 ? launch_bwd_io<float, true, true>(a, s) : launch_bwd_io<bf16, true, true>(a, s))
+                  : (io == 0 ? launch_bwd_io<float, false, true>(a, s) : launch_bwd_io<bf16, false, true>(a, s));
+        if (e == cudaSuccess) {
+            const int64_t total = 2 * a.batch * a.dstate * a.seqlen + a.dim * a.dstate + 2 * a.dim;
+            int64_t blocks = (total + 255) / 256;
+            if (blocks > 148 * 16) blocks = 148 * 16;
+            bwd_det_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(a);
+            e = cudaGetLastError();
+        }
+        const cudaError_t ef = cudaFreeAsync(ws, s);
+        return e != cudaSuccess ? e : ef;
+    }
+    const ScanBwdArgs& a = a0;
+    // dA, dB, dC (and dD, d bias) are sums that the kernel adds into: start them at zero.
     if ((e = cudaMemsetAsync(a.dA, 0, (size_t)a.dim * a.dstate * 4, s)) != cudaSuccess) return e;
     const size_t bc = (size_t)a.batch * a.dstate * a.seqlen * 4;
     if ((e = cudaMemsetAsync(a.dB, 0, bc, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.dC, 0, bc, s)) != cudaSuccess) return e;
     if (a.dD && (e = cudaMemsetAsync(a.dD, 0, (size_t)a.dim * 4, s)) != cudaSuccess) return e;
     if (a.ddbias && (e = cudaMemsetAsync(a.ddbias, 0, (size_t)a.dim * 4, s)) != cudaSuccess) return e;
-    if (a.ext) return io == 0 ? launch_bwd_io<float, true>(a, s) : launch_bwd_io<bf16, true>(a, s);
-    return io == 0 ? launch_bwd_io<float, false>(a, s) : launch_bwd_io<bf16, false>(a, s);
+    if (a.ext) return io == 0 ? launch_bwd_io<float, true, false>(a, s) : launch_bwd_io<bf16, true, false>(a, s);
+    return io == 0 ? launch_bwd_io<float, false, false>(a, s) : launch_bwd_io<bf16, false, false>(a, s);
 }
 
 unsigned int scan_bwd_read_and_clear_device_error() {

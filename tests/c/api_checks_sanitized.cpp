@@ -38,6 +38,8 @@ ScanTileChoice choose_scan_tile(int64_t, int64_t, int64_t dstate, int, int, int,
 }
 cudaError_t launch_scan_fwd(const ScanArgs&, const ScanTileChoice&, int, cudaStream_t) { ++g_launches; return cudaSuccess; }
 cudaError_t launch_scan_bwd(const ScanBwdArgs&, int, cudaStream_t) { ++g_launches; return cudaSuccess; }
+int64_t scan_bwd_det_workspace_bytes(int64_t, int64_t, int, int64_t) { return 1024; }
+bool stream_capturing(cudaStream_t) { return false; }
 cudaError_t launch_scan_step(const ScanStepArgs&, int, cudaStream_t) { ++g_launches; return cudaSuccess; }
 cudaError_t launch_ssd_fwd(const SSDArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }
 cudaError_t launch_ssd_mom(const SSDMomArgs&, cudaStream_t) { ++g_launches; return cudaSuccess; }

@@ -365,6 +365,8 @@ cudaError_t launch_scan_seg(const ScanArgs& a, int io, int64_t, bool, cudaStream
 }
 int64_t scan_seg_default_len(int64_t, int64_t) { return 64; }
 cudaError_t launch_scan_bwd(const ScanBwdArgs&, int, cudaStream_t) { return cudaErrorInvalidValue; }
+int64_t scan_bwd_det_workspace_bytes(int64_t, int64_t, int, int64_t) { return 1024; }
+bool stream_capturing(cudaStream_t) { return false; }
 cudaError_t launch_scan_step(const ScanStepArgs&, int, cudaStream_t) { return cudaErrorInvalidValue; }
 cudaError_t launch_ssd_fwd(const SSDArgs& a, cudaStream_t s) {
     ++g_launches;

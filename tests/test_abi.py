@@ -231,6 +231,13 @@ def test_set_tile(lib):
     assert lib.mm_scan_set_tile(0, 0, 0) == 0
 
 
+def test_deterministic_switch(lib):
+    assert lib.mm_scan_set_deterministic(2) == 6
+    assert lib.mm_scan_set_deterministic(-1) == 6
+    assert lib.mm_scan_set_deterministic(1) == 0
+    assert lib.mm_scan_set_deterministic(0) == 0
+
+
 def test_set_path_and_segment_length_query(lib):
     assert lib.mm_scan_set_path(4, 0) == 6
     assert lib.mm_scan_set_path(3, 0) == 0                        # the sequence split as one fused launch
