@@ -283,6 +283,7 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
     gradient out."""
     import torch
     import selective_state_space_momentum_b200 as mm
+    mm.mm_scan_set_deterministic(bool(args.deterministic))
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = wl.scan_inputs(w, seed=rank_seed(w.seed_index, rank))
     iodt = torch.float32 if w.io == "f32" else torch.bfloat16
@@ -387,13 +388,16 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.io, "data": "synthetic",
             "config": {"workload": w.name, "pass": "backward", **({"extras": GATED_EXTRAS} if args.gated else {}),
+                       **({"sums": "deterministic"} if args.deterministic else {}),
                        "batch": w.batch, "seq_len": w.seqlen,
                        "dim": w.dim, "dstate": w.dstate, "beta": beta, "alpha": alpha, "io": w.io,
                        "global_batch": w.batch * world, "parallelism": f"dp{world}",
                        "l2": l2_note(step_bytes)},
             "roofline": {"bound": "alu", "kernel": "scan_bwd_kernel",
                          "achieved": achieved / 1e9, "peak": alu_peak / 1e9, "unit": "Gop/s",
-                         "frac": achieved / alu_peak, "traffic": None,
+                         "frac": achieved / alu_peak,
+                         "traffic": (None if args.gated or args.deterministic
+                                     else measured_traffic("scan_bwd_kernel", w.name)),
                          "peak_source": f"128 fp32 lanes/clk/SM x 148 SMs x {sm_max:.0f} MHz; "
                                         f"{BWD_OPS_PER_UPDATE} fp32 ops per state update",
                          "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -401,7 +405,8 @@ def run_scan_bwd(args, w, beta, alpha, rank, world):
                                  "algorithmic_bytes": step_bytes}},
             "e2e": {"value": whole_job_rate(w.updates, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps,
+            # the deterministic form adds the fixed-order sums as a second launch
+            "gpu_launches": args.steps * (2 if args.deterministic else 1),
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -1125,6 +1130,8 @@ def main(argv=None):
                     help="time mm_scan_fwd_gated with D, z, delta_bias and softplus (scan workloads)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward mm_scan_bwd (scan workloads)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="with --backward: the fixed-order sums of mm_scan_set_deterministic(1)")
     ap.add_argument("--tile", default=None, help="force SPTxWARPS[xTIME_LANES], e.g. 4x2 or 4x2x2 (tuning)")
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="scan path: 0 automatic, 1 register-resident, 2 sequence-split, 3 sequence-split "
@@ -1170,6 +1177,8 @@ def main(argv=None):
         return rc
     if args.backward and args.impl == "reference":
         ap.error("--impl reference times the forward")
+    if args.deterministic and not args.backward:
+        ap.error("--deterministic applies to --backward")
     if isinstance(w, wl.SSDWorkload):
         if args.impl == "reference":
             return run_reference(args, w)

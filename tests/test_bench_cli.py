@@ -49,6 +49,7 @@ def test_reference_arm_prints_one_json_line(workload):
     ("--workload", "ssd", "--gated"),                  # the extras belong to the scan
     ("--workload", "ssd", "--backward"),
     ("--backward", "--impl", "reference"),             # the reference arm times the forward
+    ("--deterministic",),                               # the fixed-order sums belong to the backward
     ("--workload", "decode", "--impl", "reference"),
 ])
 def test_bad_arguments_are_refused(args):

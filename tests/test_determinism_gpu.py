@@ -8,8 +8,9 @@ L2 flushed between) and compares every output bit for bit: the
 register-resident scan, the sequence-split scan in both launch forms, its
 split across emulated ranks, the gated scan, the decode step, the SSD form
 and the momentum SSD form.  (The backward's parameter gradients are float
-atomics and are not run-to-run reproducible; its other outputs are, and are
-compared.)
+atomics by default and not run-to-run reproducible; its other outputs are,
+and are compared.  With mm_scan_set_deterministic(1) they are too: see
+test_scan_bwd_det_gpu.py.)
 """
 import numpy as np
 import pytest
