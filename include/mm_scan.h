@@ -9,7 +9,9 @@
  *   of the current device; the caller allocates and owns every buffer.  The
  *   library's only device memory of its own is the stream-ordered record
  *   memory of mm_scan_fwd's sequence-split path (a pool per device, see
- *   mm_scan_fwd) and the fixed array of mm_scan_fwd_noalloc; it keeps no
+ *   mm_scan_fwd), the workspace of the deterministic backward (another pool
+ *   per device, see mm_scan_set_deterministic; only when switched on) and
+ *   the fixed array of mm_scan_fwd_noalloc; it keeps no
  *   other state between calls except a per-thread copy of the last error
  *   message (mm_last_error), the process-wide tuning switches
  *   (mm_scan_set_tile, mm_scan_set_path, mm_scan_set_deterministic) and the
