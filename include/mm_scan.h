@@ -498,9 +498,16 @@ mm_status mm_scan_set_tile(int states_per_thread, int warps_per_block, int time_
  * register-resident kernel, 2 the sequence-split kernel (used where it
  * applies: no extras, no checkpoints, dstate <= 16, rows of a whole number of
  * 16-byte pieces), 3 the same as one fused launch (no records, see
- * mm_scan_fwd) -- and its segment length (0: automatic; else a power of
- * two in [32, 2^30]; bf16 calls use at least 64, one staged chunk of the
- * kernel).  Process-wide, not thread-safe with concurrent calls.
+ * mm_scan_fwd) -- and its segment length (0: automatic, a power of two;
+ * else a multiple of 32 in [32, 2^30], rounded up to a multiple of 64 for
+ * bf16 calls, one staged chunk of the kernel).  Streaming calls keep
+ * bit-identical final states only when split at multiples of S (see
+ * mm_scan_fwd), so a forced length that does not divide a caller's split
+ * points trades that for the segment count it sets: on one row of 2048
+ * channels and 131072 steps (split point 65536), 14592
+ * cuts the sequence into nine segments, which fill two one-warp CTAs on each
+ * warp scheduler of 148 SMs and ran 9% faster than the automatic eight.
+ * Process-wide, not thread-safe with concurrent calls.
  * MM_ERR_UNSUPPORTED for other values.
  */
 mm_status mm_scan_set_path(int path, int64_t seg_len);

@@ -63,7 +63,7 @@ int64_t seg_len_for(int64_t batch, int64_t L, int64_t dim, int64_t dstate, int i
     int64_t S = forced > 0 ? forced : mmscan::scan_seg_default_len(batch, dim);
     // a segment is a whole number of staged chunks (64 steps for bf16)
     const int64_t chunk = mmscan::scan_seg_chunk_steps(io == MM_F32 ? 0 : 1);
-    if (S < chunk) S = chunk;
+    S = (S + chunk - 1) / chunk * chunk;
     if (path == 0 && L <= S) return 0;
     return S;
 }
@@ -285,8 +285,8 @@ mm_status mm_scan_set_tile(int spt, int warps, int time_lanes) {
 mm_status mm_scan_set_path(int path, int64_t seg_len) {
     if (path < 0 || path > 3)
         return fail(MM_ERR_UNSUPPORTED, "scan path %d is not 0 (automatic), 1, 2 or 3", path);
-    if (seg_len != 0 && (seg_len < 32 || seg_len > (int64_t(1) << 30) || (seg_len & (seg_len - 1)) != 0))
-        return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not 0 or a power of two in [32, 2^30]",
+    if (seg_len != 0 && (seg_len < 32 || seg_len > (int64_t(1) << 30) || seg_len % 32 != 0))
+        return fail(MM_ERR_UNSUPPORTED, "segment length %lld is not 0 or a multiple of 32 in [32, 2^30]",
                     (long long)seg_len);
     g_forced_path = path;
     g_forced_seg_len = seg_len;

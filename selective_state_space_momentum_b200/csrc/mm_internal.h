@@ -123,6 +123,7 @@ struct ScanTileChoice {
 // absolute multiples of it, one per CTA of a cluster of at most
 // kSegMaxCluster CTAs, joined through their 2x2 affine carry maps.
 constexpr int kSegMaxCluster = 8;
+constexpr int kSegMaxRound = 256;     // segments of a channel tile per round of a plain grid
 constexpr int64_t kSegMinLen = 16384;
 int64_t scan_seg_default_len(int64_t batch, int64_t dim);
 // The sequence-split path of mm_scan_fwd: by default two launches (the main

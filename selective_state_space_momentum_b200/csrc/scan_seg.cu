@@ -946,13 +946,42 @@ namespace {
 constexpr int kSegWarps = 1;
 constexpr int kSegStages = 2;
 
+// SMs of the current device (148 on B200; that count when no device answers).
+int device_sms() {
+    static std::atomic<int> sms_of[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    int n = sms_of[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    sms_of[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 template <typename IO, bool SC, int MODE>
 cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, cudaStream_t stream) {
     using TL = SegTile<IO, kSegWarps, kSegStages>;
     ScanArgs a = a0;
     a.tiles_per_batch = (int)((a.dim + TL::CH - 1) / TL::CH);
     const int64_t nseg = (a.seqlen + seg_len - 1) / seg_len;
-    const int csize = (int)(nseg < kSegMaxCluster ? nseg : kSegMaxCluster);
+    // A launch in clusters holds at most kSegMaxCluster segments of a channel
+    // tile at a time.  A plain grid (the CTAs share nothing) holds as many as
+    // fill two one-warp CTAs on every warp scheduler, if that is more: a forced
+    // length cutting the long workload into nine segments then runs them in one
+    // round (eight per round would leave the ninth to a second round alone).
+    const bool clustered = MODE == 0 || (MODE == 2 && sp.seg_first > 0);
+    int64_t cap = kSegMaxCluster;
+    if (!clustered) {
+        const int64_t fill = (int64_t)8 * device_sms() / (a.batch * a.tiles_per_batch);
+        if (fill > cap) cap = fill < kSegMaxRound ? fill : kSegMaxRound;
+    }
+    const int csize = (int)(nseg < cap ? nseg : cap);
     const int64_t grid = (int64_t)csize * a.batch * a.tiles_per_batch;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     CUtensorMap mx, md, mB, mC;
@@ -1004,7 +1033,7 @@ cudaError_t launch_seg(const ScanArgs& a0, int64_t seg_len, const SegSplit& sp, 
     // the split launches run as plain grids, placed freely, except the second
     // launch of a piece after the first, whose tiles share one fold of the
     // earlier pieces' records in a cluster
-    cfg.numAttrs = (MODE == 0 || (MODE == 2 && sp.seg_first > 0)) ? 2 : 0;
+    cfg.numAttrs = clustered ? 2 : 0;
     return cudaLaunchKernelEx(&cfg, kern, mx, md, mB, mC, a, seg_len, csize, sp);
 }
 

@@ -245,8 +245,9 @@ def test_set_path_and_segment_length_query(lib):
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg3)) == 0
     assert seg3.value == 16384                                    # forced onto the sequence-split path
     assert lib.mm_scan_set_path(0, 0) == 0
-    assert lib.mm_scan_set_path(2, 48) == 6                       # not a power of two
+    assert lib.mm_scan_set_path(2, 48) == 6                       # not a multiple of 32
     assert lib.mm_scan_set_path(2, 16) == 6                       # below 32
+    assert lib.mm_scan_set_path(2, (1 << 30) + 32) == 6           # above 2^30
     seg = ctypes.c_int64(-1)
     dims = mm.ScanDims(1, 131072, 2048, 16, 0)
     assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 16384
@@ -257,6 +258,11 @@ def test_set_path_and_segment_length_query(lib):
     assert lib.mm_scan_set_path(2, 256) == 0
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(4, 2048, 1536, 16, 0)), ctypes.byref(seg)) == 0
     assert seg.value == 256                                       # forced onto the sequence-split path
+    assert lib.mm_scan_set_path(2, 14592) == 0                    # any whole number of 32-step chunks
+    assert lib.mm_scan_segment_len(ctypes.byref(dims), ctypes.byref(seg)) == 0 and seg.value == 14592
+    assert lib.mm_scan_set_path(2, 96) == 0
+    assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 2048, 64, 16, 1)), ctypes.byref(seg)) == 0
+    assert seg.value == 128                                       # bf16: rounded up to whole 64-step chunks
     assert lib.mm_scan_set_path(2, 32) == 0
     assert lib.mm_scan_segment_len(ctypes.byref(mm.ScanDims(1, 2048, 64, 16, 1)), ctypes.byref(seg)) == 0
     assert seg.value == 64                                        # bf16: at least one 64-step chunk

@@ -91,11 +91,13 @@ def _check(io, got, inp, beta, alpha, h0=None, v0=None, what=""):
 
 
 @pytest.mark.parametrize("path", [2, 3], ids=["two-launch", "fused"])
-@pytest.mark.parametrize("L,seg", [(256, 32), (1000, 64), (4096, 128), (4133 // 4 * 4, 256), (96, 128)])
+@pytest.mark.parametrize("L,seg", [(256, 32), (1000, 64), (4096, 128), (4133 // 4 * 4, 256), (96, 128), (2000, 160)])
 @pytest.mark.parametrize("beta,alpha", [(0.9, 1.0), (0.0, 1.0), (0.99, 0.5), (0.3, 2.0), (0.5, 1.0)])
 def test_segments_rounds_and_ragged_ends(seg_path, L, seg, beta, alpha, path):
     # beta >= 1/2 runs the scaled form of the recurrence, smaller beta the plain one
-    # up to 32 segments: several rounds of an 8-CTA cluster, a ragged last chunk
+    # up to 32 segments: rounds of an 8-CTA cluster (fused) or of a plain grid
+    # (two launches), a ragged last chunk, a forced length that is not a power of
+    # two (13 segments of 160 steps, the last of 80)
     seg_path(seg, path)
     inp = _inputs(2, L, 40, 16, seed=7 + L)
     _check("f32", _run(_dev(inp, "f32"), beta, alpha), inp, beta, alpha, what=f"L={L} S={seg}")
@@ -137,7 +139,7 @@ def test_growing_modes_are_not_cut_short(seg_path):
     _check("f32", _run(_dev(inp, "f32"), 0.5, 1.0), inp, 0.5, 1.0, what="A > 0")
 
 
-@pytest.mark.parametrize("seg", [64, 256])
+@pytest.mark.parametrize("seg", [64, 256, 160])
 def test_streaming_split_at_segment_multiples_is_bit_identical(seg_path, seg):
     seg_path(seg)
     L, L1 = 2048, 4 * seg
@@ -197,7 +199,8 @@ def test_segment_length_query():
 
 
 @pytest.mark.parametrize("L,seg,beta,io", [(4096, 128, 0.99, "f32"), (1000, 64, 0.3, "f32"),
-                                           (2048, 256, 0.9, "bf16"), (8192, 64, 0.999, "f32")])
+                                           (2048, 256, 0.9, "bf16"), (8192, 64, 0.999, "f32"),
+                                           (2000, 160, 0.99, "f32"), (4096, 448, 0.9, "bf16")])
 def test_two_launch_and_fused_forms_are_bit_identical(seg_path, L, seg, beta, io):
     law = wl.SCAN_MEDIUM if io == "f32" else wl.SCAN_BF16
     inp = _inputs(2, L, 40, 16, seed=L + seg, io=io, law=law)
