@@ -1137,7 +1137,7 @@ def main(argv=None):
                     help="scan path: 0 automatic, 1 register-resident, 2 sequence-split, 3 sequence-split "
                          "as one fused launch (tuning)")
     ap.add_argument("--seg-len", type=int, default=0,
-                    help="segment length of the sequence-split path (power of two; 0 automatic)")
+                    help="segment length of the sequence-split path (a multiple of 32; 0 automatic)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (exploration; renames the workload)")
     ap.add_argument("--seqlen", type=int, default=None,
